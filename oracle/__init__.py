@@ -1,0 +1,100 @@
+"""fp64 CPU oracle for the selective scan and the recurrent state update.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by the smoke check and by the
+benchmark's CPU-baseline leg, never by the product library.  The arithmetic
+lives in `ssm_oracle.c` (plain C, double precision); this module only moves
+numpy arrays across ctypes.  It follows the zero-order-hold discretisation and
+recurrence of "Mamba SSM Nedir? Transformer Alternatifi Rehberi (2026)",
+sections "State Space Model Temelleri" and "Ayrık Zamana Geçiş".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_c_f64p = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+
+
+class Oracle:
+    """One loaded copy of the oracle library (a test may load a modified copy)."""
+
+    def __init__(self, lib_path: str | None = None):
+        path = lib_path or _build.build()
+        self.path = path
+        self._lib = ctypes.CDLL(os.path.abspath(path))
+        self._lib.oracle_scan.restype = ctypes.c_int
+        self._lib.oracle_scan.argtypes = [_c_f64p] * 9 + [_i64] * 4 + [ctypes.c_int]
+        self._lib.oracle_state_update.restype = ctypes.c_int
+        self._lib.oracle_state_update.argtypes = [_c_f64p] * 8 + [_i64] * 3 + [ctypes.c_int]
+        self._lib.oracle_max_threads.restype = ctypes.c_int
+
+    @staticmethod
+    def _ptr(a):
+        return None if a is None else a.ctypes.data_as(_c_f64p)
+
+    @staticmethod
+    def _f64(a):
+        return None if a is None else np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+    def scan(self, u, delta, A, B, C, D=None, h0=None, want_y=True, nthreads=0):
+        """Selective scan.  u, delta: (batch, len, channels); B, C: (batch, len,
+        nstate); A: (channels, nstate); D: (channels,) or None; h0: (batch,
+        channels, nstate) or None.  Returns (y, h_final) in float64."""
+        u, delta, A, B, C, D, h0 = map(self._f64, (u, delta, A, B, C, D, h0))
+        batch, length, channels = u.shape
+        nstate = A.shape[1]
+        assert delta.shape == u.shape and A.shape == (channels, nstate)
+        assert B.shape == (batch, length, nstate) and C.shape == B.shape
+        assert D is None or D.shape == (channels,)
+        assert h0 is None or h0.shape == (batch, channels, nstate)
+        y = np.empty_like(u) if want_y else None
+        hf = np.empty((batch, channels, nstate), dtype=np.float64)
+        rc = self._lib.oracle_scan(self._ptr(u), self._ptr(delta), self._ptr(A), self._ptr(B),
+                                   self._ptr(C), self._ptr(D), self._ptr(h0), self._ptr(y),
+                                   self._ptr(hf), batch, length, channels, nstate, int(nthreads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_scan failed ({rc})")
+        return y, hf
+
+    def state_update(self, state, x, delta, A, B, C, D=None, nthreads=0):
+        """One recurrent step.  state: (batch, channels, nstate) float64, updated
+        in place; x, delta: (batch, channels); B, C: (batch, nstate).  Returns y."""
+        assert state.dtype == np.float64 and state.flags.c_contiguous
+        x, delta, A, B, C, D = map(self._f64, (x, delta, A, B, C, D))
+        batch, channels, nstate = state.shape
+        assert x.shape == (batch, channels) and delta.shape == x.shape
+        assert A.shape == (channels, nstate) and B.shape == (batch, nstate) and C.shape == B.shape
+        y = np.empty_like(x)
+        rc = self._lib.oracle_state_update(self._ptr(state), self._ptr(x), self._ptr(delta),
+                                           self._ptr(A), self._ptr(B), self._ptr(C), self._ptr(D),
+                                           self._ptr(y), batch, channels, nstate, int(nthreads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_state_update failed ({rc})")
+        return y
+
+    def max_threads(self) -> int:
+        return int(self._lib.oracle_max_threads())
+
+
+_default: Oracle | None = None
+
+
+def get() -> Oracle:
+    """The oracle built from `ssm_oracle.c` (compiled on first use)."""
+    global _default
+    if _default is None:
+        _default = Oracle()
+    return _default
+
+
+def scan(*args, **kwargs):
+    return get().scan(*args, **kwargs)
+
+
+def state_update(*args, **kwargs):
+    return get().state_update(*args, **kwargs)

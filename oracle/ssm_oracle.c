@@ -1,0 +1,177 @@
+/*
+ * ssm_oracle.c -- fp64 CPU oracle for the selective-scan hot path.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, includes or
+ * calls this file; only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg do.  It shares no code, header, table or helper with the CUDA
+ * path.  It is deliberately plain and slow: one (batch, channel) row at a time,
+ * time as the outer loop, state index as the inner loop, every quantity in
+ * double precision, libm's exp/expm1.
+ *
+ * What it computes follows the web page "Mamba SSM Nedir? Transformer
+ * Alternatifi Rehberi (2026)" (yapayzekasozluk.tr):
+ *   - section "State Space Model Temelleri": the continuous system
+ *         h'(t) = A h(t) + B x(t),   y(t) = C h(t) + D x(t)
+ *   - section "Ayrık Zamana Geçiş": zero-order-hold discretisation with step
+ *     size Delta,
+ *         Abar = exp(Delta A)
+ *         Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B
+ *     followed by the recurrence  h_t = Abar h_{t-1} + Bbar x_t,  y_t = C h_t
+ *   - section "Mamba'nın Yeniliği: Selective SSM": B, C and Delta are produced
+ *     per token (B_t, C_t, Delta_t); A stays a fixed parameter.
+ *
+ * Readings taken where the pages are silent or disagree (each is listed in the
+ * design notes of the repository):
+ *   - A is diagonal, one value per (channel, state): A[d][n].  The discretised
+ *     quantities are then per state: Abar_n = exp(Delta A_n) and
+ *     Bbar_n = (Delta A_n)^-1 (exp(Delta A_n) - 1) Delta B_n.
+ *   - Delta is per (batch, token, channel); B_t and C_t are per (batch, token,
+ *     state) and shared by every channel.
+ *   - The discrete output keeps the D x_t skip term of the continuous form:
+ *     y_t = C_t . h_t + D_d x_t, with h_t the state AFTER the update at t.
+ *   - The scan starts from h = 0 unless an initial state is given.
+ *   - Delta A = 0 (outside the stable domain A < 0) uses the limit
+ *     (e^z - 1)/z -> 1, i.e. Bbar = Delta B.
+ *
+ * Layouts (row-major, last index fastest):
+ *   u, delta, y   : [batch][len][channels]
+ *   B, C          : [batch][len][nstate]
+ *   A             : [channels][nstate]
+ *   D             : [channels]                (may be NULL: no skip term)
+ *   h0, h_final   : [batch][channels][nstate] (h0 may be NULL: zeros)
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <stdlib.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* One zero-order-hold step for a single state of a diagonal system, exactly
+ * as the "Ayrık Zamana Geçiş" section writes it, with z = Delta * A_n:
+ *   Abar = exp(z)
+ *   Bbar = z^-1 (exp(z) - 1) Delta B_n
+ * exp(z) - 1 is evaluated with expm1 so that small z keeps full precision.   */
+static void zoh_discretise(double delta, double a, double b, double *abar, double *bbar)
+{
+    double z = delta * a;
+    *abar = exp(z);
+    double phi = (z == 0.0) ? 1.0 : expm1(z) / z; /* (Delta A)^-1 (e^{Delta A} - 1) */
+    *bbar = phi * delta * b;
+}
+
+/* The recurrence of one (batch, channel) row over `len` tokens.
+ * h (length nstate) holds the running state in and out.  `stride` is the
+ * distance between consecutive tokens in u/delta/y (the channel count).      */
+static void scan_row(const double *u, const double *delta, const double *A_row,
+                     const double *B, const double *C, double D_d, int has_D,
+                     double *y, double *h, int64_t len, int64_t stride, int64_t nstate)
+{
+    for (int64_t t = 0; t < len; ++t) {
+        double x = u[t * stride];
+        double dt = delta[t * stride];
+        const double *Bt = B + t * nstate;
+        const double *Ct = C + t * nstate;
+        double acc = 0.0;
+        for (int64_t n = 0; n < nstate; ++n) {
+            double abar, bbar;
+            zoh_discretise(dt, A_row[n], Bt[n], &abar, &bbar);
+            h[n] = abar * h[n] + bbar * x;    /* h_t = Abar h_{t-1} + Bbar x_t */
+            acc += Ct[n] * h[n];              /* C_t . h_t                     */
+        }
+        if (has_D)
+            acc += D_d * x;                   /* + D x_t                       */
+        if (y)
+            y[t * stride] = acc;
+    }
+}
+
+/* Selective scan over whole sequences.  Returns 0 on success, -1 on a bad
+ * argument.  nthreads <= 0 uses the OpenMP default.                          */
+int oracle_scan(const double *u, const double *delta, const double *A,
+                const double *B, const double *C, const double *D,
+                const double *h0, double *y, double *h_final,
+                int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                int nthreads)
+{
+    if (batch < 0 || len < 0 || channels < 0 || nstate <= 0)
+        return -1;
+    if ((len > 0 && (!u || !delta || !B || !C)) || !A)
+        return -1;
+    int64_t rows = batch * channels;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = 0;
+#pragma omp parallel
+    {
+        double *h = (double *)malloc(sizeof(double) * (size_t)nstate);
+        if (!h) {
+#pragma omp atomic write
+            status = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < rows; ++r) {
+            if (!h)
+                continue;
+            int64_t b = r / channels, d = r % channels;
+            for (int64_t n = 0; n < nstate; ++n)
+                h[n] = h0 ? h0[(b * channels + d) * nstate + n] : 0.0;
+            const size_t tok0 = (size_t)(b * len) * (size_t)channels + (size_t)d;
+            scan_row(len ? u + tok0 : NULL, len ? delta + tok0 : NULL, A + d * nstate,
+                     len ? B + (size_t)(b * len) * (size_t)nstate : NULL,
+                     len ? C + (size_t)(b * len) * (size_t)nstate : NULL,
+                     D ? D[d] : 0.0, D != NULL, (y && len) ? y + tok0 : NULL, h,
+                     len, channels, nstate);
+            if (h_final)
+                for (int64_t n = 0; n < nstate; ++n)
+                    h_final[(b * channels + d) * nstate + n] = h[n];
+        }
+        free(h);
+    }
+    return status;
+}
+
+/* One recurrent (generation-time) step for every (batch, channel) row: the
+ * O(1)-memory update the pages describe for inference ("Karmaşıklık
+ * Karşılaştırması": a fixed-size hidden state is updated per token).
+ * state [batch][channels][nstate] is updated in place; x, delta and y are
+ * [batch][channels]; B, C are [batch][nstate].                              */
+int oracle_state_update(double *state, const double *x, const double *delta,
+                        const double *A, const double *B, const double *C,
+                        const double *D, double *y,
+                        int64_t batch, int64_t channels, int64_t nstate, int nthreads)
+{
+    if (batch < 0 || channels < 0 || nstate <= 0 || !state || !x || !delta || !A || !B || !C)
+        return -1;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int64_t rows = batch * channels;
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        int64_t b = r / channels, d = r % channels;
+        scan_row(x + r, delta + r, A + d * nstate, B + b * nstate, C + b * nstate,
+                 D ? D[d] : 0.0, D != NULL, y ? y + r : NULL, state + r * nstate,
+                 1, channels, nstate);
+    }
+    return 0;
+}
+
+/* Threads the OpenMP runtime would use (for reporting the CPU baseline). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,56 @@
+"""The pins must be strong enough to catch plausible mistakes in the oracle.
+
+Each case below copies oracle/ssm_oracle.c, plants one mistake by text
+substitution, builds the copy on the CPU and runs every pin of
+test_oracle_pins.py against it: at least one pin has to fail.
+"""
+import os
+import shutil
+
+import pytest
+
+import oracle
+from oracle import build as oracle_build
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
+
+MUTANTS = {
+    "drop_skip_term": ("acc += D_d * x;", "(void)D_d;"),
+    "output_uses_previous_state": ("h[n] = abar * h[n] + bbar * x;    /* h_t = Abar h_{t-1} + Bbar x_t */\n"
+                                   "            acc += Ct[n] * h[n];",
+                                   "acc += Ct[n] * h[n];\n            h[n] = abar * h[n] + bbar * x;"),
+    "decay_sign_flipped": ("*abar = exp(z);", "*abar = exp(-z);"),
+    "euler_input_matrix": ("*bbar = phi * delta * b;", "*bbar = delta * b;"),
+    "input_matrix_missing_delta": ("*bbar = phi * delta * b;", "*bbar = phi * b;"),
+    "b_and_c_swapped": ("const double *Bt = B + t * nstate;\n        const double *Ct = C + t * nstate;",
+                        "const double *Bt = C + t * nstate;\n        const double *Ct = B + t * nstate;"),
+    "state_not_reset_per_row": ("h[n] = h0 ? h0[(b * channels + d) * nstate + n] : 0.0;",
+                                "h[n] = h0 ? h0[(b * channels + d) * nstate + n] : (r == 0 ? 0.0 : h[n]);"),
+    "token_stride_ignored": ("double x = u[t * stride];", "double x = u[t];"),
+    "a_row_of_wrong_channel": ("A + d * nstate, ", "A + ((d + 1) % channels) * nstate, "),
+    "b_uses_wrong_batch": ("len ? B + (size_t)(b * len) * (size_t)nstate : NULL,",
+                           "len ? B : NULL,"),
+    "expm1_replaced_by_exp": ("expm1(z) / z", "exp(z) / z"),
+}
+
+PIN_TESTS = [getattr(pins, name) for name in dir(pins) if name.startswith("test_")]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    text = open(SRC).read()
+    assert text.count(old) == 1, f"mutation anchor for {name} not found exactly once"
+    src = tmp_path / "mutant.c"
+    src.write_text(text.replace(old, new))
+    lib = oracle_build.build(str(src), str(tmp_path / "libmutant.so"), force=True)
+    mutant = oracle.Oracle(lib)
+    failed = []
+    for test in PIN_TESTS:
+        try:
+            test(mutant)
+        except Exception:          # an assertion or a shape/NaN failure both count
+            failed.append(test.__name__)
+    assert failed, f"no pin caught mutant {name}"
+    shutil.rmtree(tmp_path, ignore_errors=True)
