@@ -1,0 +1,164 @@
+/*
+ * mamba_ssm.h -- C ABI of the B200 (sm_100a) selective-scan library.
+ *
+ * The library computes the hot path of the Mamba selective state-space model
+ * described on the web page "Mamba SSM Nedir? Transformer Alternatifi Rehberi
+ * (2026)":
+ *   - section "State Space Model Temelleri": continuous system
+ *       h'(t) = A h(t) + B x(t),  y(t) = C h(t) + D x(t);
+ *   - section "Ayrık Zamana Geçiş": zero-order-hold discretisation
+ *       Abar = exp(Delta A),  Bbar = (Delta A)^-1 (exp(Delta A) - I) Delta B,
+ *     and the recurrence h_t = Abar h_{t-1} + Bbar x_t,  y_t = C h_t;
+ *   - section "Mamba'nın Yeniliği: Selective SSM": B_t, C_t and Delta_t are
+ *     given per token (the projections that produce them are not part of
+ *     this library);
+ *   - section "Paralel Tarama Algoritması": the recurrence is evaluated with a
+ *     chunked scan whose chunk results are combined associatively.
+ *
+ * A is diagonal and real: one value A[d][n] per (channel, state), expected
+ * negative (the stability condition of the same page's "Sınırlılıklar ve Açık
+ * Sorular" section; not checked).  Each output is y_t = C_t . h_t + D_d x_t
+ * with h_t the state after the update at token t.
+ *
+ * Conventions for every entry point
+ *   - Pointers named device memory must be CUDA device (or managed) memory of
+ *     the current device, owned by the caller; the library never frees them.
+ *   - Layouts are dense row-major with the last index fastest:
+ *       u, delta, y            [batch][len][channels]
+ *       B, C                   [batch][len][nstate]   (shared by all channels)
+ *       A                      [channels][nstate]     float32
+ *       D                      [channels]             float32
+ *       states                 [batch][channels][nstate] float32
+ *   - `dtype` (mamba_dtype_t) is the element type of u, delta, B, C and y
+ *     (x, delta, B, C, y for the state update).  A, D and states are float32.
+ *     All arithmetic is float32; y is rounded to `dtype` (round to nearest even).
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream): they
+ *     validate arguments on the host, enqueue kernels and return.  They never
+ *     synchronise.
+ *   - Return value: a mamba_status_t.  Argument errors are reported before
+ *     anything is enqueued.  A kernel-launch failure returns MAMBA_ERR_CUDA.
+ *     A bounded device-side wait that ran out records MAMBA_ERR_TIMEOUT in a
+ *     device error word that mamba_get_device_error() reports.  No call traps
+ *     or aborts on the device.
+ *   - y must not overlap any input.  u/delta/B/C/A/D may alias one another
+ *     (they are only read).
+ *   - Not checked (preconditions): A < 0; delta > 0 (delta is the output of
+ *     a softplus in the model); finite inputs.
+ */
+#ifndef MAMBA_SSM_H
+#define MAMBA_SSM_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so the header needs no CUDA include. */
+typedef struct CUstream_st *mamba_stream_t;
+
+typedef enum {
+    MAMBA_F32 = 0,  /* float32 */
+    MAMBA_BF16 = 1  /* bfloat16 */
+} mamba_dtype_t;
+
+typedef enum {
+    MAMBA_OK = 0,
+    MAMBA_ERR_INVALID_ARG = 1,  /* null required pointer, negative size, unknown dtype, bad alignment */
+    MAMBA_ERR_UNSUPPORTED = 2,  /* valid request this build does not implement (e.g. nstate) */
+    MAMBA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed */
+    MAMBA_ERR_TIMEOUT = 4       /* a bounded device wait ran out (see mamba_get_device_error) */
+} mamba_status_t;
+
+/* Flags for mamba_selective_scan_ex. */
+#define MAMBA_SCAN_GENERAL_A 1u  /* never take the path for A[d][n] = (n+1) A[d][0] */
+
+/*
+ * Selective scan over whole sequences (sections "Ayrık Zamana Geçiş" and
+ * "Paralel Tarama Algoritması" of the page above), starting from h = 0.
+ *
+ *   u, delta     device, dtype, [batch][len][channels]       (x_t and Delta_t)
+ *   A            device, float32, [channels][nstate]
+ *   B, C         device, dtype, [batch][len][nstate]
+ *   D            device, float32, [channels], or NULL for no skip term
+ *   y            device, dtype, [batch][len][channels]       (output)
+ *   final_state  device, float32, [batch][channels][nstate], or NULL; receives
+ *                h after the last token (zeros when len == 0)
+ *   nstate       1..64 (see mamba_scan_supported_nstate)
+ *   stream       CUDA stream the work is ordered on
+ *
+ * Alignment: every pointer must be aligned to its element size.  Sequences
+ * with few (batch x channel) rows relative to the GPU are split into time
+ * chunks; that path allocates and frees stream-ordered scratch on `stream`
+ * (cudaMallocAsync / cudaFreeAsync) of about batch*channels*chunks*(nstate+1)
+ * floats.  batch == 0 or channels == 0 is a no-op that returns MAMBA_OK.
+ */
+int mamba_selective_scan(const void *u, const void *delta, const float *A,
+                         const void *B, const void *C, const float *D,
+                         void *y, float *final_state,
+                         int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                         int dtype, mamba_stream_t stream);
+
+/*
+ * As mamba_selective_scan, plus:
+ *   initial_state  device, float32, [batch][channels][nstate], or NULL (zeros):
+ *                  the scan resumes from this state (e.g. prefill continued in
+ *                  pieces, or a hand-off from recurrent decoding)
+ *   chunk_len      > 0: split every sequence into chunks of this many tokens
+ *                  (the associative chunk combine is then always used);
+ *                  0: chosen automatically
+ *   flags          bitwise OR of MAMBA_SCAN_* flags
+ */
+int mamba_selective_scan_ex(const void *u, const void *delta, const float *A,
+                            const void *B, const void *C, const float *D,
+                            const float *initial_state, void *y, float *final_state,
+                            int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                            int64_t chunk_len, unsigned flags,
+                            int dtype, mamba_stream_t stream);
+
+/*
+ * One recurrent step for every (batch, channel) row: the fixed-size-state
+ * update used for generation (section "Karmaşıklık Karşılaştırması": the
+ * hidden state does not grow with the sequence).  For each row and state n:
+ *   h_n <- exp(Delta A_n) h_n + (Delta A_n)^-1 (exp(Delta A_n) - 1) Delta B_n x
+ *   y    = sum_n C_n h_n + D x
+ *
+ *   state   device, float32, [batch][channels][nstate], updated in place
+ *   x, delta device, dtype, [batch][channels]
+ *   A       device, float32, [channels][nstate]
+ *   B, C    device, dtype, [batch][nstate]
+ *   D       device, float32, [channels], or NULL
+ *   y       device, dtype, [batch][channels] (output; must not overlap inputs)
+ */
+int mamba_state_update(float *state, const void *x, const void *delta,
+                       const float *A, const void *B, const void *C, const float *D,
+                       void *y, int64_t batch, int64_t channels, int64_t nstate,
+                       int dtype, mamba_stream_t stream);
+
+/* Static description of a status code (never NULL). */
+const char *mamba_status_string(int status);
+
+/* 1 if `nstate` is implemented by the scan and state-update kernels. */
+int mamba_scan_supported_nstate(int64_t nstate);
+
+/*
+ * Synchronises the current device, then returns the device error word
+ * (MAMBA_OK if no bounded wait has run out since the last clear).  With
+ * clear != 0 the word is reset to MAMBA_OK.
+ */
+int mamba_get_device_error(int clear);
+
+/*
+ * Diagnostic: enqueues one kernel that waits on a barrier nothing will ever
+ * complete, with a wait limit of `limit_ns` nanoseconds (clamped to
+ * [1 us, 1 s]).  The wait runs out, the kernel records MAMBA_ERR_TIMEOUT in
+ * the device error word and returns normally; the context stays usable.
+ * Used by the tests of the timeout path.
+ */
+int mamba_debug_expire_wait(int64_t limit_ns, mamba_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBA_SSM_H */

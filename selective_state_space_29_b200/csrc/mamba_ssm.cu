@@ -1,0 +1,368 @@
+// mamba_ssm.cu -- C ABI entry points: argument checks, planning of the
+// chunked scan, tensor-map set-up, stream-ordered scratch and launches.
+// Every arithmetic step of the path runs in the kernels of scan.cuh and
+// decode.cuh; nothing here touches tensor data on the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mamba_ssm.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "scan.cuh"
+
+namespace mamba {
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s: far above any legitimate wait
+
+int elem_size(int dtype) { return dtype == MAMBA_BF16 ? 2 : 4; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// --- device properties, cached per device ---------------------------------
+struct DeviceInfo {
+  int sms = 0;
+  bool ok = false;
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[64];
+
+int current_sms(int* sms) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MAMBA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (!g_dev[dev].ok) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MAMBA_ERR_CUDA;
+    g_dev[dev].sms = v;
+    g_dev[dev].ok = true;
+  }
+  *sms = g_dev[dev].sms;
+  return MAMBA_OK;
+}
+
+// --- tensor maps through the driver entry point (no link to libcuda) -------
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D map over a row-major [rows][cols] array, box [box_rows][box_cols].
+bool make_map_2d(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uint64_t rows, uint32_t box_cols,
+                 uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * (uint64_t)elem_size(dtype)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt =
+      dtype == MAMBA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// --- scan configuration per element type -----------------------------------
+template <typename TIO>
+struct ScanCfg;
+template <>
+struct ScanCfg<__nv_bfloat16> {
+  static constexpr int kTile = 32, kStages = 4;
+};
+template <>
+struct ScanCfg<float> {
+  static constexpr int kTile = 16, kStages = 4;
+};
+
+struct Plan {
+  int supers = 1;
+  int64_t super_len = 0;
+  int64_t chunk_len = 0;
+  int chunks_full = 1, chunks_last = 1;
+};
+
+Plan plan_scan(int64_t len, int groups, int warps_total, int tile, int64_t user_chunk) {
+  Plan pl;
+  if (user_chunk > 0) {
+    pl.super_len = std::min<int64_t>(user_chunk, len);
+  } else {
+    int64_t s = 1;
+    if (groups < warps_total) s = (warps_total + groups - 1) / groups;
+    s = std::min<int64_t>(s, std::max<int64_t>(1, len / (4 * tile)));
+    pl.super_len = (len + s - 1) / s;
+    pl.super_len = ((pl.super_len + tile - 1) / tile) * tile;
+  }
+  pl.super_len = std::max<int64_t>(1, pl.super_len);
+  pl.supers = (int)((len + pl.super_len - 1) / pl.super_len);
+  // chunks inside a super-chunk: enough jobs (about 8 per warp) for balance,
+  // but at least two tiles per job
+  const int64_t streams = (int64_t)pl.supers * groups;
+  int64_t k = (8LL * warps_total + streams - 1) / streams;
+  k = std::max<int64_t>(1, std::min<int64_t>(k, pl.super_len / (2 * tile)));
+  int64_t cl = (pl.super_len + k - 1) / k;
+  cl = ((cl + tile - 1) / tile) * tile;
+  pl.chunk_len = std::max<int64_t>(1, std::min<int64_t>(cl, pl.super_len));
+  pl.chunks_full = (int)((pl.super_len + pl.chunk_len - 1) / pl.chunk_len);
+  const int64_t last_len = len - (int64_t)(pl.supers - 1) * pl.super_len;
+  pl.chunks_last = (int)((last_len + pl.chunk_len - 1) / pl.chunk_len);
+  return pl;
+}
+
+template <typename TIO, int NS>
+int launch_scan(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
+                const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
+                int64_t user_chunk, unsigned flags, int dtype, cudaStream_t stream) {
+  constexpr int TILE = ScanCfg<TIO>::kTile;
+  constexpr int STAGES = ScanCfg<TIO>::kStages;
+  int sms = 0;
+  if (int st = current_sms(&sms)) return st;
+  const int warps_total = sms * kWarpsPerCta;
+  const int groups_d = (int)((channels + kGroup - 1) / kGroup);
+  const int64_t groups64 = batch * groups_d;
+  if (groups64 > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
+  const int groups = (int)groups64;
+  const Plan pl = plan_scan(len, groups, warps_total, TILE, user_chunk);
+
+  const size_t es = sizeof(TIO);
+  const bool use_tma = aligned(u, 16) && aligned(delta, 16) && aligned(B, 16) && aligned(C, 16) &&
+                       (channels * (int64_t)es) % 16 == 0 && (NS * es) % 16 == 0 && encode_fn() != nullptr;
+  CUtensorMap mu, mdl, mb, mc;
+  std::memset(&mu, 0, sizeof(mu));
+  std::memset(&mdl, 0, sizeof(mdl));
+  std::memset(&mb, 0, sizeof(mb));
+  std::memset(&mc, 0, sizeof(mc));
+  bool tma = use_tma;
+  if (tma) {
+    const uint64_t rows = (uint64_t)batch * (uint64_t)len;
+    tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
+          make_map_2d(&mdl, delta, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
+          make_map_2d(&mb, B, dtype, NS, rows, NS, TILE) && make_map_2d(&mc, C, dtype, NS, rows, NS, TILE);
+  }
+
+  // scratch: [counters x2][done x2][ring][ring_sd][agg_h][agg_sd][hin]
+  const int64_t S = pl.supers;
+  const int64_t streams_full = S * groups;
+  const int64_t streams_agg = (S - 1) * groups;
+  auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+  const size_t sz_ctr = al(4 * sizeof(int));
+  const size_t sz_done = al(sizeof(int) * (size_t)(streams_full + streams_agg));
+  const size_t sz_ring = al(sizeof(float) * (size_t)streams_full * 2 * kGroup * NS);
+  const size_t sz_ring_sd = al(sizeof(float) * (size_t)streams_full * 2 * kGroup);
+  const size_t sz_agg_h = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup * NS);
+  const size_t sz_agg_sd = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup);
+  const size_t sz_hin = S > 1 ? al(sizeof(float) * (size_t)streams_full * kGroup * NS) : 0;
+  const size_t total = sz_ctr + sz_done + sz_ring + sz_ring_sd + sz_agg_h + sz_agg_sd + sz_hin;
+  unsigned char* scratch = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+  unsigned char* cur = scratch;
+  int* counters = reinterpret_cast<int*>(cur); cur += sz_ctr;
+  int* done = reinterpret_cast<int*>(cur); cur += sz_done;
+  float* ring = reinterpret_cast<float*>(cur); cur += sz_ring;
+  float* ring_sd = reinterpret_cast<float*>(cur); cur += sz_ring_sd;
+  float* agg_h = reinterpret_cast<float*>(cur); cur += sz_agg_h;
+  float* agg_sd = reinterpret_cast<float*>(cur); cur += sz_agg_sd;
+  float* hin = sz_hin ? reinterpret_cast<float*>(cur) : nullptr;
+  int status = MAMBA_OK;
+  if (cudaMemsetAsync(scratch, 0, sz_ctr + sz_done, stream) != cudaSuccess) status = MAMBA_ERR_CUDA;
+
+  ScanParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.h0 = h0; p.y = y;
+  p.final_state = final_state;
+  p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd; p.hin = hin;
+  p.batch = batch; p.len = len; p.channels = channels;
+  p.groups_d = groups_d; p.groups = groups;
+  p.supers = pl.supers; p.super_len = pl.super_len; p.chunk_len = pl.chunk_len;
+  p.chunks_full = pl.chunks_full; p.chunks_last = pl.chunks_last;
+  p.use_tma = tma ? 1 : 0;
+  p.force_general = (flags & MAMBA_SCAN_GENERAL_A) ? 1 : 0;
+  p.wait_limit_ns = kWaitLimitNs;
+
+  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES>();
+  auto kern = scan_chunks_kernel<TIO, NS, TILE, STAGES>;
+  static bool attr_set = false;  // per instantiation
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+      status = MAMBA_ERR_CUDA;
+    else
+      attr_set = true;
+  }
+
+  auto run_pass = [&](int mode, int streams, int64_t jobs, int* ctr, int* dn) {
+    if (status != MAMBA_OK || jobs <= 0) return;
+    ScanParams q = p;
+    q.mode = mode;
+    q.streams = streams;
+    q.jobs = jobs;
+    q.counters = ctr;
+    q.done = dn;
+    const int64_t ctas = std::min<int64_t>(sms, (jobs + kWarpsPerCta - 1) / kWarpsPerCta);
+    kern<<<(unsigned)ctas, kWarpsPerCta * 32, smem, stream>>>(q, mu, mdl, mb, mc);
+    if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
+  };
+
+  if (S > 1) {
+    // aggregate pass over every super-chunk but the last, then the combine
+    run_pass(kModeAggregate, (int)streams_agg, streams_agg * pl.chunks_full, counters + 2, done + streams_full);
+    if (status == MAMBA_OK) {
+      const int64_t threads = (int64_t)groups * kGroup * NS;
+      scan_combine_kernel<NS><<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p, hin);
+      if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
+    }
+  }
+  const int64_t jobs_full =
+      (int64_t)pl.chunks_last * streams_full + (int64_t)(pl.chunks_full - pl.chunks_last) * streams_agg;
+  run_pass(kModeFull, (int)streams_full, jobs_full, counters, done);
+
+  if (cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) status = MAMBA_ERR_CUDA;
+  return status;
+}
+
+__global__ void expire_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    // nothing ever arrives on `bar`: the bounded wait must run out
+    if (!mbar_wait_bounded(&bar, 0, limit_ns)) record_device_error(MAMBA_ERR_TIMEOUT);
+  }
+}
+
+}  // namespace
+}  // namespace mamba
+
+using namespace mamba;
+
+extern "C" {
+
+const char* mamba_status_string(int status) {
+  switch (status) {
+    case MAMBA_OK: return "ok";
+    case MAMBA_ERR_INVALID_ARG: return "invalid argument";
+    case MAMBA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MAMBA_ERR_CUDA: return "CUDA error";
+    case MAMBA_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int mamba_scan_supported_nstate(int64_t nstate) { return nstate == 16 ? 1 : 0; }
+
+int mamba_selective_scan_ex(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                            const float* D, const float* initial_state, void* y, float* final_state,
+                            int64_t batch, int64_t len, int64_t channels, int64_t nstate, int64_t chunk_len,
+                            unsigned flags, int dtype, mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || len < 0 || channels < 0 || nstate <= 0 || chunk_len < 0) return MAMBA_ERR_INVALID_ARG;
+  if (flags & ~MAMBA_SCAN_GENERAL_A) return MAMBA_ERR_INVALID_ARG;
+  if (!mamba_scan_supported_nstate(nstate)) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || channels == 0) return MAMBA_OK;
+  const size_t es = (size_t)elem_size(dtype);
+  if (len > 0) {
+    if (!u || !delta || !B || !C || !y || !A) return MAMBA_ERR_INVALID_ARG;
+    if (!aligned(u, es) || !aligned(delta, es) || !aligned(B, es) || !aligned(C, es) || !aligned(y, es))
+      return MAMBA_ERR_INVALID_ARG;
+  }
+  if ((A && !aligned(A, 4)) || (D && !aligned(D, 4)) || (final_state && !aligned(final_state, 4)) ||
+      (initial_state && !aligned(initial_state, 4)))
+    return MAMBA_ERR_INVALID_ARG;
+  if (batch * len >= (int64_t(1) << 31) || channels >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+
+  cudaGetLastError();  // clear a stale, non-sticky error so the status below is ours
+  const size_t state_bytes = sizeof(float) * (size_t)batch * (size_t)channels * (size_t)nstate;
+  if (len == 0) {
+    if (!final_state) return MAMBA_OK;
+    cudaError_t e = initial_state
+                        ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, stream)
+                        : cudaMemsetAsync(final_state, 0, state_bytes, stream);
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+  }
+  if (dtype == MAMBA_BF16)
+    return launch_scan<__nv_bfloat16, 16>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels,
+                                          chunk_len, flags, dtype, stream);
+  return launch_scan<float, 16>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels, chunk_len,
+                                flags, dtype, stream);
+}
+
+int mamba_selective_scan(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                         const float* D, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
+                         int64_t nstate, int dtype, mamba_stream_t stream) {
+  return mamba_selective_scan_ex(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, nstate, 0, 0u,
+                                 dtype, stream);
+}
+
+int mamba_state_update(float* state, const void* x, const void* delta, const float* A, const void* B, const void* C,
+                       const float* D, void* y, int64_t batch, int64_t channels, int64_t nstate, int dtype,
+                       mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || channels < 0 || nstate <= 0) return MAMBA_ERR_INVALID_ARG;
+  if (!mamba_scan_supported_nstate(nstate)) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || channels == 0) return MAMBA_OK;
+  if (!state || !x || !delta || !A || !B || !C || !y) return MAMBA_ERR_INVALID_ARG;
+  const size_t es = (size_t)elem_size(dtype);
+  if (!aligned(state, 16) || !aligned(A, 16) || (D && !aligned(D, 4)) || !aligned(x, es) || !aligned(delta, es) ||
+      !aligned(y, es) || !aligned(B, 4 * es) || !aligned(C, 4 * es))
+    return MAMBA_ERR_INVALID_ARG;
+  int sms = 0;
+  if (int st = current_sms(&sms)) return st;
+  cudaGetLastError();
+  const int64_t rows = batch * channels;
+  constexpr int kThreads = 256, kRowsPerThread = 2;
+  const int64_t row_groups = (rows + 7) / 8;  // a warp covers 8 rows per access
+  int64_t blocks = (row_groups + (kThreads / 32) * kRowsPerThread - 1) / ((kThreads / 32) * kRowsPerThread);
+  blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, (int64_t)sms * 64));
+  if (dtype == MAMBA_BF16) {
+    DecodeArgs<__nv_bfloat16, 16> a{state, static_cast<const __nv_bfloat16*>(x),
+                                    static_cast<const __nv_bfloat16*>(delta), A,
+                                    static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
+                                    static_cast<__nv_bfloat16*>(y), batch, channels};
+    state_update_kernel<__nv_bfloat16, 16, kRowsPerThread><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+  } else {
+    DecodeArgs<float, 16> a{state, static_cast<const float*>(x), static_cast<const float*>(delta), A,
+                            static_cast<const float*>(B), static_cast<const float*>(C), D,
+                            static_cast<float*>(y), batch, channels};
+    state_update_kernel<float, 16, kRowsPerThread><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+  }
+  return cudaGetLastError() == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+int mamba_get_device_error(int clear) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return MAMBA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return MAMBA_ERR_CUDA;
+  if (clear) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &z, sizeof(int)) != cudaSuccess) return MAMBA_ERR_CUDA;
+  }
+  return v;
+}
+
+int mamba_debug_expire_wait(int64_t limit_ns, mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  const int64_t lim = std::min<int64_t>(std::max<int64_t>(limit_ns, 1000), 1000000000);
+  cudaGetLastError();
+  expire_wait_kernel<<<1, 32, 0, stream>>>((uint64_t)lim);
+  return cudaGetLastError() == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+}
+
+}  // extern "C"

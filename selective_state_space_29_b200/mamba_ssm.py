@@ -1,0 +1,181 @@
+"""Python binding of the C ABI in include/mamba_ssm.h (argument marshalling only).
+
+Every function named like a C entry point forwards its arguments to the
+library unchanged: tensors become device pointers, torch streams become
+`cudaStream_t` handles, a non-zero status raises `MambaError`.  The
+tensor-level helpers `selective_scan` and `state_update` only allocate the
+outputs with torch and then make the same C calls.  There is no fallback: if
+the library is missing or cannot load, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG_DIR, "libmamba_ssm_b200.so")
+
+MAMBA_F32 = 0
+MAMBA_BF16 = 1
+MAMBA_OK = 0
+MAMBA_ERR_INVALID_ARG = 1
+MAMBA_ERR_UNSUPPORTED = 2
+MAMBA_ERR_CUDA = 3
+MAMBA_ERR_TIMEOUT = 4
+MAMBA_SCAN_GENERAL_A = 1
+
+# (name, restype, argtypes) for every entry point of include/mamba_ssm.h
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIGNATURES = [
+    ("mamba_selective_scan", ctypes.c_int,
+     [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int, _P]),
+    ("mamba_selective_scan_ex", ctypes.c_int,
+     [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_uint, ctypes.c_int, _P]),
+    ("mamba_state_update", ctypes.c_int,
+     [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P]),
+    ("mamba_status_string", ctypes.c_char_p, [ctypes.c_int]),
+    ("mamba_scan_supported_nstate", ctypes.c_int, [_I64]),
+    ("mamba_get_device_error", ctypes.c_int, [ctypes.c_int]),
+    ("mamba_debug_expire_wait", ctypes.c_int, [_I64, _P]),
+]
+
+
+class MambaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def library() -> ctypes.CDLL:
+    """Load libmamba_ssm_b200.so (built by `python -m selective_state_space_29_b200.build`)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing; build it with "
+                              "`python -m selective_state_space_29_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, res, args in _SIGNATURES:
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return library().mamba_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, what: str):
+    if status != MAMBA_OK:
+        raise MambaError(status, what)
+
+
+def dtype_code(torch_dtype) -> int:
+    import torch
+    if torch_dtype == torch.float32:
+        return MAMBA_F32
+    if torch_dtype == torch.bfloat16:
+        return MAMBA_BF16
+    raise ValueError(f"unsupported dtype {torch_dtype}")
+
+
+# --- the C entry points -------------------------------------------------------
+
+def mamba_selective_scan(u, delta, A, B, C, D, y, final_state, batch, len, channels, nstate, dtype,
+                         stream=None):
+    st = library().mamba_selective_scan(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
+                                        _ptr(final_state), batch, len, channels, nstate, dtype,
+                                        _stream(stream))
+    _check(st, "mamba_selective_scan")
+
+
+def mamba_selective_scan_ex(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels, nstate,
+                            chunk_len, flags, dtype, stream=None):
+    st = library().mamba_selective_scan_ex(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                           _ptr(initial_state), _ptr(y), _ptr(final_state), batch, len,
+                                           channels, nstate, chunk_len, flags, dtype, _stream(stream))
+    _check(st, "mamba_selective_scan_ex")
+
+
+def mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, dtype, stream=None):
+    st = library().mamba_state_update(_ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                      _ptr(y), batch, channels, nstate, dtype, _stream(stream))
+    _check(st, "mamba_state_update")
+
+
+def mamba_status_string(status: int) -> str:
+    return status_string(status)
+
+
+def mamba_scan_supported_nstate(nstate: int) -> bool:
+    return bool(library().mamba_scan_supported_nstate(int(nstate)))
+
+
+def mamba_get_device_error(clear: bool = False) -> int:
+    return int(library().mamba_get_device_error(1 if clear else 0))
+
+
+def mamba_debug_expire_wait(limit_ns: int, stream=None):
+    _check(library().mamba_debug_expire_wait(int(limit_ns), _stream(stream)), "mamba_debug_expire_wait")
+
+
+# --- tensor-level helpers ---------------------------------------------------------
+
+def selective_scan(u, delta, A, B, C, D=None, initial_state=None, return_final_state=True, chunk_len=0,
+                   general_a=False, y=None, final_state=None, stream=None):
+    """y, final_state = selective_scan(u, delta, A, B, C, D) on CUDA tensors.
+
+    u, delta: (batch, len, channels); B, C: (batch, len, nstate) of one dtype
+    (float32 or bfloat16); A: (channels, nstate) float32; D: (channels,) or
+    None; initial_state: (batch, channels, nstate) float32 or None."""
+    import torch
+    batch, length, channels = u.shape
+    nstate = A.shape[1]
+    for t in (u, delta, A, B, C, D, initial_state):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if y is None:
+        y = torch.empty_like(u)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((batch, channels, nstate), device=u.device, dtype=torch.float32)
+    flags = MAMBA_SCAN_GENERAL_A if general_a else 0
+    if initial_state is None and chunk_len == 0 and flags == 0:
+        mamba_selective_scan(u, delta, A, B, C, D, y, final_state, batch, length, channels, nstate,
+                             dtype_code(u.dtype), stream)
+    else:
+        mamba_selective_scan_ex(u, delta, A, B, C, D, initial_state, y, final_state, batch, length, channels,
+                                nstate, chunk_len, flags, dtype_code(u.dtype), stream)
+    return y, final_state
+
+
+def state_update(state, x, delta, A, B, C, D=None, y=None, stream=None):
+    """One recurrent step in place on `state` (batch, channels, nstate) float32;
+    returns y (batch, channels) in the dtype of x."""
+    import torch
+    batch, channels, nstate = state.shape
+    if y is None:
+        y = torch.empty_like(x)
+    mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, dtype_code(x.dtype), stream)
+    return y

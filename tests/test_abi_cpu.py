@@ -1,0 +1,116 @@
+"""Host-side checks of the C ABI (no GPU needed, no compute calls).
+
+The library is built in-tree for sm_100a (nvcc cross-compiles without a GPU),
+loaded with ctypes, and every entry point that include/mamba_ssm.h declares
+must be exported.  Only calls that return before touching the device are
+made here: status strings, the supported-nstate query, and argument checks
+that reject or short-circuit a call on the host.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from selective_state_space_29_b200 import build as lib_build
+from selective_state_space_29_b200 import mamba_ssm as m
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mamba_ssm.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    lib_build.build()
+    return m.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mamba_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for want in ("mamba_selective_scan", "mamba_selective_scan_ex", "mamba_state_update",
+                 "mamba_status_string", "mamba_get_device_error"):
+        assert want in names
+
+
+def test_library_exports_every_declared_function(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/mamba_ssm.h but not exported"
+    # and the binding wraps each of them under the same name
+    for name in declared_functions():
+        assert hasattr(m, name), f"binding lacks {name}"
+
+
+def test_status_strings(lib):
+    assert m.status_string(m.MAMBA_OK) == "ok"
+    assert "invalid" in m.status_string(m.MAMBA_ERR_INVALID_ARG)
+    assert "timed out" in m.status_string(m.MAMBA_ERR_TIMEOUT)
+    assert m.status_string(12345) == "unknown status"
+
+
+def test_supported_nstate(lib):
+    assert m.mamba_scan_supported_nstate(16)
+    assert not m.mamba_scan_supported_nstate(0)
+    assert not m.mamba_scan_supported_nstate(17)
+
+
+def _scan_ex(lib, **kw):
+    a = dict(u=1024, delta=1024, A=1024, B=1024, C=1024, D=None, h0=None, y=2048, fs=None, batch=1, len=4,
+             channels=8, nstate=16, chunk=0, flags=0, dtype=m.MAMBA_BF16)
+    a.update(kw)
+    return lib.mamba_selective_scan_ex(a["u"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["h0"], a["y"],
+                                       a["fs"], a["batch"], a["len"], a["channels"], a["nstate"], a["chunk"],
+                                       a["flags"], a["dtype"], None)
+
+
+def test_scan_argument_errors_on_host(lib):
+    # every case below is rejected before any CUDA call is made
+    assert _scan_ex(lib, dtype=7) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, batch=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, len=-3) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, channels=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, chunk=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, flags=8) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, nstate=0) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, nstate=12) == m.MAMBA_ERR_UNSUPPORTED
+    assert _scan_ex(lib, u=None) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, y=None) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, A=None) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, u=1025) == m.MAMBA_ERR_INVALID_ARG            # misaligned bf16 pointer
+    assert _scan_ex(lib, dtype=m.MAMBA_F32, u=1026) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, batch=1 << 20, len=1 << 12) == m.MAMBA_ERR_UNSUPPORTED   # batch*len >= 2^31
+    # empty problems are valid no-ops
+    assert _scan_ex(lib, batch=0) == m.MAMBA_OK
+    assert _scan_ex(lib, channels=0) == m.MAMBA_OK
+    assert _scan_ex(lib, len=0, fs=None) == m.MAMBA_OK
+
+
+def test_state_update_argument_errors_on_host(lib):
+    f = lib.mamba_state_update
+    ok = dict(state=4096, x=1024, delta=1024, A=4096, B=1024, C=1024, D=None, y=2048, batch=2, channels=8,
+              nstate=16, dtype=m.MAMBA_BF16)
+
+    def call(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return f(a["state"], a["x"], a["delta"], a["A"], a["B"], a["C"], a["D"], a["y"], a["batch"],
+                 a["channels"], a["nstate"], a["dtype"], None)
+
+    assert call(dtype=3) == m.MAMBA_ERR_INVALID_ARG
+    assert call(batch=-2) == m.MAMBA_ERR_INVALID_ARG
+    assert call(nstate=8) == m.MAMBA_ERR_UNSUPPORTED
+    assert call(state=None) == m.MAMBA_ERR_INVALID_ARG
+    assert call(state=4100) == m.MAMBA_ERR_INVALID_ARG                   # state must be 16-byte aligned
+    assert call(B=1026) == m.MAMBA_ERR_INVALID_ARG
+    assert call(batch=0) == m.MAMBA_OK
+
+
+def test_library_links_no_torch(lib):
+    # the product library is plain C ABI over CUDA: no torch / python symbols needed
+    out = os.popen(f"nm -D --undefined-only {lib_build.LIB}").read()
+    assert "torch" not in out and "Py" not in out
