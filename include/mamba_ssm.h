@@ -84,14 +84,18 @@ typedef enum {
  *   y            device, dtype, [batch][len][channels]       (output)
  *   final_state  device, float32, [batch][channels][nstate], or NULL; receives
  *                h after the last token (zeros when len == 0)
- *   nstate       1..64 (see mamba_scan_supported_nstate)
+ *   nstate       number of states per channel; 16 in this build
+ *                (mamba_scan_supported_nstate tells)
  *   stream       CUDA stream the work is ordered on
  *
- * Alignment: every pointer must be aligned to its element size.  Sequences
- * with few (batch x channel) rows relative to the GPU are split into time
- * chunks; that path allocates and frees stream-ordered scratch on `stream`
- * (cudaMallocAsync / cudaFreeAsync) of about batch*channels*chunks*(nstate+1)
- * floats.  batch == 0 or channels == 0 is a no-op that returns MAMBA_OK.
+ * Alignment: every pointer must be aligned to its element size; tiles are
+ * staged with TMA when u, delta, B and C are 16-byte aligned and a row of
+ * channels is a multiple of 16 bytes, with plain loads otherwise.
+ * Scratch: every call allocates and frees stream-ordered scratch on `stream`
+ * (cudaMallocAsync / cudaFreeAsync): job counters, the buffer that hands the
+ * state from one time chunk to the next, and, when sequences are split into
+ * independent super-chunks, their aggregates (mamba_scan_plan reports the
+ * size).  batch == 0 or channels == 0 is a no-op that returns MAMBA_OK.
  */
 int mamba_selective_scan(const void *u, const void *delta, const float *A,
                          const void *B, const void *C, const float *D,
@@ -129,11 +133,33 @@ int mamba_selective_scan_ex(const void *u, const void *delta, const float *A,
  *   B, C    device, dtype, [batch][nstate]
  *   D       device, float32, [channels], or NULL
  *   y       device, dtype, [batch][channels] (output; must not overlap inputs)
+ *
+ * Alignment: state and A 16-byte aligned; B and C aligned to 4 elements;
+ * the rest to their element size.  No scratch memory is used.
  */
 int mamba_state_update(float *state, const void *x, const void *delta,
                        const float *A, const void *B, const void *C, const float *D,
                        void *y, int64_t batch, int64_t channels, int64_t nstate,
                        int dtype, mamba_stream_t stream);
+
+/* How mamba_selective_scan_ex would split a problem (host-side planning only). */
+typedef struct {
+    int64_t supers;        /* independent super-chunks per sequence (1: no aggregate/combine pass) */
+    int64_t super_len;     /* tokens per super-chunk (all but the last) */
+    int64_t chunk_len;     /* tokens per job of the main pass */
+    int64_t jobs;          /* jobs of the main pass */
+    int64_t kernels;       /* kernels one call launches */
+    int64_t scratch_bytes; /* stream-ordered scratch one call allocates */
+    int64_t ctas;          /* CTAs of the main pass (persistent: at most one per SM) */
+} mamba_scan_plan_t;
+
+/*
+ * Fills *out with the split that a scan of this shape would use.
+ * sm_count > 0 plans for that many SMs; sm_count <= 0 queries the current
+ * device.  Makes no device calls when sm_count > 0.
+ */
+int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate, int64_t chunk_len,
+                    int dtype, int sm_count, mamba_scan_plan_t *out);
 
 /* Static description of a status code (never NULL). */
 const char *mamba_status_string(int status);

@@ -126,6 +126,35 @@ Plan plan_scan(int64_t len, int groups, int warps_total, int tile, int64_t user_
   return pl;
 }
 
+struct ScratchLayout {
+  size_t ctr, done, ring, ring_sd, agg_h, agg_sd, hin, total;
+};
+
+ScratchLayout scratch_layout(const Plan& pl, int groups, int ns) {
+  auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+  const int64_t S = pl.supers;
+  const int64_t streams_full = S * groups;
+  const int64_t streams_agg = (S - 1) * groups;
+  ScratchLayout s;
+  s.ctr = al(4 * sizeof(int));
+  s.done = al(sizeof(int) * (size_t)(streams_full + streams_agg));
+  s.ring = al(sizeof(float) * (size_t)streams_full * 2 * kGroup * ns);
+  s.ring_sd = al(sizeof(float) * (size_t)streams_full * 2 * kGroup);
+  s.agg_h = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup * ns);
+  s.agg_sd = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup);
+  s.hin = S > 1 ? al(sizeof(float) * (size_t)streams_full * kGroup * ns) : 0;
+  s.total = s.ctr + s.done + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.hin;
+  return s;
+}
+
+int64_t full_jobs(const Plan& pl, int groups) {
+  const int64_t streams_full = (int64_t)pl.supers * groups;
+  const int64_t streams_agg = (int64_t)(pl.supers - 1) * groups;
+  return (int64_t)pl.chunks_last * streams_full + (int64_t)(pl.chunks_full - pl.chunks_last) * streams_agg;
+}
+
+int tile_for(int dtype) { return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16>::kTile : ScanCfg<float>::kTile; }
+
 template <typename TIO, int NS>
 int launch_scan(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
                 const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
@@ -161,27 +190,19 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   const int64_t S = pl.supers;
   const int64_t streams_full = S * groups;
   const int64_t streams_agg = (S - 1) * groups;
-  auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
-  const size_t sz_ctr = al(4 * sizeof(int));
-  const size_t sz_done = al(sizeof(int) * (size_t)(streams_full + streams_agg));
-  const size_t sz_ring = al(sizeof(float) * (size_t)streams_full * 2 * kGroup * NS);
-  const size_t sz_ring_sd = al(sizeof(float) * (size_t)streams_full * 2 * kGroup);
-  const size_t sz_agg_h = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup * NS);
-  const size_t sz_agg_sd = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup);
-  const size_t sz_hin = S > 1 ? al(sizeof(float) * (size_t)streams_full * kGroup * NS) : 0;
-  const size_t total = sz_ctr + sz_done + sz_ring + sz_ring_sd + sz_agg_h + sz_agg_sd + sz_hin;
+  const ScratchLayout sl = scratch_layout(pl, groups, NS);
   unsigned char* scratch = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
   unsigned char* cur = scratch;
-  int* counters = reinterpret_cast<int*>(cur); cur += sz_ctr;
-  int* done = reinterpret_cast<int*>(cur); cur += sz_done;
-  float* ring = reinterpret_cast<float*>(cur); cur += sz_ring;
-  float* ring_sd = reinterpret_cast<float*>(cur); cur += sz_ring_sd;
-  float* agg_h = reinterpret_cast<float*>(cur); cur += sz_agg_h;
-  float* agg_sd = reinterpret_cast<float*>(cur); cur += sz_agg_sd;
-  float* hin = sz_hin ? reinterpret_cast<float*>(cur) : nullptr;
+  int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
+  int* done = reinterpret_cast<int*>(cur); cur += sl.done;
+  float* ring = reinterpret_cast<float*>(cur); cur += sl.ring;
+  float* ring_sd = reinterpret_cast<float*>(cur); cur += sl.ring_sd;
+  float* agg_h = reinterpret_cast<float*>(cur); cur += sl.agg_h;
+  float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
+  float* hin = sl.hin ? reinterpret_cast<float*>(cur) : nullptr;
   int status = MAMBA_OK;
-  if (cudaMemsetAsync(scratch, 0, sz_ctr + sz_done, stream) != cudaSuccess) status = MAMBA_ERR_CUDA;
+  if (cudaMemsetAsync(scratch, 0, sl.ctr + sl.done, stream) != cudaSuccess) status = MAMBA_ERR_CUDA;
 
   ScanParams p;
   std::memset(&p, 0, sizeof(p));
@@ -228,9 +249,7 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
       if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
     }
   }
-  const int64_t jobs_full =
-      (int64_t)pl.chunks_last * streams_full + (int64_t)(pl.chunks_full - pl.chunks_last) * streams_agg;
-  run_pass(kModeFull, (int)streams_full, jobs_full, counters, done);
+  run_pass(kModeFull, (int)streams_full, full_jobs(pl, groups), counters, done);
 
   if (cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) status = MAMBA_ERR_CUDA;
   return status;
@@ -265,6 +284,29 @@ const char* mamba_status_string(int status) {
 }
 
 int mamba_scan_supported_nstate(int64_t nstate) { return nstate == 16 ? 1 : 0; }
+
+int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate, int64_t chunk_len, int dtype,
+                    int sm_count, mamba_scan_plan_t* out) {
+  if (!out || (dtype != MAMBA_F32 && dtype != MAMBA_BF16)) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || len < 0 || channels < 0 || nstate <= 0 || chunk_len < 0) return MAMBA_ERR_INVALID_ARG;
+  if (!mamba_scan_supported_nstate(nstate)) return MAMBA_ERR_UNSUPPORTED;
+  std::memset(out, 0, sizeof(*out));
+  if (batch == 0 || channels == 0 || len == 0) return MAMBA_OK;  // nothing is launched
+  int sms = sm_count;
+  if (sms <= 0) {
+    if (int st = current_sms(&sms)) return st;
+  }
+  const int groups = (int)(batch * ((channels + kGroup - 1) / kGroup));
+  const Plan pl = plan_scan(len, groups, sms * kWarpsPerCta, tile_for(dtype), chunk_len);
+  out->supers = pl.supers;
+  out->super_len = pl.super_len;
+  out->chunk_len = pl.chunk_len;
+  out->jobs = full_jobs(pl, groups);
+  out->kernels = pl.supers > 1 ? 3 : 1;
+  out->scratch_bytes = (int64_t)scratch_layout(pl, groups, (int)nstate).total;
+  out->ctas = std::min<int64_t>(sms, (out->jobs + kWarpsPerCta - 1) / kWarpsPerCta);
+  return MAMBA_OK;
+}
 
 int mamba_selective_scan_ex(const void* u, const void* delta, const float* A, const void* B, const void* C,
                             const float* D, const float* initial_state, void* y, float* final_state,

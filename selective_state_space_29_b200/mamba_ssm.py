@@ -24,6 +24,16 @@ MAMBA_ERR_CUDA = 3
 MAMBA_ERR_TIMEOUT = 4
 MAMBA_SCAN_GENERAL_A = 1
 
+class ScanPlan(ctypes.Structure):
+    """mamba_scan_plan_t"""
+    _fields_ = [("supers", ctypes.c_int64), ("super_len", ctypes.c_int64), ("chunk_len", ctypes.c_int64),
+                ("jobs", ctypes.c_int64), ("kernels", ctypes.c_int64), ("scratch_bytes", ctypes.c_int64),
+                ("ctas", ctypes.c_int64)]
+
+    def as_dict(self):
+        return {k: int(getattr(self, k)) for k, _ in self._fields_}
+
+
 # (name, restype, argtypes) for every entry point of include/mamba_ssm.h
 _P = ctypes.c_void_p
 _I64 = ctypes.c_int64
@@ -34,6 +44,8 @@ _SIGNATURES = [
      [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_uint, ctypes.c_int, _P]),
     ("mamba_state_update", ctypes.c_int,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P]),
+    ("mamba_scan_plan", ctypes.c_int,
+     [_I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ScanPlan)]),
     ("mamba_status_string", ctypes.c_char_p, [ctypes.c_int]),
     ("mamba_scan_supported_nstate", ctypes.c_int, [_I64]),
     ("mamba_get_device_error", ctypes.c_int, [ctypes.c_int]),
@@ -123,6 +135,13 @@ def mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, 
     st = library().mamba_state_update(_ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
                                       _ptr(y), batch, channels, nstate, dtype, _stream(stream))
     _check(st, "mamba_state_update")
+
+
+def mamba_scan_plan(batch, len, channels, nstate, chunk_len, dtype, sm_count=0) -> ScanPlan:
+    out = ScanPlan()
+    _check(library().mamba_scan_plan(batch, len, channels, nstate, chunk_len, dtype, sm_count,
+                                     ctypes.byref(out)), "mamba_scan_plan")
+    return out
 
 
 def mamba_status_string(status: int) -> str:

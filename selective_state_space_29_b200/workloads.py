@@ -187,6 +187,19 @@ def decode_step_inputs(w: DecodeWorkload, step: int, device="cpu", seed: int | N
     return {"x": x, "delta": delta, "B": B, "C": C}
 
 
+def decode_chain_inputs_bulk(w: DecodeWorkload, steps: int, device="cpu", seed: int | None = None) -> dict:
+    """`steps` steps of fresh inputs drawn in one go (a different random stream
+    from decode_step_inputs, same distributions): x, delta (steps, batch,
+    channels); B, C (steps, batch, nstate)."""
+    s = w.seed if seed is None else seed
+    dt = w.torch_dtype
+    return {"x": _normal((steps, w.batch, w.channels), _gen(device, s, 901), device, dt),
+            "delta": _log_uniform((steps, w.batch, w.channels), _gen(device, s, 902), device, dt,
+                                  w.delta_lo, w.delta_hi),
+            "B": _normal((steps, w.batch, w.nstate), _gen(device, s, 903), device, dt),
+            "C": _normal((steps, w.batch, w.nstate), _gen(device, s, 904), device, dt)}
+
+
 def decode_chain_inputs(w: DecodeWorkload, device="cpu", seed: int | None = None) -> dict:
     """All steps' inputs stacked: x, delta (steps, batch, channels); B, C
     (steps, batch, nstate)."""
