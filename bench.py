@@ -199,13 +199,24 @@ def barrier(dist, world):
         dist.barrier()
 
 
-def max_over_ranks(dist, world, value: float) -> float:
+def max_over_ranks(dist, world, value: float, device="cuda") -> float:
+    """Slowest rank's time: every rank calls this at the same point."""
     if world == 1:
         return value
     import torch
-    t = torch.tensor([value], device="cuda", dtype=torch.float64)
+    t = torch.tensor([value], device=device, dtype=torch.float64)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def weak_scaling_value(world: int, units_per_rank: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput: units all ranks processed / the slowest rank's time."""
+    return world * units_per_rank / (ms_per_step_max * 1e-3)
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own independent workload."""
+    return base + 1000 * rank
 
 
 # --- algorithmic work -------------------------------------------------------------------
@@ -286,7 +297,7 @@ def run_ours(args):
     hbm_src = "measured" if "hbm_gbs" in peaks else "fallback"
 
     w = wl.SCAN_WORKLOADS[args.workload]
-    inp = wl.scan_inputs(w, dev, seed=w.seed + 1000 * rank)
+    inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
     y = torch.empty_like(inp["u"])
     hf = torch.empty((w.batch, w.channels, w.nstate), device=dev, dtype=torch.float32)
     dtc = m.dtype_code(w.torch_dtype)
@@ -326,7 +337,7 @@ def run_ours(args):
     total_ms_max = max_over_ranks(dist, world, total_ms)
     ms_step = total_ms_max / K
     tc = w.batch * w.length * w.channels
-    value = world * tc / (ms_step * 1e-3)
+    value = weak_scaling_value(world, tc, ms_step)
     if m.mamba_get_device_error(clear=False) != 0:
         raise RuntimeError("device error word set during the benchmark")
     clocks = sampler.summary()
@@ -416,8 +427,8 @@ def run_decode(args, dev, stream, dist, world, rank, hbm_peak, hbm_src):
 
     w = wl.DECODE_WORKLOADS["decode_bf16"]
     steps = args.decode_steps
-    prm = wl.decode_params(w, dev, seed=w.seed + 1000 * rank)
-    chain = wl.decode_chain_inputs_bulk(w, steps, dev, seed=w.seed + 1000 * rank)
+    prm = wl.decode_params(w, dev, seed=rank_seed(w.seed, rank))
+    chain = wl.decode_chain_inputs_bulk(w, steps, dev, seed=rank_seed(w.seed, rank))
     state = prm["state"].clone()
     y = torch.empty((steps, w.batch, w.channels), device=dev, dtype=w.torch_dtype)
     lib = m.library()

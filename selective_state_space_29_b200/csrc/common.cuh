@@ -8,7 +8,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include "../../include/mamba_ssm.h"
+#include "mamba_ssm.h"
 
 namespace mamba {
 
@@ -131,24 +131,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
-}
-
-// exp(z) - 1 for z <= 0.  For |z| <= 0.25 a degree-7 Taylor polynomial in
-// Horner form (truncation error below 2^-26 relative there); outside it the
-// hardware exp2 minus one, whose absolute error is small against |e^z - 1|
-// > 0.22 there.  The constants are the Taylor coefficients 1/k!.
-__device__ __forceinline__ float expm1_taylor7(float z) {
-  float p = fmaf(z, 1.0f / 5040.0f, 1.0f / 720.0f);
-  p = fmaf(z, p, 1.0f / 120.0f);
-  p = fmaf(z, p, 1.0f / 24.0f);
-  p = fmaf(z, p, 1.0f / 6.0f);
-  p = fmaf(z, p, 0.5f);
-  p = p * z;
-  return fmaf(z, p, z);
-}
-__device__ __forceinline__ float expm1_neg(float z) {
-  if (fabsf(z) <= 0.25f) return expm1_taylor7(z);
-  return ex2_approx(z * 1.4426950408889634f) - 1.0f;
 }
 
 }  // namespace mamba

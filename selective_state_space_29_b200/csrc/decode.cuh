@@ -11,10 +11,14 @@
 // The kernel is bound by HBM traffic: each update reads and writes the row's
 // N fp32 states (128 bytes at N = 16) and touches only a few bytes more.
 // Layout: NS/4 consecutive lanes share one row, each holding four states as
-// one float4, so a warp moves 512 contiguous bytes per access.
+// one float4, so a warp moves 512 contiguous bytes per access.  A thread
+// keeps its channel's A and D in registers and walks ROWS batch rows, whose
+// loads are all issued before any arithmetic (ROWS x 16 bytes of state in
+// flight per thread).
 #pragma once
 
 #include "common.cuh"
+#include "scan.cuh"  // expm1_small / expm1_fast
 
 namespace mamba {
 
@@ -34,70 +38,79 @@ struct DecodeArgs {
 template <typename TIO>
 __device__ __forceinline__ void load4(const TIO* p, float (&v)[4]) {
   if constexpr (sizeof(TIO) == 4) {
-    v[0] = p[0]; v[1] = p[1]; v[2] = p[2]; v[3] = p[3];
+    const float4 f = *reinterpret_cast<const float4*>(p);
+    v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
   } else {
-    const __nv_bfloat162 lo = reinterpret_cast<const __nv_bfloat162*>(p)[0];
-    const __nv_bfloat162 hi = reinterpret_cast<const __nv_bfloat162*>(p)[1];
-    v[0] = __low2float(lo); v[1] = __high2float(lo);
-    v[2] = __low2float(hi); v[3] = __high2float(hi);
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    v[0] = __uint_as_float(w.x << 16); v[1] = __uint_as_float(w.x & 0xffff0000u);
+    v[2] = __uint_as_float(w.y << 16); v[3] = __uint_as_float(w.y & 0xffff0000u);
   }
 }
 
-template <typename TIO, int NS, int ROWS_PER_THREAD>
-__global__ void __launch_bounds__(256)
-state_update_kernel(const DecodeArgs<TIO, NS> a) {
-  constexpr int QPR = NS / 4;  // lanes per row
-  static_assert(32 % QPR == 0, "a row must not straddle a warp");
-  constexpr int RPW = 32 / QPR;  // rows per warp access
-  const int64_t rows = a.batch * a.channels;
-  const int lane = threadIdx.x & 31;
-  const int q = lane % QPR;
-  const int lane_row = lane / QPR;
-  const int64_t warp_g = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+constexpr int kDecodeWarps = 8;  // warps per CTA
 
-  // the loop bound is uniform across the warp (the shuffles below need it)
-  for (int64_t wb = warp_g; wb * RPW < rows; wb += nwarps * ROWS_PER_THREAD) {
-    float4 h[ROWS_PER_THREAD];
-    float av[ROWS_PER_THREAD][4], bv[ROWS_PER_THREAD][4], cv[ROWS_PER_THREAD][4];
-    float xv[ROWS_PER_THREAD], dv[ROWS_PER_THREAD], Dd[ROWS_PER_THREAD];
-    bool ok[ROWS_PER_THREAD];
-    // issue every load first (two rows in flight per thread)
+// grid: x over channel tiles of kDecodeWarps * 32 / (NS/4) channels,
+//       y over batch tiles of ROWS batch rows.
+// FASTQ: exp(z) - 1 from the hardware exp2 (bf16 data); otherwise the
+// branch-free accurate form.
+template <typename TIO, int NS, int ROWS, bool FASTQ>
+__global__ void __launch_bounds__(kDecodeWarps * 32)
+state_update_kernel(const DecodeArgs<TIO, NS> a) {
+  constexpr int QPR = NS / 4;           // lanes per row
+  constexpr int CPW = 32 / QPR;         // channels per warp
+  static_assert(32 % QPR == 0, "a row must not straddle a warp");
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int q = lane % QPR;
+  const int64_t d = ((int64_t)blockIdx.x * kDecodeWarps + warp) * CPW + lane / QPR;
+  const bool dok = d < a.channels;
+  const int64_t b0 = (int64_t)blockIdx.y * ROWS;
+
+  float av[4] = {-1.f, -1.f, -1.f, -1.f};
+  float Dd = 0.0f;
+  if (dok) {
+    const float4 A4 = __ldg(reinterpret_cast<const float4*>(a.A + d * NS) + q);
+    av[0] = A4.x; av[1] = A4.y; av[2] = A4.z; av[3] = A4.w;
+    Dd = a.D ? __ldg(a.D + d) : 0.0f;
+  }
+  float inva[4];
 #pragma unroll
-    for (int k = 0; k < ROWS_PER_THREAD; ++k) {
-      const int64_t r = (wb + (int64_t)k * nwarps) * RPW + lane_row;
-      ok[k] = r < rows;
-      const int64_t rr = ok[k] ? r : 0;
-      const int64_t b = rr / a.channels;
-      const int64_t d = rr - b * a.channels;
-      h[k] = reinterpret_cast<const float4*>(a.state + rr * NS)[q];
-      const float4 A4 = __ldg(reinterpret_cast<const float4*>(a.A + d * NS) + q);
-      av[k][0] = A4.x; av[k][1] = A4.y; av[k][2] = A4.z; av[k][3] = A4.w;
-      load4<TIO>(a.B + b * NS + 4 * q, bv[k]);
-      load4<TIO>(a.C + b * NS + 4 * q, cv[k]);
-      xv[k] = to_f32(a.x[rr]);
-      dv[k] = to_f32(a.delta[rr]);
-      Dd[k] = a.D ? __ldg(a.D + d) : 0.0f;
+  for (int i = 0; i < 4; ++i) inva[i] = 1.0f / av[i];
+
+  // issue every load first
+  float4 h[ROWS];
+  float bv[ROWS][4], cv[ROWS][4], xv[ROWS], dv[ROWS];
+  bool ok[ROWS];
+#pragma unroll
+  for (int k = 0; k < ROWS; ++k) {
+    const int64_t b = b0 + k;
+    ok[k] = dok && b < a.batch;
+    const int64_t r = ok[k] ? b * a.channels + d : 0;
+    const int64_t bb = ok[k] ? b : 0;
+    h[k] = ok[k] ? reinterpret_cast<const float4*>(a.state + r * NS)[q] : make_float4(0.f, 0.f, 0.f, 0.f);
+    load4<TIO>(a.B + bb * NS + 4 * q, bv[k]);
+    load4<TIO>(a.C + bb * NS + 4 * q, cv[k]);
+    xv[k] = ok[k] ? to_f32(a.x[r]) : 0.0f;
+    dv[k] = ok[k] ? to_f32(a.delta[r]) : 0.0f;
+  }
+#pragma unroll
+  for (int k = 0; k < ROWS; ++k) {
+    float hv[4] = {h[k].x, h[k].y, h[k].z, h[k].w};
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float z = dv[k] * av[i];
+      const float e = FASTQ ? expm1_fast(z) : expm1_small(z);   // exp(Delta A_n) - 1
+      const float phi = e * inva[i];              // (Delta A_n)^-1 (exp(Delta A_n) - 1) Delta
+      hv[i] = fmaf(phi, bv[k][i] * xv[k], fmaf(e, hv[i], hv[i]));
+      acc = fmaf(cv[k][i], hv[i], acc);
     }
 #pragma unroll
-    for (int k = 0; k < ROWS_PER_THREAD; ++k) {
-      float hv[4] = {h[k].x, h[k].y, h[k].z, h[k].w};
-      float acc = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float z = dv[k] * av[k][i];
-        const float e = expm1_neg(z);                     // exp(Delta A_n) - 1
-        const float phi = (av[k][i] != 0.0f) ? e / av[k][i] : dv[k];  // (Delta A)^-1 (e^{Delta A} - 1) Delta
-        hv[i] = fmaf(phi, bv[k][i] * xv[k], fmaf(e, hv[i], hv[i]));
-        acc = fmaf(cv[k][i], hv[i], acc);
-      }
-#pragma unroll
-      for (int off = 1; off < QPR; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      if (ok[k]) {
-        const int64_t r = (wb + (int64_t)k * nwarps) * RPW + lane_row;
-        reinterpret_cast<float4*>(a.state + r * NS)[q] = make_float4(hv[0], hv[1], hv[2], hv[3]);
-        if (q == 0) a.y[r] = from_f32<TIO>(fmaf(Dd[k], xv[k], acc));
-      }
+    for (int off = 1; off < QPR; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (ok[k]) {
+      const int64_t r = (b0 + k) * a.channels + d;
+      reinterpret_cast<float4*>(a.state + r * NS)[q] = make_float4(hv[0], hv[1], hv[2], hv[3]);
+      if (q == 0) a.y[r] = from_f32<TIO>(fmaf(Dd, xv[k], acc));
     }
   }
 }

@@ -10,7 +10,7 @@
 #include <cstring>
 #include <mutex>
 
-#include "../../include/mamba_ssm.h"
+#include "mamba_ssm.h"
 #include "common.cuh"
 #include "decode.cuh"
 #include "scan.cuh"
@@ -83,9 +83,12 @@ bool make_map_2d(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uin
 // --- scan configuration per element type -----------------------------------
 template <typename TIO>
 struct ScanCfg;
+#ifndef MAMBA_SCAN_STAGES
+#define MAMBA_SCAN_STAGES 4
+#endif
 template <>
 struct ScanCfg<__nv_bfloat16> {
-  static constexpr int kTile = 32, kStages = 4;
+  static constexpr int kTile = 32, kStages = MAMBA_SCAN_STAGES;
 };
 template <>
 struct ScanCfg<float> {
@@ -127,10 +130,10 @@ Plan plan_scan(int64_t len, int groups, int warps_total, int tile, int64_t user_
 }
 
 struct ScratchLayout {
-  size_t ctr, done, ring, ring_sd, agg_h, agg_sd, hin, total;
+  size_t ctr, done, ring, ring_sd, agg_h, agg_sd, hin, cs, total;
 };
 
-ScratchLayout scratch_layout(const Plan& pl, int groups, int ns) {
+ScratchLayout scratch_layout(const Plan& pl, int groups, int ns, int64_t batch, int64_t len) {
   auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
   const int64_t S = pl.supers;
   const int64_t streams_full = S * groups;
@@ -143,7 +146,8 @@ ScratchLayout scratch_layout(const Plan& pl, int groups, int ns) {
   s.agg_h = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup * ns);
   s.agg_sd = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup);
   s.hin = S > 1 ? al(sizeof(float) * (size_t)streams_full * kGroup * ns) : 0;
-  s.total = s.ctr + s.done + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.hin;
+  s.cs = al(sizeof(float) * (size_t)batch * (size_t)len * (size_t)ns);
+  s.total = s.ctr + s.done + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.hin + s.cs;
   return s;
 }
 
@@ -170,8 +174,27 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   const int groups = (int)groups64;
   const Plan pl = plan_scan(len, groups, warps_total, TILE, user_chunk);
 
+  // scratch: [counters x2][done x2][ring][ring_sd][agg_h][agg_sd][hin][C']
+  const int64_t S = pl.supers;
+  const int64_t streams_full = S * groups;
+  const int64_t streams_agg = (S - 1) * groups;
+  const ScratchLayout sl = scratch_layout(pl, groups, NS, batch, len);
+  unsigned char* scratch = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+  unsigned char* cur = scratch;
+  int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
+  int* done = reinterpret_cast<int*>(cur); cur += sl.done;
+  float* ring = reinterpret_cast<float*>(cur); cur += sl.ring;
+  float* ring_sd = reinterpret_cast<float*>(cur); cur += sl.ring_sd;
+  float* agg_h = reinterpret_cast<float*>(cur); cur += sl.agg_h;
+  float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
+  float* hin = sl.hin ? reinterpret_cast<float*>(cur) : nullptr;
+  cur += sl.hin;
+  float* cs = reinterpret_cast<float*>(cur);
+
+  // tile loads through TMA when every operand can be described by a tensor map
   const size_t es = sizeof(TIO);
-  const bool use_tma = aligned(u, 16) && aligned(delta, 16) && aligned(B, 16) && aligned(C, 16) &&
+  const bool use_tma = aligned(u, 16) && aligned(delta, 16) && aligned(B, 16) &&
                        (channels * (int64_t)es) % 16 == 0 && (NS * es) % 16 == 0 && encode_fn() != nullptr;
   CUtensorMap mu, mdl, mb, mc;
   std::memset(&mu, 0, sizeof(mu));
@@ -183,30 +206,14 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
     const uint64_t rows = (uint64_t)batch * (uint64_t)len;
     tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
           make_map_2d(&mdl, delta, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
-          make_map_2d(&mb, B, dtype, NS, rows, NS, TILE) && make_map_2d(&mc, C, dtype, NS, rows, NS, TILE);
+          make_map_2d(&mb, B, dtype, NS, rows, NS, TILE) && make_map_2d(&mc, cs, MAMBA_F32, NS, rows, NS, TILE);
   }
-
-  // scratch: [counters x2][done x2][ring][ring_sd][agg_h][agg_sd][hin]
-  const int64_t S = pl.supers;
-  const int64_t streams_full = S * groups;
-  const int64_t streams_agg = (S - 1) * groups;
-  const ScratchLayout sl = scratch_layout(pl, groups, NS);
-  unsigned char* scratch = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
-  unsigned char* cur = scratch;
-  int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
-  int* done = reinterpret_cast<int*>(cur); cur += sl.done;
-  float* ring = reinterpret_cast<float*>(cur); cur += sl.ring;
-  float* ring_sd = reinterpret_cast<float*>(cur); cur += sl.ring_sd;
-  float* agg_h = reinterpret_cast<float*>(cur); cur += sl.agg_h;
-  float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
-  float* hin = sl.hin ? reinterpret_cast<float*>(cur) : nullptr;
   int status = MAMBA_OK;
   if (cudaMemsetAsync(scratch, 0, sl.ctr + sl.done, stream) != cudaSuccess) status = MAMBA_ERR_CUDA;
 
   ScanParams p;
   std::memset(&p, 0, sizeof(p));
-  p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.D = D; p.h0 = h0; p.y = y;
+  p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.cs = cs; p.D = D; p.h0 = h0; p.y = y;
   p.final_state = final_state;
   p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd; p.hin = hin;
   p.batch = batch; p.len = len; p.channels = channels;
@@ -229,10 +236,14 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
 
   auto run_pass = [&](int mode, int streams, int64_t jobs, int* ctr, int* dn) {
     if (status != MAMBA_OK || jobs <= 0) return;
+    if (jobs > 0x7fffffff) {
+      status = MAMBA_ERR_UNSUPPORTED;
+      return;
+    }
     ScanParams q = p;
     q.mode = mode;
     q.streams = streams;
-    q.jobs = jobs;
+    q.jobs = (int)jobs;
     q.counters = ctr;
     q.done = dn;
     const int64_t ctas = std::min<int64_t>(sms, (jobs + kWarpsPerCta - 1) / kWarpsPerCta);
@@ -240,6 +251,13 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
     if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
   };
 
+  // C' = C / (n+1) in fp32 for the output sums
+  if (status == MAMBA_OK) {
+    const int64_t total_c = batch * len * NS;
+    scan_prep_c_kernel<TIO, NS><<<(unsigned)((total_c + 255) / 256), 256, 0, stream>>>(
+        static_cast<const TIO*>(C), cs, total_c);
+    if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
+  }
   if (S > 1) {
     // aggregate pass over every super-chunk but the last, then the combine
     run_pass(kModeAggregate, (int)streams_agg, streams_agg * pl.chunks_full, counters + 2, done + streams_full);
@@ -302,8 +320,8 @@ int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate
   out->super_len = pl.super_len;
   out->chunk_len = pl.chunk_len;
   out->jobs = full_jobs(pl, groups);
-  out->kernels = pl.supers > 1 ? 3 : 1;
-  out->scratch_bytes = (int64_t)scratch_layout(pl, groups, (int)nstate).total;
+  out->kernels = pl.supers > 1 ? 4 : 2;  // C' pre-pass, [aggregate, combine,] main pass
+  out->scratch_bytes = (int64_t)scratch_layout(pl, groups, (int)nstate, batch, len).total;
   out->ctas = std::min<int64_t>(sms, (out->jobs + kWarpsPerCta - 1) / kWarpsPerCta);
   return MAMBA_OK;
 }
@@ -368,22 +386,24 @@ int mamba_state_update(float* state, const void* x, const void* delta, const flo
   int sms = 0;
   if (int st = current_sms(&sms)) return st;
   cudaGetLastError();
-  const int64_t rows = batch * channels;
-  constexpr int kThreads = 256, kRowsPerThread = 2;
-  const int64_t row_groups = (rows + 7) / 8;  // a warp covers 8 rows per access
-  int64_t blocks = (row_groups + (kThreads / 32) * kRowsPerThread - 1) / ((kThreads / 32) * kRowsPerThread);
-  blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, (int64_t)sms * 64));
+  constexpr int kRows = 4;                                  // batch rows per thread
+  constexpr int kChanPerCta = kDecodeWarps * (32 / (16 / 4));  // 64 channels per CTA at 16 states
+  const int64_t gx = (channels + kChanPerCta - 1) / kChanPerCta;
+  const int64_t gy = (batch + kRows - 1) / kRows;
+  if (gy > 65535 || gx > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)gx, (unsigned)gy);
+  (void)sms;
   if (dtype == MAMBA_BF16) {
     DecodeArgs<__nv_bfloat16, 16> a{state, static_cast<const __nv_bfloat16*>(x),
                                     static_cast<const __nv_bfloat16*>(delta), A,
                                     static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
                                     static_cast<__nv_bfloat16*>(y), batch, channels};
-    state_update_kernel<__nv_bfloat16, 16, kRowsPerThread><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+    state_update_kernel<__nv_bfloat16, 16, kRows, true><<<grid, kDecodeWarps * 32, 0, stream>>>(a);
   } else {
     DecodeArgs<float, 16> a{state, static_cast<const float*>(x), static_cast<const float*>(delta), A,
                             static_cast<const float*>(B), static_cast<const float*>(C), D,
                             static_cast<float*>(y), batch, channels};
-    state_update_kernel<float, 16, kRowsPerThread><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+    state_update_kernel<float, 16, kRows, false><<<grid, kDecodeWarps * 32, 0, stream>>>(a);
   }
   return cudaGetLastError() == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
