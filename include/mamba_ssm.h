@@ -142,6 +142,39 @@ int mamba_state_update(float *state, const void *x, const void *delta,
                        void *y, int64_t batch, int64_t channels, int64_t nstate,
                        int dtype, mamba_stream_t stream);
 
+/*
+ * mamba_selective_scan without any device allocation.  (The pages describe
+ * no such call; it serves callers of this library, not the method.)
+ *
+ * Same arguments, layouts, results and asynchrony as mamba_selective_scan.
+ * It is for callers that may not allocate device memory inside an operation:
+ * inference runtimes and plugin hosts that plan all device memory ahead and
+ * hand an operation only its inputs and outputs, deployments held to a fixed
+ * memory budget, and processes whose device memory is owned by another
+ * allocator (a framework's caching pool), where an allocation made by a
+ * library can fail at any point.
+ *
+ * Its scratch is one file-scope device array of 16 MiB, reserved on every GPU
+ * that loads the library until the process exits; it never calls
+ * cudaMalloc, cudaMallocAsync or cudaFree.  A problem whose scratch (see
+ * mamba_scan_plan: scratch_bytes) exceeds 16 MiB is rejected with
+ * MAMBA_ERR_UNSUPPORTED before anything is enqueued; at 16 states that
+ * covers, e.g., 8 x 2048 x 3072 and 4 x 8192 x 5120, not 1 x 1,048,576 x 2048.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call uses the same array, which keeps what the previous
+ * call left in it: the call clears the parts that must start at zero on
+ * `stream`.  Calls that can overlap on the GPU (other streams, other host
+ * threads without ordering) race on the array and corrupt each other's
+ * results: order them.
+ */
+int mamba_selective_scan_noalloc(const void *u, const void *delta, const float *A,
+                                 const void *B, const void *C, const float *D,
+                                 void *y, float *final_state,
+                                 int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                                 int dtype, mamba_stream_t stream);
+
 /* How mamba_selective_scan_ex would split a problem (host-side planning only). */
 typedef struct {
     int64_t supers;        /* independent super-chunks per sequence (1: no aggregate/combine pass) */

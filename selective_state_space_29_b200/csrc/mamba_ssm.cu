@@ -273,6 +273,158 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   return status;
 }
 
+// ---------------------------------------------------------------------------
+// Scan without any allocation (mamba_selective_scan_noalloc).
+//
+// Some callers may not allocate device memory inside an operation: inference
+// runtimes and plugin hosts that plan every byte of device memory ahead of
+// time and hand operations only their inputs and outputs, deployments with a
+// fixed, audited memory budget, and processes whose device memory is held by
+// another allocator (a framework's caching pool), where a driver allocation
+// can fail at an arbitrary point.  For them the scan's scratch (job counters,
+// the chunk-to-chunk state hand-off, super-chunk aggregates and C/(n+1))
+// lives in one file-scope device array of fixed size, reserved on every GPU
+// that loads the library for as long as the process lives.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(16) << 20;  // 16 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the array's name only stands in for the symbol, so the address is looked
+// up once per device (with that device current) and cached.
+int noalloc_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MAMBA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) return MAMBA_ERR_CUDA;
+    g_noalloc_addr[dev] = ptr;
+  }
+  *out = g_noalloc_addr[dev];
+  return MAMBA_OK;
+}
+
+std::mutex g_noalloc_attr_mu;
+bool g_noalloc_attr_set[2][64] = {};
+
+template <typename TIO, int NS>
+int launch_scan_noalloc(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                        const float* D, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
+                        int dtype, cudaStream_t stream) {
+  constexpr int TILE = ScanCfg<TIO>::kTile;
+  constexpr int STAGES = ScanCfg<TIO>::kStages;
+  int sms = 0;
+  if (int st = current_sms(&sms)) return st;
+  const int groups_d = (int)((channels + kGroup - 1) / kGroup);
+  const int64_t groups64 = batch * groups_d;
+  if (groups64 > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
+  const int groups = (int)groups64;
+  const Plan pl = plan_scan(len, groups, sms * kWarpsPerCta, TILE, 0);
+  const ScratchLayout sl = scratch_layout(pl, groups, NS, batch, len);
+  if (sl.total > kNoAllocScratchBytes) return MAMBA_ERR_UNSUPPORTED;  // problem needs more scratch than reserved
+
+  void* base = nullptr;
+  if (int st = noalloc_scratch_address(&base)) return st;
+  unsigned char* scratch = static_cast<unsigned char*>(base);
+  unsigned char* cur = scratch;
+  int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
+  int* done = reinterpret_cast<int*>(cur); cur += sl.done;
+  float* ring = reinterpret_cast<float*>(cur); cur += sl.ring;
+  float* ring_sd = reinterpret_cast<float*>(cur); cur += sl.ring_sd;
+  float* agg_h = reinterpret_cast<float*>(cur); cur += sl.agg_h;
+  float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
+  float* hin = sl.hin ? reinterpret_cast<float*>(cur) : nullptr;
+  cur += sl.hin;
+  float* cs = reinterpret_cast<float*>(cur);
+
+  const size_t es = sizeof(TIO);
+  bool tma = aligned(u, 16) && aligned(delta, 16) && aligned(B, 16) && (channels * (int64_t)es) % 16 == 0 &&
+             (NS * es) % 16 == 0 && encode_fn() != nullptr;
+  CUtensorMap mu, mdl, mb, mc;
+  std::memset(&mu, 0, sizeof(mu));
+  std::memset(&mdl, 0, sizeof(mdl));
+  std::memset(&mb, 0, sizeof(mb));
+  std::memset(&mc, 0, sizeof(mc));
+  if (tma) {
+    const uint64_t rows = (uint64_t)batch * (uint64_t)len;
+    tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
+          make_map_2d(&mdl, delta, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
+          make_map_2d(&mb, B, dtype, NS, rows, NS, TILE) && make_map_2d(&mc, cs, MAMBA_F32, NS, rows, NS, TILE);
+  }
+
+  // the array keeps whatever the previous call left: the counters and the
+  // per-stream progress flags must start at zero
+  if (cudaMemsetAsync(scratch, 0, sl.ctr + sl.done, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+
+  ScanParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.cs = cs; p.D = D; p.h0 = nullptr; p.y = y;
+  p.final_state = final_state;
+  p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd; p.hin = hin;
+  p.batch = batch; p.len = len; p.channels = channels;
+  p.groups_d = groups_d; p.groups = groups;
+  p.supers = pl.supers; p.super_len = pl.super_len; p.chunk_len = pl.chunk_len;
+  p.chunks_full = pl.chunks_full; p.chunks_last = pl.chunks_last;
+  p.use_tma = tma ? 1 : 0;
+  p.force_general = 0;
+  p.wait_limit_ns = kWaitLimitNs;
+
+  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES>();
+  auto kern = scan_chunks_kernel<TIO, NS, TILE, STAGES>;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MAMBA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_attr_mu);
+    bool& set = g_noalloc_attr_set[sizeof(TIO) == 2 ? 1 : 0][dev];
+    if (!set) {
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+        return MAMBA_ERR_CUDA;
+      set = true;
+    }
+  }
+
+  const int64_t S = pl.supers;
+  const int64_t streams_full = S * groups;
+  const int64_t streams_agg = (S - 1) * groups;
+  int status = MAMBA_OK;
+  auto run_pass = [&](int mode, int64_t streams, int64_t jobs, int* ctr, int* dn) {
+    if (status != MAMBA_OK || jobs <= 0) return;
+    if (jobs > 0x7fffffff) {
+      status = MAMBA_ERR_UNSUPPORTED;
+      return;
+    }
+    ScanParams q = p;
+    q.mode = mode;
+    q.streams = (int)streams;
+    q.jobs = (int)jobs;
+    q.counters = ctr;
+    q.done = dn;
+    const int64_t ctas = std::min<int64_t>(sms, (jobs + kWarpsPerCta - 1) / kWarpsPerCta);
+    kern<<<(unsigned)ctas, kWarpsPerCta * 32, smem, stream>>>(q, mu, mdl, mb, mc);
+    if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
+  };
+  {
+    const int64_t total_c = batch * len * NS;
+    scan_prep_c_kernel<TIO, NS><<<(unsigned)((total_c + 255) / 256), 256, 0, stream>>>(
+        static_cast<const TIO*>(C), cs, total_c);
+    if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
+  }
+  if (S > 1) {
+    run_pass(kModeAggregate, streams_agg, streams_agg * pl.chunks_full, counters + 2, done + streams_full);
+    if (status == MAMBA_OK) {
+      const int64_t threads = (int64_t)groups * kGroup * NS;
+      scan_combine_kernel<NS><<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p, hin);
+      if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
+    }
+  }
+  run_pass(kModeFull, streams_full, full_jobs(pl, groups), counters, done);
+  return status;
+}
+
 __global__ void expire_wait_kernel(uint64_t limit_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -368,6 +520,35 @@ int mamba_selective_scan(const void* u, const void* delta, const float* A, const
                          int64_t nstate, int dtype, mamba_stream_t stream) {
   return mamba_selective_scan_ex(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, nstate, 0, 0u,
                                  dtype, stream);
+}
+
+int mamba_selective_scan_noalloc(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                                 const float* D, void* y, float* final_state, int64_t batch, int64_t len,
+                                 int64_t channels, int64_t nstate, int dtype, mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || len < 0 || channels < 0 || nstate <= 0) return MAMBA_ERR_INVALID_ARG;
+  if (!mamba_scan_supported_nstate(nstate)) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || channels == 0) return MAMBA_OK;
+  const size_t es = (size_t)elem_size(dtype);
+  if (len > 0) {
+    if (!u || !delta || !B || !C || !y || !A) return MAMBA_ERR_INVALID_ARG;
+    if (!aligned(u, es) || !aligned(delta, es) || !aligned(B, es) || !aligned(C, es) || !aligned(y, es))
+      return MAMBA_ERR_INVALID_ARG;
+  }
+  if ((A && !aligned(A, 4)) || (D && !aligned(D, 4)) || (final_state && !aligned(final_state, 4)))
+    return MAMBA_ERR_INVALID_ARG;
+  if (batch * len >= (int64_t(1) << 31) || channels >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+  cudaGetLastError();
+  if (len == 0) {
+    if (!final_state) return MAMBA_OK;
+    const size_t state_bytes = sizeof(float) * (size_t)batch * (size_t)channels * (size_t)nstate;
+    return cudaMemsetAsync(final_state, 0, state_bytes, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+  }
+  if (dtype == MAMBA_BF16)
+    return launch_scan_noalloc<__nv_bfloat16, 16>(u, delta, A, B, C, D, y, final_state, batch, len, channels, dtype,
+                                                  stream);
+  return launch_scan_noalloc<float, 16>(u, delta, A, B, C, D, y, final_state, batch, len, channels, dtype, stream);
 }
 
 int mamba_state_update(float* state, const void* x, const void* delta, const float* A, const void* B, const void* C,

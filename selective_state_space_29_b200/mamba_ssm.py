@@ -42,6 +42,8 @@ _SIGNATURES = [
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_selective_scan_ex", ctypes.c_int,
      [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_uint, ctypes.c_int, _P]),
+    ("mamba_selective_scan_noalloc", ctypes.c_int,
+     [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_state_update", ctypes.c_int,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_scan_plan", ctypes.c_int,
@@ -129,6 +131,17 @@ def mamba_selective_scan_ex(u, delta, A, B, C, D, initial_state, y, final_state,
                                            _ptr(initial_state), _ptr(y), _ptr(final_state), batch, len,
                                            channels, nstate, chunk_len, flags, dtype, _stream(stream))
     _check(st, "mamba_selective_scan_ex")
+
+
+def mamba_selective_scan_noalloc(u, delta, A, B, C, D, y, final_state, batch, len, channels, nstate, dtype,
+                                 stream=None):
+    """The scan with its scratch in the library's fixed 16 MiB device array:
+    no device allocation, for callers that may not allocate inside an
+    operation.  Calls that overlap on the GPU race on that array."""
+    st = library().mamba_selective_scan_noalloc(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
+                                                _ptr(final_state), batch, len, channels, nstate, dtype,
+                                                _stream(stream))
+    _check(st, "mamba_selective_scan_noalloc")
 
 
 def mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, dtype, stream=None):
