@@ -65,6 +65,10 @@ state_update_kernel(const DecodeArgs<TIO, NS> a) {
   const int64_t d = ((int64_t)blockIdx.x * kDecodeWarps + warp) * CPW + lane / QPR;
   const bool dok = d < a.channels;
   const int64_t b0 = (int64_t)blockIdx.y * ROWS;
+  // the next step's kernel may be scheduled as this one's CTAs retire; every
+  // input of this one may come from the previous kernel of the stream
+  griddep_launch_dependents();
+  griddep_wait();
 
   float av[4] = {-1.f, -1.f, -1.f, -1.f};
   float Dd = 0.0f;

@@ -81,44 +81,57 @@ bool make_map_2d(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uin
 }
 
 // --- scan configuration per element type -----------------------------------
+// A CTA is kScanConsumers consumer warps (one per SM sub-partition) and one
+// producer warp; a consumer's ring holds kStages tiles of kTile tokens.
 template <typename TIO>
 struct ScanCfg;
-#ifndef MAMBA_SCAN_STAGES
-#define MAMBA_SCAN_STAGES 4
-#endif
 template <>
 struct ScanCfg<__nv_bfloat16> {
-  static constexpr int kTile = 32, kStages = MAMBA_SCAN_STAGES;
+  static constexpr int kTile = 64, kStages = 3;
 };
 template <>
 struct ScanCfg<float> {
-  static constexpr int kTile = 16, kStages = 4;
+  static constexpr int kTile = 32, kStages = 3;
 };
+constexpr int kScanConsumers = 4;
+constexpr int kJobsPerWarp = 8;  // chunks per consumer warp, for dynamic balance
 
 struct Plan {
+  int groups_d = 0;         // ceil(channels / 32)
+  int64_t groups = 0;       // batch * groups_d
+  int warps_total = 0;      // resident consumer warps: SMs * kScanConsumers
   int supers = 1;
   int64_t super_len = 0;
   int64_t chunk_len = 0;
   int chunks_full = 1, chunks_last = 1;
 };
 
-Plan plan_scan(int64_t len, int groups, int warps_total, int tile, int64_t user_chunk) {
+// How a scan is laid out and split.  Every consumer warp needs a stream of
+// its own (a 32-channel group over a stretch of time); when the groups are
+// fewer than the resident consumer warps, sequences are cut into
+// super-chunks joined by the associative combine.  Within a stream the
+// sequence is cut into chunks so that there are about kJobsPerWarp jobs per
+// warp for dynamic balance, each at least two tiles long.  A positive
+// `user_chunk` forces super-chunks of that length.
+Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, int64_t user_chunk) {
   Plan pl;
+  pl.warps_total = sms * kScanConsumers;
+  pl.groups_d = (int)((channels + kCPW - 1) / kCPW);
+  pl.groups = batch * pl.groups_d;
+  const int64_t groups = std::max<int64_t>(1, pl.groups);
   if (user_chunk > 0) {
     pl.super_len = std::min<int64_t>(user_chunk, len);
   } else {
     int64_t s = 1;
-    if (groups < warps_total) s = (warps_total + groups - 1) / groups;
+    if (groups < pl.warps_total) s = (pl.warps_total + groups - 1) / groups;
     s = std::min<int64_t>(s, std::max<int64_t>(1, len / (4 * tile)));
     pl.super_len = (len + s - 1) / s;
     pl.super_len = ((pl.super_len + tile - 1) / tile) * tile;
   }
   pl.super_len = std::max<int64_t>(1, pl.super_len);
   pl.supers = (int)((len + pl.super_len - 1) / pl.super_len);
-  // chunks inside a super-chunk: enough jobs (about 8 per warp) for balance,
-  // but at least two tiles per job
   const int64_t streams = (int64_t)pl.supers * groups;
-  int64_t k = (8LL * warps_total + streams - 1) / streams;
+  int64_t k = ((int64_t)kJobsPerWarp * pl.warps_total + streams - 1) / streams;
   k = std::max<int64_t>(1, std::min<int64_t>(k, pl.super_len / (2 * tile)));
   int64_t cl = (pl.super_len + k - 1) / k;
   cl = ((cl + tile - 1) / tile) * tile;
@@ -130,151 +143,59 @@ Plan plan_scan(int64_t len, int groups, int warps_total, int tile, int64_t user_
 }
 
 struct ScratchLayout {
-  size_t ctr, done, ring, ring_sd, agg_h, agg_sd, hin, cs, total;
+  size_t ctr, done, ring, ring_sd, agg_h, agg_sd, hin, cs, chan, total;
 };
 
-ScratchLayout scratch_layout(const Plan& pl, int groups, int ns, int64_t batch, int64_t len) {
+ScratchLayout scratch_layout(const Plan& pl, int ns, int64_t batch, int64_t len) {
   auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
   const int64_t S = pl.supers;
-  const int64_t streams_full = S * groups;
-  const int64_t streams_agg = (S - 1) * groups;
+  const int64_t streams_full = S * pl.groups;
+  const int64_t streams_agg = (S - 1) * pl.groups;
   ScratchLayout s;
   s.ctr = al(4 * sizeof(int));
   s.done = al(sizeof(int) * (size_t)(streams_full + streams_agg));
-  s.ring = al(sizeof(float) * (size_t)streams_full * 2 * kGroup * ns);
-  s.ring_sd = al(sizeof(float) * (size_t)streams_full * 2 * kGroup);
-  s.agg_h = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup * ns);
-  s.agg_sd = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kGroup);
-  s.hin = S > 1 ? al(sizeof(float) * (size_t)streams_full * kGroup * ns) : 0;
+  s.ring = al(sizeof(float) * (size_t)streams_full * 2 * kCPW * ns);
+  s.ring_sd = al(sizeof(float) * (size_t)streams_full * 2 * kCPW);
+  s.agg_h = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kCPW * ns);
+  s.agg_sd = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kCPW);
+  s.hin = S > 1 ? al(sizeof(float) * (size_t)streams_full * kCPW * ns) : 0;
   s.cs = al(sizeof(float) * (size_t)batch * (size_t)len * (size_t)ns);
-  s.total = s.ctr + s.done + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.hin + s.cs;
+  s.chan = al(sizeof(float) * 4 * (size_t)pl.groups_d * (size_t)kCPW);
+  s.total = s.ctr + s.done + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.hin + s.cs + s.chan;
   return s;
 }
 
-int64_t full_jobs(const Plan& pl, int groups) {
-  const int64_t streams_full = (int64_t)pl.supers * groups;
-  const int64_t streams_agg = (int64_t)(pl.supers - 1) * groups;
+int64_t full_jobs(const Plan& pl) {
+  const int64_t streams_full = (int64_t)pl.supers * pl.groups;
+  const int64_t streams_agg = (int64_t)(pl.supers - 1) * pl.groups;
   return (int64_t)pl.chunks_last * streams_full + (int64_t)(pl.chunks_full - pl.chunks_last) * streams_agg;
 }
 
 int tile_for(int dtype) { return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16>::kTile : ScanCfg<float>::kTile; }
 
-template <typename TIO, int NS>
-int launch_scan(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
-                const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
-                int64_t user_chunk, unsigned flags, int dtype, cudaStream_t stream) {
-  constexpr int TILE = ScanCfg<TIO>::kTile;
-  constexpr int STAGES = ScanCfg<TIO>::kStages;
-  int sms = 0;
-  if (int st = current_sms(&sms)) return st;
-  const int warps_total = sms * kWarpsPerCta;
-  const int groups_d = (int)((channels + kGroup - 1) / kGroup);
-  const int64_t groups64 = batch * groups_d;
-  if (groups64 > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
-  const int groups = (int)groups64;
-  const Plan pl = plan_scan(len, groups, warps_total, TILE, user_chunk);
+int64_t kernels_per_call(const Plan& pl) { return pl.supers > 1 ? 4 : 2; }  // pre-pass, [aggregate, combine,] main
 
-  // scratch: [counters x2][done x2][ring][ring_sd][agg_h][agg_sd][hin][C']
-  const int64_t S = pl.supers;
-  const int64_t streams_full = S * groups;
-  const int64_t streams_agg = (S - 1) * groups;
-  const ScratchLayout sl = scratch_layout(pl, groups, NS, batch, len);
-  unsigned char* scratch = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
-  unsigned char* cur = scratch;
-  int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
-  int* done = reinterpret_cast<int*>(cur); cur += sl.done;
-  float* ring = reinterpret_cast<float*>(cur); cur += sl.ring;
-  float* ring_sd = reinterpret_cast<float*>(cur); cur += sl.ring_sd;
-  float* agg_h = reinterpret_cast<float*>(cur); cur += sl.agg_h;
-  float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
-  float* hin = sl.hin ? reinterpret_cast<float*>(cur) : nullptr;
-  cur += sl.hin;
-  float* cs = reinterpret_cast<float*>(cur);
-
-  // tile loads through TMA when every operand can be described by a tensor map
-  const size_t es = sizeof(TIO);
-  const bool use_tma = aligned(u, 16) && aligned(delta, 16) && aligned(B, 16) &&
-                       (channels * (int64_t)es) % 16 == 0 && (NS * es) % 16 == 0 && encode_fn() != nullptr;
-  CUtensorMap mu, mdl, mb, mc;
-  std::memset(&mu, 0, sizeof(mu));
-  std::memset(&mdl, 0, sizeof(mdl));
-  std::memset(&mb, 0, sizeof(mb));
-  std::memset(&mc, 0, sizeof(mc));
-  bool tma = use_tma;
-  if (tma) {
-    const uint64_t rows = (uint64_t)batch * (uint64_t)len;
-    tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
-          make_map_2d(&mdl, delta, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
-          make_map_2d(&mb, B, dtype, NS, rows, NS, TILE) && make_map_2d(&mc, cs, MAMBA_F32, NS, rows, NS, TILE);
-  }
-  int status = MAMBA_OK;
-  if (cudaMemsetAsync(scratch, 0, sl.ctr + sl.done, stream) != cudaSuccess) status = MAMBA_ERR_CUDA;
-
-  ScanParams p;
-  std::memset(&p, 0, sizeof(p));
-  p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.cs = cs; p.D = D; p.h0 = h0; p.y = y;
-  p.final_state = final_state;
-  p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd; p.hin = hin;
-  p.batch = batch; p.len = len; p.channels = channels;
-  p.groups_d = groups_d; p.groups = groups;
-  p.supers = pl.supers; p.super_len = pl.super_len; p.chunk_len = pl.chunk_len;
-  p.chunks_full = pl.chunks_full; p.chunks_last = pl.chunks_last;
-  p.use_tma = tma ? 1 : 0;
-  p.force_general = (flags & MAMBA_SCAN_GENERAL_A) ? 1 : 0;
-  p.wait_limit_ns = kWaitLimitNs;
-
-  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES>();
-  auto kern = scan_chunks_kernel<TIO, NS, TILE, STAGES>;
-  static bool attr_set = false;  // per instantiation
-  if (!attr_set) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-      status = MAMBA_ERR_CUDA;
-    else
-      attr_set = true;
-  }
-
-  auto run_pass = [&](int mode, int streams, int64_t jobs, int* ctr, int* dn) {
-    if (status != MAMBA_OK || jobs <= 0) return;
-    if (jobs > 0x7fffffff) {
-      status = MAMBA_ERR_UNSUPPORTED;
-      return;
-    }
-    ScanParams q = p;
-    q.mode = mode;
-    q.streams = streams;
-    q.jobs = (int)jobs;
-    q.counters = ctr;
-    q.done = dn;
-    const int64_t ctas = std::min<int64_t>(sms, (jobs + kWarpsPerCta - 1) / kWarpsPerCta);
-    kern<<<(unsigned)ctas, kWarpsPerCta * 32, smem, stream>>>(q, mu, mdl, mb, mc);
-    if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
-  };
-
-  // C' = C / (n+1) in fp32 for the output sums
-  if (status == MAMBA_OK) {
-    const int64_t total_c = batch * len * NS;
-    scan_prep_c_kernel<TIO, NS><<<(unsigned)((total_c + 255) / 256), 256, 0, stream>>>(
-        static_cast<const TIO*>(C), cs, total_c);
-    if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
-  }
-  if (S > 1) {
-    // aggregate pass over every super-chunk but the last, then the combine
-    run_pass(kModeAggregate, (int)streams_agg, streams_agg * pl.chunks_full, counters + 2, done + streams_full);
-    if (status == MAMBA_OK) {
-      const int64_t threads = (int64_t)groups * kGroup * NS;
-      scan_combine_kernel<NS><<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p, hin);
-      if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
-    }
-  }
-  run_pass(kModeFull, (int)streams_full, full_jobs(pl, groups), counters, done);
-
-  if (cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) status = MAMBA_ERR_CUDA;
-  return status;
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel of the stream finishes; it waits for that kernel's
+// writes (griddepcontrol.wait) before it reads or writes global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------------------
-// Scan without any allocation (mamba_selective_scan_noalloc).
+// Scratch for mamba_selective_scan_noalloc.
 //
 // Some callers may not allocate device memory inside an operation: inference
 // runtimes and plugin hosts that plan every byte of device memory ahead of
@@ -308,28 +229,16 @@ int noalloc_scratch_address(void** out) {
   return MAMBA_OK;
 }
 
-std::mutex g_noalloc_attr_mu;
-bool g_noalloc_attr_set[2][64] = {};
-
+// Enqueue one scan with the given plan on caller-provided scratch (laid out
+// by scratch_layout): pre-pass, [aggregate pass, combine,] main pass.
 template <typename TIO, int NS>
-int launch_scan_noalloc(const void* u, const void* delta, const float* A, const void* B, const void* C,
-                        const float* D, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
-                        int dtype, cudaStream_t stream) {
+int launch_scan_on(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
+                   const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
+                   unsigned flags, int dtype, cudaStream_t stream, const Plan& pl, int sms,
+                   unsigned char* scratch) {
   constexpr int TILE = ScanCfg<TIO>::kTile;
   constexpr int STAGES = ScanCfg<TIO>::kStages;
-  int sms = 0;
-  if (int st = current_sms(&sms)) return st;
-  const int groups_d = (int)((channels + kGroup - 1) / kGroup);
-  const int64_t groups64 = batch * groups_d;
-  if (groups64 > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
-  const int groups = (int)groups64;
-  const Plan pl = plan_scan(len, groups, sms * kWarpsPerCta, TILE, 0);
-  const ScratchLayout sl = scratch_layout(pl, groups, NS, batch, len);
-  if (sl.total > kNoAllocScratchBytes) return MAMBA_ERR_UNSUPPORTED;  // problem needs more scratch than reserved
-
-  void* base = nullptr;
-  if (int st = noalloc_scratch_address(&base)) return st;
-  unsigned char* scratch = static_cast<unsigned char*>(base);
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len);
   unsigned char* cur = scratch;
   int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
   int* done = reinterpret_cast<int*>(cur); cur += sl.done;
@@ -339,8 +248,10 @@ int launch_scan_noalloc(const void* u, const void* delta, const float* A, const 
   float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
   float* hin = sl.hin ? reinterpret_cast<float*>(cur) : nullptr;
   cur += sl.hin;
-  float* cs = reinterpret_cast<float*>(cur);
+  float* cs = reinterpret_cast<float*>(cur); cur += sl.cs;
+  float4* chan = reinterpret_cast<float4*>(cur);
 
+  // tile loads through TMA when every operand can be described by a tensor map
   const size_t es = sizeof(TIO);
   bool tma = aligned(u, 16) && aligned(delta, 16) && aligned(B, 16) && (channels * (int64_t)es) % 16 == 0 &&
              (NS * es) % 16 == 0 && encode_fn() != nullptr;
@@ -351,77 +262,106 @@ int launch_scan_noalloc(const void* u, const void* delta, const float* A, const 
   std::memset(&mc, 0, sizeof(mc));
   if (tma) {
     const uint64_t rows = (uint64_t)batch * (uint64_t)len;
-    tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
-          make_map_2d(&mdl, delta, dtype, (uint64_t)channels, rows, kGroup, TILE) &&
+    tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows, kCPW, TILE) &&
+          make_map_2d(&mdl, delta, dtype, (uint64_t)channels, rows, kCPW, TILE) &&
           make_map_2d(&mb, B, dtype, NS, rows, NS, TILE) && make_map_2d(&mc, cs, MAMBA_F32, NS, rows, NS, TILE);
   }
 
-  // the array keeps whatever the previous call left: the counters and the
-  // per-stream progress flags must start at zero
-  if (cudaMemsetAsync(scratch, 0, sl.ctr + sl.done, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
-
   ScanParams p;
   std::memset(&p, 0, sizeof(p));
-  p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.cs = cs; p.D = D; p.h0 = nullptr; p.y = y;
+  p.u = u; p.delta = delta; p.A = A; p.B = B; p.cs = cs; p.chan = chan; p.h0 = h0; p.y = y;
   p.final_state = final_state;
   p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd; p.hin = hin;
   p.batch = batch; p.len = len; p.channels = channels;
-  p.groups_d = groups_d; p.groups = groups;
+  p.groups_d = pl.groups_d; p.groups = (int)pl.groups;
   p.supers = pl.supers; p.super_len = pl.super_len; p.chunk_len = pl.chunk_len;
   p.chunks_full = pl.chunks_full; p.chunks_last = pl.chunks_last;
   p.use_tma = tma ? 1 : 0;
-  p.force_general = 0;
   p.wait_limit_ns = kWaitLimitNs;
 
-  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES>();
-  auto kern = scan_chunks_kernel<TIO, NS, TILE, STAGES>;
+  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES, kScanConsumers>();
+  static_assert(smem <= 232448, "scan CTA exceeds the shared memory of an SM");
+  auto kern = scan_chunks_kernel<TIO, NS, kScanConsumers, TILE, STAGES>;
   {
+    // the dynamic shared-memory limit is a per-device attribute of the kernel
+    static std::mutex mu_attr;
+    static bool attr_set[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MAMBA_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_noalloc_attr_mu);
-    bool& set = g_noalloc_attr_set[sizeof(TIO) == 2 ? 1 : 0][dev];
-    if (!set) {
+    std::lock_guard<std::mutex> lk(mu_attr);
+    if (!attr_set[dev]) {
       if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
         return MAMBA_ERR_CUDA;
-      set = true;
+      attr_set[dev] = true;
     }
   }
 
   const int64_t S = pl.supers;
-  const int64_t streams_full = S * groups;
-  const int64_t streams_agg = (S - 1) * groups;
-  int status = MAMBA_OK;
-  auto run_pass = [&](int mode, int64_t streams, int64_t jobs, int* ctr, int* dn) {
-    if (status != MAMBA_OK || jobs <= 0) return;
-    if (jobs > 0x7fffffff) {
-      status = MAMBA_ERR_UNSUPPORTED;
-      return;
-    }
+  const int64_t streams_full = S * pl.groups;
+  const int64_t streams_agg = (S - 1) * pl.groups;
+  if (full_jobs(pl) > 0x7fffffff || streams_agg * pl.chunks_full > 0x7fffffff || streams_full > 0x7fffffff)
+    return MAMBA_ERR_UNSUPPORTED;
+  auto run_pass = [&](int mode, int64_t streams, int64_t jobs, int* ctr, int* dn) -> cudaError_t {
     ScanParams q = p;
     q.mode = mode;
     q.streams = (int)streams;
     q.jobs = (int)jobs;
     q.counters = ctr;
     q.done = dn;
-    const int64_t ctas = std::min<int64_t>(sms, (jobs + kWarpsPerCta - 1) / kWarpsPerCta);
-    kern<<<(unsigned)ctas, kWarpsPerCta * 32, smem, stream>>>(q, mu, mdl, mb, mc);
-    if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
+    const int64_t ctas = std::min<int64_t>(sms, (jobs + kScanConsumers - 1) / kScanConsumers);
+    return launch_pdl(kern, dim3((unsigned)ctas), dim3((kScanConsumers + 1) * 32), smem, stream, q, mu, mdl, mb, mc);
   };
+
+  // pre-pass: zero the counters and progress flags, C' = C / (n+1) in fp32,
+  // and the per-channel constants
   {
+    const int64_t zero_words = (int64_t)((sl.ctr + sl.done) / sizeof(int));
     const int64_t total_c = batch * len * NS;
-    scan_prep_c_kernel<TIO, NS><<<(unsigned)((total_c + 255) / 256), 256, 0, stream>>>(
-        static_cast<const TIO*>(C), cs, total_c);
-    if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
+    const int64_t chan_padded = (int64_t)pl.groups_d * kCPW;
+    const int64_t total = zero_words + total_c + chan_padded;
+    if ((total + 255) / 256 > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
+    scan_prep_kernel<TIO, NS><<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
+        counters, zero_words, static_cast<const TIO*>(C), cs, total_c, A, D, chan, channels, chan_padded,
+        (flags & MAMBA_SCAN_GENERAL_A) ? 1 : 0);
+    if (cudaGetLastError() != cudaSuccess) return MAMBA_ERR_CUDA;
   }
   if (S > 1) {
-    run_pass(kModeAggregate, streams_agg, streams_agg * pl.chunks_full, counters + 2, done + streams_full);
-    if (status == MAMBA_OK) {
-      const int64_t threads = (int64_t)groups * kGroup * NS;
-      scan_combine_kernel<NS><<<(unsigned)((threads + 255) / 256), 256, 0, stream>>>(p, hin);
-      if (cudaGetLastError() != cudaSuccess) status = MAMBA_ERR_CUDA;
-    }
+    // aggregate pass over every super-chunk but the last, then the combine
+    if (run_pass(kModeAggregate, streams_agg, streams_agg * pl.chunks_full, counters + 2, done + streams_full) !=
+        cudaSuccess)
+      return MAMBA_ERR_CUDA;
+    const int64_t threads = pl.groups * kCPW * NS;
+    if (launch_pdl(scan_combine_kernel<NS>, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, stream, p, hin) !=
+        cudaSuccess)
+      return MAMBA_ERR_CUDA;
   }
-  run_pass(kModeFull, streams_full, full_jobs(pl, groups), counters, done);
+  if (run_pass(kModeFull, streams_full, full_jobs(pl), counters, done) != cudaSuccess) return MAMBA_ERR_CUDA;
+  return MAMBA_OK;
+}
+
+// Plan, get scratch (stream-ordered allocation, or the fixed array when
+// `noalloc`), enqueue, release the allocation.
+template <typename TIO, int NS>
+int launch_scan(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
+                const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
+                int64_t user_chunk, unsigned flags, int dtype, cudaStream_t stream, bool noalloc) {
+  int sms = 0;
+  if (int st = current_sms(&sms)) return st;
+  const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO>::kTile, user_chunk);
+  if (pl.groups > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len);
+  unsigned char* scratch = nullptr;
+  if (noalloc) {
+    if (sl.total > kNoAllocScratchBytes) return MAMBA_ERR_UNSUPPORTED;  // needs more than the fixed array
+    void* base = nullptr;
+    if (int st = noalloc_scratch_address(&base)) return st;
+    scratch = static_cast<unsigned char*>(base);
+  } else {
+    if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+  }
+  const int status = launch_scan_on<TIO, NS>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags,
+                                             dtype, stream, pl, sms, scratch);
+  if (!noalloc && cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) return MAMBA_ERR_CUDA;
   return status;
 }
 
@@ -466,15 +406,14 @@ int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate
   if (sms <= 0) {
     if (int st = current_sms(&sms)) return st;
   }
-  const int groups = (int)(batch * ((channels + kGroup - 1) / kGroup));
-  const Plan pl = plan_scan(len, groups, sms * kWarpsPerCta, tile_for(dtype), chunk_len);
+  const Plan pl = plan_scan(batch, len, channels, sms, tile_for(dtype), chunk_len);
   out->supers = pl.supers;
   out->super_len = pl.super_len;
   out->chunk_len = pl.chunk_len;
-  out->jobs = full_jobs(pl, groups);
-  out->kernels = pl.supers > 1 ? 4 : 2;  // C' pre-pass, [aggregate, combine,] main pass
-  out->scratch_bytes = (int64_t)scratch_layout(pl, groups, (int)nstate, batch, len).total;
-  out->ctas = std::min<int64_t>(sms, (out->jobs + kWarpsPerCta - 1) / kWarpsPerCta);
+  out->jobs = full_jobs(pl);
+  out->kernels = kernels_per_call(pl);
+  out->scratch_bytes = (int64_t)scratch_layout(pl, (int)nstate, batch, len).total;
+  out->ctas = std::min<int64_t>(sms, (out->jobs + kScanConsumers - 1) / kScanConsumers);
   return MAMBA_OK;
 }
 
@@ -510,9 +449,9 @@ int mamba_selective_scan_ex(const void* u, const void* delta, const float* A, co
   }
   if (dtype == MAMBA_BF16)
     return launch_scan<__nv_bfloat16, 16>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels,
-                                          chunk_len, flags, dtype, stream);
+                                          chunk_len, flags, dtype, stream, false);
   return launch_scan<float, 16>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels, chunk_len,
-                                flags, dtype, stream);
+                                flags, dtype, stream, false);
 }
 
 int mamba_selective_scan(const void* u, const void* delta, const float* A, const void* B, const void* C,
@@ -546,9 +485,10 @@ int mamba_selective_scan_noalloc(const void* u, const void* delta, const float* 
     return cudaMemsetAsync(final_state, 0, state_bytes, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
   }
   if (dtype == MAMBA_BF16)
-    return launch_scan_noalloc<__nv_bfloat16, 16>(u, delta, A, B, C, D, y, final_state, batch, len, channels, dtype,
-                                                  stream);
-  return launch_scan_noalloc<float, 16>(u, delta, A, B, C, D, y, final_state, batch, len, channels, dtype, stream);
+    return launch_scan<__nv_bfloat16, 16>(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, 0, 0u,
+                                          dtype, stream, true);
+  return launch_scan<float, 16>(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, 0, 0u, dtype,
+                                stream, true);
 }
 
 int mamba_state_update(float* state, const void* x, const void* delta, const float* A, const void* B, const void* C,
@@ -564,29 +504,29 @@ int mamba_state_update(float* state, const void* x, const void* delta, const flo
   if (!aligned(state, 16) || !aligned(A, 16) || (D && !aligned(D, 4)) || !aligned(x, es) || !aligned(delta, es) ||
       !aligned(y, es) || !aligned(B, 4 * es) || !aligned(C, 4 * es))
     return MAMBA_ERR_INVALID_ARG;
-  int sms = 0;
-  if (int st = current_sms(&sms)) return st;
   cudaGetLastError();
-  constexpr int kRows = 4;                                  // batch rows per thread
+  constexpr int kRows = 4;                                     // batch rows per thread
   constexpr int kChanPerCta = kDecodeWarps * (32 / (16 / 4));  // 64 channels per CTA at 16 states
   const int64_t gx = (channels + kChanPerCta - 1) / kChanPerCta;
   const int64_t gy = (batch + kRows - 1) / kRows;
   if (gy > 65535 || gx > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
   const dim3 grid((unsigned)gx, (unsigned)gy);
-  (void)sms;
+  // programmatic launch: a step's setup overlaps the end of the previous
+  // kernel of the stream (the kernel waits for it before touching memory)
+  cudaError_t err;
   if (dtype == MAMBA_BF16) {
     DecodeArgs<__nv_bfloat16, 16> a{state, static_cast<const __nv_bfloat16*>(x),
                                     static_cast<const __nv_bfloat16*>(delta), A,
                                     static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
                                     static_cast<__nv_bfloat16*>(y), batch, channels};
-    state_update_kernel<__nv_bfloat16, 16, kRows, true><<<grid, kDecodeWarps * 32, 0, stream>>>(a);
+    err = launch_pdl(state_update_kernel<__nv_bfloat16, 16, kRows, true>, grid, dim3(kDecodeWarps * 32), 0, stream, a);
   } else {
     DecodeArgs<float, 16> a{state, static_cast<const float*>(x), static_cast<const float*>(delta), A,
                             static_cast<const float*>(B), static_cast<const float*>(C), D,
                             static_cast<float*>(y), batch, channels};
-    state_update_kernel<float, 16, kRows, false><<<grid, kDecodeWarps * 32, 0, stream>>>(a);
+    err = launch_pdl(state_update_kernel<float, 16, kRows, false>, grid, dim3(kDecodeWarps * 32), 0, stream, a);
   }
-  return cudaGetLastError() == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+  return err == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
 }
 
 int mamba_get_device_error(int clear) {

@@ -9,22 +9,26 @@
 //     y[b,t,d] = sum_n C[b,t,n] h[n] + D[d] u[b,t,d]
 //
 // Work decomposition
-//   * A "group" is 32 consecutive channels of one batch row; one warp owns a
-//     group and each lane owns one channel with its N states in registers.
+//   * A "group" is 32 consecutive channels of one batch row.  A consumer warp
+//     owns a group while it runs a job, each lane one channel with its N
+//     states in registers.
 //   * The sequence of a group is cut into chunks.  A job is (stream, chunk):
 //     a warp runs the recurrence over the chunk's tokens starting from the
 //     state the previous chunk of the same stream ended with.  Jobs are
 //     handed out by an atomic ticket in chunk-major order, so the predecessor
 //     of every job was taken earlier by a running warp: waits always end.
-//     The grid is persistent (one warp per SM sub-partition), which keeps
-//     every sub-partition busy whatever the group count.
-//   * When there are fewer groups than warps, the sequence is also cut into
-//     "super-chunks" that run as independent streams.  Their starting states
-//     come from the associative combine of the page's parallel prefix scan
-//     ("Paralel Tarama Algoritması"): an aggregate pass computes, per
-//     super-chunk, the end state from zero H_j and sum of Delta; a combine
-//     pass runs h_{j+1} = exp(A sum Delta_j) h_j + H_j; the main pass then
-//     runs every super-chunk from its own starting state.
+//   * The grid is persistent, one CTA per SM: four consumer warps (one per SM
+//     sub-partition) and one producer warp.  The producer pulls the tickets,
+//     streams each consumer's tiles into its shared-memory ring by TMA and
+//     publishes the consumers' chunk-to-chunk hand-off flags, so a consumer
+//     only waits for a tile, computes, and hands the slot back.
+//   * When there are fewer groups than consumer warps, the sequence is also
+//     cut into "super-chunks" that run as independent streams.  Their
+//     starting states come from the associative combine of the page's
+//     parallel prefix scan ("Paralel Tarama Algoritması"): an aggregate pass
+//     computes, per super-chunk, the end state from zero H_j and sum of
+//     Delta; a combine pass runs h_{j+1} = exp(A sum Delta_j) h_j + H_j; the
+//     main pass then runs every super-chunk from its own starting state.
 //
 // Arithmetic per token and state (all fp32; the state is kept scaled,
 // g_n = A_n h_n, so that 1/A_n leaves the inner loop):
@@ -34,26 +38,25 @@
 // When A[d,n] == (n+1) A[d,0] for every n of every channel in the warp (the
 // S4D-real structure), e_n comes from one exact-arithmetic identity,
 //     e^{(n+1) z} - 1 = e^z (e^{n z} - 1) + (e^z - 1),
-// i.e. e_n = r e_{n-1} + q with q = expm1(Delta A[d,0]), r = 1 + q: one FMA per
+// i.e. e_n = r e_{n-1} + q with r = exp(Delta A[d,0]), q = r - 1: one FMA per
 // state instead of an exponential; then C_n / A_n = (C_n / (n+1)) / A_0.
 // Otherwise every e_n is computed from its own exponential.
 //
 // Data path of a tile: u, Delta and B in the I/O type, and C' = C / (n+1) as
-// fp32 (one small pre-pass per call), staged by TMA.  With bf16 data the
-// input term B_n x is one mixed-precision FMA on the raw bf16 operands
-// (their product is exact in fp32); nothing is converted in shared memory.
-// Each lane reads the whole B and C' row of every token, so the bytes
-// broadcast from shared memory per token are the other limit next to the
-// FMA pipe: 32 B of B and 64 B of C' at N = 16.
+// fp32 (a small pre-pass per call), staged by TMA.  With bf16 data the input
+// term B_n x is one mixed-precision FMA on the raw bf16 operands (their
+// product is exact in fp32); nothing is converted in shared memory.  Every
+// lane reads the whole B and C' row of every token (broadcast loads).  y is
+// stored by each lane with a predicated store: no branch inside the token
+// loop, which keeps a tile's tokens in one scheduling region.
 #pragma once
 
 #include "common.cuh"
 
 namespace mamba {
 
-constexpr int kWarpsPerCta = 4;   // one warp per SM sub-partition
-constexpr int kGroup = 32;        // channels per warp
-constexpr int kMaxRing = 8;       // jobs a warp may have pulled ahead of its compute
+constexpr int kCPW = 32;   // channels per warp: one lane per channel
+constexpr int kHandQ = 8;  // hand-off flags a consumer may leave for the producer to publish
 
 enum ScanMode : int { kModeFull = 0, kModeAggregate = 1 };
 
@@ -63,15 +66,14 @@ struct ScanParams {
   const void* delta;
   const float* A;
   const void* B;
-  const void* C;
   const float* cs;          // C' = C / (n+1), fp32 [batch*len][N] (scratch, written by the pre-pass)
-  const float* D;           // nullable
+  const float4* chan;       // per channel {A[d,0], 1/A[d,0], D[d], structured}, padded to groups_d*32
   const float* h0;          // nullable: initial state [b][d][n]
   void* y;
   float* final_state;       // nullable
-  // scratch (stream-ordered, zeroed where noted)
-  int* counters;            // [0] job ticket, [1] abort flag (zeroed)
-  int* done;                // [streams] chunks completed per stream (zeroed)
+  // scratch (stream-ordered; the pre-pass zeroes counters and done)
+  int* counters;            // [0] job ticket, [1] abort flag
+  int* done;                // [streams] chunks completed per stream
   float* ring;              // [streams][2][32][N] states handed between chunks
   float* ring_sd;           // [streams][2][32] running sum of Delta (aggregate mode)
   float* agg_h;             // [(S-1)*G][32][N] aggregate end states
@@ -90,7 +92,6 @@ struct ScanParams {
   int streams;              // streams active in this pass
   int jobs;                 // jobs in this pass (fits int32, checked on the host)
   int use_tma;
-  int force_general;
   uint64_t wait_limit_ns;
 };
 
@@ -129,7 +130,7 @@ __device__ __forceinline__ Job decode_job(const ScanParams& p, int j_in, int til
   jb.super_idx = (int)(s / (uint32_t)p.groups);
   const int grp = (int)(s - (uint32_t)jb.super_idx * (uint32_t)p.groups);
   jb.b = grp / p.groups_d;
-  jb.d0 = (grp - jb.b * p.groups_d) * kGroup;
+  jb.d0 = (grp - jb.b * p.groups_d) * kCPW;
   const int64_t s_begin = (int64_t)jb.super_idx * p.super_len;
   const int64_t s_end = (s_begin + p.super_len < p.len) ? s_begin + p.super_len : p.len;
   jb.t0 = s_begin + (int64_t)k * p.chunk_len;
@@ -141,27 +142,37 @@ __device__ __forceinline__ Job decode_job(const ScanParams& p, int j_in, int til
 }
 
 // ---------------------------------------------------------------------------
-// shared-memory layout of one warp: STAGES tile slots (TMA destinations,
-// 128-byte aligned), their full barriers, the warp's job queue
+// shared-memory block of one consumer warp: STAGES tile slots (TMA
+// destinations, 128-byte aligned) with the per-channel constants of the
+// job, full / empty barriers, the job of each slot, and the queue of
+// hand-off flags the producer publishes
 // ---------------------------------------------------------------------------
 template <typename TIO, int NS, int TILE, int STAGES>
 struct alignas(128) WarpSmem {
-  TIO u[STAGES][TILE][kGroup];
-  TIO dl[STAGES][TILE][kGroup];
+  TIO u[STAGES][TILE][kCPW];
+  TIO dl[STAGES][TILE][kCPW];
   TIO b[STAGES][TILE][NS];
   float cs[STAGES][TILE][NS];
-  uint64_t full[STAGES];
-  int ring_jobs[kMaxRing];
+  float4 chan[STAGES][kCPW];  // loaded with tile 0 of a job
+  uint64_t full[STAGES];      // producer -> consumer: the tile has landed
+  uint64_t empty[STAGES];     // consumer -> producer: the slot has been read
+  int job[STAGES];            // job of the slot's tile; -1: no more jobs
+  int hq_stream[kHandQ];      // hand-off flags: done[stream] = value
+  int hq_value[kHandQ];
+  int hq_head;                // entries pushed by the consumer
+  int hq_tail;                // entries published by the producer
+  int finished;               // the consumer has left its loop
 };
 
-template <typename TIO, int NS, int TILE, int STAGES>
+template <typename TIO, int NS, int TILE, int STAGES, int CW>
 constexpr size_t scan_smem_bytes() {
-  return sizeof(WarpSmem<TIO, NS, TILE, STAGES>) * kWarpsPerCta + 128;
+  return sizeof(WarpSmem<TIO, NS, TILE, STAGES>) * CW + 128;
 }
 
+// bytes one tile brings in: u and Delta columns, the B row (I/O type), the C' row (fp32)
 template <typename TIO, int NS>
 __host__ __device__ constexpr uint32_t tile_bytes(int tile) {
-  return (uint32_t)(tile * (2 * kGroup * sizeof(TIO) + NS * sizeof(TIO) + NS * sizeof(float)));
+  return (uint32_t)(tile * (2 * kCPW * sizeof(TIO) + NS * sizeof(TIO) + NS * sizeof(float)));
 }
 
 // ---------------------------------------------------------------------------
@@ -188,6 +199,8 @@ __device__ __forceinline__ float expm1_fast(float z) { return ex2_approx(z * 1.4
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
+__device__ __forceinline__ uint16_t raw16(__nv_bfloat16 v) { return __bfloat16_as_ushort(v); }
+
 // d = lo16(w) * x + c and d = hi16(w) * x + c with bf16 multiplicands and an
 // fp32 addend (the bf16 x bf16 product is exact in fp32).
 __device__ __forceinline__ float fma_bf16_lo(uint32_t w, uint16_t x, float c) {
@@ -203,17 +216,28 @@ __device__ __forceinline__ float fma_bf16_hi(uint32_t w, uint16_t x, float c) {
   return d;
 }
 
+// Store v at p when pred holds, as one predicated instruction (a branch
+// around a plain store would split the token loop into scheduling regions).
+__device__ __forceinline__ void st_global_pred(__nv_bfloat16* p, __nv_bfloat16 v, bool pred) {
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q st.global.b16 [%0], %1;\n\t}" ::"l"(p),
+               "h"(raw16(v)), "r"((int)pred));
+}
+__device__ __forceinline__ void st_global_pred(float* p, float v, bool pred) {
+  asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %2, 0;\n\t@q st.global.f32 [%0], %1;\n\t}" ::"l"(p),
+               "f"(v), "r"((int)pred));
+}
+
 // e2[k] = (exp((2k+1) z) - 1, exp((2k+2) z) - 1) for k < NS/2 from
-// q = exp(z) - 1, using exp((m+k) z) - 1 = (exp(k z) - 1) + exp(k z)(exp(m z) - 1):
+// r = exp(z) and q = exp(z) - 1, using
+//     exp((m+k) z) - 1 = (exp(k z) - 1) + exp(k z)(exp(m z) - 1):
 // the first four by steps of z, the rest by steps of 4z in four independent
 // chains (dependency depth 7 instead of NS - 1).
 template <int NS>
-__device__ __forceinline__ void decay_chain2(float q, float2 (&e2)[NS / 2]) {
+__device__ __forceinline__ void decay_chain(float r, float q, float2 (&e2)[NS / 2]) {
   static_assert(NS % 4 == 0, "NS multiple of 4");
-  const float r1 = 1.0f + q;
-  const float e1 = fmaf(r1, q, q);
-  const float e2s = fmaf(r1, e1, q);
-  const float e3 = fmaf(r1, e2s, q);
+  const float e1 = fmaf(r, q, q);
+  const float e2s = fmaf(r, e1, q);
+  const float e3 = fmaf(r, e2s, q);
   e2[0] = f2(q, e1);
   e2[1] = f2(e2s, e3);
   const float2 r4 = f2(1.0f + e3, 1.0f + e3);
@@ -221,8 +245,6 @@ __device__ __forceinline__ void decay_chain2(float q, float2 (&e2)[NS / 2]) {
 #pragma unroll
   for (int k = 2; k < NS / 2; ++k) e2[k] = __ffma2_rn(r4, e2[k - 2], q4);
 }
-
-__device__ __forceinline__ uint16_t raw16(__nv_bfloat16 v) { return __bfloat16_as_ushort(v); }
 
 // One token for one lane: g <- g + e (g + B x) for all states; returns
 // sum_n C'_n g_n.  States as N/2 float2 pairs, every state step a packed
@@ -269,31 +291,39 @@ __device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const T
   return (acc0.x + acc0.y) + (acc1.x + acc1.y);
 }
 
-// Rows [0, rows) of one tile, structured A.  FULL: write y; otherwise
-// accumulate sum(Delta).  FASTQ: expm1(Delta A_0) from the hardware exp2.
-// Two tokens per step: their decay chains are independent work for the
-// scheduler while the state updates wait on each other.
+// Rows [0, rows) of one tile, structured A, for one lane: its channel column
+// `su`/`sdl` (stride 32) and all its states.  FULL: store y (predicated on
+// the channel being inside the tensor); otherwise accumulate sum(Delta).
+// FASTQ (bf16 data): r from the hardware exp2 of Delta A_0 log2(e), q = r - 1;
+// otherwise q from the accurate expm1 and r = 1 + q.  Two tokens per step:
+// their decay chains are independent work for the scheduler while the state
+// updates wait on each other.
 template <typename TIO, int NS, int TILE, bool FULL, bool FASTQ>
 __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, const TIO (*bt)[NS],
                                                 const float (*ct)[NS], int rows, float a0, float inv_a0, float Dd,
                                                 float2 (&g)[NS / 2], float& sd, TIO* yp, int64_t ystride,
                                                 bool active) {
-  const float a0l2e = a0 * 1.4426950408889634f;
+  const float a0l = a0 * 1.4426950408889634f;
   auto chain = [&](float dt, float2 (&e)[NS / 2]) {
-    const float q = FASTQ ? ex2_approx(dt * a0l2e) - 1.0f : expm1_small(dt * a0);
-    decay_chain2<NS>(q, e);
+    if constexpr (FASTQ) {
+      const float r = ex2_approx(dt * a0l);
+      decay_chain<NS>(r, r - 1.0f, e);
+    } else {
+      const float q = expm1_small(dt * a0);
+      decay_chain<NS>(1.0f + q, q, e);
+    }
   };
   auto emit = [&](float s, TIO xr, float dt) {
     if constexpr (FULL) {
-      if (active) *yp = from_f32<TIO>(fmaf(s, inv_a0, Dd * to_f32(xr)));
+      st_global_pred(yp, from_f32<TIO>(fmaf(s, inv_a0, Dd * to_f32(xr))), active);
       yp += ystride;
     } else {
       sd += dt;
     }
   };
   auto pair = [&](int r) {
-    const TIO x0 = su[r * kGroup], x1 = su[(r + 1) * kGroup];
-    const float d0 = to_f32(sdl[r * kGroup]), d1 = to_f32(sdl[(r + 1) * kGroup]);
+    const TIO x0 = su[r * kCPW], x1 = su[(r + 1) * kCPW];
+    const float d0 = to_f32(sdl[r * kCPW]), d1 = to_f32(sdl[(r + 1) * kCPW]);
     float2 e0[NS / 2], e1[NS / 2];
     chain(d0, e0);
     chain(d1, e1);
@@ -309,8 +339,8 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
   } else {
     for (; r + 1 < rows; r += 2) pair(r);
     if (r < rows) {
-      const TIO x0 = su[r * kGroup];
-      const float d0 = to_f32(sdl[r * kGroup]);
+      const TIO x0 = su[r * kCPW];
+      const float d0 = to_f32(sdl[r * kCPW]);
       float2 e0[NS / 2];
       chain(d0, e0);
       emit(token_update<TIO, NS>(e0, bt[r], ct[r], x0, g), x0, d0);
@@ -326,8 +356,8 @@ __device__ __forceinline__ void tile_general(const TIO* su, const TIO* sdl, cons
                                              const float (&kC)[NS], float Dd, float2 (&g)[NS / 2], float& sd,
                                              TIO* yp, int64_t ystride, bool active) {
   for (int r = 0; r < rows; ++r) {
-    const TIO xr = su[r * kGroup];
-    const float dt = to_f32(sdl[r * kGroup]);
+    const TIO xr = su[r * kCPW];
+    const float dt = to_f32(sdl[r * kCPW]);
     float2 e[NS / 2];
 #pragma unroll
     for (int k = 0; k < NS / 2; ++k) {
@@ -343,10 +373,10 @@ __device__ __forceinline__ void tile_general(const TIO* su, const TIO* sdl, cons
     }
     float crow[NS];
 #pragma unroll
-    for (int n = 0; n < NS; ++n) crow[n] = ct[r][n] * kC[n];
+    for (int k = 0; k < NS; ++k) crow[k] = ct[r][k] * kC[k];
     const float s = token_update<TIO, NS>(e, bt[r], crow, xr, g);
     if constexpr (FULL) {
-      if (active) *yp = from_f32<TIO>(s + Dd * to_f32(xr));
+      st_global_pred(yp, from_f32<TIO>(s + Dd * to_f32(xr)), active);
       yp += ystride;
     } else {
       sd += dt;
@@ -355,89 +385,60 @@ __device__ __forceinline__ void tile_general(const TIO* su, const TIO* sdl, cons
 }
 
 // ---------------------------------------------------------------------------
-// per-warp context: tile pipeline (producer in lane 0) and job queue
+// consumer side of one warp's tile pipeline
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void abort_scan(const ScanParams& p) {
+  record_device_error(MAMBA_ERR_TIMEOUT);
+  atomicExch(&p.counters[1], 1);
+}
+
 template <typename TIO, int NS, int TILE, int STAGES>
-struct WarpCtx {
+struct Consumer {
   using Smem = WarpSmem<TIO, NS, TILE, STAGES>;
   const ScanParams& p;
   Smem& sm;
-  const CUtensorMap* mu;
-  const CUtensorMap* mdl;
-  const CUtensorMap* mb;
-  const CUtensorMap* mc;
   int lane;
-  // producer (meaningful in lane 0): ring index of the job being loaded,
-  // its next tile, jobs pulled so far; tiles issued / consumed
-  uint32_t ld_ring = 0, pulled = 0, cm_ring = 0;
-  int ld_tile = 0, ld_ntiles = 0, ld_row0 = 0, ld_d0 = 0;
-  bool ld_done = false;
-  uint32_t ld_seq = 0, cm_seq = 0;
+  uint32_t seq = 0;  // tiles consumed
+  int hq_head = 0;   // lane 0: hand-off entries pushed
 
-  __device__ WarpCtx(const ScanParams& p_, Smem& sm_, const CUtensorMap* a, const CUtensorMap* b,
-                     const CUtensorMap* c, const CUtensorMap* d, int lane_)
-      : p(p_), sm(sm_), mu(a), mdl(b), mb(c), mc(d), lane(lane_) {}
+  __device__ Consumer(const ScanParams& p_, Smem& sm_, int lane_) : p(p_), sm(sm_), lane(lane_) {}
 
-  __device__ int pull_job() {  // lane 0
-    int j = atomicAdd(&p.counters[0], 1);
-    if (j >= p.jobs || ld_volatile(&p.counters[1]) != 0) j = -1;
-    sm.ring_jobs[pulled % kMaxRing] = j;
-    ++pulled;
-    return j;
-  }
-
-  // issue loads until STAGES tiles are ahead of the compute side (lane 0)
-  __device__ void produce() {
-    while (!ld_done && ld_seq < cm_seq + STAGES) {
-      if (ld_tile >= ld_ntiles) {
-        if (ld_ring + 1 >= pulled) {
-          if (pulled - cm_ring >= (uint32_t)kMaxRing) break;  // queue full
-          if (pull_job() < 0) { ld_done = true; break; }
-        }
-        ++ld_ring;
-        const int j = sm.ring_jobs[ld_ring % kMaxRing];
-        if (j < 0) { ld_done = true; break; }
-        const Job jb = decode_job(p, j, TILE);
-        ld_tile = 0;
-        ld_ntiles = jb.ntiles;
-        ld_row0 = (int)(jb.b * p.len + jb.t0);
-        ld_d0 = jb.d0;
-        continue;
-      }
-      const int slot = ld_seq % STAGES;
-      const int row = ld_row0 + ld_tile * TILE;
-      if (p.use_tma) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&sm.full[slot], tile_bytes<TIO, NS>(TILE));
-        tma_load_2d(&sm.u[slot][0][0], mu, &sm.full[slot], ld_d0, row);
-        tma_load_2d(&sm.dl[slot][0][0], mdl, &sm.full[slot], ld_d0, row);
-        tma_load_2d(&sm.b[slot][0][0], mb, &sm.full[slot], 0, row);
-        tma_load_2d(&sm.cs[slot][0][0], mc, &sm.full[slot], 0, row);
-      } else {
-        mbar_arrive(&sm.full[slot]);  // the warp fetches the tile itself at consume time
-      }
-      ++ld_tile;
-      ++ld_seq;
+  // wait for the next tile; its slot, or -1 when the wait gave up
+  __device__ int wait_tile() {
+    const int s = seq % STAGES;
+    bool ok = mbar_wait_bounded(&sm.full[s], (seq / STAGES) & 1u, p.wait_limit_ns);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) {
+      if (lane == 0) abort_scan(p);
+      return -1;
     }
+    return s;
   }
 
-  // next job id for the compute side (all lanes), -1 when done
-  __device__ int next_job() {
-    ++cm_ring;
-    int jsel = -1;
-    if (lane == 0) {
-      produce();
-      while (!ld_done && cm_ring >= pulled) {
-        if (pull_job() < 0) ld_done = true;
-      }
-      jsel = (cm_ring < pulled) ? sm.ring_jobs[cm_ring % kMaxRing] : -1;
+  // the tile is read: hand its slot back to the producer
+  __device__ void release_tile() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.empty[seq % STAGES]);
+    ++seq;
+  }
+
+  // without TMA the warp fetches its tile itself (rows of this job only)
+  __device__ void fetch_tile(int s, const Job& jb, int64_t tt0, int rows, int d, bool active) {
+    const TIO* gu = static_cast<const TIO*>(p.u);
+    const TIO* gdl = static_cast<const TIO*>(p.delta);
+    const TIO* gB = static_cast<const TIO*>(p.B);
+    const int64_t rowbase = (int64_t)jb.b * p.len + tt0;
+    for (int r = 0; r < rows; ++r) {
+      const int64_t off = (rowbase + r) * p.channels + d;
+      sm.u[s][r][lane] = active ? gu[off] : from_f32<TIO>(0.0f);
+      sm.dl[s][r][lane] = active ? gdl[off] : from_f32<TIO>(0.0f);
     }
-    return __shfl_sync(0xffffffffu, jsel, 0);
-  }
-
-  __device__ void abort_all() {  // lane 0
-    record_device_error(MAMBA_ERR_TIMEOUT);
-    atomicExch(&p.counters[1], 1);
+    for (int i = lane; i < rows * NS; i += 32) {
+      const int r = i / NS, n = i - r * NS;
+      sm.b[s][r][n] = gB[(rowbase + r) * NS + n];
+      sm.cs[s][r][n] = p.cs[(rowbase + r) * NS + n];
+    }
+    __syncwarp();
   }
 
   // wait until the previous chunk of the stream has handed its state on
@@ -449,67 +450,170 @@ struct WarpCtx {
       while (ld_acquire(&p.done[jb.stream]) < jb.chunk) {
         if (ld_volatile(&p.counters[1]) != 0) { aborted = true; break; }
         if ((++spins & 31u) == 0 && globaltimer_ns() - t_start > p.wait_limit_ns) {
-          abort_all();
+          abort_scan(p);
           aborted = true;
           break;
         }
         __nanosleep(spins < 64 ? 32 : 256);
       }
     }
+    // lane 0's acquire, then the warp barrier, orders the state reads below
+    // after the predecessor's release; they bypass L1 (ld.cg) so no stale
+    // line of an earlier chunk can be hit
     aborted = __shfl_sync(0xffffffffu, (int)aborted, 0) != 0;
-    if (!aborted) (void)ld_acquire(&p.done[jb.stream]);  // every lane acquires before reading the state
     return !aborted;
   }
 
-  // wait for the next tile; the plain-load path fetches it here
-  __device__ bool acquire_tile(const Job& jb, int64_t tt0, int rows, int d, bool active) {
-    const int slot = cm_seq % STAGES;
-    bool ok = mbar_wait_bounded(&sm.full[slot], (cm_seq / STAGES) & 1u, p.wait_limit_ns);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) {
-      if (lane == 0) abort_all();
-      return false;
+  // Lane 0, after a __syncwarp that follows every lane's state stores:
+  // done[stream] = value.  The producer warp publishes it (its gpu-scope
+  // release covers the stores, which it observed through this cta-scope
+  // release), so the consumer does not wait for the fence; if the queue is
+  // full the consumer publishes it itself.
+  __device__ void publish(int stream, int value) {
+    if (hq_head - ld_relaxed_cta_smem(&sm.hq_tail) < kHandQ) {
+      sm.hq_stream[hq_head % kHandQ] = stream;
+      sm.hq_value[hq_head % kHandQ] = value;
+      ++hq_head;
+      st_release_cta_smem(&sm.hq_head, hq_head);
+    } else {
+      st_release(&p.done[stream], value);
     }
-    if (!p.use_tma) {
-      const TIO* gu = static_cast<const TIO*>(p.u);
-      const TIO* gdl = static_cast<const TIO*>(p.delta);
-      const TIO* gB = static_cast<const TIO*>(p.B);
-      const int64_t rowbase = (int64_t)jb.b * p.len + tt0;
-      for (int r = 0; r < rows; ++r) {
-        const int64_t off = (rowbase + r) * p.channels + d;
-        sm.u[slot][r][lane] = active ? gu[off] : from_f32<TIO>(0.0f);
-        sm.dl[slot][r][lane] = active ? gdl[off] : from_f32<TIO>(0.0f);
-      }
-      for (int i = lane; i < rows * NS; i += 32) {
-        const int r = i / NS, n = i - r * NS;
-        sm.b[slot][r][n] = gB[(rowbase + r) * NS + n];
-        sm.cs[slot][r][n] = p.cs[(rowbase + r) * NS + n];
-      }
-      __syncwarp();
-    }
-    return true;
-  }
-
-  // the tile is consumed: refill its slot
-  __device__ void release_tile() {
-    __syncwarp();
-    ++cm_seq;
-    if (lane == 0) produce();
-    __syncwarp();
   }
 };
 
-// One job: the recurrence over the chunk's tokens for the warp's 32 channels,
+// ---------------------------------------------------------------------------
+// producer warp (lane 0): pulls jobs from the global ticket, decodes them and
+// streams their tiles into every consumer's slots (TMA, or a bare arrive
+// when the consumer fetches by itself); publishes the consumers' hand-off
+// flags; ends each consumer's stream with a job id of -1.
+// ---------------------------------------------------------------------------
+template <typename TIO, int NS, int CW, int TILE, int STAGES>
+__device__ void producer_loop(const ScanParams& p, WarpSmem<TIO, NS, TILE, STAGES>* sms, const CUtensorMap* mu,
+                              const CUtensorMap* mdl, const CUtensorMap* mb, const CUtensorMap* mc) {
+  struct Feed {
+    uint32_t seq;   // tiles (and the end mark) issued
+    int job, tile, ntiles;
+    int row0, d0;
+    int hq_tail;    // hand-off entries published
+    bool ended;     // end mark issued (or the consumer left)
+    bool fin;       // the consumer has left its loop
+  };
+  Feed f[CW];
+#pragma unroll
+  for (int w = 0; w < CW; ++w) f[w] = Feed{0u, -1, 0, 0, 0, 0, 0, false, false};
+  int ticket = atomicAdd(&p.counters[0], 1);  // one ticket ahead hides the atomic's latency
+  bool stop = false;                          // some warp gave up: hand out no more jobs
+  uint32_t idle = 0;
+  uint64_t idle_since = 0;
+  for (;;) {
+    bool progress = false, all_done = true;
+#pragma unroll
+    for (int w = 0; w < CW; ++w) {
+      auto& sm = sms[w];
+      // consumer state first, then its queue: seeing `finished` makes every
+      // entry it pushed before visible to the queue read that follows
+      if (!f[w].fin) f[w].fin = ld_acquire_cta_smem(&sm.finished) != 0;
+      const int head = ld_acquire_cta_smem(&sm.hq_head);
+      if (f[w].hq_tail != head) {
+        for (; f[w].hq_tail != head; ++f[w].hq_tail) {
+          const int e = f[w].hq_tail % kHandQ;
+          st_release(&p.done[sm.hq_stream[e]], sm.hq_value[e]);
+        }
+        st_relaxed_cta_smem(&sm.hq_tail, f[w].hq_tail);
+        progress = true;
+      }
+      if (f[w].fin) f[w].ended = true;  // left early (gave up): feed it no more
+      if (!f[w].ended) {
+        const uint32_t k = f[w].seq;
+        const int s = (int)(k % STAGES);
+        if (k < (uint32_t)STAGES || mbar_test_wait(&sm.empty[s], ((k / STAGES) - 1u) & 1u)) {
+          bool issue = true;
+          if (f[w].tile >= f[w].ntiles) {
+            if (!stop && ticket < p.jobs) {
+              const Job jb = decode_job(p, ticket, TILE);
+              f[w].job = ticket;
+              f[w].tile = 0;
+              f[w].ntiles = jb.ntiles;
+              f[w].row0 = (int)(jb.b * p.len + jb.t0);
+              f[w].d0 = jb.d0;
+              ticket = atomicAdd(&p.counters[0], 1);
+            } else {
+              sm.job[s] = -1;  // end of this consumer's work
+              mbar_arrive(&sm.full[s]);
+              f[w].seq = k + 1;
+              f[w].ended = true;
+              issue = false;
+            }
+          }
+          if (issue) {
+            sm.job[s] = f[w].job;
+            if (p.use_tma) {
+              const int row = f[w].row0 + f[w].tile * TILE;
+              const bool first = f[w].tile == 0;
+              constexpr uint32_t kChanBytes = kCPW * sizeof(float4);
+              mbar_arrive_expect_tx(&sm.full[s], tile_bytes<TIO, NS>(TILE) + (first ? kChanBytes : 0u));
+              tma_load_2d(&sm.u[s][0][0], mu, &sm.full[s], f[w].d0, row);
+              tma_load_2d(&sm.dl[s][0][0], mdl, &sm.full[s], f[w].d0, row);
+              tma_load_2d(&sm.b[s][0][0], mb, &sm.full[s], 0, row);
+              tma_load_2d(&sm.cs[s][0][0], mc, &sm.full[s], 0, row);
+              if (first) bulk_load(&sm.chan[s][0], p.chan + f[w].d0, kChanBytes, &sm.full[s]);
+            } else {
+              mbar_arrive(&sm.full[s]);
+            }
+            ++f[w].tile;
+            f[w].seq = k + 1;
+          }
+          progress = true;
+        }
+      }
+      all_done = all_done && f[w].fin && f[w].hq_tail == head;
+    }
+    if (all_done) break;
+    if (progress) {
+      idle = 0;
+      continue;
+    }
+    // nothing to do: back off (the consumers run on the same sub-partitions)
+    const uint64_t now = globaltimer_ns();
+    if (idle == 0) idle_since = now;
+    ++idle;
+    if (!stop && (idle & 15u) == 0 && ld_volatile(&p.counters[1]) != 0) stop = true;
+    if (now - idle_since > 2 * p.wait_limit_ns) {  // the consumers' own limits expire first
+      abort_scan(p);
+      break;
+    }
+    __nanosleep(idle < 8 ? 64 : 256);
+  }
+  // every TMA load issued must land before the CTA exits: wait for the last
+  // issue into each slot (a consumer that gave up may have left some unread)
+#pragma unroll
+  for (int w = 0; w < CW; ++w) {
+    for (int s = 0; s < STAGES; ++s) {
+      if ((uint32_t)s >= f[w].seq) break;
+      const uint32_t k_last = f[w].seq - 1u - ((f[w].seq - 1u - (uint32_t)s) % STAGES);
+      if (!mbar_wait_bounded(&sms[w].full[s], (k_last / STAGES) & 1u, p.wait_limit_ns)) {
+        record_device_error(MAMBA_ERR_TIMEOUT);
+        return;
+      }
+    }
+  }
+}
+
+// One job: the recurrence over the chunk's tokens for the warp's channels,
 // from the state the previous chunk handed on, then hand the end state on.
-// STRUCT: A[d,n] = (n+1) A[d,0] on every lane (see decay_chain2).
+// Lane l serves channel d0 + l and all its states.  STRUCT: A[d,n] = (n+1)
+// A[d,0] on every lane (see decay_chain).  Tile 0 is already in slot s0;
+// cm = {A[d,0], 1/A[d,0], D[d], structured}.
 template <typename TIO, int NS, int TILE, int STAGES, bool STRUCT, bool FULL>
-__device__ __forceinline__ bool run_job(WarpCtx<TIO, NS, TILE, STAGES>& cx, const Job& jb, float a0) {
+__device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, const Job& jb, int s0,
+                                        const float4 cm) {
   const ScanParams& p = cx.p;
   auto& sm = cx.sm;
-  const int lane = cx.lane;
-  const int d = jb.d0 + lane;
+  const int c = cx.lane;
+  const int d = jb.d0 + c;
   const bool active = d < p.channels;
-  const float Dd = (FULL && active && p.D) ? __ldg(p.D + d) : 0.0f;
+  const float a0 = cm.x;
+  const float Dd = FULL ? cm.z : 0.0f;
   const float* Arow = p.A + (int64_t)(active ? d : 0) * NS;
 
   if (!jb.first && !cx.wait_predecessor(jb)) return false;
@@ -521,10 +625,10 @@ __device__ __forceinline__ bool run_job(WarpCtx<TIO, NS, TILE, STAGES>& cx, cons
     const float* src = nullptr;
     if (!jb.first) {
       const int64_t slot_i = (int64_t)jb.stream * 2 + ((jb.chunk - 1) & 1);
-      src = p.ring + slot_i * (kGroup * NS) + lane * NS;
-      if (!FULL) sd = p.ring_sd[slot_i * kGroup + lane];
+      src = p.ring + slot_i * (kCPW * NS) + c * NS;
+      if (!FULL) sd = __ldcg(p.ring_sd + slot_i * kCPW + c);
     } else if (FULL) {
-      if (jb.super_idx > 0) src = p.hin + ((int64_t)jb.stream * kGroup + lane) * NS;
+      if (jb.super_idx > 0) src = p.hin + ((int64_t)jb.stream * kCPW + c) * NS;
       else if (p.h0 && active) src = p.h0 + ((int64_t)jb.b * p.channels + d) * NS;
     }
 #pragma unroll
@@ -537,7 +641,16 @@ __device__ __forceinline__ bool run_job(WarpCtx<TIO, NS, TILE, STAGES>& cx, cons
         ak0 = active ? __ldg(Arow + 2 * k) : -1.0f;
         ak1 = active ? __ldg(Arow + 2 * k + 1) : -1.0f;
       }
-      g[k] = src ? f2(src[2 * k] * ak0, src[2 * k + 1] * ak1) : f2(0.0f, 0.0f);
+      g[k] = src ? f2(__ldcg(src + 2 * k) * ak0, __ldcg(src + 2 * k + 1) * ak1) : f2(0.0f, 0.0f);
+    }
+  }
+  float kA[STRUCT ? 1 : NS], kC[STRUCT ? 1 : NS];
+  if constexpr (!STRUCT) {
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+      const float an = active ? __ldg(Arow + k) : -1.0f;
+      kA[k] = an * 1.4426950408889634f;
+      kC[k] = (float)(k + 1) / an;
     }
   }
 
@@ -545,22 +658,16 @@ __device__ __forceinline__ bool run_job(WarpCtx<TIO, NS, TILE, STAGES>& cx, cons
   for (int it = 0; it < jb.ntiles; ++it) {
     const int64_t tt0 = jb.t0 + (int64_t)it * TILE;
     const int rows = (int)(jb.t1 - tt0 < (int64_t)TILE ? jb.t1 - tt0 : (int64_t)TILE);
-    if (!cx.acquire_tile(jb, tt0, rows, d, active)) return false;
-    const int slot = cx.cm_seq % STAGES;
-    const TIO* su = &sm.u[slot][0][lane];
-    const TIO* sdl = &sm.dl[slot][0][lane];
+    const int slot = it == 0 ? s0 : cx.wait_tile();
+    if (slot < 0) return false;
+    if (!p.use_tma) cx.fetch_tile(slot, jb, tt0, rows, d, active);
+    const TIO* su = &sm.u[slot][0][c];
+    const TIO* sdl = &sm.dl[slot][0][c];
     if constexpr (STRUCT) {
-      constexpr bool kFastQ = sizeof(TIO) == 2;  // bf16 data: hardware exp2 for expm1(Delta A_0)
-      tile_structured<TIO, NS, TILE, FULL, kFastQ>(su, sdl, sm.b[slot], sm.cs[slot], rows, a0, 1.0f / a0, Dd, g,
-                                                   sd, yrow, p.channels, active);
+      constexpr bool kFastQ = sizeof(TIO) == 2;  // bf16 data: hardware exp2 for expm1
+      tile_structured<TIO, NS, TILE, FULL, kFastQ>(su, sdl, sm.b[slot], sm.cs[slot], rows, a0, cm.y, Dd, g, sd, yrow,
+                                                   p.channels, active);
     } else {
-      float kA[NS], kC[NS];
-#pragma unroll
-      for (int n = 0; n < NS; ++n) {
-        const float an = active ? __ldg(Arow + n) : -1.0f;
-        kA[n] = an * 1.4426950408889634f;
-        kC[n] = (float)(n + 1) / an;
-      }
       tile_general<TIO, NS, FULL>(su, sdl, sm.b[slot], sm.cs[slot], rows, kA, kC, Dd, g, sd, yrow, p.channels,
                                   active);
     }
@@ -573,47 +680,50 @@ __device__ __forceinline__ bool run_job(WarpCtx<TIO, NS, TILE, STAGES>& cx, cons
   float* dst_sd = nullptr;
   if (!jb.last) {
     const int64_t slot_i = (int64_t)jb.stream * 2 + (jb.chunk & 1);
-    dst = p.ring + slot_i * (kGroup * NS) + lane * NS;
-    if (!FULL) dst_sd = p.ring_sd + slot_i * kGroup + lane;
+    dst = p.ring + slot_i * (kCPW * NS) + c * NS;
+    if (!FULL) dst_sd = p.ring_sd + slot_i * kCPW + c;
   } else if (FULL) {
     dst = (p.final_state && active && jb.super_idx == p.supers - 1)
               ? p.final_state + ((int64_t)jb.b * p.channels + d) * NS
               : nullptr;
   } else {
-    dst = p.agg_h + ((int64_t)jb.stream * kGroup + lane) * NS;
-    dst_sd = p.agg_sd + (int64_t)jb.stream * kGroup + lane;
+    dst = p.agg_h + ((int64_t)jb.stream * kCPW + c) * NS;
+    dst_sd = p.agg_sd + (int64_t)jb.stream * kCPW + c;
   }
   if (dst) {
 #pragma unroll
-    for (int n = 0; n < NS; ++n) {
+    for (int k = 0; k < NS; ++k) {
       float inv;
-      if constexpr (STRUCT) inv = 1.0f / ((float)(n + 1) * a0);
-      else inv = active ? 1.0f / __ldg(Arow + n) : -1.0f;
-      dst[n] = ((n & 1) ? g[n >> 1].y : g[n >> 1].x) * inv;
+      if constexpr (STRUCT) inv = 1.0f / ((float)(k + 1) * a0);
+      else inv = active ? 1.0f / __ldg(Arow + k) : -1.0f;
+      dst[k] = ((k & 1) ? g[k >> 1].y : g[k >> 1].x) * inv;
     }
   }
   if (dst_sd) *dst_sd = sd;
   if (!jb.last) {
-    __threadfence();
+    // the warp barrier orders every lane's state stores before lane 0's
+    // hand-off, which releases them with the flag
     __syncwarp();
-    if (lane == 0) st_release(&p.done[jb.stream], jb.chunk + 1);
+    if (c == 0) cx.publish(jb.stream, jb.chunk + 1);
   }
   __syncwarp();
   return true;
 }
 
 // ---------------------------------------------------------------------------
-// the persistent chunked scan kernel
+// the persistent chunked scan kernel: CW consumer warps (one job at a time
+// each) and one producer warp (index CW) per CTA
 // ---------------------------------------------------------------------------
-template <typename TIO, int NS, int TILE, int STAGES>
-__global__ void __launch_bounds__(kWarpsPerCta * 32, 1)
+template <typename TIO, int NS, int CW, int TILE, int STAGES>
+__global__ void __launch_bounds__((CW + 1) * 32, 1)
 scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__ CUtensorMap map_u,
                    const __grid_constant__ CUtensorMap map_dl, const __grid_constant__ CUtensorMap map_b,
                    const __grid_constant__ CUtensorMap map_c) {
   using Smem = WarpSmem<TIO, NS, TILE, STAGES>;
   // TMA destinations must start on 128-byte boundaries
   static_assert(sizeof(Smem) % 128 == 0, "per-warp block keeps 128-byte alignment");
-  static_assert((sizeof(TIO) * TILE * kGroup) % 128 == 0 && (sizeof(TIO) * TILE * NS) % 128 == 0,
+  static_assert((sizeof(TIO) * TILE * kCPW) % 128 == 0 && (sizeof(TIO) * TILE * NS) % 128 == 0 &&
+                    (sizeof(float) * TILE * NS) % 128 == 0,
                 "tile slots keep 128-byte alignment");
   extern __shared__ __align__(128) unsigned char smem_raw[];
   const int warp = threadIdx.x >> 5;
@@ -621,76 +731,97 @@ scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__
   // align to 128 bytes by pointer arithmetic (an integer round trip would
   // hide from the compiler that these are shared-memory addresses)
   unsigned char* smem_base = smem_raw + ((128u - (smem_addr(smem_raw) & 127u)) & 127u);
-  Smem& sm = reinterpret_cast<Smem*>(smem_base)[warp];
+  Smem* sms = reinterpret_cast<Smem*>(smem_base);
 
-  if (lane == 0) {
-    for (int s = 0; s < STAGES; ++s) mbar_init(&sm.full[s], 1);
-    fence_mbar_init();
-    if (p.use_tma) {
-      tma_prefetch_desc(&map_u);
-      tma_prefetch_desc(&map_dl);
-      tma_prefetch_desc(&map_b);
-      tma_prefetch_desc(&map_c);
+  if (threadIdx.x < CW) {
+    Smem& s = sms[threadIdx.x];
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
     }
+    s.hq_head = 0;
+    s.hq_tail = 0;
+    s.finished = 0;
+    fence_mbar_init();
   }
-  __syncwarp();
-
-  WarpCtx<TIO, NS, TILE, STAGES> cx(p, sm, &map_u, &map_dl, &map_b, &map_c, lane);
-  // ring entry 0 is a sentinel "before the first job": the first produce()
-  // pulls job #1 into entry 1
-  if (lane == 0) {
-    sm.ring_jobs[0] = -1;
-    cx.pulled = 1;
-    cx.produce();
+  if (threadIdx.x == CW * 32 && p.use_tma) {
+    tma_prefetch_desc(&map_u);
+    tma_prefetch_desc(&map_dl);
+    tma_prefetch_desc(&map_b);
+    tma_prefetch_desc(&map_c);
   }
-  __syncwarp();
+  // the setup above overlaps the end of the previous kernel (programmatic
+  // launch); everything below reads what it wrote
+  griddep_wait();
+  __syncthreads();
 
+  if (warp == CW) {
+    if (lane == 0) producer_loop<TIO, NS, CW, TILE, STAGES>(p, sms, &map_u, &map_dl, &map_b, &map_c);
+    return;
+  }
+
+  Consumer<TIO, NS, TILE, STAGES> cx(p, sms[warp], lane);
   const bool full_mode = (p.mode == kModeFull);
   for (;;) {
-    const int j = cx.next_job();
-    if (j < 0) break;
+    const int s0 = cx.wait_tile();
+    if (s0 < 0) break;
+    const int j = cx.sm.job[s0];
+    if (j < 0) break;  // the producer's end mark
     const Job jb = decode_job(p, j, TILE);
-    const int d = jb.d0 + lane;
-    const bool active = d < p.channels;
-    // structured A: A[d,n] == (n+1) A[d,0] exactly, on every lane of the warp
-    const float* Arow = p.A + (int64_t)(active ? d : 0) * NS;
-    const float a0 = active ? __ldg(Arow) : -1.0f;
-    bool structured = !p.force_general && a0 < 0.0f;
-#pragma unroll
-    for (int n = 1; n < NS; ++n) structured = structured && (!active || __ldg(Arow + n) == (float)(n + 1) * a0);
-    structured = __all_sync(0xffffffffu, structured);
+    const float4 cm = p.use_tma ? cx.sm.chan[s0][lane] : __ldg(p.chan + jb.d0 + lane);
+    // structured A on every channel of the warp (decided per channel by the pre-pass)
+    const bool structured = __all_sync(0xffffffffu, cm.w != 0.0f);
     bool ok;
     if (structured)
-      ok = full_mode ? run_job<TIO, NS, TILE, STAGES, true, true>(cx, jb, a0)
-                     : run_job<TIO, NS, TILE, STAGES, true, false>(cx, jb, a0);
+      ok = full_mode ? run_job<TIO, NS, TILE, STAGES, true, true>(cx, jb, s0, cm)
+                     : run_job<TIO, NS, TILE, STAGES, true, false>(cx, jb, s0, cm);
     else
-      ok = full_mode ? run_job<TIO, NS, TILE, STAGES, false, true>(cx, jb, a0)
-                     : run_job<TIO, NS, TILE, STAGES, false, false>(cx, jb, a0);
+      ok = full_mode ? run_job<TIO, NS, TILE, STAGES, false, true>(cx, jb, s0, cm)
+                     : run_job<TIO, NS, TILE, STAGES, false, false>(cx, jb, s0, cm);
     if (!ok) break;
   }
-
-  // Drain: every TMA load this warp issued must land before the CTA exits.
   __syncwarp();
-  if (lane == 0 && p.use_tma) {
-    for (uint32_t s = cx.cm_seq; s < cx.ld_seq; ++s) {
-      if (!mbar_wait_bounded(&sm.full[s % STAGES], (s / STAGES) & 1u, p.wait_limit_ns)) {
-        record_device_error(MAMBA_ERR_TIMEOUT);
-        break;
-      }
-    }
-  }
-  __syncwarp();
+  if (lane == 0) st_release_cta_smem(&cx.sm.finished, 1);
 }
 
 // ---------------------------------------------------------------------------
-// pre-pass: C' = C / (n+1) in fp32, one thread per (token row, state)
+// pre-pass, one thread per element of three ranges:
+//   [0, zero_words):          the job counters and progress flags = 0
+//   C' = C / (n+1) in fp32 for every (token row, state)
+//   per channel {A[d,0], 1/A[d,0], D[d], structured}, where "structured"
+//   means A[d,n] == (n+1) A[d,0] exactly for every n, A[d,0] < 0 and the
+//   general path was not forced; padding channels get {-1, -1, 0, 1}.
 // ---------------------------------------------------------------------------
 template <typename TIO, int NS>
-__global__ void scan_prep_c_kernel(const TIO* __restrict__ C, float* __restrict__ cs, int64_t total) {
-  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  if (i >= total) return;
-  const int n = (int)(i % NS);
-  cs[i] = to_f32(C[i]) / (float)(n + 1);
+__global__ void scan_prep_kernel(int* __restrict__ zero, int64_t zero_words, const TIO* __restrict__ C,
+                                 float* __restrict__ cs, int64_t total_c, const float* __restrict__ A,
+                                 const float* __restrict__ D, float4* __restrict__ chan, int64_t channels,
+                                 int64_t chan_padded, int force_general) {
+  griddep_launch_dependents();  // the scan kernel may start its setup
+  int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  griddep_wait();  // the scratch may still be in use by the previous kernel of the stream
+  if (i < zero_words) {
+    zero[i] = 0;
+    return;
+  }
+  i -= zero_words;
+  if (i < total_c) {
+    const int n = (int)(i % NS);
+    cs[i] = to_f32(C[i]) / (float)(n + 1);
+    return;
+  }
+  const int64_t d = i - total_c;
+  if (d >= chan_padded) return;
+  if (d >= channels) {
+    chan[d] = make_float4(-1.0f, -1.0f, 0.0f, 1.0f);
+    return;
+  }
+  const float* row = A + d * NS;
+  const float a0 = row[0];
+  bool structured = !force_general && a0 < 0.0f;
+#pragma unroll
+  for (int n = 1; n < NS; ++n) structured &= (row[n] == (float)(n + 1) * a0);
+  chan[d] = make_float4(a0, 1.0f / a0, D ? D[d] : 0.0f, structured ? 1.0f : 0.0f);
 }
 
 // ---------------------------------------------------------------------------
@@ -700,23 +831,25 @@ __global__ void scan_prep_c_kernel(const TIO* __restrict__ C, float* __restrict_
 // ---------------------------------------------------------------------------
 template <int NS>
 __global__ void scan_combine_kernel(const ScanParams p, float* hin) {
+  griddep_launch_dependents();
   const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  const int64_t total = (int64_t)p.groups * kGroup * NS;
+  griddep_wait();
+  const int64_t total = (int64_t)p.groups * kCPW * NS;
   if (tid >= total) return;
   const int n = (int)(tid % NS);
-  const int lane = (int)((tid / NS) % kGroup);
-  const int grp = (int)(tid / ((int64_t)NS * kGroup));
+  const int c = (int)((tid / NS) % kCPW);
+  const int grp = (int)(tid / ((int64_t)NS * kCPW));
   const int b = grp / p.groups_d;
-  const int d = (grp - b * p.groups_d) * kGroup + lane;
+  const int d = (grp - b * p.groups_d) * kCPW + c;
   const bool active = d < p.channels;
   const float a = active ? p.A[(int64_t)d * NS + n] : -1.0f;
   float h = (active && p.h0) ? p.h0[((int64_t)b * p.channels + d) * NS + n] : 0.0f;
   for (int j = 0; j + 1 < p.supers; ++j) {
     const int64_t s = (int64_t)j * p.groups + grp;
-    const float sdj = p.agg_sd[s * kGroup + lane];
-    const float H = p.agg_h[(s * kGroup + lane) * NS + n];
+    const float sdj = p.agg_sd[s * kCPW + c];
+    const float H = p.agg_h[(s * kCPW + c) * NS + n];
     h = fmaf(expf(a * sdj), h, H);
-    hin[(((int64_t)(j + 1) * p.groups + grp) * kGroup + lane) * NS + n] = h;
+    hin[(((int64_t)(j + 1) * p.groups + grp) * kCPW + c) * NS + n] = h;
   }
 }
 

@@ -166,3 +166,14 @@ def test_workload_sampled(name, count):
     assert hf.shape == (w.batch, w.channels, w.nstate)
     del inp, y, hf
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("a_mode", ["channel", "random"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_scan_more_groups_than_warps(a_mode, dtype):
+    # 40 x 32 groups of 32 channels: more streams than resident consumer warps,
+    # so every warp runs several groups, without super-chunks
+    w = SMALL.with_(batch=40, length=96, channels=1024, a_mode=a_mode, dtype=dtype)
+    plan = m.mamba_scan_plan(w.batch, w.length, w.channels, 16, 0, m.dtype_code(w.torch_dtype))
+    assert plan.supers == 1
+    _check_full(w)
