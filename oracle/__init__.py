@@ -5,7 +5,9 @@ benchmark's CPU-baseline leg, never by the product library.  The arithmetic
 lives in `ssm_oracle.c` (plain C, double precision); this module only moves
 numpy arrays across ctypes.  It follows the zero-order-hold discretisation and
 recurrence of "Mamba SSM Nedir? Transformer Alternatifi Rehberi (2026)",
-sections "State Space Model Temelleri" and "Ayrık Zamana Geçiş".
+sections "State Space Model Temelleri" and "Ayrık Zamana Geçiş", and, as
+options, the exponential-Euler and trapezoidal discretisations that the
+Mamba-3 page names in "Geliştirilmiş Ayrıklaştırma Şeması".
 """
 from __future__ import annotations
 
@@ -29,6 +31,8 @@ class Oracle:
         self._lib = ctypes.CDLL(os.path.abspath(path))
         self._lib.oracle_scan.restype = ctypes.c_int
         self._lib.oracle_scan.argtypes = [_c_f64p] * 9 + [_i64] * 4 + [ctypes.c_int]
+        self._lib.oracle_scan_method.restype = ctypes.c_int
+        self._lib.oracle_scan_method.argtypes = [_c_f64p] * 9 + [_i64] * 4 + [ctypes.c_int, ctypes.c_int]
         self._lib.oracle_state_update.restype = ctypes.c_int
         self._lib.oracle_state_update.argtypes = [_c_f64p] * 8 + [_i64] * 3 + [ctypes.c_int]
         self._lib.oracle_max_threads.restype = ctypes.c_int
@@ -41,10 +45,15 @@ class Oracle:
     def _f64(a):
         return None if a is None else np.ascontiguousarray(np.asarray(a, dtype=np.float64))
 
-    def scan(self, u, delta, A, B, C, D=None, h0=None, want_y=True, nthreads=0):
+    # discretisations (oracle_scan_method): zero-order hold, exponential
+    # Euler, trapezoidal -- see ssm_oracle.c for the readings
+    ZOH, EULER, TRAPEZOID = 0, 1, 2
+
+    def scan(self, u, delta, A, B, C, D=None, h0=None, want_y=True, nthreads=0, method=0):
         """Selective scan.  u, delta: (batch, len, channels); B, C: (batch, len,
         nstate); A: (channels, nstate); D: (channels,) or None; h0: (batch,
-        channels, nstate) or None.  Returns (y, h_final) in float64."""
+        channels, nstate) or None; method: ZOH, EULER or TRAPEZOID.  Returns
+        (y, h_final) in float64."""
         u, delta, A, B, C, D, h0 = map(self._f64, (u, delta, A, B, C, D, h0))
         batch, length, channels = u.shape
         nstate = A.shape[1]
@@ -54,9 +63,15 @@ class Oracle:
         assert h0 is None or h0.shape == (batch, channels, nstate)
         y = np.empty_like(u) if want_y else None
         hf = np.empty((batch, channels, nstate), dtype=np.float64)
-        rc = self._lib.oracle_scan(self._ptr(u), self._ptr(delta), self._ptr(A), self._ptr(B),
-                                   self._ptr(C), self._ptr(D), self._ptr(h0), self._ptr(y),
-                                   self._ptr(hf), batch, length, channels, nstate, int(nthreads))
+        if method == self.ZOH:
+            rc = self._lib.oracle_scan(self._ptr(u), self._ptr(delta), self._ptr(A), self._ptr(B),
+                                       self._ptr(C), self._ptr(D), self._ptr(h0), self._ptr(y),
+                                       self._ptr(hf), batch, length, channels, nstate, int(nthreads))
+        else:
+            rc = self._lib.oracle_scan_method(self._ptr(u), self._ptr(delta), self._ptr(A), self._ptr(B),
+                                              self._ptr(C), self._ptr(D), self._ptr(h0), self._ptr(y),
+                                              self._ptr(hf), batch, length, channels, nstate, int(method),
+                                              int(nthreads))
         if rc != 0:
             raise RuntimeError(f"oracle_scan failed ({rc})")
         return y, hf

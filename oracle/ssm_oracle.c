@@ -166,6 +166,113 @@ int oracle_state_update(double *state, const double *x, const double *delta,
     return 0;
 }
 
+/* ------------------------------------------------------------------------
+ * Discretisations other than zero-order hold.
+ *
+ * The Mamba-3 page (bitig.info, section "Geliştirilmiş Ayrıklaştırma
+ * Şeması") says Mamba-1 and Mamba-2 discretised the continuous system with
+ * "the Euler method" and Mamba-3 with the trapezoidal rule, and gives no
+ * formula for either.  Readings (listed in the design notes):
+ *   method 1, exponential Euler: the state transition stays exp(Delta A)
+ *     (as in the zero-order hold of "Ayrık Zamana Geçiş"), the input term is
+ *     taken to first order, Bbar = Delta B:
+ *         h_t = exp(Delta_t A) h_{t-1} + Delta_t B_t x_t
+ *   method 2, trapezoidal: the exact step is
+ *         h_t = exp(Delta A) h_{t-1} + int_0^Delta exp(A (Delta - s)) B(s) x(s) ds
+ *     and the trapezoid rule takes the integral from its two end points, the
+ *     previous token at s = 0 and the current one at s = Delta:
+ *         h_t = exp(Delta_t A) h_{t-1}
+ *               + (Delta_t / 2) (exp(Delta_t A) B_{t-1} x_{t-1} + B_t x_t)
+ *     with B_{-1} x_{-1} = 0: the first token of a call has no predecessor,
+ *     also when an initial state is given.
+ * For every method y_t = C_t . h_t + D x_t.
+ * ------------------------------------------------------------------------ */
+static void scan_row_method(const double *u, const double *delta, const double *A_row,
+                            const double *B, const double *C, double D_d, int has_D,
+                            double *y, double *h, int64_t len, int64_t stride, int64_t nstate,
+                            int method)
+{
+    for (int64_t t = 0; t < len; ++t) {
+        double x = u[t * stride];
+        double dt = delta[t * stride];
+        const double *Bt = B + t * nstate;
+        const double *Ct = C + t * nstate;
+        double acc = 0.0;
+        for (int64_t n = 0; n < nstate; ++n) {
+            double abar = exp(dt * A_row[n]);
+            double input;
+            if (method == 1) {
+                input = dt * Bt[n] * x;
+            } else {
+                double previous = 0.0;   /* exp(Delta_t A) B_{t-1} x_{t-1} */
+                if (t > 0)
+                    previous = abar * B[(t - 1) * nstate + n] * u[(t - 1) * stride];
+                input = 0.5 * dt * (previous + Bt[n] * x);
+            }
+            h[n] = abar * h[n] + input;
+            acc += Ct[n] * h[n];
+        }
+        if (has_D)
+            acc += D_d * x;
+        if (y)
+            y[t * stride] = acc;
+    }
+}
+
+/* Selective scan with the discretisation `method` (0: zero-order hold, the
+ * same as oracle_scan; 1: exponential Euler; 2: trapezoidal).  Returns 0, or
+ * -1 on a bad argument.                                                       */
+int oracle_scan_method(const double *u, const double *delta, const double *A,
+                       const double *B, const double *C, const double *D,
+                       const double *h0, double *y, double *h_final,
+                       int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                       int method, int nthreads)
+{
+    if (method == 0)
+        return oracle_scan(u, delta, A, B, C, D, h0, y, h_final, batch, len, channels, nstate, nthreads);
+    if (method != 1 && method != 2)
+        return -1;
+    if (batch < 0 || len < 0 || channels < 0 || nstate <= 0)
+        return -1;
+    if ((len > 0 && (!u || !delta || !B || !C)) || !A)
+        return -1;
+    int64_t rows = batch * channels;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = 0;
+#pragma omp parallel
+    {
+        double *h = (double *)malloc(sizeof(double) * (size_t)nstate);
+        if (!h) {
+#pragma omp atomic write
+            status = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < rows; ++r) {
+            if (!h)
+                continue;
+            int64_t b = r / channels, d = r % channels;
+            for (int64_t n = 0; n < nstate; ++n)
+                h[n] = h0 ? h0[(b * channels + d) * nstate + n] : 0.0;
+            const size_t tok0 = (size_t)(b * len) * (size_t)channels + (size_t)d;
+            scan_row_method(len ? u + tok0 : NULL, len ? delta + tok0 : NULL, A + d * nstate,
+                            len ? B + (size_t)(b * len) * (size_t)nstate : NULL,
+                            len ? C + (size_t)(b * len) * (size_t)nstate : NULL,
+                            D ? D[d] : 0.0, D != NULL, (y && len) ? y + tok0 : NULL, h,
+                            len, channels, nstate, method);
+            if (h_final)
+                for (int64_t n = 0; n < nstate; ++n)
+                    h_final[(b * channels + d) * nstate + n] = h[n];
+        }
+        free(h);
+    }
+    return status;
+}
+
 /* Threads the OpenMP runtime would use (for reporting the CPU baseline). */
 int oracle_max_threads(void)
 {

@@ -302,3 +302,94 @@ def test_empty_sequence(oracle_lib):
     u = np.zeros((2, 0, 3))
     _, hf = oracle_lib.scan(u, u, -np.ones((3, 4)), np.zeros((2, 0, 4)), np.zeros((2, 0, 4)), None)
     assert hf.shape == (2, 3, 4) and not hf.any()
+
+
+# --- discretisations named on the Mamba-3 page -----------------------------------------
+# "Geliştirilmiş Ayrıklaştırma Şeması": Mamba-1/2 used the Euler method, Mamba-3 the
+# trapezoidal rule.  Readings (ssm_oracle.c): exponential Euler keeps exp(Delta A) and
+# takes Bbar = Delta B; the trapezoid rule takes the step's input integral from the
+# previous token (weighted by exp(Delta A)) and the current one, Delta/2 each.
+
+def _impulse_inputs(L, delta, a, b, c):
+    x = np.zeros((1, L, 1))
+    x[0, 0, 0] = 1.0
+    x[0, 7, 0] = -0.5                                   # a second impulse: superposition
+    return (x, np.full((1, L, 1), delta), np.array([a]), np.tile(np.array(b), (1, L, 1)),
+            np.tile(np.array(c), (1, L, 1)))
+
+
+@pytest.mark.parametrize("method", ["euler", "trapezoid"])
+def test_methods_impulse_response_closed_form(oracle_lib, method):
+    """Constant Delta, B, C: the response to an impulse at t=0 is, in closed form,
+    exponential Euler  h_k = Abar^k Delta B          (k >= 0)
+    trapezoid          h_0 = Delta/2 B,  h_k = Abar^k Delta B  (k >= 1)
+    (the previous-token term of step 1 carries the other half, decayed once);
+    a second impulse adds its shifted, scaled copy."""
+    L, dt = 20, 0.3
+    a, b, c = [-0.5, -2.0, -7.0], [1.0, -0.4, 0.25], [0.3, 1.1, -0.8]
+    u, delta, A, B, C = _impulse_inputs(L, dt, a, b, c)
+    m = oracle_lib.EULER if method == "euler" else oracle_lib.TRAPEZOID
+    y, _ = oracle_lib.scan(u, delta, A, B, C, None, method=m)
+    abar = np.exp(dt * np.array(a))
+    k = np.arange(L)[:, None]
+    resp = (abar[None, :] ** k) * dt * np.array(b)[None, :]        # Abar^k Delta B
+    if method == "trapezoid":
+        resp[0] = 0.5 * dt * np.array(b)
+    kernel = resp @ np.array(c)                                      # C . h_k
+    expect = kernel.copy()
+    expect[7:] += -0.5 * kernel[:L - 7]
+    np.testing.assert_allclose(y[0, :, 0], expect, rtol=1e-13, atol=1e-15)
+
+
+def test_methods_order_of_accuracy(oracle_lib):
+    """Against the continuous system h' = A h + B x(t) with a smooth input that
+    starts at x(0) = 0 (solved by scipy to 1e-12): zero-order hold and exponential
+    Euler converge at first order in Delta, the trapezoidal rule at second order."""
+    a = np.array([-1.0, -3.0])
+    b = np.array([1.0, 0.5])
+    c = np.array([1.0, 1.0])
+    T = 4.0
+
+    def xf(t):
+        return np.sin(2.0 * t) + 0.5 * np.sin(0.7 * t)
+
+    def exact(ts):
+        sol = scipy.integrate.solve_ivp(lambda t, h: a * h + b * xf(t), (0.0, T), [0.0, 0.0],
+                                        t_eval=ts, rtol=1e-12, atol=1e-14, method="DOP853")
+        return c @ sol.y
+
+    errs = {}
+    for dt in (0.02, 0.01):
+        L = int(round(T / dt))
+        ts = dt * np.arange(1, L + 1)            # token t closes the step ending at (t+1) Delta
+        ref = exact(ts)
+        u = xf(ts).reshape(1, L, 1)
+        delta = np.full((1, L, 1), dt)
+        B = np.tile(b, (1, L, 1))
+        C = np.tile(c, (1, L, 1))
+        for name, m in (("zoh", oracle_lib.ZOH), ("euler", oracle_lib.EULER), ("trap", oracle_lib.TRAPEZOID)):
+            y, _ = oracle_lib.scan(u, delta, a[None, :], B, C, None, method=m)
+            errs[(name, dt)] = np.max(np.abs(y[0, :, 0] - ref))
+    for name, lo, hi in (("zoh", 1.6, 2.4), ("euler", 1.6, 2.4), ("trap", 3.3, 4.7)):
+        ratio = errs[(name, 0.02)] / errs[(name, 0.01)]
+        assert lo < ratio < hi, f"{name}: error ratio {ratio:.2f} for halved Delta"
+    assert errs[("trap", 0.01)] < 0.1 * errs[("euler", 0.01)]
+
+
+@pytest.mark.parametrize("method", ["euler", "trapezoid"])
+def test_methods_share_the_zoh_transition(oracle_lib, method):
+    """All three discretisations keep Abar = exp(Delta A), so the part of y that an
+    initial state contributes (y(h0) - y(0), linear in h0) is the same as under
+    zero-order hold; and as Delta -> 0 the output tends to D x."""
+    rng = np.random.default_rng(11)
+    u, delta, A, B, C, D = _rand_inputs(rng, 2, 30, 3, 4)
+    h0 = rng.standard_normal((2, 3, 4))
+    m = oracle_lib.EULER if method == "euler" else oracle_lib.TRAPEZOID
+    y1, _ = oracle_lib.scan(u, delta, A, B, C, D, h0=h0, method=m)
+    y0, _ = oracle_lib.scan(u, delta, A, B, C, D, method=m)
+    z1, _ = oracle_lib.scan(u, delta, A, B, C, D, h0=h0)
+    z0, _ = oracle_lib.scan(u, delta, A, B, C, D)
+    np.testing.assert_allclose(y1 - y0, z1 - z0, rtol=1e-10, atol=1e-12)
+    tiny = np.full_like(delta, 1e-14)
+    yt, _ = oracle_lib.scan(u, tiny, A, B, C, D, method=m)
+    np.testing.assert_allclose(yt, u * D[None, None, :], rtol=0, atol=1e-12)
