@@ -57,6 +57,9 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--length-sweep", action="store_true",
+                    help="instead of the benchmark line: ns per token-channel of the long-context workload's "
+                         "generator (1 x L x 2048, bf16) for L = 2^14 .. 2^20 (linear scaling in length)")
     return ap.parse_args()
 
 
@@ -280,6 +283,24 @@ def oracle_sample_rate(inp, w, budget_s: float, max_rows=None):
     return best, orc.max_threads()
 
 
+def oracle_single_thread_tiny(budget_s: float = 1.0) -> dict:
+    """tc/s of the fp64 oracle on one host thread over the tiny fp32 workload."""
+    import oracle
+    from selective_state_space_29_b200 import workloads as wl
+    orc = oracle.get()
+    w = wl.SCAN_WORKLOADS["tiny_f32"]
+    inp = {k: v.to("cpu", copy=True).double().numpy() for k, v in wl.scan_inputs(w, "cpu").items()}
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        orc.scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], nthreads=1)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= budget_s:
+            break
+    tc = w.batch * w.length * w.channels
+    return {"value": reps * tc / dt, "unit": UNIT, "cores": 1, "reps": reps}
+
+
 # --- our implementation ---------------------------------------------------------------
 
 def run_ours(args):
@@ -412,7 +433,8 @@ def run_ours(args):
         best, cores = oracle_sample_rate(inp, w, budget_s=10.0)
         out["cpu_baseline"] = {"value": best["value"], "unit": UNIT, "cores": cores, "kind": "oracle",
                                "sample": f"{best['rows']} of {w.batch * w.channels} (batch, channel) rows x "
-                                         f"{w.length} tokens of {w.name} ({best['seconds']:.1f} s, fp64)"}
+                                         f"{w.length} tokens of {w.name} ({best['seconds']:.1f} s, fp64)",
+                               "single_thread_tiny_f32": oracle_single_thread_tiny()}
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -530,10 +552,60 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_length_sweep(args):
+    """Time per token·channel against sequence length: one input of the
+    long-context generator at the largest length, scanned over its first L
+    tokens (contiguous prefixes for batch 1)."""
+    import torch
+
+    from selective_state_space_29_b200 import mamba_ssm as m
+    from selective_state_space_29_b200 import workloads as wl
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    w = wl.SCAN_WORKLOADS["long_bf16"]
+    inp = wl.scan_inputs(w, dev)
+    y = torch.empty_like(inp["u"])
+    hf = torch.empty((w.batch, w.channels, w.nstate), device=dev, dtype=torch.float32)
+    lib = m.library()
+    dtc = m.dtype_code(w.torch_dtype)
+    stream = torch.cuda.current_stream(dev)
+    rows = []
+    L = 1 << 14
+    while L <= w.length:
+        def step():
+            st = lib.mamba_selective_scan(inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(),
+                                          inp["B"].data_ptr(), inp["C"].data_ptr(), inp["D"].data_ptr(),
+                                          y.data_ptr(), hf.data_ptr(), w.batch, L, w.channels, w.nstate, dtc,
+                                          stream.cuda_stream)
+            if st != 0:
+                raise m.MambaError(st, "mamba_selective_scan")
+        for _ in range(max(args.warmup, 3)):
+            step()
+        reps = max(5, min(args.steps, int(2e9 // (w.channels * L))))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(reps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b) / reps
+        plan = m.mamba_scan_plan(w.batch, L, w.channels, w.nstate, 0, dtc)
+        rows.append({"len": L, "ms": round(ms, 5), "ns_per_tc": round(ms * 1e6 / (w.channels * L), 6),
+                     "reps": reps, "supers": int(plan.supers)})
+        L *= 2
+    v = [r["ns_per_tc"] for r in rows]
+    print(json.dumps({"length_sweep": rows, "workload": f"{w.name} generator, batch 1, {w.channels} channels",
+                      "max_over_min_ns_per_tc": round(max(v) / min(v), 4)}), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.length_sweep:
+        run_length_sweep(args)
     else:
         run_ours(args)
 

@@ -54,7 +54,7 @@ constexpr int kDecodeWarps = 8;  // warps per CTA
 // FASTQ: exp(z) - 1 from the hardware exp2 (bf16 data); otherwise the
 // branch-free accurate form.
 template <typename TIO, int NS, int ROWS, bool FASTQ>
-__global__ void __launch_bounds__(kDecodeWarps * 32)
+__global__ void __launch_bounds__(kDecodeWarps * 32, 1)
 state_update_kernel(const DecodeArgs<TIO, NS> a) {
   constexpr int QPR = NS / 4;           // lanes per row
   constexpr int CPW = 32 / QPR;         // channels per warp
