@@ -72,6 +72,24 @@ typedef enum {
 
 /* Flags for mamba_selective_scan_ex. */
 #define MAMBA_SCAN_GENERAL_A 1u  /* never take the path for A[d][n] = (n+1) A[d][0] */
+/*
+ * Discretisation (default: zero-order hold, section "Ayrık Zamana Geçiş").
+ * The Mamba-3 page (bitig.info, "Geliştirilmiş Ayrıklaştırma Şeması") names
+ * the Euler method (Mamba-1/2) and the trapezoidal rule (Mamba-3) without
+ * formulas; these flags implement the readings
+ *   MAMBA_SCAN_EULER      exponential Euler: Abar = exp(Delta A), Bbar = Delta B
+ *                         h_t = exp(Delta_t A) h_{t-1} + Delta_t B_t x_t
+ *   MAMBA_SCAN_TRAPEZOID  trapezoid rule on the step's input integral:
+ *                         h_t = exp(Delta_t A) h_{t-1}
+ *                               + Delta_t/2 (exp(Delta_t A) B_{t-1} x_{t-1} + B_t x_t),
+ *                         no previous-token term at t = 0 (also with an
+ *                         initial state)
+ * y_t = C_t . h_t + D x_t in all cases.  Both run the general-A kernel path
+ * (one exponential per state); setting both is MAMBA_ERR_INVALID_ARG.
+ * mamba_state_update is zero-order hold only.
+ */
+#define MAMBA_SCAN_EULER 2u
+#define MAMBA_SCAN_TRAPEZOID 4u
 
 /*
  * Selective scan over whole sequences (sections "Ayrık Zamana Geçiş" and
@@ -111,7 +129,8 @@ int mamba_selective_scan(const void *u, const void *delta, const float *A,
  *   chunk_len      > 0: split every sequence into chunks of this many tokens
  *                  (the associative chunk combine is then always used);
  *                  0: chosen automatically
- *   flags          bitwise OR of MAMBA_SCAN_* flags
+ *   flags          bitwise OR of MAMBA_SCAN_* flags; unknown bits, or EULER
+ *                  together with TRAPEZOID, give MAMBA_ERR_INVALID_ARG
  */
 int mamba_selective_scan_ex(const void *u, const void *delta, const float *A,
                             const void *B, const void *C, const float *D,

@@ -231,7 +231,7 @@ int noalloc_scratch_address(void** out) {
 
 // Enqueue one scan with the given plan on caller-provided scratch (laid out
 // by scratch_layout): pre-pass, [aggregate pass, combine,] main pass.
-template <typename TIO, int NS>
+template <typename TIO, int NS, int METHOD>
 int launch_scan_on(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
                    const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
                    unsigned flags, int dtype, cudaStream_t stream, const Plan& pl, int sms,
@@ -281,7 +281,7 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
 
   constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES, kScanConsumers>();
   static_assert(smem <= 232448, "scan CTA exceeds the shared memory of an SM");
-  auto kern = scan_chunks_kernel<TIO, NS, kScanConsumers, TILE, STAGES>;
+  auto kern = scan_chunks_kernel<TIO, NS, kScanConsumers, TILE, STAGES, METHOD>;
   {
     // the dynamic shared-memory limit is a per-device attribute of the kernel
     static std::mutex mu_attr;
@@ -359,8 +359,16 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   } else {
     if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
   }
-  const int status = launch_scan_on<TIO, NS>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags,
+  int status;
+  if (flags & MAMBA_SCAN_EULER)
+    status = launch_scan_on<TIO, NS, kEuler>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags,
                                              dtype, stream, pl, sms, scratch);
+  else if (flags & MAMBA_SCAN_TRAPEZOID)
+    status = launch_scan_on<TIO, NS, kTrapezoid>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels,
+                                                 flags, dtype, stream, pl, sms, scratch);
+  else
+    status = launch_scan_on<TIO, NS, kZOH>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags,
+                                           dtype, stream, pl, sms, scratch);
   if (!noalloc && cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) return MAMBA_ERR_CUDA;
   return status;
 }
@@ -424,7 +432,8 @@ int mamba_selective_scan_ex(const void* u, const void* delta, const float* A, co
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
   if (batch < 0 || len < 0 || channels < 0 || nstate <= 0 || chunk_len < 0) return MAMBA_ERR_INVALID_ARG;
-  if (flags & ~MAMBA_SCAN_GENERAL_A) return MAMBA_ERR_INVALID_ARG;
+  if (flags & ~(MAMBA_SCAN_GENERAL_A | MAMBA_SCAN_EULER | MAMBA_SCAN_TRAPEZOID)) return MAMBA_ERR_INVALID_ARG;
+  if ((flags & MAMBA_SCAN_EULER) && (flags & MAMBA_SCAN_TRAPEZOID)) return MAMBA_ERR_INVALID_ARG;
   if (!mamba_scan_supported_nstate(nstate)) return MAMBA_ERR_UNSUPPORTED;
   if (batch == 0 || channels == 0) return MAMBA_OK;
   const size_t es = (size_t)elem_size(dtype);

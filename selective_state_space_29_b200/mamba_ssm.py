@@ -23,6 +23,8 @@ MAMBA_ERR_UNSUPPORTED = 2
 MAMBA_ERR_CUDA = 3
 MAMBA_ERR_TIMEOUT = 4
 MAMBA_SCAN_GENERAL_A = 1
+MAMBA_SCAN_EULER = 2
+MAMBA_SCAN_TRAPEZOID = 4
 
 class ScanPlan(ctypes.Structure):
     """mamba_scan_plan_t"""
@@ -175,13 +177,17 @@ def mamba_debug_expire_wait(limit_ns: int, stream=None):
 
 # --- tensor-level helpers ---------------------------------------------------------
 
+_METHOD_FLAGS = {"zoh": 0, "euler": MAMBA_SCAN_EULER, "trapezoid": MAMBA_SCAN_TRAPEZOID}
+
+
 def selective_scan(u, delta, A, B, C, D=None, initial_state=None, return_final_state=True, chunk_len=0,
-                   general_a=False, y=None, final_state=None, stream=None):
+                   general_a=False, y=None, final_state=None, stream=None, method="zoh"):
     """y, final_state = selective_scan(u, delta, A, B, C, D) on CUDA tensors.
 
     u, delta: (batch, len, channels); B, C: (batch, len, nstate) of one dtype
     (float32 or bfloat16); A: (channels, nstate) float32; D: (channels,) or
-    None; initial_state: (batch, channels, nstate) float32 or None."""
+    None; initial_state: (batch, channels, nstate) float32 or None; method:
+    "zoh" (default), "euler" or "trapezoid" (see MAMBA_SCAN_EULER)."""
     import torch
     batch, length, channels = u.shape
     nstate = A.shape[1]
@@ -192,7 +198,7 @@ def selective_scan(u, delta, A, B, C, D=None, initial_state=None, return_final_s
         y = torch.empty_like(u)
     if final_state is None and return_final_state:
         final_state = torch.empty((batch, channels, nstate), device=u.device, dtype=torch.float32)
-    flags = MAMBA_SCAN_GENERAL_A if general_a else 0
+    flags = (MAMBA_SCAN_GENERAL_A if general_a else 0) | _METHOD_FLAGS[method]
     if initial_state is None and chunk_len == 0 and flags == 0:
         mamba_selective_scan(u, delta, A, B, C, D, y, final_state, batch, length, channels, nstate,
                              dtype_code(u.dtype), stream)

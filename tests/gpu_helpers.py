@@ -31,17 +31,21 @@ def row_error(gpu: np.ndarray, ref: np.ndarray, axis: int) -> float:
     return float((num / den).max()) if num.size else 0.0
 
 
-def gpu_scan(inp: dict, D=True, h0=None, chunk_len=0, general_a=False):
+def gpu_scan(inp: dict, D=True, h0=None, chunk_len=0, general_a=False, method="zoh"):
     y, hf = m.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"],
                              inp["D"] if D else None, initial_state=h0, chunk_len=chunk_len,
-                             general_a=general_a)
+                             general_a=general_a, method=method)
     torch.cuda.synchronize()
     return y, hf
 
 
-def oracle_scan_full(inp: dict, D=True, h0=None):
+ORACLE_METHOD = {"zoh": 0, "euler": 1, "trapezoid": 2}
+
+
+def oracle_scan_full(inp: dict, D=True, h0=None, method="zoh"):
     y, hf = oracle.scan(f64(inp["u"]), f64(inp["delta"]), f64(inp["A"]), f64(inp["B"]), f64(inp["C"]),
-                        f64(inp["D"]) if D else None, h0=None if h0 is None else f64(h0))
+                        f64(inp["D"]) if D else None, h0=None if h0 is None else f64(h0),
+                        method=ORACLE_METHOD[method])
     return y, hf
 
 

@@ -76,6 +76,7 @@ def test_scan_argument_errors_on_host(lib):
     assert _scan_ex(lib, channels=-1) == m.MAMBA_ERR_INVALID_ARG
     assert _scan_ex(lib, chunk=-1) == m.MAMBA_ERR_INVALID_ARG
     assert _scan_ex(lib, flags=8) == m.MAMBA_ERR_INVALID_ARG
+    assert _scan_ex(lib, flags=m.MAMBA_SCAN_EULER | m.MAMBA_SCAN_TRAPEZOID) == m.MAMBA_ERR_INVALID_ARG
     assert _scan_ex(lib, nstate=0) == m.MAMBA_ERR_INVALID_ARG
     assert _scan_ex(lib, nstate=12) == m.MAMBA_ERR_UNSUPPORTED
     assert _scan_ex(lib, u=None) == m.MAMBA_ERR_INVALID_ARG

@@ -19,14 +19,14 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 
-def _check_full(w: wl.ScanWorkload, chunk_len=0, general_a=False, D=True, h0_std=None, seed=None):
+def _check_full(w: wl.ScanWorkload, chunk_len=0, general_a=False, D=True, h0_std=None, seed=None, method="zoh"):
     inp = wl.scan_inputs(w, DEV, seed)
     h0 = None
     if h0_std is not None:
         g = torch.Generator(device=DEV).manual_seed(7)
         h0 = h0_std * torch.randn((w.batch, w.channels, w.nstate), generator=g, device=DEV)
-    y, hf = gpu_scan(inp, D=D, h0=h0, chunk_len=chunk_len, general_a=general_a)
-    yr, hr = oracle_scan_full(inp, D=D, h0=h0)
+    y, hf = gpu_scan(inp, D=D, h0=h0, chunk_len=chunk_len, general_a=general_a, method=method)
+    yr, hr = oracle_scan_full(inp, D=D, h0=h0, method=method)
     ey = row_error(f64(y), yr, axis=1)
     eh = row_error(f64(hf), hr, axis=2)
     tol = TOL[w.dtype]
@@ -177,3 +177,34 @@ def test_scan_more_groups_than_warps(a_mode, dtype):
     plan = m.mamba_scan_plan(w.batch, w.length, w.channels, 16, 0, m.dtype_code(w.torch_dtype))
     assert plan.supers == 1
     _check_full(w)
+
+
+# --- exponential-Euler and trapezoidal discretisations (flags of mamba_selective_scan_ex) ---
+
+@pytest.mark.parametrize("method", ["euler", "trapezoid"])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("a_mode", ["s4d", "random"])
+def test_scan_methods_small(method, dtype, a_mode):
+    _check_full(SMALL.with_(dtype=dtype, a_mode=a_mode), method=method)
+
+
+@pytest.mark.parametrize("chunk_len", [1, 37, 999])
+def test_scan_trapezoid_across_chunks(chunk_len):
+    # the previous token's input term crosses every chunk and super-chunk border
+    _check_full(SMALL.with_(length=600 if chunk_len == 1 else 1000), chunk_len=chunk_len, method="trapezoid")
+
+
+@pytest.mark.parametrize("method", ["euler", "trapezoid"])
+def test_scan_methods_initial_state_and_super_chunks(method):
+    _check_full(SMALL.with_(dtype="f32", length=400), chunk_len=100, h0_std=0.5, method=method)
+    _check_full(SMALL.with_(batch=1, length=20000, channels=64, delta_lo=1e-4), D=False, method=method)
+
+
+def test_scan_methods_flags_rejected_together():
+    inp = wl.scan_inputs(SMALL, DEV)
+    y = torch.empty_like(inp["u"])
+    st = m.library().mamba_selective_scan_ex(
+        inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(), inp["B"].data_ptr(),
+        inp["C"].data_ptr(), inp["D"].data_ptr(), None, y.data_ptr(), None, SMALL.batch, SMALL.length,
+        SMALL.channels, 16, 0, m.MAMBA_SCAN_EULER | m.MAMBA_SCAN_TRAPEZOID, m.MAMBA_BF16, None)
+    assert st == m.MAMBA_ERR_INVALID_ARG
