@@ -196,13 +196,13 @@ int mamba_selective_scan_noalloc(const void *u, const void *delta, const float *
 
 /* How mamba_selective_scan_ex would split a problem (host-side planning only). */
 typedef struct {
-    int64_t supers;        /* independent super-chunks per sequence (1: no aggregate/combine pass) */
+    int64_t supers;        /* independent super-chunks per sequence (1: no aggregate jobs) */
     int64_t super_len;     /* tokens per super-chunk (all but the last) */
     int64_t chunk_len;     /* tokens per job of the main pass */
-    int64_t jobs;          /* jobs of the main pass */
+    int64_t jobs;          /* jobs of the chunked kernel (aggregate and main) */
     int64_t kernels;       /* kernels one call launches */
     int64_t scratch_bytes; /* stream-ordered scratch one call allocates */
-    int64_t ctas;          /* CTAs of the main pass (persistent: at most one per SM) */
+    int64_t ctas;          /* CTAs of the chunked kernel (persistent: at most one per SM) */
 } mamba_scan_plan_t;
 
 /*

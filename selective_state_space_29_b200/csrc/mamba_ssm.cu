@@ -143,7 +143,7 @@ Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, 
 }
 
 struct ScratchLayout {
-  size_t ctr, done, ring, ring_sd, agg_h, agg_sd, hin, cs, chan, total;
+  size_t ctr, done, ring, ring_sd, agg_h, agg_sd, cs, chan, total;
 };
 
 ScratchLayout scratch_layout(const Plan& pl, int ns, int64_t batch, int64_t len) {
@@ -154,14 +154,13 @@ ScratchLayout scratch_layout(const Plan& pl, int ns, int64_t batch, int64_t len)
   ScratchLayout s;
   s.ctr = al(4 * sizeof(int));
   s.done = al(sizeof(int) * (size_t)(streams_full + streams_agg));
-  s.ring = al(sizeof(float) * (size_t)streams_full * 2 * kCPW * ns);
-  s.ring_sd = al(sizeof(float) * (size_t)streams_full * 2 * kCPW);
+  s.ring = al(sizeof(float) * (size_t)(streams_full + streams_agg) * 2 * kCPW * ns);
+  s.ring_sd = al(sizeof(float) * (size_t)(streams_full + streams_agg) * 2 * kCPW);
   s.agg_h = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kCPW * ns);
   s.agg_sd = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kCPW);
-  s.hin = S > 1 ? al(sizeof(float) * (size_t)streams_full * kCPW * ns) : 0;
   s.cs = al(sizeof(float) * (size_t)batch * (size_t)len * (size_t)ns);
   s.chan = al(sizeof(float) * 4 * (size_t)pl.groups_d * (size_t)kCPW);
-  s.total = s.ctr + s.done + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.hin + s.cs + s.chan;
+  s.total = s.ctr + s.done + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.cs + s.chan;
   return s;
 }
 
@@ -173,7 +172,7 @@ int64_t full_jobs(const Plan& pl) {
 
 int tile_for(int dtype) { return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16>::kTile : ScanCfg<float>::kTile; }
 
-int64_t kernels_per_call(const Plan& pl) { return pl.supers > 1 ? 4 : 2; }  // pre-pass, [aggregate, combine,] main
+int64_t kernels_per_call(const Plan&) { return 2; }  // pre-pass, chunked scan
 
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel of the stream finishes; it waits for that kernel's
@@ -246,8 +245,6 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   float* ring_sd = reinterpret_cast<float*>(cur); cur += sl.ring_sd;
   float* agg_h = reinterpret_cast<float*>(cur); cur += sl.agg_h;
   float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
-  float* hin = sl.hin ? reinterpret_cast<float*>(cur) : nullptr;
-  cur += sl.hin;
   float* cs = reinterpret_cast<float*>(cur); cur += sl.cs;
   float4* chan = reinterpret_cast<float4*>(cur);
 
@@ -271,7 +268,7 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   std::memset(&p, 0, sizeof(p));
   p.u = u; p.delta = delta; p.A = A; p.B = B; p.cs = cs; p.chan = chan; p.h0 = h0; p.y = y;
   p.final_state = final_state;
-  p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd; p.hin = hin;
+  p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd;
   p.batch = batch; p.len = len; p.channels = channels;
   p.groups_d = pl.groups_d; p.groups = (int)pl.groups;
   p.supers = pl.supers; p.super_len = pl.super_len; p.chunk_len = pl.chunk_len;
@@ -299,18 +296,16 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   const int64_t S = pl.supers;
   const int64_t streams_full = S * pl.groups;
   const int64_t streams_agg = (S - 1) * pl.groups;
-  if (full_jobs(pl) > 0x7fffffff || streams_agg * pl.chunks_full > 0x7fffffff || streams_full > 0x7fffffff)
-    return MAMBA_ERR_UNSUPPORTED;
-  auto run_pass = [&](int mode, int64_t streams, int64_t jobs, int* ctr, int* dn) -> cudaError_t {
-    ScanParams q = p;
-    q.mode = mode;
-    q.streams = (int)streams;
-    q.jobs = (int)jobs;
-    q.counters = ctr;
-    q.done = dn;
-    const int64_t ctas = std::min<int64_t>(sms, (jobs + kScanConsumers - 1) / kScanConsumers);
-    return launch_pdl(kern, dim3((unsigned)ctas), dim3((kScanConsumers + 1) * 32), smem, stream, q, mu, mdl, mb, mc);
-  };
+  const int64_t jobs_agg = streams_agg * pl.chunks_full;
+  const int64_t jobs = jobs_agg + full_jobs(pl);
+  if (jobs > 0x7fffffff || streams_full + streams_agg > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
+  p.streams_agg = (int)streams_agg;
+  p.streams_full = (int)streams_full;
+  p.jobs_agg = (int)jobs_agg;
+  p.jobs = (int)jobs;
+  p.counters = counters;
+  p.done = done;
+  p.done_agg = done + streams_full;
 
   // pre-pass: zero the counters and progress flags, C' = C / (n+1) in fp32,
   // and the per-channel constants
@@ -325,17 +320,12 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
         (flags & MAMBA_SCAN_GENERAL_A) ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return MAMBA_ERR_CUDA;
   }
-  if (S > 1) {
-    // aggregate pass over every super-chunk but the last, then the combine
-    if (run_pass(kModeAggregate, streams_agg, streams_agg * pl.chunks_full, counters + 2, done + streams_full) !=
-        cudaSuccess)
-      return MAMBA_ERR_CUDA;
-    const int64_t threads = pl.groups * kCPW * NS;
-    if (launch_pdl(scan_combine_kernel<NS>, dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, stream, p, hin) !=
-        cudaSuccess)
-      return MAMBA_ERR_CUDA;
-  }
-  if (run_pass(kModeFull, streams_full, full_jobs(pl), counters, done) != cudaSuccess) return MAMBA_ERR_CUDA;
+  // one persistent pass: the aggregate jobs of super-chunks 0..S-2 hold the
+  // first tickets, the main jobs follow
+  const int64_t ctas = std::min<int64_t>(sms, (jobs + kScanConsumers - 1) / kScanConsumers);
+  if (launch_pdl(kern, dim3((unsigned)ctas), dim3((kScanConsumers + 1) * 32), smem, stream, p, mu, mdl, mb, mc) !=
+      cudaSuccess)
+    return MAMBA_ERR_CUDA;
   return MAMBA_OK;
 }
 
@@ -418,7 +408,7 @@ int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate
   out->supers = pl.supers;
   out->super_len = pl.super_len;
   out->chunk_len = pl.chunk_len;
-  out->jobs = full_jobs(pl);
+  out->jobs = (int64_t)(pl.supers - 1) * pl.groups * pl.chunks_full + full_jobs(pl);
   out->kernels = kernels_per_call(pl);
   out->scratch_bytes = (int64_t)scratch_layout(pl, (int)nstate, batch, len).total;
   out->ctas = std::min<int64_t>(sms, (out->jobs + kScanConsumers - 1) / kScanConsumers);

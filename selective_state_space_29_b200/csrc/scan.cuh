@@ -25,10 +25,12 @@
 //   * When there are fewer groups than consumer warps, the sequence is also
 //     cut into "super-chunks" that run as independent streams.  Their
 //     starting states come from the associative combine of the page's
-//     parallel prefix scan ("Paralel Tarama Algoritması"): an aggregate pass
-//     computes, per super-chunk, the end state from zero H_j and sum of
-//     Delta; a combine pass runs h_{j+1} = exp(A sum Delta_j) h_j + H_j; the
-//     main pass then runs every super-chunk from its own starting state.
+//     parallel prefix scan ("Paralel Tarama Algoritması"): aggregate jobs
+//     (the first tickets) compute, per super-chunk but the last, the end
+//     state from zero H_j and the sum of Delta; the first main job of
+//     super-chunk j waits for the aggregates of super-chunks 0..j-1 and runs
+//     h <- exp(A sum Delta_i) h + H_i over them for its starting state.  All
+//     of it is one launch; every wait is for an earlier ticket.
 //
 // Arithmetic per token and state (all fp32; the state is kept scaled,
 // g_n = A_n h_n, so that 1/A_n leaves the inner loop):
@@ -58,7 +60,6 @@ namespace mamba {
 constexpr int kCPW = 32;   // channels per warp: one lane per channel
 constexpr int kHandQ = 8;  // hand-off flags a consumer may leave for the producer to publish
 
-enum ScanMode : int { kModeFull = 0, kModeAggregate = 1 };
 enum Discretisation : int { kZOH = 0, kEuler = 1, kTrapezoid = 2 };
 
 struct ScanParams {
@@ -74,12 +75,12 @@ struct ScanParams {
   float* final_state;       // nullable
   // scratch (stream-ordered; the pre-pass zeroes counters and done)
   int* counters;            // [0] job ticket, [1] abort flag
-  int* done;                // [streams] chunks completed per stream
-  float* ring;              // [streams][2][32][N] states handed between chunks
-  float* ring_sd;           // [streams][2][32] running sum of Delta (aggregate mode)
+  int* done;                // [S*G] chunks completed per main stream
+  int* done_agg;            // [(S-1)*G] chunks completed per aggregate stream
+  float* ring;              // [S*G + (S-1)*G][2][32][N] states handed between chunks
+  float* ring_sd;           // [S*G + (S-1)*G][2][32] running sum of Delta (aggregate jobs)
   float* agg_h;             // [(S-1)*G][32][N] aggregate end states
   float* agg_sd;            // [(S-1)*G][32]    aggregate sum of Delta
-  const float* hin;         // [S*G][32][N] starting state of each super-chunk (S > 1)
   // sizes
   int64_t batch, len, channels;
   int groups_d;             // ceil(channels / 32)
@@ -88,10 +89,11 @@ struct ScanParams {
   int64_t super_len;        // tokens per super-chunk (all but the last)
   int64_t chunk_len;        // tokens per chunk
   int chunks_full;          // chunks of a full super-chunk
-  int chunks_last;          // chunks of the last super-chunk (full mode)
-  int mode;
-  int streams;              // streams active in this pass
-  int jobs;                 // jobs in this pass (fits int32, checked on the host)
+  int chunks_last;          // chunks of the last super-chunk (main jobs)
+  int streams_agg;          // (S-1)*G aggregate streams: super-chunks 0..S-2 from zero
+  int streams_full;         // S*G main streams
+  int jobs_agg;             // aggregate jobs: tickets [0, jobs_agg)
+  int jobs;                 // all jobs (fits int32, checked on the host)
   int use_tma;
   uint64_t wait_limit_ns;
 };
@@ -100,7 +102,8 @@ struct ScanParams {
 // job bookkeeping
 // ---------------------------------------------------------------------------
 struct Job {
-  int stream;      // super * groups + group
+  bool agg;        // aggregate job (super-chunk end state from zero) or main job
+  int stream;      // super * groups + group (within its kind)
   int chunk;       // chunk index inside the stream
   int b, d0;       // batch row and first channel of the group
   int64_t t0, t1;  // token range [t0, t1) of this job
@@ -112,10 +115,11 @@ struct Job {
 __device__ __forceinline__ Job decode_job(const ScanParams& p, int j_in, int tile) {
   // 32-bit arithmetic: the host guarantees jobs, streams and b*len fit in int32
   Job jb;
-  const uint32_t j = (uint32_t)j_in;
-  const uint32_t n_all = (uint32_t)p.streams;
-  const uint32_t n_full = (p.mode == kModeFull) ? (uint32_t)(p.supers - 1) * (uint32_t)p.groups : n_all;
-  const uint32_t kmin = (uint32_t)((p.mode == kModeFull) ? p.chunks_last : p.chunks_full);
+  jb.agg = j_in < p.jobs_agg;
+  const uint32_t j = (uint32_t)(jb.agg ? j_in : j_in - p.jobs_agg);
+  const uint32_t n_all = (uint32_t)(jb.agg ? p.streams_agg : p.streams_full);
+  const uint32_t n_full = jb.agg ? n_all : (uint32_t)(p.supers - 1) * (uint32_t)p.groups;
+  const uint32_t kmin = (uint32_t)(jb.agg ? p.chunks_full : p.chunks_last);
   uint32_t k, s;
   if (j < kmin * n_all) {
     k = j / n_all;
@@ -158,7 +162,7 @@ struct alignas(128) WarpSmem {
   uint64_t full[STAGES];      // producer -> consumer: the tile has landed
   uint64_t empty[STAGES];     // consumer -> producer: the slot has been read
   int job[STAGES];            // job of the slot's tile; -1: no more jobs
-  int hq_stream[kHandQ];      // hand-off flags: done[stream] = value
+  int* hq_flag[kHandQ];       // hand-off flags: *flag = value
   int hq_value[kHandQ];
   int hq_head;                // entries pushed by the consumer
   int hq_tail;                // entries published by the producer
@@ -467,18 +471,30 @@ struct Consumer {
     __syncwarp();
   }
 
-  // wait until the previous chunk of the stream has handed its state on
-  __device__ bool wait_predecessor(const Job& jb) {
+  // wait until *flag >= target (the previous chunk of a stream, or a whole
+  // aggregate stream, has handed its state on)
+  // The limit counts time without progress of the whole grid: a wait for an
+  // aggregate stream can legitimately last as long as the aggregate jobs
+  // ahead of it, so the deadline restarts whenever the job ticket moves.
+  __device__ bool wait_flag(const int* flag, int target) {
     bool aborted = false;
     if (lane == 0) {
-      const uint64_t t_start = globaltimer_ns();
+      uint64_t t_start = globaltimer_ns();
+      int ticket = ld_volatile(&p.counters[0]);
       uint32_t spins = 0;
-      while (ld_acquire(&p.done[jb.stream]) < jb.chunk) {
+      while (ld_acquire(flag) < target) {
         if (ld_volatile(&p.counters[1]) != 0) { aborted = true; break; }
-        if ((++spins & 31u) == 0 && globaltimer_ns() - t_start > p.wait_limit_ns) {
-          abort_scan(p);
-          aborted = true;
-          break;
+        if ((++spins & 31u) == 0) {
+          const uint64_t now = globaltimer_ns();
+          const int t = ld_volatile(&p.counters[0]);
+          if (t != ticket) {
+            ticket = t;
+            t_start = now;
+          } else if (now - t_start > p.wait_limit_ns) {
+            abort_scan(p);
+            aborted = true;
+            break;
+          }
         }
         __nanosleep(spins < 64 ? 32 : 256);
       }
@@ -491,18 +507,18 @@ struct Consumer {
   }
 
   // Lane 0, after a __syncwarp that follows every lane's state stores:
-  // done[stream] = value.  The producer warp publishes it (its gpu-scope
-  // release covers the stores, which it observed through this cta-scope
-  // release), so the consumer does not wait for the fence; if the queue is
-  // full the consumer publishes it itself.
-  __device__ void publish(int stream, int value) {
+  // *flag = value.  The producer warp publishes it (its gpu-scope release
+  // covers the stores, which it observed through this cta-scope release), so
+  // the consumer does not wait for the fence; if the queue is full the
+  // consumer publishes it itself.
+  __device__ void publish(int* flag, int value) {
     if (hq_head - ld_relaxed_cta_smem(&sm.hq_tail) < kHandQ) {
-      sm.hq_stream[hq_head % kHandQ] = stream;
+      sm.hq_flag[hq_head % kHandQ] = flag;
       sm.hq_value[hq_head % kHandQ] = value;
       ++hq_head;
       st_release_cta_smem(&sm.hq_head, hq_head);
     } else {
-      st_release(&p.done[stream], value);
+      st_release(flag, value);
     }
   }
 };
@@ -531,6 +547,7 @@ __device__ void producer_loop(const ScanParams& p, WarpSmem<TIO, NS, TILE, STAGE
   bool stop = false;                          // some warp gave up: hand out no more jobs
   uint32_t idle = 0;
   uint64_t idle_since = 0;
+  int seen_ticket = -1;
   for (;;) {
     bool progress = false, all_done = true;
 #pragma unroll
@@ -543,7 +560,7 @@ __device__ void producer_loop(const ScanParams& p, WarpSmem<TIO, NS, TILE, STAGE
       if (f[w].hq_tail != head) {
         for (; f[w].hq_tail != head; ++f[w].hq_tail) {
           const int e = f[w].hq_tail % kHandQ;
-          st_release(&p.done[sm.hq_stream[e]], sm.hq_value[e]);
+          st_release(sm.hq_flag[e], sm.hq_value[e]);
         }
         st_relaxed_cta_smem(&sm.hq_tail, f[w].hq_tail);
         progress = true;
@@ -599,11 +616,21 @@ __device__ void producer_loop(const ScanParams& p, WarpSmem<TIO, NS, TILE, STAGE
       idle = 0;
       continue;
     }
-    // nothing to do: back off (the consumers run on the same sub-partitions)
+    // nothing to do: back off (the consumers run on the same sub-partitions).
+    // Idle time counts only while the whole grid makes no progress (the job
+    // ticket does not move): this CTA's consumers may legitimately wait for
+    // other CTAs' aggregate jobs for a long time.
     const uint64_t now = globaltimer_ns();
     if (idle == 0) idle_since = now;
     ++idle;
-    if (!stop && (idle & 15u) == 0 && ld_volatile(&p.counters[1]) != 0) stop = true;
+    if ((idle & 15u) == 0) {
+      if (!stop && ld_volatile(&p.counters[1]) != 0) stop = true;
+      const int t = ld_volatile(&p.counters[0]);
+      if (t != seen_ticket) {
+        seen_ticket = t;
+        idle_since = now;
+      }
+    }
     if (now - idle_since > 2 * p.wait_limit_ns) {  // the consumers' own limits expire first
       abort_scan(p);
       break;
@@ -643,33 +670,52 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, con
   const float Dd = FULL ? cm.z : 0.0f;
   const float* Arow = p.A + (int64_t)(active ? d : 0) * NS;
 
-  if (!jb.first && !cx.wait_predecessor(jb)) return false;
+  // the stream's slot pair in the hand-off ring and its progress flag
+  // (aggregate streams come after the main streams in the ring)
+  const int64_t ring_stream = FULL ? jb.stream : (int64_t)p.streams_full + jb.stream;
+  int* flag = (FULL ? p.done : p.done_agg) + jb.stream;
+  if (!jb.first && !cx.wait_flag(flag, jb.chunk)) return false;
 
   // starting state, kept scaled: g_n = A_n h_n
   float2 g[NS / 2];
   float sd = 0.0f;
   {
-    const float* src = nullptr;
+    float an[NS];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) {
+      if constexpr (STRUCT) an[k] = (float)(k + 1) * a0;
+      else an[k] = active ? __ldg(Arow + k) : -1.0f;
+    }
+    float h[NS];
+#pragma unroll
+    for (int k = 0; k < NS; ++k) h[k] = 0.0f;
     if (!jb.first) {
-      const int64_t slot_i = (int64_t)jb.stream * 2 + ((jb.chunk - 1) & 1);
-      src = p.ring + slot_i * (kCPW * NS) + c * NS;
+      const int64_t slot_i = ring_stream * 2 + ((jb.chunk - 1) & 1);
+      const float* src = p.ring + slot_i * (kCPW * NS) + c * NS;
+#pragma unroll
+      for (int k = 0; k < NS; ++k) h[k] = __ldcg(src + k);
       if (!FULL) sd = __ldcg(p.ring_sd + slot_i * kCPW + c);
     } else if (FULL) {
-      if (jb.super_idx > 0) src = p.hin + ((int64_t)jb.stream * kCPW + c) * NS;
-      else if (p.h0 && active) src = p.h0 + ((int64_t)jb.b * p.channels + d) * NS;
+      // first chunk of a super-chunk: the initial state, carried over the
+      // super-chunks before this one with their aggregates (the monoid
+      // h <- exp(A sum Delta_j) h + H_j of the page's parallel prefix scan)
+      if (p.h0 && active) {
+        const float* src = p.h0 + ((int64_t)jb.b * p.channels + d) * NS;
+#pragma unroll
+        for (int k = 0; k < NS; ++k) h[k] = __ldcg(src + k);
+      }
+      const int grp = jb.stream - jb.super_idx * p.groups;
+      for (int j = 0; j < jb.super_idx; ++j) {
+        const int sa = j * p.groups + grp;  // aggregate stream of super-chunk j
+        if (!cx.wait_flag(p.done_agg + sa, p.chunks_full)) return false;
+        const float sdj = __ldcg(p.agg_sd + (int64_t)sa * kCPW + c);
+        const float* H = p.agg_h + ((int64_t)sa * kCPW + c) * NS;
+#pragma unroll
+        for (int k = 0; k < NS; ++k) h[k] = fmaf(expf(an[k] * sdj), h[k], __ldcg(H + k));
+      }
     }
 #pragma unroll
-    for (int k = 0; k < NS / 2; ++k) {
-      float ak0, ak1;
-      if constexpr (STRUCT) {
-        ak0 = (float)(2 * k + 1) * a0;
-        ak1 = (float)(2 * k + 2) * a0;
-      } else {
-        ak0 = active ? __ldg(Arow + 2 * k) : -1.0f;
-        ak1 = active ? __ldg(Arow + 2 * k + 1) : -1.0f;
-      }
-      g[k] = src ? f2(__ldcg(src + 2 * k) * ak0, __ldcg(src + 2 * k + 1) * ak1) : f2(0.0f, 0.0f);
-    }
+    for (int k = 0; k < NS / 2; ++k) g[k] = f2(h[2 * k] * an[2 * k], h[2 * k + 1] * an[2 * k + 1]);
   }
   float kA[STRUCT ? 1 : NS], kC[STRUCT ? 1 : NS];
   if constexpr (!STRUCT) {
@@ -716,7 +762,7 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, con
   float* dst;
   float* dst_sd = nullptr;
   if (!jb.last) {
-    const int64_t slot_i = (int64_t)jb.stream * 2 + (jb.chunk & 1);
+    const int64_t slot_i = ring_stream * 2 + (jb.chunk & 1);
     dst = p.ring + slot_i * (kCPW * NS) + c * NS;
     if (!FULL) dst_sd = p.ring_sd + slot_i * kCPW + c;
   } else if (FULL) {
@@ -737,11 +783,12 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, con
     }
   }
   if (dst_sd) *dst_sd = sd;
-  if (!jb.last) {
+  if (!jb.last || !FULL) {
     // the warp barrier orders every lane's state stores before lane 0's
-    // hand-off, which releases them with the flag
+    // hand-off, which releases them with the flag (an aggregate stream's
+    // last chunk publishes its aggregate the same way)
     __syncwarp();
-    if (c == 0) cx.publish(jb.stream, jb.chunk + 1);
+    if (c == 0) cx.publish(flag, jb.chunk + 1);
   }
   __syncwarp();
   return true;
@@ -800,7 +847,6 @@ scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__
   }
 
   Consumer<TIO, NS, TILE, STAGES> cx(p, sms[warp], lane);
-  const bool full_mode = (p.mode == kModeFull);
   for (;;) {
     const int s0 = cx.wait_tile();
     if (s0 < 0) break;
@@ -810,6 +856,7 @@ scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__
     const float4 cm = p.use_tma ? cx.sm.chan[s0][lane] : __ldg(p.chan + jb.d0 + lane);
     // structured A on every channel of the warp (decided per channel by the pre-pass)
     const bool structured = __all_sync(0xffffffffu, cm.w != 0.0f);
+    const bool full_mode = !jb.agg;
     bool ok;
     if constexpr (METHOD != kZOH)  // other discretisations: the general-A path
       ok = full_mode ? run_job<TIO, NS, TILE, STAGES, false, true, METHOD>(cx, jb, s0, cm)
@@ -864,35 +911,6 @@ __global__ void scan_prep_kernel(int* __restrict__ zero, int64_t zero_words, con
 #pragma unroll
   for (int n = 1; n < NS; ++n) structured &= (row[n] == (float)(n + 1) * a0);
   chan[d] = make_float4(a0, 1.0f / a0, D ? D[d] : 0.0f, structured ? 1.0f : 0.0f);
-}
-
-// ---------------------------------------------------------------------------
-// combine pass: starting state of every super-chunk from the aggregates,
-//   h_{j+1} = exp(A * sumDelta_j) h_j + H_j,   h_0 = initial state or 0
-// one thread per (group, lane, state).
-// ---------------------------------------------------------------------------
-template <int NS>
-__global__ void scan_combine_kernel(const ScanParams p, float* hin) {
-  griddep_launch_dependents();
-  const int64_t tid = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-  griddep_wait();
-  const int64_t total = (int64_t)p.groups * kCPW * NS;
-  if (tid >= total) return;
-  const int n = (int)(tid % NS);
-  const int c = (int)((tid / NS) % kCPW);
-  const int grp = (int)(tid / ((int64_t)NS * kCPW));
-  const int b = grp / p.groups_d;
-  const int d = (grp - b * p.groups_d) * kCPW + c;
-  const bool active = d < p.channels;
-  const float a = active ? p.A[(int64_t)d * NS + n] : -1.0f;
-  float h = (active && p.h0) ? p.h0[((int64_t)b * p.channels + d) * NS + n] : 0.0f;
-  for (int j = 0; j + 1 < p.supers; ++j) {
-    const int64_t s = (int64_t)j * p.groups + grp;
-    const float sdj = p.agg_sd[s * kCPW + c];
-    const float H = p.agg_h[(s * kCPW + c) * NS + n];
-    h = fmaf(expf(a * sdj), h, H);
-    hin[(((int64_t)(j + 1) * p.groups + grp) * kCPW + c) * NS + n] = h;
-  }
 }
 
 }  // namespace mamba
