@@ -109,7 +109,8 @@ struct Plan {
 // How a scan is laid out and split.  Every consumer warp needs a stream of
 // its own (a 32-channel group over a stretch of time); when the groups are
 // fewer than the resident consumer warps, sequences are cut into
-// super-chunks joined by the associative combine.  Within a stream the
+// super-chunks joined by the associative combine (about twice as many
+// streams as warps).  Within a stream the
 // sequence is cut into chunks so that there are about kJobsPerWarp jobs per
 // warp for dynamic balance, each at least two tiles long.  A positive
 // `user_chunk` forces super-chunks of that length.
@@ -123,7 +124,10 @@ Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, 
     pl.super_len = std::min<int64_t>(user_chunk, len);
   } else {
     int64_t s = 1;
-    if (groups < pl.warps_total) s = (pl.warps_total + groups - 1) / groups;
+    // twice as many streams as warps: a super-chunk's aggregate and main
+    // jobs form a sequential path of about 1.6 super-chunk lengths, which
+    // then stays well below each warp's share of the work
+    if (groups < pl.warps_total) s = (2 * (int64_t)pl.warps_total + groups - 1) / groups;
     s = std::min<int64_t>(s, std::max<int64_t>(1, len / (4 * tile)));
     pl.super_len = (len + s - 1) / s;
     pl.super_len = ((pl.super_len + tile - 1) / tile) * tile;
