@@ -194,6 +194,37 @@ int mamba_selective_scan_noalloc(const void *u, const void *delta, const float *
                                  int64_t batch, int64_t len, int64_t channels, int64_t nstate,
                                  int dtype, mamba_stream_t stream);
 
+/*
+ * mamba_selective_scan on HOST buffers, with the copies overlapped with the
+ * scan.  The pages have no counterpart of this call; it serves callers whose
+ * sequences live in host memory (prefill from host-resident activations,
+ * offline batch scoring).
+ *
+ *   u, delta, B, C, y, A, D, final_state   host memory, same layouts and
+ *                types as mamba_selective_scan (final_state and D may be NULL)
+ *   piece_len    > 0: tokens per piece; 0: about len / 8 (at least 256)
+ *
+ * The sequence is cut into time pieces.  Piece k's host->device copies
+ * (cudaMemcpy2DAsync of rows [t0, t0+n) of every batch), its scan and the
+ * device->host copy of its y run on one of two streams (`stream` and an
+ * internal non-blocking stream, created once per device), so copies overlap
+ * the neighbouring pieces' scans; piece k starts from piece k-1's final state
+ * (ordered by an event), which is the same recurrence as one scan.
+ *
+ * Host buffers should be page-locked (cudaHostAlloc / cudaHostRegister): with
+ * pageable memory the copies do not overlap.  The call is asynchronous on
+ * `stream` (which waits for the internal stream at the end): the host
+ * buffers must stay valid, and y / final_state may be read only after
+ * `stream` has been synchronised.  Device memory (two pieces' buffers, A, D)
+ * is allocated and freed stream-ordered on `stream`.  len == 0 writes zeros
+ * to final_state on the host before returning.
+ */
+int mamba_selective_scan_host(const void *u, const void *delta, const float *A,
+                              const void *B, const void *C, const float *D,
+                              void *y, float *final_state,
+                              int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                              int64_t piece_len, int dtype, mamba_stream_t stream);
+
 /* How mamba_selective_scan_ex would split a problem (host-side planning only). */
 typedef struct {
     int64_t supers;        /* independent super-chunks per sequence (1: no aggregate jobs) */

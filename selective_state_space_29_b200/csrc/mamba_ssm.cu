@@ -367,6 +367,113 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   return status;
 }
 
+// ---------------------------------------------------------------------------
+// Host-resident data: the sequence is cut into time pieces; piece k's
+// host->device copies, scan and device->host copy of y run on stream k % 2,
+// so one piece's copies overlap the neighbouring pieces' scans (the two copy
+// directions use separate copy engines).  Piece k resumes from piece k-1's
+// final state (an event orders the two streams), which is the same
+// recurrence as one scan over the whole sequence.
+// ---------------------------------------------------------------------------
+std::mutex g_aux_mu;
+cudaStream_t g_aux_stream[64] = {};
+
+int aux_stream(cudaStream_t* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MAMBA_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_aux_mu);
+  if (!g_aux_stream[dev] && cudaStreamCreateWithFlags(&g_aux_stream[dev], cudaStreamNonBlocking) != cudaSuccess)
+    return MAMBA_ERR_CUDA;
+  *out = g_aux_stream[dev];
+  return MAMBA_OK;
+}
+
+// Rows [t0, t0 + n) of every batch of a host array [batch][len][width]
+// to/from a packed device array [batch][n][width].
+cudaError_t copy_piece(void* dst, const void* src, bool to_device, int64_t batch, int64_t len, int64_t t0, int64_t n,
+                       size_t row_bytes, cudaStream_t st) {
+  const size_t piece_pitch = (size_t)n * row_bytes, full_pitch = (size_t)len * row_bytes;
+  if (to_device)
+    return cudaMemcpy2DAsync(dst, piece_pitch, static_cast<const char*>(src) + (size_t)t0 * row_bytes, full_pitch,
+                             piece_pitch, (size_t)batch, cudaMemcpyHostToDevice, st);
+  return cudaMemcpy2DAsync(static_cast<char*>(dst) + (size_t)t0 * row_bytes, full_pitch, src, piece_pitch,
+                           piece_pitch, (size_t)batch, cudaMemcpyDeviceToHost, st);
+}
+
+int scan_host_pipelined(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                        const float* D, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
+                        int64_t nstate, int64_t piece_len, int dtype, cudaStream_t s0) {
+  cudaStream_t s1 = nullptr;
+  if (int st = aux_stream(&s1)) return st;
+  const size_t es = (size_t)elem_size(dtype);
+  int64_t P = piece_len > 0 ? piece_len : std::max<int64_t>(256, ((len + 7) / 8 + 63) / 64 * 64);
+  P = std::min<int64_t>(P, len);
+  const int64_t pieces = (len + P - 1) / P;
+  const size_t xb = (size_t)batch * (size_t)P * (size_t)channels * es;  // u, delta or y of one piece
+  const size_t bb = (size_t)batch * (size_t)P * (size_t)nstate * es;    // B or C of one piece
+  const size_t hb = sizeof(float) * (size_t)batch * (size_t)channels * (size_t)nstate;
+  const size_t ab = sizeof(float) * (size_t)channels * (size_t)(nstate + 1);
+  auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+  const size_t per_set = 3 * al(xb) + 2 * al(bb) + al(hb);
+  const size_t total = 2 * per_set + al(ab);
+  cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};  // s0 ready for s1, state ready on s0 / s1
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return MAMBA_ERR_CUDA;
+  int status = MAMBA_OK;
+  auto fail = [&](cudaError_t e) {
+    if (e != cudaSuccess && status == MAMBA_OK) status = MAMBA_ERR_CUDA;
+    return status != MAMBA_OK;
+  };
+  unsigned char* mem = nullptr;
+  if (!fail(cudaMallocAsync(reinterpret_cast<void**>(&mem), total, s0))) {
+    float* dA = reinterpret_cast<float*>(mem + 2 * per_set);
+    float* dD = D ? dA + (size_t)channels * nstate : nullptr;
+    fail(cudaMemcpyAsync(dA, A, sizeof(float) * (size_t)channels * nstate, cudaMemcpyHostToDevice, s0));
+    if (D) fail(cudaMemcpyAsync(dD, D, sizeof(float) * (size_t)channels, cudaMemcpyHostToDevice, s0));
+    // s1 starts after everything enqueued on s0 so far (the caller's work, the allocation, A and D)
+    fail(cudaEventRecord(ev[0], s0));
+    fail(cudaStreamWaitEvent(s1, ev[0], 0));
+    float* state_prev = nullptr;
+    for (int64_t k = 0; k < pieces && status == MAMBA_OK; ++k) {
+      cudaStream_t st = (k & 1) ? s1 : s0;
+      unsigned char* set = mem + (size_t)(k & 1) * per_set;
+      void* du = set;
+      void* ddl = set + al(xb);
+      void* dy = set + 2 * al(xb);
+      void* dB = set + 3 * al(xb);
+      void* dC = set + 3 * al(xb) + al(bb);
+      float* dh = reinterpret_cast<float*>(set + 3 * al(xb) + 2 * al(bb));
+      const int64_t t0 = k * P, n = std::min<int64_t>(P, len - t0);
+      fail(copy_piece(du, u, true, batch, len, t0, n, (size_t)channels * es, st));
+      fail(copy_piece(ddl, delta, true, batch, len, t0, n, (size_t)channels * es, st));
+      fail(copy_piece(dB, B, true, batch, len, t0, n, (size_t)nstate * es, st));
+      fail(copy_piece(dC, C, true, batch, len, t0, n, (size_t)nstate * es, st));
+      if (k > 0) fail(cudaStreamWaitEvent(st, ev[1 + ((k - 1) & 1)], 0));  // piece k-1's final state
+      if (status != MAMBA_OK) break;
+      const int sc = dtype == MAMBA_BF16
+                         ? launch_scan<__nv_bfloat16, 16>(du, ddl, dA, dB, dC, dD, state_prev, dy, dh, batch, n,
+                                                          channels, 0, 0u, dtype, st, false)
+                         : launch_scan<float, 16>(du, ddl, dA, dB, dC, dD, state_prev, dy, dh, batch, n, channels, 0,
+                                                  0u, dtype, st, false);
+      if (sc != MAMBA_OK) {
+        status = sc;
+        break;
+      }
+      fail(cudaEventRecord(ev[1 + (k & 1)], st));
+      fail(copy_piece(y, dy, false, batch, len, t0, n, (size_t)channels * es, st));
+      state_prev = dh;
+      if (k == pieces - 1 && final_state)
+        fail(cudaMemcpyAsync(final_state, dh, hb, cudaMemcpyDeviceToHost, st));
+    }
+    // join: s0 continues after everything on s1, then the memory goes back
+    fail(cudaEventRecord(ev[0], s1));
+    fail(cudaStreamWaitEvent(s0, ev[0], 0));
+    fail(cudaFreeAsync(mem, s0));
+  }
+  for (auto& e : ev) cudaEventDestroy(e);
+  return status;
+}
+
 __global__ void expire_wait_kernel(uint64_t limit_ns) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
@@ -462,6 +569,29 @@ int mamba_selective_scan(const void* u, const void* delta, const float* A, const
                          int64_t nstate, int dtype, mamba_stream_t stream) {
   return mamba_selective_scan_ex(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, nstate, 0, 0u,
                                  dtype, stream);
+}
+
+int mamba_selective_scan_host(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                              const float* D, void* y, float* final_state, int64_t batch, int64_t len,
+                              int64_t channels, int64_t nstate, int64_t piece_len, int dtype,
+                              mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || len < 0 || channels < 0 || nstate <= 0 || piece_len < 0) return MAMBA_ERR_INVALID_ARG;
+  if (!mamba_scan_supported_nstate(nstate)) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || channels == 0) return MAMBA_OK;
+  if (!A) return MAMBA_ERR_INVALID_ARG;
+  if (len > 0 && (!u || !delta || !B || !C || !y)) return MAMBA_ERR_INVALID_ARG;
+  if (batch * len >= (int64_t(1) << 31) || channels >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+  cudaGetLastError();
+  if (len == 0) {
+    if (!final_state) return MAMBA_OK;
+    const size_t hb = sizeof(float) * (size_t)batch * (size_t)channels * (size_t)nstate;
+    std::memset(final_state, 0, hb);  // h_0 = 0 and no token: the final state is zero
+    return MAMBA_OK;
+  }
+  return scan_host_pipelined(u, delta, A, B, C, D, y, final_state, batch, len, channels, nstate, piece_len, dtype,
+                             stream);
 }
 
 int mamba_selective_scan_noalloc(const void* u, const void* delta, const float* A, const void* B, const void* C,

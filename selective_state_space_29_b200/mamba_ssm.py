@@ -46,6 +46,8 @@ _SIGNATURES = [
      [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_uint, ctypes.c_int, _P]),
     ("mamba_selective_scan_noalloc", ctypes.c_int,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int, _P]),
+    ("mamba_selective_scan_host", ctypes.c_int,
+     [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_state_update", ctypes.c_int,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_scan_plan", ctypes.c_int,
@@ -146,6 +148,16 @@ def mamba_selective_scan_noalloc(u, delta, A, B, C, D, y, final_state, batch, le
     _check(st, "mamba_selective_scan_noalloc")
 
 
+def mamba_selective_scan_host(u, delta, A, B, C, D, y, final_state, batch, len, channels, nstate, piece_len,
+                              dtype, stream=None):
+    """The scan on host buffers (page-locked for overlap), copies pipelined
+    with the scan piece by piece; asynchronous on `stream`."""
+    st = library().mamba_selective_scan_host(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(y),
+                                             _ptr(final_state), batch, len, channels, nstate, piece_len, dtype,
+                                             _stream(stream))
+    _check(st, "mamba_selective_scan_host")
+
+
 def mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, dtype, stream=None):
     st = library().mamba_state_update(_ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
                                       _ptr(y), batch, channels, nstate, dtype, _stream(stream))
@@ -217,3 +229,25 @@ def state_update(state, x, delta, A, B, C, D=None, y=None, stream=None):
         y = torch.empty_like(x)
     mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, dtype_code(x.dtype), stream)
     return y
+
+
+def selective_scan_host(u, delta, A, B, C, D=None, y=None, final_state=None, piece_len=0, stream=None,
+                        synchronize=True):
+    """y, final_state = the scan of host tensors (CPU, ideally pinned), with
+    the host<->device copies overlapped with the scan; outputs are host
+    tensors (allocated pinned when not given)."""
+    import torch
+    batch, length, channels = u.shape
+    nstate = A.shape[1]
+    for t in (u, delta, A, B, C, D):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError("host tensors must be contiguous CPU tensors")
+    if y is None:
+        y = torch.empty(u.shape, dtype=u.dtype, pin_memory=True)
+    if final_state is None:
+        final_state = torch.empty((batch, channels, nstate), dtype=torch.float32, pin_memory=True)
+    mamba_selective_scan_host(u, delta, A, B, C, D, y, final_state, batch, length, channels, nstate, piece_len,
+                              dtype_code(u.dtype), stream)
+    if synchronize:
+        torch.cuda.synchronize()
+    return y, final_state

@@ -111,6 +111,23 @@ def test_state_update_argument_errors_on_host(lib):
     assert call(batch=0) == m.MAMBA_OK
 
 
+def test_host_scan_argument_errors(lib):
+    # rejected on the host before any CUDA call
+    f = lib.mamba_selective_scan_host
+    args = [1024, 1024, 1024, 1024, 1024, None, 2048, None, 1, 4, 8, 16, 0, m.MAMBA_BF16, None]
+    def call(i, v):
+        a = list(args)
+        a[i] = v
+        return f(*a)
+    assert call(13, 5) == m.MAMBA_ERR_INVALID_ARG       # dtype
+    assert call(8, -1) == m.MAMBA_ERR_INVALID_ARG       # batch
+    assert call(12, -1) == m.MAMBA_ERR_INVALID_ARG      # piece_len
+    assert call(11, 12) == m.MAMBA_ERR_UNSUPPORTED      # nstate
+    assert call(2, None) == m.MAMBA_ERR_INVALID_ARG     # A
+    assert call(0, None) == m.MAMBA_ERR_INVALID_ARG     # u
+    assert call(8, 0) == m.MAMBA_OK                     # empty
+
+
 def test_library_links_no_torch(lib):
     # the product library is plain C ABI over CUDA: no torch / python symbols needed
     out = os.popen(f"nm -D --undefined-only {lib_build.LIB}").read()
