@@ -102,8 +102,9 @@ typedef enum {
  *   y            device, dtype, [batch][len][channels]       (output)
  *   final_state  device, float32, [batch][channels][nstate], or NULL; receives
  *                h after the last token (zeros when len == 0)
- *   nstate       number of states per channel; 16 in this build
- *                (mamba_scan_supported_nstate tells)
+ *   nstate       number of states per channel: 4, 8, 16 or 32 in this build
+ *                (mamba_scan_supported_nstate tells); bf16 with 4 states
+ *                loads its tiles without TMA (a B row is 8 bytes)
  *   stream       CUDA stream the work is ordered on
  *
  * Alignment: every pointer must be aligned to its element size; tiles are

@@ -9,6 +9,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "mamba_ssm.h"
 #include "common.cuh"
@@ -80,18 +81,15 @@ bool make_map_2d(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// --- scan configuration per element type -----------------------------------
+// --- scan configuration per element type and state count -------------------
 // A CTA is kScanConsumers consumer warps (one per SM sub-partition) and one
-// producer warp; a consumer's ring holds kStages tiles of kTile tokens.
-template <typename TIO>
-struct ScanCfg;
-template <>
-struct ScanCfg<__nv_bfloat16> {
-  static constexpr int kTile = 64, kStages = 3;
-};
-template <>
-struct ScanCfg<float> {
-  static constexpr int kTile = 32, kStages = 3;
+// producer warp; a consumer's ring holds kStages tiles of kTile tokens (the
+// ring of four consumers fits the 227 KB of shared memory of a CTA).
+template <typename TIO, int NS>
+struct ScanCfg {
+  static constexpr bool kBf16 = sizeof(TIO) == 2;
+  static constexpr int kTile = kBf16 ? 64 : 32;
+  static constexpr int kStages = (kBf16 && NS >= 32) ? 2 : 3;
 };
 constexpr int kScanConsumers = 4;
 constexpr int kJobsPerWarp = 8;  // chunks per consumer warp, for dynamic balance
@@ -174,7 +172,19 @@ int64_t full_jobs(const Plan& pl) {
   return (int64_t)pl.chunks_last * streams_full + (int64_t)(pl.chunks_full - pl.chunks_last) * streams_agg;
 }
 
-int tile_for(int dtype) { return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16>::kTile : ScanCfg<float>::kTile; }
+int tile_for(int dtype) { return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16, 16>::kTile : ScanCfg<float, 16>::kTile; }
+
+// state counts the kernels are built for
+template <typename F>
+int dispatch_nstate(int64_t nstate, F&& f) {
+  switch (nstate) {
+    case 4: return f(std::integral_constant<int, 4>{});
+    case 8: return f(std::integral_constant<int, 8>{});
+    case 16: return f(std::integral_constant<int, 16>{});
+    case 32: return f(std::integral_constant<int, 32>{});
+    default: return MAMBA_ERR_UNSUPPORTED;
+  }
+}
 
 int64_t kernels_per_call(const Plan&) { return 2; }  // pre-pass, chunked scan
 
@@ -239,8 +249,8 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
                    const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
                    unsigned flags, int dtype, cudaStream_t stream, const Plan& pl, int sms,
                    unsigned char* scratch) {
-  constexpr int TILE = ScanCfg<TIO>::kTile;
-  constexpr int STAGES = ScanCfg<TIO>::kStages;
+  constexpr int TILE = ScanCfg<TIO, NS>::kTile;
+  constexpr int STAGES = ScanCfg<TIO, NS>::kStages;
   const ScratchLayout sl = scratch_layout(pl, NS, batch, len);
   unsigned char* cur = scratch;
   int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
@@ -341,7 +351,7 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
                 int64_t user_chunk, unsigned flags, int dtype, cudaStream_t stream, bool noalloc) {
   int sms = 0;
   if (int st = current_sms(&sms)) return st;
-  const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO>::kTile, user_chunk);
+  const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO, NS>::kTile, user_chunk);
   if (pl.groups > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
   const ScratchLayout sl = scratch_layout(pl, NS, batch, len);
   unsigned char* scratch = nullptr;
@@ -450,11 +460,13 @@ int scan_host_pipelined(const void* u, const void* delta, const float* A, const 
       fail(copy_piece(dC, C, true, batch, len, t0, n, (size_t)nstate * es, st));
       if (k > 0) fail(cudaStreamWaitEvent(st, ev[1 + ((k - 1) & 1)], 0));  // piece k-1's final state
       if (status != MAMBA_OK) break;
-      const int sc = dtype == MAMBA_BF16
-                         ? launch_scan<__nv_bfloat16, 16>(du, ddl, dA, dB, dC, dD, state_prev, dy, dh, batch, n,
-                                                          channels, 0, 0u, dtype, st, false)
-                         : launch_scan<float, 16>(du, ddl, dA, dB, dC, dD, state_prev, dy, dh, batch, n, channels, 0,
-                                                  0u, dtype, st, false);
+      const int sc = dispatch_nstate(nstate, [&](auto ns) {
+        constexpr int NS = decltype(ns)::value;
+        return dtype == MAMBA_BF16 ? launch_scan<__nv_bfloat16, NS>(du, ddl, dA, dB, dC, dD, state_prev, dy, dh, batch,
+                                                                    n, channels, 0, 0u, dtype, st, false)
+                                   : launch_scan<float, NS>(du, ddl, dA, dB, dC, dD, state_prev, dy, dh, batch, n,
+                                                            channels, 0, 0u, dtype, st, false);
+      });
       if (sc != MAMBA_OK) {
         status = sc;
         break;
@@ -502,7 +514,9 @@ const char* mamba_status_string(int status) {
   }
 }
 
-int mamba_scan_supported_nstate(int64_t nstate) { return nstate == 16 ? 1 : 0; }
+int mamba_scan_supported_nstate(int64_t nstate) {
+  return (nstate == 4 || nstate == 8 || nstate == 16 || nstate == 32) ? 1 : 0;
+}
 
 int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate, int64_t chunk_len, int dtype,
                     int sm_count, mamba_scan_plan_t* out) {
@@ -557,11 +571,14 @@ int mamba_selective_scan_ex(const void* u, const void* delta, const float* A, co
                         : cudaMemsetAsync(final_state, 0, state_bytes, stream);
     return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
   }
-  if (dtype == MAMBA_BF16)
-    return launch_scan<__nv_bfloat16, 16>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels,
-                                          chunk_len, flags, dtype, stream, false);
-  return launch_scan<float, 16>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels, chunk_len,
-                                flags, dtype, stream, false);
+  return dispatch_nstate(nstate, [&](auto ns) {
+    constexpr int NS = decltype(ns)::value;
+    if (dtype == MAMBA_BF16)
+      return launch_scan<__nv_bfloat16, NS>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels,
+                                            chunk_len, flags, dtype, stream, false);
+    return launch_scan<float, NS>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels,
+                                  chunk_len, flags, dtype, stream, false);
+  });
 }
 
 int mamba_selective_scan(const void* u, const void* delta, const float* A, const void* B, const void* C,
@@ -617,11 +634,14 @@ int mamba_selective_scan_noalloc(const void* u, const void* delta, const float* 
     const size_t state_bytes = sizeof(float) * (size_t)batch * (size_t)channels * (size_t)nstate;
     return cudaMemsetAsync(final_state, 0, state_bytes, stream) == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
   }
-  if (dtype == MAMBA_BF16)
-    return launch_scan<__nv_bfloat16, 16>(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, 0, 0u,
-                                          dtype, stream, true);
-  return launch_scan<float, 16>(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, 0, 0u, dtype,
-                                stream, true);
+  return dispatch_nstate(nstate, [&](auto ns) {
+    constexpr int NS = decltype(ns)::value;
+    if (dtype == MAMBA_BF16)
+      return launch_scan<__nv_bfloat16, NS>(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, 0,
+                                            0u, dtype, stream, true);
+    return launch_scan<float, NS>(u, delta, A, B, C, D, nullptr, y, final_state, batch, len, channels, 0, 0u, dtype,
+                                  stream, true);
+  });
 }
 
 int mamba_state_update(float* state, const void* x, const void* delta, const float* A, const void* B, const void* C,
@@ -638,28 +658,32 @@ int mamba_state_update(float* state, const void* x, const void* delta, const flo
       !aligned(y, es) || !aligned(B, 4 * es) || !aligned(C, 4 * es))
     return MAMBA_ERR_INVALID_ARG;
   cudaGetLastError();
-  constexpr int kRows = 4;                                     // batch rows per thread
-  constexpr int kChanPerCta = kDecodeWarps * (32 / (16 / 4));  // 64 channels per CTA at 16 states
-  const int64_t gx = (channels + kChanPerCta - 1) / kChanPerCta;
-  const int64_t gy = (batch + kRows - 1) / kRows;
-  if (gy > 65535 || gx > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
-  const dim3 grid((unsigned)gx, (unsigned)gy);
+  constexpr int kRows = 4;  // batch rows per thread
   // programmatic launch: a step's setup overlaps the end of the previous
   // kernel of the stream (the kernel waits for it before touching memory)
-  cudaError_t err;
-  if (dtype == MAMBA_BF16) {
-    DecodeArgs<__nv_bfloat16, 16> a{state, static_cast<const __nv_bfloat16*>(x),
-                                    static_cast<const __nv_bfloat16*>(delta), A,
-                                    static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
-                                    static_cast<__nv_bfloat16*>(y), batch, channels};
-    err = launch_pdl(state_update_kernel<__nv_bfloat16, 16, kRows, true>, grid, dim3(kDecodeWarps * 32), 0, stream, a);
-  } else {
-    DecodeArgs<float, 16> a{state, static_cast<const float*>(x), static_cast<const float*>(delta), A,
-                            static_cast<const float*>(B), static_cast<const float*>(C), D,
-                            static_cast<float*>(y), batch, channels};
-    err = launch_pdl(state_update_kernel<float, 16, kRows, false>, grid, dim3(kDecodeWarps * 32), 0, stream, a);
-  }
-  return err == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+  return dispatch_nstate(nstate, [&](auto ns) {
+    constexpr int NS = decltype(ns)::value;
+    constexpr int kChanPerCta = kDecodeWarps * (32 / (NS / 4));  // NS/4 lanes per (batch, channel) row
+    const int64_t gx = (channels + kChanPerCta - 1) / kChanPerCta;
+    const int64_t gy = (batch + kRows - 1) / kRows;
+    if (gy > 65535 || gx > 0x7fffffff) return (int)MAMBA_ERR_UNSUPPORTED;
+    const dim3 grid((unsigned)gx, (unsigned)gy);
+    cudaError_t err;
+    if (dtype == MAMBA_BF16) {
+      DecodeArgs<__nv_bfloat16, NS> a{state, static_cast<const __nv_bfloat16*>(x),
+                                      static_cast<const __nv_bfloat16*>(delta), A,
+                                      static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
+                                      static_cast<__nv_bfloat16*>(y), batch, channels};
+      err = launch_pdl(state_update_kernel<__nv_bfloat16, NS, kRows, true>, grid, dim3(kDecodeWarps * 32), 0, stream,
+                       a);
+    } else {
+      DecodeArgs<float, NS> a{state, static_cast<const float*>(x), static_cast<const float*>(delta), A,
+                              static_cast<const float*>(B), static_cast<const float*>(C), D,
+                              static_cast<float*>(y), batch, channels};
+      err = launch_pdl(state_update_kernel<float, NS, kRows, false>, grid, dim3(kDecodeWarps * 32), 0, stream, a);
+    }
+    return err == cudaSuccess ? (int)MAMBA_OK : (int)MAMBA_ERR_CUDA;
+  });
 }
 
 int mamba_get_device_error(int clear) {

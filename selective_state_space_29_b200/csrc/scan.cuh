@@ -261,10 +261,18 @@ __device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const T
   if constexpr (sizeof(TIO) == 2) {
     const uint16_t xh = raw16(xr);
     uint32_t bw[NS / 2];
+    if constexpr (NS % 8 == 0) {
 #pragma unroll
-    for (int k8 = 0; k8 < NS / 8; ++k8) {
-      const uint4 w = reinterpret_cast<const uint4*>(brow)[k8];
-      bw[4 * k8] = w.x; bw[4 * k8 + 1] = w.y; bw[4 * k8 + 2] = w.z; bw[4 * k8 + 3] = w.w;
+      for (int k8 = 0; k8 < NS / 8; ++k8) {
+        const uint4 w = reinterpret_cast<const uint4*>(brow)[k8];
+        bw[4 * k8] = w.x; bw[4 * k8 + 1] = w.y; bw[4 * k8 + 2] = w.z; bw[4 * k8 + 3] = w.w;
+      }
+    } else {
+#pragma unroll
+      for (int k4 = 0; k4 < NS / 4; ++k4) {
+        const uint2 w = reinterpret_cast<const uint2*>(brow)[k4];
+        bw[2 * k4] = w.x; bw[2 * k4 + 1] = w.y;
+      }
     }
 #pragma unroll
     for (int n4 = 0; n4 < NS / 4; ++n4) {

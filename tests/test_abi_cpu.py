@@ -54,9 +54,10 @@ def test_status_strings(lib):
 
 
 def test_supported_nstate(lib):
-    assert m.mamba_scan_supported_nstate(16)
-    assert not m.mamba_scan_supported_nstate(0)
-    assert not m.mamba_scan_supported_nstate(17)
+    for n in (4, 8, 16, 32):
+        assert m.mamba_scan_supported_nstate(n)
+    for n in (0, 1, 2, 12, 17, 64):
+        assert not m.mamba_scan_supported_nstate(n)
 
 
 def _scan_ex(lib, **kw):
@@ -104,7 +105,7 @@ def test_state_update_argument_errors_on_host(lib):
 
     assert call(dtype=3) == m.MAMBA_ERR_INVALID_ARG
     assert call(batch=-2) == m.MAMBA_ERR_INVALID_ARG
-    assert call(nstate=8) == m.MAMBA_ERR_UNSUPPORTED
+    assert call(nstate=12) == m.MAMBA_ERR_UNSUPPORTED
     assert call(state=None) == m.MAMBA_ERR_INVALID_ARG
     assert call(state=4100) == m.MAMBA_ERR_INVALID_ARG                   # state must be 16-byte aligned
     assert call(B=1026) == m.MAMBA_ERR_INVALID_ARG

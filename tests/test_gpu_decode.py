@@ -108,3 +108,12 @@ def test_decode_workload_sampled():
     print(f"decode chain: y err {ey:.2e}, state err {eh:.2e} over {len(rows)} rows")
     assert ey <= TOL["bf16"] and eh <= TOL["bf16"]
     assert torch.isfinite(state).all()
+
+
+@pytest.mark.parametrize("nstate", [4, 8, 32])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_other_state_counts(nstate, dtype):
+    # nstate/4 lanes per (batch, channel) row: 1, 2 and 8 lanes
+    w = wl.DecodeWorkload("n", batch=5, channels=300, nstate=nstate, steps=20, dtype=dtype, a_mode="random")
+    ey, eh, _ = _chain(w)
+    assert ey <= TOL[dtype] and eh <= TOL[dtype], (ey, eh)

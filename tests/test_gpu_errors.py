@@ -19,7 +19,7 @@ def test_argument_errors_raise():
     assert ei.value.status == m.MAMBA_ERR_INVALID_ARG
     with pytest.raises(m.MambaError) as ei:
         m.mamba_selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], None, inp["u"], None,
-                               1, 16, 32, 8, m.MAMBA_BF16)
+                               1, 16, 32, 12, m.MAMBA_BF16)
     assert ei.value.status == m.MAMBA_ERR_UNSUPPORTED
 
 

@@ -208,3 +208,24 @@ def test_scan_methods_flags_rejected_together():
         inp["C"].data_ptr(), inp["D"].data_ptr(), None, y.data_ptr(), None, SMALL.batch, SMALL.length,
         SMALL.channels, 16, 0, m.MAMBA_SCAN_EULER | m.MAMBA_SCAN_TRAPEZOID, m.MAMBA_BF16, None)
     assert st == m.MAMBA_ERR_INVALID_ARG
+
+
+# --- other state counts -------------------------------------------------------------------
+
+@pytest.mark.parametrize("nstate", [4, 8, 32])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("a_mode", ["s4d", "random"])
+def test_scan_other_state_counts(nstate, dtype, a_mode):
+    _check_full(SMALL.with_(nstate=nstate, dtype=dtype, a_mode=a_mode))
+
+
+@pytest.mark.parametrize("nstate", [4, 32])
+def test_scan_other_state_counts_chunked_and_initial_state(nstate):
+    _check_full(SMALL.with_(nstate=nstate, length=700), chunk_len=100, h0_std=0.5)
+    _check_full(SMALL.with_(nstate=nstate, batch=1, length=20000, channels=64, delta_lo=1e-4), D=False)
+
+
+@pytest.mark.parametrize("nstate", [8, 32])
+def test_scan_other_state_counts_methods(nstate):
+    _check_full(SMALL.with_(nstate=nstate, length=500), method="trapezoid", chunk_len=123)
+    _check_full(SMALL.with_(nstate=nstate, length=500, dtype="f32"), method="euler")
