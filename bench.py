@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the timings of the scan's options (general A, other discretisations, state counts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--length-sweep", action="store_true",
                     help="instead of the benchmark line: ns per token-channel of the long-context workload's "
@@ -444,6 +446,11 @@ def run_ours(args):
                                       "call": "copies of whole tensors around mamba_selective_scan"}}
         del host, dbuf
 
+    # the scan's options on the same shape: general-A path, the other
+    # discretisations, other state counts (device-timed calls, events)
+    if not args.no_variants:
+        out["variants"] = run_variants(w, dev, stream, dist, world, rank)
+
     # decode: 1000 single-token steps on 256 x 5120 x 16 states
     if not args.no_decode:
         out["decode"] = run_decode(args, dev, stream, dist, world, rank, hbm_peak, hbm_src)
@@ -525,6 +532,54 @@ def run_decode(args, dev, stream, dist, world, rank, hbm_peak, hbm_src):
                          "algorithmic_bytes_per_launch": nb, "peak_source": hbm_src,
                          "note": "the 84 MB state fits in L2; DRAM traffic per launch is in the ncu summary"},
             "gpu_launches": steps}
+
+
+def run_variants(w, dev, stream, dist, world, rank, reps: int = 20):
+    """ms per call and token·channels/s of the scan's options on the workload's
+    shape: MAMBA_SCAN_GENERAL_A, MAMBA_SCAN_EULER, MAMBA_SCAN_TRAPEZOID, and 4, 8
+    and 32 states (zero-order hold, structured A)."""
+    import torch
+
+    from selective_state_space_29_b200 import mamba_ssm as m
+    from selective_state_space_29_b200 import workloads as wl
+
+    lib = m.library()
+    dtc = m.dtype_code(w.torch_dtype)
+    tc = w.batch * w.length * w.channels
+    cases = [("general_a", w, m.MAMBA_SCAN_GENERAL_A), ("euler", w, m.MAMBA_SCAN_EULER),
+             ("trapezoid", w, m.MAMBA_SCAN_TRAPEZOID)]
+    cases += [(f"nstate_{n}", w.with_(nstate=n), 0) for n in (4, 8, 32)]
+    res = {}
+    for name, wv, flags in cases:
+        inp = wl.scan_inputs(wv, dev, seed=rank_seed(wv.seed, rank))
+        y = torch.empty_like(inp["u"])
+        hf = torch.empty((wv.batch, wv.channels, wv.nstate), device=dev, dtype=torch.float32)
+
+        def step():
+            st = lib.mamba_selective_scan_ex(inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(),
+                                             inp["B"].data_ptr(), inp["C"].data_ptr(), inp["D"].data_ptr(), None,
+                                             y.data_ptr(), hf.data_ptr(), wv.batch, wv.length, wv.channels,
+                                             wv.nstate, 0, flags, dtc, stream.cuda_stream)
+            if st != 0:
+                raise m.MambaError(st, "mamba_selective_scan_ex")
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        barrier(dist, world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(dist, world, a.elapsed_time(b)) / reps
+        res[name] = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
+                     "nstate": wv.nstate}
+        del inp, y, hf
+    res["note"] = (f"{w.name} shape; general A and the other discretisations take one exp2 per state "
+                   f"(MUFU); nstate_* are zero-order hold with structured A")
+    return res
 
 
 # --- reference arm: the fp64 oracle on the host cores ------------------------------------
