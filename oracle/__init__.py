@@ -33,6 +33,8 @@ class Oracle:
         self._lib.oracle_scan.argtypes = [_c_f64p] * 9 + [_i64] * 4 + [ctypes.c_int]
         self._lib.oracle_scan_method.restype = ctypes.c_int
         self._lib.oracle_scan_method.argtypes = [_c_f64p] * 9 + [_i64] * 4 + [ctypes.c_int, ctypes.c_int]
+        self._lib.oracle_scan_backward.restype = ctypes.c_int
+        self._lib.oracle_scan_backward.argtypes = [_c_f64p] * 16 + [_i64] * 4
         self._lib.oracle_state_update.restype = ctypes.c_int
         self._lib.oracle_state_update.argtypes = [_c_f64p] * 8 + [_i64] * 3 + [ctypes.c_int]
         self._lib.oracle_max_threads.restype = ctypes.c_int
@@ -75,6 +77,27 @@ class Oracle:
         if rc != 0:
             raise RuntimeError(f"oracle_scan failed ({rc})")
         return y, hf
+
+    def scan_backward(self, u, delta, A, B, C, D, dy, h0=None, dh_final=None):
+        """Gradients of the zero-order-hold scan for an upstream gradient dy of
+        y (and dh_final of the final state): returns a dict with du, ddelta,
+        dA, dB, dC, dD (None when D is None) and dh0, all float64."""
+        u, delta, A, B, C, D, dy, h0, dh_final = map(self._f64, (u, delta, A, B, C, D, dy, h0, dh_final))
+        batch, length, channels = u.shape
+        nstate = A.shape[1]
+        assert dy.shape == u.shape
+        out = {"du": np.empty_like(u), "ddelta": np.empty_like(u), "dA": np.empty_like(A),
+               "dB": np.empty_like(B), "dC": np.empty_like(C),
+               "dD": None if D is None else np.empty_like(D),
+               "dh0": np.empty((batch, channels, nstate), dtype=np.float64)}
+        rc = self._lib.oracle_scan_backward(
+            self._ptr(u), self._ptr(delta), self._ptr(A), self._ptr(B), self._ptr(C), self._ptr(D), self._ptr(h0),
+            self._ptr(dy), self._ptr(dh_final), self._ptr(out["du"]), self._ptr(out["ddelta"]), self._ptr(out["dA"]),
+            self._ptr(out["dB"]), self._ptr(out["dC"]), self._ptr(out["dD"]), self._ptr(out["dh0"]),
+            batch, length, channels, nstate)
+        if rc != 0:
+            raise RuntimeError(f"oracle_scan_backward failed ({rc})")
+        return out
 
     def state_update(self, state, x, delta, A, B, C, D=None, nthreads=0):
         """One recurrent step.  state: (batch, channels, nstate) float64, updated

@@ -273,6 +273,106 @@ int oracle_scan_method(const double *u, const double *delta, const double *A,
     return status;
 }
 
+/* ------------------------------------------------------------------------
+ * Backward of the zero-order-hold scan (training).  The pages imply training
+ * ("Mamba'nın Yeniliği: Selective SSM": Delta, B and C are learned
+ * projections of the input) but print no gradient; this is reverse-mode
+ * differentiation of exactly the recurrence of oracle_scan, written out by
+ * the chain rule.  With lam_t = dL/dh_t (the adjoint), per state n and token
+ * t (z = Delta_t A_n, r = exp(z), Bbar = (r - 1)/A_n B_{t,n}):
+ *   lam_t     = C_t dy_t + r_{t+1} lam_{t+1}      (+ dh_final at t = L-1)
+ *   du_t      = sum_n lam_t Bbar + D dy_t
+ *   dDelta_t  = sum_n lam_t r (A_n h_{t-1} + B_{t,n} x_t)
+ *   dA_n     += lam_t (Delta_t r h_{t-1} + x_t B_{t,n} Delta_t^2 psi(z))
+ *               with psi(z) = (z e^z - (e^z - 1)) / z^2  (d Bbar / d A_n)
+ *   dB_{t,n} += lam_t x_t (r - 1)/A_n          (summed over channels)
+ *   dC_{t,n} += dy_t h_t                       (summed over channels)
+ *   dD       += dy_t x_t
+ *   dh0       = r_0 lam_0
+ * Single-threaded: dB, dC and dA are sums over rows.
+ * ------------------------------------------------------------------------ */
+static double psi(double z)
+{
+    if (fabs(z) < 1e-3)  /* series: 1/2 + z/3 + z^2/8 + z^3/30 */
+        return 0.5 + z * (1.0 / 3.0 + z * (1.0 / 8.0 + z / 30.0));
+    return (z * exp(z) - expm1(z)) / (z * z);
+}
+
+int oracle_scan_backward(const double *u, const double *delta, const double *A,
+                         const double *B, const double *C, const double *D,
+                         const double *h0, const double *dy, const double *dh_final,
+                         double *du, double *ddelta, double *dA, double *dB, double *dC,
+                         double *dD, double *dh0,
+                         int64_t batch, int64_t len, int64_t channels, int64_t nstate)
+{
+    if (batch < 0 || len < 0 || channels < 0 || nstate <= 0 || !A || !dA || !dB || !dC || !dh0)
+        return -1;
+    if (len > 0 && (!u || !delta || !B || !C || !dy || !du || !ddelta))
+        return -1;
+    for (int64_t i = 0; i < channels * nstate; ++i)
+        dA[i] = 0.0;
+    for (int64_t i = 0; i < batch * len * nstate; ++i)
+        dB[i] = dC[i] = 0.0;
+    if (dD)
+        for (int64_t d = 0; d < channels; ++d)
+            dD[d] = 0.0;
+    double *hs = (double *)malloc(sizeof(double) * (size_t)((len + 1) * nstate));
+    double *lam = (double *)malloc(sizeof(double) * (size_t)nstate);
+    if (!hs || !lam) {
+        free(hs);
+        free(lam);
+        return -1;
+    }
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < channels; ++d) {
+            const double *Ad = A + d * nstate;
+            /* forward: hs[(t+1)*N + n] = h_t, hs[n] = h_{-1} */
+            for (int64_t n = 0; n < nstate; ++n)
+                hs[n] = h0 ? h0[(b * channels + d) * nstate + n] : 0.0;
+            for (int64_t t = 0; t < len; ++t) {
+                const size_t k = (size_t)(b * len + t);
+                double x = u[k * channels + d], dt = delta[k * channels + d];
+                for (int64_t n = 0; n < nstate; ++n) {
+                    double abar, bbar;
+                    zoh_discretise(dt, Ad[n], B[k * nstate + n], &abar, &bbar);
+                    hs[(t + 1) * nstate + n] = abar * hs[t * nstate + n] + bbar * x;
+                }
+            }
+            /* reverse */
+            for (int64_t n = 0; n < nstate; ++n)
+                lam[n] = dh_final ? dh_final[(b * channels + d) * nstate + n] : 0.0;
+            for (int64_t t = len - 1; t >= 0; --t) {
+                const size_t k = (size_t)(b * len + t);
+                double x = u[k * channels + d], dt = delta[k * channels + d], g = dy[k * channels + d];
+                double dut = D ? D[d] * g : 0.0, ddt = 0.0;
+                if (dD)
+                    dD[d] += g * x;
+                for (int64_t n = 0; n < nstate; ++n) {
+                    double a = Ad[n], bn = B[k * nstate + n];
+                    double hprev = hs[t * nstate + n], ht = hs[(t + 1) * nstate + n];
+                    dC[k * nstate + n] += g * ht;              /* y_t = C_t . h_t + D x_t      */
+                    lam[n] += C[k * nstate + n] * g;           /* lam_t                       */
+                    double z = dt * a, r = exp(z);
+                    double phi = (z == 0.0) ? 1.0 : expm1(z) / z;
+                    double bbar = phi * dt * bn;
+                    dut += lam[n] * bbar;
+                    ddt += lam[n] * r * (a * hprev + bn * x);
+                    dA[d * nstate + n] += lam[n] * (dt * r * hprev + x * bn * dt * dt * psi(z));
+                    dB[k * nstate + n] += lam[n] * x * phi * dt;
+                    lam[n] *= r;                               /* towards lam_{t-1}           */
+                }
+                du[k * channels + d] = dut;
+                ddelta[k * channels + d] = ddt;
+            }
+            for (int64_t n = 0; n < nstate; ++n)
+                dh0[(b * channels + d) * nstate + n] = lam[n];
+        }
+    }
+    free(hs);
+    free(lam);
+    return 0;
+}
+
 /* Threads the OpenMP runtime would use (for reporting the CPU baseline). */
 int oracle_max_threads(void)
 {

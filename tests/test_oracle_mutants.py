@@ -40,6 +40,14 @@ MUTANTS = {
     "trapezoid_previous_is_current_x": ("abar * B[(t - 1) * nstate + n] * u[(t - 1) * stride]",
                                         "abar * B[(t - 1) * nstate + n] * u[t * stride]"),
     "methods_decay_sign_flipped": ("double abar = exp(dt * A_row[n]);", "double abar = exp(-dt * A_row[n]);"),
+    # the backward
+    "backward_adjoint_not_decayed": ("lam[n] *= r;", "(void)r;"),
+    "backward_dc_from_previous_state": ("dC[k * nstate + n] += g * ht;", "dC[k * nstate + n] += g * hprev;"),
+    "backward_psi_sign": ("return (z * exp(z) - expm1(z)) / (z * z);", "return (z * exp(z) + expm1(z)) / (z * z);"),
+    "backward_db_missing_x": ("dB[k * nstate + n] += lam[n] * x * phi * dt;", "dB[k * nstate + n] += lam[n] * phi * dt;"),
+    "backward_ddelta_missing_a": ("ddt += lam[n] * r * (a * hprev + bn * x);", "ddt += lam[n] * r * (hprev + bn * x);"),
+    "backward_adjoint_before_output": ("lam[n] += C[k * nstate + n] * g;           /* lam_t                       */",
+                                       "(void)0;"),
 }
 
 PIN_TESTS = [getattr(pins, name) for name in dir(pins) if name.startswith("test_")]

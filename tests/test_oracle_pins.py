@@ -393,3 +393,62 @@ def test_methods_share_the_zoh_transition(oracle_lib, method):
     tiny = np.full_like(delta, 1e-14)
     yt, _ = oracle_lib.scan(u, tiny, A, B, C, D, method=m)
     np.testing.assert_allclose(yt, u * D[None, None, :], rtol=0, atol=1e-12)
+
+
+# --- backward of the zero-order-hold scan -------------------------------------------------
+# Reverse mode of the same recurrence (training).  Pinned by finite differences of the
+# forward oracle (itself pinned above), by the LTI closed form of du (a correlation with the
+# convolution kernel), and by linearity in the upstream gradient.
+
+def _loss(oracle_lib, args, dy, dh):
+    u, delta, A, B, C, D, h0 = args
+    y, hf = oracle_lib.scan(u, delta, A, B, C, D, h0=h0)
+    return float((y * dy).sum() + (hf * dh).sum())
+
+
+def test_backward_matches_finite_differences(oracle_lib):
+    rng = np.random.default_rng(21)
+    u, delta, A, B, C, D = _rand_inputs(rng, 2, 5, 3, 4, dlo=0.05, dhi=0.5)
+    h0 = rng.standard_normal((2, 3, 4))
+    dy = rng.standard_normal(u.shape)
+    dh = rng.standard_normal(h0.shape)
+    g = oracle_lib.scan_backward(u, delta, A, B, C, D, dy, h0=h0, dh_final=dh)
+    args = [u, delta, A, B, C, D, h0]
+    names = ["du", "ddelta", "dA", "dB", "dC", "dD", "dh0"]
+    for i, name in enumerate(names):
+        base = args[i]
+        fd = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            step = 1e-6 * max(1.0, abs(base[idx]))
+            plus, minus = base.copy(), base.copy()
+            plus[idx] += step
+            minus[idx] -= step
+            a_p, a_m = list(args), list(args)
+            a_p[i], a_m[i] = plus, minus
+            fd[idx] = (_loss(oracle_lib, a_p, dy, dh) - _loss(oracle_lib, a_m, dy, dh)) / (2 * step)
+        np.testing.assert_allclose(g[name], fd, rtol=2e-6, atol=1e-8, err_msg=name)
+
+
+def test_backward_lti_du_is_correlation_with_kernel(oracle_lib):
+    """Constant Delta, B, C: y = K * x + D x, so du_t = sum_k K_k dy_{t+k} + D dy_t."""
+    rng = np.random.default_rng(22)
+    L, N = 48, 4
+    u, delta, A, B, C, Bv, Cv = _lti_inputs(rng, L, N, 0.07)
+    D = np.array([0.3])
+    dy = rng.standard_normal(u.shape)
+    g = oracle_lib.scan_backward(u, delta, A, B, C, D, dy)
+    ab, bb = _zoh_van_loan(A[0], Bv, 0.07)
+    K = np.array([(Cv * ab ** k * bb).sum() for k in range(L)])
+    ref = np.array([sum(K[k] * dy[0, t + k, 0] for k in range(L - t)) for t in range(L)]) + 0.3 * dy[0, :, 0]
+    np.testing.assert_allclose(g["du"][0, :, 0], ref, rtol=1e-10, atol=1e-12)
+
+
+def test_backward_linear_in_upstream_gradient(oracle_lib):
+    rng = np.random.default_rng(23)
+    u, delta, A, B, C, D = _rand_inputs(rng, 2, 9, 3, 4)
+    d1, d2 = rng.standard_normal(u.shape), rng.standard_normal(u.shape)
+    g1 = oracle_lib.scan_backward(u, delta, A, B, C, D, d1)
+    g2 = oracle_lib.scan_backward(u, delta, A, B, C, D, d2)
+    g12 = oracle_lib.scan_backward(u, delta, A, B, C, D, 2.0 * d1 - d2)
+    for k in ("du", "ddelta", "dA", "dB", "dC", "dD", "dh0"):
+        np.testing.assert_allclose(g12[k], 2.0 * g1[k] - g2[k], rtol=1e-10, atol=1e-12, err_msg=k)
