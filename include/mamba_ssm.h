@@ -115,6 +115,9 @@ typedef enum {
  * state from one time chunk to the next, and, when sequences are split into
  * independent super-chunks, their aggregates (mamba_scan_plan reports the
  * size).  batch == 0 or channels == 0 is a no-op that returns MAMBA_OK.
+ * The call enqueues only stream-ordered work (allocation, kernels, free), so
+ * it can be captured in a CUDA graph once a first call on the device has run
+ * outside capture (that call sets the kernels' shared-memory attribute).
  */
 int mamba_selective_scan(const void *u, const void *delta, const float *A,
                          const void *B, const void *C, const float *D,

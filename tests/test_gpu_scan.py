@@ -229,3 +229,24 @@ def test_scan_other_state_counts_chunked_and_initial_state(nstate):
 def test_scan_other_state_counts_methods(nstate):
     _check_full(SMALL.with_(nstate=nstate, length=500), method="trapezoid", chunk_len=123)
     _check_full(SMALL.with_(nstate=nstate, length=500, dtype="f32"), method="euler")
+
+
+@pytest.mark.parametrize("shape", ["groups", "super_chunks"])
+def test_scan_capture_in_cuda_graph(shape):
+    # the call only enqueues stream work (stream-ordered scratch, kernels), so
+    # it can be captured once and replayed; replays equal the eager call bit for bit
+    w = SMALL if shape == "groups" else SMALL.with_(batch=1, length=20000, channels=64)
+    inp = wl.scan_inputs(w, DEV)
+    y0, h0 = gpu_scan(inp)
+    y = torch.empty_like(y0)
+    hf = torch.empty_like(h0)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        m.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], y=y, final_state=hf)
+    for _ in range(2):
+        y.zero_()
+        hf.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y0) and torch.equal(hf, h0)
+    del g
