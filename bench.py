@@ -577,6 +577,36 @@ def run_variants(w, dev, stream, dist, world, rank, reps: int = 20):
         res[name] = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
                      "nstate": wv.nstate}
         del inp, y, hf
+    # the backward (gradients of every input from dy), zero-order hold
+    inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
+    dy = torch.randn(inp["u"].shape, device=dev).to(inp["u"].dtype)
+    f32 = dict(device=dev, dtype=torch.float32)
+    outs = [torch.empty_like(inp["u"]), torch.empty_like(inp["u"]), torch.empty(inp["A"].shape, **f32),
+            torch.empty(inp["B"].shape, **f32), torch.empty(inp["C"].shape, **f32), torch.empty(inp["D"].shape, **f32),
+            torch.empty((w.batch, w.channels, w.nstate), **f32)]
+
+    def bwd():
+        st = lib.mamba_selective_scan_backward(
+            inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(), inp["B"].data_ptr(),
+            inp["C"].data_ptr(), inp["D"].data_ptr(), None, dy.data_ptr(), None, *[o.data_ptr() for o in outs],
+            w.batch, w.length, w.channels, w.nstate, dtc, stream.cuda_stream)
+        if st != 0:
+            raise m.MambaError(st, "mamba_selective_scan_backward")
+
+    for _ in range(2):
+        bwd()
+    torch.cuda.synchronize()
+    barrier(dist, world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(5):
+        bwd()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(dist, world, a.elapsed_time(b)) / 5
+    res["backward"] = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
+                       "nstate": w.nstate, "includes": "checkpointing forward pass + reverse pass"}
+    del inp, dy, outs
     res["note"] = (f"{w.name} shape; general A and the other discretisations take one exp2 per state "
                    f"(MUFU); nstate_* are zero-order hold with structured A")
     return res

@@ -229,6 +229,46 @@ int mamba_selective_scan_host(const void *u, const void *delta, const float *A,
                               int64_t batch, int64_t len, int64_t channels, int64_t nstate,
                               int64_t piece_len, int dtype, mamba_stream_t stream);
 
+/*
+ * Backward of the zero-order-hold scan (training): the gradients of
+ * L(y, h_final) with respect to every input, given dy = dL/dy and
+ * d_final_state = dL/dh_final (NULL: zero).  The pages imply training but
+ * print no gradient; this is reverse-mode differentiation of the recurrence
+ * of mamba_selective_scan (per state n, z = Delta_t A_n, r = e^z):
+ *   lam_t = C_t dy_t + r_{t+1} lam_{t+1}          (the adjoint of h_t)
+ *   du_t = sum_n lam_t (r - 1)/A_n B_{t,n} + D dy_t
+ *   dDelta_t = sum_n lam_t r (A_n h_{t-1} + B_{t,n} x_t)
+ *   dA_n = sum over (b, t) of lam_t (Delta r h_{t-1} + x B Delta^2 psi(z)),
+ *          psi(z) = (z e^z - (e^z - 1)) / z^2
+ *   dB_{t,n} = sum over channels of lam_t x_t (r - 1)/A_n
+ *   dC_{t,n} = sum over channels of dy_t h_t,   dD = sum dy x,   dh0 = r_0 lam_0
+ *
+ *   u, delta, B, C, dy      device, dtype, layouts as the forward
+ *   A, D, initial_state     as the forward (D and initial_state may be NULL)
+ *   d_final_state           device, float32, [batch][channels][nstate], or NULL
+ *   du, ddelta              device, dtype, [batch][len][channels] (outputs)
+ *   dA                      device, float32, [channels][nstate] (output)
+ *   dB, dC                  device, float32, [batch][len][nstate] (outputs)
+ *   dD                      device, float32, [channels]; required when D is given
+ *   d_initial_state         device, float32, [batch][channels][nstate], or NULL
+ *   nstate                  4, 8 or 16 (32: MAMBA_ERR_UNSUPPORTED)
+ *
+ * It runs the forward scan once more, keeping only the state before every
+ * tile, then one warp per (batch, 32-channel group) walks the sequence in
+ * reverse, recomputing each tile's states from its checkpoint (stream-ordered
+ * scratch: the checkpoints and [T][32][nstate] floats per warp).  dA, dB,
+ * dC and dD are accumulated with atomic adds, so their last bits can vary
+ * from call to call.  Asynchronous on `stream`.
+ */
+int mamba_selective_scan_backward(const void *u, const void *delta, const float *A,
+                                  const void *B, const void *C, const float *D,
+                                  const float *initial_state, const void *dy,
+                                  const float *d_final_state,
+                                  void *du, void *ddelta, float *dA, float *dB, float *dC,
+                                  float *dD, float *d_initial_state,
+                                  int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                                  int dtype, mamba_stream_t stream);
+
 /* How mamba_selective_scan_ex would split a problem (host-side planning only). */
 typedef struct {
     int64_t supers;        /* independent super-chunks per sequence (1: no aggregate jobs) */

@@ -1,0 +1,192 @@
+// backward.cuh -- gradients of the zero-order-hold selective scan (training).
+//
+// The pages imply training (page "Mamba SSM Nedir? Transformer Alternatifi
+// Rehberi (2026)", section "Mamba'nın Yeniliği: Selective SSM": Delta, B and C
+// are learned projections of the input) but print no gradient.  This is
+// reverse-mode differentiation of the recurrence of section "Ayrık Zamana
+// Geçiş".  Per state n and token t, with z = Delta_t A_n, r = exp(z),
+// q = r - 1, lam = dL/dh_t (the adjoint):
+//     lam_t      = C_t dy_t + r_{t+1} lam_{t+1}          (+ d h_final at the end)
+//     du_t       = sum_n lam_t (q / A_n) B_{t,n} + D dy_t
+//     dDelta_t   = sum_n lam_t r (A_n h_{t-1} + B_{t,n} x_t)
+//     dA_n      += lam_t (Delta_t r h_{t-1} + x_t B_{t,n} Delta_t^2 psi(z)),
+//                  psi(z) = (z e^z - (e^z - 1)) / z^2
+//     dB_{t,n}  += lam_t x_t q / A_n                      (summed over channels)
+//     dC_{t,n}  += dy_t h_t                               (summed over channels)
+//     dD        += dy_t x_t,        dh0 = r_0 lam_0
+//
+// Work decomposition: a warp takes a (batch row, 32-channel group) stream at
+// a time, a lane per channel, and walks its tokens in reverse.  The states
+// are recomputed tile by tile: the forward kernel leaves the state before
+// every tile of T tokens in a checkpoint array; the warp re-runs a tile
+// forward from its checkpoint, writing h_t for each token to a per-warp
+// scratch area ([T][32][N], 64 bytes per lane and token at N = 16, small
+// enough to stay in L2), then takes the tile's reverse steps reading the
+// states back.  The channel sums for dB and dC are a warp reduce-scatter
+// (lane i ends with the sum of value i) and one atomic add per lane.
+#pragma once
+
+#include "common.cuh"
+#include "scan.cuh"  // expm1_small
+
+namespace mamba {
+
+template <typename TIO>
+struct BwdArgs {
+  const TIO* u;
+  const TIO* delta;
+  const float* A;
+  const TIO* B;
+  const TIO* C;
+  const float* D;          // nullable
+  const TIO* dy;
+  const float* dh_final;   // nullable
+  const float* ckpt;       // [batch][ntiles][channels][N]
+  float* scratch;          // [warps of the grid][T][32][N]
+  TIO* du;
+  TIO* ddelta;
+  float* dA;               // [channels][N], accumulated (zeroed by the host)
+  float* dB;               // [batch][len][N], accumulated
+  float* dC;               // [batch][len][N], accumulated
+  float* dD;               // [channels] or nullptr, accumulated
+  float* dh0;              // [batch][channels][N] or nullptr
+  int64_t batch, len, channels;
+  int groups_d;            // ceil(channels / 32)
+  int tile;                // checkpoint spacing T
+};
+
+// (z e^z - (e^z - 1)) / z^2 given q = e^z - 1, with its Taylor series
+// 1/2 + z/3 + z^2/8 + z^3/30 + z^4/144 for |z| < 1/4
+__device__ __forceinline__ float psi_f(float z, float q) {
+  if (fabsf(z) < 0.25f)
+    return fmaf(z, fmaf(z, fmaf(z, fmaf(z, 1.0f / 144.0f, 1.0f / 30.0f), 0.125f), 1.0f / 3.0f), 0.5f);
+  return (z * (1.0f + q) - q) / (z * z);
+}
+
+// Sum over the 32 lanes of v[0..31]; lane i returns the sum of v[i]
+// (butterfly reduce-scatter: at each step a lane keeps the half of its
+// values whose index has the lane's bit, and receives the partner's copy).
+__device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int w = 16; w >= 1; w >>= 1) {
+    const bool upper = (lane & w) != 0;
+#pragma unroll
+    for (int i = 0; i < w; ++i) {
+      const float send = upper ? v[i] : v[i + w];
+      const float keep = upper ? v[i + w] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+    }
+  }
+  return v[0];
+}
+
+constexpr int kBwdWarps = 8;  // warps per CTA of the backward kernel
+
+template <typename TIO, int NS>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+scan_backward_kernel(const BwdArgs<TIO> a) {
+  static_assert(2 * NS <= 32, "dB and dC of a token are reduced in one 32-lane pass");
+  griddep_wait();  // the checkpoints come from the previous kernel of the stream
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t wid = (int64_t)blockIdx.x * kBwdWarps + warp;
+  const int64_t nwarps = (int64_t)gridDim.x * kBwdWarps;
+  const int64_t streams = a.batch * a.groups_d;
+  const int T = a.tile;
+  const int64_t ntiles = (a.len + T - 1) / T;
+  float* S = a.scratch + (size_t)wid * (size_t)T * 32 * NS + (size_t)lane * NS;  // + k * 32 * NS
+
+  for (int64_t stream = wid; stream < streams; stream += nwarps) {
+    const int64_t b = stream / a.groups_d;
+    const int64_t d = (stream - b * a.groups_d) * 32 + lane;
+    const bool active = d < a.channels;
+    float An[NS], lam[NS], dA[NS];
+#pragma unroll
+    for (int n = 0; n < NS; ++n) {
+      An[n] = active ? __ldg(a.A + d * NS + n) : -1.0f;
+      lam[n] = (active && a.dh_final) ? a.dh_final[(b * a.channels + d) * NS + n] : 0.0f;
+      dA[n] = 0.0f;
+    }
+    const float Dd = (active && a.D) ? __ldg(a.D + d) : 0.0f;
+    float dD = 0.0f;
+
+    for (int64_t tile = ntiles - 1; tile >= 0; --tile) {
+      const int64_t t0 = tile * T;
+      const int rows = (int)(a.len - t0 < (int64_t)T ? a.len - t0 : (int64_t)T);
+      const float* ck = a.ckpt + ((b * ntiles + tile) * a.channels + (active ? d : 0)) * NS;
+      // forward over the tile: S[k] = h after token t0 + k
+      float h[NS];
+#pragma unroll
+      for (int n = 0; n < NS; ++n) h[n] = active ? ck[n] : 0.0f;
+      for (int k = 0; k < rows; ++k) {
+        const int64_t tok = b * a.len + t0 + k;
+        const float x = active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
+        const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+          const float q = expm1_small(dt * An[n]);
+          h[n] = fmaf(1.0f + q, h[n], (q / An[n]) * to_f32(a.B[tok * NS + n]) * x);
+        }
+#pragma unroll
+        for (int n = 0; n < NS; n += 4)
+          *reinterpret_cast<float4*>(S + (size_t)k * 32 * NS + n) = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
+      }
+      // reverse over the tile; h holds h_t, hp is read back as h_{t-1}
+      for (int k = rows - 1; k >= 0; --k) {
+        const int64_t tok = b * a.len + t0 + k;
+        float hp[NS];
+        if (k > 0) {
+#pragma unroll
+          for (int n = 0; n < NS; n += 4) {
+            const float4 v = *reinterpret_cast<const float4*>(S + (size_t)(k - 1) * 32 * NS + n);
+            hp[n] = v.x; hp[n + 1] = v.y; hp[n + 2] = v.z; hp[n + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int n = 0; n < NS; ++n) hp[n] = active ? ck[n] : 0.0f;
+        }
+        const float x = active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
+        const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+        const float gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
+        float du = Dd * gy, ddt = 0.0f;
+        dD = fmaf(gy, x, dD);
+        float red[32];
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+          const float bn = to_f32(a.B[tok * NS + n]);
+          const float z = dt * An[n];
+          const float q = expm1_small(z);
+          const float r = 1.0f + q;
+          const float qa = q / An[n];
+          red[NS + n] = gy * h[n];                      // dC_{t,n} part: dy_t h_t
+          lam[n] = fmaf(to_f32(a.C[tok * NS + n]), gy, lam[n]);
+          du = fmaf(lam[n], qa * bn, du);
+          ddt = fmaf(lam[n] * r, fmaf(An[n], hp[n], bn * x), ddt);
+          dA[n] = fmaf(lam[n], fmaf(dt * r, hp[n], x * bn * dt * dt * psi_f(z, q)), dA[n]);
+          red[n] = lam[n] * x * qa;                     // dB_{t,n} part
+          lam[n] *= r;
+          h[n] = hp[n];
+        }
+#pragma unroll
+        for (int n = 2 * NS; n < 32; ++n) red[n] = 0.0f;
+        if (active) {
+          a.du[tok * a.channels + d] = from_f32<TIO>(du);
+          a.ddelta[tok * a.channels + d] = from_f32<TIO>(ddt);
+        }
+        const float s = reduce_scatter32(red, lane);
+        if (lane < NS) atomicAdd(a.dB + tok * NS + lane, s);
+        else if (lane < 2 * NS) atomicAdd(a.dC + tok * NS + (lane - NS), s);
+      }
+    }
+    if (active) {
+#pragma unroll
+      for (int n = 0; n < NS; ++n) atomicAdd(a.dA + d * NS + n, dA[n]);
+      if (a.dD) atomicAdd(a.dD + d, dD);
+      if (a.dh0) {
+#pragma unroll
+        for (int n = 0; n < NS; ++n) a.dh0[(b * a.channels + d) * NS + n] = lam[n];
+      }
+    }
+  }
+}
+
+}  // namespace mamba

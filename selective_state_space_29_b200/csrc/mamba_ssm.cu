@@ -13,6 +13,7 @@
 
 #include "mamba_ssm.h"
 #include "common.cuh"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "scan.cuh"
 
@@ -248,7 +249,7 @@ template <typename TIO, int NS, int METHOD>
 int launch_scan_on(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
                    const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
                    unsigned flags, int dtype, cudaStream_t stream, const Plan& pl, int sms,
-                   unsigned char* scratch) {
+                   unsigned char* scratch, float* ckpt = nullptr) {
   constexpr int TILE = ScanCfg<TIO, NS>::kTile;
   constexpr int STAGES = ScanCfg<TIO, NS>::kStages;
   const ScratchLayout sl = scratch_layout(pl, NS, batch, len);
@@ -282,6 +283,7 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   std::memset(&p, 0, sizeof(p));
   p.u = u; p.delta = delta; p.A = A; p.B = B; p.cs = cs; p.chan = chan; p.h0 = h0; p.y = y;
   p.final_state = final_state;
+  p.ckpt = ckpt;
   p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd;
   p.batch = batch; p.len = len; p.channels = channels;
   p.groups_d = pl.groups_d; p.groups = (int)pl.groups;
@@ -348,7 +350,8 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
 template <typename TIO, int NS>
 int launch_scan(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
                 const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
-                int64_t user_chunk, unsigned flags, int dtype, cudaStream_t stream, bool noalloc) {
+                int64_t user_chunk, unsigned flags, int dtype, cudaStream_t stream, bool noalloc,
+                float* ckpt = nullptr) {
   int sms = 0;
   if (int st = current_sms(&sms)) return st;
   const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO, NS>::kTile, user_chunk);
@@ -372,7 +375,7 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
                                                  flags, dtype, stream, pl, sms, scratch);
   else
     status = launch_scan_on<TIO, NS, kZOH>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags,
-                                           dtype, stream, pl, sms, scratch);
+                                           dtype, stream, pl, sms, scratch, ckpt);
   if (!noalloc && cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) return MAMBA_ERR_CUDA;
   return status;
 }
@@ -609,6 +612,85 @@ int mamba_selective_scan_host(const void* u, const void* delta, const float* A, 
   }
   return scan_host_pipelined(u, delta, A, B, C, D, y, final_state, batch, len, channels, nstate, piece_len, dtype,
                              stream);
+}
+
+int mamba_selective_scan_backward(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                                  const float* D, const float* initial_state, const void* dy,
+                                  const float* d_final_state, void* du, void* ddelta, float* dA, float* dB,
+                                  float* dC, float* dD, float* d_initial_state, int64_t batch, int64_t len,
+                                  int64_t channels, int64_t nstate, int dtype, mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || len < 0 || channels < 0 || nstate <= 0) return MAMBA_ERR_INVALID_ARG;
+  if (nstate != 4 && nstate != 8 && nstate != 16) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || channels == 0) return MAMBA_OK;
+  if (!A || !dA || !dB || !dC || (D && !dD)) return MAMBA_ERR_INVALID_ARG;
+  const size_t es = (size_t)elem_size(dtype);
+  if (len > 0) {
+    if (!u || !delta || !B || !C || !dy || !du || !ddelta) return MAMBA_ERR_INVALID_ARG;
+    if (!aligned(u, es) || !aligned(delta, es) || !aligned(B, es) || !aligned(C, es) || !aligned(dy, es) ||
+        !aligned(du, es) || !aligned(ddelta, es))
+      return MAMBA_ERR_INVALID_ARG;
+  }
+  if (!aligned(A, 4) || !aligned(dA, 4) || !aligned(dB, 4) || !aligned(dC, 4) || (D && !aligned(D, 4)) ||
+      (dD && !aligned(dD, 4)) || (initial_state && !aligned(initial_state, 4)) ||
+      (d_final_state && !aligned(d_final_state, 4)) || (d_initial_state && !aligned(d_initial_state, 4)))
+    return MAMBA_ERR_INVALID_ARG;
+  if (batch * len >= (int64_t(1) << 31) || channels >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+  cudaGetLastError();
+  const size_t state_bytes = sizeof(float) * (size_t)batch * (size_t)channels * (size_t)nstate;
+  // gradients that are sums start at zero
+  if (cudaMemsetAsync(dA, 0, sizeof(float) * (size_t)channels * (size_t)nstate, stream) != cudaSuccess ||
+      cudaMemsetAsync(dB, 0, sizeof(float) * (size_t)batch * (size_t)len * (size_t)nstate, stream) != cudaSuccess ||
+      cudaMemsetAsync(dC, 0, sizeof(float) * (size_t)batch * (size_t)len * (size_t)nstate, stream) != cudaSuccess ||
+      (dD && D && cudaMemsetAsync(dD, 0, sizeof(float) * (size_t)channels, stream) != cudaSuccess))
+    return MAMBA_ERR_CUDA;
+  if (len == 0) {
+    if (!d_initial_state) return MAMBA_OK;
+    const cudaError_t e = d_final_state ? cudaMemcpyAsync(d_initial_state, d_final_state, state_bytes,
+                                                          cudaMemcpyDeviceToDevice, stream)
+                                        : cudaMemsetAsync(d_initial_state, 0, state_bytes, stream);
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+  }
+  int sms = 0;
+  if (int st = current_sms(&sms)) return st;
+  return dispatch_nstate(nstate, [&](auto ns) -> int {
+    constexpr int NS = decltype(ns)::value;
+    if constexpr (NS > 16) {
+      return MAMBA_ERR_UNSUPPORTED;
+    } else {
+      auto run = [&](auto tio) -> int {
+        using TIO = decltype(tio);
+        constexpr int T = ScanCfg<TIO, NS>::kTile;
+        const int64_t ntiles = (len + T - 1) / T;
+        const int64_t groups_d = (channels + 31) / 32;
+        const int64_t streams = batch * groups_d;
+        const int64_t ctas = std::min<int64_t>((streams + kBwdWarps - 1) / kBwdWarps, 2 * (int64_t)sms);
+        auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
+        const size_t ck_bytes = al(sizeof(float) * (size_t)batch * (size_t)ntiles * (size_t)channels * NS);
+        const size_t sc_bytes = al(sizeof(float) * (size_t)ctas * kBwdWarps * T * 32 * NS);
+        unsigned char* mem = nullptr;
+        if (cudaMallocAsync(reinterpret_cast<void**>(&mem), ck_bytes + sc_bytes, stream) != cudaSuccess)
+          return MAMBA_ERR_CUDA;
+        float* ckpt = reinterpret_cast<float*>(mem);
+        // forward pass that only leaves the state before every tile
+        int st = launch_scan<TIO, NS>(u, delta, A, B, C, D, initial_state, nullptr, nullptr, batch, len, channels, 0,
+                                      0u, dtype, stream, false, ckpt);
+        if (st == MAMBA_OK) {
+          BwdArgs<TIO> a{static_cast<const TIO*>(u), static_cast<const TIO*>(delta), A, static_cast<const TIO*>(B),
+                         static_cast<const TIO*>(C), D, static_cast<const TIO*>(dy), d_final_state, ckpt,
+                         reinterpret_cast<float*>(mem + ck_bytes), static_cast<TIO*>(du), static_cast<TIO*>(ddelta),
+                         dA, dB, dC, D ? dD : nullptr, d_initial_state, batch, len, channels, (int)groups_d, T};
+          if (launch_pdl(scan_backward_kernel<TIO, NS>, dim3((unsigned)ctas), dim3(kBwdWarps * 32), 0, stream, a) !=
+              cudaSuccess)
+            st = MAMBA_ERR_CUDA;
+        }
+        if (cudaFreeAsync(mem, stream) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+        return st;
+      };
+      return dtype == MAMBA_BF16 ? run(__nv_bfloat16{}) : run(float{});
+    }
+  });
 }
 
 int mamba_selective_scan_noalloc(const void* u, const void* delta, const float* A, const void* B, const void* C,

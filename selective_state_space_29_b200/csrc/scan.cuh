@@ -71,8 +71,9 @@ struct ScanParams {
   const float* cs;          // C' = C / (n+1), fp32 [batch*len][N] (scratch, written by the pre-pass)
   const float4* chan;       // per channel {A[d,0], 1/A[d,0], D[d], structured}, padded to groups_d*32
   const float* h0;          // nullable: initial state [b][d][n]
-  void* y;
+  void* y;                  // nullable: no output (checkpoint-only runs for the backward)
   float* final_state;       // nullable
+  float* ckpt;              // nullable: [batch][ceil(len/TILE)][channels][N] state before every tile
   // scratch (stream-ordered; the pre-pass zeroes counters and done)
   int* counters;            // [0] job ticket, [1] abort flag
   int* done;                // [S*G] chunks completed per main stream
@@ -745,10 +746,20 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, con
       vp[k] = has_prev ? to_f32(static_cast<const TIO*>(p.B)[prow * NS + k]) * xprev : 0.0f;
   }
 
+  const bool store_y = active && p.y != nullptr;
   TIO* yrow = static_cast<TIO*>(p.y) + ((int64_t)jb.b * p.len + jb.t0) * p.channels + d;
   for (int it = 0; it < jb.ntiles; ++it) {
     const int64_t tt0 = jb.t0 + (int64_t)it * TILE;
     const int rows = (int)(jb.t1 - tt0 < (int64_t)TILE ? jb.t1 - tt0 : (int64_t)TILE);
+    if (FULL && p.ckpt && active) {
+      // the state before this tile, unscaled (tiles start at multiples of TILE)
+      float* ck = p.ckpt + (((int64_t)jb.b * ((p.len + TILE - 1) / TILE) + tt0 / TILE) * p.channels + d) * NS;
+#pragma unroll
+      for (int k = 0; k < NS; ++k) {
+        const float an = STRUCT ? (float)(k + 1) * a0 : __ldg(Arow + k);
+        ck[k] = ((k & 1) ? g[k >> 1].y : g[k >> 1].x) / an;
+      }
+    }
     const int slot = it == 0 ? s0 : cx.wait_tile();
     if (slot < 0) return false;
     if (!p.use_tma) cx.fetch_tile(slot, jb, tt0, rows, d, active);
@@ -757,10 +768,10 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, con
     if constexpr (STRUCT) {
       constexpr bool kFastQ = sizeof(TIO) == 2;  // bf16 data: hardware exp2 for expm1
       tile_structured<TIO, NS, TILE, FULL, kFastQ>(su, sdl, sm.b[slot], sm.cs[slot], rows, a0, cm.y, Dd, g, sd, yrow,
-                                                   p.channels, active);
+                                                   p.channels, store_y);
     } else {
       tile_general<TIO, NS, FULL, METHOD>(su, sdl, sm.b[slot], sm.cs[slot], rows, kA, kC, Dd, g, sd, vp, yrow,
-                                          p.channels, active);
+                                          p.channels, store_y);
     }
     yrow += (int64_t)rows * p.channels;
     cx.release_tile();

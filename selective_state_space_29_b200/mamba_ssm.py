@@ -48,6 +48,8 @@ _SIGNATURES = [
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_selective_scan_host", ctypes.c_int,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I64, _I64, ctypes.c_int, _P]),
+    ("mamba_selective_scan_backward", ctypes.c_int,
+     [_P] * 16 + [_I64, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_state_update", ctypes.c_int,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_scan_plan", ctypes.c_int,
@@ -158,6 +160,15 @@ def mamba_selective_scan_host(u, delta, A, B, C, D, y, final_state, batch, len, 
     _check(st, "mamba_selective_scan_host")
 
 
+def mamba_selective_scan_backward(u, delta, A, B, C, D, initial_state, dy, d_final_state, du, ddelta, dA, dB, dC,
+                                  dD, d_initial_state, batch, len, channels, nstate, dtype, stream=None):
+    st = library().mamba_selective_scan_backward(
+        _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(initial_state), _ptr(dy), _ptr(d_final_state),
+        _ptr(du), _ptr(ddelta), _ptr(dA), _ptr(dB), _ptr(dC), _ptr(dD), _ptr(d_initial_state), batch, len, channels,
+        nstate, dtype, _stream(stream))
+    _check(st, "mamba_selective_scan_backward")
+
+
 def mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, dtype, stream=None):
     st = library().mamba_state_update(_ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
                                       _ptr(y), batch, channels, nstate, dtype, _stream(stream))
@@ -251,3 +262,25 @@ def selective_scan_host(u, delta, A, B, C, D=None, y=None, final_state=None, pie
     if synchronize:
         torch.cuda.synchronize()
     return y, final_state
+
+
+def selective_scan_backward(u, delta, A, B, C, D, dy, initial_state=None, d_final_state=None, stream=None):
+    """Gradients of the zero-order-hold scan for an upstream gradient dy of y
+    (and d_final_state of the final state), on CUDA tensors.  Returns a dict:
+    du, ddelta (dtype of u), dA, dB, dC, dD (None without D), d_initial_state
+    (float32)."""
+    import torch
+    batch, length, channels = u.shape
+    nstate = A.shape[1]
+    for t in (u, delta, A, B, C, D, dy, initial_state, d_final_state):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    f32 = dict(device=u.device, dtype=torch.float32)
+    out = {"du": torch.empty_like(u), "ddelta": torch.empty_like(delta), "dA": torch.empty(A.shape, **f32),
+           "dB": torch.empty(B.shape, **f32), "dC": torch.empty(C.shape, **f32),
+           "dD": None if D is None else torch.empty(D.shape, **f32),
+           "d_initial_state": torch.empty((batch, channels, nstate), **f32)}
+    mamba_selective_scan_backward(u, delta, A, B, C, D, initial_state, dy, d_final_state, out["du"], out["ddelta"],
+                                  out["dA"], out["dB"], out["dC"], out["dD"], out["d_initial_state"], batch, length,
+                                  channels, nstate, dtype_code(u.dtype), stream)
+    return out

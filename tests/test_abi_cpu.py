@@ -129,6 +129,30 @@ def test_host_scan_argument_errors(lib):
     assert call(8, 0) == m.MAMBA_OK                     # empty
 
 
+def test_backward_argument_errors(lib):
+    f = lib.mamba_selective_scan_backward
+    base = [1024] * 16 + [1, 4, 8, 16, m.MAMBA_BF16, None]
+    base[5] = None   # D
+    base[6] = None   # initial state
+    base[8] = None   # d_final_state
+    base[14] = None  # dD
+    base[15] = None  # d_initial_state
+
+    def call(i, v):
+        a = list(base)
+        a[i] = v
+        return f(*a)
+    assert call(20, 9) == m.MAMBA_ERR_INVALID_ARG      # dtype
+    assert call(16, -1) == m.MAMBA_ERR_INVALID_ARG     # batch
+    assert call(19, 12) == m.MAMBA_ERR_UNSUPPORTED     # nstate
+    assert call(19, 32) == m.MAMBA_ERR_UNSUPPORTED     # nstate 32: forward only
+    assert call(7, None) == m.MAMBA_ERR_INVALID_ARG    # dy
+    assert call(11, None) == m.MAMBA_ERR_INVALID_ARG   # dA
+    assert call(5, 1024) == m.MAMBA_ERR_INVALID_ARG    # D given without dD
+    assert call(9, 1025) == m.MAMBA_ERR_INVALID_ARG    # misaligned du
+    assert call(16, 0) == m.MAMBA_OK                   # empty
+
+
 def test_library_links_no_torch(lib):
     # the product library is plain C ABI over CUDA: no torch / python symbols needed
     out = os.popen(f"nm -D --undefined-only {lib_build.LIB}").read()
