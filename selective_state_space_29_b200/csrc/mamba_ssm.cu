@@ -665,7 +665,7 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
         const int64_t ntiles = (len + T - 1) / T;
         const int64_t groups_d = (channels + 31) / 32;
         const int64_t streams = batch * groups_d;
-        const int64_t ctas = std::min<int64_t>((streams + kBwdWarps - 1) / kBwdWarps, 2 * (int64_t)sms);
+        const int64_t ctas = std::min<int64_t>((streams + kBwdWarps - 1) / kBwdWarps, 3 * (int64_t)sms);
         auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
         const size_t ck_bytes = al(sizeof(float) * (size_t)batch * (size_t)ntiles * (size_t)channels * NS);
         const size_t sc_bytes = al(sizeof(float) * (size_t)ctas * kBwdWarps * T * 32 * NS);
@@ -680,7 +680,8 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
           BwdArgs<TIO> a{static_cast<const TIO*>(u), static_cast<const TIO*>(delta), A, static_cast<const TIO*>(B),
                          static_cast<const TIO*>(C), D, static_cast<const TIO*>(dy), d_final_state, ckpt,
                          reinterpret_cast<float*>(mem + ck_bytes), static_cast<TIO*>(du), static_cast<TIO*>(ddelta),
-                         dA, dB, dC, D ? dD : nullptr, d_initial_state, batch, len, channels, (int)groups_d, T};
+                         dA, dB, dC, D ? dD : nullptr, d_initial_state, batch, len, channels, (int)groups_d, T,
+                         (aligned(B, 16) && aligned(C, 16) && (NS * sizeof(TIO)) % 16 == 0) ? 1 : 0};
           if (launch_pdl(scan_backward_kernel<TIO, NS>, dim3((unsigned)ctas), dim3(kBwdWarps * 32), 0, stream, a) !=
               cudaSuccess)
             st = MAMBA_ERR_CUDA;
