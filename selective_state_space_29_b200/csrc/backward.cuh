@@ -54,6 +54,10 @@ struct BwdArgs {
   int groups_d;            // ceil(channels / 32)
   int tile;                // checkpoint spacing T
   int vec_rows;            // B and C rows may be read with 16-byte vector loads
+  int supers;              // S: the sequence is cut into S super-chunks of super_tiles tiles
+  int super_tiles;
+  float* agg_mu;           // [S][streams][32][N] outgoing adjoint of super-chunk j from zero
+  float* agg_sd;           // [S][streams][32] sum of Delta over super-chunk j
 };
 
 // (z e^z - (e^z - 1)) / z^2 given q = e^z - 1 and inv_z2 = 1/z^2: its Taylor
@@ -117,6 +121,51 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
 
 constexpr int kBwdWarps = 4;  // warps per CTA of the backward kernel
 
+// Outgoing adjoint of each super-chunk j >= 1 from a zero incoming adjoint,
+// M_j (after its first token, multiplied by that token's exp(Delta A)), and
+// its sum of Delta: the reverse counterpart of the forward aggregates.  Only
+// C, dy and Delta enter (no state).  One warp per (super-chunk, stream).
+template <typename TIO, int NS>
+__global__ void __launch_bounds__(kBwdWarps * 32)
+scan_backward_aggregate_kernel(const BwdArgs<TIO> a) {
+  griddep_wait();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t streams = a.batch * a.groups_d;
+  const int64_t item = (int64_t)blockIdx.x * kBwdWarps + warp;  // (j - 1) * streams + stream
+  if (item >= (int64_t)(a.supers - 1) * streams) return;
+  const int j = 1 + (int)(item / streams);
+  const int64_t stream = item - (int64_t)(j - 1) * streams;
+  const int64_t b = stream / a.groups_d;
+  const int64_t d = (stream - b * a.groups_d) * 32 + lane;
+  const bool active = d < a.channels;
+  const int T = a.tile;
+  const int64_t ntiles = (a.len + T - 1) / T;
+  const int64_t t_lo = (int64_t)j * a.super_tiles * T;
+  const int64_t t_hi = (j == a.supers - 1) ? a.len : (int64_t)(j + 1) * a.super_tiles * T;
+  (void)ntiles;
+  float An[NS], mu[NS];
+#pragma unroll
+  for (int n = 0; n < NS; ++n) {
+    An[n] = active ? __ldg(a.A + d * NS + n) : -1.0f;
+    mu[n] = 0.0f;
+  }
+  float sd = 0.0f;
+  for (int64_t t = t_hi - 1; t >= t_lo; --t) {
+    const int64_t tok = b * a.len + t;
+    const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+    const float gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
+    float cv[NS];
+    load_row<TIO, NS>(a.C + tok * NS, cv, a.vec_rows);
+    sd += dt;
+#pragma unroll
+    for (int n = 0; n < NS; ++n) mu[n] = (1.0f + expm1_small(dt * An[n])) * fmaf(cv[n], gy, mu[n]);
+  }
+  const size_t base = ((size_t)j * streams + stream) * 32 + lane;
+  a.agg_sd[base] = sd;
+#pragma unroll
+  for (int n = 0; n < NS; ++n) a.agg_mu[base * NS + n] = mu[n];
+}
+
 template <typename TIO, int NS>
 __global__ void __launch_bounds__(kBwdWarps * 32)
 scan_backward_kernel(const BwdArgs<TIO> a) {
@@ -130,7 +179,10 @@ scan_backward_kernel(const BwdArgs<TIO> a) {
   const int64_t ntiles = (a.len + T - 1) / T;
   float* S = a.scratch + (size_t)wid * (size_t)T * 32 * NS + (size_t)lane * NS;  // + k * 32 * NS
 
-  for (int64_t stream = wid; stream < streams; stream += nwarps) {
+  // work item = (super-chunk j, stream), the later super-chunks first
+  for (int64_t item = wid; item < (int64_t)a.supers * streams; item += nwarps) {
+    const int j = a.supers - 1 - (int)(item / streams);
+    const int64_t stream = item - (int64_t)(a.supers - 1 - j) * streams;
     const int64_t b = stream / a.groups_d;
     const int64_t d = (stream - b * a.groups_d) * 32 + lane;
     const bool active = d < a.channels;
@@ -142,10 +194,20 @@ scan_backward_kernel(const BwdArgs<TIO> a) {
       lam[n] = (active && a.dh_final) ? a.dh_final[(b * a.channels + d) * NS + n] : 0.0f;
       dA[n] = 0.0f;
     }
+    // the adjoint entering super-chunk j from the later ones:
+    //   mu <- M_k + exp(A sumDelta_k) mu,  k = S-1 .. j+1,  mu_S = d h_final
+    for (int k = a.supers - 1; k > j; --k) {
+      const size_t base = ((size_t)k * streams + stream) * 32 + lane;
+      const float sdk = a.agg_sd[base];
+#pragma unroll
+      for (int n = 0; n < NS; ++n) lam[n] = fmaf(expf(An[n] * sdk), lam[n], a.agg_mu[base * NS + n]);
+    }
     const float Dd = (active && a.D) ? __ldg(a.D + d) : 0.0f;
     float dD = 0.0f;
 
-    for (int64_t tile = ntiles - 1; tile >= 0; --tile) {
+    const int64_t tile_lo = (int64_t)j * a.super_tiles;
+    const int64_t tile_hi = (j == a.supers - 1) ? ntiles : tile_lo + a.super_tiles;
+    for (int64_t tile = tile_hi - 1; tile >= tile_lo; --tile) {
       const int64_t t0 = tile * T;
       const int rows = (int)(a.len - t0 < (int64_t)T ? a.len - t0 : (int64_t)T);
       const float* ck = a.ckpt + ((b * ntiles + tile) * a.channels + (active ? d : 0)) * NS;
@@ -224,7 +286,7 @@ scan_backward_kernel(const BwdArgs<TIO> a) {
 #pragma unroll
       for (int n = 0; n < NS; ++n) atomicAdd(a.dA + d * NS + n, dA[n]);
       if (a.dD) atomicAdd(a.dD + d, dD);
-      if (a.dh0) {
+      if (a.dh0 && j == 0) {
 #pragma unroll
         for (int n = 0; n < NS; ++n) a.dh0[(b * a.channels + d) * NS + n] = lam[n];
       }

@@ -665,12 +665,23 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
         const int64_t ntiles = (len + T - 1) / T;
         const int64_t groups_d = (channels + 31) / 32;
         const int64_t streams = batch * groups_d;
-        const int64_t ctas = std::min<int64_t>((streams + kBwdWarps - 1) / kBwdWarps, 3 * (int64_t)sms);
+        // the sequence is cut into S super-chunks run in parallel (about two
+        // work items per resident warp); their incoming adjoints come from
+        // the reverse aggregates of the later super-chunks
+        const int64_t resident = 3 * (int64_t)sms * kBwdWarps;
+        const int64_t S = std::max<int64_t>(1, std::min<int64_t>((2 * resident + streams - 1) / streams, ntiles));
+        const int64_t super_tiles = (ntiles + S - 1) / S;
+        const int64_t supers = (ntiles + super_tiles - 1) / super_tiles;
+        const int64_t items = supers * streams;
+        const int64_t ctas = std::min<int64_t>((items + kBwdWarps - 1) / kBwdWarps, 3 * (int64_t)sms);
         auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
         const size_t ck_bytes = al(sizeof(float) * (size_t)batch * (size_t)ntiles * (size_t)channels * NS);
         const size_t sc_bytes = al(sizeof(float) * (size_t)ctas * kBwdWarps * T * 32 * NS);
+        const size_t mu_bytes = al(sizeof(float) * (size_t)supers * (size_t)streams * 32 * NS);
+        const size_t sd_bytes = al(sizeof(float) * (size_t)supers * (size_t)streams * 32);
         unsigned char* mem = nullptr;
-        if (cudaMallocAsync(reinterpret_cast<void**>(&mem), ck_bytes + sc_bytes, stream) != cudaSuccess)
+        if (cudaMallocAsync(reinterpret_cast<void**>(&mem), ck_bytes + sc_bytes + mu_bytes + sd_bytes, stream) !=
+            cudaSuccess)
           return MAMBA_ERR_CUDA;
         float* ckpt = reinterpret_cast<float*>(mem);
         // forward pass that only leaves the state before every tile
@@ -681,9 +692,19 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
                          static_cast<const TIO*>(C), D, static_cast<const TIO*>(dy), d_final_state, ckpt,
                          reinterpret_cast<float*>(mem + ck_bytes), static_cast<TIO*>(du), static_cast<TIO*>(ddelta),
                          dA, dB, dC, D ? dD : nullptr, d_initial_state, batch, len, channels, (int)groups_d, T,
-                         (aligned(B, 16) && aligned(C, 16) && (NS * sizeof(TIO)) % 16 == 0) ? 1 : 0};
-          if (launch_pdl(scan_backward_kernel<TIO, NS>, dim3((unsigned)ctas), dim3(kBwdWarps * 32), 0, stream, a) !=
-              cudaSuccess)
+                         (aligned(B, 16) && aligned(C, 16) && (NS * sizeof(TIO)) % 16 == 0) ? 1 : 0, (int)supers,
+                         (int)super_tiles, reinterpret_cast<float*>(mem + ck_bytes + sc_bytes),
+                         reinterpret_cast<float*>(mem + ck_bytes + sc_bytes + mu_bytes)};
+          if (supers > 1) {
+            const int64_t agg_items = (supers - 1) * streams;
+            if (launch_pdl(scan_backward_aggregate_kernel<TIO, NS>,
+                           dim3((unsigned)((agg_items + kBwdWarps - 1) / kBwdWarps)), dim3(kBwdWarps * 32), 0, stream,
+                           a) != cudaSuccess)
+              st = MAMBA_ERR_CUDA;
+          }
+          if (st == MAMBA_OK &&
+              launch_pdl(scan_backward_kernel<TIO, NS>, dim3((unsigned)ctas), dim3(kBwdWarps * 32), 0, stream, a) !=
+                  cudaSuccess)
             st = MAMBA_ERR_CUDA;
         }
         if (cudaFreeAsync(mem, stream) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;

@@ -1,7 +1,8 @@
 """GPU parity of the scan's backward (mamba_selective_scan_backward) against the
 fp64 oracle's reverse-mode gradients, through the C ABI: every gradient, both
-dtypes, 4/8/16 states, initial state and final-state gradient, several tiles
-and ragged channel groups."""
+dtypes, 4/8/16 states, initial state and final-state gradient, several tiles,
+ragged channel groups, and sequences cut into super-chunks of one and of
+several tiles (the last shape: 256 streams, 16 tiles)."""
 import numpy as np
 import pytest
 import torch
@@ -22,7 +23,8 @@ def _rel(g, r):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("shape", [(2, 300, 100, 16), (1, 1000, 64, 8), (3, 200, 40, 4), (1, 64, 32, 16)])
+@pytest.mark.parametrize("shape", [(2, 300, 100, 16), (1, 1000, 64, 8), (3, 200, 40, 4), (1, 64, 32, 16),
+                                   (8, 1024, 1024, 16)])
 @pytest.mark.parametrize("extras", [False, True])
 def test_backward_matches_oracle(dtype, shape, extras):
     b, L, ch, n = shape
