@@ -9,11 +9,16 @@
 //     lam_t      = C_t dy_t + r_{t+1} lam_{t+1}          (+ d h_final at the end)
 //     du_t       = sum_n lam_t (q / A_n) B_{t,n} + D dy_t
 //     dDelta_t   = sum_n lam_t r (A_n h_{t-1} + B_{t,n} x_t)
-//     dA_n      += lam_t (Delta_t r h_{t-1} + x_t B_{t,n} Delta_t^2 psi(z)),
-//                  psi(z) = (z e^z - (e^z - 1)) / z^2
+//     dA_n      += lam_t (Delta_t r (h_{t-1} + B_{t,n} x_t / A_n) - q B_{t,n} x_t / A_n^2)
 //     dB_{t,n}  += lam_t x_t q / A_n                      (summed over channels)
 //     dC_{t,n}  += dy_t h_t                               (summed over channels)
 //     dD        += dy_t x_t,        dh0 = r_0 lam_0
+//
+// (the dA term is d h_t / d A_n at fixed Delta, with the derivative of
+// (e^z - 1)/A_n written out; its two parts nearly cancel only when the term
+// itself is small, so the sum over tokens keeps fp32 accuracy).  With
+// structured A (A[d,n] = (n+1) A[d,0]) the decays come from one exponential
+// per token and the forward kernel's decay chain.
 //
 // Work decomposition: a warp takes a (batch row, 32-channel group) stream at
 // a time, a lane per channel, and walks its tokens in reverse.  The states
@@ -59,15 +64,6 @@ struct BwdArgs {
   float* agg_mu;           // [S][streams][32][N] outgoing adjoint of super-chunk j from zero
   float* agg_sd;           // [S][streams][32] sum of Delta over super-chunk j
 };
-
-// (z e^z - (e^z - 1)) / z^2 given q = e^z - 1 and inv_z2 = 1/z^2: its Taylor
-// series 1/2 + z/3 + z^2/8 + z^3/30 + z^4/144 for |z| < 1/4 (truncation below
-// 2e-6 relative there), the closed form otherwise; both evaluated, one selected
-__device__ __forceinline__ float psi_f(float z, float q, float inv_z2) {
-  const float series = fmaf(z, fmaf(z, fmaf(z, fmaf(z, 1.0f / 144.0f, 1.0f / 30.0f), 0.125f), 1.0f / 3.0f), 0.5f);
-  const float closed = fmaf(z, 1.0f + q, -q) * inv_z2;
-  return fabsf(z) < 0.25f ? series : closed;
-}
 
 // the B (or C) row of a token as NS floats: vector loads of the raw row
 template <typename TIO, int NS>
@@ -121,10 +117,67 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
 
 constexpr int kBwdWarps = 4;  // warps per CTA of the backward kernel
 
-// Outgoing adjoint of each super-chunk j >= 1 from a zero incoming adjoint,
-// M_j (after its first token, multiplied by that token's exp(Delta A)), and
-// its sum of Delta: the reverse counterpart of the forward aggregates.  Only
-// C, dy and Delta enter (no state).  One warp per (super-chunk, stream).
+// q_n = exp(Delta A_n) - 1 for all states of one lane and token.  STRUCT
+// (A[d,n] = (n+1) A[d,0] on every lane of the warp): one accurate expm1 and
+// the decay chain of the forward kernel; otherwise one expm1 per state.
+template <int NS, bool STRUCT>
+__device__ __forceinline__ void decays(float dt, const float (&An)[NS], float (&q)[NS]) {
+  if constexpr (STRUCT) {
+    const float q0 = expm1_small(dt * An[0]);
+    float2 e2[NS / 2];
+    decay_chain<NS>(1.0f + q0, q0, e2);
+#pragma unroll
+    for (int k = 0; k < NS / 2; ++k) {
+      q[2 * k] = e2[k].x;
+      q[2 * k + 1] = e2[k].y;
+    }
+  } else {
+#pragma unroll
+    for (int n = 0; n < NS; ++n) q[n] = expm1_small(dt * An[n]);
+  }
+}
+
+// A work item's channel group has structured A (every lane, exact fp32 test)
+template <int NS>
+__device__ __forceinline__ bool group_structured(const float (&An)[NS]) {
+  bool ok = An[0] < 0.0f;
+#pragma unroll
+  for (int n = 1; n < NS; ++n) ok &= (An[n] == (float)(n + 1) * An[0]);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Outgoing adjoint of super-chunk j >= 1 from a zero incoming adjoint, M_j
+// (after its first token, multiplied by that token's exp(Delta A)), and its
+// sum of Delta: the reverse counterpart of the forward aggregates.  Only C,
+// dy and Delta enter (no state).
+template <typename TIO, int NS, bool STRUCT>
+__device__ __forceinline__ void bwd_aggregate_item(const BwdArgs<TIO>& a, int j, int64_t stream, int64_t b,
+                                                   int64_t d, bool active, int lane, const float (&An)[NS]) {
+  const int64_t streams = a.batch * a.groups_d;
+  const int T = a.tile;
+  const int64_t t_lo = (int64_t)j * a.super_tiles * T;
+  const int64_t t_hi = (j == a.supers - 1) ? a.len : (int64_t)(j + 1) * a.super_tiles * T;
+  float mu[NS];
+#pragma unroll
+  for (int n = 0; n < NS; ++n) mu[n] = 0.0f;
+  float sd = 0.0f;
+  for (int64_t t = t_hi - 1; t >= t_lo; --t) {
+    const int64_t tok = b * a.len + t;
+    const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+    const float gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
+    float cv[NS], q[NS];
+    load_row<TIO, NS>(a.C + tok * NS, cv, a.vec_rows);
+    decays<NS, STRUCT>(dt, An, q);
+    sd += dt;
+#pragma unroll
+    for (int n = 0; n < NS; ++n) mu[n] = (1.0f + q[n]) * fmaf(cv[n], gy, mu[n]);
+  }
+  const size_t base = ((size_t)j * streams + stream) * 32 + lane;
+  a.agg_sd[base] = sd;
+#pragma unroll
+  for (int n = 0; n < NS; ++n) a.agg_mu[base * NS + n] = mu[n];
+}
+
 template <typename TIO, int NS>
 __global__ void __launch_bounds__(kBwdWarps * 32)
 scan_backward_aggregate_kernel(const BwdArgs<TIO> a) {
@@ -138,47 +191,133 @@ scan_backward_aggregate_kernel(const BwdArgs<TIO> a) {
   const int64_t b = stream / a.groups_d;
   const int64_t d = (stream - b * a.groups_d) * 32 + lane;
   const bool active = d < a.channels;
-  const int T = a.tile;
-  const int64_t ntiles = (a.len + T - 1) / T;
-  const int64_t t_lo = (int64_t)j * a.super_tiles * T;
-  const int64_t t_hi = (j == a.supers - 1) ? a.len : (int64_t)(j + 1) * a.super_tiles * T;
-  (void)ntiles;
-  float An[NS], mu[NS];
+  float An[NS];
 #pragma unroll
-  for (int n = 0; n < NS; ++n) {
-    An[n] = active ? __ldg(a.A + d * NS + n) : -1.0f;
-    mu[n] = 0.0f;
-  }
-  float sd = 0.0f;
-  for (int64_t t = t_hi - 1; t >= t_lo; --t) {
-    const int64_t tok = b * a.len + t;
-    const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
-    const float gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
-    float cv[NS];
-    load_row<TIO, NS>(a.C + tok * NS, cv, a.vec_rows);
-    sd += dt;
-#pragma unroll
-    for (int n = 0; n < NS; ++n) mu[n] = (1.0f + expm1_small(dt * An[n])) * fmaf(cv[n], gy, mu[n]);
-  }
-  const size_t base = ((size_t)j * streams + stream) * 32 + lane;
-  a.agg_sd[base] = sd;
-#pragma unroll
-  for (int n = 0; n < NS; ++n) a.agg_mu[base * NS + n] = mu[n];
+  for (int n = 0; n < NS; ++n) An[n] = active ? __ldg(a.A + d * NS + n) : -(float)(n + 1);
+  if (group_structured<NS>(An)) bwd_aggregate_item<TIO, NS, true>(a, j, stream, b, d, active, lane, An);
+  else bwd_aggregate_item<TIO, NS, false>(a, j, stream, b, d, active, lane, An);
 }
 
+// One work item: super-chunk j of one stream, tiles in reverse.
+template <typename TIO, int NS, bool STRUCT>
+__device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t stream, int64_t b, int64_t d,
+                                         bool active, int lane, const float (&An)[NS], float* S) {
+  const int64_t streams = a.batch * a.groups_d;
+  const int T = a.tile;
+  const int64_t ntiles = (a.len + T - 1) / T;
+  float iA[NS], lam[NS], dA[NS];
+#pragma unroll
+  for (int n = 0; n < NS; ++n) {
+    iA[n] = 1.0f / An[n];
+    lam[n] = (active && a.dh_final) ? a.dh_final[(b * a.channels + d) * NS + n] : 0.0f;
+    dA[n] = 0.0f;
+  }
+  // the adjoint entering super-chunk j from the later ones:
+  //   mu <- M_k + exp(A sumDelta_k) mu,  k = S-1 .. j+1,  mu_S = d h_final
+  for (int k = a.supers - 1; k > j; --k) {
+    const size_t base = ((size_t)k * streams + stream) * 32 + lane;
+    const float sdk = a.agg_sd[base];
+#pragma unroll
+    for (int n = 0; n < NS; ++n) lam[n] = fmaf(expf(An[n] * sdk), lam[n], a.agg_mu[base * NS + n]);
+  }
+  const float Dd = (active && a.D) ? __ldg(a.D + d) : 0.0f;
+  float dD = 0.0f;
+
+  const int64_t tile_lo = (int64_t)j * a.super_tiles;
+  const int64_t tile_hi = (j == a.supers - 1) ? ntiles : tile_lo + a.super_tiles;
+  for (int64_t tile = tile_hi - 1; tile >= tile_lo; --tile) {
+    const int64_t t0 = tile * T;
+    const int rows = (int)(a.len - t0 < (int64_t)T ? a.len - t0 : (int64_t)T);
+    const float* ck = a.ckpt + ((b * ntiles + tile) * a.channels + (active ? d : 0)) * NS;
+    // forward over the tile: S[k] = h after token t0 + k
+    float h[NS];
+#pragma unroll
+    for (int n = 0; n < NS; ++n) h[n] = active ? ck[n] : 0.0f;
+    for (int k = 0; k < rows; ++k) {
+      const int64_t tok = b * a.len + t0 + k;
+      const float x = active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
+      const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+      float bv[NS], q[NS];
+      load_row<TIO, NS>(a.B + tok * NS, bv, a.vec_rows);
+      decays<NS, STRUCT>(dt, An, q);
+#pragma unroll
+      for (int n = 0; n < NS; ++n) h[n] = fmaf(1.0f + q[n], h[n], q[n] * iA[n] * bv[n] * x);
+#pragma unroll
+      for (int n = 0; n < NS; n += 4)
+        *reinterpret_cast<float4*>(S + (size_t)k * 32 * NS + n) = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
+    }
+    // reverse over the tile; h holds h_t, hp is read back as h_{t-1}
+    for (int k = rows - 1; k >= 0; --k) {
+      const int64_t tok = b * a.len + t0 + k;
+      float hp[NS];
+      if (k > 0) {
+#pragma unroll
+        for (int n = 0; n < NS; n += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(S + (size_t)(k - 1) * 32 * NS + n);
+          hp[n] = v.x; hp[n + 1] = v.y; hp[n + 2] = v.z; hp[n + 3] = v.w;
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < NS; ++n) hp[n] = active ? ck[n] : 0.0f;
+      }
+      const float x = active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
+      const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+      const float gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
+      float du = Dd * gy, ddt = 0.0f;
+      dD = fmaf(gy, x, dD);
+      float bv[NS], cv[NS], q[NS];
+      load_row<TIO, NS>(a.B + tok * NS, bv, a.vec_rows);
+      load_row<TIO, NS>(a.C + tok * NS, cv, a.vec_rows);
+      decays<NS, STRUCT>(dt, An, q);
+      float red[32];
+#pragma unroll
+      for (int n = 0; n < NS; ++n) {
+        const float r = 1.0f + q[n];
+        const float bx = bv[n] * x;
+        const float qa = q[n] * iA[n];
+        red[NS + n] = gy * h[n];                      // dC_{t,n} part: dy_t h_t
+        lam[n] = fmaf(cv[n], gy, lam[n]);
+        du = fmaf(lam[n], qa * bv[n], du);
+        ddt = fmaf(lam[n] * r, fmaf(An[n], hp[n], bx), ddt);
+        // d h_t / d A_n = Delta r (h_{t-1} + B x / A_n) - q B x / A_n^2
+        dA[n] = fmaf(lam[n], fmaf(dt * r, fmaf(bx, iA[n], hp[n]), -qa * iA[n] * bx), dA[n]);
+        red[n] = lam[n] * x * qa;                     // dB_{t,n} part
+        lam[n] *= r;
+        h[n] = hp[n];
+      }
+#pragma unroll
+      for (int n = 2 * NS; n < 32; ++n) red[n] = 0.0f;
+      if (active) {
+        a.du[tok * a.channels + d] = from_f32<TIO>(du);
+        a.ddelta[tok * a.channels + d] = from_f32<TIO>(ddt);
+      }
+      const float s = reduce_scatter32(red, lane);
+      if (lane < NS) atomicAdd(a.dB + tok * NS + lane, s);
+      else if (lane < 2 * NS) atomicAdd(a.dC + tok * NS + (lane - NS), s);
+    }
+  }
+  if (active) {
+#pragma unroll
+    for (int n = 0; n < NS; ++n) atomicAdd(a.dA + d * NS + n, dA[n]);
+    if (a.dD) atomicAdd(a.dD + d, dD);
+    if (a.dh0 && j == 0) {
+#pragma unroll
+      for (int n = 0; n < NS; ++n) a.dh0[(b * a.channels + d) * NS + n] = lam[n];
+    }
+  }
+}
+
+// at least three CTAs per SM: the occupancy is worth a few spilled registers
 template <typename TIO, int NS>
-__global__ void __launch_bounds__(kBwdWarps * 32)
+__global__ void __launch_bounds__(kBwdWarps * 32, 3)
 scan_backward_kernel(const BwdArgs<TIO> a) {
   static_assert(2 * NS <= 32, "dB and dC of a token are reduced in one 32-lane pass");
-  griddep_wait();  // the checkpoints come from the previous kernel of the stream
+  griddep_wait();  // the aggregates and checkpoints come from the previous kernels of the stream
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t wid = (int64_t)blockIdx.x * kBwdWarps + warp;
   const int64_t nwarps = (int64_t)gridDim.x * kBwdWarps;
   const int64_t streams = a.batch * a.groups_d;
-  const int T = a.tile;
-  const int64_t ntiles = (a.len + T - 1) / T;
-  float* S = a.scratch + (size_t)wid * (size_t)T * 32 * NS + (size_t)lane * NS;  // + k * 32 * NS
-
+  float* S = a.scratch + (size_t)wid * (size_t)a.tile * 32 * NS + (size_t)lane * NS;  // + k * 32 * NS
   // work item = (super-chunk j, stream), the later super-chunks first
   for (int64_t item = wid; item < (int64_t)a.supers * streams; item += nwarps) {
     const int j = a.supers - 1 - (int)(item / streams);
@@ -186,111 +325,11 @@ scan_backward_kernel(const BwdArgs<TIO> a) {
     const int64_t b = stream / a.groups_d;
     const int64_t d = (stream - b * a.groups_d) * 32 + lane;
     const bool active = d < a.channels;
-    float An[NS], iA[NS], lam[NS], dA[NS];
+    float An[NS];
 #pragma unroll
-    for (int n = 0; n < NS; ++n) {
-      An[n] = active ? __ldg(a.A + d * NS + n) : -1.0f;
-      iA[n] = 1.0f / An[n];
-      lam[n] = (active && a.dh_final) ? a.dh_final[(b * a.channels + d) * NS + n] : 0.0f;
-      dA[n] = 0.0f;
-    }
-    // the adjoint entering super-chunk j from the later ones:
-    //   mu <- M_k + exp(A sumDelta_k) mu,  k = S-1 .. j+1,  mu_S = d h_final
-    for (int k = a.supers - 1; k > j; --k) {
-      const size_t base = ((size_t)k * streams + stream) * 32 + lane;
-      const float sdk = a.agg_sd[base];
-#pragma unroll
-      for (int n = 0; n < NS; ++n) lam[n] = fmaf(expf(An[n] * sdk), lam[n], a.agg_mu[base * NS + n]);
-    }
-    const float Dd = (active && a.D) ? __ldg(a.D + d) : 0.0f;
-    float dD = 0.0f;
-
-    const int64_t tile_lo = (int64_t)j * a.super_tiles;
-    const int64_t tile_hi = (j == a.supers - 1) ? ntiles : tile_lo + a.super_tiles;
-    for (int64_t tile = tile_hi - 1; tile >= tile_lo; --tile) {
-      const int64_t t0 = tile * T;
-      const int rows = (int)(a.len - t0 < (int64_t)T ? a.len - t0 : (int64_t)T);
-      const float* ck = a.ckpt + ((b * ntiles + tile) * a.channels + (active ? d : 0)) * NS;
-      // forward over the tile: S[k] = h after token t0 + k
-      float h[NS];
-#pragma unroll
-      for (int n = 0; n < NS; ++n) h[n] = active ? ck[n] : 0.0f;
-      for (int k = 0; k < rows; ++k) {
-        const int64_t tok = b * a.len + t0 + k;
-        const float x = active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
-        const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
-        float bv[NS];
-        load_row<TIO, NS>(a.B + tok * NS, bv, a.vec_rows);
-#pragma unroll
-        for (int n = 0; n < NS; ++n) {
-          const float q = expm1_small(dt * An[n]);
-          h[n] = fmaf(1.0f + q, h[n], q * iA[n] * bv[n] * x);
-        }
-#pragma unroll
-        for (int n = 0; n < NS; n += 4)
-          *reinterpret_cast<float4*>(S + (size_t)k * 32 * NS + n) = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
-      }
-      // reverse over the tile; h holds h_t, hp is read back as h_{t-1}
-      for (int k = rows - 1; k >= 0; --k) {
-        const int64_t tok = b * a.len + t0 + k;
-        float hp[NS];
-        if (k > 0) {
-#pragma unroll
-          for (int n = 0; n < NS; n += 4) {
-            const float4 v = *reinterpret_cast<const float4*>(S + (size_t)(k - 1) * 32 * NS + n);
-            hp[n] = v.x; hp[n + 1] = v.y; hp[n + 2] = v.z; hp[n + 3] = v.w;
-          }
-        } else {
-#pragma unroll
-          for (int n = 0; n < NS; ++n) hp[n] = active ? ck[n] : 0.0f;
-        }
-        const float x = active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
-        const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
-        const float gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
-        float du = Dd * gy, ddt = 0.0f;
-        dD = fmaf(gy, x, dD);
-        float bv[NS], cv[NS];
-        load_row<TIO, NS>(a.B + tok * NS, bv, a.vec_rows);
-        load_row<TIO, NS>(a.C + tok * NS, cv, a.vec_rows);
-        const float inv_dt2 = active ? 1.0f / (dt * dt) : 0.0f;  // psi's closed form: 1/z^2 = 1/(dt^2 A^2)
-        float red[32];
-#pragma unroll
-        for (int n = 0; n < NS; ++n) {
-          const float bn = bv[n];
-          const float z = dt * An[n];
-          const float q = expm1_small(z);
-          const float r = 1.0f + q;
-          const float qa = q * iA[n];
-          red[NS + n] = gy * h[n];                      // dC_{t,n} part: dy_t h_t
-          lam[n] = fmaf(cv[n], gy, lam[n]);
-          du = fmaf(lam[n], qa * bn, du);
-          ddt = fmaf(lam[n] * r, fmaf(An[n], hp[n], bn * x), ddt);
-          const float ps = psi_f(z, q, inv_dt2 * iA[n] * iA[n]);
-          dA[n] = fmaf(lam[n], fmaf(dt * r, hp[n], x * bn * dt * dt * ps), dA[n]);
-          red[n] = lam[n] * x * qa;                     // dB_{t,n} part
-          lam[n] *= r;
-          h[n] = hp[n];
-        }
-#pragma unroll
-        for (int n = 2 * NS; n < 32; ++n) red[n] = 0.0f;
-        if (active) {
-          a.du[tok * a.channels + d] = from_f32<TIO>(du);
-          a.ddelta[tok * a.channels + d] = from_f32<TIO>(ddt);
-        }
-        const float s = reduce_scatter32(red, lane);
-        if (lane < NS) atomicAdd(a.dB + tok * NS + lane, s);
-        else if (lane < 2 * NS) atomicAdd(a.dC + tok * NS + (lane - NS), s);
-      }
-    }
-    if (active) {
-#pragma unroll
-      for (int n = 0; n < NS; ++n) atomicAdd(a.dA + d * NS + n, dA[n]);
-      if (a.dD) atomicAdd(a.dD + d, dD);
-      if (a.dh0 && j == 0) {
-#pragma unroll
-        for (int n = 0; n < NS; ++n) a.dh0[(b * a.channels + d) * NS + n] = lam[n];
-      }
-    }
+    for (int n = 0; n < NS; ++n) An[n] = active ? __ldg(a.A + d * NS + n) : -(float)(n + 1);
+    if (group_structured<NS>(An)) bwd_item<TIO, NS, true>(a, j, stream, b, d, active, lane, An, S);
+    else bwd_item<TIO, NS, false>(a, j, stream, b, d, active, lane, An, S);
   }
 }
 

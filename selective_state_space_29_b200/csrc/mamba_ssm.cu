@@ -245,7 +245,7 @@ int noalloc_scratch_address(void** out) {
 
 // Enqueue one scan with the given plan on caller-provided scratch (laid out
 // by scratch_layout): pre-pass, [aggregate pass, combine,] main pass.
-template <typename TIO, int NS, int METHOD>
+template <typename TIO, int NS, int METHOD, bool CKPT = false>
 int launch_scan_on(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
                    const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
                    unsigned flags, int dtype, cudaStream_t stream, const Plan& pl, int sms,
@@ -294,7 +294,7 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
 
   constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES, kScanConsumers>();
   static_assert(smem <= 232448, "scan CTA exceeds the shared memory of an SM");
-  auto kern = scan_chunks_kernel<TIO, NS, kScanConsumers, TILE, STAGES, METHOD>;
+  auto kern = scan_chunks_kernel<TIO, NS, kScanConsumers, TILE, STAGES, METHOD, CKPT>;
   {
     // the dynamic shared-memory limit is a per-device attribute of the kernel
     static std::mutex mu_attr;
@@ -373,9 +373,12 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   else if (flags & MAMBA_SCAN_TRAPEZOID)
     status = launch_scan_on<TIO, NS, kTrapezoid>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels,
                                                  flags, dtype, stream, pl, sms, scratch);
+  else if (ckpt)
+    status = launch_scan_on<TIO, NS, kZOH, true>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels,
+                                                 flags, dtype, stream, pl, sms, scratch, ckpt);
   else
     status = launch_scan_on<TIO, NS, kZOH>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags,
-                                           dtype, stream, pl, sms, scratch, ckpt);
+                                           dtype, stream, pl, sms, scratch);
   if (!noalloc && cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) return MAMBA_ERR_CUDA;
   return status;
 }

@@ -73,7 +73,7 @@ struct ScanParams {
   const float* h0;          // nullable: initial state [b][d][n]
   void* y;                  // nullable: no output (checkpoint-only runs for the backward)
   float* final_state;       // nullable
-  float* ckpt;              // nullable: [batch][ceil(len/TILE)][channels][N] state before every tile
+  float* ckpt;              // [batch][ceil(len/TILE)][channels][N] state before every tile (CKPT kernels)
   // scratch (stream-ordered; the pre-pass zeroes counters and done)
   int* counters;            // [0] job ticket, [1] abort flag
   int* done;                // [S*G] chunks completed per main stream
@@ -666,7 +666,7 @@ __device__ void producer_loop(const ScanParams& p, WarpSmem<TIO, NS, TILE, STAGE
 // Lane l serves channel d0 + l and all its states.  STRUCT: A[d,n] = (n+1)
 // A[d,0] on every lane (see decay_chain).  Tile 0 is already in slot s0;
 // cm = {A[d,0], 1/A[d,0], D[d], structured}.
-template <typename TIO, int NS, int TILE, int STAGES, bool STRUCT, bool FULL, int METHOD = kZOH>
+template <typename TIO, int NS, int TILE, int STAGES, bool STRUCT, bool FULL, int METHOD = kZOH, bool CKPT = false>
 __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, const Job& jb, int s0,
                                         const float4 cm) {
   static_assert(!STRUCT || METHOD == kZOH, "the structured-A path is zero-order hold only");
@@ -751,7 +751,7 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, con
   for (int it = 0; it < jb.ntiles; ++it) {
     const int64_t tt0 = jb.t0 + (int64_t)it * TILE;
     const int rows = (int)(jb.t1 - tt0 < (int64_t)TILE ? jb.t1 - tt0 : (int64_t)TILE);
-    if (FULL && p.ckpt && active) {
+    if (CKPT && FULL && active) {
       // the state before this tile, unscaled (tiles start at multiples of TILE)
       float* ck = p.ckpt + (((int64_t)jb.b * ((p.len + TILE - 1) / TILE) + tt0 / TILE) * p.channels + d) * NS;
 #pragma unroll
@@ -817,9 +817,10 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES>& cx, con
 // the persistent chunked scan kernel: CW consumer warps (one job at a time
 // each) and one producer warp (index CW) per CTA; METHOD is the
 // discretisation (zero-order hold, or the general-A path with exponential
-// Euler or the trapezoid rule)
+// Euler or the trapezoid rule); CKPT kernels also leave the state before
+// every tile in p.ckpt (for the backward)
 // ---------------------------------------------------------------------------
-template <typename TIO, int NS, int CW, int TILE, int STAGES, int METHOD>
+template <typename TIO, int NS, int CW, int TILE, int STAGES, int METHOD, bool CKPT>
 __global__ void __launch_bounds__((CW + 1) * 32, 1)
 scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__ CUtensorMap map_u,
                    const __grid_constant__ CUtensorMap map_dl, const __grid_constant__ CUtensorMap map_b,
@@ -881,11 +882,11 @@ scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__
       ok = full_mode ? run_job<TIO, NS, TILE, STAGES, false, true, METHOD>(cx, jb, s0, cm)
                      : run_job<TIO, NS, TILE, STAGES, false, false, METHOD>(cx, jb, s0, cm);
     else if (structured)
-      ok = full_mode ? run_job<TIO, NS, TILE, STAGES, true, true>(cx, jb, s0, cm)
-                     : run_job<TIO, NS, TILE, STAGES, true, false>(cx, jb, s0, cm);
+      ok = full_mode ? run_job<TIO, NS, TILE, STAGES, true, true, kZOH, CKPT>(cx, jb, s0, cm)
+                     : run_job<TIO, NS, TILE, STAGES, true, false, kZOH, CKPT>(cx, jb, s0, cm);
     else
-      ok = full_mode ? run_job<TIO, NS, TILE, STAGES, false, true>(cx, jb, s0, cm)
-                     : run_job<TIO, NS, TILE, STAGES, false, false>(cx, jb, s0, cm);
+      ok = full_mode ? run_job<TIO, NS, TILE, STAGES, false, true, kZOH, CKPT>(cx, jb, s0, cm)
+                     : run_job<TIO, NS, TILE, STAGES, false, false, kZOH, CKPT>(cx, jb, s0, cm);
     if (!ok) break;
   }
   __syncwarp();
