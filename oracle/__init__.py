@@ -115,6 +115,41 @@ class Oracle:
             raise RuntimeError(f"oracle_state_update failed ({rc})")
         return y
 
+    # --- Mamba-2's restricted form (state space duality) -----------------
+    @staticmethod
+    def _ssd_channel_head(channels: int, headdim: int) -> np.ndarray:
+        """Head of every channel: channels are grouped into heads of
+        `headdim` consecutive channels, so channel d belongs to head d // headdim."""
+        return np.arange(channels) // headdim
+
+    def ssd_scan(self, x, dt, A_head, B, C, D=None, h0=None, headdim=64, want_y=True, nthreads=0, method=0):
+        """The scan of Mamba-2's restricted SSM.
+
+        The Mamba-3 page (bitig.info), "Karmaşık Değerli Durum Güncellemesi":
+        Mamba-2 reduces the state transition to real scalars; "Mamba SSM
+        Nedir? Transformer Alternatifi Rehberi (2026)", "Mamba-2 ve Güncel
+        Gelişmeler", and "Albert Gu: Mamba'nın Mucidi ...", "Mamba-2 (2024)":
+        under that restriction the SSM equals a masked attention-like form
+        (state space duality).  Read plainly: head h has one negative
+        scalar a_h, every channel of the head uses A = a_h * I over its
+        states, and one step dt[b, t, h] is shared by the head's channels.
+        Everything else (discretisation, recurrence, output, skip term) is the
+        selective scan's.  So the definition is the scan oracle on inputs
+        broadcast to channels: A[d, n] = a_{h(d)}, delta[b, t, d] = dt[b, t, h(d)].
+
+        x: (batch, len, heads*headdim); dt: (batch, len, heads); A_head:
+        (heads,); B, C: (batch, len, nstate); D: (channels,) or None; h0:
+        (batch, channels, nstate) or None.  Returns (y, h_final) in float64."""
+        x, dt, A_head, B = map(self._f64, (x, dt, A_head, B))
+        batch, length, channels = x.shape
+        heads = A_head.shape[0]
+        assert channels == heads * headdim and dt.shape == (batch, length, heads)
+        nstate = B.shape[2]
+        head_of = self._ssd_channel_head(channels, headdim)
+        delta = np.ascontiguousarray(dt[:, :, head_of])
+        A = np.ascontiguousarray(np.repeat(A_head[head_of][:, None], nstate, axis=1))
+        return self.scan(x, delta, A, B, C, D, h0, want_y=want_y, nthreads=nthreads, method=method)
+
     def max_threads(self) -> int:
         return int(self._lib.oracle_max_threads())
 
@@ -136,3 +171,7 @@ def scan(*args, **kwargs):
 
 def state_update(*args, **kwargs):
     return get().state_update(*args, **kwargs)
+
+
+def ssd_scan(*args, **kwargs):
+    return get().ssd_scan(*args, **kwargs)

@@ -13,6 +13,8 @@ Workloads (one scan or one decode chain each):
   long_bf16    batch 1, channels 2048, state 16, length 1,048,576,  bf16, delta in [1e-4, 1e-1]
   decode_bf16  256 sequences x 5120 channels x 16 states, 1000 single-token steps,
                fp32 state, bf16 x / delta / B / C / y
+  ssd_mid_bf16 / ssd_long_bf16  the mid and long shapes as Mamba-2 heads of 64
+               channels (48 and 32 heads): one scalar A and one step per head
 
 Distributions: x ~ N(0,1); delta log-uniform in [lo, hi] (uniform exponent);
 B, C ~ N(0,1) per (batch, token, state), shared by all channels; D ~ N(0,1) per
@@ -82,11 +84,48 @@ class DecodeWorkload:
         return dataclasses.replace(self, **kw)
 
 
+@dataclasses.dataclass(frozen=True)
+class SsdWorkload:
+    """Mamba-2's restricted scan: heads of `headdim` channels, one scalar A
+    and one step dt per (batch, token, head)."""
+    name: str
+    batch: int
+    length: int
+    heads: int
+    headdim: int
+    nstate: int
+    dtype: str = "bf16"        # dtype of x, dt, B, C and y
+    delta_lo: float = 1e-3
+    delta_hi: float = 1e-1
+    final_state: bool = True
+    seed: int = 34
+
+    @property
+    def torch_dtype(self):
+        return _DTYPES[self.dtype]
+
+    @property
+    def channels(self) -> int:
+        return self.heads * self.headdim
+
+    @property
+    def token_channels(self) -> int:
+        return self.batch * self.length * self.channels
+
+    def with_(self, **kw) -> "SsdWorkload":
+        return dataclasses.replace(self, **kw)
+
+
 SCAN_WORKLOADS = {
     "tiny_f32": ScanWorkload("tiny_f32", 1, 256, 64, 16, "f32", a_mode="s4d", seed=29),
     "mid_bf16": ScanWorkload("mid_bf16", 8, 2048, 3072, 16, "bf16", seed=30),
     "large_bf16": ScanWorkload("large_bf16", 4, 8192, 5120, 16, "bf16", seed=31),
     "long_bf16": ScanWorkload("long_bf16", 1, 1 << 20, 2048, 16, "bf16", delta_lo=1e-4, seed=32),
+}
+# the mid and long scan shapes with their channels grouped into heads of 64
+SSD_WORKLOADS = {
+    "ssd_mid_bf16": SsdWorkload("ssd_mid_bf16", 8, 2048, 48, 64, 16, seed=34),
+    "ssd_long_bf16": SsdWorkload("ssd_long_bf16", 1, 1 << 20, 32, 64, 16, delta_lo=1e-4, seed=35),
 }
 DECODE_WORKLOADS = {
     "decode_bf16": DecodeWorkload("decode_bf16", 256, 5120, 16, 1000, seed=33),
@@ -205,3 +244,30 @@ def decode_chain_inputs(w: DecodeWorkload, device="cpu", seed: int | None = None
     (steps, batch, nstate)."""
     steps = [decode_step_inputs(w, i, device, seed) for i in range(w.steps)]
     return {k: torch.stack([st[k] for st in steps]) for k in ("x", "delta", "B", "C")}
+
+
+def ssd_inputs(w: SsdWorkload, device="cpu", seed: int | None = None) -> dict:
+    """x (batch, len, heads*headdim); dt (batch, len, heads); B, C (batch,
+    len, nstate) in the workload dtype; A (heads,) and D (channels,) fp32.
+    A per head is log-uniform in [-16, -1] (no distribution is given for a
+    scalar A; this spans the decay rates of the per-state A of the scan
+    workloads, -(n+1) for n < 16)."""
+    s = w.seed if seed is None else seed
+    dt_ = w.torch_dtype
+    shp_x = (w.batch, w.length, w.channels)
+    shp_dt = (w.batch, w.length, w.heads)
+    shp_bc = (w.batch, w.length, w.nstate)
+    if w.length == 0 or w.batch == 0:
+        x = torch.empty(shp_x, dtype=dt_, device=device)
+        dt = torch.empty(shp_dt, dtype=dt_, device=device)
+        B = torch.empty(shp_bc, dtype=dt_, device=device)
+        C = torch.empty(shp_bc, dtype=dt_, device=device)
+    else:
+        x = _normal(shp_x, _gen(device, s, 1), device, dt_)
+        dt = _log_uniform(shp_dt, _gen(device, s, 2), device, dt_, w.delta_lo, w.delta_hi)
+        B = _normal(shp_bc, _gen(device, s, 3), device, dt_)
+        C = _normal(shp_bc, _gen(device, s, 4), device, dt_)
+    A = -torch.exp(torch.empty((w.heads,), device=device, dtype=torch.float32)
+                   .uniform_(0.0, math.log(16.0), generator=_gen(device, s, 5)))
+    D = torch.randn((w.channels,), generator=_gen(device, s, 6), device=device, dtype=torch.float32)
+    return {"x": x, "dt": dt, "A": A, "B": B, "C": C, "D": D}
