@@ -41,6 +41,7 @@ if ROOT not in sys.path:
 METRIC = "selective-scan token·channels/s and achieved HBM GB/s (% of B200 peak)"
 UNIT = "token·channels/s"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 FMA_LANES_PER_SM = 128          # FP32 FMA results per clock per SM (sm_100)
 FLOP_PER_STATE_STEP = 8         # 4 FMA per state and token: decay, input term, state update, output
 FLOP_PER_TOKEN_CHANNEL = 4      # skip term and output scaling
@@ -59,6 +60,9 @@ def parse_args():
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the timings of the scan's options (general A, other discretisations, state counts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-ssd", action="store_true", help="skip Mamba-2's scalar-A scan (state space duality) leg")
+    ap.add_argument("--only-ssd", action="store_true",
+                    help="run only the scalar-A scan leg (steps/warmup as given) and print its object")
     ap.add_argument("--length-sweep", action="store_true",
                     help="instead of the benchmark line: ns per token-channel of the long-context workload's "
                          "generator (1 x L x 2048, bf16) for L = 2^14 .. 2^20 (linear scaling in length)")
@@ -79,6 +83,7 @@ def measured_peaks():
 KERNEL_SOURCES = {
     "scan_chunks_kernel": ("common.cuh", "scan.cuh"),
     "state_update_kernel": ("common.cuh", "scan.cuh", "decode.cuh"),
+    "ssd_chunk_kernel": ("common.cuh", "ssd.cuh"),
 }
 
 
@@ -451,6 +456,10 @@ def run_ours(args):
     if not args.no_variants:
         out["variants"] = run_variants(w, dev, stream, dist, world, rank)
 
+    # Mamba-2's scalar-A scan in its chunked tensor-core form, on the same shape
+    if not args.no_ssd:
+        out["ssd"] = run_ssd(args, dev, stream, dist, world, rank, hbm_peak, hbm_src, peaks)
+
     # decode: 1000 single-token steps on 256 x 5120 x 16 states
     if not args.no_decode:
         out["decode"] = run_decode(args, dev, stream, dist, world, rank, hbm_peak, hbm_src)
@@ -532,6 +541,86 @@ def run_decode(args, dev, stream, dist, world, rank, hbm_peak, hbm_src):
                          "algorithmic_bytes_per_launch": nb, "peak_source": hbm_src,
                          "note": "the 84 MB state fits in L2; DRAM traffic per launch is in the ncu summary"},
             "gpu_launches": steps}
+
+
+def ssd_bytes(w) -> int:
+    """Algorithmic bytes of one scalar-A scan call: x read, y written, dt, B,
+    C, the final state, A and D."""
+    es = 2
+    return (w.batch * w.length * w.channels * es * 2 + w.batch * w.length * w.heads * es
+            + 2 * w.batch * w.length * w.nstate * es + w.batch * w.channels * w.nstate * 4
+            + w.heads * 4 + w.channels * 4)
+
+
+SSD_CHUNK = 64    # tokens per chunk of mamba_ssd_scan
+
+
+def ssd_mma_flops(w) -> int:
+    """Tensor-core FLOPs of the chunked form per call: per chunk of Q tokens
+    and head, C S_in (Q x N x 64), the causal 16 x 16 blocks of C B^T (nb
+    blocks of 16 x N x 16) and of M X (nb of 16 x 16 x 64), and B_w^T X
+    (N x Q x 64); nb = k(k+1)/2 with k = Q/16."""
+    q, p, n = SSD_CHUNK, 64, w.nstate
+    nb = (q // 16) * (q // 16 + 1) // 2
+    per_chunk = 2 * (q * n * p + nb * 16 * n * 16 + nb * 16 * 16 * p + n * q * p)
+    chunks = -(-w.length // q)
+    return w.batch * w.heads * chunks * per_chunk
+
+
+def run_ssd(args, dev, stream, dist, world, rank, hbm_peak, hbm_src, peaks):
+    """Mamba-2's scalar-A scan (mamba_ssd_scan) on the mid shape as 48 heads
+    of 64 channels (device-timed per call, K calls), and on the long shape."""
+    import torch
+
+    from selective_state_space_29_b200 import mamba_ssm as m
+    from selective_state_space_29_b200 import workloads as wl
+
+    lib = m.library()
+    sh = stream.cuda_stream
+    res = {}
+    for name, K in (("ssd_mid_bf16", max(args.steps, 3)), ("ssd_long_bf16", 3)):
+        if args.only_ssd and name != "ssd_mid_bf16":
+            continue
+        w = wl.SSD_WORKLOADS[name]
+        inp = wl.ssd_inputs(w, dev, seed=rank_seed(w.seed, rank))
+        y = torch.empty_like(inp["x"])
+        hf = torch.empty((w.batch, w.channels, w.nstate), device=dev, dtype=torch.float32)
+        ptrs = [inp[k].data_ptr() for k in ("x", "dt", "A", "B", "C", "D")] + [None, y.data_ptr(), hf.data_ptr()]
+
+        def step():
+            st = lib.mamba_ssd_scan(*ptrs, w.batch, w.length, w.heads, w.headdim, w.nstate, 0, 0, m.MAMBA_BF16, sh)
+            if st != 0:
+                raise m.MambaError(st, "mamba_ssd_scan")
+
+        for _ in range(max(args.warmup, 3)):
+            step()
+        torch.cuda.synchronize()
+        barrier(dist, world)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for i in range(K):
+            ev[i][0].record(stream)
+            step()
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+        call_ms = max_over_ranks(dist, world, statistics.mean(a.elapsed_time(b) for a, b in ev))
+        nb, fl = ssd_bytes(w), ssd_mma_flops(w)
+        ach = nb / (call_ms * 1e-3) / 1e9
+        tpk = float(peaks.get("bf16_tflops", FALLBACK_BF16_TFLOPS))
+        tfl = fl / (call_ms * 1e-3) / 1e12
+        res[name] = {
+            "workload": f"{w.name}: batch {w.batch}, len {w.length}, {w.heads} heads x {w.headdim} channels, "
+                        f"state {w.nstate}, bf16 I/O, fp32 state",
+            "ms_per_call": round(call_ms, 5), "calls": K,
+            "token_channels_per_s": world * w.token_channels / (call_ms * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                         "frac": round(ach / hbm_peak, 4), "traffic": profiled_traffic("ssd_chunk_kernel", w.name),
+                         "algorithmic_bytes_per_launch": nb, "peak_source": hbm_src,
+                         "tensor": {"achieved": round(tfl, 2), "peak": tpk, "unit": "TFLOP/s",
+                                    "frac": round(tfl / tpk, 4), "flop_per_launch": fl,
+                                    "peak_source": "measured bf16" if "bf16_tflops" in peaks else "fallback"}},
+            "l2": f"inputs larger than L2 ({nb / 1e6:.0f} MB per call), no flush"}
+        del inp, y, hf
+    return res
 
 
 def run_variants(w, dev, stream, dist, world, rank, reps: int = 20):
@@ -709,6 +798,19 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.only_ssd:
+        import torch
+        rank, world, local = dist_setup(args.gpus)
+        torch.cuda.set_device(local)
+        dist = init_pg(world, local)
+        peaks = measured_peaks()
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+        res = run_ssd(args, torch.device("cuda", local), torch.cuda.current_stream(), dist, world, rank, hbm,
+                      "measured" if "hbm_gbs" in peaks else "fallback", peaks)
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"ssd": res}), flush=True)
     elif args.length_sweep:
         run_length_sweep(args)
     else:

@@ -111,7 +111,9 @@ typedef enum {
  * staged with TMA when u, delta, B and C are 16-byte aligned and a row of
  * channels is a multiple of 16 bytes, with plain loads otherwise.
  * Scratch: every call allocates and frees stream-ordered scratch on `stream`
- * (cudaMallocAsync / cudaFreeAsync): job counters, the buffer that hands the
+ * (from a memory pool the library creates on the device, which keeps up to
+ * 1 GiB of freed memory for later calls; inside a stream capture, from
+ * cudaMallocAsync, and freed with cudaFreeAsync): job counters, the buffer that hands the
  * state from one time chunk to the next, and, when sequences are split into
  * independent super-chunks, their aggregates (mamba_scan_plan reports the
  * size).  batch == 0 or channels == 0 is a no-op that returns MAMBA_OK.
@@ -268,6 +270,55 @@ int mamba_selective_scan_backward(const void *u, const void *delta, const float 
                                   float *dD, float *d_initial_state,
                                   int64_t batch, int64_t len, int64_t channels, int64_t nstate,
                                   int dtype, mamba_stream_t stream);
+
+/*
+ * Mamba-2's restricted scan in its chunked matrix form (state space duality),
+ * on the tensor cores.
+ *
+ * Defined by: the Mamba-3 page (bitig.info), "Karmaşık Değerli Durum
+ * Güncellemesi" (Mamba-2 reduces the state transition to real scalars), and
+ * "Mamba SSM Nedir? Transformer Alternatifi Rehberi (2026)", "Mamba-2 ve
+ * Güncel Gelişmeler" (with that restriction the SSM equals a masked,
+ * attention-like matrix form).  Channels are grouped into `heads` heads of
+ * `headdim` consecutive channels; head h has one scalar A[h] < 0 and one
+ * step dt[b][t][h] shared by its channels, and every channel d of head h
+ * runs the selective scan with A[d][n] = A[h] for all n and delta[b][t][d]
+ * = dt[b][t][h]:
+ *   h_t = exp(dt A) h_{t-1} + w_t B_t x_t,  y_t = C_t . h_t + D x_t,
+ *   w_t = (exp(dt A) - 1)/A (zero-order hold) or dt (flag MAMBA_SCAN_EULER).
+ * The kernel evaluates it chunk by chunk as matrix products (64-token
+ * chunks; the decay-masked C B^T of a chunk times its x, plus the entering
+ * state), with bf16 operands and fp32 accumulation; the state carried from
+ * chunk to chunk is fp32, its bf16 copy feeds the C . h term.
+ *
+ * Layouts (row-major, contiguous): x, y [batch][len][heads*headdim] bf16;
+ * dt [batch][len][heads] bf16; A [heads] fp32; B, C [batch][len][nstate]
+ * bf16 (shared by all heads); D [heads*headdim] fp32 or NULL;
+ * initial_state / final_state [batch][heads*headdim][nstate] fp32 or NULL
+ * (the selective scan's state layout).  x, B, C and y must be 16-byte
+ * aligned, D 8-byte aligned.  All pointers are caller-owned device memory.
+ *
+ * supers: super-chunks per (batch row, head) run in parallel (0 = chosen
+ * from the shape and the device; a forced value is clamped to the chunk
+ * count).  With more than one, a first kernel computes each super-chunk's
+ * end state from zero (stream-ordered scratch of 4 (64 nstate + 1) bytes per
+ * super-chunk) and the main kernel folds them in.
+ *
+ * Supported: dtype MAMBA_BF16, headdim 64, nstate 16, 32 or 64, flags 0 or
+ * MAMBA_SCAN_EULER (MAMBA_SCAN_GENERAL_A is accepted and has no effect: A
+ * has no state structure here).  Otherwise MAMBA_ERR_UNSUPPORTED
+ * (MAMBA_SCAN_TRAPEZOID, fp32 I/O, other headdim or nstate); malformed
+ * arguments (NULL tensors with len > 0, negative sizes, misalignment,
+ * unknown flags, EULER with TRAPEZOID) give MAMBA_ERR_INVALID_ARG.  len == 0
+ * copies initial_state (or zeros) to final_state.  Asynchronous on `stream`.
+ */
+int mamba_ssd_scan(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                   const float *D, const float *initial_state, void *y, float *final_state,
+                   int64_t batch, int64_t len, int64_t heads, int64_t headdim, int64_t nstate,
+                   int64_t supers, unsigned flags, int dtype, mamba_stream_t stream);
+
+/* 1 if `nstate` is implemented by mamba_ssd_scan. */
+int mamba_ssd_supported_nstate(int64_t nstate);
 
 /* How mamba_selective_scan_ex would split a problem (host-side planning only). */
 typedef struct {

@@ -16,6 +16,7 @@
 #include "backward.cuh"
 #include "decode.cuh"
 #include "scan.cuh"
+#include "ssd.cuh"
 
 namespace mamba {
 
@@ -47,6 +48,43 @@ int current_sms(int* sms) {
   }
   *sms = g_dev[dev].sms;
   return MAMBA_OK;
+}
+
+// --- stream-ordered scratch -------------------------------------------------
+// Scratch comes from a memory pool the library owns on each device, which
+// keeps up to kPoolKeepBytes of freed memory across synchronisations: the
+// device's default pool returns freed memory to the system at every
+// synchronisation, and mapping it again on the next call costs host time
+// during which the GPU waits.  Inside a stream capture the allocation is a
+// plain cudaMallocAsync (a graph memory node).
+constexpr uint64_t kPoolKeepBytes = uint64_t(1) << 30;
+std::mutex g_pool_mu;
+cudaMemPool_t g_pool[64] = {};
+
+cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return cudaErrorUnknown;
+  int dev = 0;
+  if (cs != cudaStreamCaptureStatusNone || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return cudaMallocAsync(p, bytes, stream);
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    if (!g_pool[dev]) {
+      cudaMemPoolProps props = {};
+      props.allocType = cudaMemAllocationTypePinned;
+      props.handleTypes = cudaMemHandleTypeNone;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      cudaMemPool_t np = nullptr;
+      if (cudaMemPoolCreate(&np, &props) != cudaSuccess) return cudaMallocAsync(p, bytes, stream);
+      uint64_t keep = kPoolKeepBytes;
+      cudaMemPoolSetAttribute(np, cudaMemPoolAttrReleaseThreshold, &keep);
+      g_pool[dev] = np;
+    }
+    pool = g_pool[dev];
+  }
+  return cudaMallocFromPoolAsync(p, bytes, pool, stream);
 }
 
 // --- tensor maps through the driver entry point (no link to libcuda) -------
@@ -364,7 +402,7 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
     if (int st = noalloc_scratch_address(&base)) return st;
     scratch = static_cast<unsigned char*>(base);
   } else {
-    if (cudaMallocAsync(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+    if (scratch_alloc(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
   }
   int status;
   if (flags & MAMBA_SCAN_EULER)
@@ -441,7 +479,7 @@ int scan_host_pipelined(const void* u, const void* delta, const float* A, const 
     return status != MAMBA_OK;
   };
   unsigned char* mem = nullptr;
-  if (!fail(cudaMallocAsync(reinterpret_cast<void**>(&mem), total, s0))) {
+  if (!fail(scratch_alloc(reinterpret_cast<void**>(&mem), total, s0))) {
     float* dA = reinterpret_cast<float*>(mem + 2 * per_set);
     float* dD = D ? dA + (size_t)channels * nstate : nullptr;
     fail(cudaMemcpyAsync(dA, A, sizeof(float) * (size_t)channels * nstate, cudaMemcpyHostToDevice, s0));
@@ -500,6 +538,58 @@ __global__ void expire_wait_kernel(uint64_t limit_ns) {
     // nothing ever arrives on `bar`: the bounded wait must run out
     if (!mbar_wait_bounded(&bar, 0, limit_ns)) record_device_error(MAMBA_ERR_TIMEOUT);
   }
+}
+
+// --- Mamba-2's restricted scan (ssd.cuh) ------------------------------------
+// Super-chunks per (batch row, head): one when the (batch row, head) pairs
+// fill at least half of the resident CTA slots, else as many as fit the
+// slots in one wave (each super-chunk but the last costs an extra,
+// state-only pass over its x and B).
+int64_t ssd_supers(int64_t seqs, int64_t chunks, int64_t slots, int64_t requested) {
+  int64_t s = requested > 0 ? requested : (seqs * 2 >= slots ? 1 : std::max<int64_t>(1, slots / seqs));
+  return std::max<int64_t>(1, std::min(s, chunks));
+}
+
+template <int N>
+int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream) {
+  using L = SsdSmem<N>;
+  auto main_k = ssd_chunk_kernel<N, false>;
+  auto agg_k = ssd_chunk_kernel<N, true>;
+  if (cudaFuncSetAttribute(main_k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(agg_k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+    return MAMBA_ERR_CUDA;
+  int sms = 0, per_sm = 0;
+  if (current_sms(&sms) != MAMBA_OK) return MAMBA_ERR_CUDA;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, main_k, kSsdWarps * 32, L::kBytes) != cudaSuccess ||
+      per_sm < 1)
+    return MAMBA_ERR_CUDA;
+  const int64_t seqs = batch * a.heads;
+  const int64_t chunks = (a.len + kSsdQ - 1) / kSsdQ;
+  int64_t S = ssd_supers(seqs, chunks, (int64_t)sms * per_sm, supers_req);
+  const int64_t per = (chunks + S - 1) / S;
+  S = (chunks + per - 1) / per;
+  a.super_len = per * kSsdQ;
+  a.supers = (int)S;
+  if (seqs * S >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+  unsigned char* mem = nullptr;
+  if (S > 1) {
+    const size_t n_agg = (size_t)seqs * (size_t)(S - 1);
+    const size_t st_bytes = n_agg * kSsdP * N * sizeof(float);
+    if (scratch_alloc(reinterpret_cast<void**>(&mem), st_bytes + n_agg * sizeof(float), stream) != cudaSuccess)
+      return MAMBA_ERR_CUDA;
+    a.agg_state = reinterpret_cast<float*>(mem);
+    a.agg_decay = reinterpret_cast<float*>(mem + st_bytes);
+    if (launch_pdl(agg_k, dim3((unsigned)(seqs * (S - 1))), dim3(kSsdWarps * 32), L::kBytes, stream, a) !=
+        cudaSuccess) {
+      cudaFreeAsync(mem, stream);
+      return MAMBA_ERR_CUDA;
+    }
+  }
+  int st = MAMBA_OK;
+  if (launch_pdl(main_k, dim3((unsigned)(seqs * S)), dim3(kSsdWarps * 32), L::kBytes, stream, a) != cudaSuccess)
+    st = MAMBA_ERR_CUDA;
+  if (mem && cudaFreeAsync(mem, stream) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  return st;
 }
 
 }  // namespace
@@ -683,7 +773,7 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
         const size_t mu_bytes = al(sizeof(float) * (size_t)supers * (size_t)streams * 32 * NS);
         const size_t sd_bytes = al(sizeof(float) * (size_t)supers * (size_t)streams * 32);
         unsigned char* mem = nullptr;
-        if (cudaMallocAsync(reinterpret_cast<void**>(&mem), ck_bytes + sc_bytes + mu_bytes + sd_bytes, stream) !=
+        if (scratch_alloc(reinterpret_cast<void**>(&mem), ck_bytes + sc_bytes + mu_bytes + sd_bytes, stream) !=
             cudaSuccess)
           return MAMBA_ERR_CUDA;
         float* ckpt = reinterpret_cast<float*>(mem);
@@ -791,6 +881,61 @@ int mamba_state_update(float* state, const void* x, const void* delta, const flo
     }
     return err == cudaSuccess ? (int)MAMBA_OK : (int)MAMBA_ERR_CUDA;
   });
+}
+
+int mamba_ssd_supported_nstate(int64_t nstate) { return nstate == 16 || nstate == 32 || nstate == 64; }
+
+int mamba_ssd_scan(const void* x, const void* dt, const float* A, const void* B, const void* C, const float* D,
+                   const float* initial_state, void* y, float* final_state, int64_t batch, int64_t len,
+                   int64_t heads, int64_t headdim, int64_t nstate, int64_t supers, unsigned flags, int dtype,
+                   mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || len < 0 || heads < 0 || headdim <= 0 || nstate <= 0 || supers < 0) return MAMBA_ERR_INVALID_ARG;
+  if (flags & ~(MAMBA_SCAN_GENERAL_A | MAMBA_SCAN_EULER | MAMBA_SCAN_TRAPEZOID)) return MAMBA_ERR_INVALID_ARG;
+  if ((flags & MAMBA_SCAN_EULER) && (flags & MAMBA_SCAN_TRAPEZOID)) return MAMBA_ERR_INVALID_ARG;
+  if (flags & MAMBA_SCAN_TRAPEZOID) return MAMBA_ERR_UNSUPPORTED;
+  if (dtype != MAMBA_BF16 || headdim != kSsdP || !mamba_ssd_supported_nstate(nstate)) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || heads == 0) return MAMBA_OK;
+  if (len > 0) {
+    if (!x || !dt || !A || !B || !C || !y) return MAMBA_ERR_INVALID_ARG;
+    // x, B, C and y move in 16-byte pieces; dt in 2-byte ones
+    if (!aligned(x, 16) || !aligned(B, 16) || !aligned(C, 16) || !aligned(y, 16) || !aligned(dt, 2))
+      return MAMBA_ERR_INVALID_ARG;
+  }
+  if ((A && !aligned(A, 4)) || (D && !aligned(D, 8)) || (final_state && !aligned(final_state, 4)) ||
+      (initial_state && !aligned(initial_state, 4)))
+    return MAMBA_ERR_INVALID_ARG;
+  if (batch * len >= (int64_t(1) << 31) || heads * headdim >= (int64_t(1) << 31) || batch * heads >= (int64_t(1) << 31))
+    return MAMBA_ERR_UNSUPPORTED;
+
+  cudaGetLastError();  // clear a stale, non-sticky error so the status below is ours
+  const size_t state_bytes = sizeof(float) * (size_t)batch * (size_t)(heads * headdim) * (size_t)nstate;
+  if (len == 0) {
+    if (!final_state) return MAMBA_OK;
+    cudaError_t e = initial_state
+                        ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, stream)
+                        : cudaMemsetAsync(final_state, 0, state_bytes, stream);
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+  }
+  SsdArgs a = {};
+  a.x = static_cast<const __nv_bfloat16*>(x);
+  a.dt = static_cast<const __nv_bfloat16*>(dt);
+  a.A = A;
+  a.B = static_cast<const __nv_bfloat16*>(B);
+  a.C = static_cast<const __nv_bfloat16*>(C);
+  a.D = D;
+  a.h0 = initial_state;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.final_state = final_state;
+  a.len = len;
+  a.heads = (int)heads;
+  a.euler = (flags & MAMBA_SCAN_EULER) ? 1 : 0;
+  switch (nstate) {
+    case 16: return launch_ssd<16>(a, batch, supers, stream);
+    case 32: return launch_ssd<32>(a, batch, supers, stream);
+    default: return launch_ssd<64>(a, batch, supers, stream);
+  }
 }
 
 int mamba_get_device_error(int clear) {

@@ -3,7 +3,7 @@
 Every function named like a C entry point forwards its arguments to the
 library unchanged: tensors become device pointers, torch streams become
 `cudaStream_t` handles, a non-zero status raises `MambaError`.  The
-tensor-level helpers `selective_scan` and `state_update` only allocate the
+tensor-level helpers (`selective_scan`, `ssd_scan`, `state_update`, ...) only allocate the
 outputs with torch and then make the same C calls.  There is no fallback: if
 the library is missing or cannot load, every call raises.
 """
@@ -52,6 +52,9 @@ _SIGNATURES = [
      [_P] * 16 + [_I64, _I64, _I64, _I64, ctypes.c_int, _P]),
     ("mamba_state_update", ctypes.c_int,
      [_P, _P, _P, _P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, _P]),
+    ("mamba_ssd_scan", ctypes.c_int,
+     [_P] * 9 + [_I64] * 6 + [ctypes.c_uint, ctypes.c_int, _P]),
+    ("mamba_ssd_supported_nstate", ctypes.c_int, [_I64]),
     ("mamba_scan_plan", ctypes.c_int,
      [_I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ScanPlan)]),
     ("mamba_status_string", ctypes.c_char_p, [ctypes.c_int]),
@@ -175,6 +178,18 @@ def mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, 
     _check(st, "mamba_state_update")
 
 
+def mamba_ssd_scan(x, dt, A, B, C, D, initial_state, y, final_state, batch, len, heads, headdim, nstate, supers,
+                   flags, dtype, stream=None):
+    st = library().mamba_ssd_scan(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(initial_state),
+                                  _ptr(y), _ptr(final_state), batch, len, heads, headdim, nstate, supers, flags,
+                                  dtype, _stream(stream))
+    _check(st, "mamba_ssd_scan")
+
+
+def mamba_ssd_supported_nstate(nstate: int) -> bool:
+    return bool(library().mamba_ssd_supported_nstate(int(nstate)))
+
+
 def mamba_scan_plan(batch, len, channels, nstate, chunk_len, dtype, sm_count=0) -> ScanPlan:
     out = ScanPlan()
     _check(library().mamba_scan_plan(batch, len, channels, nstate, chunk_len, dtype, sm_count,
@@ -240,6 +255,32 @@ def state_update(state, x, delta, A, B, C, D=None, y=None, stream=None):
         y = torch.empty_like(x)
     mamba_state_update(state, x, delta, A, B, C, D, y, batch, channels, nstate, dtype_code(x.dtype), stream)
     return y
+
+
+def ssd_scan(x, dt, A, B, C, D=None, initial_state=None, return_final_state=True, headdim=64, supers=0,
+             method="zoh", y=None, final_state=None, stream=None):
+    """y, final_state = Mamba-2's scalar-A scan on CUDA tensors.
+
+    x: (batch, len, heads*headdim) bfloat16; dt: (batch, len, heads)
+    bfloat16; A: (heads,) float32; B, C: (batch, len, nstate) bfloat16; D:
+    (heads*headdim,) float32 or None; initial_state: (batch,
+    heads*headdim, nstate) float32 or None; method "zoh" or "euler"."""
+    import torch
+    batch, length, channels = x.shape
+    heads = A.shape[0]
+    nstate = B.shape[2]
+    for t in (x, dt, A, B, C, D, initial_state):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if channels != heads * headdim:
+        raise ValueError("x must have heads*headdim channels")
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((batch, channels, nstate), device=x.device, dtype=torch.float32)
+    mamba_ssd_scan(x, dt, A, B, C, D, initial_state, y, final_state, batch, length, heads, headdim, nstate, supers,
+                   _METHOD_FLAGS[method], dtype_code(x.dtype), stream)
+    return y, final_state
 
 
 def selective_scan_host(u, delta, A, B, C, D=None, y=None, final_state=None, piece_len=0, stream=None,

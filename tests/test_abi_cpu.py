@@ -92,6 +92,46 @@ def test_scan_argument_errors_on_host(lib):
     assert _scan_ex(lib, len=0, fs=None) == m.MAMBA_OK
 
 
+def _ssd(lib, **kw):
+    a = dict(x=1024, dt=1024, A=1024, B=1024, C=1024, D=None, h0=None, y=2048, fs=None, batch=1, len=4,
+             heads=2, headdim=64, nstate=16, supers=0, flags=0, dtype=m.MAMBA_BF16)
+    a.update(kw)
+    return lib.mamba_ssd_scan(a["x"], a["dt"], a["A"], a["B"], a["C"], a["D"], a["h0"], a["y"], a["fs"],
+                              a["batch"], a["len"], a["heads"], a["headdim"], a["nstate"], a["supers"],
+                              a["flags"], a["dtype"], None)
+
+
+def test_ssd_argument_errors_on_host(lib):
+    # every case below is rejected (or is a no-op) before any CUDA call is made
+    assert _ssd(lib, dtype=7) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, batch=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, len=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, heads=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, headdim=0) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, supers=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, flags=8) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, flags=m.MAMBA_SCAN_EULER | m.MAMBA_SCAN_TRAPEZOID) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, flags=m.MAMBA_SCAN_TRAPEZOID) == m.MAMBA_ERR_UNSUPPORTED
+    assert _ssd(lib, dtype=m.MAMBA_F32) == m.MAMBA_ERR_UNSUPPORTED
+    assert _ssd(lib, headdim=32) == m.MAMBA_ERR_UNSUPPORTED
+    for n in (4, 8, 12, 128):
+        assert _ssd(lib, nstate=n) == m.MAMBA_ERR_UNSUPPORTED
+    for n in (16, 32, 64):
+        assert m.mamba_ssd_supported_nstate(n)
+    assert _ssd(lib, x=None) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, dt=None) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, y=None) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, x=1032) == m.MAMBA_ERR_INVALID_ARG          # x not 16-byte aligned
+    assert _ssd(lib, B=1040 + 2) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, y=2056) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, dt=1025) == m.MAMBA_ERR_INVALID_ARG
+    assert _ssd(lib, D=1028) == m.MAMBA_ERR_INVALID_ARG          # D not 8-byte aligned
+    assert _ssd(lib, batch=1 << 20, len=1 << 12) == m.MAMBA_ERR_UNSUPPORTED
+    assert _ssd(lib, batch=0) == m.MAMBA_OK
+    assert _ssd(lib, heads=0) == m.MAMBA_OK
+    assert _ssd(lib, len=0, fs=None) == m.MAMBA_OK
+
+
 def test_state_update_argument_errors_on_host(lib):
     f = lib.mamba_state_update
     ok = dict(state=4096, x=1024, delta=1024, A=4096, B=1024, C=1024, D=None, y=2048, batch=2, channels=8,
