@@ -50,7 +50,36 @@ MUTANTS = {
                                        "(void)0;"),
 }
 
-PIN_TESTS = [getattr(pins, name) for name in dir(pins) if name.startswith("test_")]
+def _pin_calls(module):
+    """Every (name, function, keyword arguments) a pin module's tests run
+    with: parametrized pins are expanded over their parameter values."""
+    calls = []
+    for name in sorted(dir(module)):
+        if not name.startswith("test_"):
+            continue
+        fn = getattr(module, name)
+        combos = [{}]
+        for mark in getattr(fn, "pytestmark", []):
+            if mark.name != "parametrize":
+                continue
+            argnames, values = mark.args[0], mark.args[1]
+            keys = [k.strip() for k in argnames.split(",")] if isinstance(argnames, str) else list(argnames)
+            rows = [v if len(keys) > 1 else (v,) for v in values]
+            combos = [dict(c, **dict(zip(keys, r))) for c in combos for r in rows]
+        for kw in combos:
+            calls.append((name, fn, kw))
+    return calls
+
+
+PIN_CALLS = _pin_calls(pins)
+
+
+def test_every_pin_call_binds():
+    """The harness calls each pin with the oracle and its parameters only; a
+    call that cannot bind would count as a catch for every mutant."""
+    import inspect
+    for name, fn, kw in PIN_CALLS:
+        inspect.signature(fn).bind(None, **kw)
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
@@ -65,10 +94,10 @@ def test_pins_catch_mutant(name, tmp_path):
     lib = oracle_build.build(str(src), str(tmp_path / "libmutant.so"), force=True)
     mutant = oracle.Oracle(lib)
     failed = []
-    for test in PIN_TESTS:
+    for pin_name, test, kw in PIN_CALLS:
         try:
-            test(mutant)
+            test(mutant, **kw)
         except Exception:          # an assertion or a shape/NaN failure both count
-            failed.append(test.__name__)
+            failed.append(pin_name)
     assert failed, f"no pin caught mutant {name}"
     shutil.rmtree(tmp_path, ignore_errors=True)
