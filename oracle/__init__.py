@@ -37,6 +37,8 @@ class Oracle:
         self._lib.oracle_scan_backward.argtypes = [_c_f64p] * 16 + [_i64] * 4
         self._lib.oracle_state_update.restype = ctypes.c_int
         self._lib.oracle_state_update.argtypes = [_c_f64p] * 8 + [_i64] * 3 + [ctypes.c_int]
+        self._lib.oracle_scan_complex.restype = ctypes.c_int
+        self._lib.oracle_scan_complex.argtypes = [_c_f64p] * 10 + [_i64] * 4 + [ctypes.c_int]
         self._lib.oracle_max_threads.restype = ctypes.c_int
 
     @staticmethod
@@ -115,6 +117,28 @@ class Oracle:
             raise RuntimeError(f"oracle_state_update failed ({rc})")
         return y
 
+    def scan_complex(self, u, delta, A_re, A_im, B, C, D=None, h0=None, want_y=True, nthreads=0):
+        """Selective scan with a complex diagonal A = A_re + i A_im and a
+        complex state (the Mamba-3 page, "Karmaşık Değerli Durum
+        Güncellemesi"; the reading is in ssm_oracle.c).  h0 and the returned
+        final state are (batch, channels, nstate, 2) float64, (re, im)
+        adjacent.  Returns (y, h_final)."""
+        u, delta, A_re, A_im, B, C, D, h0 = map(self._f64, (u, delta, A_re, A_im, B, C, D, h0))
+        batch, length, channels = u.shape
+        nstate = A_re.shape[1]
+        assert delta.shape == u.shape and A_re.shape == (channels, nstate) and A_im.shape == A_re.shape
+        assert B.shape == (batch, length, nstate) and C.shape == B.shape
+        assert D is None or D.shape == (channels,)
+        assert h0 is None or h0.shape == (batch, channels, nstate, 2)
+        y = np.empty_like(u) if want_y else None
+        hf = np.empty((batch, channels, nstate, 2), dtype=np.float64)
+        rc = self._lib.oracle_scan_complex(self._ptr(u), self._ptr(delta), self._ptr(A_re), self._ptr(A_im),
+                                           self._ptr(B), self._ptr(C), self._ptr(D), self._ptr(h0), self._ptr(y),
+                                           self._ptr(hf), batch, length, channels, nstate, int(nthreads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_scan_complex failed ({rc})")
+        return y, hf
+
     # --- Mamba-2's restricted form (state space duality) -----------------
     @staticmethod
     def _ssd_channel_head(channels: int, headdim: int) -> np.ndarray:
@@ -175,3 +199,7 @@ def state_update(*args, **kwargs):
 
 def ssd_scan(*args, **kwargs):
     return get().ssd_scan(*args, **kwargs)
+
+
+def scan_complex(*args, **kwargs):
+    return get().scan_complex(*args, **kwargs)

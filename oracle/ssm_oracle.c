@@ -40,6 +40,7 @@
  *   D             : [channels]                (may be NULL: no skip term)
  *   h0, h_final   : [batch][channels][nstate] (h0 may be NULL: zeros)
  */
+#include <complex.h>
 #include <math.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -374,6 +375,102 @@ int oracle_scan_backward(const double *u, const double *delta, const double *A,
 }
 
 /* Threads the OpenMP runtime would use (for reporting the CPU baseline). */
+/* ---------------------------------------------------------------------------
+ * Complex-valued state.
+ *
+ * The Mamba-3 page (bitig.info), section "Karmaşık Değerli Durum
+ * Güncellemesi": the state update uses complex numbers; complex eigenvalues
+ * of the transition represent oscillation and rotation, and the page relates
+ * them to data-dependent rotary embeddings.  It prints no formula.  Reading
+ * taken: A stays diagonal with complex entries A[d][n] = A_re + i A_im
+ * (A_re < 0); the zero-order hold of "Ayrık Zamana Geçiş" applies unchanged
+ * in complex arithmetic,
+ *     Abar = exp(Delta A),   Bbar = (Delta A)^-1 (exp(Delta A) - 1) Delta B,
+ * with B and C real as in the selective scan; the state is complex and the
+ * output takes its real part,
+ *     y_t = sum_n C_t[n] Re(h_t[n]) + D x_t.
+ * Each step turns a state by the angle Delta_t A_im: the rotation depends on
+ * the input through Delta.
+ *
+ * Layouts: A_re, A_im [channels][nstate]; h0, h_final
+ * [batch][channels][nstate][2] with (re, im) adjacent; the rest as above.
+ * ------------------------------------------------------------------------- */
+static void scan_row_complex(const double *u, const double *delta, const double *Are_row,
+                             const double *Aim_row, const double *B, const double *C, double D_d,
+                             int has_D, double *y, double complex *h, int64_t len, int64_t stride,
+                             int64_t nstate)
+{
+    for (int64_t t = 0; t < len; ++t) {
+        double x = u[t * stride];
+        double dt = delta[t * stride];
+        const double *Bt = B + t * nstate;
+        const double *Ct = C + t * nstate;
+        double acc = 0.0;
+        for (int64_t n = 0; n < nstate; ++n) {
+            double complex a = Are_row[n] + I * Aim_row[n];
+            double complex z = dt * a;
+            double complex abar = cexp(z);
+            double complex phi = (z == 0.0) ? 1.0 : (abar - 1.0) / z;  /* (Delta A)^-1 (e^{Delta A} - 1) */
+            double complex bbar = phi * dt * Bt[n];
+            h[n] = abar * h[n] + bbar * x;
+            acc += Ct[n] * creal(h[n]);
+        }
+        if (has_D)
+            acc += D_d * x;
+        if (y)
+            y[t * stride] = acc;
+    }
+}
+
+int oracle_scan_complex(const double *u, const double *delta, const double *A_re, const double *A_im,
+                        const double *B, const double *C, const double *D, const double *h0,
+                        double *y, double *h_final, int64_t batch, int64_t len, int64_t channels,
+                        int64_t nstate, int nthreads)
+{
+    if (batch < 0 || len < 0 || channels < 0 || nstate <= 0)
+        return -1;
+    if ((len > 0 && (!u || !delta || !B || !C)) || !A_re || !A_im)
+        return -1;
+    int64_t rows = batch * channels;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = 0;
+#pragma omp parallel
+    {
+        double complex *h = (double complex *)malloc(sizeof(double complex) * (size_t)nstate);
+        if (!h) {
+#pragma omp atomic write
+            status = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < rows; ++r) {
+            if (!h)
+                continue;
+            int64_t b = r / channels, d = r % channels;
+            for (int64_t n = 0; n < nstate; ++n) {
+                const double *s0 = h0 ? h0 + ((b * channels + d) * nstate + n) * 2 : NULL;
+                h[n] = s0 ? s0[0] + I * s0[1] : 0.0;
+            }
+            const size_t tok0 = (size_t)(b * len) * (size_t)channels + (size_t)d;
+            scan_row_complex(len ? u + tok0 : NULL, len ? delta + tok0 : NULL, A_re + d * nstate,
+                             A_im + d * nstate, len ? B + (size_t)(b * len) * (size_t)nstate : NULL,
+                             len ? C + (size_t)(b * len) * (size_t)nstate : NULL, D ? D[d] : 0.0,
+                             D != NULL, (y && len) ? y + tok0 : NULL, h, len, channels, nstate);
+            if (h_final)
+                for (int64_t n = 0; n < nstate; ++n) {
+                    h_final[((b * channels + d) * nstate + n) * 2] = creal(h[n]);
+                    h_final[((b * channels + d) * nstate + n) * 2 + 1] = cimag(h[n]);
+                }
+        }
+        free(h);
+    }
+    return status;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

@@ -2,7 +2,8 @@
 
 Each case below copies oracle/ssm_oracle.c, plants one mistake by text
 substitution (in every copy of the line), builds the copy on the CPU and runs
-every pin of test_oracle_pins.py against it: at least one pin has to fail.
+every pin of test_oracle_pins.py and test_oracle_complex_pins.py against it: at
+least one pin has to fail.
 """
 import os
 import shutil
@@ -11,6 +12,7 @@ import pytest
 
 import oracle
 from oracle import build as oracle_build
+from tests import test_oracle_complex_pins as complex_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
@@ -48,6 +50,13 @@ MUTANTS = {
     "backward_ddelta_missing_a": ("ddt += lam[n] * r * (a * hprev + bn * x);", "ddt += lam[n] * r * (hprev + bn * x);"),
     "backward_adjoint_before_output": ("lam[n] += C[k * nstate + n] * g;           /* lam_t                       */",
                                        "(void)0;"),
+    # the complex-valued state
+    "complex_output_from_imaginary_part": ("acc += Ct[n] * creal(h[n]);", "acc += Ct[n] * cimag(h[n]);"),
+    "complex_rotation_sign": ("double complex a = Are_row[n] + I * Aim_row[n];",
+                              "double complex a = Are_row[n] - I * Aim_row[n];"),
+    "complex_input_missing_division": ("(abar - 1.0) / z;", "(abar - 1.0);"),
+    "complex_rotation_dropped": ("double complex abar = cexp(z);", "double complex abar = exp(creal(z));"),
+    "complex_state_layout_swapped": ("h[n] = s0 ? s0[0] + I * s0[1] : 0.0;", "h[n] = s0 ? s0[1] + I * s0[0] : 0.0;"),
 }
 
 def _pin_calls(module):
@@ -71,7 +80,7 @@ def _pin_calls(module):
     return calls
 
 
-PIN_CALLS = _pin_calls(pins)
+PIN_CALLS = _pin_calls(pins) + _pin_calls(complex_pins)
 
 
 def test_every_pin_call_binds():
