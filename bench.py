@@ -666,6 +666,35 @@ def run_variants(w, dev, stream, dist, world, rank, reps: int = 20):
         res[name] = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
                      "nstate": wv.nstate}
         del inp, y, hf
+    # the complex-valued state (A_im = pi n), the same shape
+    inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
+    A_im = wl.complex_a_imag(w.channels, w.nstate, dev)
+    y = torch.empty_like(inp["u"])
+    hf = torch.empty((w.batch, w.channels, w.nstate, 2), device=dev, dtype=torch.float32)
+
+    def cstep():
+        st = lib.mamba_selective_scan_complex(inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(),
+                                              A_im.data_ptr(), inp["B"].data_ptr(), inp["C"].data_ptr(),
+                                              inp["D"].data_ptr(), None, y.data_ptr(), hf.data_ptr(), w.batch,
+                                              w.length, w.channels, w.nstate, 0, dtc, stream.cuda_stream)
+        if st != 0:
+            raise m.MambaError(st, "mamba_selective_scan_complex")
+
+    for _ in range(3):
+        cstep()
+    torch.cuda.synchronize()
+    barrier(dist, world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        cstep()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(dist, world, a.elapsed_time(b)) / reps
+    res["complex_state"] = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
+                            "nstate": w.nstate, "note": "complex diagonal A (imaginary parts pi n), complex state"}
+    del inp, A_im, y, hf
+
     # the backward (gradients of every input from dy), zero-order hold
     inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
     dy = torch.randn(inp["u"].shape, device=dev).to(inp["u"].dtype)

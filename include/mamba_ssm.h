@@ -320,6 +320,39 @@ int mamba_ssd_scan(const void *x, const void *dt, const float *A, const void *B,
 /* 1 if `nstate` is implemented by mamba_ssd_scan. */
 int mamba_ssd_supported_nstate(int64_t nstate);
 
+/*
+ * The selective scan with a complex diagonal A and a complex state.
+ *
+ * Defined by: the Mamba-3 page (bitig.info), "Karmaşık Değerli Durum
+ * Güncellemesi" (complex state update; complex eigenvalues let the state
+ * rotate and oscillate).  The page prints no formula; the reading taken is
+ * A[d][n] = A_re[d][n] + i A_im[d][n] (A_re < 0) with the zero-order hold of
+ * mamba_selective_scan in complex arithmetic and real B, C:
+ *   h_t = exp(delta A) h_{t-1} + (exp(delta A) - 1)/A * B_t x_t
+ *   y_t = sum_n C_t[n] Re(h_t[n]) + D x_t
+ * so a state turns by delta_t * A_im per token.
+ *
+ * Layouts as mamba_selective_scan (u, delta, y [batch][len][channels]; B, C
+ * [batch][len][nstate]; one dtype for them, fp32 or bf16); A_re, A_im
+ * [channels][nstate] fp32; D [channels] fp32 or NULL; initial_state and
+ * final_state [batch][channels][nstate][2] fp32 with (re, im) adjacent
+ * (8-byte aligned), or NULL.  supers: super-chunks per sequence run in
+ * parallel (0 = chosen from the shape and the device); with more than one,
+ * stream-ordered scratch of 8 nstate + 8 bytes per (batch, super-chunk,
+ * channel) holds their end states and step sums.  nstate 4, 8 or 16
+ * (otherwise MAMBA_ERR_UNSUPPORTED).  All arithmetic fp32 (the sum of steps
+ * of a super-chunk in double).  Errors and len == 0 as for
+ * mamba_selective_scan_ex.  Asynchronous on `stream`.
+ */
+int mamba_selective_scan_complex(const void *u, const void *delta, const float *A_re,
+                                 const float *A_im, const void *B, const void *C, const float *D,
+                                 const float *initial_state, void *y, float *final_state,
+                                 int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                                 int64_t supers, int dtype, mamba_stream_t stream);
+
+/* 1 if `nstate` is implemented by mamba_selective_scan_complex. */
+int mamba_complex_supported_nstate(int64_t nstate);
+
 /* How mamba_selective_scan_ex would split a problem (host-side planning only). */
 typedef struct {
     int64_t supers;        /* independent super-chunks per sequence (1: no aggregate jobs) */

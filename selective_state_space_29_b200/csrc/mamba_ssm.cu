@@ -17,6 +17,7 @@
 #include "decode.cuh"
 #include "scan.cuh"
 #include "ssd.cuh"
+#include "complex_scan.cuh"
 
 namespace mamba {
 
@@ -592,6 +593,52 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
   return st;
 }
 
+// --- complex-valued state (complex_scan.cuh) ---------------------------------
+template <typename TIO, int N>
+int launch_complex(ComplexArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream) {
+  using L = ComplexSmem<TIO, N>;
+  auto main_k = complex_scan_kernel<TIO, N, false>;
+  auto agg_k = complex_scan_kernel<TIO, N, true>;
+  if (cudaFuncSetAttribute(main_k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(agg_k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+    return MAMBA_ERR_CUDA;
+  int sms = 0, per_sm = 0;
+  if (current_sms(&sms) != MAMBA_OK) return MAMBA_ERR_CUDA;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, main_k, kCplxWarps * 32, L::kBytes) != cudaSuccess ||
+      per_sm < 1)
+    return MAMBA_ERR_CUDA;
+  const int64_t seqs = batch * a.groups;  // one warp each
+  const int64_t blocks = (a.len + kCplxBlock - 1) / kCplxBlock;
+  int64_t S = ssd_supers(seqs, blocks, (int64_t)sms * per_sm * kCplxWarps, supers_req);
+  const int64_t per = (blocks + S - 1) / S;
+  S = (blocks + per - 1) / per;
+  a.super_len = per * kCplxBlock;
+  a.supers = (int)S;
+  if (seqs * S >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+  unsigned char* mem = nullptr;
+  if (S > 1) {
+    const size_t slots = (size_t)batch * (size_t)(S - 1) * (size_t)a.channels;
+    const size_t h_bytes = (slots * N * 2 * sizeof(float) + 15) / 16 * 16;
+    if (scratch_alloc(reinterpret_cast<void**>(&mem), h_bytes + slots * sizeof(double), stream) != cudaSuccess)
+      return MAMBA_ERR_CUDA;
+    a.agg_h = reinterpret_cast<float*>(mem);
+    a.agg_sd = reinterpret_cast<double*>(mem + h_bytes);
+    a.jobs = seqs * (S - 1);
+    if (launch_pdl(agg_k, dim3((unsigned)((a.jobs + kCplxWarps - 1) / kCplxWarps)), dim3(kCplxWarps * 32), L::kBytes,
+                   stream, a) != cudaSuccess) {
+      cudaFreeAsync(mem, stream);
+      return MAMBA_ERR_CUDA;
+    }
+  }
+  a.jobs = seqs * S;
+  int st = MAMBA_OK;
+  if (launch_pdl(main_k, dim3((unsigned)((a.jobs + kCplxWarps - 1) / kCplxWarps)), dim3(kCplxWarps * 32), L::kBytes,
+                 stream, a) != cudaSuccess)
+    st = MAMBA_ERR_CUDA;
+  if (mem && cudaFreeAsync(mem, stream) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
+  return st;
+}
+
 }  // namespace
 }  // namespace mamba
 
@@ -935,6 +982,65 @@ int mamba_ssd_scan(const void* x, const void* dt, const float* A, const void* B,
     case 16: return launch_ssd<16>(a, batch, supers, stream);
     case 32: return launch_ssd<32>(a, batch, supers, stream);
     default: return launch_ssd<64>(a, batch, supers, stream);
+  }
+}
+
+int mamba_complex_supported_nstate(int64_t nstate) { return nstate == 4 || nstate == 8 || nstate == 16; }
+
+int mamba_selective_scan_complex(const void* u, const void* delta, const float* A_re, const float* A_im,
+                                 const void* B, const void* C, const float* D, const float* initial_state, void* y,
+                                 float* final_state, int64_t batch, int64_t len, int64_t channels, int64_t nstate,
+                                 int64_t supers, int dtype, mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || len < 0 || channels < 0 || nstate <= 0 || supers < 0) return MAMBA_ERR_INVALID_ARG;
+  if (!mamba_complex_supported_nstate(nstate)) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || channels == 0) return MAMBA_OK;
+  const size_t es = (size_t)elem_size(dtype);
+  if (!A_re || !A_im) return MAMBA_ERR_INVALID_ARG;
+  if (len > 0) {
+    if (!u || !delta || !B || !C || !y) return MAMBA_ERR_INVALID_ARG;
+    if (!aligned(u, es) || !aligned(delta, es) || !aligned(B, es) || !aligned(C, es) || !aligned(y, es))
+      return MAMBA_ERR_INVALID_ARG;
+  }
+  if (!aligned(A_re, 4) || !aligned(A_im, 4) || (D && !aligned(D, 4)) || (final_state && !aligned(final_state, 8)) ||
+      (initial_state && !aligned(initial_state, 8)))
+    return MAMBA_ERR_INVALID_ARG;
+  if (batch * len >= (int64_t(1) << 31) || channels >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+
+  cudaGetLastError();  // clear a stale, non-sticky error so the status below is ours
+  const size_t state_bytes = 2 * sizeof(float) * (size_t)batch * (size_t)channels * (size_t)nstate;
+  if (len == 0) {
+    if (!final_state) return MAMBA_OK;
+    cudaError_t e = initial_state
+                        ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, stream)
+                        : cudaMemsetAsync(final_state, 0, state_bytes, stream);
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+  }
+  ComplexArgs a = {};
+  a.u = u;
+  a.delta = delta;
+  a.A_re = A_re;
+  a.A_im = A_im;
+  a.B = B;
+  a.C = C;
+  a.D = D;
+  a.h0 = initial_state;
+  a.y = y;
+  a.final_state = final_state;
+  a.len = len;
+  a.channels = (int)channels;
+  const int cpw = nstate >= 8 ? 16 : 32;  // channels per warp (ComplexSmem::kCPW)
+  a.groups = (int)((channels + cpw - 1) / cpw);
+  auto go = [&](auto ns) {
+    constexpr int NS = decltype(ns)::value;
+    return dtype == MAMBA_BF16 ? launch_complex<__nv_bfloat16, NS>(a, batch, supers, stream)
+                               : launch_complex<float, NS>(a, batch, supers, stream);
+  };
+  switch (nstate) {
+    case 4: return go(std::integral_constant<int, 4>{});
+    case 8: return go(std::integral_constant<int, 8>{});
+    default: return go(std::integral_constant<int, 16>{});
   }
 }
 

@@ -55,6 +55,9 @@ _SIGNATURES = [
     ("mamba_ssd_scan", ctypes.c_int,
      [_P] * 9 + [_I64] * 6 + [ctypes.c_uint, ctypes.c_int, _P]),
     ("mamba_ssd_supported_nstate", ctypes.c_int, [_I64]),
+    ("mamba_selective_scan_complex", ctypes.c_int,
+     [_P] * 10 + [_I64] * 5 + [ctypes.c_int, _P]),
+    ("mamba_complex_supported_nstate", ctypes.c_int, [_I64]),
     ("mamba_scan_plan", ctypes.c_int,
      [_I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ScanPlan)]),
     ("mamba_status_string", ctypes.c_char_p, [ctypes.c_int]),
@@ -190,6 +193,18 @@ def mamba_ssd_supported_nstate(nstate: int) -> bool:
     return bool(library().mamba_ssd_supported_nstate(int(nstate)))
 
 
+def mamba_selective_scan_complex(u, delta, A_re, A_im, B, C, D, initial_state, y, final_state, batch, len, channels,
+                                 nstate, supers, dtype, stream=None):
+    st = library().mamba_selective_scan_complex(_ptr(u), _ptr(delta), _ptr(A_re), _ptr(A_im), _ptr(B), _ptr(C),
+                                                _ptr(D), _ptr(initial_state), _ptr(y), _ptr(final_state), batch, len,
+                                                channels, nstate, supers, dtype, _stream(stream))
+    _check(st, "mamba_selective_scan_complex")
+
+
+def mamba_complex_supported_nstate(nstate: int) -> bool:
+    return bool(library().mamba_complex_supported_nstate(int(nstate)))
+
+
 def mamba_scan_plan(batch, len, channels, nstate, chunk_len, dtype, sm_count=0) -> ScanPlan:
     out = ScanPlan()
     _check(library().mamba_scan_plan(batch, len, channels, nstate, chunk_len, dtype, sm_count,
@@ -280,6 +295,29 @@ def ssd_scan(x, dt, A, B, C, D=None, initial_state=None, return_final_state=True
         final_state = torch.empty((batch, channels, nstate), device=x.device, dtype=torch.float32)
     mamba_ssd_scan(x, dt, A, B, C, D, initial_state, y, final_state, batch, length, heads, headdim, nstate, supers,
                    _METHOD_FLAGS[method], dtype_code(x.dtype), stream)
+    return y, final_state
+
+
+def selective_scan_complex(u, delta, A_re, A_im, B, C, D=None, initial_state=None, return_final_state=True,
+                           supers=0, y=None, final_state=None, stream=None):
+    """y, final_state = the scan with a complex diagonal A = A_re + i A_im.
+
+    u, delta: (batch, len, channels); B, C: (batch, len, nstate) of one dtype
+    (float32 or bfloat16); A_re, A_im: (channels, nstate) float32; D:
+    (channels,) or None; initial_state and the returned final state:
+    (batch, channels, nstate, 2) float32, (re, im) in the last index."""
+    import torch
+    batch, length, channels = u.shape
+    nstate = A_re.shape[1]
+    for t in (u, delta, A_re, A_im, B, C, D, initial_state):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if y is None:
+        y = torch.empty_like(u)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((batch, channels, nstate, 2), device=u.device, dtype=torch.float32)
+    mamba_selective_scan_complex(u, delta, A_re, A_im, B, C, D, initial_state, y, final_state, batch, length,
+                                 channels, nstate, supers, dtype_code(u.dtype), stream)
     return y, final_state
 
 

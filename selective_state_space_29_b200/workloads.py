@@ -181,6 +181,14 @@ def a_matrix(channels: int, nstate: int, mode: str, gen, device) -> torch.Tensor
     raise ValueError(f"unknown A mode {mode!r}")
 
 
+def complex_a_imag(channels: int, nstate: int, device) -> torch.Tensor:
+    """Rotation rates of a complex diagonal A (imaginary parts), pi * n for
+    state n: the pages give none; these are the S4D-Lin imaginary parts, so
+    the real parts of the scan workloads' A pair with evenly spaced
+    frequencies."""
+    return (math.pi * torch.arange(nstate, device=device, dtype=torch.float32)).expand(channels, nstate).contiguous()
+
+
 def scan_inputs(w: ScanWorkload, device="cpu", seed: int | None = None) -> dict:
     """u, delta (batch, len, channels); B, C (batch, len, nstate) in the
     workload dtype; A (channels, nstate) and D (channels,) in fp32."""

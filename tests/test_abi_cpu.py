@@ -132,6 +132,36 @@ def test_ssd_argument_errors_on_host(lib):
     assert _ssd(lib, len=0, fs=None) == m.MAMBA_OK
 
 
+def _cplx(lib, **kw):
+    a = dict(u=1024, delta=1024, Are=1024, Aim=1024, B=1024, C=1024, D=None, h0=None, y=2048, fs=None, batch=1,
+             len=4, channels=8, nstate=16, supers=0, dtype=m.MAMBA_BF16)
+    a.update(kw)
+    return lib.mamba_selective_scan_complex(a["u"], a["delta"], a["Are"], a["Aim"], a["B"], a["C"], a["D"],
+                                            a["h0"], a["y"], a["fs"], a["batch"], a["len"], a["channels"],
+                                            a["nstate"], a["supers"], a["dtype"], None)
+
+
+def test_complex_scan_argument_errors_on_host(lib):
+    assert _cplx(lib, dtype=7) == m.MAMBA_ERR_INVALID_ARG
+    assert _cplx(lib, batch=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _cplx(lib, len=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _cplx(lib, channels=-1) == m.MAMBA_ERR_INVALID_ARG
+    assert _cplx(lib, supers=-1) == m.MAMBA_ERR_INVALID_ARG
+    for n in (2, 12, 32):
+        assert _cplx(lib, nstate=n) == m.MAMBA_ERR_UNSUPPORTED
+    for n in (4, 8, 16):
+        assert m.mamba_complex_supported_nstate(n)
+    assert _cplx(lib, Aim=None) == m.MAMBA_ERR_INVALID_ARG
+    assert _cplx(lib, u=None) == m.MAMBA_ERR_INVALID_ARG
+    assert _cplx(lib, u=1025) == m.MAMBA_ERR_INVALID_ARG
+    assert _cplx(lib, dtype=m.MAMBA_F32, B=1026) == m.MAMBA_ERR_INVALID_ARG
+    assert _cplx(lib, h0=1028) == m.MAMBA_ERR_INVALID_ARG          # complex state: 8-byte aligned
+    assert _cplx(lib, batch=1 << 20, len=1 << 12) == m.MAMBA_ERR_UNSUPPORTED
+    assert _cplx(lib, batch=0) == m.MAMBA_OK
+    assert _cplx(lib, channels=0) == m.MAMBA_OK
+    assert _cplx(lib, len=0, fs=None) == m.MAMBA_OK
+
+
 def test_state_update_argument_errors_on_host(lib):
     f = lib.mamba_state_update
     ok = dict(state=4096, x=1024, delta=1024, A=4096, B=1024, C=1024, D=None, y=2048, batch=2, channels=8,

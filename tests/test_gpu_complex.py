@@ -1,0 +1,137 @@
+"""GPU parity of the complex-state scan (`mamba_selective_scan_complex`)
+against the fp64 oracle (`Oracle.scan_complex`), through the C ABI.
+
+Whole outputs on small cases (a ragged 32-channel group, ragged token
+blocks, one and several super-chunks, 4, 8 and 16 states, fp32 and bf16, an
+initial state, no skip term, fast and slow rotations), the real scan when
+every rotation is zero, and sampled channels of the mid workload.
+Tolerances as for the scan: 1e-4 (fp32), 2e-2 (bf16), per (batch, channel)
+row, normwise.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_29_b200 import mamba_ssm as m
+from selective_state_space_29_b200 import workloads as wl
+from tests.gpu_helpers import TOL, f64, row_error
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _a_imag(w, mode, seed=3):
+    if mode == "s4d_lin":
+        return wl.complex_a_imag(w.channels, w.nstate, DEV)
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    hi = {"slow": 2.0, "fast": 40.0}[mode]
+    return torch.empty((w.channels, w.nstate), device=DEV).uniform_(-hi, hi, generator=g).contiguous()
+
+
+def _check(w, supers=0, D=True, h0_std=None, a_imag="s4d_lin"):
+    """Rows shorter than a block of 32 tokens are gated normwise over the
+    whole output: a row of one or a few tokens makes the row measure an
+    elementwise relative error, which cancellation in C.Re(h) + D x can make
+    arbitrarily large for any rounding."""
+    inp = wl.scan_inputs(w, DEV)
+    A_im = _a_imag(w, a_imag)
+    h0 = None
+    if h0_std is not None:
+        g = torch.Generator(device=DEV).manual_seed(9)
+        h0 = h0_std * torch.randn((w.batch, w.channels, w.nstate, 2), generator=g, device=DEV)
+    y, hf = m.selective_scan_complex(inp["u"], inp["delta"], inp["A"], A_im, inp["B"], inp["C"],
+                                     inp["D"] if D else None, initial_state=h0, supers=supers)
+    torch.cuda.synchronize()
+    yr, hr = oracle.scan_complex(f64(inp["u"]), f64(inp["delta"]), f64(inp["A"]), f64(A_im), f64(inp["B"]),
+                                 f64(inp["C"]), f64(inp["D"]) if D else None, h0=None if h0 is None else f64(h0))
+    yg, hg = f64(y), f64(hf)
+    assert np.isfinite(yg).all() and np.isfinite(hg).all()
+    tol = TOL[w.dtype]
+    ey = row_error(yg, yr, axis=1) if w.length >= 32 else float(np.abs(yg - yr).max() / np.abs(yr).max())
+    eh = row_error(hg.reshape(w.batch, w.channels, -1), hr.reshape(w.batch, w.channels, -1), axis=2)
+    assert ey <= tol, f"y error {ey:.3e} > {tol}"
+    assert eh <= tol, f"final state error {eh:.3e} > {tol}"
+
+
+SMALL = wl.ScanWorkload("cplx_small", batch=2, length=1000, channels=200, nstate=16, dtype="f32", seed=301)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("supers", [0, 1, 3])
+def test_complex_small(dtype, supers):
+    _check(SMALL.with_(dtype=dtype), supers=supers)
+
+
+@pytest.mark.parametrize("nstate", [4, 8, 16])
+@pytest.mark.parametrize("a_imag", ["slow", "fast"])
+def test_complex_state_counts_and_rotation_rates(nstate, a_imag):
+    _check(SMALL.with_(nstate=nstate, length=500, a_mode="state"), a_imag=a_imag)
+
+
+@pytest.mark.parametrize("supers", [1, 4])
+def test_complex_initial_state_and_no_skip(supers):
+    _check(SMALL.with_(length=600), supers=supers, h0_std=0.3)
+    _check(SMALL.with_(length=600), supers=supers, D=False)
+
+
+@pytest.mark.parametrize("length", [1, 31, 32, 33])
+def test_complex_short_lengths(length):
+    w = SMALL.with_(length=length, channels=40)
+    _check(w, supers=1, h0_std=0.3)
+    _check(w, supers=0)
+
+
+def test_complex_without_rotation_is_the_real_scan():
+    w = SMALL.with_(length=700)
+    inp = wl.scan_inputs(w, DEV)
+    zero = torch.zeros_like(inp["A"])
+    y, hf = m.selective_scan_complex(inp["u"], inp["delta"], inp["A"], zero, inp["B"], inp["C"], inp["D"])
+    yr, hr = m.selective_scan(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], general_a=True)
+    torch.cuda.synchronize()
+    assert row_error(f64(y), f64(yr), axis=1) <= TOL["f32"]
+    assert row_error(f64(hf[..., 0]), f64(hr), axis=2) <= TOL["f32"]
+    assert torch.count_nonzero(hf[..., 1]) == 0
+
+
+def test_complex_len_zero_copies_initial_state():
+    w = SMALL.with_(length=0)
+    inp = wl.scan_inputs(w, DEV)
+    h0 = torch.randn((w.batch, w.channels, w.nstate, 2), device=DEV)
+    _, hf = m.selective_scan_complex(inp["u"], inp["delta"], inp["A"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                     initial_state=h0)
+    torch.cuda.synchronize()
+    assert torch.equal(hf, h0)
+
+
+def test_complex_mid_workload_sampled_channels():
+    w = wl.SCAN_WORKLOADS["mid_bf16"]
+    inp = wl.scan_inputs(w, DEV)
+    A_im = wl.complex_a_imag(w.channels, w.nstate, DEV)
+    y, hf = m.selective_scan_complex(inp["u"], inp["delta"], inp["A"], A_im, inp["B"], inp["C"], inp["D"])
+    torch.cuda.synchronize()
+    ch = torch.tensor([0, 31, 32, 1777, w.channels - 1], device=DEV)
+    yr, hr = oracle.scan_complex(f64(inp["u"].index_select(2, ch)), f64(inp["delta"].index_select(2, ch)),
+                                 f64(inp["A"].index_select(0, ch)), f64(A_im.index_select(0, ch)), f64(inp["B"]),
+                                 f64(inp["C"]), f64(inp["D"].index_select(0, ch)))
+    ey = row_error(f64(y.index_select(2, ch)), yr, axis=1)
+    eh = row_error(f64(hf.index_select(1, ch)).reshape(w.batch, len(ch), -1), hr.reshape(w.batch, len(ch), -1), 2)
+    assert ey <= TOL["bf16"] and eh <= TOL["bf16"], (ey, eh)
+
+
+def test_complex_graph_capture_replays_the_eager_result():
+    w = SMALL.with_(length=700)
+    inp = wl.scan_inputs(w, DEV)
+    A_im = wl.complex_a_imag(w.channels, w.nstate, DEV)
+    args = (inp["u"], inp["delta"], inp["A"], A_im, inp["B"], inp["C"], inp["D"])
+    y0, h0 = m.selective_scan_complex(*args, supers=4)
+    y, hf = torch.empty_like(y0), torch.empty_like(h0)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        m.selective_scan_complex(*args, supers=4, y=y, final_state=hf)
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0) and torch.equal(hf, h0)

@@ -159,3 +159,19 @@ def test_ssd_mid_workload_sampled_heads():
 def test_ssd_long_workload_sampled_head():
     w = wl.SSD_WORKLOADS["ssd_long_bf16"]
     _check(w, heads=[w.heads - 1])
+
+
+def test_ssd_graph_capture_replays_the_eager_result():
+    # the small shape uses several super-chunks, so the captured call also
+    # allocates and frees its aggregate scratch inside the graph
+    inp = wl.ssd_inputs(SMALL, DEV)
+    args = (inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"], inp["D"])
+    y0, h0 = m.ssd_scan(*args)
+    y, hf = torch.empty_like(y0), torch.empty_like(h0)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        m.ssd_scan(*args, y=y, final_state=hf)
+    y.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0) and torch.equal(hf, h0)
