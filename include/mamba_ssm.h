@@ -258,7 +258,10 @@ int mamba_selective_scan_host(const void *u, const void *delta, const float *A,
  * It runs the forward scan once more, keeping only the state before every
  * tile, then one warp per (batch, 32-channel group) walks the sequence in
  * reverse, recomputing each tile's states from its checkpoint (stream-ordered
- * scratch: the checkpoints and [T][32][nstate] floats per warp).  dA, dB,
+ * scratch: the checkpoints and [T][32][nstate] floats per warp).  With
+ * 16-byte aligned rows (channels * element size and nstate * element size
+ * multiples of 16, tensors 16-byte aligned) each tile's inputs are first
+ * staged in shared memory (16 KB per warp).  dA, dB,
  * dC and dD are accumulated with atomic adds, so their last bits can vary
  * from call to call.  Asynchronous on `stream`.
  */

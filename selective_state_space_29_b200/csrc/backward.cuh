@@ -28,7 +28,11 @@
 // scratch area ([T][32][N], 64 bytes per lane and token at N = 16, small
 // enough to stay in L2), then takes the tile's reverse steps reading the
 // states back.  The channel sums for dB and dC are a warp reduce-scatter
-// (lane i ends with the sum of value i) and one atomic add per lane.
+// (lane i ends with the sum of value i) and one atomic add per lane.  When
+// rows are 16-byte aligned, the warp first copies the tile's u, Delta and
+// dy rows and its B, C rows into its shared memory (one round of 16-byte
+// cp.async copies), so both passes over the tile read shared memory
+// instead of waiting on a global load per token.
 #pragma once
 
 #include "common.cuh"
@@ -63,7 +67,47 @@ struct BwdArgs {
   int super_tiles;
   float* agg_mu;           // [S][streams][32][N] outgoing adjoint of super-chunk j from zero
   float* agg_sd;           // [S][streams][32] sum of Delta over super-chunk j
+  int staged;              // tiles are staged in shared memory (rows 16-byte aligned)
 };
+
+// Bytes of one warp's staged tile: u, Delta and dy rows of 32 channels, then
+// the B and C rows, for T tokens.
+template <typename TIO, int NS>
+__host__ __device__ constexpr int bwd_stage_bytes(int T) {
+  return (3 * 32 + 2 * NS) * T * (int)sizeof(TIO);
+}
+
+// 16-byte asynchronous copy of which the first `bytes` (0..16) come from src
+// and the rest is zero-filled
+__device__ __forceinline__ void bwd_cp_async(uint32_t dst, const void* src, int bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
+}
+
+// the B (or C) row of a token from shared memory as NS floats
+template <typename TIO, int NS>
+__device__ __forceinline__ void load_row_smem(const TIO* row, float (&v)[NS]) {
+  if constexpr (sizeof(TIO) == 2 && NS % 8 == 0) {
+#pragma unroll
+    for (int i = 0; i < NS / 8; ++i) {
+      const uint4 w = reinterpret_cast<const uint4*>(row)[i];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * i + 2 * j] = __uint_as_float(ws[j] << 16);
+        v[8 * i + 2 * j + 1] = __uint_as_float(ws[j] & 0xffff0000u);
+      }
+    }
+  } else if constexpr (sizeof(TIO) == 4 && NS % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < NS / 4; ++i) {
+      const float4 w = reinterpret_cast<const float4*>(row)[i];
+      v[4 * i] = w.x; v[4 * i + 1] = w.y; v[4 * i + 2] = w.z; v[4 * i + 3] = w.w;
+    }
+  } else {
+#pragma unroll
+    for (int n = 0; n < NS; ++n) v[n] = to_f32(row[n]);
+  }
+}
 
 // the B (or C) row of a token as NS floats: vector loads of the raw row
 template <typename TIO, int NS>
@@ -198,10 +242,11 @@ scan_backward_aggregate_kernel(const BwdArgs<TIO> a) {
   else bwd_aggregate_item<TIO, NS, false>(a, j, stream, b, d, active, lane, An);
 }
 
-// One work item: super-chunk j of one stream, tiles in reverse.
-template <typename TIO, int NS, bool STRUCT>
+// One work item: super-chunk j of one stream, tiles in reverse.  STAGED:
+// the tile's inputs are copied to `stg` (this warp's shared memory) first.
+template <typename TIO, int NS, bool STRUCT, bool STAGED>
 __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t stream, int64_t b, int64_t d,
-                                         bool active, int lane, const float (&An)[NS], float* S) {
+                                         bool active, int lane, const float (&An)[NS], float* S, TIO* stg) {
   const int64_t streams = a.batch * a.groups_d;
   const int T = a.tile;
   const int64_t ntiles = (a.len + T - 1) / T;
@@ -229,16 +274,69 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
     const int64_t t0 = tile * T;
     const int rows = (int)(a.len - t0 < (int64_t)T ? a.len - t0 : (int64_t)T);
     const float* ck = a.ckpt + ((b * ntiles + tile) * a.channels + (active ? d : 0)) * NS;
+    const TIO* su = stg;                 // staged rows: u, Delta, dy [T][32], then B, C [T][NS]
+    const TIO* sdl = stg + T * 32;
+    const TIO* sdy = stg + 2 * T * 32;
+    const TIO* sB = stg + 3 * T * 32;
+    const TIO* sC = sB + T * NS;
+    if constexpr (STAGED) {
+      __syncwarp();  // every lane is done with the previous tile's rows
+      constexpr int P = 32 * (int)sizeof(TIO) / 16;  // 16-byte pieces per row of 32 channels
+      constexpr int EPP = 16 / (int)sizeof(TIO);      // channels per piece
+      constexpr int RB = 32 * (int)sizeof(TIO);       // bytes per staged row
+      const uint32_t s0 = smem_addr(stg);
+      const int64_t ch_base = d - lane;
+      for (int i = lane; i < rows * P; i += 32) {
+        const int r = i / P, pc = i % P;
+        const int64_t ch = ch_base + pc * EPP;
+        const bool ok = ch < a.channels;  // whole pieces: the channel count is a multiple of EPP here
+        const int64_t off = (b * a.len + t0 + r) * a.channels + ch;
+        const uint32_t o = (uint32_t)(r * RB + pc * 16);
+        bwd_cp_async(s0 + o, ok ? (const void*)(a.u + off) : (const void*)a.u, ok ? 16 : 0);
+        bwd_cp_async(s0 + T * RB + o, ok ? (const void*)(a.delta + off) : (const void*)a.delta, ok ? 16 : 0);
+        bwd_cp_async(s0 + 2 * T * RB + o, ok ? (const void*)(a.dy + off) : (const void*)a.dy, ok ? 16 : 0);
+      }
+      const int nbytes = rows * NS * (int)sizeof(TIO);  // a multiple of 16 here
+      const char* gB = reinterpret_cast<const char*>(a.B + (b * a.len + t0) * NS);
+      const char* gC = reinterpret_cast<const char*>(a.C + (b * a.len + t0) * NS);
+      const uint32_t sbB = s0 + 3 * T * RB, sbC = sbB + T * NS * (int)sizeof(TIO);
+      for (int i = lane * 16; i < nbytes; i += 32 * 16) {
+        bwd_cp_async(sbB + i, gB + i, 16);
+        bwd_cp_async(sbC + i, gC + i, 16);
+      }
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncwarp();
+    }
+    auto get_x = [&](int k, int64_t tok) -> float {
+      if constexpr (STAGED) return to_f32(su[k * 32 + lane]);
+      else return active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
+    };
+    auto get_dt = [&](int k, int64_t tok) -> float {
+      if constexpr (STAGED) return to_f32(sdl[k * 32 + lane]);
+      else return active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+    };
+    auto get_dy = [&](int k, int64_t tok) -> float {
+      if constexpr (STAGED) return to_f32(sdy[k * 32 + lane]);
+      else return active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
+    };
+    auto get_B = [&](int k, int64_t tok, float (&v)[NS]) {
+      if constexpr (STAGED) load_row_smem<TIO, NS>(sB + k * NS, v);
+      else load_row<TIO, NS>(a.B + tok * NS, v, a.vec_rows);
+    };
+    auto get_C = [&](int k, int64_t tok, float (&v)[NS]) {
+      if constexpr (STAGED) load_row_smem<TIO, NS>(sC + k * NS, v);
+      else load_row<TIO, NS>(a.C + tok * NS, v, a.vec_rows);
+    };
     // forward over the tile: S[k] = h after token t0 + k
     float h[NS];
 #pragma unroll
     for (int n = 0; n < NS; ++n) h[n] = active ? ck[n] : 0.0f;
     for (int k = 0; k < rows; ++k) {
       const int64_t tok = b * a.len + t0 + k;
-      const float x = active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
-      const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+      const float x = get_x(k, tok);
+      const float dt = get_dt(k, tok);
       float bv[NS], q[NS];
-      load_row<TIO, NS>(a.B + tok * NS, bv, a.vec_rows);
+      get_B(k, tok, bv);
       decays<NS, STRUCT>(dt, An, q);
 #pragma unroll
       for (int n = 0; n < NS; ++n) h[n] = fmaf(1.0f + q[n], h[n], q[n] * iA[n] * bv[n] * x);
@@ -260,14 +358,14 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
 #pragma unroll
         for (int n = 0; n < NS; ++n) hp[n] = active ? ck[n] : 0.0f;
       }
-      const float x = active ? to_f32(a.u[tok * a.channels + d]) : 0.0f;
-      const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
-      const float gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
+      const float x = get_x(k, tok);
+      const float dt = get_dt(k, tok);
+      const float gy = get_dy(k, tok);
       float du = Dd * gy, ddt = 0.0f;
       dD = fmaf(gy, x, dD);
       float bv[NS], cv[NS], q[NS];
-      load_row<TIO, NS>(a.B + tok * NS, bv, a.vec_rows);
-      load_row<TIO, NS>(a.C + tok * NS, cv, a.vec_rows);
+      get_B(k, tok, bv);
+      get_C(k, tok, cv);
       decays<NS, STRUCT>(dt, An, q);
       float red[32];
 #pragma unroll
@@ -312,8 +410,10 @@ template <typename TIO, int NS>
 __global__ void __launch_bounds__(kBwdWarps * 32, 3)
 scan_backward_kernel(const BwdArgs<TIO> a) {
   static_assert(2 * NS <= 32, "dB and dC of a token are reduced in one 32-lane pass");
+  extern __shared__ __align__(16) unsigned char bwd_smem[];
   griddep_wait();  // the aggregates and checkpoints come from the previous kernels of the stream
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  TIO* stg = reinterpret_cast<TIO*>(bwd_smem + warp * bwd_stage_bytes<TIO, NS>(a.tile));
   const int64_t wid = (int64_t)blockIdx.x * kBwdWarps + warp;
   const int64_t nwarps = (int64_t)gridDim.x * kBwdWarps;
   const int64_t streams = a.batch * a.groups_d;
@@ -328,8 +428,14 @@ scan_backward_kernel(const BwdArgs<TIO> a) {
     float An[NS];
 #pragma unroll
     for (int n = 0; n < NS; ++n) An[n] = active ? __ldg(a.A + d * NS + n) : -(float)(n + 1);
-    if (group_structured<NS>(An)) bwd_item<TIO, NS, true>(a, j, stream, b, d, active, lane, An, S);
-    else bwd_item<TIO, NS, false>(a, j, stream, b, d, active, lane, An, S);
+    const bool st = group_structured<NS>(An);
+    if (a.staged) {
+      if (st) bwd_item<TIO, NS, true, true>(a, j, stream, b, d, active, lane, An, S, stg);
+      else bwd_item<TIO, NS, false, true>(a, j, stream, b, d, active, lane, An, S, stg);
+    } else {
+      if (st) bwd_item<TIO, NS, true, false>(a, j, stream, b, d, active, lane, An, S, stg);
+      else bwd_item<TIO, NS, false, false>(a, j, stream, b, d, active, lane, An, S, stg);
+    }
   }
 }
 

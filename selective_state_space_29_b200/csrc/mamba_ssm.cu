@@ -842,9 +842,20 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
                            a) != cudaSuccess)
               st = MAMBA_ERR_CUDA;
           }
+          // tiles staged in shared memory when every row piece is a whole,
+          // aligned 16-byte copy
+          a.staged = ((channels * (int64_t)es) % 16 == 0 && (NS * es) % 16 == 0 && aligned(u, 16) &&
+                      aligned(delta, 16) && aligned(dy, 16) && aligned(B, 16) && aligned(C, 16))
+                         ? 1
+                         : 0;
+          const int smem = a.staged ? kBwdWarps * bwd_stage_bytes<TIO, NS>(T) : 0;
+          if (st == MAMBA_OK && smem > 0 &&
+              cudaFuncSetAttribute(scan_backward_kernel<TIO, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   smem) != cudaSuccess)
+            st = MAMBA_ERR_CUDA;
           if (st == MAMBA_OK &&
-              launch_pdl(scan_backward_kernel<TIO, NS>, dim3((unsigned)ctas), dim3(kBwdWarps * 32), 0, stream, a) !=
-                  cudaSuccess)
+              launch_pdl(scan_backward_kernel<TIO, NS>, dim3((unsigned)ctas), dim3(kBwdWarps * 32), (size_t)smem,
+                         stream, a) != cudaSuccess)
             st = MAMBA_ERR_CUDA;
         }
         if (cudaFreeAsync(mem, stream) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
