@@ -344,20 +344,28 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
       for (int n = 0; n < NS; n += 4)
         *reinterpret_cast<float4*>(S + (size_t)k * 32 * NS + n) = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
     }
-    // reverse over the tile; h holds h_t, hp is read back as h_{t-1}
-    for (int k = rows - 1; k >= 0; --k) {
-      const int64_t tok = b * a.len + t0 + k;
-      float hp[NS];
+    // reverse over the tile; h holds h_t, hp is read back as h_{t-1}, one
+    // token ahead of its use (hn)
+    auto read_prev = [&](int k, float (&v)[NS]) {  // h_{t0+k-1}
       if (k > 0) {
 #pragma unroll
         for (int n = 0; n < NS; n += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(S + (size_t)(k - 1) * 32 * NS + n);
-          hp[n] = v.x; hp[n + 1] = v.y; hp[n + 2] = v.z; hp[n + 3] = v.w;
+          const float4 w = *reinterpret_cast<const float4*>(S + (size_t)(k - 1) * 32 * NS + n);
+          v[n] = w.x; v[n + 1] = w.y; v[n + 2] = w.z; v[n + 3] = w.w;
         }
       } else {
 #pragma unroll
-        for (int n = 0; n < NS; ++n) hp[n] = active ? ck[n] : 0.0f;
+        for (int n = 0; n < NS; ++n) v[n] = active ? ck[n] : 0.0f;
       }
+    };
+    float hn[NS];
+    read_prev(rows - 1, hn);
+    for (int k = rows - 1; k >= 0; --k) {
+      const int64_t tok = b * a.len + t0 + k;
+      float hp[NS];
+#pragma unroll
+      for (int n = 0; n < NS; ++n) hp[n] = hn[n];
+      if (k > 0) read_prev(k - 1, hn);
       const float x = get_x(k, tok);
       const float dt = get_dt(k, tok);
       const float gy = get_dy(k, tok);
