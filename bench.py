@@ -61,6 +61,8 @@ def parse_args():
                     help="skip the timings of the scan's options (general A, other discretisations, state counts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-ssd", action="store_true", help="skip Mamba-2's scalar-A scan (state space duality) leg")
+    ap.add_argument("--only-backward", action="store_true",
+                    help="run only the backward on the workload's shape (steps = timed calls) and print its object")
     ap.add_argument("--only-ssd", action="store_true",
                     help="run only the scalar-A scan leg (steps/warmup as given) and print its object")
     ap.add_argument("--length-sweep", action="store_true",
@@ -84,6 +86,7 @@ KERNEL_SOURCES = {
     "scan_chunks_kernel": ("common.cuh", "scan.cuh"),
     "state_update_kernel": ("common.cuh", "scan.cuh", "decode.cuh"),
     "ssd_chunk_kernel": ("common.cuh", "ssd.cuh"),
+    "scan_backward_kernel": ("common.cuh", "scan.cuh", "backward.cuh"),
 }
 
 
@@ -695,7 +698,33 @@ def run_variants(w, dev, stream, dist, world, rank, reps: int = 20):
                             "nstate": w.nstate, "note": "complex diagonal A (imaginary parts pi n), complex state"}
     del inp, A_im, y, hf
 
-    # the backward (gradients of every input from dy), zero-order hold
+    res["backward"] = run_backward(w, dev, stream, dist, world, rank)
+    res["note"] = (f"{w.name} shape; general A and the other discretisations take one exp2 per state "
+                   f"(MUFU); nstate_* are zero-order hold with structured A")
+    return res
+
+
+def backward_bytes(w) -> int:
+    """Algorithmic bytes of one backward call: u, delta, dy, B, C read; du,
+    ddelta written (I/O dtype); dB, dC (fp32) written; A, D and their
+    gradients."""
+    es = 2 if w.dtype == "bf16" else 4
+    tc = w.batch * w.length * w.channels
+    bc = w.batch * w.length * w.nstate
+    return tc * es * 5 + bc * (2 * es + 2 * 4) + w.channels * (w.nstate + 1) * 4 * 2
+
+
+def run_backward(w, dev, stream, dist, world, rank, reps: int = 5):
+    """ms per call of the backward (gradients of every input from dy, zero-order
+    hold) on the workload's shape, with its bytes against the HBM peak."""
+    import torch
+
+    from selective_state_space_29_b200 import mamba_ssm as m
+    from selective_state_space_29_b200 import workloads as wl
+
+    lib = m.library()
+    dtc = m.dtype_code(w.torch_dtype)
+    tc = w.batch * w.length * w.channels
     inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
     dy = torch.randn(inp["u"].shape, device=dev).to(inp["u"].dtype)
     f32 = dict(device=dev, dtype=torch.float32)
@@ -717,17 +746,21 @@ def run_variants(w, dev, stream, dist, world, rank, reps: int = 20):
     barrier(dist, world)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record(stream)
-    for _ in range(5):
+    for _ in range(reps):
         bwd()
     b.record(stream)
     torch.cuda.synchronize()
-    ms = max_over_ranks(dist, world, a.elapsed_time(b)) / 5
-    res["backward"] = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
-                       "nstate": w.nstate, "includes": "checkpointing forward pass + reverse pass"}
+    ms = max_over_ranks(dist, world, a.elapsed_time(b)) / reps
     del inp, dy, outs
-    res["note"] = (f"{w.name} shape; general A and the other discretisations take one exp2 per state "
-                   f"(MUFU); nstate_* are zero-order hold with structured A")
-    return res
+    peaks = measured_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    nb = backward_bytes(w)
+    ach = nb / (ms * 1e-3) / 1e9
+    return {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3), "nstate": w.nstate,
+            "includes": "checkpointing forward pass + reverse aggregates + reverse pass",
+            "hbm": {"achieved": round(ach, 1), "peak": hbm, "unit": "GB/s", "frac": round(ach / hbm, 4),
+                    "algorithmic_bytes_per_call": nb,
+                    "traffic_reverse_kernel": profiled_traffic("scan_backward_kernel", w.name)}}
 
 
 # --- reference arm: the fp64 oracle on the host cores ------------------------------------
@@ -827,6 +860,18 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.only_backward:
+        import torch
+        from selective_state_space_29_b200 import workloads as wl
+        rank, world, local = dist_setup(args.gpus)
+        torch.cuda.set_device(local)
+        dist = init_pg(world, local)
+        res = run_backward(wl.SCAN_WORKLOADS[args.workload], torch.device("cuda", local),
+                           torch.cuda.current_stream(), dist, world, rank, reps=max(1, args.steps))
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps({"backward": res}), flush=True)
     elif args.only_ssd:
         import torch
         rank, world, local = dist_setup(args.gpus)
