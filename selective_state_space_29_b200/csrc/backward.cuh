@@ -83,6 +83,36 @@ __device__ __forceinline__ void bwd_cp_async(uint32_t dst, const void* src, int 
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(bytes) : "memory");
 }
 
+// Stage `rows` token rows of the 32 channels from ch_base on (one row is
+// 32 elements, 16-byte pieces; pieces past the last channel are zero-filled)
+// to dst, [rows][32]: row r of token t0 + r.  The channel count is a multiple
+// of the elements in a piece and the rows are 16-byte aligned on this path.
+template <typename TIO>
+__device__ __forceinline__ void bwd_stage_rows(uint32_t dst, const TIO* src, int64_t tok0, int rows,
+                                               int64_t ch_base, int64_t channels, int lane) {
+  constexpr int P = 32 * (int)sizeof(TIO) / 16;  // pieces per row
+  constexpr int EPP = 16 / (int)sizeof(TIO);      // channels per piece
+  for (int i = lane; i < rows * P; i += 32) {
+    const int r = i / P, pc = i % P;
+    const int64_t ch = ch_base + pc * EPP;
+    const bool ok = ch < channels;
+    bwd_cp_async(dst + (uint32_t)(r * 32 * (int)sizeof(TIO) + pc * 16),
+                 ok ? (const void*)(src + (tok0 + r) * channels + ch) : (const void*)src, ok ? 16 : 0);
+  }
+}
+
+// Stage `nbytes` (a multiple of 16) contiguous bytes
+__device__ __forceinline__ void bwd_stage_contig(uint32_t dst, const void* src, int nbytes, int lane) {
+  for (int i = lane * 16; i < nbytes; i += 32 * 16) bwd_cp_async(dst + i, static_cast<const char*>(src) + i, 16);
+}
+
+// Bytes of one warp's staged tile in the aggregate kernel: Delta and dy rows,
+// then the C rows
+template <typename TIO, int NS>
+__host__ __device__ constexpr int bwd_agg_stage_bytes(int T) {
+  return (2 * 32 + NS) * T * (int)sizeof(TIO);
+}
+
 // the B (or C) row of a token from shared memory as NS floats
 template <typename TIO, int NS>
 __device__ __forceinline__ void load_row_smem(const TIO* row, float (&v)[NS]) {
@@ -194,9 +224,10 @@ __device__ __forceinline__ bool group_structured(const float (&An)[NS]) {
 // (after its first token, multiplied by that token's exp(Delta A)), and its
 // sum of Delta: the reverse counterpart of the forward aggregates.  Only C,
 // dy and Delta enter (no state).
-template <typename TIO, int NS, bool STRUCT>
+template <typename TIO, int NS, bool STRUCT, bool STAGED>
 __device__ __forceinline__ void bwd_aggregate_item(const BwdArgs<TIO>& a, int j, int64_t stream, int64_t b,
-                                                   int64_t d, bool active, int lane, const float (&An)[NS]) {
+                                                   int64_t d, bool active, int lane, const float (&An)[NS],
+                                                   TIO* stg) {
   const int64_t streams = a.batch * a.groups_d;
   const int T = a.tile;
   const int64_t t_lo = (int64_t)j * a.super_tiles * T;
@@ -205,16 +236,40 @@ __device__ __forceinline__ void bwd_aggregate_item(const BwdArgs<TIO>& a, int j,
 #pragma unroll
   for (int n = 0; n < NS; ++n) mu[n] = 0.0f;
   float sd = 0.0f;
-  for (int64_t t = t_hi - 1; t >= t_lo; --t) {
-    const int64_t tok = b * a.len + t;
-    const float dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
-    const float gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
-    float cv[NS], q[NS];
-    load_row<TIO, NS>(a.C + tok * NS, cv, a.vec_rows);
-    decays<NS, STRUCT>(dt, An, q);
-    sd += dt;
+  // tiles in reverse (t_lo is a tile boundary; the last tile may be short)
+  for (int64_t tt0 = t_lo + ((t_hi - 1 - t_lo) / T) * T; tt0 >= t_lo; tt0 -= T) {
+    const int rows = (int)(t_hi - tt0 < (int64_t)T ? t_hi - tt0 : (int64_t)T);
+    const TIO* sdl = stg;  // staged rows: Delta, dy [T][32], then C [T][NS]
+    const TIO* sdy = stg + T * 32;
+    const TIO* sC = stg + 2 * T * 32;
+    if constexpr (STAGED) {
+      __syncwarp();
+      constexpr int RB = 32 * (int)sizeof(TIO);
+      const uint32_t s0 = smem_addr(stg);
+      const int64_t tok0 = b * a.len + tt0;
+      bwd_stage_rows<TIO>(s0, a.delta, tok0, rows, d - lane, a.channels, lane);
+      bwd_stage_rows<TIO>(s0 + T * RB, a.dy, tok0, rows, d - lane, a.channels, lane);
+      bwd_stage_contig(s0 + 2 * T * RB, a.C + tok0 * NS, rows * NS * (int)sizeof(TIO), lane);
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncwarp();
+    }
+    for (int k = rows - 1; k >= 0; --k) {
+      const int64_t tok = b * a.len + tt0 + k;
+      float dt, gy, cv[NS], q[NS];
+      if constexpr (STAGED) {
+        dt = to_f32(sdl[k * 32 + lane]);
+        gy = to_f32(sdy[k * 32 + lane]);
+        load_row_smem<TIO, NS>(sC + k * NS, cv);
+      } else {
+        dt = active ? to_f32(a.delta[tok * a.channels + d]) : 0.0f;
+        gy = active ? to_f32(a.dy[tok * a.channels + d]) : 0.0f;
+        load_row<TIO, NS>(a.C + tok * NS, cv, a.vec_rows);
+      }
+      decays<NS, STRUCT>(dt, An, q);
+      sd += dt;
 #pragma unroll
-    for (int n = 0; n < NS; ++n) mu[n] = (1.0f + q[n]) * fmaf(cv[n], gy, mu[n]);
+      for (int n = 0; n < NS; ++n) mu[n] = (1.0f + q[n]) * fmaf(cv[n], gy, mu[n]);
+    }
   }
   const size_t base = ((size_t)j * streams + stream) * 32 + lane;
   a.agg_sd[base] = sd;
@@ -225,8 +280,10 @@ __device__ __forceinline__ void bwd_aggregate_item(const BwdArgs<TIO>& a, int j,
 template <typename TIO, int NS>
 __global__ void __launch_bounds__(kBwdWarps * 32)
 scan_backward_aggregate_kernel(const BwdArgs<TIO> a) {
+  extern __shared__ __align__(16) unsigned char bwd_agg_smem[];
   griddep_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  TIO* stg = reinterpret_cast<TIO*>(bwd_agg_smem + warp * bwd_agg_stage_bytes<TIO, NS>(a.tile));
   const int64_t streams = a.batch * a.groups_d;
   const int64_t item = (int64_t)blockIdx.x * kBwdWarps + warp;  // (j - 1) * streams + stream
   if (item >= (int64_t)(a.supers - 1) * streams) return;
@@ -238,8 +295,14 @@ scan_backward_aggregate_kernel(const BwdArgs<TIO> a) {
   float An[NS];
 #pragma unroll
   for (int n = 0; n < NS; ++n) An[n] = active ? __ldg(a.A + d * NS + n) : -(float)(n + 1);
-  if (group_structured<NS>(An)) bwd_aggregate_item<TIO, NS, true>(a, j, stream, b, d, active, lane, An);
-  else bwd_aggregate_item<TIO, NS, false>(a, j, stream, b, d, active, lane, An);
+  const bool st = group_structured<NS>(An);
+  if (a.staged) {
+    if (st) bwd_aggregate_item<TIO, NS, true, true>(a, j, stream, b, d, active, lane, An, stg);
+    else bwd_aggregate_item<TIO, NS, false, true>(a, j, stream, b, d, active, lane, An, stg);
+  } else {
+    if (st) bwd_aggregate_item<TIO, NS, true, false>(a, j, stream, b, d, active, lane, An, stg);
+    else bwd_aggregate_item<TIO, NS, false, false>(a, j, stream, b, d, active, lane, An, stg);
+  }
 }
 
 // One work item: super-chunk j of one stream, tiles in reverse.  STAGED:
@@ -281,29 +344,15 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
     const TIO* sC = sB + T * NS;
     if constexpr (STAGED) {
       __syncwarp();  // every lane is done with the previous tile's rows
-      constexpr int P = 32 * (int)sizeof(TIO) / 16;  // 16-byte pieces per row of 32 channels
-      constexpr int EPP = 16 / (int)sizeof(TIO);      // channels per piece
-      constexpr int RB = 32 * (int)sizeof(TIO);       // bytes per staged row
+      constexpr int RB = 32 * (int)sizeof(TIO);  // bytes per staged row
       const uint32_t s0 = smem_addr(stg);
-      const int64_t ch_base = d - lane;
-      for (int i = lane; i < rows * P; i += 32) {
-        const int r = i / P, pc = i % P;
-        const int64_t ch = ch_base + pc * EPP;
-        const bool ok = ch < a.channels;  // whole pieces: the channel count is a multiple of EPP here
-        const int64_t off = (b * a.len + t0 + r) * a.channels + ch;
-        const uint32_t o = (uint32_t)(r * RB + pc * 16);
-        bwd_cp_async(s0 + o, ok ? (const void*)(a.u + off) : (const void*)a.u, ok ? 16 : 0);
-        bwd_cp_async(s0 + T * RB + o, ok ? (const void*)(a.delta + off) : (const void*)a.delta, ok ? 16 : 0);
-        bwd_cp_async(s0 + 2 * T * RB + o, ok ? (const void*)(a.dy + off) : (const void*)a.dy, ok ? 16 : 0);
-      }
-      const int nbytes = rows * NS * (int)sizeof(TIO);  // a multiple of 16 here
-      const char* gB = reinterpret_cast<const char*>(a.B + (b * a.len + t0) * NS);
-      const char* gC = reinterpret_cast<const char*>(a.C + (b * a.len + t0) * NS);
+      const int64_t tok0 = b * a.len + t0;
+      bwd_stage_rows<TIO>(s0, a.u, tok0, rows, d - lane, a.channels, lane);
+      bwd_stage_rows<TIO>(s0 + T * RB, a.delta, tok0, rows, d - lane, a.channels, lane);
+      bwd_stage_rows<TIO>(s0 + 2 * T * RB, a.dy, tok0, rows, d - lane, a.channels, lane);
       const uint32_t sbB = s0 + 3 * T * RB, sbC = sbB + T * NS * (int)sizeof(TIO);
-      for (int i = lane * 16; i < nbytes; i += 32 * 16) {
-        bwd_cp_async(sbB + i, gB + i, 16);
-        bwd_cp_async(sbC + i, gC + i, 16);
-      }
+      bwd_stage_contig(sbB, a.B + tok0 * NS, rows * NS * (int)sizeof(TIO), lane);
+      bwd_stage_contig(sbC, a.C + tok0 * NS, rows * NS * (int)sizeof(TIO), lane);
       asm volatile("cp.async.wait_all;" ::: "memory");
       __syncwarp();
     }

@@ -835,19 +835,25 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
                          (aligned(B, 16) && aligned(C, 16) && (NS * sizeof(TIO)) % 16 == 0) ? 1 : 0, (int)supers,
                          (int)super_tiles, reinterpret_cast<float*>(mem + ck_bytes + sc_bytes),
                          reinterpret_cast<float*>(mem + ck_bytes + sc_bytes + mu_bytes)};
-          if (supers > 1) {
-            const int64_t agg_items = (supers - 1) * streams;
-            if (launch_pdl(scan_backward_aggregate_kernel<TIO, NS>,
-                           dim3((unsigned)((agg_items + kBwdWarps - 1) / kBwdWarps)), dim3(kBwdWarps * 32), 0, stream,
-                           a) != cudaSuccess)
-              st = MAMBA_ERR_CUDA;
-          }
           // tiles staged in shared memory when every row piece is a whole,
           // aligned 16-byte copy
           a.staged = ((channels * (int64_t)es) % 16 == 0 && (NS * es) % 16 == 0 && aligned(u, 16) &&
                       aligned(delta, 16) && aligned(dy, 16) && aligned(B, 16) && aligned(C, 16))
                          ? 1
                          : 0;
+          if (supers > 1) {
+            const int64_t agg_items = (supers - 1) * streams;
+            const int agg_smem = a.staged ? kBwdWarps * bwd_agg_stage_bytes<TIO, NS>(T) : 0;
+            if (agg_smem > 0 && cudaFuncSetAttribute(scan_backward_aggregate_kernel<TIO, NS>,
+                                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     agg_smem) != cudaSuccess)
+              st = MAMBA_ERR_CUDA;
+            if (st == MAMBA_OK &&
+                launch_pdl(scan_backward_aggregate_kernel<TIO, NS>,
+                           dim3((unsigned)((agg_items + kBwdWarps - 1) / kBwdWarps)), dim3(kBwdWarps * 32),
+                           (size_t)agg_smem, stream, a) != cudaSuccess)
+              st = MAMBA_ERR_CUDA;
+          }
           const int smem = a.staged ? kBwdWarps * bwd_stage_bytes<TIO, NS>(T) : 0;
           if (st == MAMBA_OK && smem > 0 &&
               cudaFuncSetAttribute(scan_backward_kernel<TIO, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
