@@ -25,9 +25,9 @@
 // are recomputed tile by tile: the forward kernel leaves the state before
 // every tile of T tokens in a checkpoint array; the warp re-runs a tile
 // forward from its checkpoint, writing h_t for each token to a per-warp
-// scratch area ([T][32][N], 64 bytes per lane and token at N = 16, small
-// enough to stay in L2), then takes the tile's reverse steps reading the
-// states back.  The channel sums for dB and dC are a warp reduce-scatter
+// scratch area ([T][32][N], 64 bytes per lane and token at N = 16, read
+// back one token ahead of use; 227 MB over the resident warps, so it lives
+// in DRAM), then walks the tile in reverse.  dB and dC are a reduce-scatter
 // (lane i ends with the sum of value i) and one atomic add per lane.  When
 // rows are 16-byte aligned, the warp first copies the tile's u, Delta and
 // dy rows and its B, C rows into its shared memory (one round of 16-byte
