@@ -112,7 +112,7 @@ complex_scan_kernel(const ComplexArgs a) {
   constexpr int LPC = L::kLPC;    // lanes per channel
   constexpr int CPW = L::kCPW;    // channels per warp
   constexpr int NH = N / LPC;     // states per lane
-  extern __shared__ __align__(16) unsigned char smem[];
+  extern __shared__ __align__(16) unsigned char cplx_smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int64_t job = (int64_t)blockIdx.x * kCplxWarps + warp;
@@ -132,10 +132,10 @@ complex_scan_kernel(const ComplexArgs a) {
   const int64_t t_begin = (int64_t)j * a.super_len;
   const int64_t t_end = t_begin + a.super_len < a.len ? t_begin + a.super_len : a.len;
 
-  float* su = reinterpret_cast<float*>(smem + warp * L::kWarp + L::kU);
-  float* sdt = reinterpret_cast<float*>(smem + warp * L::kWarp + L::kDt);
-  float* sB = reinterpret_cast<float*>(smem + warp * L::kWarp + L::kB);
-  float* sC = reinterpret_cast<float*>(smem + warp * L::kWarp + L::kC);
+  float* su = reinterpret_cast<float*>(cplx_smem + warp * L::kWarp + L::kU);
+  float* sdt = reinterpret_cast<float*>(cplx_smem + warp * L::kWarp + L::kDt);
+  float* sB = reinterpret_cast<float*>(cplx_smem + warp * L::kWarp + L::kB);
+  float* sC = reinterpret_cast<float*>(cplx_smem + warp * L::kWarp + L::kC);
 
   // per state: a, w / 2, and 1/A = conj(A) / |A|^2
   float ar[NH], wh[NH], iar[NH], iai[NH];

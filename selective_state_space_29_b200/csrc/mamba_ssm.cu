@@ -834,7 +834,7 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
                          dA, dB, dC, D ? dD : nullptr, d_initial_state, batch, len, channels, (int)groups_d, T,
                          (aligned(B, 16) && aligned(C, 16) && (NS * sizeof(TIO)) % 16 == 0) ? 1 : 0, (int)supers,
                          (int)super_tiles, reinterpret_cast<float*>(mem + ck_bytes + sc_bytes),
-                         reinterpret_cast<float*>(mem + ck_bytes + sc_bytes + mu_bytes)};
+                         reinterpret_cast<float*>(mem + ck_bytes + sc_bytes + mu_bytes), 0};
           // tiles staged in shared memory when every row piece is a whole,
           // aligned 16-byte copy
           a.staged = ((channels * (int64_t)es) % 16 == 0 && (NS * es) % 16 == 0 && aligned(u, 16) &&
