@@ -132,3 +132,26 @@ def test_complex_initial_state_response(oracle_lib):
     yb, hb = _real_block_scan(u, delta, A_re, A_im, B, C, None, h0=h0)
     assert _rel(y, yb) < 1e-11
     assert _rel(hf, hb) < 1e-11
+
+
+def test_complex_quarter_turn_halving_closed_form(oracle_lib):
+    """Delta = 1, A = -ln 2 + i pi/2: exp(Delta A) = i/2 exactly (half a
+    magnitude, a quarter turn per step).  With B = C = 1 and an impulse
+    x_0 = 1, h_t = (i/2)^t Bbar with Bbar = (i/2 - 1) / A; in real arithmetic
+    (a + ib)/(c + id) = ((ac + bd) + i(bc - ad)) / (c^2 + d^2), so
+    Re Bbar = (ln 2 + pi/4) / (ln^2 2 + pi^2/4), Im Bbar = (pi/2 - ln 2 / 2) / (same).
+    Then y_0 = Re Bbar, y_1 = -Im Bbar / 2, y_{t+2} = -y_t / 4, and after six
+    tokens h_5 = (i/32) Bbar = (-Im Bbar / 32, Re Bbar / 32)."""
+    L = 6
+    ln2, hp = math.log(2.0), math.pi / 2
+    den = ln2 * ln2 + hp * hp
+    re_b, im_b = (ln2 + math.pi / 4) / den, (hp - ln2 / 2) / den
+    u = np.zeros((1, L, 1))
+    u[0, 0, 0] = 1.0
+    y, hf = oracle_lib.scan_complex(u, np.ones((1, L, 1)), np.array([[-ln2]]), np.array([[hp]]),
+                                    np.ones((1, L, 1)), np.ones((1, L, 1)), None)
+    want = [re_b, -im_b / 2]
+    for t in range(2, L):
+        want.append(-want[t - 2] / 4)
+    assert np.max(np.abs(y[0, :, 0] - np.array(want))) < 1e-14
+    assert abs(hf[0, 0, 0, 0] - (-im_b / 32)) < 1e-15 and abs(hf[0, 0, 0, 1] - re_b / 32) < 1e-15
