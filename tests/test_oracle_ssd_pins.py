@@ -147,17 +147,19 @@ def test_ssd_heads_are_independent(oracle_lib):
     assert _rel(y1[:, :, 2:4], y2[:, :, 2:4]) > 1e-3
 
 
-def test_ssd_one_state_constant_step_closed_form(oracle_lib):
+@pytest.mark.parametrize("method", [0, 1], ids=["zoh", "euler"])
+def test_ssd_one_state_constant_step_closed_form(oracle_lib, method):
     """One head of one channel, one state, constant dt, B = C = 1, x = 1:
-    h_t = w (1 - r^(t+1)) / (1 - r) with r = exp(a dt), w = (r - 1)/a."""
+    h_t = w (1 - r^(t+1)) / (1 - r) with r = exp(a dt) and the input weight
+    w = (r - 1)/a (zero-order hold) or w = dt (exponential Euler)."""
     L, a, d = 30, -2.0, 0.05
     x = np.ones((1, L, 1))
     dt = np.full((1, L, 1), d)
     B = np.ones((1, L, 1))
     C = np.ones((1, L, 1))
-    y, hf = oracle_lib.ssd_scan(x, dt, np.array([a]), B, C, None, headdim=1)
+    y, hf = oracle_lib.ssd_scan(x, dt, np.array([a]), B, C, None, headdim=1, method=method)
     r = math.exp(a * d)
-    w = (r - 1.0) / a
+    w = (r - 1.0) / a if method == 0 else d
     want = np.array([w * (1 - r ** (t + 1)) / (1 - r) for t in range(L)])
     assert np.max(np.abs(y[0, :, 0] - want)) < 1e-14
     assert abs(hf[0, 0, 0] - want[-1]) < 1e-14
