@@ -20,18 +20,26 @@
  *   - section "Mamba'nın Yeniliği: Selective SSM": B, C and Delta are produced
  *     per token (B_t, C_t, Delta_t); A stays a fixed parameter.
  *
- * Readings taken where the pages are silent or disagree (each is listed in the
- * design notes of the repository):
- *   - A is diagonal, one value per (channel, state): A[d][n].  The discretised
- *     quantities are then per state: Abar_n = exp(Delta A_n) and
+ * Readings taken where the pages are silent or disagree, each with the
+ * passage it rests on:
+ *   - A is diagonal, one value per (channel, state): A[d][n] ("Ayrık Zamana
+ *     Geçiş" writes exp(Delta A) and (Delta A)^-1 as matrix functions; with a
+ *     diagonal A they act state by state).  The discretised quantities are
+ *     then per state: Abar_n = exp(Delta A_n) and
  *     Bbar_n = (Delta A_n)^-1 (exp(Delta A_n) - 1) Delta B_n.
  *   - Delta is per (batch, token, channel); B_t and C_t are per (batch, token,
- *     state) and shared by every channel.
- *   - The discrete output keeps the D x_t skip term of the continuous form:
- *     y_t = C_t . h_t + D_d x_t, with h_t the state AFTER the update at t.
- *   - The scan starts from h = 0 unless an initial state is given.
- *   - Delta A = 0 (outside the stable domain A < 0) uses the limit
- *     (e^z - 1)/z -> 1, i.e. Bbar = Delta B.
+ *     state) and shared by every channel ("Mamba'nın Yeniliği: Selective SSM"
+ *     lists B, C and Delta as the quantities computed from the input; A is
+ *     not among them).
+ *   - The discrete output keeps the D x_t skip term of the continuous form of
+ *     "State Space Model Temelleri": y_t = C_t . h_t + D_d x_t, with h_t the
+ *     state AFTER the update at t (the order in which "Ayrık Zamana Geçiş"
+ *     writes the two equations).
+ *   - The scan starts from h = 0 unless an initial state is given (no page
+ *     states an initial state).
+ *   - Delta A = 0 lies outside the stable domain A < 0 ("Sınırlılıklar ve
+ *     Açık Sorular"); there the limit (e^z - 1)/z -> 1 is used, i.e.
+ *     Bbar = Delta B.
  *
  * Layouts (row-major, last index fastest):
  *   u, delta, y   : [batch][len][channels]
@@ -173,7 +181,8 @@ int oracle_state_update(double *state, const double *x, const double *delta,
  * The Mamba-3 page (bitig.info, section "Geliştirilmiş Ayrıklaştırma
  * Şeması") says Mamba-1 and Mamba-2 discretised the continuous system with
  * "the Euler method" and Mamba-3 with the trapezoidal rule, and gives no
- * formula for either.  Readings (listed in the design notes):
+ * formula for either.  Readings taken (the plainest forms that keep the
+ * transition exp(Delta A) of "Ayrık Zamana Geçiş"):
  *   method 1, exponential Euler: the state transition stays exp(Delta A)
  *     (as in the zero-order hold of "Ayrık Zamana Geçiş"), the input term is
  *     taken to first order, Bbar = Delta B:

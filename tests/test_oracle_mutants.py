@@ -46,6 +46,9 @@ MUTANTS = {
     "backward_adjoint_not_decayed": ("lam[n] *= r;", "(void)r;"),
     "backward_dc_from_previous_state": ("dC[k * nstate + n] += g * ht;", "dC[k * nstate + n] += g * hprev;"),
     "backward_psi_sign": ("return (z * exp(z) - expm1(z)) / (z * z);", "return (z * exp(z) + expm1(z)) / (z * z);"),
+    "backward_psi_series_coefficient": ("1.0 / 8.0 + z / 30.0", "1.0 / 6.0 + z / 30.0"),
+    "backward_psi_series_cubic_term": ("1.0 / 8.0 + z / 30.0", "1.0 / 8.0 + z / 24.0"),
+    "backward_psi_series_range": ("if (fabs(z) < 1e-3)", "if (fabs(z) < 1e-1)"),
     "backward_db_missing_x": ("dB[k * nstate + n] += lam[n] * x * phi * dt;", "dB[k * nstate + n] += lam[n] * phi * dt;"),
     "backward_ddelta_missing_a": ("ddt += lam[n] * r * (a * hprev + bn * x);", "ddt += lam[n] * r * (hprev + bn * x);"),
     "backward_adjoint_before_output": ("lam[n] += C[k * nstate + n] * g;           /* lam_t                       */",

@@ -429,6 +429,36 @@ def test_backward_matches_finite_differences(oracle_lib):
         np.testing.assert_allclose(g[name], fd, rtol=2e-6, atol=1e-8, err_msg=name)
 
 
+def _dbbar_da_series(dt, a, terms=40):
+    """d/dA of (exp(dt A) - 1)/A from the power series of exp, term by term:
+    (e^{dt A} - 1)/A = sum_{k>=1} dt^k A^{k-1}/k!, so its derivative is
+    sum_{k>=2} (k-1) dt^k A^{k-2}/k!.  No closed form, no psi()."""
+    total, fact = 0.0, 1.0
+    for k in range(1, terms + 1):
+        fact *= k
+        if k >= 2:
+            total += (k - 1) * dt ** k * a ** (k - 2) / fact
+    return total
+
+
+@pytest.mark.parametrize("dt, a", [(1e-3, -1e-3), (1e-3, -0.1), (1e-3, -0.9), (1e-3, -5.0), (0.05, -1.0)])
+def test_backward_da_small_z(oracle_lib, dt, a):
+    """One token from h = 0: dA comes from d Bbar / dA alone, at |Delta A| from
+    1e-6 to 5e-2, on both sides of the oracle's switch to a series for small
+    |z|.  Reference: the power series of exp differentiated term by term."""
+    rng = np.random.default_rng(24)
+    N = 3
+    u = np.array([[[0.7]]])
+    delta = np.array([[[dt]]])
+    A = np.full((1, N), a) * np.array([[1.0, 1.5, 2.0]])
+    B = rng.standard_normal((1, 1, N))
+    C = rng.standard_normal((1, 1, N))
+    dy = np.array([[[1.3]]])
+    g = oracle_lib.scan_backward(u, delta, A, B, C, np.zeros(1), dy)
+    ref = np.array([1.3 * C[0, 0, n] * B[0, 0, n] * 0.7 * _dbbar_da_series(dt, A[0, n]) for n in range(N)])
+    np.testing.assert_allclose(g["dA"][0], ref, rtol=1e-12, atol=0)
+
+
 def test_backward_lti_du_is_correlation_with_kernel(oracle_lib):
     """Constant Delta, B, C: y = K * x + D x, so du_t = sum_k K_k dy_{t+k} + D dy_t."""
     rng = np.random.default_rng(22)
