@@ -3,23 +3,29 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one selective scan (discretise, recurrence, output, final state)
-over the mid workload: batch 8, length 2048, 3072 channels, 16 states, bf16
-inputs/outputs with fp32 state and arithmetic.  Inputs stay resident in HBM
-and are larger than L2 (305 MB per step), so no L2 flush is needed between
+over the long-context workload, the largest single-GPU configuration: batch
+1, length 1,048,576, 2048 channels, 16 states, bf16 inputs/outputs with fp32
+state and arithmetic (12.95 GB of algorithmic traffic per step).  Inputs stay
+resident in HBM and are far larger than L2, so no L2 flush is needed between
 steps.  Timing is by CUDA events on the launching stream; for N > 1 (one
 process per GPU under torchrun) every rank runs its own independent
 workload, there is no collective on the data path, and the time is the max
 over ranks.
 
 Also reported on the same line:
-  roofline   the scan kernel against its binding roof (the FP32 FMA pipe) and,
-             under "hbm", its algorithmic HBM bytes against the measured copy
-             bandwidth
+  roofline   the scan call's algorithmic HBM bytes against the measured copy
+             bandwidth (the metric's roof), with the FP32 FMA pipe under "alu"
+  configs    every configuration of the workload list: tiny fp32, mid, large,
+             long (the headline) and the decode chain, each with its time,
+             token-channels/s and HBM fraction
+  length_sweep  ns per token-channel of the long workload's generator for
+             L = 2^14 .. 2^20 (linear scaling in length)
   e2e        the same metric through the public API from pinned host buffers,
              host<->device copies of each step's inputs and outputs included
   decode     the single-token state update on 256 x 5120 x 16 states, 1000
              steps with fresh inputs, captured in a CUDA graph
-  cpu_baseline  the fp64 CPU oracle on a bounded sample of the same workload
+  variants, ssd  the scan's options and Mamba-2's scalar-A scan on the mid shape
+  cpu_baseline  the fp64 CPU oracle on a strided channel subset of the workload
   clocks     SM clock and clock-event reasons sampled during the timed region
 """
 from __future__ import annotations
@@ -50,16 +56,18 @@ FLOP_PER_TOKEN_CHANNEL = 4      # skip term and output scaling
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mid_bf16")
+    ap.add_argument("--workload", default="long_bf16")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the timings of the scan's options (general A, other discretisations, state counts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration timings")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the length sweep of the line")
     ap.add_argument("--no-ssd", action="store_true", help="skip Mamba-2's scalar-A scan (state space duality) leg")
     ap.add_argument("--only-backward", action="store_true",
                     help="run only the backward on the workload's shape (steps = timed calls) and print its object")
@@ -266,40 +274,6 @@ def decode_bytes_per_step(w) -> int:
 
 # --- CPU oracle baseline -------------------------------------------------------------------
 
-def oracle_sample_rate(inp, w, budget_s: float, max_rows=None):
-    """tc/s of the fp64 oracle over whole (batch, channel) rows of the workload,
-    growing the sample until it takes budget_s seconds or covers every row."""
-    import numpy as np
-    import torch
-
-    import oracle
-    orc = oracle.get()
-    total_rows = w.batch * w.channels
-    cap = total_rows if max_rows is None else min(total_rows, max_rows)
-    rows = min(cap, 64)
-    best = None
-    while True:
-        per_b = max(1, rows // w.batch)
-        nb = min(w.batch, max(1, rows // per_b))
-        ch = torch.arange(per_b, device=inp["u"].device)
-        u = inp["u"][:nb].index_select(2, ch).to(torch.float64).cpu().numpy()
-        dl = inp["delta"][:nb].index_select(2, ch).to(torch.float64).cpu().numpy()
-        A = inp["A"].index_select(0, ch).to(torch.float64).cpu().numpy()
-        D = inp["D"].index_select(0, ch).to(torch.float64).cpu().numpy()
-        B = inp["B"][:nb].to(torch.float64).cpu().numpy()
-        C = inp["C"][:nb].to(torch.float64).cpu().numpy()
-        t0 = time.perf_counter()
-        orc.scan(u, dl, A, B, C, D)
-        dt = time.perf_counter() - t0
-        tc = nb * per_b * w.length
-        best = {"value": tc / dt, "rows": nb * per_b, "seconds": dt, "tc": tc}
-        if dt >= budget_s or nb * per_b >= cap:
-            break
-        rows = min(cap, max(rows * 2, int(rows * budget_s / max(dt, 1e-3) * 1.1)))
-    del u, dl, B, C
-    return best, orc.max_threads()
-
-
 def oracle_single_thread_tiny(budget_s: float = 1.0) -> dict:
     """tc/s of the fp64 oracle on one host thread over the tiny fp32 workload."""
     import oracle
@@ -319,6 +293,128 @@ def oracle_single_thread_tiny(budget_s: float = 1.0) -> dict:
 
 
 # --- our implementation ---------------------------------------------------------------
+
+def time_calls(fn, stream, dist, world, reps: int, warmup: int = 3) -> float:
+    """Mean device time of one call (ms), CUDA events on the launching stream
+    around each call, max over ranks."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    barrier(dist, world)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return max_over_ranks(dist, world, statistics.mean(a.elapsed_time(b) for a, b in ev))
+
+
+def scan_caller(lib, m, inp, y, hf, w, length, stream):
+    """One mamba_selective_scan call over the first `length` tokens of the
+    workload's tensors (contiguous prefixes for batch 1)."""
+    dtc = m.dtype_code(w.torch_dtype)
+    ptrs = [inp[k].data_ptr() for k in ("u", "delta", "A", "B", "C", "D")] + [y.data_ptr(), hf.data_ptr()]
+    sh = stream.cuda_stream
+
+    def call():
+        st = lib.mamba_selective_scan(*ptrs, w.batch, length, w.channels, w.nstate, dtc, sh)
+        if st != 0:
+            raise m.MambaError(st, "mamba_selective_scan")
+    return call
+
+
+def hbm_entry(nbytes: int, ms: float, hbm_peak: float) -> dict:
+    ach = nbytes / (ms * 1e-3) / 1e9
+    return {"achieved_gbs": round(ach, 1), "frac": round(ach / hbm_peak, 4), "algorithmic_bytes": nbytes}
+
+
+def run_configs(args, headline, dev, stream, dist, world, rank, hbm_peak, decode_res):
+    """Time, token-channels/s and HBM fraction of every configuration of the
+    workload list; the headline's own figures are reused, not re-measured."""
+    import torch
+
+    from selective_state_space_29_b200 import mamba_ssm as m
+    from selective_state_space_29_b200 import workloads as wl
+    lib = m.library()
+    res = {}
+    reps = {"tiny_f32": 200, "mid_bf16": 50, "large_bf16": 20}
+    for name in ("tiny_f32", "mid_bf16", "large_bf16", "long_bf16"):
+        w = wl.SCAN_WORKLOADS[name]
+        if name == headline["name"]:
+            ms = headline["ms"]
+        else:
+            inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
+            y = torch.empty_like(inp["u"])
+            hf = torch.empty((w.batch, w.channels, w.nstate), device=dev, dtype=torch.float32)
+            ms = time_calls(scan_caller(lib, m, inp, y, hf, w, w.length, stream), stream, dist, world,
+                            reps.get(name, 5))
+            del inp, y, hf
+        tc = w.batch * w.length * w.channels
+        e = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
+             "shape": f"batch {w.batch}, len {w.length}, channels {w.channels}, state {w.nstate}, {w.dtype} I/O"}
+        e.update({"hbm_" + k: v for k, v in hbm_entry(scan_bytes(w), ms, hbm_peak).items()})
+        if name == "tiny_f32":
+            e["note"] = "16,384 token-channels: launch latency, not bandwidth, sets the time"
+        res[name] = e
+    if decode_res is not None:
+        r = decode_res["roofline"]
+        res["decode_bf16"] = {"ms_per_step": decode_res["ms_per_step"],
+                              "updates_per_s": decode_res["updates_per_s"],
+                              "hbm_achieved_gbs": r["achieved"], "hbm_frac": r["frac"],
+                              "hbm_algorithmic_bytes": r["algorithmic_bytes_per_launch"]}
+    return res
+
+
+def run_length_sweep_on(inp, y, hf, w, dev, stream, dist, world, steps: int = 20) -> dict:
+    """ns per token-channel of the long workload's generator over its first L
+    tokens, L = 2^14 .. len, on the already resident input."""
+    from selective_state_space_29_b200 import mamba_ssm as m
+    lib = m.library()
+    dtc = m.dtype_code(w.torch_dtype)
+    rows = []
+    L = 1 << 14
+    while L <= w.length:
+        reps = max(5, min(steps, int(2e9 // (w.channels * L))))
+        ms = time_calls(scan_caller(lib, m, inp, y, hf, w, L, stream), stream, dist, world, reps)
+        plan = m.mamba_scan_plan(w.batch, L, w.channels, w.nstate, 0, dtc)
+        rows.append({"len": L, "ms": round(ms, 5), "ns_per_tc": round(ms * 1e6 / (w.channels * L), 6),
+                     "reps": reps, "supers": int(plan.supers)})
+        L *= 2
+    v = [r["ns_per_tc"] for r in rows]
+    ref = v[-1]
+    return {"rows": rows, "workload": f"{w.name} generator, batch 1, {w.channels} channels, prefixes of one input",
+            "max_over_min_ns_per_tc": round(max(v) / min(v), 4),
+            "max_dev_from_longest": round(max(abs(x / ref - 1.0) for x in v), 4),
+            "linear_within_10pct": bool(all(abs(x / ref - 1.0) <= 0.10 for x in v))}
+
+
+def oracle_strided_rate(inp, w, stride: int, budget_s: float):
+    """tc/s of the fp64 oracle over every `stride`-th channel of batch row 0
+    (whole rows: per-channel independence makes each exact), growing the
+    number of channels until it takes budget_s seconds or covers the stride."""
+    import torch
+
+    import oracle
+    orc = oracle.get()
+    all_ch = list(range(0, w.channels, stride))
+    n = min(len(all_ch), 16)
+    while True:
+        ch = torch.tensor(all_ch[:n], device=inp["u"].device)
+        arrs = [inp["u"][:1].index_select(2, ch), inp["delta"][:1].index_select(2, ch),
+                inp["A"].index_select(0, ch), inp["B"][:1], inp["C"][:1], inp["D"].index_select(0, ch)]
+        arrs = [a.to(torch.float64).cpu().numpy() for a in arrs]
+        t0 = time.perf_counter()
+        orc.scan(*arrs)
+        dt = time.perf_counter() - t0
+        del arrs
+        if dt >= budget_s or n >= len(all_ch):
+            break
+        n = min(len(all_ch), max(2 * n, int(n * budget_s / max(dt, 1e-3))))
+    tc = n * w.length
+    return {"value": tc / dt, "rows": n, "seconds": dt, "tc": tc}, orc.max_threads()
+
 
 def run_ours(args):
     import torch
@@ -342,13 +438,7 @@ def run_ours(args):
     plan = m.mamba_scan_plan(w.batch, w.length, w.channels, w.nstate, 0, dtc)
     lib = m.library()
     stream = torch.cuda.current_stream(dev)
-    sh = stream.cuda_stream
-    ptrs = [inp[k].data_ptr() for k in ("u", "delta", "A", "B", "C", "D")] + [y.data_ptr(), hf.data_ptr()]
-
-    def step():
-        st = lib.mamba_selective_scan(*ptrs, w.batch, w.length, w.channels, w.nstate, dtc, sh)
-        if st != 0:
-            raise m.MambaError(st, "mamba_selective_scan")
+    step = scan_caller(lib, m, inp, y, hf, w, w.length, stream)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -380,7 +470,8 @@ def run_ours(args):
         raise RuntimeError("device error word set during the benchmark")
     clocks = sampler.summary()
 
-    # roofline of the scan kernel (per launch, from the per-call event timing)
+    # roofline of the scan call (per launch, from the per-call event timing):
+    # the metric's roof is HBM; the FP32 pipe figure is kept beside it
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     max_mhz = clocks.get("sm_max_mhz") or float(peaks.get("sm_max_mhz", 1965.0))
     alu_peak = sms * FMA_LANES_PER_SM * 2 * max_mhz * 1e6 / 1e12        # TFLOP/s
@@ -388,14 +479,17 @@ def run_ours(args):
     nbytes = scan_bytes(w)
     alu_ach = flops / (call_ms * 1e-3) / 1e12
     hbm_ach = nbytes / (call_ms * 1e-3) / 1e9
-    traffic = profiled_traffic("scan_chunks_kernel", args.workload)
-    roofline = {"bound": "alu", "achieved": round(alu_ach, 3), "peak": round(alu_peak, 3), "unit": "TFLOP/s",
-                "frac": round(alu_ach / alu_peak, 4), "traffic": traffic,
-                "peak_source": f"derived: {sms} SMs x {FMA_LANES_PER_SM} FP32 FMA/clk x 2 x {max_mhz:.0f} MHz",
-                "kernel": "scan_chunks_kernel", "call_ms": round(call_ms, 5),
-                "flop_per_launch": flops, "algorithmic_bytes_per_launch": nbytes,
-                "hbm": {"achieved": round(hbm_ach, 1), "peak": hbm_peak, "unit": "GB/s",
-                        "frac": round(hbm_ach / hbm_peak, 4), "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)"}}
+    roofline = {"bound": "hbm", "achieved": round(hbm_ach, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(hbm_ach / hbm_peak, 4),
+                "traffic": profiled_traffic("scan_chunks_kernel", args.workload),
+                "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)",
+                "kernel": "scan_chunks_kernel (timed per call: the call's pre-pass included)",
+                "call_ms": round(call_ms, 5), "algorithmic_bytes_per_launch": nbytes,
+                "bytes_per_tc": round(nbytes / tc, 4),
+                "alu": {"achieved": round(alu_ach, 3), "peak": round(alu_peak, 3), "unit": "TFLOP/s",
+                        "frac": round(alu_ach / alu_peak, 4), "flop_per_launch": flops,
+                        "peak_source": f"derived: {sms} SMs x {FMA_LANES_PER_SM} FP32 FMA/clk x 2 x "
+                                       f"{max_mhz:.0f} MHz"}}
 
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -403,10 +497,14 @@ def run_ours(args):
            "config": {"workload": f"{w.name}: batch {w.batch}, len {w.length}, channels {w.channels}, "
                                   f"state {w.nstate}, {w.dtype} I/O, fp32 state",
                       "batch": w.batch, "len": w.length, "channels": w.channels, "nstate": w.nstate,
-                      "io_dtype": w.dtype, "global_batch": w.batch * world,
+                      "io_dtype": w.dtype, "state_dtype": "f32", "global_batch": w.batch * world,
                       "l2": f"inputs larger than L2 ({nbytes / 1e6:.0f} MB per step), no flush",
                       "parallelism": f"independent workload per GPU x{world}", "plan": plan.as_dict()},
            "roofline": roofline, "gpu_launches": int(K * plan.kernels), "clocks": clocks}
+
+    # the long workload's length sweep, on the resident input (batch 1 only)
+    if not args.no_sweep and w.batch == 1 and w.length >= (1 << 15):
+        out["length_sweep"] = run_length_sweep_on(inp, y, hf, w, dev, stream, dist, world)
 
     # end to end through the public API from pinned host buffers, copies timed:
     # mamba_selective_scan_host (copies pipelined with the scan piece by
@@ -418,7 +516,7 @@ def run_ours(args):
         hf_host = torch.empty(hf.shape, dtype=hf.dtype).pin_memory()
         h2d = sum(v.numel() * v.element_size() for v in host.values())
         d2h = y_host.numel() * y_host.element_size() + hf_host.numel() * hf_host.element_size()
-        Ke = max(3, min(K, 30))
+        Ke = max(3, min(K, 30 if nbytes < 2e9 else 5))
 
         def e2e_step():
             m.mamba_selective_scan_host(host["u"], host["delta"], host["A"], host["B"], host["C"], host["D"],
@@ -452,28 +550,36 @@ def run_ours(args):
                       "call": "mamba_selective_scan_host (pinned host buffers, copies overlapped piecewise)",
                       "unpipelined": {"value": world * tc / (plain_ms * 1e-3), "ms_per_step": plain_ms,
                                       "call": "copies of whole tensors around mamba_selective_scan"}}
-        del host, dbuf
+        del host, dbuf, y_host, hf_host
 
-    # the scan's options on the same shape: general-A path, the other
-    # discretisations, other state counts (device-timed calls, events)
+    # CPU oracle on every 16th channel of the headline workload (rank 0, single GPU only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        best, cores = oracle_strided_rate(inp, w, stride=16, budget_s=15.0)
+        out["cpu_baseline"] = {"value": best["value"], "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": f"{best['rows']} channels (every 16th) of batch row 0 x {w.length} "
+                                         f"tokens of {w.name} ({best['seconds']:.1f} s, fp64)",
+                               "single_thread_tiny_f32": oracle_single_thread_tiny()}
+    headline = {"name": w.name, "ms": call_ms}
+    del inp, y, hf
+    torch.cuda.empty_cache()
+
+    # the scan's options and Mamba-2's scalar-A scan, on the mid shape
+    mid = wl.SCAN_WORKLOADS["mid_bf16"]
     if not args.no_variants:
-        out["variants"] = run_variants(w, dev, stream, dist, world, rank)
-
-    # Mamba-2's scalar-A scan in its chunked tensor-core form, on the same shape
+        out["variants"] = run_variants(mid, dev, stream, dist, world, rank)
     if not args.no_ssd:
         out["ssd"] = run_ssd(args, dev, stream, dist, world, rank, hbm_peak, hbm_src, peaks)
 
     # decode: 1000 single-token steps on 256 x 5120 x 16 states
+    decode_res = None
     if not args.no_decode:
-        out["decode"] = run_decode(args, dev, stream, dist, world, rank, hbm_peak, hbm_src)
+        decode_res = run_decode(args, dev, stream, dist, world, rank, hbm_peak, hbm_src)
+        out["decode"] = decode_res
 
-    # CPU oracle on a bounded sample (rank 0, single GPU only)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        best, cores = oracle_sample_rate(inp, w, budget_s=10.0)
-        out["cpu_baseline"] = {"value": best["value"], "unit": UNIT, "cores": cores, "kind": "oracle",
-                               "sample": f"{best['rows']} of {w.batch * w.channels} (batch, channel) rows x "
-                                         f"{w.length} tokens of {w.name} ({best['seconds']:.1f} s, fp64)",
-                               "single_thread_tiny_f32": oracle_single_thread_tiny()}
+    # every configuration of the workload list
+    if not args.no_configs:
+        out["configs"] = run_configs(args, headline, dev, stream, dist, world, rank, hbm_peak, decode_res)
+
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -772,31 +878,30 @@ def run_reference(args):
         return
     import torch
 
+    import oracle
     from selective_state_space_29_b200 import workloads as wl
     w = wl.SCAN_WORKLOADS[args.workload]
     inp = wl.scan_inputs(w, "cpu" if not torch.cuda.is_available() else "cuda")
-    # each step: whole rows of the workload, sized so K + W steps fit in about three minutes
+    # each step: whole (batch row 0, channel) rows, every 16th channel, as many
+    # as fit a step budget that keeps K + W steps within about three minutes
     budget = max(0.5, 180.0 / max(1, args.steps + args.warmup))
-    best, cores = oracle_sample_rate(inp, w, budget_s=budget)
-    rows = best["rows"]
-    import numpy as np
-    import oracle
+    best, cores = oracle_strided_rate(inp, w, stride=16, budget_s=budget)
+    n = best["rows"]
     orc = oracle.get()
-    per_b = max(1, rows // w.batch)
-    nb = min(w.batch, max(1, rows // per_b))
-    ch = torch.arange(per_b, device=inp["u"].device)
-    arrs = [inp["u"][:nb].index_select(2, ch), inp["delta"][:nb].index_select(2, ch),
-            inp["A"].index_select(0, ch), inp["B"][:nb], inp["C"][:nb], inp["D"].index_select(0, ch)]
+    ch = torch.arange(0, 16 * n, 16, device=inp["u"].device)
+    arrs = [inp["u"][:1].index_select(2, ch), inp["delta"][:1].index_select(2, ch),
+            inp["A"].index_select(0, ch), inp["B"][:1], inp["C"][:1], inp["D"].index_select(0, ch)]
     arrs = [a.to(torch.float64).cpu().numpy() for a in arrs]
+    del inp
     for _ in range(args.warmup):
         orc.scan(*arrs)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         orc.scan(*arrs)
     dt = (time.perf_counter() - t0) / max(1, args.steps)
-    tc = nb * per_b * w.length
+    tc = n * w.length
     value = tc / dt
-    sample = f"{nb * per_b} of {w.batch * w.channels} (batch, channel) rows x {w.length} tokens of {w.name} per step"
+    sample = f"{n} channels (every 16th) of batch row 0 x {w.length} tokens of {w.name} per step"
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -809,51 +914,18 @@ def run_reference(args):
 
 
 def run_length_sweep(args):
-    """Time per token·channel against sequence length: one input of the
-    long-context generator at the largest length, scanned over its first L
-    tokens (contiguous prefixes for batch 1)."""
+    """The length sweep alone (its object, one JSON line)."""
     import torch
 
-    from selective_state_space_29_b200 import mamba_ssm as m
     from selective_state_space_29_b200 import workloads as wl
-
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     w = wl.SCAN_WORKLOADS["long_bf16"]
     inp = wl.scan_inputs(w, dev)
     y = torch.empty_like(inp["u"])
     hf = torch.empty((w.batch, w.channels, w.nstate), device=dev, dtype=torch.float32)
-    lib = m.library()
-    dtc = m.dtype_code(w.torch_dtype)
-    stream = torch.cuda.current_stream(dev)
-    rows = []
-    L = 1 << 14
-    while L <= w.length:
-        def step():
-            st = lib.mamba_selective_scan(inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(),
-                                          inp["B"].data_ptr(), inp["C"].data_ptr(), inp["D"].data_ptr(),
-                                          y.data_ptr(), hf.data_ptr(), w.batch, L, w.channels, w.nstate, dtc,
-                                          stream.cuda_stream)
-            if st != 0:
-                raise m.MambaError(st, "mamba_selective_scan")
-        for _ in range(max(args.warmup, 3)):
-            step()
-        reps = max(5, min(args.steps, int(2e9 // (w.channels * L))))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        a.record(stream)
-        for _ in range(reps):
-            step()
-        b.record(stream)
-        torch.cuda.synchronize()
-        ms = a.elapsed_time(b) / reps
-        plan = m.mamba_scan_plan(w.batch, L, w.channels, w.nstate, 0, dtc)
-        rows.append({"len": L, "ms": round(ms, 5), "ns_per_tc": round(ms * 1e6 / (w.channels * L), 6),
-                     "reps": reps, "supers": int(plan.supers)})
-        L *= 2
-    v = [r["ns_per_tc"] for r in rows]
-    print(json.dumps({"length_sweep": rows, "workload": f"{w.name} generator, batch 1, {w.channels} channels",
-                      "max_over_min_ns_per_tc": round(max(v) / min(v), 4)}), flush=True)
+    res = run_length_sweep_on(inp, y, hf, w, dev, torch.cuda.current_stream(dev), None, 1, args.steps)
+    print(json.dumps({"length_sweep": res}), flush=True)
 
 
 def main():

@@ -382,11 +382,33 @@ const char *mamba_status_string(int status);
 int mamba_scan_supported_nstate(int64_t nstate);
 
 /*
- * Synchronises the current device, then returns the device error word
- * (MAMBA_OK if no bounded wait has run out since the last clear).  With
- * clear != 0 the word is reset to MAMBA_OK.
+ * The device error word of the current device: MAMBA_OK, or MAMBA_ERR_TIMEOUT
+ * when a bounded device wait has run out since the word was last cleared.
+ * The word is read (and, with clear != 0, reset to MAMBA_OK) by copies
+ * enqueued on `stream`, so it reflects every kernel enqueued on `stream`
+ * before the call; the call then waits for `stream` alone (it synchronises
+ * no other stream, unless `stream` is the legacy default stream, which is
+ * ordered with every blocking stream).  MAMBA_ERR_CUDA if a copy or the wait
+ * fails.
  */
-int mamba_get_device_error(int clear);
+int mamba_get_device_error(mamba_stream_t stream, int clear);
+
+/*
+ * Diagnostic: how many device scratch allocations (stream-ordered, from the
+ * library's pool or cudaMallocAsync) the library has made in this process.
+ * Lets a test show that a call allocated nothing.
+ */
+int64_t mamba_debug_scratch_allocations(void);
+
+/*
+ * Returns to the system the freed scratch that the library's memory pool on
+ * the current device keeps for later calls (up to 1 GiB; see
+ * mamba_selective_scan).  Scratch still in use by enqueued work stays.  The
+ * pool keeps freed memory because mapping it again on every call costs host
+ * time during which the GPU waits; a caller that wants the memory back
+ * between phases calls this.  MAMBA_OK, or MAMBA_ERR_CUDA.
+ */
+int mamba_trim_scratch_pool(void);
 
 /*
  * Diagnostic: enqueues one kernel that waits on a barrier nothing will ever

@@ -9,14 +9,14 @@
 //     lam_t      = C_t dy_t + r_{t+1} lam_{t+1}          (+ d h_final at the end)
 //     du_t       = sum_n lam_t (q / A_n) B_{t,n} + D dy_t
 //     dDelta_t   = sum_n lam_t r (A_n h_{t-1} + B_{t,n} x_t)
-//     dA_n      += lam_t (Delta_t r (h_{t-1} + B_{t,n} x_t / A_n) - q B_{t,n} x_t / A_n^2)
+//     dA_n      += lam_t (Delta_t r h_{t-1} + B_{t,n} x_t Delta_t^2 psi(z)),
+//                  psi(z) = (z e^z - (e^z - 1)) / z^2
 //     dB_{t,n}  += lam_t x_t q / A_n                      (summed over channels)
 //     dC_{t,n}  += dy_t h_t                               (summed over channels)
 //     dD        += dy_t x_t,        dh0 = r_0 lam_0
 //
-// (the dA term is d h_t / d A_n at fixed Delta, with the derivative of
-// (e^z - 1)/A_n written out; its two parts nearly cancel only when the term
-// itself is small, so the sum over tokens keeps fp32 accuracy).  With
+// (the dA term is d h_t / d A_n at fixed Delta; psi is evaluated by its
+// series where the closed form would cancel, see psi_f).  With
 // structured A (A[d,n] = (n+1) A[d,0]) the decays come from one exponential
 // per token and the forward kernel's decay chain.
 //
@@ -209,6 +209,21 @@ __device__ __forceinline__ void decays(float dt, const float (&An)[NS], float (&
 #pragma unroll
     for (int n = 0; n < NS; ++n) q[n] = expm1_small(dt * An[n]);
   }
+}
+
+// psi(z) = (z e^z - (e^z - 1)) / z^2 = d/dA [(e^{Delta A} - 1)/A] / Delta^2,
+// given q = e^z - 1.  The closed form cancels for small |z| (relative error
+// about 2 eps / |z|), so |z| <= 1/4 takes the series
+// sum_k (k+1) z^k / (k+2)! through z^6 (truncation below 3e-9 relative).
+__device__ __forceinline__ float psi_f(float z, float q) {
+  float s = fmaf(z, 1.0f / 5760.0f, 1.0f / 840.0f);
+  s = fmaf(z, s, 1.0f / 144.0f);
+  s = fmaf(z, s, 1.0f / 30.0f);
+  s = fmaf(z, s, 1.0f / 8.0f);
+  s = fmaf(z, s, 1.0f / 3.0f);
+  s = fmaf(z, s, 0.5f);
+  const float closed = (fmaf(z, q, z) - q) / (z * z);
+  return fabsf(z) <= 0.25f ? s : closed;
 }
 
 // A work item's channel group has structured A (every lane, exact fp32 test)
@@ -434,8 +449,8 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
         lam[n] = fmaf(cv[n], gy, lam[n]);
         du = fmaf(lam[n], qa * bv[n], du);
         ddt = fmaf(lam[n] * r, fmaf(An[n], hp[n], bx), ddt);
-        // d h_t / d A_n = Delta r (h_{t-1} + B x / A_n) - q B x / A_n^2
-        dA[n] = fmaf(lam[n], fmaf(dt * r, fmaf(bx, iA[n], hp[n]), -qa * iA[n] * bx), dA[n]);
+        // d h_t / d A_n = Delta r h_{t-1} + B x Delta^2 psi(Delta A_n)
+        dA[n] = fmaf(lam[n], fmaf(dt * r, hp[n], bx * (dt * dt) * psi_f(dt * An[n], q[n])), dA[n]);
         red[n] = lam[n] * x * qa;                     // dB_{t,n} part
         lam[n] *= r;
         h[n] = hp[n];

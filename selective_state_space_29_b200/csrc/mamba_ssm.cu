@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 #include <mutex>
@@ -62,7 +63,10 @@ constexpr uint64_t kPoolKeepBytes = uint64_t(1) << 30;
 std::mutex g_pool_mu;
 cudaMemPool_t g_pool[64] = {};
 
+std::atomic<int64_t> g_scratch_allocs{0};  // scratch allocations made by this process
+
 cudaError_t scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
+  g_scratch_allocs.fetch_add(1);
   cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
   if (cudaStreamIsCapturing(stream, &cs) != cudaSuccess) return cudaErrorUnknown;
   int dev = 0;
@@ -1061,15 +1065,35 @@ int mamba_selective_scan_complex(const void* u, const void* delta, const float* 
   }
 }
 
-int mamba_get_device_error(int clear) {
-  if (cudaDeviceSynchronize() != cudaSuccess) return MAMBA_ERR_CUDA;
+int mamba_get_device_error(mamba_stream_t stream_, int clear) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  // the read (and the clear) are ordered after the work already on `stream`;
+  // only that stream is waited for
   int v = 0;
-  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return MAMBA_ERR_CUDA;
+  if (cudaMemcpyFromSymbolAsync(&v, g_device_error, sizeof(int), 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+    return MAMBA_ERR_CUDA;
   if (clear) {
-    const int z = 0;
-    if (cudaMemcpyToSymbol(g_device_error, &z, sizeof(int)) != cudaSuccess) return MAMBA_ERR_CUDA;
+    static const int kZero = 0;
+    if (cudaMemcpyToSymbolAsync(g_device_error, &kZero, sizeof(int), 0, cudaMemcpyHostToDevice, stream) !=
+        cudaSuccess)
+      return MAMBA_ERR_CUDA;
   }
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return MAMBA_ERR_CUDA;
   return v;
+}
+
+int64_t mamba_debug_scratch_allocations(void) { return g_scratch_allocs.load(); }
+
+int mamba_trim_scratch_pool(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MAMBA_ERR_CUDA;
+  cudaMemPool_t pool = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_pool_mu);
+    pool = g_pool[dev];
+  }
+  if (pool && cudaMemPoolTrimTo(pool, 0) != cudaSuccess) return MAMBA_ERR_CUDA;
+  return MAMBA_OK;
 }
 
 int mamba_debug_expire_wait(int64_t limit_ns, mamba_stream_t stream_) {

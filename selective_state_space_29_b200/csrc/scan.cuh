@@ -199,9 +199,15 @@ __device__ __forceinline__ float expm1_small(float z) {
   return fabsf(z) <= 0.25f ? poly : viaexp2;
 }
 
-// exp(z) - 1 from the hardware exp2 (no branch): absolute error about 1e-7,
-// i.e. a relative error below 1e-4 once |z| > 1e-3.  Used for bf16 data.
-__device__ __forceinline__ float expm1_fast(float z) { return ex2_approx(z * 1.4426950408889634f) - 1.0f; }
+// exp(z) - 1 for z <= 0 without a branch, for bf16 data: the hardware exp2
+// minus one (absolute error about 2.4e-7, so below 7.7e-6 relative once
+// |z| >= 1/32), and for |z| < 1/32 the series z + z^2/2 + z^3/6 (truncation
+// below 1.3e-6 relative there).  Both are evaluated and one is selected.
+__device__ __forceinline__ float expm1_series3(float z) { return z * fmaf(z, fmaf(z, 1.0f / 6.0f, 0.5f), 1.0f); }
+__device__ __forceinline__ float expm1_fast(float z) {
+  const float viaexp2 = ex2_approx(z * 1.4426950408889634f) - 1.0f;
+  return fabsf(z) < 0.03125f ? expm1_series3(z) : viaexp2;
+}
 
 __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b); }
 
@@ -308,8 +314,9 @@ __device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const T
 // Rows [0, rows) of one tile, structured A, for one lane: its channel column
 // `su`/`sdl` (stride 32) and all its states.  FULL: store y (predicated on
 // the channel being inside the tensor); otherwise accumulate sum(Delta).
-// FASTQ (bf16 data): r from the hardware exp2 of Delta A_0 log2(e), q = r - 1;
-// otherwise q from the accurate expm1 and r = 1 + q.  Two tokens per step:
+// FASTQ (bf16 data): r from the hardware exp2 of Delta A_0 log2(e), q = r - 1
+// (a short series for |Delta A_0| < 1/32); otherwise q from the accurate
+// expm1 and r = 1 + q.  Two tokens per step:
 // their decay chains are independent work for the scheduler while the state
 // updates wait on each other.
 template <typename TIO, int NS, int TILE, bool FULL, bool FASTQ>
@@ -320,8 +327,12 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
   const float a0l = a0 * 1.4426950408889634f;
   auto chain = [&](float dt, float2 (&e)[NS / 2]) {
     if constexpr (FASTQ) {
+      // r from the hardware exp2; q = r - 1 from the same value, or from the
+      // series where that subtraction would lose the small |Delta A_0|
       const float r = ex2_approx(dt * a0l);
-      decay_chain<NS>(r, r - 1.0f, e);
+      const float z = dt * a0;
+      const float q = fabsf(z) < 0.03125f ? expm1_series3(z) : r - 1.0f;
+      decay_chain<NS>(r, q, e);
     } else {
       const float q = expm1_small(dt * a0);
       decay_chain<NS>(1.0f + q, q, e);
@@ -384,7 +395,7 @@ __device__ __forceinline__ void tile_general(const TIO* su, const TIO* sdl, cons
     for (int k = 0; k < NS; ++k) {
       zv[k] = dt * (kA[k] * 0.69314718055994531f);  // Delta A_n
       if constexpr (sizeof(TIO) == 4) ev[k] = expm1_small(zv[k]);  // fp32 data: accurate expm1
-      else ev[k] = ex2_approx(dt * kA[k]) - 1.0f;
+      else ev[k] = expm1_fast(zv[k]);
     }
     float crow[NS];
 #pragma unroll

@@ -62,7 +62,9 @@ _SIGNATURES = [
      [_I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ScanPlan)]),
     ("mamba_status_string", ctypes.c_char_p, [ctypes.c_int]),
     ("mamba_scan_supported_nstate", ctypes.c_int, [_I64]),
-    ("mamba_get_device_error", ctypes.c_int, [ctypes.c_int]),
+    ("mamba_get_device_error", ctypes.c_int, [_P, ctypes.c_int]),
+    ("mamba_debug_scratch_allocations", ctypes.c_int64, []),
+    ("mamba_trim_scratch_pool", ctypes.c_int, []),
     ("mamba_debug_expire_wait", ctypes.c_int, [_I64, _P]),
 ]
 
@@ -220,8 +222,16 @@ def mamba_scan_supported_nstate(nstate: int) -> bool:
     return bool(library().mamba_scan_supported_nstate(int(nstate)))
 
 
-def mamba_get_device_error(clear: bool = False) -> int:
-    return int(library().mamba_get_device_error(1 if clear else 0))
+def mamba_get_device_error(clear: bool = False, stream=None) -> int:
+    return int(library().mamba_get_device_error(_stream(stream), 1 if clear else 0))
+
+
+def mamba_debug_scratch_allocations() -> int:
+    return int(library().mamba_debug_scratch_allocations())
+
+
+def mamba_trim_scratch_pool():
+    _check(library().mamba_trim_scratch_pool(), "mamba_trim_scratch_pool")
 
 
 def mamba_debug_expire_wait(limit_ns: int, stream=None):

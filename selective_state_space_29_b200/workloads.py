@@ -174,6 +174,15 @@ def a_matrix(channels: int, nstate: int, mode: str, gen, device) -> torch.Tensor
     if mode == "state":
         scale = 1.0 + 0.1 * torch.rand((channels, nstate), generator=gen, device=device, dtype=torch.float32)
         return (-(ramp * scale)).contiguous()
+    if mode == "small":
+        # slow decay: |A[d, 0]| log-uniform in [1e-3, 1e-2] per channel, A[d, n] = (n+1) A[d, 0]
+        scale = torch.exp(torch.empty((channels, 1), device=device, dtype=torch.float32)
+                          .uniform_(math.log(1e-3), math.log(1e-2), generator=gen))
+        return (-(ramp * scale)).contiguous()
+    if mode == "small_state":
+        # slow decay without structure across n: |A[d, n]| log-uniform in [1e-3, 1e-2]
+        return (-torch.exp(torch.empty((channels, nstate), device=device, dtype=torch.float32)
+                           .uniform_(math.log(1e-3), math.log(1e-2), generator=gen))).contiguous()
     if mode == "random":
         # arbitrary negative values over three decades, no structure across n
         return (-torch.exp(torch.empty((channels, nstate), device=device, dtype=torch.float32)

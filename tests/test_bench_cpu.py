@@ -21,6 +21,24 @@ def test_scan_bytes_of_the_mid_workload():
     assert 300e6 < bench.scan_bytes(w) < 310e6       # ~6.06 bytes per token-channel
 
 
+def test_scan_bytes_of_the_long_workload():
+    w = wl.SCAN_WORKLOADS["long_bf16"]
+    tc = w.batch * w.length * w.channels
+    assert tc == 2_147_483_648
+    # 3 x 2 bytes per token-channel, B and C 64 bytes per token, A, D, final state
+    want = 6 * tc + 64 * w.length + w.channels * 17 * 4 + w.channels * 16 * 4
+    assert bench.scan_bytes(w) == want
+    assert 12.95e9 < bench.scan_bytes(w) < 12.96e9
+
+
+def test_bench_defaults_to_the_largest_single_gpu_config(monkeypatch):
+    monkeypatch.setattr("sys.argv", ["bench.py"])
+    args = bench.parse_args()
+    assert args.workload == "long_bf16"
+    big = max(wl.SCAN_WORKLOADS.values(), key=bench.scan_bytes)
+    assert big.name == args.workload
+
+
 def test_ssd_bytes_of_the_mid_workload():
     w = wl.SSD_WORKLOADS["ssd_mid_bf16"]
     x_and_y = 2 * w.batch * w.length * w.channels * 2
