@@ -7,7 +7,8 @@ numpy arrays across ctypes.  It follows the zero-order-hold discretisation and
 recurrence of "Mamba SSM Nedir? Transformer Alternatifi Rehberi (2026)",
 sections "State Space Model Temelleri" and "Ayrık Zamana Geçiş", and, as
 options, the exponential-Euler and trapezoidal discretisations that the
-Mamba-3 page names in "Geliştirilmiş Ayrıklaştırma Şeması".
+Mamba-3 page names in "Geliştirilmiş Ayrıklaştırma Şeması"; also the
+complex-valued and the multi-input multi-output (MIMO) state of that page.
 """
 from __future__ import annotations
 
@@ -39,6 +40,8 @@ class Oracle:
         self._lib.oracle_state_update.argtypes = [_c_f64p] * 8 + [_i64] * 3 + [ctypes.c_int]
         self._lib.oracle_scan_complex.restype = ctypes.c_int
         self._lib.oracle_scan_complex.argtypes = [_c_f64p] * 10 + [_i64] * 4 + [ctypes.c_int]
+        self._lib.oracle_scan_mimo.restype = ctypes.c_int
+        self._lib.oracle_scan_mimo.argtypes = [_c_f64p] * 9 + [_i64] * 5 + [ctypes.c_int]
         self._lib.oracle_max_threads.restype = ctypes.c_int
 
     @staticmethod
@@ -139,6 +142,28 @@ class Oracle:
             raise RuntimeError(f"oracle_scan_complex failed ({rc})")
         return y, hf
 
+    def scan_mimo(self, u, delta, A, B, C, D=None, h0=None, want_y=True, nthreads=0):
+        """Multi-input multi-output scan (the Mamba-3 page, "MIMO Mekanizmasının
+        İşleyişi"; the reading is in ssm_oracle.c).  u: (batch, len, ranks,
+        channels); delta: (batch, len, channels); B, C: (batch, len, ranks,
+        nstate); A: (channels, nstate); D: (channels,) or None; h0: (batch,
+        channels, nstate) or None.  Returns (y, h_final), y shaped like u."""
+        u, delta, A, B, C, D, h0 = map(self._f64, (u, delta, A, B, C, D, h0))
+        batch, length, ranks, channels = u.shape
+        nstate = A.shape[1]
+        assert delta.shape == (batch, length, channels) and A.shape == (channels, nstate)
+        assert B.shape == (batch, length, ranks, nstate) and C.shape == B.shape
+        assert D is None or D.shape == (channels,)
+        assert h0 is None or h0.shape == (batch, channels, nstate)
+        y = np.empty_like(u) if want_y else None
+        hf = np.empty((batch, channels, nstate), dtype=np.float64)
+        rc = self._lib.oracle_scan_mimo(self._ptr(u), self._ptr(delta), self._ptr(A), self._ptr(B), self._ptr(C),
+                                        self._ptr(D), self._ptr(h0), self._ptr(y), self._ptr(hf), batch, length,
+                                        channels, nstate, ranks, int(nthreads))
+        if rc != 0:
+            raise RuntimeError(f"oracle_scan_mimo failed ({rc})")
+        return y, hf
+
     # --- Mamba-2's restricted form (state space duality) -----------------
     @staticmethod
     def _ssd_channel_head(channels: int, headdim: int) -> np.ndarray:
@@ -203,3 +228,7 @@ def ssd_scan(*args, **kwargs):
 
 def scan_complex(*args, **kwargs):
     return get().scan_complex(*args, **kwargs)
+
+
+def scan_mimo(*args, **kwargs):
+    return get().scan_mimo(*args, **kwargs)

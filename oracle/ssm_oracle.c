@@ -480,6 +480,113 @@ int oracle_scan_complex(const double *u, const double *delta, const double *A_re
     return status;
 }
 
+/* ------------------------------------------------------------------------
+ * Multi-input multi-output (MIMO) state update.
+ *
+ * The Mamba-3 page (bitig.info), sections "MIMO Mekanizmasının İşleyişi"
+ * and "Seçici Durum Güncellemesindeki İyileştirmeler", says that MIMO
+ * updates the hidden state once per step for several outputs at once,
+ * widens what the state holds without enlarging the state transition
+ * matrix or adding parameters, and gives every output channel its own
+ * selective gate deciding how much of the state that output uses; it
+ * prints no formula.  Reading taken (the plainest one that keeps the
+ * zero-order hold of "Ayrık Zamana Geçiş" as written, with B a matrix):
+ * per channel d the continuous system of "State Space Model Temelleri" has
+ * R inputs and R outputs,
+ *     h'(t) = A h(t) + B x(t),   y(t) = C h(t) + D x(t),
+ * x(t), y(t) in R^R, B_t in R^{N x R} (columns B_t^(r)), C_t in R^{R x N}
+ * (rows C_t^(r): the per-output selective gates), D = D_d I; A stays the
+ * diagonal N x N transition with one step Delta_t per (token, channel), so
+ *     Abar = exp(Delta A),
+ *     Bbar x = (Delta A)^-1 (exp(Delta A) - I) Delta B x
+ *            = sum_r (Delta A)^-1 (exp(Delta A) - I) Delta B^(r) x^(r),
+ *     h_t = Abar h_{t-1} + sum_r Bbar^(r) x_t^(r),
+ *     y_t^(r) = C_t^(r) . h_t + D_d x_t^(r).
+ * B and C are per (batch, token, input/output r, state), shared by all
+ * channels, as in the single-input scan.  With R = 1 this is oracle_scan,
+ * operation for operation.
+ *
+ * Layouts: u, y [batch][len][ranks][channels]; delta [batch][len][channels];
+ * B, C [batch][len][ranks][nstate]; A [channels][nstate]; D [channels] or
+ * NULL; h0, h_final [batch][channels][nstate] (h0 may be NULL).
+ * ------------------------------------------------------------------------ */
+static void scan_row_mimo(const double *u, const double *delta, const double *A_row,
+                          const double *B, const double *C, double D_d, int has_D,
+                          double *y, double *h, int64_t len, int64_t channels, int64_t nstate,
+                          int64_t ranks)
+{
+    for (int64_t t = 0; t < len; ++t) {
+        const double dt = delta[t * channels];
+        const double *xt = u + t * ranks * channels;         /* x_t^(r) = xt[r * channels] */
+        const double *Bt = B + t * ranks * nstate;           /* B_t^(r)[n] = Bt[r * nstate + n] */
+        const double *Ct = C + t * ranks * nstate;
+        for (int64_t n = 0; n < nstate; ++n) {
+            double abar = 1.0, in = 0.0;
+            for (int64_t r = 0; r < ranks; ++r) {
+                double bbar;
+                zoh_discretise(dt, A_row[n], Bt[r * nstate + n], &abar, &bbar);
+                in += bbar * xt[r * channels];               /* sum_r Bbar^(r) x_t^(r) */
+            }
+            h[n] = abar * h[n] + in;                         /* h_t = Abar h_{t-1} + Bbar x_t */
+        }
+        for (int64_t r = 0; r < ranks; ++r) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < nstate; ++n)
+                acc += Ct[r * nstate + n] * h[n];            /* C_t^(r) . h_t */
+            if (has_D)
+                acc += D_d * xt[r * channels];               /* + D x_t^(r)   */
+            if (y)
+                y[(t * ranks + r) * channels] = acc;
+        }
+    }
+}
+
+int oracle_scan_mimo(const double *u, const double *delta, const double *A,
+                     const double *B, const double *C, const double *D,
+                     const double *h0, double *y, double *h_final,
+                     int64_t batch, int64_t len, int64_t channels, int64_t nstate, int64_t ranks,
+                     int nthreads)
+{
+    if (batch < 0 || len < 0 || channels < 0 || nstate <= 0 || ranks <= 0)
+        return -1;
+    if ((len > 0 && (!u || !delta || !B || !C)) || !A)
+        return -1;
+    int64_t rows = batch * channels;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+    int status = 0;
+#pragma omp parallel
+    {
+        double *h = (double *)malloc(sizeof(double) * (size_t)nstate);
+        if (!h) {
+#pragma omp atomic write
+            status = -1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t r = 0; r < rows; ++r) {
+            if (!h)
+                continue;
+            int64_t b = r / channels, d = r % channels;
+            for (int64_t n = 0; n < nstate; ++n)
+                h[n] = h0 ? h0[(b * channels + d) * nstate + n] : 0.0;
+            const size_t x0 = (size_t)(b * len) * (size_t)(ranks * channels) + (size_t)d;
+            const size_t bc0 = (size_t)(b * len) * (size_t)(ranks * nstate);
+            scan_row_mimo(len ? u + x0 : NULL, len ? delta + (size_t)(b * len) * (size_t)channels + (size_t)d : NULL,
+                          A + d * nstate, len ? B + bc0 : NULL, len ? C + bc0 : NULL, D ? D[d] : 0.0,
+                          D != NULL, (y && len) ? y + x0 : NULL, h, len, channels, nstate, ranks);
+            if (h_final)
+                for (int64_t n = 0; n < nstate; ++n)
+                    h_final[(b * channels + d) * nstate + n] = h[n];
+        }
+        free(h);
+    }
+    return status;
+}
+
 int oracle_max_threads(void)
 {
 #ifdef _OPENMP

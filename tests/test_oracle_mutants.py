@@ -2,7 +2,8 @@
 
 Each case below copies oracle/ssm_oracle.c, plants one mistake by text
 substitution (in every copy of the line), builds the copy on the CPU and runs
-every pin of test_oracle_pins.py and test_oracle_complex_pins.py against it: at
+every pin of test_oracle_pins.py, test_oracle_complex_pins.py and
+test_oracle_mimo_pins.py against it: at
 least one pin has to fail.
 """
 import os
@@ -13,6 +14,7 @@ import pytest
 import oracle
 from oracle import build as oracle_build
 from tests import test_oracle_complex_pins as complex_pins
+from tests import test_oracle_mimo_pins as mimo_pins
 from tests import test_oracle_pins as pins
 
 SRC = os.path.join(os.path.dirname(oracle.__file__), "ssm_oracle.c")
@@ -60,6 +62,14 @@ MUTANTS = {
     "complex_input_missing_division": ("(abar - 1.0) / z;", "(abar - 1.0);"),
     "complex_rotation_dropped": ("double complex abar = cexp(z);", "double complex abar = exp(creal(z));"),
     "complex_state_layout_swapped": ("h[n] = s0 ? s0[0] + I * s0[1] : 0.0;", "h[n] = s0 ? s0[1] + I * s0[0] : 0.0;"),
+    # the multi-input multi-output state
+    "mimo_input_sum_keeps_last_rank": ("in += bbar * xt[r * channels];", "in = bbar * xt[r * channels];"),
+    "mimo_output_gate_shared": ("acc += Ct[r * nstate + n] * h[n];", "acc += Ct[n] * h[n];"),
+    "mimo_input_column_mismatched": ("zoh_discretise(dt, A_row[n], Bt[r * nstate + n], &abar, &bbar);",
+                                     "zoh_discretise(dt, A_row[n], Bt[((r + 1) % ranks) * nstate + n], &abar, &bbar);"),
+    "mimo_skip_from_first_input": ("acc += D_d * xt[r * channels];", "acc += D_d * xt[0];"),
+    "mimo_input_rank_stride": ("in += bbar * xt[r * channels];", "in += bbar * xt[r];"),
+    "mimo_output_rank_layout": ("y[(t * ranks + r) * channels] = acc;", "y[(r * len + t) * channels] = acc;"),
 }
 
 def _pin_calls(module):
@@ -83,7 +93,7 @@ def _pin_calls(module):
     return calls
 
 
-PIN_CALLS = _pin_calls(pins) + _pin_calls(complex_pins)
+PIN_CALLS = _pin_calls(pins) + _pin_calls(complex_pins) + _pin_calls(mimo_pins)
 
 
 def test_every_pin_call_binds():
