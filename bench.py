@@ -67,6 +67,7 @@ def parse_args():
                     help="skip the timings of the scan's options (general A, other discretisations, state counts)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration timings")
+    ap.add_argument("--no-mimo", action="store_true", help="skip the multi-input multi-output leg")
     ap.add_argument("--no-sweep", action="store_true", help="skip the length sweep of the line")
     ap.add_argument("--no-ssd", action="store_true", help="skip Mamba-2's scalar-A scan (state space duality) leg")
     ap.add_argument("--only-backward", action="store_true",
@@ -569,6 +570,8 @@ def run_ours(args):
         out["variants"] = run_variants(mid, dev, stream, dist, world, rank)
     if not args.no_ssd:
         out["ssd"] = run_ssd(args, dev, stream, dist, world, rank, hbm_peak, hbm_src, peaks)
+    if not args.no_mimo:
+        out["mimo"] = run_mimo(dev, stream, dist, world, rank, hbm_peak)
 
     # decode: 1000 single-token steps on 256 x 5120 x 16 states
     decode_res = None
@@ -729,6 +732,85 @@ def run_ssd(args, dev, stream, dist, world, rank, hbm_peak, hbm_src, peaks):
                                     "peak_source": "measured bf16" if "bf16_tflops" in peaks else "fallback"}},
             "l2": f"inputs larger than L2 ({nb / 1e6:.0f} MB per call), no flush"}
         del inp, y, hf
+    return res
+
+
+def mimo_bytes(w) -> int:
+    """Algorithmic bytes of one multi-input multi-output scan call: R inputs
+    read and R outputs written per token and channel, Delta, the R rows of B
+    and C per token, A, D and the final state."""
+    es = 2 if w.dtype == "bf16" else 4
+    tc = w.batch * w.length * w.channels
+    return (2 * w.ranks * tc * es + tc * es + 2 * w.batch * w.length * w.ranks * w.nstate * es
+            + w.channels * (w.nstate + 1) * 4 + w.batch * w.channels * w.nstate * 4)
+
+
+def mimo_decode_bytes_per_step(batch, ranks, channels, nstate, es=2) -> int:
+    rows = batch * channels
+    return (2 * rows * nstate * 4 + (2 * ranks + 1) * rows * es + 2 * batch * ranks * nstate * es
+            + channels * (nstate + 1) * 4)
+
+
+def run_mimo(dev, stream, dist, world, rank, hbm_peak, reps: int = 20) -> dict:
+    """The multi-input multi-output scan on the mid shape with 4 inputs and
+    outputs per channel, and its single-token step on the decode shape
+    (256 x 5120 x 16 states, 4 inputs and outputs per row)."""
+    import torch
+
+    from selective_state_space_29_b200 import mamba_ssm as m
+    from selective_state_space_29_b200 import workloads as wl
+    lib = m.library()
+    w = wl.MIMO_WORKLOADS["mimo_mid_bf16"]
+    inp = wl.mimo_inputs(w, dev, seed=rank_seed(w.seed, rank))
+    y = torch.empty_like(inp["u"])
+    hf = torch.empty((w.batch, w.channels, w.nstate), device=dev, dtype=torch.float32)
+    dtc = m.dtype_code(w.torch_dtype)
+
+    def call():
+        st = lib.mamba_selective_scan_mimo(inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(),
+                                           inp["B"].data_ptr(), inp["C"].data_ptr(), inp["D"].data_ptr(), None,
+                                           y.data_ptr(), hf.data_ptr(), w.batch, w.length, w.ranks, w.channels,
+                                           w.nstate, 0, dtc, stream.cuda_stream)
+        if st != 0:
+            raise m.MambaError(st, "mamba_selective_scan_mimo")
+
+    ms = time_calls(call, stream, dist, world, reps)
+    tc = w.token_channels
+    res = {"scan": {"workload": f"{w.name}: batch {w.batch}, len {w.length}, {w.ranks} inputs/outputs x "
+                                f"{w.channels} channels, state {w.nstate}, {w.dtype} I/O, fp32 state",
+                    "ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
+                    "outputs_per_s": world * tc * w.ranks / (ms * 1e-3),
+                    **{"hbm_" + k: v for k, v in hbm_entry(mimo_bytes(w), ms, hbm_peak).items()}}}
+    del inp, y, hf
+    # decode step: 256 x 5120 rows, 4 inputs and outputs each, 200 steps with fresh inputs
+    B_, R_, C_, N_, steps = 256, 4, 5120, 16, 200
+    g = torch.Generator(device=dev).manual_seed(rank_seed(37, rank))
+    A = -(torch.arange(1, N_ + 1, device=dev, dtype=torch.float32) * (1.0 + 0.1 * torch.rand((C_, 1), generator=g, device=dev))).contiguous()
+    D = torch.randn(C_, generator=g, device=dev)
+    state = 0.1 * torch.randn((B_, C_, N_), generator=g, device=dev)
+    x = torch.randn((steps, B_, R_, C_), generator=g, device=dev).to(torch.bfloat16)
+    dl = torch.exp(torch.empty((steps, B_, C_), device=dev).uniform_(math.log(1e-3), math.log(1e-1), generator=g)).to(torch.bfloat16)
+    Bm = torch.randn((steps, B_, R_, N_), generator=g, device=dev).to(torch.bfloat16)
+    Cm = torch.randn((steps, B_, R_, N_), generator=g, device=dev).to(torch.bfloat16)
+    yd = torch.empty((steps, B_, R_, C_), device=dev, dtype=torch.bfloat16)
+    sx, sd, sb = x[0].numel() * 2, dl[0].numel() * 2, Bm[0].numel() * 2
+
+    def chain():
+        for s in range(steps):
+            st = lib.mamba_state_update_mimo(state.data_ptr(), x.data_ptr() + s * sx, dl.data_ptr() + s * sd,
+                                             A.data_ptr(), Bm.data_ptr() + s * sb, Cm.data_ptr() + s * sb,
+                                             D.data_ptr(), yd.data_ptr() + s * sx, B_, R_, C_, N_, m.MAMBA_BF16,
+                                             stream.cuda_stream)
+            if st != 0:
+                raise m.MambaError(st, "mamba_state_update_mimo")
+
+    ms_d = time_calls(chain, stream, dist, world, 3, warmup=1) / steps
+    nb = mimo_decode_bytes_per_step(B_, R_, C_, N_)
+    res["decode"] = {"workload": f"{B_} sequences x {C_} channels x {N_} states, {R_} inputs/outputs per row, "
+                                 f"{steps} steps, fp32 state, bf16 x/delta/B/C/y (plain launches)",
+                     "ms_per_step": round(ms_d, 5), "outputs_per_s": world * B_ * C_ * R_ / (ms_d * 1e-3),
+                     **{"hbm_" + k: v for k, v in hbm_entry(nb, ms_d, hbm_peak).items()}}
+    del state, x, dl, Bm, Cm, yd
     return res
 
 

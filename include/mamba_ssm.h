@@ -112,11 +112,15 @@ typedef enum {
  * channels is a multiple of 16 bytes, with plain loads otherwise.
  * Scratch: every call allocates and frees stream-ordered scratch on `stream`
  * (from a memory pool the library creates on the device, which keeps up to
- * 1 GiB of freed memory for later calls; inside a stream capture, from
- * cudaMallocAsync, and freed with cudaFreeAsync): job counters, the buffer that hands the
- * state from one time chunk to the next, and, when sequences are split into
- * independent super-chunks, their aggregates (mamba_scan_plan reports the
- * size).  batch == 0 or channels == 0 is a no-op that returns MAMBA_OK.
+ * 1 GiB of freed memory for later calls, see mamba_trim_scratch_pool;
+ * inside a stream capture, from cudaMallocAsync, and freed with
+ * cudaFreeAsync): job counters, the buffer that hands the state from one
+ * time chunk to the next, and, when sequences are split into super-chunks
+ * that run side by side, their end states and step sums (mamba_scan_plan
+ * reports the size).  With super-chunks a third kernel adds the state
+ * entering each super-chunk to its outputs; it walks a super-chunk only
+ * until that state's decay underflows to zero in fp32.  batch == 0 or
+ * channels == 0 is a no-op that returns MAMBA_OK.
  * The call enqueues only stream-ordered work (allocation, kernels, free), so
  * it can be captured in a CUDA graph once a first call on the device has run
  * outside capture (that call sets the kernels' shared-memory attribute).
@@ -356,13 +360,70 @@ int mamba_selective_scan_complex(const void *u, const void *delta, const float *
 /* 1 if `nstate` is implemented by mamba_selective_scan_complex. */
 int mamba_complex_supported_nstate(int64_t nstate);
 
+/*
+ * Multi-input multi-output (MIMO) selective scan.
+ *
+ * Defined by: the Mamba-3 page (bitig.info), "MIMO Mekanizmasının İşleyişi"
+ * (the state is updated once per step for several outputs, holds several
+ * output predictions without a larger state transition matrix or more
+ * parameters) and "Seçici Durum Güncellemesindeki İyileştirmeler" (a
+ * separate selective gate per output channel).  The page prints no
+ * formula; the reading taken is the zero-order hold of mamba_selective_scan
+ * with R inputs and R outputs per channel sharing one state and one step:
+ *   h_t = exp(Delta_t A) h_{t-1} + sum_r (Delta_t A)^-1 (exp(Delta_t A) - 1) Delta_t B_t^(r) x_t^(r)
+ *   y_t^(r) = C_t^(r) . h_t + D x_t^(r)          (C^(r): the gate of output r)
+ *
+ *   u, y          device, dtype, [batch][len][ranks][channels]   (x_t^(r), y_t^(r))
+ *   delta         device, dtype, [batch][len][channels]          (one step per token and channel)
+ *   A             device, float32, [channels][nstate]
+ *   B, C          device, dtype, [batch][len][ranks][nstate]     (shared by all channels)
+ *   D             device, float32, [channels], or NULL
+ *   initial_state, final_state   device, float32, [batch][channels][nstate], or NULL
+ *   ranks         R: 2 or 4 in this build, with nstate 16 (mamba_mimo_supported)
+ *   flags         0 or MAMBA_SCAN_GENERAL_A (zero-order hold only: EULER or
+ *                 TRAPEZOID give MAMBA_ERR_UNSUPPORTED)
+ *
+ * The same kernels as mamba_selective_scan (a tile of 64/R bf16 or 32/R fp32
+ * tokens), the same scratch, asynchrony, alignment and errors;
+ * batch * len * ranks must stay below 2^31.
+ */
+int mamba_selective_scan_mimo(const void *u, const void *delta, const float *A,
+                              const void *B, const void *C, const float *D,
+                              const float *initial_state, void *y, float *final_state,
+                              int64_t batch, int64_t len, int64_t ranks, int64_t channels, int64_t nstate,
+                              unsigned flags, int dtype, mamba_stream_t stream);
+
+/*
+ * One multi-input multi-output recurrent step for every (batch, channel)
+ * row (the decode step of mamba_selective_scan_mimo; the Mamba-3 page says
+ * MIMO's point is to serve several outputs per state update):
+ *   h_n <- exp(Delta A_n) h_n + (Delta A_n)^-1 (exp(Delta A_n) - 1) Delta sum_r B^(r)_n x^(r)
+ *   y^(r) = sum_n C^(r)_n h_n + D x^(r)
+ *
+ *   state   device, float32, [batch][channels][nstate], updated in place
+ *   x, y    device, dtype, [batch][ranks][channels]
+ *   delta   device, dtype, [batch][channels]
+ *   A       device, float32, [channels][nstate]
+ *   B, C    device, dtype, [batch][ranks][nstate]
+ *   D       device, float32, [channels], or NULL
+ * ranks and nstate as mamba_mimo_supported.  Alignment as mamba_state_update.
+ * No scratch memory is used.  Zero-order hold.
+ */
+int mamba_state_update_mimo(float *state, const void *x, const void *delta,
+                            const float *A, const void *B, const void *C, const float *D,
+                            void *y, int64_t batch, int64_t ranks, int64_t channels, int64_t nstate,
+                            int dtype, mamba_stream_t stream);
+
+/* 1 if mamba_selective_scan_mimo implements this number of inputs/outputs and states. */
+int mamba_mimo_supported(int64_t ranks, int64_t nstate);
+
 /* How mamba_selective_scan_ex would split a problem (host-side planning only). */
 typedef struct {
-    int64_t supers;        /* independent super-chunks per sequence (1: no aggregate jobs) */
+    int64_t supers;        /* super-chunks per sequence, run side by side from zero (1: no correction kernel) */
     int64_t super_len;     /* tokens per super-chunk (all but the last) */
-    int64_t chunk_len;     /* tokens per job of the main pass */
-    int64_t jobs;          /* jobs of the chunked kernel (aggregate and main) */
-    int64_t kernels;       /* kernels one call launches */
+    int64_t chunk_len;     /* tokens per job of the chunked kernel */
+    int64_t jobs;          /* jobs of the chunked kernel */
+    int64_t kernels;       /* kernels one call launches (pre-pass, chunked scan, correction when supers > 1) */
     int64_t scratch_bytes; /* stream-ordered scratch one call allocates */
     int64_t ctas;          /* CTAs of the chunked kernel (persistent: at most one per SM) */
 } mamba_scan_plan_t;

@@ -190,6 +190,12 @@ __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
 }
 
 constexpr int kBwdWarps = 4;  // warps per CTA of the backward kernel
+// resident CTAs per SM of the reverse kernel: the per-warp state scratch of
+// all resident warps should stay in L2
+#ifndef MAMBA_BWD_CTAS_PER_SM
+#define MAMBA_BWD_CTAS_PER_SM 3
+#endif
+constexpr int kBwdCtasPerSm = MAMBA_BWD_CTAS_PER_SM;
 
 // q_n = exp(Delta A_n) - 1 for all states of one lane and token.  STRUCT
 // (A[d,n] = (n+1) A[d,0] on every lane of the warp): one accurate expm1 and
@@ -479,7 +485,7 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
 
 // at least three CTAs per SM: the occupancy is worth a few spilled registers
 template <typename TIO, int NS>
-__global__ void __launch_bounds__(kBwdWarps * 32, 3)
+__global__ void __launch_bounds__(kBwdWarps * 32, kBwdCtasPerSm)
 scan_backward_kernel(const BwdArgs<TIO> a) {
   static_assert(2 * NS <= 32, "dB and dC of a token are reduced in one 32-lane pass");
   extern __shared__ __align__(16) unsigned char bwd_smem[];

@@ -14,6 +14,11 @@
 // dt w / 2 and m = expm1(dt a),
 //   Re E = m (1 - 2 s^2) - 2 s^2,   Im E = (1 + m) 2 s c.
 // Each step turns the state by dt w: the rotation follows the input through dt.
+// When A[n] = (n+1) a + i n w exactly for every state of every channel of a
+// warp (the S4D-Lin form), E_{n+1} = E_n + F + E_n F with F = exp(dt (a +
+// i w)) - 1 (exp(dt A_{n+1}) = exp(dt A_n) exp(dt (a + i w))): two complex
+// exponentials per token and lane instead of one per state, which moves
+// the work from the special-function unit to the FMA pipe.
 //
 // One warp per (batch row, channel group, super-chunk); with 8 or more
 // states two lanes share a channel (half of its states each, 16 channels
@@ -86,6 +91,18 @@ __device__ __forceinline__ void sincos_reduced(float v, float* s, float* c) {
   __sincosf(fmaf(k, 1.7484556e-7f, r), s, c);                // + k * (fp32(2 pi) - 2 pi)
 }
 
+// exp(x + 2 i v) - 1 without cancellation for small arguments: with s, c =
+// sin, cos of v and m = expm1(x),
+//   Re = m (1 - 2 s^2) - 2 s^2,   Im = (1 + m) 2 s c.
+__device__ __forceinline__ void expm1_complex(float x, float v, float* re, float* im) {
+  const float m = expm1_small(x);
+  float s, c;
+  sincos_reduced(v, &s, &c);
+  const float s2 = 2.0f * s * s;
+  *re = fmaf(m, 1.0f - s2, -s2);
+  *im = (1.0f + m) * (2.0f * s * c);
+}
+
 // Stage one B or C row of N values (converted to fp32): 16-byte loads when
 // the row allows them, else element by element.
 template <typename TIO, int N>
@@ -147,6 +164,22 @@ complex_scan_kernel(const ComplexArgs a) {
     wh[i] = 0.5f * im;
     iar[i] = re * inv;
     iai[i] = -im * inv;
+  }
+  // S4D-Lin structure on every channel of the warp: A[n] = (n+1) a + i n w
+  // exactly (fp32), i.e. A[n+1] - A[n] = a + i w for all n: then
+  // exp(dt A[n+1]) = exp(dt A[n]) exp(dt (a + i w)), and a lane needs two
+  // complex exponentials per token instead of one per state
+  float sa, sw;  // a and w / 2 of the step a + i w
+  bool structured;
+  {
+    const float a0 = __ldg(a.A_re + (int64_t)dc * N), w1 = N > 1 ? __ldg(a.A_im + (int64_t)dc * N + 1) : 0.0f;
+    bool ok = a0 < 0.0f;
+    for (int n = 0; n < N; ++n)
+      ok &= __ldg(a.A_re + (int64_t)dc * N + n) == (float)(n + 1) * a0 &&
+            __ldg(a.A_im + (int64_t)dc * N + n) == (float)n * w1;
+    structured = __all_sync(0xffffffffu, ok);
+    sa = a0;
+    sw = 0.5f * w1;
   }
   float hr[NH], hi[NH];
 #pragma unroll
@@ -217,14 +250,24 @@ complex_scan_kernel(const ComplexArgs a) {
       const float* Bt = sB + k * N + n0;
       const float* Ct = sC + k * N + n0;
       float acc = 0.0f;
+      // structured: E of the lane's first state and F = exp(dt (a + i w)) - 1
+      // from the exponentials, the others by the product chain
+      float er = 0.0f, ei = 0.0f, fr = 0.0f, fi = 0.0f;
+      if (structured) {
+        expm1_complex(dt * ar[0], dt * wh[0], &er, &ei);
+        expm1_complex(dt * sa, dt * sw, &fr, &fi);
+      }
 #pragma unroll
       for (int i = 0; i < NH; ++i) {
-        const float m = expm1_small(dt * ar[i]);
-        float s, c;
-        sincos_reduced(dt * wh[i], &s, &c);
-        const float s2 = 2.0f * s * s;
-        const float er = fmaf(m, 1.0f - s2, -s2);        // Re(exp(dt A) - 1)
-        const float ei = (1.0f + m) * (2.0f * s * c);    // Im(exp(dt A) - 1)
+        if (!structured) {
+          expm1_complex(dt * ar[i], dt * wh[i], &er, &ei);  // exp(dt A) - 1
+        } else if (i > 0) {
+          // exp(dt A_{n+1}) - 1 = E + F + E F   (exp(dt A_{n+1}) = exp(dt A_n) exp(dt (a + i w)))
+          const float nr = er + fr + fmaf(er, fr, -ei * fi);
+          const float ni = ei + fi + fmaf(er, fi, ei * fr);
+          er = nr;
+          ei = ni;
+        }
         const float bx = Bt[i] * x;
         const float gr = fmaf(er, iar[i], -ei * iai[i]) * bx;  // Re((E / A) B x)
         const float gi = fmaf(er, iai[i], ei * iar[i]) * bx;   // Im((E / A) B x)

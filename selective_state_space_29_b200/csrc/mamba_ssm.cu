@@ -129,14 +129,22 @@ bool make_map_2d(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uin
 // A CTA is kScanConsumers consumer warps (one per SM sub-partition) and one
 // producer warp; a consumer's ring holds kStages tiles of kTile tokens (the
 // ring of four consumers fits the 227 KB of shared memory of a CTA).
-template <typename TIO, int NS>
+// With R inputs per token (multi-input multi-output) a tile holds 1/R as
+// many tokens, so that its u, B and C' rows stay the same size.
+template <typename TIO, int NS, int R = 1>
 struct ScanCfg {
   static constexpr bool kBf16 = sizeof(TIO) == 2;
-  static constexpr int kTile = kBf16 ? 64 : 32;
+  static constexpr int kTile = (kBf16 ? 64 : 32) / R;
   static constexpr int kStages = (kBf16 && NS >= 32) ? 2 : 3;
 };
 constexpr int kScanConsumers = 4;
 constexpr int kJobsPerWarp = 8;  // chunks per consumer warp, for dynamic balance
+// streams (channel group x super-chunk) per resident consumer warp, in percent,
+// below which sequences are cut into super-chunks
+#ifndef MAMBA_SCAN_STREAMS_PCT
+#define MAMBA_SCAN_STREAMS_PCT 100
+#endif
+constexpr int64_t kStreamsPerWarpPct = MAMBA_SCAN_STREAMS_PCT;
 
 struct Plan {
   int groups_d = 0;         // ceil(channels / 32)
@@ -151,11 +159,13 @@ struct Plan {
 // How a scan is laid out and split.  Every consumer warp needs a stream of
 // its own (a 32-channel group over a stretch of time); when the groups are
 // fewer than the resident consumer warps, sequences are cut into
-// super-chunks joined by the associative combine (about twice as many
-// streams as warps).  Within a stream the
-// sequence is cut into chunks so that there are about kJobsPerWarp jobs per
-// warp for dynamic balance, each at least two tiles long.  A positive
-// `user_chunk` forces super-chunks of that length.
+// super-chunks that run from zero side by side and are joined afterwards by
+// the correction kernel (about as many streams as warps: each extra
+// super-chunk adds a correction walk, which is short once the decay has
+// underflowed).  Within a stream the sequence is cut into chunks so that
+// there are about kJobsPerWarp jobs per warp for dynamic balance, each at
+// least two tiles long.  A positive `user_chunk` forces super-chunks of that
+// length.
 Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, int64_t user_chunk) {
   Plan pl;
   pl.warps_total = sms * kScanConsumers;
@@ -166,10 +176,8 @@ Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, 
     pl.super_len = std::min<int64_t>(user_chunk, len);
   } else {
     int64_t s = 1;
-    // twice as many streams as warps: a super-chunk's aggregate and main
-    // jobs form a sequential path of about 1.6 super-chunk lengths, which
-    // then stays well below each warp's share of the work
-    if (groups < pl.warps_total) s = (2 * (int64_t)pl.warps_total + groups - 1) / groups;
+    const int64_t want = (int64_t)pl.warps_total * kStreamsPerWarpPct / 100;  // streams wanted
+    if (groups < want) s = (want + groups - 1) / groups;
     s = std::min<int64_t>(s, std::max<int64_t>(1, len / (4 * tile)));
     pl.super_len = (len + s - 1) / s;
     pl.super_len = ((pl.super_len + tile - 1) / tile) * tile;
@@ -189,31 +197,36 @@ Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, 
 }
 
 struct ScratchLayout {
-  size_t ctr, done, ring, ring_sd, agg_h, agg_sd, cs, chan, total;
+  size_t ctr, done, fix_segs, ring, ring_sd, agg_h, agg_sd, cum, cs, chan, total;
+  int64_t segs_max;  // correction segments of a full super-chunk
 };
 
-ScratchLayout scratch_layout(const Plan& pl, int ns, int64_t batch, int64_t len) {
+ScratchLayout scratch_layout(const Plan& pl, int ns, int64_t batch, int64_t len, int tile, int ranks = 1) {
   auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
   const int64_t S = pl.supers;
-  const int64_t streams_full = S * pl.groups;
-  const int64_t streams_agg = (S - 1) * pl.groups;
+  const int64_t streams = S * pl.groups;
+  const int64_t aggs = S > 1 ? streams : 0;  // aggregates, segment sums: only with super-chunks
   ScratchLayout s;
+  const int64_t seg = (int64_t)kFixSegTiles * tile;
+  s.segs_max = (pl.super_len + seg - 1) / seg;
   s.ctr = al(4 * sizeof(int));
-  s.done = al(sizeof(int) * (size_t)(streams_full + streams_agg));
-  s.ring = al(sizeof(float) * (size_t)(streams_full + streams_agg) * 2 * kCPW * ns);
-  s.ring_sd = al(sizeof(float) * (size_t)(streams_full + streams_agg) * 2 * kCPW);
-  s.agg_h = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kCPW * ns);
-  s.agg_sd = al(sizeof(float) * (size_t)std::max<int64_t>(streams_agg, 1) * kCPW);
-  s.cs = al(sizeof(float) * (size_t)batch * (size_t)len * (size_t)ns);
+  s.done = al(sizeof(int) * (size_t)streams);
+  s.fix_segs = al(sizeof(int) * (size_t)aggs);
+  s.ring = al(sizeof(float) * (size_t)streams * 2 * kCPW * ns);
+  s.ring_sd = al(sizeof(float) * (size_t)streams * 2 * kCPW);
+  s.agg_h = al(sizeof(float) * (size_t)aggs * kCPW * ns);
+  s.agg_sd = al(sizeof(float) * (size_t)aggs * kCPW);
+  s.cum = al(sizeof(float) * (size_t)aggs * (size_t)s.segs_max * kCPW);
+  s.cs = al(sizeof(float) * (size_t)batch * (size_t)len * (size_t)ranks * (size_t)ns);
   s.chan = al(sizeof(float) * 4 * (size_t)pl.groups_d * (size_t)kCPW);
-  s.total = s.ctr + s.done + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.cs + s.chan;
+  s.total = s.ctr + s.done + s.fix_segs + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.cum + s.cs + s.chan;
   return s;
 }
 
 int64_t full_jobs(const Plan& pl) {
-  const int64_t streams_full = (int64_t)pl.supers * pl.groups;
-  const int64_t streams_agg = (int64_t)(pl.supers - 1) * pl.groups;
-  return (int64_t)pl.chunks_last * streams_full + (int64_t)(pl.chunks_full - pl.chunks_last) * streams_agg;
+  const int64_t streams = (int64_t)pl.supers * pl.groups;
+  const int64_t streams_early = (int64_t)(pl.supers - 1) * pl.groups;  // super-chunks 0..S-2
+  return (int64_t)pl.chunks_last * streams + (int64_t)(pl.chunks_full - pl.chunks_last) * streams_early;
 }
 
 int tile_for(int dtype) { return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16, 16>::kTile : ScanCfg<float, 16>::kTile; }
@@ -230,7 +243,8 @@ int dispatch_nstate(int64_t nstate, F&& f) {
   }
 }
 
-int64_t kernels_per_call(const Plan&) { return 2; }  // pre-pass, chunked scan
+// pre-pass, chunked scan, and the correction kernel when there are super-chunks
+int64_t kernels_per_call(const Plan& pl) { return pl.supers > 1 ? 3 : 2; }
 
 // Launch with programmatic stream serialization: the kernel may start while
 // the previous kernel of the stream finishes; it waits for that kernel's
@@ -287,22 +301,26 @@ int noalloc_scratch_address(void** out) {
 }
 
 // Enqueue one scan with the given plan on caller-provided scratch (laid out
-// by scratch_layout): pre-pass, [aggregate pass, combine,] main pass.
-template <typename TIO, int NS, int METHOD, bool CKPT = false>
+// by scratch_layout): pre-pass, chunked pass, [correction].  R > 1: the
+// multi-input multi-output scan (u, y [batch][len][R][channels], B, C
+// [batch][len][R][nstate]).
+template <typename TIO, int NS, int METHOD, bool CKPT = false, int R = 1>
 int launch_scan_on(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
                    const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
                    unsigned flags, int dtype, cudaStream_t stream, const Plan& pl, int sms,
                    unsigned char* scratch, float* ckpt = nullptr) {
-  constexpr int TILE = ScanCfg<TIO, NS>::kTile;
-  constexpr int STAGES = ScanCfg<TIO, NS>::kStages;
-  const ScratchLayout sl = scratch_layout(pl, NS, batch, len);
+  constexpr int TILE = ScanCfg<TIO, NS, R>::kTile;
+  constexpr int STAGES = ScanCfg<TIO, NS, R>::kStages;
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, TILE, R);
   unsigned char* cur = scratch;
   int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
   int* done = reinterpret_cast<int*>(cur); cur += sl.done;
+  int* fix_segs = reinterpret_cast<int*>(cur); cur += sl.fix_segs;
   float* ring = reinterpret_cast<float*>(cur); cur += sl.ring;
   float* ring_sd = reinterpret_cast<float*>(cur); cur += sl.ring_sd;
   float* agg_h = reinterpret_cast<float*>(cur); cur += sl.agg_h;
   float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
+  float* cum = reinterpret_cast<float*>(cur); cur += sl.cum;
   float* cs = reinterpret_cast<float*>(cur); cur += sl.cs;
   float4* chan = reinterpret_cast<float4*>(cur);
 
@@ -317,17 +335,19 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   std::memset(&mc, 0, sizeof(mc));
   if (tma) {
     const uint64_t rows = (uint64_t)batch * (uint64_t)len;
-    tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows, kCPW, TILE) &&
+    tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows * R, kCPW, TILE * R) &&
           make_map_2d(&mdl, delta, dtype, (uint64_t)channels, rows, kCPW, TILE) &&
-          make_map_2d(&mb, B, dtype, NS, rows, NS, TILE) && make_map_2d(&mc, cs, MAMBA_F32, NS, rows, NS, TILE);
+          make_map_2d(&mb, B, dtype, NS, rows * R, NS, TILE * R) &&
+          make_map_2d(&mc, cs, MAMBA_F32, NS, rows * R, NS, TILE * R);
   }
 
   ScanParams p;
   std::memset(&p, 0, sizeof(p));
-  p.u = u; p.delta = delta; p.A = A; p.B = B; p.cs = cs; p.chan = chan; p.h0 = h0; p.y = y;
+  p.u = u; p.delta = delta; p.A = A; p.B = B; p.C = C; p.cs = cs; p.chan = chan; p.h0 = h0; p.y = y;
   p.final_state = final_state;
   p.ckpt = ckpt;
-  p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd;
+  p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd; p.cum = cum; p.fix_segs = fix_segs;
+  p.segs_max = (int)sl.segs_max;
   p.batch = batch; p.len = len; p.channels = channels;
   p.groups_d = pl.groups_d; p.groups = (int)pl.groups;
   p.supers = pl.supers; p.super_len = pl.super_len; p.chunk_len = pl.chunk_len;
@@ -335,9 +355,9 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   p.use_tma = tma ? 1 : 0;
   p.wait_limit_ns = kWaitLimitNs;
 
-  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES, kScanConsumers>();
+  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES, kScanConsumers, R>();
   static_assert(smem <= 232448, "scan CTA exceeds the shared memory of an SM");
-  auto kern = scan_chunks_kernel<TIO, NS, kScanConsumers, TILE, STAGES, METHOD, CKPT>;
+  auto kern = scan_chunks_kernel<TIO, NS, kScanConsumers, TILE, STAGES, METHOD, CKPT, R>;
   {
     // the dynamic shared-memory limit is a per-device attribute of the kernel
     static std::mutex mu_attr;
@@ -353,24 +373,22 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   }
 
   const int64_t S = pl.supers;
-  const int64_t streams_full = S * pl.groups;
-  const int64_t streams_agg = (S - 1) * pl.groups;
-  const int64_t jobs_agg = streams_agg * pl.chunks_full;
-  const int64_t jobs = jobs_agg + full_jobs(pl);
-  if (jobs > 0x7fffffff || streams_full + streams_agg > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
-  p.streams_agg = (int)streams_agg;
-  p.streams_full = (int)streams_full;
-  p.jobs_agg = (int)jobs_agg;
+  const int64_t streams = S * pl.groups;
+  const int64_t jobs = full_jobs(pl);
+  const int64_t fix_phases = std::min<int64_t>(sl.segs_max, kFixPhases);
+  const int64_t fix_warps = (S - 1) * pl.groups * fix_phases;
+  if (jobs > 0x7fffffff || streams > 0x7fffffff || fix_warps > 0x7fffffffLL || sl.segs_max > 0x7fffffff)
+    return MAMBA_ERR_UNSUPPORTED;
+  p.streams = (int)streams;
   p.jobs = (int)jobs;
   p.counters = counters;
   p.done = done;
-  p.done_agg = done + streams_full;
 
   // pre-pass: zero the counters and progress flags, C' = C / (n+1) in fp32,
   // and the per-channel constants
   {
-    const int64_t zero_words = (int64_t)((sl.ctr + sl.done) / sizeof(int));
-    const int64_t total_c = batch * len * NS;
+    const int64_t zero_words = (int64_t)((sl.ctr + sl.done + sl.fix_segs) / sizeof(int));
+    const int64_t total_c = batch * len * R * NS;
     const int64_t chan_padded = (int64_t)pl.groups_d * kCPW;
     const int64_t total = zero_words + total_c + chan_padded;
     if ((total + 255) / 256 > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
@@ -379,12 +397,21 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
         (flags & MAMBA_SCAN_GENERAL_A) ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return MAMBA_ERR_CUDA;
   }
-  // one persistent pass: the aggregate jobs of super-chunks 0..S-2 hold the
-  // first tickets, the main jobs follow
+  // one persistent pass over every super-chunk from zero (super-chunk 0
+  // from the initial state) ...
   const int64_t ctas = std::min<int64_t>(sms, (jobs + kScanConsumers - 1) / kScanConsumers);
   if (launch_pdl(kern, dim3((unsigned)ctas), dim3((kScanConsumers + 1) * 32), smem, stream, p, mu, mdl, mb, mc) !=
       cudaSuccess)
     return MAMBA_ERR_CUDA;
+  // ... then the states entering super-chunks 1..S-1 and their effect on y
+  // (and on the checkpoints), and the final state
+  if (S > 1) {
+    const int phases = (int)fix_phases;
+    const int64_t blocks = (fix_warps + kFixWarps - 1) / kFixWarps;
+    if (launch_pdl(scan_fix_kernel<TIO, NS, TILE, CKPT, R>, dim3((unsigned)blocks), dim3(kFixWarps * 32), 0, stream,
+                   p, phases) != cudaSuccess)
+      return MAMBA_ERR_CUDA;
+  }
   return MAMBA_OK;
 }
 
@@ -399,7 +426,7 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   if (int st = current_sms(&sms)) return st;
   const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO, NS>::kTile, user_chunk);
   if (pl.groups > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
-  const ScratchLayout sl = scratch_layout(pl, NS, batch, len);
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, ScanCfg<TIO, NS>::kTile);
   unsigned char* scratch = nullptr;
   if (noalloc) {
     if (sl.total > kNoAllocScratchBytes) return MAMBA_ERR_UNSUPPORTED;  // needs more than the fixed array
@@ -423,6 +450,24 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
     status = launch_scan_on<TIO, NS, kZOH>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags,
                                            dtype, stream, pl, sms, scratch);
   if (!noalloc && cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) return MAMBA_ERR_CUDA;
+  return status;
+}
+
+// The multi-input multi-output scan: plan, stream-ordered scratch, enqueue.
+template <typename TIO, int NS, int R>
+int launch_scan_mimo(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                     const float* D, const float* h0, void* y, float* final_state, int64_t batch, int64_t len,
+                     int64_t channels, unsigned flags, int dtype, cudaStream_t stream) {
+  int sms = 0;
+  if (int st = current_sms(&sms)) return st;
+  const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO, NS, R>::kTile, 0);
+  if (pl.groups > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, ScanCfg<TIO, NS, R>::kTile, R);
+  unsigned char* scratch = nullptr;
+  if (scratch_alloc(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
+  const int status = launch_scan_on<TIO, NS, kZOH, false, R>(u, delta, A, B, C, D, h0, y, final_state, batch, len,
+                                                             channels, flags, dtype, stream, pl, sms, scratch);
+  if (cudaFreeAsync(scratch, stream) != cudaSuccess && status == MAMBA_OK) return MAMBA_ERR_CUDA;
   return status;
 }
 
@@ -568,7 +613,11 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, main_k, kSsdWarps * 32, L::kBytes) != cudaSuccess ||
       per_sm < 1)
     return MAMBA_ERR_CUDA;
-  const int64_t seqs = batch * a.heads;
+  // tensor memory: kSsdTmemCols columns per CTA out of 512 per SM
+  per_sm = std::min(per_sm, 512 / kSsdTmemCols);
+  a.head_pairs = (a.heads + kSsdHeads - 1) / kSsdHeads;
+  a.wait_limit_ns = kWaitLimitNs;
+  const int64_t seqs = batch * a.head_pairs;  // one CTA per (batch row, head pair, super-chunk)
   const int64_t chunks = (a.len + kSsdQ - 1) / kSsdQ;
   int64_t S = ssd_supers(seqs, chunks, (int64_t)sms * per_sm, supers_req);
   const int64_t per = (chunks + S - 1) / S;
@@ -578,7 +627,7 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
   if (seqs * S >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
   unsigned char* mem = nullptr;
   if (S > 1) {
-    const size_t n_agg = (size_t)seqs * (size_t)(S - 1);
+    const size_t n_agg = (size_t)(batch * a.heads) * (size_t)(S - 1);
     const size_t st_bytes = n_agg * kSsdP * N * sizeof(float);
     if (scratch_alloc(reinterpret_cast<void**>(&mem), st_bytes + n_agg * sizeof(float), stream) != cudaSuccess)
       return MAMBA_ERR_CUDA;
@@ -680,9 +729,9 @@ int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate
   out->supers = pl.supers;
   out->super_len = pl.super_len;
   out->chunk_len = pl.chunk_len;
-  out->jobs = (int64_t)(pl.supers - 1) * pl.groups * pl.chunks_full + full_jobs(pl);
+  out->jobs = full_jobs(pl);
   out->kernels = kernels_per_call(pl);
-  out->scratch_bytes = (int64_t)scratch_layout(pl, (int)nstate, batch, len).total;
+  out->scratch_bytes = (int64_t)scratch_layout(pl, (int)nstate, batch, len, tile_for(dtype)).total;
   out->ctas = std::min<int64_t>(sms, (out->jobs + kScanConsumers - 1) / kScanConsumers);
   return MAMBA_OK;
 }
@@ -726,6 +775,54 @@ int mamba_selective_scan_ex(const void* u, const void* delta, const float* A, co
     return launch_scan<float, NS>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels,
                                   chunk_len, flags, dtype, stream, false);
   });
+}
+
+int mamba_mimo_supported(int64_t ranks, int64_t nstate) {
+  return ((ranks == 2 || ranks == 4) && nstate == 16) ? 1 : 0;
+}
+
+int mamba_selective_scan_mimo(const void* u, const void* delta, const float* A, const void* B, const void* C,
+                              const float* D, const float* initial_state, void* y, float* final_state,
+                              int64_t batch, int64_t len, int64_t ranks, int64_t channels, int64_t nstate,
+                              unsigned flags, int dtype, mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || len < 0 || channels < 0 || nstate <= 0 || ranks <= 0) return MAMBA_ERR_INVALID_ARG;
+  if (flags & ~MAMBA_SCAN_GENERAL_A) {
+    if (flags & ~(MAMBA_SCAN_GENERAL_A | MAMBA_SCAN_EULER | MAMBA_SCAN_TRAPEZOID)) return MAMBA_ERR_INVALID_ARG;
+    return MAMBA_ERR_UNSUPPORTED;  // zero-order hold only
+  }
+  if (!mamba_mimo_supported(ranks, nstate)) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || channels == 0) return MAMBA_OK;
+  const size_t es = (size_t)elem_size(dtype);
+  if (len > 0) {
+    if (!u || !delta || !B || !C || !y || !A) return MAMBA_ERR_INVALID_ARG;
+    if (!aligned(u, es) || !aligned(delta, es) || !aligned(B, es) || !aligned(C, es) || !aligned(y, es))
+      return MAMBA_ERR_INVALID_ARG;
+  }
+  if ((A && !aligned(A, 4)) || (D && !aligned(D, 4)) || (final_state && !aligned(final_state, 4)) ||
+      (initial_state && !aligned(initial_state, 4)))
+    return MAMBA_ERR_INVALID_ARG;
+  if (batch * len * ranks >= (int64_t(1) << 31) || channels >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
+
+  cudaGetLastError();  // clear a stale, non-sticky error so the status below is ours
+  const size_t state_bytes = sizeof(float) * (size_t)batch * (size_t)channels * (size_t)nstate;
+  if (len == 0) {
+    if (!final_state) return MAMBA_OK;
+    cudaError_t e = initial_state
+                        ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, stream)
+                        : cudaMemsetAsync(final_state, 0, state_bytes, stream);
+    return e == cudaSuccess ? MAMBA_OK : MAMBA_ERR_CUDA;
+  }
+  auto go = [&](auto rk) {
+    constexpr int R = decltype(rk)::value;
+    if (dtype == MAMBA_BF16)
+      return launch_scan_mimo<__nv_bfloat16, 16, R>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len,
+                                                    channels, flags, dtype, stream);
+    return launch_scan_mimo<float, 16, R>(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, channels,
+                                          flags, dtype, stream);
+  };
+  return ranks == 2 ? go(std::integral_constant<int, 2>{}) : go(std::integral_constant<int, 4>{});
 }
 
 int mamba_selective_scan(const void* u, const void* delta, const float* A, const void* B, const void* C,
@@ -812,12 +909,12 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
         // the sequence is cut into S super-chunks run in parallel (about two
         // work items per resident warp); their incoming adjoints come from
         // the reverse aggregates of the later super-chunks
-        const int64_t resident = 3 * (int64_t)sms * kBwdWarps;
+        const int64_t resident = kBwdCtasPerSm * (int64_t)sms * kBwdWarps;
         const int64_t S = std::max<int64_t>(1, std::min<int64_t>((2 * resident + streams - 1) / streams, ntiles));
         const int64_t super_tiles = (ntiles + S - 1) / S;
         const int64_t supers = (ntiles + super_tiles - 1) / super_tiles;
         const int64_t items = supers * streams;
-        const int64_t ctas = std::min<int64_t>((items + kBwdWarps - 1) / kBwdWarps, 3 * (int64_t)sms);
+        const int64_t ctas = std::min<int64_t>((items + kBwdWarps - 1) / kBwdWarps, kBwdCtasPerSm * (int64_t)sms);
         auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
         const size_t ck_bytes = al(sizeof(float) * (size_t)batch * (size_t)ntiles * (size_t)channels * NS);
         const size_t sc_bytes = al(sizeof(float) * (size_t)ctas * kBwdWarps * T * 32 * NS);
@@ -949,6 +1046,49 @@ int mamba_state_update(float* state, const void* x, const void* delta, const flo
     }
     return err == cudaSuccess ? (int)MAMBA_OK : (int)MAMBA_ERR_CUDA;
   });
+}
+
+int mamba_state_update_mimo(float* state, const void* x, const void* delta, const float* A, const void* B,
+                            const void* C, const float* D, void* y, int64_t batch, int64_t ranks, int64_t channels,
+                            int64_t nstate, int dtype, mamba_stream_t stream_) {
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  if (dtype != MAMBA_F32 && dtype != MAMBA_BF16) return MAMBA_ERR_INVALID_ARG;
+  if (batch < 0 || channels < 0 || nstate <= 0 || ranks <= 0) return MAMBA_ERR_INVALID_ARG;
+  if (!mamba_mimo_supported(ranks, nstate)) return MAMBA_ERR_UNSUPPORTED;
+  if (batch == 0 || channels == 0) return MAMBA_OK;
+  if (!state || !x || !delta || !A || !B || !C || !y) return MAMBA_ERR_INVALID_ARG;
+  const size_t es = (size_t)elem_size(dtype);
+  if (!aligned(state, 16) || !aligned(A, 16) || (D && !aligned(D, 4)) || !aligned(x, es) || !aligned(delta, es) ||
+      !aligned(y, es) || !aligned(B, 4 * es) || !aligned(C, 4 * es))
+    return MAMBA_ERR_INVALID_ARG;
+  cudaGetLastError();
+  constexpr int NS = 16;
+  constexpr int kRows = 2;  // batch rows per thread
+  constexpr int kChanPerCta = kDecodeWarps * (32 / (NS / 4));
+  const int64_t gx = (channels + kChanPerCta - 1) / kChanPerCta;
+  const int64_t gy = (batch + kRows - 1) / kRows;
+  if (gy > 65535 || gx > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)gx, (unsigned)gy);
+  auto go = [&](auto rk) {
+    constexpr int R = decltype(rk)::value;
+    cudaError_t err;
+    if (dtype == MAMBA_BF16) {
+      DecodeArgs<__nv_bfloat16, NS> a{state, static_cast<const __nv_bfloat16*>(x),
+                                      static_cast<const __nv_bfloat16*>(delta), A,
+                                      static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C), D,
+                                      static_cast<__nv_bfloat16*>(y), batch, channels};
+      err = launch_pdl(state_update_mimo_kernel<__nv_bfloat16, NS, R, kRows, true>, grid, dim3(kDecodeWarps * 32), 0,
+                       stream, a);
+    } else {
+      DecodeArgs<float, NS> a{state, static_cast<const float*>(x), static_cast<const float*>(delta), A,
+                              static_cast<const float*>(B), static_cast<const float*>(C), D,
+                              static_cast<float*>(y), batch, channels};
+      err = launch_pdl(state_update_mimo_kernel<float, NS, R, kRows, false>, grid, dim3(kDecodeWarps * 32), 0, stream,
+                       a);
+    }
+    return err == cudaSuccess ? (int)MAMBA_OK : (int)MAMBA_ERR_CUDA;
+  };
+  return ranks == 2 ? go(std::integral_constant<int, 2>{}) : go(std::integral_constant<int, 4>{});
 }
 
 int mamba_ssd_supported_nstate(int64_t nstate) { return nstate == 16 || nstate == 32 || nstate == 64; }

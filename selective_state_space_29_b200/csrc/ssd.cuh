@@ -1,5 +1,6 @@
 // ssd.cuh -- Mamba-2's restricted scan (one scalar A per head, one step per
-// (token, head)) in its chunked matrix form, on the tensor cores.
+// (token, head)) in its chunked matrix form, on the 5th-generation tensor
+// cores (tcgen05, accumulators in tensor memory).
 //
 // With A = a_h * I the decay from token s to token t is the same scalar for
 // every state and channel of head h, so within a chunk of Q tokens
@@ -12,26 +13,29 @@
 // the input weight of the discretisation: (e^{a dt} - 1)/a for the
 // zero-order hold, dt for exponential Euler.
 //
-// A CTA of four warps owns one (batch row, head, super-chunk) and walks its
-// chunks of 64 tokens in order; warp w owns the chunk's rows 16w..16w+15.
-// Per chunk (mma.sync m16n8k16, bf16 operands, fp32 accumulators):
-//   Y   = C S_in                         [16 x 64] += [16 x N][N x 64]
-//   Y  *= e^{a cum_t} (per row)
-//   G   = C B^T                          [16 x 16(k+1)], causal blocks only
-//   M   = G o e^{a(cum_t - cum_s)} o w_s (masked s > t), rounded to bf16 in
-//         registers: the accumulator fragment is the next MMA's A fragment
-//   Y  += M X                            [16 x 64] += [16 x 16(w+1)][.. x 64]
-//   y   = Y + D x  -> bf16 -> shared -> 16-byte stores
-//   dS  = Bw^T X, Bw_s = e^{a(cum_end - cum_s)} w_s B_s     (warp w: 16 channels)
-//   S   = e^{a cum_end} S + dS           (fp32 registers; a bf16 copy in
-//                                          shared memory feeds the next Y_off)
-// x, B and C stream through a 3-stage cp.async ring (16-byte copies,
-// XOR-swizzled rows so that every ldmatrix is free of bank conflicts).
+// A CTA of four warps owns two heads of one batch row over one super-chunk
+// and walks its chunks of 64 tokens in order.  Per chunk and head, all
+// products are tcgen05.mma (bf16 operands from shared memory, fp32
+// accumulators in tensor memory), issued by one thread:
+//   G   = C B^T                     64 x 64, K = N      (same for both heads)
+//   Y   = M X + C~ S_in             64 x 64, K = 64 + N  (M = G o e^{a(cum_t - cum_s)} o w_s,
+//                                                         masked s > t; C~ = e^{a cum_t} C)
+//   dS^T = X^T Bw                   64 x N,  K = 64      (Bw_s = e^{a(cum_end - cum_s)} w_s B_s)
+// The M = 64 accumulators of head 0 sit in tensor-memory lanes 0-15 of each
+// 32-lane sub-partition and those of head 1 in lanes 16-31, so every thread
+// of a warp reads one row of one head: thread i of warp w owns row (or
+// channel) 16w + i%16 of head i/16.  The warps turn G into M, form C~ and
+// Bw, and run the epilogues: y = Y + D x, and the fp32 state
+// S = e^{a cum_end} S + dS, kept in registers (a bf16 copy in shared memory
+// is the next chunk's operand).  x, B and C arrive through a ring of
+// cp.async copies into the no-swizzle core-matrix layouts the tensor core
+// reads (8 rows x 16 bytes per core matrix).
 //
-// Long sequences with few (batch, head) pairs are cut into super-chunks: an
-// aggregate kernel runs each super-chunk but the last from a zero state and
-// records its end state and total decay; the main kernel folds the
-// aggregates of the earlier super-chunks into its entering state.
+// Long sequences with few (batch row, head) pairs are cut into
+// super-chunks: an aggregate kernel (the same kernel, state only) runs each
+// super-chunk but the last from a zero state and records its end state and
+// total decay; the main kernel folds the aggregates of the earlier
+// super-chunks into its entering state.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -43,8 +47,9 @@ namespace mamba {
 
 constexpr int kSsdQ = 64;       // tokens per chunk
 constexpr int kSsdP = 64;       // channels per head
-constexpr int kSsdWarps = 4;    // warp w owns chunk rows 16w..16w+15
-constexpr int kSsdStages = 3;   // cp.async ring depth (chunks in flight)
+constexpr int kSsdWarps = 4;    // one warpgroup per CTA
+constexpr int kSsdHeads = 2;    // heads per CTA
+constexpr int kSsdTmemCols = 128;  // G / dS^T in columns [0, 64), Y in [64, 128)
 
 struct SsdArgs {
   const __nv_bfloat16* x;       // (batch, len, heads*64)
@@ -60,20 +65,12 @@ struct SsdArgs {
   float* agg_decay;             // (batch*heads, supers-1): log2 of its total decay
   int64_t len;
   int heads;
-  int supers;                   // super-chunks per (batch row, head)
+  int head_pairs;               // ceil(heads / 2)
+  int supers;                   // super-chunks per (batch row, head pair)
   int64_t super_len;            // tokens per super-chunk, a multiple of 64
   int euler;                    // input weight dt (exponential Euler) instead of the ZOH weight
+  uint64_t wait_limit_ns;
 };
-
-// Byte offset of 16-byte chunk `ch` of row `row` in a tile whose rows are R
-// chunks long: the chunk index is XORed with the row's position among the
-// rows that share a 128-byte line, so that 8 consecutive rows at one chunk
-// column fall in 8 different bank groups.
-template <int R>
-__device__ __forceinline__ uint32_t ssd_swz(int row, int ch) {
-  constexpr int kRowsPerLine = 8 / R;
-  return (uint32_t)(row * R * 16 + ((ch ^ ((row / kRowsPerLine) & (R - 1))) * 16));
-}
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
   const int n = valid ? 16 : 0;  // 0: nothing is read, the 16 bytes are zero-filled
@@ -83,398 +80,453 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
-}
-
-// D[16x8] += A[16x16] B[16x8], bf16 in, fp32 accumulate
-__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// ---------------------------------------------------------------------------
+// tcgen05 pieces
+// ---------------------------------------------------------------------------
+// Shared-memory matrix descriptor, no swizzle: start address, the byte
+// distance between core matrices along the leading dimension (LBO) and along
+// the stride dimension (SBO), all in 16-byte units; version 1 (sm_100).
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3fffu) | ((uint64_t)((lbo >> 4) & 0x3fffu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3fffu) << 32) | ((uint64_t)1 << 46);
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B, fp32 accumulator,
+// M x N, A / B K-major (0) or MN-major (1).
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int m, int n, int a_mn, int b_mn) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+         ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          bool accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"((int)accumulate)
+      : "memory");
+}
+
+// the mbarrier completes when every tcgen05.mma this thread issued so far has
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
+// shared-memory layout (bytes), every tile in the no-swizzle core-matrix
+// form: a core matrix is 8 rows x 16 bytes, stored contiguously (128 B)
+//   K-major [rows][K]:   (r/8) SBO + (k/8) 128 + (r%8) 16 + (k%8) 2,  SBO = K/8 * 128
+//   X [tok][ch] as MN-major (N or M = ch, K = tok):
+//                        (t/8) 1024 + (c/8) 128 + (t%8) 16 + (c%8) 2
+//   Bw [s][n] as MN-major (N = n, K = s):
+//                        (s/8) (N/8 * 128) + (n/8) 128 + (s%8) 16 + (n%8) 2
+// ---------------------------------------------------------------------------
 template <int N>
 struct SsdSmem {
-  static constexpr int R = N / 8;                  // 16-byte chunks per B / C row
-  static constexpr int kX = kSsdQ * kSsdP * 2;     // one x tile
-  static constexpr int kBC = kSsdQ * N * 2;        // one B or C tile
-  static constexpr int kStage = kX + 2 * kBC;
-  static constexpr int kRing = kSsdStages * kStage;
-  static constexpr int kBw = kRing;                // [64 tokens][N] bf16
-  static constexpr int kS = kBw + kBC;             // [64 channels][N] bf16 copy of the state
-  static constexpr int kY = kS + kSsdP * N * 2;    // [64][64] bf16 output staging
-  static constexpr int kCum = kY + kSsdQ * kSsdP * 2;  // per warp: cum (log2) and w for 64 tokens
-  static constexpr int kBytes = kCum + kSsdWarps * 2 * kSsdQ * 4;
-  // CTAs per SM the register budget is set for (shared memory allows 4 at
-  // 16 states, 3 at 32, 2 at 64)
-  static constexpr int kMinBlocks = N == 16 ? 4 : 2;
+  static constexpr int kStages = N >= 32 ? 2 : 3;
+  static constexpr int kX = kSsdQ * kSsdP * 2;           // one head's x tile (8 KB)
+  static constexpr int kBC = kSsdQ * N * 2;              // one B or C tile
+  static constexpr int kStage = kSsdHeads * kX + 2 * kBC;  // x of both heads, B, C
+  static constexpr int kRing = kStages * kStage;
+  static constexpr int kM = kRing;                       // [2 heads] M tiles, 64 x 64
+  static constexpr int kCt = kM + kSsdHeads * kSsdQ * kSsdQ * 2;  // [2] C~ tiles, 64 x N
+  static constexpr int kBw = kCt + kSsdHeads * kBC;      // [2] Bw tiles, 64 x N
+  static constexpr int kS = kBw + kSsdHeads * kBC;       // [2] bf16 state copies, 64 ch x N
+  static constexpr int kCum = kS + kSsdHeads * kSsdP * N * 2;  // [2][64] cum (log2), [2][64] w
+  static constexpr int kWsum = kCum + 2 * kSsdHeads * kSsdQ * 4;  // [4 warps][2 heads] partial sums
+  static constexpr int kDs = kWsum + kSsdWarps * kSsdHeads * 4;   // [2 heads][64] D
+  static constexpr int kBar = kDs + kSsdHeads * kSsdP * 4;        // 2 mbarriers
+  static constexpr int kTslot = kBar + 16;
+  static constexpr int kBytes = kTslot + 16 + 1024;      // + room to align the base to 1024
+  static constexpr int kSboBC = (N / 8) * 128;            // K-major [rows][N]
 };
 
 template <int N, bool AGG>
-__global__ void __launch_bounds__(kSsdWarps * 32, SsdSmem<N>::kMinBlocks)
+__global__ void __launch_bounds__(kSsdWarps * 32)
 ssd_chunk_kernel(const SsdArgs a) {
   using L = SsdSmem<N>;
-  constexpr int R = L::R;
-  constexpr int KS = N / 16;   // k-steps over states
-  extern __shared__ __align__(128) unsigned char smem[];
+  static_assert(N % 16 == 0 && N <= 64, "states in steps of 16, at most 64 (tensor-memory columns)");
+  extern __shared__ __align__(1024) unsigned char ssd_smem_raw[];
+  unsigned char* smem = ssd_smem_raw + ((1024u - (smem_addr(ssd_smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int g = lane >> 2, q = lane & 3;
+  const int hd = lane >> 4;                 // head of this thread within the CTA
+  const int row = 16 * warp + (lane & 15);  // its row (token) or channel
   const int64_t channels = (int64_t)a.heads * kSsdP;
 
-  // job: (batch row, head, super-chunk); the aggregate kernel has one
-  // super-chunk fewer per (batch row, head)
+  // job: (batch row, head pair, super-chunk); the aggregate kernel has one
+  // super-chunk fewer per pair
   const int per_seq = AGG ? a.supers - 1 : a.supers;
-  const int64_t seq = blockIdx.x / per_seq;
+  const int64_t seq = blockIdx.x / per_seq;  // batch row * head_pairs + pair
   const int j = (int)(blockIdx.x % per_seq);
-  const int64_t b = seq / a.heads;
-  const int h = (int)(seq % a.heads);
+  const int64_t b = seq / a.head_pairs;
+  const int hp = (int)(seq % a.head_pairs);
+  const int h = 2 * hp + hd;                // this thread's head
+  const bool hok = h < a.heads;
+  const bool pair = 2 * hp + 1 < a.heads;   // the CTA's second head exists
   const int64_t t_begin = (int64_t)j * a.super_len;
   const int64_t t_end = t_begin + a.super_len < a.len ? t_begin + a.super_len : a.len;
   const int nchunks = (int)((t_end - t_begin + kSsdQ - 1) / kSsdQ);
 
+  uint64_t* bar_g = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  uint64_t* bar_y = bar_g + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L::kTslot);
+  if (tid == 0) {
+    mbar_init(bar_g, 1);
+    mbar_init(bar_y, 1);
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tslot)),
+                 "n"(kSsdTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
   griddep_wait();  // inputs (and the aggregates) may come from the previous kernel
 
-  const float a_h = __ldg(a.A + h);
+  const int hc = hok ? h : 0;               // a valid head for reads
+  const float a_h = __ldg(a.A + hc);
   const float a2 = a_h * 1.4426950408889634f;  // a in log2 units
-  const __nv_bfloat16* xg = a.x + (b * a.len) * channels + (int64_t)h * kSsdP;
   const __nv_bfloat16* Bg = a.B + (b * a.len) * N;
   const __nv_bfloat16* Cg = a.C + (b * a.len) * N;
-  const unsigned short* dtg = reinterpret_cast<const unsigned short*>(a.dt) + (b * a.len) * a.heads + h;
+  const unsigned short* dtg = reinterpret_cast<const unsigned short*>(a.dt) + (b * a.len) * a.heads + hc;
 
-  // stage one chunk's x, B (and C) into ring slot `slot`
+  // stage one chunk's x (both heads), B (and C) into ring slot `slot`
   auto load_chunk = [&](int c, int slot) {
     const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
     const uint32_t sx = sbase + slot * L::kStage;
 #pragma unroll
-    for (int i = tid; i < kSsdQ * 8; i += kSsdWarps * 32) {
-      const int row = i >> 3, ch = i & 7;
-      const bool ok = t0 + row < t_end;
-      cp_async16(sx + ssd_swz<8>(row, ch), ok ? (const void*)(xg + (t0 + row) * channels + ch * 8) : (const void*)a.x,
+    for (int i = tid; i < kSsdHeads * kSsdQ * 8; i += kSsdWarps * 32) {
+      const int hh = i / (kSsdQ * 8), rem = i % (kSsdQ * 8);
+      const int t = rem >> 3, c8 = rem & 7;
+      const bool ok = t0 + t < t_end && 2 * hp + hh < a.heads;
+      const __nv_bfloat16* src = a.x + (b * a.len + t0 + t) * channels + (int64_t)(2 * hp + hh) * kSsdP + c8 * 8;
+      cp_async16(sx + hh * L::kX + (t >> 3) * 1024 + c8 * 128 + (t & 7) * 16, ok ? (const void*)src : (const void*)a.x,
                  ok);
     }
-    const uint32_t sb = sx + L::kX;
+    const uint32_t sb = sx + kSsdHeads * L::kX;
 #pragma unroll
-    for (int i = tid; i < kSsdQ * R; i += kSsdWarps * 32) {
-      const int row = i / R, ch = i % R;
-      const bool ok = t0 + row < t_end;
-      cp_async16(sb + ssd_swz<R>(row, ch), ok ? (const void*)(Bg + (t0 + row) * N + ch * 8) : (const void*)a.B, ok);
-      if (!AGG)
-        cp_async16(sb + L::kBC + ssd_swz<R>(row, ch),
-                   ok ? (const void*)(Cg + (t0 + row) * N + ch * 8) : (const void*)a.C, ok);
+    for (int i = tid; i < kSsdQ * (N / 8); i += kSsdWarps * 32) {
+      const int t = i / (N / 8), n8 = i % (N / 8);
+      const bool ok = t0 + t < t_end;
+      const uint32_t off = (t >> 3) * L::kSboBC + n8 * 128 + (t & 7) * 16;
+      cp_async16(sb + off, ok ? (const void*)(Bg + (t0 + t) * N + n8 * 8) : (const void*)a.B, ok);
+      if (!AGG) cp_async16(sb + L::kBC + off, ok ? (const void*)(Cg + (t0 + t) * N + n8 * 8) : (const void*)a.C, ok);
     }
   };
-  auto load_dt = [&](int c, int k) -> float {
-    const int64_t t = t_begin + (int64_t)c * kSsdQ + k;
+  auto load_dt = [&](int c) -> float {  // this thread's (token, head) step
+    const int64_t t = t_begin + (int64_t)c * kSsdQ + row;
     if (c >= nchunks || t >= t_end) return 0.0f;  // padding tokens: no decay, no input
     return __uint_as_float((uint32_t)__ldg(dtg + t * a.heads) << 16);
   };
 
-  // the state: warp w holds channels 16w..16w+15 for all N states, in the
-  // accumulator layout of dS (row = state, column = channel)
-  float S[KS][2][4];
+  // the state of this thread's (head, channel `row`): N fp32 values
+  float S[N];
 #pragma unroll
-  for (int mt = 0; mt < KS; ++mt)
-#pragma unroll
-    for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) S[mt][jj][e] = 0.0f;
-  auto s_index = [&](int mt, int jj, int e, int* n, int* p) {
-    *n = 16 * mt + g + 8 * (e >> 1);
-    *p = 16 * warp + 8 * jj + 2 * q + (e & 1);
-  };
-  if (!AGG) {
+  for (int n = 0; n < N; ++n) S[n] = 0.0f;
+  const int64_t sidx = ((b * a.heads + hc) * kSsdP + row) * N;  // (batch, channel, n) offset
+  if (!AGG && hok) {
     if (a.h0) {
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt)
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            int n, p;
-            s_index(mt, jj, e, &n, &p);
-            S[mt][jj][e] = __ldg(a.h0 + ((b * a.heads + h) * kSsdP + p) * N + n);
-          }
+      for (int n = 0; n < N; ++n) S[n] = __ldg(a.h0 + sidx + n);
     }
     // fold in the super-chunks before this one
+    const int64_t aseq = b * a.heads + h;
     for (int k = 0; k < j; ++k) {
-      const int64_t agg = seq * (a.supers - 1) + k;
+      const int64_t agg = aseq * (a.supers - 1) + k;
       const float dec = exp2f(__ldg(a.agg_decay + agg));
-      const float* as = a.agg_state + agg * (kSsdP * N);
+      const float* as = a.agg_state + (agg * kSsdP + row) * N;
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt)
-#pragma unroll
-        for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            int n, p;
-            s_index(mt, jj, e, &n, &p);
-            S[mt][jj][e] = fmaf(dec, S[mt][jj][e], __ldg(as + p * N + n));
-          }
+      for (int n = 0; n < N; ++n) S[n] = fmaf(dec, S[n], __ldg(as + n));
     }
   }
-  // bf16 copy of the state for the next chunk's C S_in (state n, channel p)
+  // bf16 copy of the state (K-major [channel][n]) for the next chunk's C~ S_in
   auto store_state_copy = [&]() {
+    unsigned char* st = smem + L::kS + hd * (kSsdP * N * 2) + (row >> 3) * L::kSboBC + (row & 7) * 16;
 #pragma unroll
-    for (int mt = 0; mt < KS; ++mt)
-#pragma unroll
-      for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          int n, p;
-          s_index(mt, jj, e, &n, &p);
-          const __nv_bfloat16 v = __float2bfloat16_rn(S[mt][jj][e]);
-          *reinterpret_cast<__nv_bfloat16*>(smem + L::kS + ssd_swz<R>(p, n >> 3) + (n & 7) * 2) = v;
-        }
+    for (int n8 = 0; n8 < N / 8; ++n8) {
+      uint4 v;
+      v.x = pack_bf16(S[8 * n8 + 0], S[8 * n8 + 1]);
+      v.y = pack_bf16(S[8 * n8 + 2], S[8 * n8 + 3]);
+      v.z = pack_bf16(S[8 * n8 + 4], S[8 * n8 + 5]);
+      v.w = pack_bf16(S[8 * n8 + 6], S[8 * n8 + 7]);
+      *reinterpret_cast<uint4*>(st + n8 * 128) = v;
+    }
   };
   if (!AGG) store_state_copy();
 
-  float* cum_w = reinterpret_cast<float*>(smem + L::kCum) + warp * 2 * kSsdQ;  // [64] cum (log2), [64] w
-  float* wt_w = cum_w + kSsdQ;
+  float* Ds = reinterpret_cast<float*>(smem + L::kDs);  // [2][64] D of both heads (0 without D)
+  Ds[hd * kSsdP + row] = (a.D && hok) ? __ldg(a.D + (int64_t)h * kSsdP + row) : 0.0f;
+  float* cum_s = reinterpret_cast<float*>(smem + L::kCum);  // [2][64]
+  float* w_s = cum_s + kSsdHeads * kSsdQ;                    // [2][64]
+  float* wsum = reinterpret_cast<float*>(smem + L::kWsum);   // [4][2]
   float total_log2 = 0.0f;
 
-  // prologue: the first kSsdStages-1 chunks
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);  // this warp's sub-partition, + lane i = thread
+  const uint32_t d_off = (uint32_t)(16 * 1) << 16;                // head 1's accumulators: lanes 16-31
+
+  // prologue: the first kStages-1 chunks
 #pragma unroll
-  for (int s = 0; s < kSsdStages - 1; ++s) {
+  for (int s = 0; s < L::kStages - 1; ++s) {
     if (s < nchunks) load_chunk(s, s);
     cp_async_commit();
   }
-  float dt0 = load_dt(0, lane), dt1 = load_dt(0, lane + 32);
+  float dt = load_dt(0);
+  bool ok_run = true;
 
-  for (int c = 0; c < nchunks; ++c) {
-    const int slot = c % kSsdStages;
+  for (int c = 0; c < nchunks && ok_run; ++c) {
+    const int slot = c % L::kStages;
     const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
-    // next chunk's steps, one chunk ahead
-    const float ndt0 = load_dt(c + 1, lane), ndt1 = load_dt(c + 1, lane + 32);
+    const float ndt = load_dt(c + 1);
 
-    // running log2 decay inside the chunk (every warp computes its own copy)
-    float v0 = dt0 * a2, v1 = dt1 * a2;
+    // running log2 decay inside the chunk for this thread's head: an
+    // inclusive scan over the 16 lanes of the half-warp, then across warps
+    float v = dt * a2;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float n0 = __shfl_up_sync(0xffffffffu, v0, o);
-      const float n1 = __shfl_up_sync(0xffffffffu, v1, o);
-      if (lane >= o) {
-        v0 += n0;
-        v1 += n1;
-      }
+    for (int o = 1; o < 16; o <<= 1) {
+      const float nb = __shfl_up_sync(0xffffffffu, v, o, 16);
+      if ((lane & 15) >= o) v += nb;
     }
-    v1 += __shfl_sync(0xffffffffu, v0, 31);
-    const float cum_end = __shfl_sync(0xffffffffu, v1, 31);
-    total_log2 += cum_end;
-    const float w0 = a.euler ? dt0 : expm1f(dt0 * a_h) / a_h;
-    const float w1 = a.euler ? dt1 : expm1f(dt1 * a_h) / a_h;
-    __syncwarp();
-    cum_w[lane] = v0;
-    cum_w[lane + 32] = v1;
-    wt_w[lane] = w0;
-    wt_w[lane + 32] = w1;
-    __syncwarp();
+    if ((lane & 15) == 15) wsum[warp * kSsdHeads + hd] = v;
+    const float wgt = a.euler ? dt : expm1f(dt * a_h) / a_h;
 
-    cp_async_wait<kSsdStages - 2>();  // this thread's copies of chunk c have landed
-    __syncthreads();                  // everyone's; and chunk c-1 is done with its slot
-    if (c + kSsdStages - 1 < nchunks) load_chunk(c + kSsdStages - 1, (c + kSsdStages - 1) % kSsdStages);
-    cp_async_commit();
+    cp_async_wait<L::kStages - 2>();  // this thread's copies of chunk c have landed
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
+    __syncthreads();                  // everyone's; the warp sums; chunk c-1 is done with its slot
+    float pre = 0.0f;
+    for (int w2 = 0; w2 < warp; ++w2) pre += wsum[w2 * kSsdHeads + hd];
+    const float cum = v + pre;
+    float cum_end = 0.0f;
+    for (int w2 = 0; w2 < kSsdWarps; ++w2) cum_end += wsum[w2 * kSsdHeads + hd];
+    total_log2 += cum_end;
+    cum_s[hd * kSsdQ + row] = cum;
+    w_s[hd * kSsdQ + row] = wgt;
 
     const uint32_t sx = sbase + slot * L::kStage;
-    const uint32_t sb = sx + L::kX;
+    const uint32_t sb = sx + kSsdHeads * L::kX;
     const uint32_t sc = sb + L::kBC;
-
-    // Bw rows of this warp's 16 tokens: e^{a(cum_end - cum_s)} w_s B_s
-    {
-      constexpr int kPer = 16 * N / 32;  // elements per lane
-      const int row = 16 * warp + lane / (32 / 16);
-      static_assert(kPer % 2 == 0, "pairs");
-      const int n0 = (lane % 2) * kPer;
-      const float f = ex2_approx(cum_end - cum_w[row]) * wt_w[row];
+    constexpr uint32_t kIdG = umma_idesc_bf16(64, 64, 0, 0);
+    if (!AGG && tid == 0) {
+      // G = C B^T for both heads (identical; one accumulator per head's lanes)
 #pragma unroll
-      for (int i = 0; i < kPer; i += 2) {
-        const int n = n0 + i;
-        const uint32_t off = ssd_swz<R>(row, n >> 3) + (n & 7) * 2;
-        const __nv_bfloat162 bv = *reinterpret_cast<const __nv_bfloat162*>(smem + (sb - sbase) + off);
-        const float2 bf = __bfloat1622float2(bv);
-        *reinterpret_cast<uint32_t*>(smem + L::kBw + off) = pack_bf16(bf.x * f, bf.y * f);
+      for (int hh = 0; hh < kSsdHeads; ++hh) {
+        if (hh == 1 && !pair) break;
+#pragma unroll
+        for (int k = 0; k < N / 16; ++k)
+          umma_bf16(tmem + hh * d_off, umma_desc(sc + k * 256, 128, L::kSboBC), umma_desc(sb + k * 256, 128, L::kSboBC),
+                    kIdG, k > 0);
+      }
+      umma_commit(bar_g);
+    }
+    __syncthreads();  // cum and w of the chunk are in shared memory
+
+    // C~ = e^{a cum_t} C_t and Bw = e^{a(cum_end - cum_s)} w_s B_s, row `row` of head hd
+    {
+      const float fB = ex2_approx(cum_end - cum) * wgt;
+      const unsigned char* brow = smem + (sb - sbase) + (row >> 3) * L::kSboBC + (row & 7) * 16;
+      // Bw [s][n] as MN-major (N = n, K = s): (s/8) (N/8 128) + (n/8) 128 + (s%8) 16 + (n%8) 2,
+      // the same bytes as the K-major [s][n] placement of B
+      unsigned char* bwrow = smem + L::kBw + hd * L::kBC + (row >> 3) * L::kSboBC + (row & 7) * 16;
+#pragma unroll
+      for (int n8 = 0; n8 < N / 8; ++n8) {
+        const uint4 bv = *reinterpret_cast<const uint4*>(brow + n8 * 128);
+        const uint32_t bw4[4] = {bv.x, bv.y, bv.z, bv.w};
+        uint32_t op[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw4[q]));
+          op[q] = pack_bf16(f.x * fB, f.y * fB);
+        }
+        *reinterpret_cast<uint4*>(bwrow + n8 * 128) = make_uint4(op[0], op[1], op[2], op[3]);
+      }
+      if (!AGG) {
+        const float fC = ex2_approx(cum);
+        const unsigned char* crow = smem + (sc - sbase) + (row >> 3) * L::kSboBC + (row & 7) * 16;
+        unsigned char* ctrow = smem + L::kCt + hd * L::kBC + (row >> 3) * L::kSboBC + (row & 7) * 16;
+#pragma unroll
+        for (int n8 = 0; n8 < N / 8; ++n8) {
+          const uint4 cv = *reinterpret_cast<const uint4*>(crow + n8 * 128);
+          const uint32_t cw4[4] = {cv.x, cv.y, cv.z, cv.w};
+          uint32_t op[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cw4[q]));
+            op[q] = pack_bf16(f.x * fC, f.y * fC);
+          }
+          *reinterpret_cast<uint4*>(ctrow + n8 * 128) = make_uint4(op[0], op[1], op[2], op[3]);
+        }
       }
     }
 
     if (!AGG) {
-      const int r0 = 16 * warp + g, r1 = r0 + 8;
-      const float cr0 = cum_w[r0], cr1 = cum_w[r1];
-      // C fragments of this warp's rows (A operand, row-major [t][n])
-      uint32_t cf[KS][4];
-#pragma unroll
-      for (int kk = 0; kk < KS; ++kk)
-        ldsm_x4(cf[kk], sc + ssd_swz<R>(16 * warp + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * kk + (lane >> 4)));
-
-      // Y = e^{a cum_t} C S_in
-      float Y[8][4];
-#pragma unroll
-      for (int jt = 0; jt < 8; ++jt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) Y[jt][e] = 0.0f;
-#pragma unroll
-      for (int kk = 0; kk < KS; ++kk)
-#pragma unroll
-        for (int jp = 0; jp < 4; ++jp) {
-          uint32_t sf[4];
-          ldsm_x4(sf, sbase + L::kS + ssd_swz<R>(16 * jp + (lane & 7) + 8 * (lane >> 4), 2 * kk + ((lane >> 3) & 1)));
-          mma_bf16(Y[2 * jp], cf[kk], sf[0], sf[1]);
-          mma_bf16(Y[2 * jp + 1], cf[kk], sf[2], sf[3]);
-        }
-      {
-        const float e0 = ex2_approx(cr0), e1 = ex2_approx(cr1);
-#pragma unroll
-        for (int jt = 0; jt < 8; ++jt) {
-          Y[jt][0] *= e0;
-          Y[jt][1] *= e0;
-          Y[jt][2] *= e1;
-          Y[jt][3] *= e1;
-        }
+      // M row `row` of head hd from G: causal mask, decay and input weight
+      bool got = mbar_wait_bounded(bar_g, (uint32_t)(c & 1), a.wait_limit_ns);
+      got = __all_sync(0xffffffffu, got);  // warp-uniform: the tensor-memory loads are warp-wide
+      if (!got) {
+        if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+        ok_run = false;
       }
-
-      // causal part, one 16-token column block at a time
+      tc_fence_after();
+      const float* cum_h = cum_s + hd * kSsdQ;
+      const float* w_h = w_s + hd * kSsdQ;
+      unsigned char* mrow = smem + L::kM + hd * (kSsdQ * kSsdQ * 2) + (row >> 3) * 1024 + (row & 7) * 16;
 #pragma unroll
-      for (int ks = 0; ks < kSsdWarps; ++ks) {
-        if (ks <= warp) {
-          // G for columns 16ks..16ks+15 (two n-tiles)
-          float G[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      for (int q4 = 0; q4 < 4 && ok_run; ++q4) {
+        float g[16];
+        tmem_ld16(t_lane + (uint32_t)(16 * q4), g);
 #pragma unroll
-          for (int kk = 0; kk < KS; ++kk) {
-            uint32_t bf[4];
-            ldsm_x4(bf, sb + ssd_swz<R>(16 * ks + (lane & 7) + 8 * (lane >> 4), 2 * kk + ((lane >> 3) & 1)));
-            mma_bf16(G[0], cf[kk], bf[0], bf[1]);
-            mma_bf16(G[1], cf[kk], bf[2], bf[3]);
+        for (int h8 = 0; h8 < 2; ++h8) {
+          uint32_t op[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int s0 = 16 * q4 + 8 * h8 + 2 * e;
+            const float m0 = s0 <= row ? g[8 * h8 + 2 * e] * ex2_approx(cum - cum_h[s0]) * w_h[s0] : 0.0f;
+            const float m1 = s0 + 1 <= row ? g[8 * h8 + 2 * e + 1] * ex2_approx(cum - cum_h[s0 + 1]) * w_h[s0 + 1] : 0.0f;
+            op[e] = pack_bf16(m0, m1);
           }
-          // M = G o e^{a(cum_t - cum_s)} o w_s, zero above the diagonal
-          uint32_t am[4];
-#pragma unroll
-          for (int half = 0; half < 2; ++half) {
-            const int s0 = 16 * ks + 8 * half + 2 * q;
-            const float2 cs = *reinterpret_cast<const float2*>(cum_w + s0);
-            const float2 ws = *reinterpret_cast<const float2*>(wt_w + s0);
-            const float x00 = s0 <= r0 ? cr0 - cs.x : -INFINITY;
-            const float x01 = s0 + 1 <= r0 ? cr0 - cs.y : -INFINITY;
-            const float x10 = s0 <= r1 ? cr1 - cs.x : -INFINITY;
-            const float x11 = s0 + 1 <= r1 ? cr1 - cs.y : -INFINITY;
-            am[2 * half + 0] = pack_bf16(G[half][0] * ex2_approx(x00) * ws.x, G[half][1] * ex2_approx(x01) * ws.y);
-            am[2 * half + 1] = pack_bf16(G[half][2] * ex2_approx(x10) * ws.x, G[half][3] * ex2_approx(x11) * ws.y);
-          }
-          // Y += M X for tokens 16ks..16ks+15
-#pragma unroll
-          for (int jp = 0; jp < 4; ++jp) {
-            uint32_t xf[4];
-            ldsm_x4_t(xf, sx + ssd_swz<8>(16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * jp + (lane >> 4)));
-            mma_bf16(Y[2 * jp], am, xf[0], xf[1]);
-            mma_bf16(Y[2 * jp + 1], am, xf[2], xf[3]);
-          }
-        }
-      }
-
-      // y = Y + D x -> bf16, staged per warp, then 16-byte row stores
-      const float* Dh = a.D ? a.D + (int64_t)h * kSsdP : nullptr;
-#pragma unroll
-      for (int jt = 0; jt < 8; ++jt) {
-        const int p = 8 * jt + 2 * q;
-        const float2 dd = Dh ? __ldg(reinterpret_cast<const float2*>(Dh + p)) : make_float2(0.f, 0.f);
-        const uint32_t o0 = ssd_swz<8>(r0, jt) + 4 * q, o1 = ssd_swz<8>(r1, jt) + 4 * q;
-        const float2 x0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + (sx - sbase) + o0));
-        const float2 x1 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(smem + (sx - sbase) + o1));
-        *reinterpret_cast<uint32_t*>(smem + L::kY + o0) =
-            pack_bf16(fmaf(dd.x, x0.x, Y[jt][0]), fmaf(dd.y, x0.y, Y[jt][1]));
-        *reinterpret_cast<uint32_t*>(smem + L::kY + o1) =
-            pack_bf16(fmaf(dd.x, x1.x, Y[jt][2]), fmaf(dd.y, x1.y, Y[jt][3]));
-      }
-      __syncwarp();
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const int i = lane + 32 * k;
-        const int row = 16 * warp + (i >> 3), ch = i & 7;
-        if (t0 + row < t_end) {
-          const uint4 v = *reinterpret_cast<const uint4*>(smem + L::kY + ssd_swz<8>(row, ch));
-          *reinterpret_cast<uint4*>(a.y + (b * a.len + t0 + row) * channels + (int64_t)h * kSsdP + ch * 8) = v;
+          *reinterpret_cast<uint4*>(mrow + (2 * q4 + h8) * 128) = make_uint4(op[0], op[1], op[2], op[3]);
         }
       }
     }
 
-    __syncthreads();  // Bw complete; every read of the state copy is done
+    // the operands built by the warps are complete: issue Y and dS^T
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0 && ok_run) {
+      constexpr uint32_t kIdY = umma_idesc_bf16(64, 64, 0, 1);     // M K-major, X MN-major
+      constexpr uint32_t kIdOff = umma_idesc_bf16(64, 64, 0, 0);   // C~ K-major, S K-major
+      constexpr uint32_t kIdS = umma_idesc_bf16(64, N, 1, 1);      // X^T MN-major, Bw MN-major
+#pragma unroll
+      for (int hh = 0; hh < kSsdHeads; ++hh) {
+        if (hh == 1 && !pair) break;
+        const uint32_t xs = sx + hh * L::kX;
+        if (!AGG) {
+          const uint32_t dy = tmem + hh * d_off + 64;
+          const uint32_t ms = sbase + L::kM + hh * (kSsdQ * kSsdQ * 2);
+#pragma unroll
+          for (int k = 0; k < kSsdQ / 16; ++k)
+            umma_bf16(dy, umma_desc(ms + k * 256, 128, 1024), umma_desc(xs + k * 2048, 1024, 128), kIdY, k > 0);
+          const uint32_t cts = sbase + L::kCt + hh * L::kBC;
+          const uint32_t ss = sbase + L::kS + hh * (kSsdP * N * 2);
+#pragma unroll
+          for (int k = 0; k < N / 16; ++k)
+            umma_bf16(dy, umma_desc(cts + k * 256, 128, L::kSboBC), umma_desc(ss + k * 256, 128, L::kSboBC), kIdOff,
+                      true);
+        }
+        const uint32_t bws = sbase + L::kBw + hh * L::kBC;
+#pragma unroll
+        for (int k = 0; k < kSsdQ / 16; ++k)
+          umma_bf16(tmem + hh * d_off, umma_desc(xs + k * 2048, 1024, 128),
+                    umma_desc(bws + k * 2 * L::kSboBC, L::kSboBC, 128), kIdS, k > 0);
+      }
+      umma_commit(bar_y);
+    }
+    // the next chunk's copies overlap the products (its slot was read by chunk c-1)
+    if (c + L::kStages - 1 < nchunks) load_chunk(c + L::kStages - 1, (c + L::kStages - 1) % L::kStages);
+    cp_async_commit();
 
-    // dS = Bw^T X for channels 16w..16w+15, then S = e^{a cum_end} S + dS
-    {
-      float dS[KS][2][4];
+    if (ok_run) {
+      bool got = mbar_wait_bounded(bar_y, (uint32_t)(c & 1), a.wait_limit_ns);
+      got = __all_sync(0xffffffffu, got);
+      if (!got) {
+        if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+        ok_run = false;
+      }
+    }
+    tc_fence_after();
+    if (ok_run) {
+      if (!AGG) {
+        // y = Y + D x for row `row` of head hd -> bf16 -> 16-byte stores
+        const float* Dh = Ds + hd * kSsdP;
+        const unsigned char* xrow = smem + (sx - sbase) + hd * L::kX + (row >> 3) * 1024 + (row & 7) * 16;
+        const bool store = hok && t0 + row < t_end;
+        __nv_bfloat16* yrow = a.y + (b * a.len + t0 + row) * channels + (int64_t)hc * kSsdP;
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt)
+        for (int q4 = 0; q4 < 4; ++q4) {
+          float yv[16];
+          tmem_ld16(t_lane + 64 + (uint32_t)(16 * q4), yv);
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj)
+          for (int h8 = 0; h8 < 2; ++h8) {
+            const int c8 = 2 * q4 + h8;
+            const uint4 xv = *reinterpret_cast<const uint4*>(xrow + c8 * 128);
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+            uint32_t op[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dS[mt][jj][e] = 0.0f;
-#pragma unroll
-      for (int ks = 0; ks < kSsdQ / 16; ++ks) {
-        uint32_t xf[4];
-        ldsm_x4_t(xf, sx + ssd_swz<8>(16 * ks + (lane & 7) + 8 * ((lane >> 3) & 1), 2 * warp + (lane >> 4)));
-#pragma unroll
-        for (int mt = 0; mt < KS; ++mt) {
-          uint32_t bw[4];
-          ldsm_x4_t(bw, sbase + L::kBw + ssd_swz<R>(16 * ks + (lane & 7) + 8 * (lane >> 4), 2 * mt + ((lane >> 3) & 1)));
-          mma_bf16(dS[mt][0], bw, xf[0], xf[1]);
-          mma_bf16(dS[mt][1], bw, xf[2], xf[3]);
+            for (int e = 0; e < 4; ++e) {
+              const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[e]));
+              const int p = 8 * c8 + 2 * e;
+              const float d0 = Dh[p], d1 = Dh[p + 1];
+              op[e] = pack_bf16(fmaf(d0, xf.x, yv[8 * h8 + 2 * e]), fmaf(d1, xf.y, yv[8 * h8 + 2 * e + 1]));
+            }
+            if (store) *reinterpret_cast<uint4*>(yrow + 8 * c8) = make_uint4(op[0], op[1], op[2], op[3]);
+          }
         }
       }
+      // S = e^{a cum_end} S + dS for channel `row` of head hd
       const float dec = ex2_approx(cum_end);
 #pragma unroll
-      for (int mt = 0; mt < KS; ++mt)
+      for (int q4 = 0; q4 < N / 16; ++q4) {
+        float ds[16];
+        tmem_ld16(t_lane + (uint32_t)(16 * q4), ds);
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) S[mt][jj][e] = fmaf(dec, S[mt][jj][e], dS[mt][jj][e]);
+        for (int i = 0; i < 16; ++i) S[16 * q4 + i] = fmaf(dec, S[16 * q4 + i], ds[i]);
+      }
     }
-    if (!AGG) store_state_copy();
-    dt0 = ndt0;
-    dt1 = ndt1;
+    tc_fence_before();
+    ok_run = __syncthreads_and(ok_run) != 0;  // every read of G / dS / Y and of the state copy is done
+    if (!AGG && ok_run) store_state_copy();
+    dt = ndt;
   }
   cp_async_wait<0>();
 
   griddep_launch_dependents();
-  if (AGG) {
-    const int64_t agg = seq * (a.supers - 1) + j;
-    float* as = a.agg_state + agg * (kSsdP * N);
+  if (ok_run && hok) {
+    if (AGG) {
+      const int64_t agg = (b * a.heads + h) * (a.supers - 1) + j;
+      float* as = a.agg_state + (agg * kSsdP + row) * N;
 #pragma unroll
-    for (int mt = 0; mt < KS; ++mt)
+      for (int n = 0; n < N; ++n) as[n] = S[n];
+      if ((lane & 15) == 0 && warp == 0) a.agg_decay[agg] = total_log2;
+    } else if (a.final_state && j == a.supers - 1) {
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          int n, p;
-          s_index(mt, jj, e, &n, &p);
-          as[p * N + n] = S[mt][jj][e];
-        }
-    if (tid == 0) a.agg_decay[agg] = total_log2;
-  } else if (a.final_state && j == a.supers - 1) {
-    float* fs = a.final_state + (b * a.heads + h) * (int64_t)(kSsdP * N);
-#pragma unroll
-    for (int mt = 0; mt < KS; ++mt)
-#pragma unroll
-      for (int jj = 0; jj < 2; ++jj)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          int n, p;
-          s_index(mt, jj, e, &n, &p);
-          fs[p * N + n] = S[mt][jj][e];
-        }
+      for (int n = 0; n < N; ++n) a.final_state[sidx + n] = S[n];
+    }
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kSsdTmemCols) : "memory");
 }
 
 }  // namespace mamba

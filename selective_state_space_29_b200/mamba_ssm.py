@@ -58,6 +58,11 @@ _SIGNATURES = [
     ("mamba_selective_scan_complex", ctypes.c_int,
      [_P] * 10 + [_I64] * 5 + [ctypes.c_int, _P]),
     ("mamba_complex_supported_nstate", ctypes.c_int, [_I64]),
+    ("mamba_selective_scan_mimo", ctypes.c_int,
+     [_P] * 9 + [_I64] * 5 + [ctypes.c_uint, ctypes.c_int, _P]),
+    ("mamba_mimo_supported", ctypes.c_int, [_I64, _I64]),
+    ("mamba_state_update_mimo", ctypes.c_int,
+     [_P] * 8 + [_I64] * 4 + [ctypes.c_int, _P]),
     ("mamba_scan_plan", ctypes.c_int,
      [_I64, _I64, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ScanPlan)]),
     ("mamba_status_string", ctypes.c_char_p, [ctypes.c_int]),
@@ -205,6 +210,24 @@ def mamba_selective_scan_complex(u, delta, A_re, A_im, B, C, D, initial_state, y
 
 def mamba_complex_supported_nstate(nstate: int) -> bool:
     return bool(library().mamba_complex_supported_nstate(int(nstate)))
+
+
+def mamba_selective_scan_mimo(u, delta, A, B, C, D, initial_state, y, final_state, batch, len, ranks, channels,
+                              nstate, flags, dtype, stream=None):
+    st = library().mamba_selective_scan_mimo(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                             _ptr(initial_state), _ptr(y), _ptr(final_state), batch, len, ranks,
+                                             channels, nstate, flags, dtype, _stream(stream))
+    _check(st, "mamba_selective_scan_mimo")
+
+
+def mamba_state_update_mimo(state, x, delta, A, B, C, D, y, batch, ranks, channels, nstate, dtype, stream=None):
+    st = library().mamba_state_update_mimo(_ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                           _ptr(y), batch, ranks, channels, nstate, dtype, _stream(stream))
+    _check(st, "mamba_state_update_mimo")
+
+
+def mamba_mimo_supported(ranks: int, nstate: int) -> bool:
+    return bool(library().mamba_mimo_supported(int(ranks), int(nstate)))
 
 
 def mamba_scan_plan(batch, len, channels, nstate, chunk_len, dtype, sm_count=0) -> ScanPlan:
@@ -373,3 +396,39 @@ def selective_scan_backward(u, delta, A, B, C, D, dy, initial_state=None, d_fina
                                   out["dA"], out["dB"], out["dC"], out["dD"], out["d_initial_state"], batch, length,
                                   channels, nstate, dtype_code(u.dtype), stream)
     return out
+
+
+def selective_scan_mimo(u, delta, A, B, C, D=None, initial_state=None, return_final_state=True, general_a=False,
+                        y=None, final_state=None, stream=None):
+    """y, final_state = selective_scan_mimo(u, delta, A, B, C, D) on CUDA tensors.
+
+    u: (batch, len, ranks, channels); delta: (batch, len, channels); B, C:
+    (batch, len, ranks, nstate), one dtype (float32 or bfloat16); A:
+    (channels, nstate) float32; D: (channels,) or None; initial_state:
+    (batch, channels, nstate) float32 or None.  y is shaped like u."""
+    import torch
+    batch, length, ranks, channels = u.shape
+    nstate = A.shape[1]
+    for t in (u, delta, A, B, C, D, initial_state):
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+    if y is None:
+        y = torch.empty_like(u)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((batch, channels, nstate), device=u.device, dtype=torch.float32)
+    mamba_selective_scan_mimo(u, delta, A, B, C, D, initial_state, y, final_state, batch, length, ranks, channels,
+                              nstate, MAMBA_SCAN_GENERAL_A if general_a else 0, dtype_code(u.dtype), stream)
+    return y, final_state
+
+
+def state_update_mimo(state, x, delta, A, B, C, D=None, y=None, stream=None):
+    """One multi-input multi-output recurrent step, state updated in place.
+    state: (batch, channels, nstate) float32; x: (batch, ranks, channels);
+    delta: (batch, channels); B, C: (batch, ranks, nstate).  Returns y, shaped like x."""
+    import torch
+    batch, ranks, channels = x.shape
+    nstate = A.shape[1]
+    if y is None:
+        y = torch.empty_like(x)
+    mamba_state_update_mimo(state, x, delta, A, B, C, D, y, batch, ranks, channels, nstate, dtype_code(x.dtype), stream)
+    return y

@@ -15,6 +15,7 @@ Workloads (one scan or one decode chain each):
                fp32 state, bf16 x / delta / B / C / y
   ssd_mid_bf16 / ssd_long_bf16  the mid and long shapes as Mamba-2 heads of 64
                channels (48 and 32 heads): one scalar A and one step per head
+  mimo_mid_bf16  the mid shape with 4 inputs and outputs per channel
 
 Distributions: x ~ N(0,1); delta log-uniform in [lo, hi] (uniform exponent);
 B, C ~ N(0,1) per (batch, token, state), shared by all channels; D ~ N(0,1) per
@@ -116,6 +117,34 @@ class SsdWorkload:
         return dataclasses.replace(self, **kw)
 
 
+@dataclasses.dataclass(frozen=True)
+class MimoWorkload:
+    """Multi-input multi-output scan: `ranks` inputs and outputs per channel
+    sharing one state and one step per (batch, token, channel)."""
+    name: str
+    batch: int
+    length: int
+    ranks: int
+    channels: int
+    nstate: int
+    dtype: str = "bf16"
+    delta_lo: float = 1e-3
+    delta_hi: float = 1e-1
+    a_mode: str = "channel"
+    seed: int = 36
+
+    @property
+    def torch_dtype(self):
+        return _DTYPES[self.dtype]
+
+    @property
+    def token_channels(self) -> int:
+        return self.batch * self.length * self.channels
+
+    def with_(self, **kw) -> "MimoWorkload":
+        return dataclasses.replace(self, **kw)
+
+
 SCAN_WORKLOADS = {
     "tiny_f32": ScanWorkload("tiny_f32", 1, 256, 64, 16, "f32", a_mode="s4d", seed=29),
     "mid_bf16": ScanWorkload("mid_bf16", 8, 2048, 3072, 16, "bf16", seed=30),
@@ -126,6 +155,11 @@ SCAN_WORKLOADS = {
 SSD_WORKLOADS = {
     "ssd_mid_bf16": SsdWorkload("ssd_mid_bf16", 8, 2048, 48, 64, 16, seed=34),
     "ssd_long_bf16": SsdWorkload("ssd_long_bf16", 1, 1 << 20, 32, 64, 16, delta_lo=1e-4, seed=35),
+}
+# the mid scan shape with four inputs and outputs per channel (the pages give
+# no MIMO sizes; four is a small rank that keeps the state update on FMA)
+MIMO_WORKLOADS = {
+    "mimo_mid_bf16": MimoWorkload("mimo_mid_bf16", 8, 2048, 4, 3072, 16, seed=36),
 }
 DECODE_WORKLOADS = {
     "decode_bf16": DecodeWorkload("decode_bf16", 256, 5120, 16, 1000, seed=33),
@@ -288,3 +322,27 @@ def ssd_inputs(w: SsdWorkload, device="cpu", seed: int | None = None) -> dict:
                    .uniform_(0.0, math.log(16.0), generator=_gen(device, s, 5)))
     D = torch.randn((w.channels,), generator=_gen(device, s, 6), device=device, dtype=torch.float32)
     return {"x": x, "dt": dt, "A": A, "B": B, "C": C, "D": D}
+
+
+def mimo_inputs(w: MimoWorkload, device="cpu", seed: int | None = None) -> dict:
+    """u (batch, len, ranks, channels); delta (batch, len, channels); B, C
+    (batch, len, ranks, nstate) in the workload dtype; A (channels, nstate)
+    and D (channels,) fp32.  Same distributions as the scan workloads."""
+    s = w.seed if seed is None else seed
+    dt = w.torch_dtype
+    shp_x = (w.batch, w.length, w.ranks, w.channels)
+    shp_dl = (w.batch, w.length, w.channels)
+    shp_bc = (w.batch, w.length, w.ranks, w.nstate)
+    if w.length == 0 or w.batch == 0:
+        u = torch.empty(shp_x, dtype=dt, device=device)
+        delta = torch.empty(shp_dl, dtype=dt, device=device)
+        B = torch.empty(shp_bc, dtype=dt, device=device)
+        C = torch.empty(shp_bc, dtype=dt, device=device)
+    else:
+        u = _normal(shp_x, _gen(device, s, 1), device, dt)
+        delta = _log_uniform(shp_dl, _gen(device, s, 2), device, dt, w.delta_lo, w.delta_hi)
+        B = _normal(shp_bc, _gen(device, s, 3), device, dt)
+        C = _normal(shp_bc, _gen(device, s, 4), device, dt)
+    A = a_matrix(w.channels, w.nstate, w.a_mode, _gen(device, s, 5), device)
+    D = torch.randn((w.channels,), generator=_gen(device, s, 6), device=device, dtype=torch.float32)
+    return {"u": u, "delta": delta, "A": A, "B": B, "C": C, "D": D}

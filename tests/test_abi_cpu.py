@@ -239,15 +239,17 @@ def test_scan_plan_host_logic(lib):
     assert p.supers == 1 and p.kernels == 2
     assert p.jobs * p.chunk_len >= 768 * 2048 and p.jobs >= 8 * 592 * 0.9
     assert p.ctas == sms
-    # long workload: 64 groups -> split into super-chunks; still one pre-pass
-    # and one chunked kernel (aggregate jobs first, then the main jobs)
+    # long workload: 64 groups -> split into super-chunks that run from zero
+    # side by side; pre-pass, chunked kernel, correction kernel
     p = m.mamba_scan_plan(1, 1 << 20, 2048, 16, 0, m.MAMBA_BF16, sms)
-    assert p.supers > 1 and p.kernels == 2
+    assert p.supers > 1 and p.kernels == 3
     assert p.supers * 64 >= 592
     assert p.super_len * p.supers >= 1 << 20 and p.super_len * (p.supers - 1) < 1 << 20
+    # every job is a chunk of a main stream: the jobs cover each stream once
+    assert p.jobs * p.chunk_len >= 64 * (1 << 20) and (p.jobs - 64 * p.supers) * p.chunk_len < 64 * (1 << 20)
     # forced chunking
     p = m.mamba_scan_plan(2, 1000, 200, 16, 37, m.MAMBA_BF16, sms)
-    assert p.super_len == 37 and p.supers == 28 and p.kernels == 2
+    assert p.super_len == 37 and p.supers == 28 and p.kernels == 3
     # tiny problem: one CTA per four jobs
     p = m.mamba_scan_plan(1, 10, 32, 16, 0, m.MAMBA_F32, sms)
     assert p.supers == 1 and p.jobs == 1 and p.ctas == 1

@@ -26,6 +26,9 @@ DEV = "cuda"
 def _a_imag(w, mode, seed=3):
     if mode == "s4d_lin":
         return wl.complex_a_imag(w.channels, w.nstate, DEV)
+    if mode == "lin_fast":
+        # n w with a fast rate: the structured path's product chain over large turns
+        return (7.3 * torch.arange(w.nstate, device=DEV, dtype=torch.float32)).expand(w.channels, w.nstate).contiguous()
     g = torch.Generator(device=DEV).manual_seed(seed)
     hi = {"slow": 2.0, "fast": 40.0}[mode]
     return torch.empty((w.channels, w.nstate), device=DEV).uniform_(-hi, hi, generator=g).contiguous()
@@ -69,6 +72,17 @@ def test_complex_small(dtype, supers):
 @pytest.mark.parametrize("a_imag", ["slow", "fast"])
 def test_complex_state_counts_and_rotation_rates(nstate, a_imag):
     _check(SMALL.with_(nstate=nstate, length=500, a_mode="state"), a_imag=a_imag)
+
+
+@pytest.mark.parametrize("nstate", [4, 8, 16])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("delta_hi", [0.1, 3.0])
+def test_complex_structured_product_chain(nstate, dtype, delta_hi):
+    """A[n] = (n+1) a + i n w on every channel: exp(dt A_n) - 1 from two
+    complex exponentials per token and the product chain, up to large turns
+    per token (dt w up to 3 x 7.3 x 15 radians)."""
+    _check(SMALL.with_(nstate=nstate, dtype=dtype, length=500, a_mode="channel", delta_hi=delta_hi),
+           a_imag="lin_fast")
 
 
 @pytest.mark.parametrize("supers", [1, 4])
