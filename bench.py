@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long_bf16")
+    ap.add_argument("--length", type=int, default=0,
+                    help="override the workload's sequence length (smaller cases of the same generator, for profiling)")
     ap.add_argument("--decode-steps", type=int, default=1000)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
@@ -432,6 +434,8 @@ def run_ours(args):
     hbm_src = "measured" if "hbm_gbs" in peaks else "fallback"
 
     w = wl.SCAN_WORKLOADS[args.workload]
+    if args.length > 0:
+        w = w.with_(length=args.length, name=f"{w.name}_len{args.length}")
     inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
     y = torch.empty_like(inp["u"])
     hf = torch.empty((w.batch, w.channels, w.nstate), device=dev, dtype=torch.float32)

@@ -130,15 +130,24 @@ bool make_map_2d(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uin
 // producer warp; a consumer's ring holds kStages tiles of kTile tokens (the
 // ring of four consumers fits the 227 KB of shared memory of a CTA).
 // With R inputs per token (multi-input multi-output) a tile holds 1/R as
-// many tokens, so that its u, B and C' rows stay the same size.
+// many tokens, so that its u, B and C' rows stay the same size.  With eight
+// consumer warps (two per sub-partition) tiles are half as long and the
+// ring two deep, so that eight rings fit the shared memory of a CTA.
+#ifndef MAMBA_SCAN_CONSUMERS
+#define MAMBA_SCAN_CONSUMERS 4
+#endif
+constexpr int kScanConsumers = MAMBA_SCAN_CONSUMERS;
+static_assert(kScanConsumers == 4 || kScanConsumers == 8, "one or two consumer warps per sub-partition");
 template <typename TIO, int NS, int R = 1>
 struct ScanCfg {
   static constexpr bool kBf16 = sizeof(TIO) == 2;
-  static constexpr int kTile = (kBf16 ? 64 : 32) / R;
-  static constexpr int kStages = (kBf16 && NS >= 32) ? 2 : 3;
+  static constexpr int kTile = (kBf16 ? 64 : 32) / R / (kScanConsumers / 4);
+  static constexpr int kStages = (kScanConsumers == 8 || (kBf16 && NS >= 32)) ? 2 : 3;
 };
-constexpr int kScanConsumers = 4;
-constexpr int kJobsPerWarp = 8;  // chunks per consumer warp, for dynamic balance
+#ifndef MAMBA_SCAN_JOBS_PER_WARP
+#define MAMBA_SCAN_JOBS_PER_WARP 8
+#endif
+constexpr int kJobsPerWarp = MAMBA_SCAN_JOBS_PER_WARP;  // chunks per consumer warp, for dynamic balance
 // streams (channel group x super-chunk) per resident consumer warp, in percent,
 // below which sequences are cut into super-chunks
 #ifndef MAMBA_SCAN_STREAMS_PCT

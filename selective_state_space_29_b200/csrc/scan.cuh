@@ -61,6 +61,10 @@
 
 namespace mamba {
 
+#ifndef MAMBA_SCAN_PIPE
+#define MAMBA_SCAN_PIPE 0
+#endif
+
 constexpr int kCPW = 32;   // channels per warp: one lane per channel
 constexpr int kFixSegTiles = 4;  // tiles per segment of the super-chunk correction
 constexpr int kHandQ = 8;  // hand-off flags a consumer may leave for the producer to publish
@@ -205,6 +209,21 @@ __device__ __forceinline__ float expm1_small(float z) {
   const float poly = fmaf(z4, hi, fmaf(z2, lo, z));
   const float viaexp2 = ex2_approx(z * 1.4426950408889634f) - 1.0f;
   return fabsf(z) <= 0.25f ? poly : viaexp2;
+}
+
+// expm1_small's q = e^z - 1 together with d = q - z, both accurate to fp32
+// relative precision: for |z| <= 1/4 d is the polynomial without its
+// leading z (no cancellation); above, q - z does not cancel much.
+__device__ __forceinline__ void expm1_parts(float z, float& q, float& d) {
+  const float z2 = z * z;
+  const float lo = fmaf(z, 1.0f / 6.0f, 0.5f);
+  const float hi = fmaf(z2, 1.0f / 720.0f, fmaf(z, 1.0f / 120.0f, 1.0f / 24.0f));
+  const float z4 = z2 * z2;
+  const float dpoly = fmaf(z4, hi, z2 * lo);
+  const float qexp = ex2_approx(z * 1.4426950408889634f) - 1.0f;
+  const bool small = fabsf(z) <= 0.25f;
+  q = small ? z + dpoly : qexp;
+  d = small ? dpoly : qexp - z;
 }
 
 // exp(z) - 1 for z <= 0 without a branch, for bf16 data: the hardware exp2
@@ -364,8 +383,46 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
   };
   int r = 0;
   if (rows == TILE) {
+#if MAMBA_SCAN_PIPE
+    // software pipeline over token pairs: the loads and decay chains of
+    // pair k+1 are issued before the state updates of pair k, so their
+    // latency (shared-memory loads, exp2) overlaps the updates
+    float2 ea[NS / 2], eb[NS / 2];
+    TIO xa = su[0], xb = su[kCPW];
+    float da = to_f32(sdl[0]), db = to_f32(sdl[kCPW]);
+    chain(da, ea);
+    chain(db, eb);
+#pragma unroll 2
+    for (; r < TILE; r += 2) {
+      float2 na[NS / 2], nb[NS / 2];
+      TIO nxa = xa, nxb = xb;
+      float nda = 0.0f, ndb = 0.0f;
+      if (r + 2 < TILE) {
+        nxa = su[(r + 2) * kCPW];
+        nxb = su[(r + 3) * kCPW];
+        nda = to_f32(sdl[(r + 2) * kCPW]);
+        ndb = to_f32(sdl[(r + 3) * kCPW]);
+        chain(nda, na);
+        chain(ndb, nb);
+      }
+      const float s0 = token_update<TIO, NS>(ea, bt[r], ct[r], xa, g);
+      const float s1 = token_update<TIO, NS>(eb, bt[r + 1], ct[r + 1], xb, g);
+      emit(s0, xa, da);
+      emit(s1, xb, db);
+#pragma unroll
+      for (int k = 0; k < NS / 2; ++k) {
+        ea[k] = na[k];
+        eb[k] = nb[k];
+      }
+      xa = nxa;
+      xb = nxb;
+      da = nda;
+      db = ndb;
+    }
+#else
 #pragma unroll 4
     for (; r < TILE; r += 2) pair(r);
+#endif
   } else {
     for (; r + 1 < rows; r += 2) pair(r);
     if (r < rows) {

@@ -49,7 +49,7 @@ constexpr int kSsdQ = 64;       // tokens per chunk
 constexpr int kSsdP = 64;       // channels per head
 constexpr int kSsdWarps = 4;    // one warpgroup per CTA
 constexpr int kSsdHeads = 2;    // heads per CTA
-constexpr int kSsdTmemCols = 128;  // G / dS^T in columns [0, 64), Y in [64, 128)
+constexpr int kSsdTmemCols = 256;  // dS^T in columns [0, 64), Y in [64, 128), G in [128, 192)
 
 struct SsdArgs {
   const __nv_bfloat16* x;       // (batch, len, heads*64)
@@ -146,6 +146,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 template <int N>
 struct SsdSmem {
   static constexpr int kStages = N >= 32 ? 2 : 3;
+  static_assert(kStages >= 2, "chunk c+1 must be resident while chunk c is finished");
   static constexpr int kX = kSsdQ * kSsdP * 2;           // one head's x tile (8 KB)
   static constexpr int kBC = kSsdQ * N * 2;              // one B or C tile
   static constexpr int kStage = kSsdHeads * kX + 2 * kBC;  // x of both heads, B, C
@@ -293,12 +294,41 @@ ssd_chunk_kernel(const SsdArgs a) {
   const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);  // this warp's sub-partition, + lane i = thread
   const uint32_t d_off = (uint32_t)(16 * 1) << 16;                // head 1's accumulators: lanes 16-31
 
-  // prologue: the first kStages-1 chunks
+  // Shared-memory descriptors, built once: a K step (or another ring slot /
+  // head) only moves the start address, the low 14 bits in 16-byte units
+  const uint64_t dBC = umma_desc(sbase, 128, L::kSboBC);      // K-major [rows][N]: C, B, C~, S
+  const uint64_t dM = umma_desc(sbase, 128, 1024);            // K-major [64][64]: M
+  const uint64_t dX = umma_desc(sbase, 1024, 128);            // MN-major x (B of Y, A of dS^T)
+  const uint64_t dBw = umma_desc(sbase, L::kSboBC, 128);      // MN-major Bw (B of dS^T)
+  auto at = [](uint64_t d, uint32_t off) { return d + (uint64_t)(off >> 4); };
+  constexpr uint32_t kIdG = umma_idesc_bf16(64, 64, 0, 0);
+  constexpr uint32_t kIdY = umma_idesc_bf16(64, 64, 0, 1);     // M K-major, x MN-major
+  constexpr uint32_t kIdOff = umma_idesc_bf16(64, 64, 0, 0);   // C~ K-major, S K-major
+  constexpr uint32_t kIdS = umma_idesc_bf16(64, N, 1, 1);      // x^T MN-major, Bw MN-major
+  constexpr uint32_t kColS = 0, kColY = 64, kColG = 128;       // tensor-memory columns
+  // G = C B^T of chunk c (slot) into columns [128, 192) of both heads' lanes
+  auto issue_g = [&](int slot) {
+    const uint32_t ob = slot * L::kStage + kSsdHeads * L::kX;  // B tile, then C tile
 #pragma unroll
-  for (int s = 0; s < L::kStages - 1; ++s) {
+    for (int hh = 0; hh < kSsdHeads; ++hh) {
+      if (hh == 1 && !pair) break;
+#pragma unroll
+      for (int k = 0; k < N / 16; ++k)
+        umma_bf16(tmem + hh * d_off + kColG, at(dBC, ob + L::kBC + k * 256), at(dBC, ob + k * 256), kIdG, k > 0);
+    }
+    umma_commit(bar_g);
+  };
+
+  // prologue: the first kStages chunks, and G of chunk 0
+#pragma unroll
+  for (int s = 0; s < L::kStages; ++s) {
     if (s < nchunks) load_chunk(s, s);
     cp_async_commit();
   }
+  cp_async_wait<L::kStages - 1>();  // chunk 0
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+  if (!AGG && tid == 0 && nchunks > 0) issue_g(0);
   float dt = load_dt(0);
   bool ok_run = true;
 
@@ -306,6 +336,9 @@ ssd_chunk_kernel(const SsdArgs a) {
     const int slot = c % L::kStages;
     const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
     const float ndt = load_dt(c + 1);
+    const uint32_t ox = slot * L::kStage;                 // x tiles of the slot
+    const uint32_t ob = ox + kSsdHeads * L::kX;           // B tile
+    const uint32_t oc = ob + L::kBC;                      // C tile
 
     // running log2 decay inside the chunk for this thread's head: an
     // inclusive scan over the 16 lanes of the half-warp, then across warps
@@ -317,10 +350,7 @@ ssd_chunk_kernel(const SsdArgs a) {
     }
     if ((lane & 15) == 15) wsum[warp * kSsdHeads + hd] = v;
     const float wgt = a.euler ? dt : expm1f(dt * a_h) / a_h;
-
-    cp_async_wait<L::kStages - 2>();  // this thread's copies of chunk c have landed
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // visible to the tensor core
-    __syncthreads();                  // everyone's; the warp sums; chunk c-1 is done with its slot
+    __syncthreads();  // the warp sums
     float pre = 0.0f;
     for (int w2 = 0; w2 < warp; ++w2) pre += wsum[w2 * kSsdHeads + hd];
     const float cum = v + pre;
@@ -330,28 +360,10 @@ ssd_chunk_kernel(const SsdArgs a) {
     cum_s[hd * kSsdQ + row] = cum;
     w_s[hd * kSsdQ + row] = wgt;
 
-    const uint32_t sx = sbase + slot * L::kStage;
-    const uint32_t sb = sx + kSsdHeads * L::kX;
-    const uint32_t sc = sb + L::kBC;
-    constexpr uint32_t kIdG = umma_idesc_bf16(64, 64, 0, 0);
-    if (!AGG && tid == 0) {
-      // G = C B^T for both heads (identical; one accumulator per head's lanes)
-#pragma unroll
-      for (int hh = 0; hh < kSsdHeads; ++hh) {
-        if (hh == 1 && !pair) break;
-#pragma unroll
-        for (int k = 0; k < N / 16; ++k)
-          umma_bf16(tmem + hh * d_off, umma_desc(sc + k * 256, 128, L::kSboBC), umma_desc(sb + k * 256, 128, L::kSboBC),
-                    kIdG, k > 0);
-      }
-      umma_commit(bar_g);
-    }
-    __syncthreads();  // cum and w of the chunk are in shared memory
-
     // C~ = e^{a cum_t} C_t and Bw = e^{a(cum_end - cum_s)} w_s B_s, row `row` of head hd
     {
       const float fB = ex2_approx(cum_end - cum) * wgt;
-      const unsigned char* brow = smem + (sb - sbase) + (row >> 3) * L::kSboBC + (row & 7) * 16;
+      const unsigned char* brow = smem + ob + (row >> 3) * L::kSboBC + (row & 7) * 16;
       // Bw [s][n] as MN-major (N = n, K = s): (s/8) (N/8 128) + (n/8) 128 + (s%8) 16 + (n%8) 2,
       // the same bytes as the K-major [s][n] placement of B
       unsigned char* bwrow = smem + L::kBw + hd * L::kBC + (row >> 3) * L::kSboBC + (row & 7) * 16;
@@ -369,7 +381,7 @@ ssd_chunk_kernel(const SsdArgs a) {
       }
       if (!AGG) {
         const float fC = ex2_approx(cum);
-        const unsigned char* crow = smem + (sc - sbase) + (row >> 3) * L::kSboBC + (row & 7) * 16;
+        const unsigned char* crow = smem + oc + (row >> 3) * L::kSboBC + (row & 7) * 16;
         unsigned char* ctrow = smem + L::kCt + hd * L::kBC + (row >> 3) * L::kSboBC + (row & 7) * 16;
 #pragma unroll
         for (int n8 = 0; n8 < N / 8; ++n8) {
@@ -385,6 +397,7 @@ ssd_chunk_kernel(const SsdArgs a) {
         }
       }
     }
+    __syncthreads();  // cum and w of the chunk are in shared memory
 
     if (!AGG) {
       // M row `row` of head hd from G: causal mask, decay and input weight
@@ -401,7 +414,7 @@ ssd_chunk_kernel(const SsdArgs a) {
 #pragma unroll
       for (int q4 = 0; q4 < 4 && ok_run; ++q4) {
         float g[16];
-        tmem_ld16(t_lane + (uint32_t)(16 * q4), g);
+        tmem_ld16(t_lane + kColG + (uint32_t)(16 * q4), g);
 #pragma unroll
         for (int h8 = 0; h8 < 2; ++h8) {
           uint32_t op[4];
@@ -417,43 +430,36 @@ ssd_chunk_kernel(const SsdArgs a) {
       }
     }
 
-    // the operands built by the warps are complete: issue Y and dS^T
+    // the operands built by the warps, and chunk c+1's copies, are complete:
+    // issue Y and dS^T of chunk c, then G of chunk c+1 behind them
+    cp_async_wait<L::kStages - 2>();
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     if (tid == 0 && ok_run) {
-      constexpr uint32_t kIdY = umma_idesc_bf16(64, 64, 0, 1);     // M K-major, X MN-major
-      constexpr uint32_t kIdOff = umma_idesc_bf16(64, 64, 0, 0);   // C~ K-major, S K-major
-      constexpr uint32_t kIdS = umma_idesc_bf16(64, N, 1, 1);      // X^T MN-major, Bw MN-major
 #pragma unroll
       for (int hh = 0; hh < kSsdHeads; ++hh) {
         if (hh == 1 && !pair) break;
-        const uint32_t xs = sx + hh * L::kX;
+        const uint32_t xs = ox + hh * L::kX;
         if (!AGG) {
-          const uint32_t dy = tmem + hh * d_off + 64;
-          const uint32_t ms = sbase + L::kM + hh * (kSsdQ * kSsdQ * 2);
+          const uint32_t dy = tmem + hh * d_off + kColY;
+          const uint32_t ms = L::kM + hh * (kSsdQ * kSsdQ * 2);
 #pragma unroll
-          for (int k = 0; k < kSsdQ / 16; ++k)
-            umma_bf16(dy, umma_desc(ms + k * 256, 128, 1024), umma_desc(xs + k * 2048, 1024, 128), kIdY, k > 0);
-          const uint32_t cts = sbase + L::kCt + hh * L::kBC;
-          const uint32_t ss = sbase + L::kS + hh * (kSsdP * N * 2);
+          for (int k = 0; k < kSsdQ / 16; ++k) umma_bf16(dy, at(dM, ms + k * 256), at(dX, xs + k * 2048), kIdY, k > 0);
+          const uint32_t cts = L::kCt + hh * L::kBC;
+          const uint32_t ss = L::kS + hh * (kSsdP * N * 2);
 #pragma unroll
-          for (int k = 0; k < N / 16; ++k)
-            umma_bf16(dy, umma_desc(cts + k * 256, 128, L::kSboBC), umma_desc(ss + k * 256, 128, L::kSboBC), kIdOff,
-                      true);
+          for (int k = 0; k < N / 16; ++k) umma_bf16(dy, at(dBC, cts + k * 256), at(dBC, ss + k * 256), kIdOff, true);
         }
-        const uint32_t bws = sbase + L::kBw + hh * L::kBC;
+        const uint32_t bws = L::kBw + hh * L::kBC;
 #pragma unroll
         for (int k = 0; k < kSsdQ / 16; ++k)
-          umma_bf16(tmem + hh * d_off, umma_desc(xs + k * 2048, 1024, 128),
-                    umma_desc(bws + k * 2 * L::kSboBC, L::kSboBC, 128), kIdS, k > 0);
+          umma_bf16(tmem + hh * d_off + kColS, at(dX, xs + k * 2048), at(dBw, bws + k * 2 * L::kSboBC), kIdS, k > 0);
       }
       umma_commit(bar_y);
+      if (!AGG && c + 1 < nchunks) issue_g((c + 1) % L::kStages);
     }
-    // the next chunk's copies overlap the products (its slot was read by chunk c-1)
-    if (c + L::kStages - 1 < nchunks) load_chunk(c + L::kStages - 1, (c + L::kStages - 1) % L::kStages);
-    cp_async_commit();
 
     if (ok_run) {
       bool got = mbar_wait_bounded(bar_y, (uint32_t)(c & 1), a.wait_limit_ns);
@@ -468,13 +474,13 @@ ssd_chunk_kernel(const SsdArgs a) {
       if (!AGG) {
         // y = Y + D x for row `row` of head hd -> bf16 -> 16-byte stores
         const float* Dh = Ds + hd * kSsdP;
-        const unsigned char* xrow = smem + (sx - sbase) + hd * L::kX + (row >> 3) * 1024 + (row & 7) * 16;
+        const unsigned char* xrow = smem + ox + hd * L::kX + (row >> 3) * 1024 + (row & 7) * 16;
         const bool store = hok && t0 + row < t_end;
         __nv_bfloat16* yrow = a.y + (b * a.len + t0 + row) * channels + (int64_t)hc * kSsdP;
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           float yv[16];
-          tmem_ld16(t_lane + 64 + (uint32_t)(16 * q4), yv);
+          tmem_ld16(t_lane + kColY + (uint32_t)(16 * q4), yv);
 #pragma unroll
           for (int h8 = 0; h8 < 2; ++h8) {
             const int c8 = 2 * q4 + h8;
@@ -492,19 +498,23 @@ ssd_chunk_kernel(const SsdArgs a) {
           }
         }
       }
-      // S = e^{a cum_end} S + dS for channel `row` of head hd
+      // S = e^{a cum_end} S + dS for channel `row` of head hd; its bf16 copy
+      // feeds the next chunk's C~ S_in (this chunk's products are done)
       const float dec = ex2_approx(cum_end);
 #pragma unroll
       for (int q4 = 0; q4 < N / 16; ++q4) {
         float ds[16];
-        tmem_ld16(t_lane + (uint32_t)(16 * q4), ds);
+        tmem_ld16(t_lane + kColS + (uint32_t)(16 * q4), ds);
 #pragma unroll
         for (int i = 0; i < 16; ++i) S[16 * q4 + i] = fmaf(dec, S[16 * q4 + i], ds[i]);
       }
+      if (!AGG) store_state_copy();
     }
     tc_fence_before();
-    ok_run = __syncthreads_and(ok_run) != 0;  // every read of G / dS / Y and of the state copy is done
-    if (!AGG && ok_run) store_state_copy();
+    ok_run = __syncthreads_and(ok_run) != 0;  // slot c is read; every read of Y / dS is done
+    // chunk c + kStages into the slot chunk c used
+    if (c + L::kStages < nchunks) load_chunk(c + L::kStages, slot);
+    cp_async_commit();
     dt = ndt;
   }
   cp_async_wait<0>();
