@@ -261,8 +261,9 @@ int mamba_selective_scan_host(const void *u, const void *delta, const float *A,
  *
  * It runs the forward scan once more, keeping only the state before every
  * tile, then one warp per (batch, 32-channel group) walks the sequence in
- * reverse, recomputing each tile's states from its checkpoint (stream-ordered
- * scratch: the checkpoints and [T][32][nstate] floats per warp).  With
+ * reverse, recomputing each tile's states from its checkpoint, half a tile at
+ * a time (stream-ordered scratch: the checkpoints and [T/2 + 1][32][nstate]
+ * floats per warp, T = 64 tokens for bf16 and 32 for float32).  With
  * 16-byte aligned rows (channels * element size and nstate * element size
  * multiples of 16, tensors 16-byte aligned) each tile's inputs are first
  * staged in shared memory (16 KB per warp).  dA, dB,

@@ -23,11 +23,12 @@
 // Work decomposition: a warp takes a (batch row, 32-channel group) stream at
 // a time, a lane per channel, and walks its tokens in reverse.  The states
 // are recomputed tile by tile: the forward kernel leaves the state before
-// every tile of T tokens in a checkpoint array; the warp re-runs a tile
-// forward from its checkpoint, writing h_t for each token to a per-warp
-// scratch area ([T][32][N], 64 bytes per lane and token at N = 16, read
-// back one token ahead of use; 227 MB over the resident warps, so it lives
-// in DRAM), then walks the tile in reverse.  dB and dC are a reduce-scatter
+// every tile of T tokens in a checkpoint array; the warp takes a tile in
+// two halves, the later first: it re-runs the tile forward from its
+// checkpoint through the half's end, writing the half's states h_t to a
+// per-warp scratch area ([T/2 + 1][32][N], 64 bytes per lane and token at
+// N = 16, read back one token ahead of use; about 78 MB over the resident
+// warps, so it stays in L2), then walks the half in reverse.  dB and dC are a reduce-scatter
 // (lane i ends with the sum of value i) and one atomic add per lane.  When
 // rows are 16-byte aligned, the warp first copies the tile's u, Delta and
 // dy rows and its B, C rows into its shared memory (one round of 16-byte
@@ -397,11 +398,26 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
       if constexpr (STAGED) load_row_smem<TIO, NS>(sC + k * NS, v);
       else load_row<TIO, NS>(a.C + tok * NS, v, a.vec_rows);
     };
-    // forward over the tile: S[k] = h after token t0 + k
+    // The tile goes in two halves, the later one first, so that the scratch
+    // holds half a tile of states (and stays in L2): for each half, a
+    // forward pass from the checkpoint through the half's end keeps
+    // S[0] = h before the half's first token and S[1 + i] = h after its
+    // token i; the reverse steps then read h_{t-1} from S one token ahead.
+    const int H = T / 2;
+    for (int half = 1; half >= 0; --half) {
+    const int start = half * H;
+    if (start >= rows) continue;
+    const int end = (start + H < rows) ? start + H : rows;
+    auto put = [&](int slot, const float (&v)[NS]) {
+#pragma unroll
+      for (int n = 0; n < NS; n += 4)
+        *reinterpret_cast<float4*>(S + (size_t)slot * 32 * NS + n) = make_float4(v[n], v[n + 1], v[n + 2], v[n + 3]);
+    };
     float h[NS];
 #pragma unroll
     for (int n = 0; n < NS; ++n) h[n] = active ? ck[n] : 0.0f;
-    for (int k = 0; k < rows; ++k) {
+    if (start == 0) put(0, h);
+    for (int k = 0; k < end; ++k) {
       const int64_t tok = b * a.len + t0 + k;
       const float x = get_x(k, tok);
       const float dt = get_dt(k, tok);
@@ -410,32 +426,26 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
       decays<NS, STRUCT>(dt, An, q);
 #pragma unroll
       for (int n = 0; n < NS; ++n) h[n] = fmaf(1.0f + q[n], h[n], q[n] * iA[n] * bv[n] * x);
-#pragma unroll
-      for (int n = 0; n < NS; n += 4)
-        *reinterpret_cast<float4*>(S + (size_t)k * 32 * NS + n) = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
+      if (k == start - 1) put(0, h);
+      if (k >= start) put(k - start + 1, h);
     }
-    // reverse over the tile; h holds h_t, hp is read back as h_{t-1}, one
+    // reverse over the half; h holds h_t, hp is read back as h_{t-1}, one
     // token ahead of its use (hn)
     auto read_prev = [&](int k, float (&v)[NS]) {  // h_{t0+k-1}
-      if (k > 0) {
 #pragma unroll
-        for (int n = 0; n < NS; n += 4) {
-          const float4 w = *reinterpret_cast<const float4*>(S + (size_t)(k - 1) * 32 * NS + n);
-          v[n] = w.x; v[n + 1] = w.y; v[n + 2] = w.z; v[n + 3] = w.w;
-        }
-      } else {
-#pragma unroll
-        for (int n = 0; n < NS; ++n) v[n] = active ? ck[n] : 0.0f;
+      for (int n = 0; n < NS; n += 4) {
+        const float4 w = *reinterpret_cast<const float4*>(S + (size_t)(k - start) * 32 * NS + n);
+        v[n] = w.x; v[n + 1] = w.y; v[n + 2] = w.z; v[n + 3] = w.w;
       }
     };
     float hn[NS];
-    read_prev(rows - 1, hn);
-    for (int k = rows - 1; k >= 0; --k) {
+    read_prev(end - 1, hn);
+    for (int k = end - 1; k >= start; --k) {
       const int64_t tok = b * a.len + t0 + k;
       float hp[NS];
 #pragma unroll
       for (int n = 0; n < NS; ++n) hp[n] = hn[n];
-      if (k > 0) read_prev(k - 1, hn);
+      if (k > start) read_prev(k - 1, hn);
       const float x = get_x(k, tok);
       const float dt = get_dt(k, tok);
       const float gy = get_dy(k, tok);
@@ -496,6 +506,7 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
       if (lane < NS) atomicAdd(a.dB + tok * NS + lane, s);
       else if (lane < 2 * NS) atomicAdd(a.dC + tok * NS + (lane - NS), s);
     }
+    }  // half
   }
   if (active) {
 #pragma unroll
@@ -520,7 +531,7 @@ scan_backward_kernel(const BwdArgs<TIO> a) {
   const int64_t wid = (int64_t)blockIdx.x * kBwdWarps + warp;
   const int64_t nwarps = (int64_t)gridDim.x * kBwdWarps;
   const int64_t streams = a.batch * a.groups_d;
-  float* S = a.scratch + (size_t)wid * (size_t)a.tile * 32 * NS + (size_t)lane * NS;  // + k * 32 * NS
+  float* S = a.scratch + (size_t)wid * (size_t)(a.tile / 2 + 1) * 32 * NS + (size_t)lane * NS;  // + k * 32 * NS
   // work item = (super-chunk j, stream), the later super-chunks first
   for (int64_t item = wid; item < (int64_t)a.supers * streams; item += nwarps) {
     const int j = a.supers - 1 - (int)(item / streams);

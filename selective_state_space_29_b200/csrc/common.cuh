@@ -183,4 +183,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// cp.async groups: close the copies issued so far into a group; wait until
+// at most N of this thread's groups are still in flight
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 }  // namespace mamba

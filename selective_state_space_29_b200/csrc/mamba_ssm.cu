@@ -206,11 +206,13 @@ Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, 
 }
 
 struct ScratchLayout {
-  size_t ctr, done, fix_segs, ring, ring_sd, agg_h, agg_sd, cum, cs, chan, total;
+  size_t ctr, done, fix_segs, ring, ring_sd, agg_h, agg_sd, cum, cs, bs, chan, total;
   int64_t segs_max;  // correction segments of a full super-chunk
 };
 
-ScratchLayout scratch_layout(const Plan& pl, int ns, int64_t batch, int64_t len, int tile, int ranks = 1) {
+// widen_b: bf16 data, whose B rows the pre-pass widens to fp32 in scratch
+ScratchLayout scratch_layout(const Plan& pl, int ns, int64_t batch, int64_t len, int tile, bool widen_b,
+                             int ranks = 1) {
   auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
   const int64_t S = pl.supers;
   const int64_t streams = S * pl.groups;
@@ -227,8 +229,9 @@ ScratchLayout scratch_layout(const Plan& pl, int ns, int64_t batch, int64_t len,
   s.agg_sd = al(sizeof(float) * (size_t)aggs * kCPW);
   s.cum = al(sizeof(float) * (size_t)aggs * (size_t)s.segs_max * kCPW);
   s.cs = al(sizeof(float) * (size_t)batch * (size_t)len * (size_t)ranks * (size_t)ns);
+  s.bs = widen_b ? s.cs : 0;
   s.chan = al(sizeof(float) * 4 * (size_t)pl.groups_d * (size_t)kCPW);
-  s.total = s.ctr + s.done + s.fix_segs + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.cum + s.cs + s.chan;
+  s.total = s.ctr + s.done + s.fix_segs + s.ring + s.ring_sd + s.agg_h + s.agg_sd + s.cum + s.cs + s.bs + s.chan;
   return s;
 }
 
@@ -320,7 +323,8 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
                    unsigned char* scratch, float* ckpt = nullptr) {
   constexpr int TILE = ScanCfg<TIO, NS, R>::kTile;
   constexpr int STAGES = ScanCfg<TIO, NS, R>::kStages;
-  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, TILE, R);
+  constexpr bool kWidenB = sizeof(TIO) == 2;
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, TILE, kWidenB, R);
   unsigned char* cur = scratch;
   int* counters = reinterpret_cast<int*>(cur); cur += sl.ctr;
   int* done = reinterpret_cast<int*>(cur); cur += sl.done;
@@ -331,12 +335,15 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   float* agg_sd = reinterpret_cast<float*>(cur); cur += sl.agg_sd;
   float* cum = reinterpret_cast<float*>(cur); cur += sl.cum;
   float* cs = reinterpret_cast<float*>(cur); cur += sl.cs;
+  float* bs = kWidenB ? reinterpret_cast<float*>(cur) : nullptr; cur += sl.bs;
   float4* chan = reinterpret_cast<float4*>(cur);
 
   // tile loads through TMA when every operand can be described by a tensor map
   const size_t es = sizeof(TIO);
-  bool tma = aligned(u, 16) && aligned(delta, 16) && aligned(B, 16) && (channels * (int64_t)es) % 16 == 0 &&
-             (NS * es) % 16 == 0 && encode_fn() != nullptr;
+  // (B rows are read as fp32: the input itself, or its widened copy)
+  const void* b32 = kWidenB ? static_cast<const void*>(bs) : B;
+  bool tma = aligned(u, 16) && aligned(delta, 16) && aligned(b32, 16) && (channels * (int64_t)es) % 16 == 0 &&
+             (NS * sizeof(float)) % 16 == 0 && encode_fn() != nullptr;
   CUtensorMap mu, mdl, mb, mc;
   std::memset(&mu, 0, sizeof(mu));
   std::memset(&mdl, 0, sizeof(mdl));
@@ -346,7 +353,7 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
     const uint64_t rows = (uint64_t)batch * (uint64_t)len;
     tma = make_map_2d(&mu, u, dtype, (uint64_t)channels, rows * R, kCPW, TILE * R) &&
           make_map_2d(&mdl, delta, dtype, (uint64_t)channels, rows, kCPW, TILE) &&
-          make_map_2d(&mb, B, dtype, NS, rows * R, NS, TILE * R) &&
+          make_map_2d(&mb, b32, MAMBA_F32, NS, rows * R, NS, TILE * R) &&
           make_map_2d(&mc, cs, MAMBA_F32, NS, rows * R, NS, TILE * R);
   }
 
@@ -357,6 +364,10 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   p.ckpt = ckpt;
   p.ring = ring; p.ring_sd = ring_sd; p.agg_h = agg_h; p.agg_sd = agg_sd; p.cum = cum; p.fix_segs = fix_segs;
   p.segs_max = (int)sl.segs_max;
+  p.fix_vec = (aligned(delta, 16) && aligned(y, 16) && aligned(C, 16) && (channels * (int64_t)es) % 16 == 0 &&
+               (NS * es) % 16 == 0)
+                  ? 1
+                  : 0;
   p.batch = batch; p.len = len; p.channels = channels;
   p.groups_d = pl.groups_d; p.groups = (int)pl.groups;
   p.supers = pl.supers; p.super_len = pl.super_len; p.chunk_len = pl.chunk_len;
@@ -394,7 +405,7 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   p.done = done;
 
   // pre-pass: zero the counters and progress flags, C' = C / (n+1) in fp32,
-  // and the per-channel constants
+  // B in fp32 (bf16 data), and the per-channel constants
   {
     const int64_t zero_words = (int64_t)((sl.ctr + sl.done + sl.fix_segs) / sizeof(int));
     const int64_t total_c = batch * len * R * NS;
@@ -402,7 +413,8 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
     const int64_t total = zero_words + total_c + chan_padded;
     if ((total + 255) / 256 > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
     scan_prep_kernel<TIO, NS><<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
-        counters, zero_words, static_cast<const TIO*>(C), cs, total_c, A, D, chan, channels, chan_padded,
+        counters, zero_words, static_cast<const TIO*>(C), cs, static_cast<const TIO*>(B), bs, total_c, A, D, chan,
+        channels, chan_padded,
         (flags & MAMBA_SCAN_GENERAL_A) ? 1 : 0);
     if (cudaGetLastError() != cudaSuccess) return MAMBA_ERR_CUDA;
   }
@@ -417,8 +429,10 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   if (S > 1) {
     const int phases = (int)fix_phases;
     const int64_t blocks = (fix_warps + kFixWarps - 1) / kFixWarps;
-    if (launch_pdl(scan_fix_kernel<TIO, NS, TILE, CKPT, R>, dim3((unsigned)blocks), dim3(kFixWarps * 32), 0, stream,
-                   p, phases) != cudaSuccess)
+    constexpr int fix_smem = kFixWarps * fix_stage_bytes<TIO, NS, TILE, R>();
+    static_assert(fix_smem <= 48 * 1024, "correction staging within the default shared-memory limit");
+    if (launch_pdl(scan_fix_kernel<TIO, NS, TILE, CKPT, R>, dim3((unsigned)blocks), dim3(kFixWarps * 32), fix_smem,
+                   stream, p, phases) != cudaSuccess)
       return MAMBA_ERR_CUDA;
   }
   return MAMBA_OK;
@@ -435,7 +449,7 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   if (int st = current_sms(&sms)) return st;
   const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO, NS>::kTile, user_chunk);
   if (pl.groups > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
-  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, ScanCfg<TIO, NS>::kTile);
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, ScanCfg<TIO, NS>::kTile, sizeof(TIO) == 2);
   unsigned char* scratch = nullptr;
   if (noalloc) {
     if (sl.total > kNoAllocScratchBytes) return MAMBA_ERR_UNSUPPORTED;  // needs more than the fixed array
@@ -471,7 +485,7 @@ int launch_scan_mimo(const void* u, const void* delta, const float* A, const voi
   if (int st = current_sms(&sms)) return st;
   const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO, NS, R>::kTile, 0);
   if (pl.groups > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
-  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, ScanCfg<TIO, NS, R>::kTile, R);
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, ScanCfg<TIO, NS, R>::kTile, sizeof(TIO) == 2, R);
   unsigned char* scratch = nullptr;
   if (scratch_alloc(reinterpret_cast<void**>(&scratch), sl.total, stream) != cudaSuccess) return MAMBA_ERR_CUDA;
   const int status = launch_scan_on<TIO, NS, kZOH, false, R>(u, delta, A, B, C, D, h0, y, final_state, batch, len,
@@ -600,12 +614,14 @@ __global__ void expire_wait_kernel(uint64_t limit_ns) {
 }
 
 // --- Mamba-2's restricted scan (ssd.cuh) ------------------------------------
-// Super-chunks per (batch row, head): one when the (batch row, head) pairs
-// fill at least half of the resident CTA slots, else as many as fit the
-// slots in one wave (each super-chunk but the last costs an extra,
-// state-only pass over its x and B).
+// Super-chunks per sequence (a CTA's unit): one when the sequences fill at
+// least half of the resident CTA slots, else enough for two waves of slots
+// (each super-chunk but the last costs an extra, state-only pass over its
+// x and B, but a CTA walks its chunks in order, so parallelism wins for
+// long sequences).
 int64_t ssd_supers(int64_t seqs, int64_t chunks, int64_t slots, int64_t requested) {
-  int64_t s = requested > 0 ? requested : (seqs * 2 >= slots ? 1 : std::max<int64_t>(1, slots / seqs));
+  int64_t s = requested > 0 ? requested
+                            : (seqs * 2 >= slots ? 1 : std::max<int64_t>(1, (2 * slots + seqs - 1) / seqs));
   return std::max<int64_t>(1, std::min(s, chunks));
 }
 
@@ -659,6 +675,10 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
 template <typename TIO, int N>
 int launch_complex(ComplexArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream) {
   using L = ComplexSmem<TIO, N>;
+  constexpr int kES = (int)sizeof(TIO);
+  a.groups = (int)((a.channels + L::kCPW - 1) / L::kCPW);
+  a.async = ((int64_t)a.channels * kES) % 16 == 0 && (N * kES) % 16 == 0 && aligned(a.u, 16) &&
+            aligned(a.delta, 16) && aligned(a.y, 16) && aligned(a.B, 16) && aligned(a.C, 16);
   auto main_k = complex_scan_kernel<TIO, N, false>;
   auto agg_k = complex_scan_kernel<TIO, N, true>;
   if (cudaFuncSetAttribute(main_k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess ||
@@ -671,7 +691,12 @@ int launch_complex(ComplexArgs a, int64_t batch, int64_t supers_req, cudaStream_
     return MAMBA_ERR_CUDA;
   const int64_t seqs = batch * a.groups;  // one warp each
   const int64_t blocks = (a.len + kCplxBlock - 1) / kCplxBlock;
-  int64_t S = ssd_supers(seqs, blocks, (int64_t)sms * per_sm * kCplxWarps, supers_req);
+  // one super-chunk per sequence when the warps fill at least half of the
+  // slots, else as many as fit the slots in one wave (the aggregate pass
+  // costs nearly a full pass here: its exponentials dominate)
+  const int64_t slots = (int64_t)sms * per_sm * kCplxWarps;
+  int64_t S = supers_req > 0 ? supers_req : (seqs * 2 >= slots ? 1 : std::max<int64_t>(1, slots / seqs));
+  S = std::max<int64_t>(1, std::min(S, blocks));
   const int64_t per = (blocks + S - 1) / S;
   S = (blocks + per - 1) / per;
   a.super_len = per * kCplxBlock;
@@ -740,7 +765,7 @@ int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate
   out->chunk_len = pl.chunk_len;
   out->jobs = full_jobs(pl);
   out->kernels = kernels_per_call(pl);
-  out->scratch_bytes = (int64_t)scratch_layout(pl, (int)nstate, batch, len, tile_for(dtype)).total;
+  out->scratch_bytes = (int64_t)scratch_layout(pl, (int)nstate, batch, len, tile_for(dtype), dtype == MAMBA_BF16).total;
   out->ctas = std::min<int64_t>(sms, (out->jobs + kScanConsumers - 1) / kScanConsumers);
   return MAMBA_OK;
 }
@@ -926,7 +951,7 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
         const int64_t ctas = std::min<int64_t>((items + kBwdWarps - 1) / kBwdWarps, kBwdCtasPerSm * (int64_t)sms);
         auto al = [](size_t b) { return (b + 255) & ~size_t(255); };
         const size_t ck_bytes = al(sizeof(float) * (size_t)batch * (size_t)ntiles * (size_t)channels * NS);
-        const size_t sc_bytes = al(sizeof(float) * (size_t)ctas * kBwdWarps * T * 32 * NS);
+        const size_t sc_bytes = al(sizeof(float) * (size_t)ctas * kBwdWarps * (T / 2 + 1) * 32 * NS);
         const size_t mu_bytes = al(sizeof(float) * (size_t)supers * (size_t)streams * 32 * NS);
         const size_t sd_bytes = al(sizeof(float) * (size_t)supers * (size_t)streams * 32);
         unsigned char* mem = nullptr;
@@ -1200,8 +1225,6 @@ int mamba_selective_scan_complex(const void* u, const void* delta, const float* 
   a.final_state = final_state;
   a.len = len;
   a.channels = (int)channels;
-  const int cpw = nstate >= 8 ? 16 : 32;  // channels per warp (ComplexSmem::kCPW)
-  a.groups = (int)((channels + cpw - 1) / cpw);
   auto go = [&](auto ns) {
     constexpr int NS = decltype(ns)::value;
     return dtype == MAMBA_BF16 ? launch_complex<__nv_bfloat16, NS>(a, batch, supers, stream)

@@ -66,7 +66,7 @@ namespace mamba {
 #endif
 
 constexpr int kCPW = 32;   // channels per warp: one lane per channel
-constexpr int kFixSegTiles = 4;  // tiles per segment of the super-chunk correction
+constexpr int kFixSegTiles = 1;  // tiles per segment of the super-chunk correction
 constexpr int kHandQ = 8;  // hand-off flags a consumer may leave for the producer to publish
 
 enum Discretisation : int { kZOH = 0, kEuler = 1, kTrapezoid = 2 };
@@ -104,6 +104,7 @@ struct ScanParams {
   int chunks_last;          // chunks of the last super-chunk
   int streams;              // S*G streams, stream = super * groups + group
   int segs_max;             // correction segments (kFixSegTiles tiles each) of a full super-chunk
+  int fix_vec;              // Delta, y and C rows can be staged in 16-byte pieces
   int jobs;                 // all jobs (fits int32, checked on the host)
   int use_tma;
   uint64_t wait_limit_ns;
@@ -163,13 +164,16 @@ __device__ __forceinline__ Job decode_job(const ScanParams& p, int j_in, int til
 // job, full / empty barriers, the job of each slot, and the queue of
 // hand-off flags the producer publishes
 // ---------------------------------------------------------------------------
-// R > 1 (multi-input multi-output): a token has R rows of u, B and C'
-// (input / output r of row t at row t R + r) and one row of Delta.
+// B and C' rows are fp32 whatever the I/O type (for bf16 data the pre-pass
+// widens B; the widening is exact), so the input term of every state step
+// is a packed FFMA2.  R > 1 (multi-input multi-output): a token has R rows
+// of u, B and C' (input / output r of row t at row t R + r) and one row of
+// Delta.
 template <typename TIO, int NS, int TILE, int STAGES, int R = 1>
 struct alignas(128) WarpSmem {
   TIO u[STAGES][TILE * R][kCPW];
   TIO dl[STAGES][TILE][kCPW];
-  TIO b[STAGES][TILE * R][NS];
+  float b[STAGES][TILE * R][NS];
   float cs[STAGES][TILE * R][NS];
   float4 chan[STAGES][kCPW];  // loaded with tile 0 of a job
   uint64_t full[STAGES];      // producer -> consumer: the tile has landed
@@ -187,10 +191,10 @@ constexpr size_t scan_smem_bytes() {
   return sizeof(WarpSmem<TIO, NS, TILE, STAGES, R>) * CW + 128;
 }
 
-// bytes one tile brings in: u and Delta columns, the B rows (I/O type), the C' rows (fp32)
+// bytes one tile brings in: u and Delta columns (I/O type), the B and C' rows (fp32)
 template <typename TIO, int NS, int R = 1>
 __host__ __device__ constexpr uint32_t tile_bytes(int tile) {
-  return (uint32_t)(tile * ((R + 1) * kCPW * sizeof(TIO) + R * NS * sizeof(TIO) + R * NS * sizeof(float)));
+  return (uint32_t)(tile * ((R + 1) * kCPW * sizeof(TIO) + 2 * R * NS * sizeof(float)));
 }
 
 // ---------------------------------------------------------------------------
@@ -231,6 +235,12 @@ __device__ __forceinline__ void expm1_parts(float z, float& q, float& d) {
 // |z| >= 1/32), and for |z| < 1/32 the series z + z^2/2 + z^3/6 (truncation
 // below 1.3e-6 relative there).  Both are evaluated and one is selected.
 __device__ __forceinline__ float expm1_series3(float z) { return z * fmaf(z, fmaf(z, 1.0f / 6.0f, 0.5f), 1.0f); }
+// the same series for z = zl ln 2 given zl (base-2 units): zl (c1 + zl (c2 + zl c3))
+// with c1 = ln 2, c2 = (ln 2)^2 / 2, c3 = (ln 2)^3 / 6; |zl| < kSeriesLimit2 is |z| < 1/32
+constexpr float kSeriesLimit2 = 0.03125f * 1.4426950408889634f;
+__device__ __forceinline__ float expm1_series3_log2(float zl) {
+  return zl * fmaf(zl, fmaf(zl, 0.0555041086648216f, 0.2402265069591007f), 0.6931471805599453f);
+}
 __device__ __forceinline__ float expm1_fast(float z) {
   const float viaexp2 = ex2_approx(z * 1.4426950408889634f) - 1.0f;
   return fabsf(z) < 0.03125f ? expm1_series3(z) : viaexp2;
@@ -240,19 +250,10 @@ __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b
 
 __device__ __forceinline__ uint16_t raw16(__nv_bfloat16 v) { return __bfloat16_as_ushort(v); }
 
-// d = lo16(w) * x + c and d = hi16(w) * x + c with bf16 multiplicands and an
-// fp32 addend (the bf16 x bf16 product is exact in fp32).
-__device__ __forceinline__ float fma_bf16_lo(uint32_t w, uint16_t x, float c) {
-  float d;
-  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, l, %2, %3;\n\t}"
-      : "=f"(d) : "r"(w), "h"(x), "f"(c));
-  return d;
-}
-__device__ __forceinline__ float fma_bf16_hi(uint32_t w, uint16_t x, float c) {
-  float d;
-  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, h, %2, %3;\n\t}"
-      : "=f"(d) : "r"(w), "h"(x), "f"(c));
-  return d;
+// 16-byte asynchronous copy global -> shared; with in == false nothing is
+// read and the 16 bytes are zero-filled
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool in) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(in ? 16 : 0) : "memory");
 }
 
 // Store v at p when pred holds, as one predicated instruction (a branch
@@ -286,54 +287,26 @@ __device__ __forceinline__ void decay_chain(float r, float q, float2 (&e2)[NS / 
 }
 
 // One token for one lane: g <- g + e (g + B x) for all states; returns
-// sum_n C'_n g_n.  States as N/2 float2 pairs, every state step a packed
-// FFMA2 except the bf16 input term (two mixed FMAs per pair).
+// sum_n C'_n g_n.  States as N/2 float2 pairs, every step a packed FFMA2
+// (B x is exact in fp32 for bf16 operands, so this equals the mixed-precision
+// product of the raw bf16 values).
 template <typename TIO, int NS>
-__device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const TIO* brow, const float* csrow, TIO xr,
+__device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const float* brow, const float* csrow, TIO xr,
                                               float2 (&g)[NS / 2]) {
   float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
-  if constexpr (sizeof(TIO) == 2) {
-    const uint16_t xh = raw16(xr);
-    uint32_t bw[NS / 2];
-    if constexpr (NS % 8 == 0) {
+  const float x = to_f32(xr);
+  const float2 x2 = f2(x, x);
 #pragma unroll
-      for (int k8 = 0; k8 < NS / 8; ++k8) {
-        const uint4 w = reinterpret_cast<const uint4*>(brow)[k8];
-        bw[4 * k8] = w.x; bw[4 * k8 + 1] = w.y; bw[4 * k8 + 2] = w.z; bw[4 * k8 + 3] = w.w;
-      }
-    } else {
-#pragma unroll
-      for (int k4 = 0; k4 < NS / 4; ++k4) {
-        const uint2 w = reinterpret_cast<const uint2*>(brow)[k4];
-        bw[2 * k4] = w.x; bw[2 * k4 + 1] = w.y;
-      }
-    }
-#pragma unroll
-    for (int n4 = 0; n4 < NS / 4; ++n4) {
-      const float4 cv = reinterpret_cast<const float4*>(csrow)[n4];
-      const int p0 = 2 * n4, p1 = 2 * n4 + 1;
-      const float2 v0 = f2(fma_bf16_lo(bw[p0], xh, g[p0].x), fma_bf16_hi(bw[p0], xh, g[p0].y));
-      const float2 v1 = f2(fma_bf16_lo(bw[p1], xh, g[p1].x), fma_bf16_hi(bw[p1], xh, g[p1].y));
-      g[p0] = __ffma2_rn(e[p0], v0, g[p0]);
-      g[p1] = __ffma2_rn(e[p1], v1, g[p1]);
-      acc0 = __ffma2_rn(f2(cv.x, cv.y), g[p0], acc0);
-      acc1 = __ffma2_rn(f2(cv.z, cv.w), g[p1], acc1);
-    }
-  } else {
-    const float x = to_f32(xr);
-    const float2 x2 = f2(x, x);
-#pragma unroll
-    for (int n4 = 0; n4 < NS / 4; ++n4) {
-      const float4 bv = reinterpret_cast<const float4*>(brow)[n4];
-      const float4 cv = reinterpret_cast<const float4*>(csrow)[n4];
-      const int p0 = 2 * n4, p1 = 2 * n4 + 1;
-      const float2 v0 = __ffma2_rn(f2(bv.x, bv.y), x2, g[p0]);
-      const float2 v1 = __ffma2_rn(f2(bv.z, bv.w), x2, g[p1]);
-      g[p0] = __ffma2_rn(e[p0], v0, g[p0]);
-      g[p1] = __ffma2_rn(e[p1], v1, g[p1]);
-      acc0 = __ffma2_rn(f2(cv.x, cv.y), g[p0], acc0);
-      acc1 = __ffma2_rn(f2(cv.z, cv.w), g[p1], acc1);
-    }
+  for (int n4 = 0; n4 < NS / 4; ++n4) {
+    const float4 bv = reinterpret_cast<const float4*>(brow)[n4];
+    const float4 cv = reinterpret_cast<const float4*>(csrow)[n4];
+    const int p0 = 2 * n4, p1 = 2 * n4 + 1;
+    const float2 v0 = __ffma2_rn(f2(bv.x, bv.y), x2, g[p0]);
+    const float2 v1 = __ffma2_rn(f2(bv.z, bv.w), x2, g[p1]);
+    g[p0] = __ffma2_rn(e[p0], v0, g[p0]);
+    g[p1] = __ffma2_rn(e[p1], v1, g[p1]);
+    acc0 = __ffma2_rn(f2(cv.x, cv.y), g[p0], acc0);
+    acc1 = __ffma2_rn(f2(cv.z, cv.w), g[p1], acc1);
   }
   return (acc0.x + acc0.y) + (acc1.x + acc1.y);
 }
@@ -347,7 +320,7 @@ __device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const T
 // their decay chains are independent work for the scheduler while the state
 // updates wait on each other.
 template <typename TIO, int NS, int TILE, bool FASTQ>
-__device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, const TIO (*bt)[NS],
+__device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, const float (*bt)[NS],
                                                 const float (*ct)[NS], int rows, float a0, float inv_a0, float Dd,
                                                 float2 (&g)[NS / 2], float& sd, TIO* yp, int64_t ystride,
                                                 bool active) {
@@ -356,9 +329,9 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
     if constexpr (FASTQ) {
       // r from the hardware exp2; q = r - 1 from the same value, or from the
       // series where that subtraction would lose the small |Delta A_0|
-      const float r = ex2_approx(dt * a0l);
-      const float z = dt * a0;
-      const float q = fabsf(z) < 0.03125f ? expm1_series3(z) : r - 1.0f;
+      const float zl = dt * a0l;
+      const float r = ex2_approx(zl);
+      const float q = fabsf(zl) < kSeriesLimit2 ? expm1_series3_log2(zl) : r - 1.0f;
       decay_chain<NS>(r, q, e);
     } else {
       const float q = expm1_small(dt * a0);
@@ -445,7 +418,7 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
 // (Mamba-3 page, "Geliştirilmiş Ayrıklaştırma Şeması", with the readings
 // given in the header).  vp carries the previous token's v across tiles.
 template <typename TIO, int NS, int METHOD>
-__device__ __forceinline__ void tile_general(const TIO* su, const TIO* sdl, const TIO (*bt)[NS],
+__device__ __forceinline__ void tile_general(const TIO* su, const TIO* sdl, const float (*bt)[NS],
                                              const float (*ct)[NS], int rows, const float (&kA)[NS],
                                              const float (&kC)[NS], float Dd, float2 (&g)[NS / 2], float& sd,
                                              float (&vp)[NS], TIO* yp, int64_t ystride, bool active) {
@@ -473,7 +446,7 @@ __device__ __forceinline__ void tile_general(const TIO* su, const TIO* sdl, cons
       s = 0.0f;
 #pragma unroll
       for (int k = 0; k < NS; ++k) {
-        const float v = to_f32(bt[r][k]) * x;  // exact for bf16 operands
+        const float v = bt[r][k] * x;  // exact for bf16 operands
         float gk = (k & 1) ? g[k >> 1].y : g[k >> 1].x;
         if constexpr (METHOD == kEuler) {
           gk = fmaf(ev[k], gk, fmaf(zv[k], v, gk));
@@ -504,7 +477,7 @@ __device__ __forceinline__ void tile_general(const TIO* su, const TIO* sdl, cons
 // x^(r) at xs[r * 32].  GEN: general A, C'^(r)_n is scaled by kC[n].
 // ---------------------------------------------------------------------------
 template <typename TIO, int NS, int R, bool GEN>
-__device__ __forceinline__ void token_update_mimo(const float2 (&e)[NS / 2], const TIO* brows, const float* csrows,
+__device__ __forceinline__ void token_update_mimo(const float2 (&e)[NS / 2], const float* brows, const float* csrows,
                                                   const TIO* xs, const float (&kC)[GEN ? NS : 1],
                                                   float2 (&g)[NS / 2], float (&acc)[R]) {
   static_assert(NS % 8 == 0, "MIMO rows are read in 16-byte pieces");
@@ -517,27 +490,13 @@ __device__ __forceinline__ void token_update_mimo(const float2 (&e)[NS / 2], con
   // input terms: sum over r of B^(r) x^(r), added to g
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    if constexpr (sizeof(TIO) == 2) {
-      const uint16_t xh = raw16(xs[r * kCPW]);
+    const float x = to_f32(xs[r * kCPW]);
+    const float2 x2 = f2(x, x);
 #pragma unroll
-      for (int k8 = 0; k8 < NS / 8; ++k8) {
-        const uint4 w = reinterpret_cast<const uint4*>(brows + r * NS)[k8];
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int k = 4 * k8 + i;
-          v[k] = f2(fma_bf16_lo(ww[i], xh, v[k].x), fma_bf16_hi(ww[i], xh, v[k].y));
-        }
-      }
-    } else {
-      const float x = to_f32(xs[r * kCPW]);
-      const float2 x2 = f2(x, x);
-#pragma unroll
-      for (int k4 = 0; k4 < NS / 4; ++k4) {
-        const float4 bv = reinterpret_cast<const float4*>(brows + r * NS)[k4];
-        v[2 * k4] = __ffma2_rn(f2(bv.x, bv.y), x2, v[2 * k4]);
-        v[2 * k4 + 1] = __ffma2_rn(f2(bv.z, bv.w), x2, v[2 * k4 + 1]);
-      }
+    for (int k4 = 0; k4 < NS / 4; ++k4) {
+      const float4 bv = reinterpret_cast<const float4*>(brows + r * NS)[k4];
+      v[2 * k4] = __ffma2_rn(f2(bv.x, bv.y), x2, v[2 * k4]);
+      v[2 * k4 + 1] = __ffma2_rn(f2(bv.z, bv.w), x2, v[2 * k4 + 1]);
     }
   }
 #pragma unroll
@@ -565,7 +524,7 @@ __device__ __forceinline__ void token_update_mimo(const float2 (&e)[NS / 2], con
 // accumulates sum(Delta) in sd.  y of token t, output q, sits at
 // yp + (t R + q) ystride.
 template <typename TIO, int NS, int R, bool STRUCT, bool FASTQ>
-__device__ __forceinline__ void tile_mimo(const TIO* su, const TIO* sdl, const TIO (*bt)[NS], const float (*ct)[NS],
+__device__ __forceinline__ void tile_mimo(const TIO* su, const TIO* sdl, const float (*bt)[NS], const float (*ct)[NS],
                                           int rows, float a0, float inv_a0, const float (&kA)[STRUCT ? 1 : NS],
                                           const float (&kC)[STRUCT ? 1 : NS], float Dd, float2 (&g)[NS / 2],
                                           float& sd, TIO* yp, int64_t ystride, bool active) {
@@ -576,9 +535,9 @@ __device__ __forceinline__ void tile_mimo(const TIO* su, const TIO* sdl, const T
     float2 e[NS / 2];
     if constexpr (STRUCT) {
       if constexpr (FASTQ) {
-        const float rr = ex2_approx(dt * a0l);
-        const float z = dt * a0;
-        decay_chain<NS>(rr, fabsf(z) < 0.03125f ? expm1_series3(z) : rr - 1.0f, e);
+        const float zl = dt * a0l;
+        const float rr = ex2_approx(zl);
+        decay_chain<NS>(rr, fabsf(zl) < kSeriesLimit2 ? expm1_series3_log2(zl) : rr - 1.0f, e);
       } else {
         const float q = expm1_small(dt * a0);
         decay_chain<NS>(1.0f + q, q, e);
@@ -657,7 +616,7 @@ struct Consumer {
     }
     for (int i = lane; i < rows * R * NS; i += 32) {
       const int r = i / NS, n = i - r * NS;
-      sm.b[s][r][n] = gB[(rowbase * R + r) * NS + n];
+      sm.b[s][r][n] = to_f32(gB[(rowbase * R + r) * NS + n]);
       sm.cs[s][r][n] = p.cs[(rowbase * R + r) * NS + n];
     }
     __syncwarp();
@@ -1094,27 +1053,32 @@ scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__
 // from zero, so each of its outputs misses
 //     sum_n C_t[n] exp(A_n cum_t) h_in[n],   cum_t = sum of Delta from the
 //                                            super-chunk's start through t.
-// The main pass left cum at the start of every segment of kFixSegTiles
-// tiles, up to the segment where exp2 of the slowest decay underflows to
-// zero on every lane (from there on the term is exactly zero in fp32), and
-// the number of such segments per stream.  One warp per (stream of a
-// super-chunk j >= 1, phase w), a lane per channel, takes segments w,
-// w + phases, ...; a segment goes in blocks of 16/R tokens whose Delta, y and
-// C rows are loaded together before the arithmetic.  Phase 0 of the last
-// super-chunk writes the final state H + exp(A sum Delta) h_in.  CKPT: the
-// state checkpointed before every tile of a walked segment gets
-// exp(A_n cum) h_in[n] added.
+// The main pass left cum at the start of every tile, up to the tile where
+// exp2 of the slowest decay underflows to zero on every lane (from there on
+// the term is exactly zero in fp32), and the number of such tiles per
+// stream.  One warp per (stream of a super-chunk j >= 1, phase w), a lane per
+// channel, takes tiles w, w + phases, ...: it stages the tile's Delta, y
+// and C rows in its shared memory (16-byte cp.async copies, all in flight
+// at once; plain loads when rows are not 16-byte pieces), adds the term
+// token by token, and writes y back.  Phase 0 of the last super-chunk writes
+// the final state H + exp(A sum Delta) h_in.  CKPT: the state checkpointed
+// before every walked tile gets exp(A_n cum) h_in[n] added.
 // ---------------------------------------------------------------------------
 constexpr int kFixWarps = 4;
 constexpr int kFixPhases = 32;
 
+template <typename TIO, int NS, int TILE, int R>
+__host__ __device__ constexpr int fix_stage_bytes() {  // one warp: Delta [TILE][32], y [TILE*R][32], C [TILE*R][NS]
+  return (TILE * kCPW + TILE * R * kCPW + TILE * R * NS) * (int)sizeof(TIO);
+}
+
 template <typename TIO, int NS, int TILE, bool CKPT, int R = 1>
 __global__ void __launch_bounds__(kFixWarps * 32)
 scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
-  constexpr int SB = 16 / R;  // tokens per block
-  __shared__ float cbuf[kFixWarps][SB * R][NS];
-  griddep_wait();  // the main pass's outputs, aggregates and segment sums
+  extern __shared__ __align__(16) unsigned char fix_smem[];
+  griddep_wait();  // the main pass's outputs, aggregates and tile sums
   constexpr float kLog2e = 1.4426950408889634f;
+  constexpr int kChunk = 16 / (int)sizeof(TIO);  // elements per 16-byte piece
   const int lane = threadIdx.x & 31;
   const int wl = threadIdx.x >> 5;
   const int64_t wg = (int64_t)blockIdx.x * kFixWarps + wl;
@@ -1155,95 +1119,122 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
     for (int k = 0; k < NS; ++k) dst[k] = fmaf(expf(an[k] * sdl), h[k], __ldcg(H + k));
   }
 
-  float kmax = an[0];
+  const float a0l = cm.x * kLog2e;  // structured: every decay is a power of exp(A_0 cum)
+  float kmax = an[0];  // the slowest decay of the lane
 #pragma unroll
   for (int k = 1; k < NS; ++k) kmax = fmaxf(kmax, an[k]);
   kmax *= kLog2e;
-  const float a0l = cm.x * kLog2e;  // structured: every decay is a power of exp(A_0 cum)
   const int64_t s_begin = (int64_t)super_idx * p.super_len;
   const int64_t s_end = (s_begin + p.super_len < p.len) ? s_begin + p.super_len : p.len;
-  const int segs = ld_volatile(p.fix_segs + stream);
+  const int tiles = ld_volatile(p.fix_segs + stream);
   const TIO* dl = static_cast<const TIO*>(p.delta);
   const TIO* Cg = static_cast<const TIO*>(p.C);
   TIO* y = static_cast<TIO*>(p.y);
-  float (*cb)[NS] = cbuf[wl];
-  constexpr int64_t kSeg = (int64_t)kFixSegTiles * TILE;
+  // this warp's staging area
+  TIO* sdl = reinterpret_cast<TIO*>(fix_smem + wl * fix_stage_bytes<TIO, NS, TILE, R>());  // [TILE][32]
+  TIO* sy = sdl + TILE * kCPW;                                                              // [TILE*R][32]
+  TIO* sc = sy + TILE * R * kCPW;                                                            // [TILE*R][NS]
+  const uint32_t s_dl = smem_addr(sdl), s_y = smem_addr(sy), s_c = smem_addr(sc);
 
-  for (int k = w; k < segs; k += phases) {
+  for (int k = w; k < tiles; k += phases) {
     float cum = __ldcg(p.cum + ((int64_t)stream * p.segs_max + k) * kCPW + lane);
-    const int64_t t0 = s_begin + (int64_t)k * kSeg;
-    const int64_t t1 = (t0 + kSeg < s_end) ? t0 + kSeg : s_end;
-    bool gone = false;
-    for (int64_t tb = t0; tb < t1 && !gone; tb += SB) {
-      const int nt = (int)(t1 - tb < SB ? t1 - tb : SB);
-      const int64_t row0 = (int64_t)b * p.len + tb;
-      // loads of the block: Delta and y of this lane's channel, the C rows (to shared memory)
-      float dv[SB], yv[SB * R];
-#pragma unroll
-      for (int i = 0; i < SB; ++i) dv[i] = (i < nt && active) ? to_f32(dl[(row0 + i) * p.channels + d]) : 0.0f;
-#pragma unroll
-      for (int i = 0; i < SB * R; ++i)
-        yv[i] = (y != nullptr && i < nt * R && active) ? to_f32(y[(row0 * R + i) * p.channels + d]) : 0.0f;
-      for (int e = lane; e < SB * R * NS; e += 32) {
-        const int r = e / NS;
-        cb[r][e - r * NS] = r < nt * R ? to_f32(Cg[row0 * R * NS + e]) : 0.0f;
+    const int64_t t0 = s_begin + (int64_t)k * TILE;
+    const int nt = (int)(s_end - t0 < TILE ? s_end - t0 : TILE);
+    const int64_t row0 = (int64_t)b * p.len + t0;
+    // stage Delta, y and the C rows of the tile
+    if (p.fix_vec) {
+      constexpr int kRowPieces = kCPW / kChunk;  // 16-byte pieces of a 32-channel row
+      for (int i = lane; i < nt * kRowPieces; i += 32) {
+        const int r = i / kRowPieces, c = i - r * kRowPieces;
+        const bool in = d0 + c * kChunk < p.channels;
+        cp_async16_zfill(s_dl + (uint32_t)(r * kCPW + c * kChunk) * sizeof(TIO),
+                         in ? (const void*)(dl + (row0 + r) * p.channels + d0 + c * kChunk) : p.delta, in);
       }
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < SB; ++i) {
-        if constexpr (CKPT) {
-          const int64_t t = tb + i;
-          if (i < nt && t % TILE == 0 && active) {
-            float* ck = p.ckpt + (((int64_t)b * ((p.len + TILE - 1) / TILE) + t / TILE) * p.channels + d) * NS;
-#pragma unroll
-            for (int k2 = 0; k2 < NS; ++k2) ck[k2] = fmaf(ex2_approx(cum * an[k2] * kLog2e), h[k2], ck[k2]);
-          }
+      if (y != nullptr)
+        for (int i = lane; i < nt * R * kRowPieces; i += 32) {
+          const int r = i / kRowPieces, c = i - r * kRowPieces;
+          const bool in = d0 + c * kChunk < p.channels;
+          cp_async16_zfill(s_y + (uint32_t)(r * kCPW + c * kChunk) * sizeof(TIO),
+                           in ? (const void*)(y + (row0 * R + r) * p.channels + d0 + c * kChunk) : p.delta, in);
         }
-        cum += dv[i];
-        // the carried state's decay to this token: rho_n = exp(A_n cum)
-        float ph[NS];
-        if (structured) {
-          const float rho = ex2_approx(cum * a0l);
-          float pw = rho;
-#pragma unroll
-          for (int n = 0; n < NS; ++n) {
-            ph[n] = pw * h[n];
-            pw *= rho;
-          }
-        } else {
-#pragma unroll
-          for (int n = 0; n < NS; ++n) ph[n] = ex2_approx(cum * an[n] * kLog2e) * h[n];
-        }
-#pragma unroll
-        for (int q = 0; q < R; ++q) {  // output q reads the state with its own C row
-          float corr = 0.0f;
-#pragma unroll
-          for (int n = 0; n < NS; ++n) corr = fmaf(cb[i * R + q][n], ph[n], corr);
-          yv[i * R + q] += corr;
-        }
-      }
-      if (p.y != nullptr && active) {
-#pragma unroll
-        for (int i = 0; i < SB * R; ++i)
-          if (i < nt * R) y[(row0 * R + i) * p.channels + d] = from_f32<TIO>(yv[i]);
-      }
-      __syncwarp();
-      gone = __all_sync(0xffffffffu, !active || ex2_approx(cum * kmax) == 0.0f);
+      constexpr int kCPieces = NS / kChunk;  // 16-byte pieces of a C row
+      for (int i = lane; i < nt * R * kCPieces; i += 32)
+        cp_async16_zfill(s_c + (uint32_t)i * 16u, Cg + row0 * R * NS + (int64_t)i * kChunk, true);
+      asm volatile("cp.async.wait_all;" ::: "memory");
+    } else {
+      for (int r = 0; r < nt; ++r) sdl[r * kCPW + lane] = active ? dl[(row0 + r) * p.channels + d] : from_f32<TIO>(0.0f);
+      if (y != nullptr)
+        for (int r = 0; r < nt * R; ++r)
+          sy[r * kCPW + lane] = active ? y[(row0 * R + r) * p.channels + d] : from_f32<TIO>(0.0f);
+      for (int i = lane; i < nt * R * NS; i += 32) sc[i] = Cg[row0 * R * NS + i];
     }
+    __syncwarp();
+    for (int r = 0; r < nt; ++r) {
+      if constexpr (CKPT) {
+        if (r == 0 && active) {  // tiles start at multiples of TILE
+          float* ck = p.ckpt + (((int64_t)b * ((p.len + TILE - 1) / TILE) + t0 / TILE) * p.channels + d) * NS;
+#pragma unroll
+          for (int k2 = 0; k2 < NS; ++k2) ck[k2] = fmaf(ex2_approx(cum * an[k2] * kLog2e), h[k2], ck[k2]);
+        }
+      }
+      cum += to_f32(sdl[r * kCPW + lane]);
+      // the carried state's decay to this token: rho_n = exp(A_n cum)
+      float ph[NS];
+      if (structured) {
+        const float rho = ex2_approx(cum * a0l);
+        float pw = rho;
+#pragma unroll
+        for (int n = 0; n < NS; ++n) {
+          ph[n] = pw * h[n];
+          pw *= rho;
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < NS; ++n) ph[n] = ex2_approx(cum * an[n] * kLog2e) * h[n];
+      }
+#pragma unroll
+      for (int q = 0; q < R; ++q) {  // output q reads the state with its own C row
+        float corr = 0.0f;
+#pragma unroll
+        for (int n = 0; n < NS; ++n) corr = fmaf(to_f32(sc[(r * R + q) * NS + n]), ph[n], corr);
+        TIO& yv = sy[(r * R + q) * kCPW + lane];
+        yv = from_f32<TIO>(to_f32(yv) + corr);
+      }
+    }
+    __syncwarp();
+    // write y back
+    if (y != nullptr) {
+      if (p.fix_vec) {
+        constexpr int kRowPieces = kCPW / kChunk;
+        for (int i = lane; i < nt * R * kRowPieces; i += 32) {
+          const int r = i / kRowPieces, c = i - r * kRowPieces;
+          if (d0 + c * kChunk < p.channels)
+            *reinterpret_cast<uint4*>(y + (row0 * R + r) * p.channels + d0 + c * kChunk) =
+                *reinterpret_cast<const uint4*>(sy + r * kCPW + c * kChunk);
+        }
+      } else if (active) {
+        for (int r = 0; r < nt * R; ++r) y[(row0 * R + r) * p.channels + d] = sy[r * kCPW + lane];
+      }
+    }
+    __syncwarp();
+    if (__all_sync(0xffffffffu, !active || ex2_approx(cum * kmax) == 0.0f))
+      break;  // later tiles of this warp add exactly zero (their cum is larger)
   }
 }
 
 // ---------------------------------------------------------------------------
 // pre-pass, one thread per element of three ranges:
 //   [0, zero_words):          the job counters and progress flags = 0
-//   C' = C / (n+1) in fp32 for every (token row, state)
+//   C' = C / (n+1) in fp32 for every (token row, state), and B widened to
+//   fp32 when bs is given (bf16 data)
 //   per channel {A[d,0], 1/A[d,0], D[d], structured}, where "structured"
 //   means A[d,n] == (n+1) A[d,0] exactly for every n, A[d,0] < 0 and the
 //   general path was not forced; padding channels get {-1, -1, 0, 1}.
 // ---------------------------------------------------------------------------
 template <typename TIO, int NS>
 __global__ void scan_prep_kernel(int* __restrict__ zero, int64_t zero_words, const TIO* __restrict__ C,
-                                 float* __restrict__ cs, int64_t total_c, const float* __restrict__ A,
+                                 float* __restrict__ cs, const TIO* __restrict__ B, float* __restrict__ bs,
+                                 int64_t total_c, const float* __restrict__ A,
                                  const float* __restrict__ D, float4* __restrict__ chan, int64_t channels,
                                  int64_t chan_padded, int force_general) {
   griddep_launch_dependents();  // the scan kernel may start its setup
@@ -1257,6 +1248,7 @@ __global__ void scan_prep_kernel(int* __restrict__ zero, int64_t zero_words, con
   if (i < total_c) {
     const int n = (int)(i % NS);
     cs[i] = to_f32(C[i]) / (float)(n + 1);
+    if (bs) bs[i] = to_f32(B[i]);
     return;
   }
   const int64_t d = i - total_c;

@@ -76,9 +76,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
   const int n = valid ? 16 : 0;  // 0: nothing is read, the 16 bytes are zero-filled
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -121,17 +118,40 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// 16 consecutive 32-bit columns of this thread's tensor-memory lane
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
+// 16 consecutive 32-bit columns of this thread's tensor-memory lane; the
+// registers are valid after tmem_wait_ld (several loads may be in flight)
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
         "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 64 consecutive columns (four loads in flight, one wait)
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
+  uint32_t r[4][16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  for (int q = 0; q < 4; ++q) tmem_ld16_nowait(taddr + 16 * q, r[q]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[16 * q + i] = __uint_as_float(r[q][i]);
+}
+
+// N consecutive columns, N a multiple of 16
+template <int N>
+__device__ __forceinline__ void tmem_ldN(uint32_t taddr, float (&v)[N]) {
+  uint32_t r[N / 16][16];
+#pragma unroll
+  for (int q = 0; q < N / 16; ++q) tmem_ld16_nowait(taddr + 16 * q, r[q]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int q = 0; q < N / 16; ++q)
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[16 * q + i] = __uint_as_float(r[q][i]);
 }
 
 // ---------------------------------------------------------------------------
@@ -155,8 +175,8 @@ struct SsdSmem {
   static constexpr int kCt = kM + kSsdHeads * kSsdQ * kSsdQ * 2;  // [2] C~ tiles, 64 x N
   static constexpr int kBw = kCt + kSsdHeads * kBC;      // [2] Bw tiles, 64 x N
   static constexpr int kS = kBw + kSsdHeads * kBC;       // [2] bf16 state copies, 64 ch x N
-  static constexpr int kCum = kS + kSsdHeads * kSsdP * N * 2;  // [2][64] cum (log2), [2][64] w
-  static constexpr int kWsum = kCum + 2 * kSsdHeads * kSsdQ * 4;  // [4 warps][2 heads] partial sums
+  static constexpr int kCum = kS + kSsdHeads * kSsdP * N * 2;  // [2][64] cum (log2), [2][64] w, [2][64] u
+  static constexpr int kWsum = kCum + 3 * kSsdHeads * kSsdQ * 4;  // [4 warps][2 heads] partial sums
   static constexpr int kDs = kWsum + kSsdWarps * kSsdHeads * 4;   // [2 heads][64] D
   static constexpr int kBar = kDs + kSsdHeads * kSsdP * 4;        // 2 mbarriers
   static constexpr int kTslot = kBar + 16;
@@ -284,6 +304,7 @@ ssd_chunk_kernel(const SsdArgs a) {
   Ds[hd * kSsdP + row] = (a.D && hok) ? __ldg(a.D + (int64_t)h * kSsdP + row) : 0.0f;
   float* cum_s = reinterpret_cast<float*>(smem + L::kCum);  // [2][64]
   float* w_s = cum_s + kSsdHeads * kSsdQ;                    // [2][64]
+  float* u_s = w_s + kSsdHeads * kSsdQ;                      // [2][64] e^{-a cum_s} w_s
   float* wsum = reinterpret_cast<float*>(smem + L::kWsum);   // [4][2]
   float total_log2 = 0.0f;
 
@@ -359,6 +380,10 @@ ssd_chunk_kernel(const SsdArgs a) {
     total_log2 += cum_end;
     cum_s[hd * kSsdQ + row] = cum;
     w_s[hd * kSsdQ + row] = wgt;
+    // the decay from s to t factors as e^{a cum_t} e^{-a cum_s} while the
+    // factors stay in range (the chunk decays by less than 2^-100)
+    const bool split = cum_end > -100.0f;
+    u_s[hd * kSsdQ + row] = split ? ex2_approx(-cum) * wgt : 0.0f;
 
     // C~ = e^{a cum_t} C_t and Bw = e^{a(cum_end - cum_s)} w_s B_s, row `row` of head hd
     {
@@ -410,22 +435,42 @@ ssd_chunk_kernel(const SsdArgs a) {
       tc_fence_after();
       const float* cum_h = cum_s + hd * kSsdQ;
       const float* w_h = w_s + hd * kSsdQ;
+      const float* u_h = u_s + hd * kSsdQ;
       unsigned char* mrow = smem + L::kM + hd * (kSsdQ * kSsdQ * 2) + (row >> 3) * 1024 + (row & 7) * 16;
+      if (ok_run) {
+        float g[64];
+        tmem_ld64(t_lane + kColG, g);
+        if (split) {
+          // M[t][s] = G[t][s] e^{a cum_t} (e^{-a cum_s} w_s), s <= t
+          const float et = ex2_approx(cum);
 #pragma unroll
-      for (int q4 = 0; q4 < 4 && ok_run; ++q4) {
-        float g[16];
-        tmem_ld16(t_lane + kColG + (uint32_t)(16 * q4), g);
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const float4 ua = *reinterpret_cast<const float4*>(u_h + 8 * c8);
+            const float4 ub = *reinterpret_cast<const float4*>(u_h + 8 * c8 + 4);
+            const float uu[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+            uint32_t op[4];
 #pragma unroll
-        for (int h8 = 0; h8 < 2; ++h8) {
-          uint32_t op[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int s0 = 16 * q4 + 8 * h8 + 2 * e;
-            const float m0 = s0 <= row ? g[8 * h8 + 2 * e] * ex2_approx(cum - cum_h[s0]) * w_h[s0] : 0.0f;
-            const float m1 = s0 + 1 <= row ? g[8 * h8 + 2 * e + 1] * ex2_approx(cum - cum_h[s0 + 1]) * w_h[s0 + 1] : 0.0f;
-            op[e] = pack_bf16(m0, m1);
+            for (int e = 0; e < 4; ++e) {
+              const int s0 = 8 * c8 + 2 * e;
+              const float m0 = s0 <= row ? g[s0] * et * uu[2 * e] : 0.0f;
+              const float m1 = s0 + 1 <= row ? g[s0 + 1] * et * uu[2 * e + 1] : 0.0f;
+              op[e] = pack_bf16(m0, m1);
+            }
+            *reinterpret_cast<uint4*>(mrow + c8 * 128) = make_uint4(op[0], op[1], op[2], op[3]);
           }
-          *reinterpret_cast<uint4*>(mrow + (2 * q4 + h8) * 128) = make_uint4(op[0], op[1], op[2], op[3]);
+        } else {
+#pragma unroll
+          for (int c8 = 0; c8 < 8; ++c8) {
+            uint32_t op[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int s0 = 8 * c8 + 2 * e;
+              const float m0 = s0 <= row ? g[s0] * ex2_approx(cum - cum_h[s0]) * w_h[s0] : 0.0f;
+              const float m1 = s0 + 1 <= row ? g[s0 + 1] * ex2_approx(cum - cum_h[s0 + 1]) * w_h[s0 + 1] : 0.0f;
+              op[e] = pack_bf16(m0, m1);
+            }
+            *reinterpret_cast<uint4*>(mrow + c8 * 128) = make_uint4(op[0], op[1], op[2], op[3]);
+          }
         }
       }
     }
@@ -477,36 +522,33 @@ ssd_chunk_kernel(const SsdArgs a) {
         const unsigned char* xrow = smem + ox + hd * L::kX + (row >> 3) * 1024 + (row & 7) * 16;
         const bool store = hok && t0 + row < t_end;
         __nv_bfloat16* yrow = a.y + (b * a.len + t0 + row) * channels + (int64_t)hc * kSsdP;
+        float yv[64];
+        tmem_ld64(t_lane + kColY, yv);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          float yv[16];
-          tmem_ld16(t_lane + kColY + (uint32_t)(16 * q4), yv);
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint4 xv = *reinterpret_cast<const uint4*>(xrow + c8 * 128);
+          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+          const float4 da = *reinterpret_cast<const float4*>(Dh + 8 * c8);
+          const float4 db = *reinterpret_cast<const float4*>(Dh + 8 * c8 + 4);
+          const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+          uint32_t op[4];
 #pragma unroll
-          for (int h8 = 0; h8 < 2; ++h8) {
-            const int c8 = 2 * q4 + h8;
-            const uint4 xv = *reinterpret_cast<const uint4*>(xrow + c8 * 128);
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-            uint32_t op[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[e]));
-              const int p = 8 * c8 + 2 * e;
-              const float d0 = Dh[p], d1 = Dh[p + 1];
-              op[e] = pack_bf16(fmaf(d0, xf.x, yv[8 * h8 + 2 * e]), fmaf(d1, xf.y, yv[8 * h8 + 2 * e + 1]));
-            }
-            if (store) *reinterpret_cast<uint4*>(yrow + 8 * c8) = make_uint4(op[0], op[1], op[2], op[3]);
+          for (int e = 0; e < 4; ++e) {
+            const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[e]));
+            const int p = 8 * c8 + 2 * e;
+            op[e] = pack_bf16(fmaf(dd[2 * e], xf.x, yv[p]), fmaf(dd[2 * e + 1], xf.y, yv[p + 1]));
           }
+          if (store) *reinterpret_cast<uint4*>(yrow + 8 * c8) = make_uint4(op[0], op[1], op[2], op[3]);
         }
       }
       // S = e^{a cum_end} S + dS for channel `row` of head hd; its bf16 copy
       // feeds the next chunk's C~ S_in (this chunk's products are done)
       const float dec = ex2_approx(cum_end);
+      {
+        float ds[N];
+        tmem_ldN<N>(t_lane + kColS, ds);
 #pragma unroll
-      for (int q4 = 0; q4 < N / 16; ++q4) {
-        float ds[16];
-        tmem_ld16(t_lane + kColS + (uint32_t)(16 * q4), ds);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) S[16 * q4 + i] = fmaf(dec, S[16 * q4 + i], ds[i]);
+        for (int i = 0; i < N; ++i) S[i] = fmaf(dec, S[i], ds[i]);
       }
       if (!AGG) store_state_copy();
     }
