@@ -640,9 +640,8 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
     return MAMBA_ERR_CUDA;
   // tensor memory: kSsdTmemCols columns per CTA out of 512 per SM
   per_sm = std::min(per_sm, 512 / kSsdTmemCols);
-  a.head_pairs = (a.heads + kSsdHeads - 1) / kSsdHeads;
   a.wait_limit_ns = kWaitLimitNs;
-  const int64_t seqs = batch * a.head_pairs;  // one CTA per (batch row, head pair, super-chunk)
+  const int64_t seqs = batch * a.heads;  // one CTA per (batch row, head, super-chunk)
   const int64_t chunks = (a.len + kSsdQ - 1) / kSsdQ;
   int64_t S = ssd_supers(seqs, chunks, (int64_t)sms * per_sm, supers_req);
   const int64_t per = (chunks + S - 1) / S;

@@ -13,23 +13,29 @@
 // the input weight of the discretisation: (e^{a dt} - 1)/a for the
 // zero-order hold, dt for exponential Euler.
 //
-// A CTA of four warps owns two heads of one batch row over one super-chunk
-// and walks its chunks of 64 tokens in order.  Per chunk and head, all
-// products are tcgen05.mma (bf16 operands from shared memory, fp32
-// accumulators in tensor memory), issued by one thread:
-//   G   = C B^T                     64 x 64, K = N      (same for both heads)
+// A CTA of four warps owns one head of one batch row over one super-chunk
+// and walks its chunks of 64 tokens in order.  Per chunk, all products are
+// tcgen05.mma (bf16 operands from shared memory, fp32 accumulators in
+// tensor memory), issued by one thread:
+//   G   = C B^T                     64 x 64, K = N
 //   Y   = M X + C~ S_in             64 x 64, K = 64 + N  (M = G o e^{a(cum_t - cum_s)} o w_s,
 //                                                         masked s > t; C~ = e^{a cum_t} C)
 //   dS^T = X^T Bw                   64 x N,  K = 64      (Bw_s = e^{a(cum_end - cum_s)} w_s B_s)
-// The M = 64 accumulators of head 0 sit in tensor-memory lanes 0-15 of each
-// 32-lane sub-partition and those of head 1 in lanes 16-31, so every thread
-// of a warp reads one row of one head: thread i of warp w owns row (or
-// channel) 16w + i%16 of head i/16.  The warps turn G into M, form C~ and
-// Bw, and run the epilogues: y = Y + D x, and the fp32 state
-// S = e^{a cum_end} S + dS, kept in registers (a bf16 copy in shared memory
-// is the next chunk's operand).  x, B and C arrive through a ring of
-// cp.async copies into the no-swizzle core-matrix layouts the tensor core
-// reads (8 rows x 16 bytes per core matrix).
+// With M = 64 an accumulator row m sits in tensor-memory lane 32(m/16) +
+// m%16; a second tile can take lanes 32(m/16) + 16 + m%16.  G and Y are each
+// issued as two 32-column halves, the first half in the low lanes and the
+// second in the high ones, so thread i of warp w owns row 16w + i%16 and
+// column half i/16 of both: it reads a half row of G (turned into M) and of
+// Y (the y epilogue).  dS^T is issued as two halves of its K (tokens 0-31
+// into the low lanes, 32-63 into the high ones); the two threads of a
+// channel swap halves of their partial sums (N/2 shuffles) and each keeps
+// half of the channel's fp32 state S = e^{a cum_end} S + dS in registers
+// (a bf16 copy in shared memory is the next chunk's operand).  The first
+// thread of a row forms C~, the second Bw.  x, B and C arrive through a ring
+// of cp.async copies into the no-swizzle core-matrix layouts the tensor core
+// reads (8 rows x 16 bytes per core matrix).  One head per CTA keeps a CTA
+// to 128 tensor-memory columns and about 52 KB of shared memory (N = 16),
+// so four CTAs share an SM and their chunk pipelines overlap.
 //
 // Long sequences with few (batch row, head) pairs are cut into
 // super-chunks: an aggregate kernel (the same kernel, state only) runs each
@@ -48,8 +54,7 @@ namespace mamba {
 constexpr int kSsdQ = 64;       // tokens per chunk
 constexpr int kSsdP = 64;       // channels per head
 constexpr int kSsdWarps = 4;    // one warpgroup per CTA
-constexpr int kSsdHeads = 2;    // heads per CTA
-constexpr int kSsdTmemCols = 256;  // dS^T in columns [0, 64), Y in [64, 128), G in [128, 192)
+constexpr int kSsdTmemCols = 128;  // dS^T in columns [0, 64), Y in [64, 96), G in [96, 128)
 
 struct SsdArgs {
   const __nv_bfloat16* x;       // (batch, len, heads*64)
@@ -65,8 +70,7 @@ struct SsdArgs {
   float* agg_decay;             // (batch*heads, supers-1): log2 of its total decay
   int64_t len;
   int heads;
-  int head_pairs;               // ceil(heads / 2)
-  int supers;                   // super-chunks per (batch row, head pair)
+  int supers;                   // super-chunks per (batch row, head)
   int64_t super_len;            // tokens per super-chunk, a multiple of 64
   int euler;                    // input weight dt (exponential Euler) instead of the ZOH weight
   uint64_t wait_limit_ns;
@@ -129,29 +133,31 @@ __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[1
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 64 consecutive columns (four loads in flight, one wait)
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-  uint32_t r[4][16];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) tmem_ld16_nowait(taddr + 16 * q, r[q]);
-  tmem_wait_ld();
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[16 * q + i] = __uint_as_float(r[q][i]);
+__device__ __forceinline__ void tmem_ld8_nowait(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
 }
 
-// N consecutive columns, N a multiple of 16
+// N consecutive columns, N a multiple of 8
 template <int N>
 __device__ __forceinline__ void tmem_ldN(uint32_t taddr, float (&v)[N]) {
-  uint32_t r[N / 16][16];
+  static_assert(N % 8 == 0, "columns in steps of 8");
+  constexpr int Q = N / 16;
+  uint32_t r[Q > 0 ? Q : 1][16];
+  uint32_t t8[8];
 #pragma unroll
-  for (int q = 0; q < N / 16; ++q) tmem_ld16_nowait(taddr + 16 * q, r[q]);
+  for (int q = 0; q < Q; ++q) tmem_ld16_nowait(taddr + 16 * q, r[q]);
+  if constexpr (N % 16 != 0) tmem_ld8_nowait(taddr + 16 * Q, t8);
   tmem_wait_ld();
 #pragma unroll
-  for (int q = 0; q < N / 16; ++q)
+  for (int q = 0; q < Q; ++q)
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[16 * q + i] = __uint_as_float(r[q][i]);
+  if constexpr (N % 16 != 0) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[16 * Q + i] = __uint_as_float(t8[i]);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -165,23 +171,23 @@ __device__ __forceinline__ void tmem_ldN(uint32_t taddr, float (&v)[N]) {
 // ---------------------------------------------------------------------------
 template <int N>
 struct SsdSmem {
-  static constexpr int kStages = N >= 32 ? 2 : 3;
+  static constexpr int kStages = N >= 64 ? 2 : 3;
   static_assert(kStages >= 2, "chunk c+1 must be resident while chunk c is finished");
-  static constexpr int kX = kSsdQ * kSsdP * 2;           // one head's x tile (8 KB)
+  static constexpr int kX = kSsdQ * kSsdP * 2;           // the head's x tile (8 KB)
   static constexpr int kBC = kSsdQ * N * 2;              // one B or C tile
-  static constexpr int kStage = kSsdHeads * kX + 2 * kBC;  // x of both heads, B, C
+  static constexpr int kStage = kX + 2 * kBC;            // x, B, C
   static constexpr int kRing = kStages * kStage;
-  static constexpr int kM = kRing;                       // [2 heads] M tiles, 64 x 64
-  static constexpr int kCt = kM + kSsdHeads * kSsdQ * kSsdQ * 2;  // [2] C~ tiles, 64 x N
-  static constexpr int kBw = kCt + kSsdHeads * kBC;      // [2] Bw tiles, 64 x N
-  static constexpr int kS = kBw + kSsdHeads * kBC;       // [2] bf16 state copies, 64 ch x N
-  static constexpr int kCum = kS + kSsdHeads * kSsdP * N * 2;  // [2][64] cum (log2), [2][64] w, [2][64] u
-  static constexpr int kWsum = kCum + 3 * kSsdHeads * kSsdQ * 4;  // [4 warps][2 heads] partial sums
-  static constexpr int kDs = kWsum + kSsdWarps * kSsdHeads * 4;   // [2 heads][64] D
-  static constexpr int kBar = kDs + kSsdHeads * kSsdP * 4;        // 2 mbarriers
+  static constexpr int kM = kRing;                       // M tile, 64 x 64
+  static constexpr int kCt = kM + kSsdQ * kSsdQ * 2;     // C~ tile, 64 x N
+  static constexpr int kBw = kCt + kBC;                  // Bw tile, 64 x N
+  static constexpr int kS = kBw + kBC;                   // bf16 state copy, 64 ch x N
+  static constexpr int kCum = kS + kSsdP * N * 2;        // [64] cum (log2), [64] w, [64] u
+  static constexpr int kWsum = kCum + 3 * kSsdQ * 4;     // [4 warps] partial sums
+  static constexpr int kDs = kWsum + 16;                 // [64] D
+  static constexpr int kBar = kDs + kSsdP * 4;           // 2 mbarriers
   static constexpr int kTslot = kBar + 16;
   static constexpr int kBytes = kTslot + 16 + 1024;      // + room to align the base to 1024
-  static constexpr int kSboBC = (N / 8) * 128;            // K-major [rows][N]
+  static constexpr int kSboBC = (N / 8) * 128;           // K-major [rows][N]
 };
 
 template <int N, bool AGG>
@@ -189,26 +195,24 @@ __global__ void __launch_bounds__(kSsdWarps * 32)
 ssd_chunk_kernel(const SsdArgs a) {
   using L = SsdSmem<N>;
   static_assert(N % 16 == 0 && N <= 64, "states in steps of 16, at most 64 (tensor-memory columns)");
+  constexpr int NH = N / 2;                 // states per thread
   extern __shared__ __align__(1024) unsigned char ssd_smem_raw[];
   unsigned char* smem = ssd_smem_raw + ((1024u - (smem_addr(ssd_smem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
-  const int hd = lane >> 4;                 // head of this thread within the CTA
+  const int ch = lane >> 4;                 // column half (and half of the states) of this thread
   const int row = 16 * warp + (lane & 15);  // its row (token) or channel
   const int64_t channels = (int64_t)a.heads * kSsdP;
 
-  // job: (batch row, head pair, super-chunk); the aggregate kernel has one
-  // super-chunk fewer per pair
+  // job: (batch row, head, super-chunk); the aggregate kernel has one
+  // super-chunk fewer per head
   const int per_seq = AGG ? a.supers - 1 : a.supers;
-  const int64_t seq = blockIdx.x / per_seq;  // batch row * head_pairs + pair
+  const int64_t seq = blockIdx.x / per_seq;  // batch row * heads + head
   const int j = (int)(blockIdx.x % per_seq);
-  const int64_t b = seq / a.head_pairs;
-  const int hp = (int)(seq % a.head_pairs);
-  const int h = 2 * hp + hd;                // this thread's head
-  const bool hok = h < a.heads;
-  const bool pair = 2 * hp + 1 < a.heads;   // the CTA's second head exists
+  const int64_t b = seq / a.heads;
+  const int h = (int)(seq % a.heads);
   const int64_t t_begin = (int64_t)j * a.super_len;
   const int64_t t_end = t_begin + a.super_len < a.len ? t_begin + a.super_len : a.len;
   const int nchunks = (int)((t_end - t_begin + kSsdQ - 1) / kSsdQ);
@@ -229,27 +233,25 @@ ssd_chunk_kernel(const SsdArgs a) {
   }
   griddep_wait();  // inputs (and the aggregates) may come from the previous kernel
 
-  const int hc = hok ? h : 0;               // a valid head for reads
-  const float a_h = __ldg(a.A + hc);
+  const float a_h = __ldg(a.A + h);
   const float a2 = a_h * 1.4426950408889634f;  // a in log2 units
   const __nv_bfloat16* Bg = a.B + (b * a.len) * N;
   const __nv_bfloat16* Cg = a.C + (b * a.len) * N;
-  const unsigned short* dtg = reinterpret_cast<const unsigned short*>(a.dt) + (b * a.len) * a.heads + hc;
+  const __nv_bfloat16* xg = a.x + (b * a.len) * channels + (int64_t)h * kSsdP;
+  const unsigned short* dtg = reinterpret_cast<const unsigned short*>(a.dt) + (b * a.len) * a.heads + h;
 
-  // stage one chunk's x (both heads), B (and C) into ring slot `slot`
+  // stage one chunk's x, B (and C) into ring slot `slot`
   auto load_chunk = [&](int c, int slot) {
     const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
     const uint32_t sx = sbase + slot * L::kStage;
 #pragma unroll
-    for (int i = tid; i < kSsdHeads * kSsdQ * 8; i += kSsdWarps * 32) {
-      const int hh = i / (kSsdQ * 8), rem = i % (kSsdQ * 8);
-      const int t = rem >> 3, c8 = rem & 7;
-      const bool ok = t0 + t < t_end && 2 * hp + hh < a.heads;
-      const __nv_bfloat16* src = a.x + (b * a.len + t0 + t) * channels + (int64_t)(2 * hp + hh) * kSsdP + c8 * 8;
-      cp_async16(sx + hh * L::kX + (t >> 3) * 1024 + c8 * 128 + (t & 7) * 16, ok ? (const void*)src : (const void*)a.x,
-                 ok);
+    for (int i = tid; i < kSsdQ * 8; i += kSsdWarps * 32) {
+      const int t = i >> 3, c8 = i & 7;
+      const bool ok = t0 + t < t_end;
+      const __nv_bfloat16* src = xg + (t0 + t) * channels + c8 * 8;
+      cp_async16(sx + (t >> 3) * 1024 + c8 * 128 + (t & 7) * 16, ok ? (const void*)src : (const void*)a.x, ok);
     }
-    const uint32_t sb = sx + kSsdHeads * L::kX;
+    const uint32_t sb = sx + L::kX;
 #pragma unroll
     for (int i = tid; i < kSsdQ * (N / 8); i += kSsdWarps * 32) {
       const int t = i / (N / 8), n8 = i % (N / 8);
@@ -259,53 +261,57 @@ ssd_chunk_kernel(const SsdArgs a) {
       if (!AGG) cp_async16(sb + L::kBC + off, ok ? (const void*)(Cg + (t0 + t) * N + n8 * 8) : (const void*)a.C, ok);
     }
   };
-  auto load_dt = [&](int c) -> float {  // this thread's (token, head) step
+  // this thread's (token, head) step as raw bf16 bits (0 for padding tokens:
+  // no decay, no input); widened where it is used, a chunk later, so the
+  // load's latency is not waited for when it is issued
+  auto load_dt = [&](int c) -> uint32_t {
     const int64_t t = t_begin + (int64_t)c * kSsdQ + row;
-    if (c >= nchunks || t >= t_end) return 0.0f;  // padding tokens: no decay, no input
-    return __uint_as_float((uint32_t)__ldg(dtg + t * a.heads) << 16);
+    if (c >= nchunks || t >= t_end) return 0u;
+    return (uint32_t)__ldg(dtg + t * a.heads);
   };
 
-  // the state of this thread's (head, channel `row`): N fp32 values
-  float S[N];
+  // this thread's half of the state of channel `row`: states ch NH ..
+  // ch NH + NH - 1, fp32
+  float S[NH];
 #pragma unroll
-  for (int n = 0; n < N; ++n) S[n] = 0.0f;
-  const int64_t sidx = ((b * a.heads + hc) * kSsdP + row) * N;  // (batch, channel, n) offset
-  if (!AGG && hok) {
+  for (int n = 0; n < NH; ++n) S[n] = 0.0f;
+  const int64_t sidx = ((b * a.heads + h) * kSsdP + row) * N + ch * NH;  // (batch, channel, n) offset
+  if (!AGG) {
     if (a.h0) {
 #pragma unroll
-      for (int n = 0; n < N; ++n) S[n] = __ldg(a.h0 + sidx + n);
+      for (int n = 0; n < NH; ++n) S[n] = __ldg(a.h0 + sidx + n);
     }
     // fold in the super-chunks before this one
     const int64_t aseq = b * a.heads + h;
     for (int k = 0; k < j; ++k) {
       const int64_t agg = aseq * (a.supers - 1) + k;
       const float dec = exp2f(__ldg(a.agg_decay + agg));
-      const float* as = a.agg_state + (agg * kSsdP + row) * N;
+      const float* as = a.agg_state + (agg * kSsdP + row) * N + ch * NH;
 #pragma unroll
-      for (int n = 0; n < N; ++n) S[n] = fmaf(dec, S[n], __ldg(as + n));
+      for (int n = 0; n < NH; ++n) S[n] = fmaf(dec, S[n], __ldg(as + n));
     }
   }
   // bf16 copy of the state (K-major [channel][n]) for the next chunk's C~ S_in
   auto store_state_copy = [&]() {
-    unsigned char* st = smem + L::kS + hd * (kSsdP * N * 2) + (row >> 3) * L::kSboBC + (row & 7) * 16;
+    unsigned char* st = smem + L::kS + (row >> 3) * L::kSboBC + (row & 7) * 16;
 #pragma unroll
-    for (int n8 = 0; n8 < N / 8; ++n8) {
+    for (int q = 0; q < NH / 8; ++q) {
       uint4 v;
-      v.x = pack_bf16(S[8 * n8 + 0], S[8 * n8 + 1]);
-      v.y = pack_bf16(S[8 * n8 + 2], S[8 * n8 + 3]);
-      v.z = pack_bf16(S[8 * n8 + 4], S[8 * n8 + 5]);
-      v.w = pack_bf16(S[8 * n8 + 6], S[8 * n8 + 7]);
-      *reinterpret_cast<uint4*>(st + n8 * 128) = v;
+      v.x = pack_bf16(S[8 * q + 0], S[8 * q + 1]);
+      v.y = pack_bf16(S[8 * q + 2], S[8 * q + 3]);
+      v.z = pack_bf16(S[8 * q + 4], S[8 * q + 5]);
+      v.w = pack_bf16(S[8 * q + 6], S[8 * q + 7]);
+      *reinterpret_cast<uint4*>(st + (ch * (NH / 8) + q) * 128) = v;
     }
   };
   if (!AGG) store_state_copy();
 
-  float* Ds = reinterpret_cast<float*>(smem + L::kDs);  // [2][64] D of both heads (0 without D)
-  Ds[hd * kSsdP + row] = (a.D && hok) ? __ldg(a.D + (int64_t)h * kSsdP + row) : 0.0f;
-  float* cum_s = reinterpret_cast<float*>(smem + L::kCum);  // [2][64]
-  float* w_s = cum_s + kSsdHeads * kSsdQ;                    // [2][64]
-  float* u_s = w_s + kSsdHeads * kSsdQ;                      // [2][64] e^{-a cum_s} w_s
-  float* wsum = reinterpret_cast<float*>(smem + L::kWsum);   // [4][2]
+  float* Ds = reinterpret_cast<float*>(smem + L::kDs);  // [64] D of the head (0 without D)
+  if (ch == 0) Ds[row] = a.D ? __ldg(a.D + (int64_t)h * kSsdP + row) : 0.0f;
+  float* cum_s = reinterpret_cast<float*>(smem + L::kCum);  // [64]
+  float* w_s = cum_s + kSsdQ;                                // [64]
+  float* u_s = w_s + kSsdQ;                                  // [64] e^{-a cum_s} w_s
+  float* wsum = reinterpret_cast<float*>(smem + L::kWsum);   // [4]
   float total_log2 = 0.0f;
 
   tc_fence_before();
@@ -313,119 +319,111 @@ ssd_chunk_kernel(const SsdArgs a) {
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t t_lane = tmem + ((uint32_t)(32 * warp) << 16);  // this warp's sub-partition, + lane i = thread
-  const uint32_t d_off = (uint32_t)(16 * 1) << 16;                // head 1's accumulators: lanes 16-31
+  const uint32_t d_off = (uint32_t)16 << 16;                     // the second half's tiles: lanes 16-31
 
-  // Shared-memory descriptors, built once: a K step (or another ring slot /
-  // head) only moves the start address, the low 14 bits in 16-byte units
+  // Shared-memory descriptors, built once: a K step (or another ring slot)
+  // only moves the start address, the low 14 bits in 16-byte units
   const uint64_t dBC = umma_desc(sbase, 128, L::kSboBC);      // K-major [rows][N]: C, B, C~, S
   const uint64_t dM = umma_desc(sbase, 128, 1024);            // K-major [64][64]: M
   const uint64_t dX = umma_desc(sbase, 1024, 128);            // MN-major x (B of Y, A of dS^T)
   const uint64_t dBw = umma_desc(sbase, L::kSboBC, 128);      // MN-major Bw (B of dS^T)
   auto at = [](uint64_t d, uint32_t off) { return d + (uint64_t)(off >> 4); };
-  constexpr uint32_t kIdG = umma_idesc_bf16(64, 64, 0, 0);
-  constexpr uint32_t kIdY = umma_idesc_bf16(64, 64, 0, 1);     // M K-major, x MN-major
-  constexpr uint32_t kIdOff = umma_idesc_bf16(64, 64, 0, 0);   // C~ K-major, S K-major
+  constexpr uint32_t kIdG = umma_idesc_bf16(64, 32, 0, 0);     // C K-major, B rows K-major
+  constexpr uint32_t kIdY = umma_idesc_bf16(64, 32, 0, 1);     // M K-major, x MN-major
+  constexpr uint32_t kIdOff = umma_idesc_bf16(64, 32, 0, 0);   // C~ K-major, S K-major
   constexpr uint32_t kIdS = umma_idesc_bf16(64, N, 1, 1);      // x^T MN-major, Bw MN-major
-  constexpr uint32_t kColS = 0, kColY = 64, kColG = 128;       // tensor-memory columns
-  // G = C B^T of chunk c (slot) into columns [128, 192) of both heads' lanes
+  constexpr uint32_t kColS = 0, kColY = 64, kColG = 96;        // tensor-memory columns
+  // G = C B^T of chunk c (slot): column half hh (s = 32 hh ..) into lanes + 16 hh
   auto issue_g = [&](int slot) {
-    const uint32_t ob = slot * L::kStage + kSsdHeads * L::kX;  // B tile, then C tile
+    const uint32_t ob = slot * L::kStage + L::kX;  // B tile, then C tile
 #pragma unroll
-    for (int hh = 0; hh < kSsdHeads; ++hh) {
-      if (hh == 1 && !pair) break;
+    for (int hh = 0; hh < 2; ++hh)
 #pragma unroll
       for (int k = 0; k < N / 16; ++k)
-        umma_bf16(tmem + hh * d_off + kColG, at(dBC, ob + L::kBC + k * 256), at(dBC, ob + k * 256), kIdG, k > 0);
-    }
+        umma_bf16(tmem + hh * d_off + kColG, at(dBC, ob + L::kBC + k * 256), at(dBC, ob + 4 * hh * L::kSboBC + k * 256),
+                  kIdG, k > 0);
     umma_commit(bar_g);
   };
 
   // prologue: the first kStages chunks, and G of chunk 0
 #pragma unroll
-  for (int s = 0; s < L::kStages; ++s) {
-    if (s < nchunks) load_chunk(s, s);
+  for (int s2 = 0; s2 < L::kStages; ++s2) {
+    if (s2 < nchunks) load_chunk(s2, s2);
     cp_async_commit();
   }
   cp_async_wait<L::kStages - 1>();  // chunk 0
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
   if (!AGG && tid == 0 && nchunks > 0) issue_g(0);
-  float dt = load_dt(0);
+  uint32_t dt_raw = load_dt(0);
   bool ok_run = true;
 
   for (int c = 0; c < nchunks && ok_run; ++c) {
     const int slot = c % L::kStages;
     const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
-    const float ndt = load_dt(c + 1);
-    const uint32_t ox = slot * L::kStage;                 // x tiles of the slot
-    const uint32_t ob = ox + kSsdHeads * L::kX;           // B tile
+    const float dt = __uint_as_float(dt_raw << 16);
+    const uint32_t ndt_raw = load_dt(c + 1);
+    const uint32_t ox = slot * L::kStage;                 // x tile of the slot
+    const uint32_t ob = ox + L::kX;                       // B tile
     const uint32_t oc = ob + L::kBC;                      // C tile
 
-    // running log2 decay inside the chunk for this thread's head: an
-    // inclusive scan over the 16 lanes of the half-warp, then across warps
+    // running log2 decay inside the chunk: an inclusive scan over the 16
+    // rows of the half-warp (both halves of a warp hold the same rows), then
+    // across warps
     float v = dt * a2;
 #pragma unroll
     for (int o = 1; o < 16; o <<= 1) {
       const float nb = __shfl_up_sync(0xffffffffu, v, o, 16);
       if ((lane & 15) >= o) v += nb;
     }
-    if ((lane & 15) == 15) wsum[warp * kSsdHeads + hd] = v;
+    if (lane == 15) wsum[warp] = v;
     const float wgt = a.euler ? dt : expm1f(dt * a_h) / a_h;
     __syncthreads();  // the warp sums
     float pre = 0.0f;
-    for (int w2 = 0; w2 < warp; ++w2) pre += wsum[w2 * kSsdHeads + hd];
+    for (int w2 = 0; w2 < warp; ++w2) pre += wsum[w2];
     const float cum = v + pre;
-    float cum_end = 0.0f;
-    for (int w2 = 0; w2 < kSsdWarps; ++w2) cum_end += wsum[w2 * kSsdHeads + hd];
+    const float cum_end = (wsum[0] + wsum[1]) + (wsum[2] + wsum[3]);
     total_log2 += cum_end;
-    cum_s[hd * kSsdQ + row] = cum;
-    w_s[hd * kSsdQ + row] = wgt;
     // the decay from s to t factors as e^{a cum_t} e^{-a cum_s} while the
     // factors stay in range (the chunk decays by less than 2^-100)
     const bool split = cum_end > -100.0f;
-    u_s[hd * kSsdQ + row] = split ? ex2_approx(-cum) * wgt : 0.0f;
+    if (ch == 0) {
+      cum_s[row] = cum;
+      w_s[row] = wgt;
+      u_s[row] = split ? ex2_approx(-cum) * wgt : 0.0f;
+    }
 
-    // C~ = e^{a cum_t} C_t and Bw = e^{a(cum_end - cum_s)} w_s B_s, row `row` of head hd
+    // C~ = e^{a cum_t} C_t and Bw = e^{a(cum_end - cum_s)} w_s B_s for row
+    // `row`: each of the row's two threads takes half of the 16-byte pieces
     {
-      const float fB = ex2_approx(cum_end - cum) * wgt;
-      const unsigned char* brow = smem + ob + (row >> 3) * L::kSboBC + (row & 7) * 16;
-      // Bw [s][n] as MN-major (N = n, K = s): (s/8) (N/8 128) + (n/8) 128 + (s%8) 16 + (n%8) 2,
-      // the same bytes as the K-major [s][n] placement of B
-      unsigned char* bwrow = smem + L::kBw + hd * L::kBC + (row >> 3) * L::kSboBC + (row & 7) * 16;
-#pragma unroll
-      for (int n8 = 0; n8 < N / 8; ++n8) {
-        const uint4 bv = *reinterpret_cast<const uint4*>(brow + n8 * 128);
-        const uint32_t bw4[4] = {bv.x, bv.y, bv.z, bv.w};
+      auto scaled = [&](const unsigned char* src, unsigned char* dst, float f) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
         uint32_t op[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&bw4[q]));
-          op[q] = pack_bf16(f.x * fB, f.y * fB);
+          const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]));
+          op[q] = pack_bf16(x2.x * f, x2.y * f);
         }
-        *reinterpret_cast<uint4*>(bwrow + n8 * 128) = make_uint4(op[0], op[1], op[2], op[3]);
-      }
-      if (!AGG) {
-        const float fC = ex2_approx(cum);
-        const unsigned char* crow = smem + oc + (row >> 3) * L::kSboBC + (row & 7) * 16;
-        unsigned char* ctrow = smem + L::kCt + hd * L::kBC + (row >> 3) * L::kSboBC + (row & 7) * 16;
+        *reinterpret_cast<uint4*>(dst) = make_uint4(op[0], op[1], op[2], op[3]);
+      };
+      const uint32_t roff = (row >> 3) * L::kSboBC + (row & 7) * 16;
+      // Bw [s][n] as MN-major (N = n, K = s): (s/8) (N/8 128) + (n/8) 128 + (s%8) 16 + (n%8) 2,
+      // the same bytes as the K-major [s][n] placement of B
+      const float fB = ex2_approx(cum_end - cum) * wgt;
+      const float fC = ex2_approx(cum);
 #pragma unroll
-        for (int n8 = 0; n8 < N / 8; ++n8) {
-          const uint4 cv = *reinterpret_cast<const uint4*>(crow + n8 * 128);
-          const uint32_t cw4[4] = {cv.x, cv.y, cv.z, cv.w};
-          uint32_t op[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cw4[q]));
-            op[q] = pack_bf16(f.x * fC, f.y * fC);
-          }
-          *reinterpret_cast<uint4*>(ctrow + n8 * 128) = make_uint4(op[0], op[1], op[2], op[3]);
-        }
+      for (int q = 0; q < N / 16; ++q) {
+        const int n8 = ch * (N / 16) + q;
+        scaled(smem + ob + roff + n8 * 128, smem + L::kBw + roff + n8 * 128, fB);
+        if (!AGG) scaled(smem + oc + roff + n8 * 128, smem + L::kCt + roff + n8 * 128, fC);
       }
     }
     __syncthreads();  // cum and w of the chunk are in shared memory
 
     if (!AGG) {
-      // M row `row` of head hd from G: causal mask, decay and input weight
+      // M row `row`, columns s = 32 ch .. 32 ch + 31, from G: causal mask,
+      // decay and input weight
       bool got = mbar_wait_bounded(bar_g, (uint32_t)(c & 1), a.wait_limit_ns);
       got = __all_sync(0xffffffffu, got);  // warp-uniform: the tensor-memory loads are warp-wide
       if (!got) {
@@ -433,43 +431,41 @@ ssd_chunk_kernel(const SsdArgs a) {
         ok_run = false;
       }
       tc_fence_after();
-      const float* cum_h = cum_s + hd * kSsdQ;
-      const float* w_h = w_s + hd * kSsdQ;
-      const float* u_h = u_s + hd * kSsdQ;
-      unsigned char* mrow = smem + L::kM + hd * (kSsdQ * kSsdQ * 2) + (row >> 3) * 1024 + (row & 7) * 16;
+      unsigned char* mrow = smem + L::kM + (row >> 3) * 1024 + (row & 7) * 16;
       if (ok_run) {
-        float g[64];
-        tmem_ld64(t_lane + kColG, g);
+        float g[32];
+        tmem_ldN<32>(t_lane + kColG, g);
+        const int sb = 32 * ch;
         if (split) {
           // M[t][s] = G[t][s] e^{a cum_t} (e^{-a cum_s} w_s), s <= t
           const float et = ex2_approx(cum);
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const float4 ua = *reinterpret_cast<const float4*>(u_h + 8 * c8);
-            const float4 ub = *reinterpret_cast<const float4*>(u_h + 8 * c8 + 4);
+          for (int c8 = 0; c8 < 4; ++c8) {
+            const float4 ua = *reinterpret_cast<const float4*>(u_s + sb + 8 * c8);
+            const float4 ub = *reinterpret_cast<const float4*>(u_s + sb + 8 * c8 + 4);
             const float uu[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
             uint32_t op[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int s0 = 8 * c8 + 2 * e;
-              const float m0 = s0 <= row ? g[s0] * et * uu[2 * e] : 0.0f;
-              const float m1 = s0 + 1 <= row ? g[s0 + 1] * et * uu[2 * e + 1] : 0.0f;
+              const int s0 = sb + 8 * c8 + 2 * e, i0 = 8 * c8 + 2 * e;
+              const float m0 = s0 <= row ? g[i0] * et * uu[2 * e] : 0.0f;
+              const float m1 = s0 + 1 <= row ? g[i0 + 1] * et * uu[2 * e + 1] : 0.0f;
               op[e] = pack_bf16(m0, m1);
             }
-            *reinterpret_cast<uint4*>(mrow + c8 * 128) = make_uint4(op[0], op[1], op[2], op[3]);
+            *reinterpret_cast<uint4*>(mrow + (4 * ch + c8) * 128) = make_uint4(op[0], op[1], op[2], op[3]);
           }
         } else {
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
+          for (int c8 = 0; c8 < 4; ++c8) {
             uint32_t op[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int s0 = 8 * c8 + 2 * e;
-              const float m0 = s0 <= row ? g[s0] * ex2_approx(cum - cum_h[s0]) * w_h[s0] : 0.0f;
-              const float m1 = s0 + 1 <= row ? g[s0 + 1] * ex2_approx(cum - cum_h[s0 + 1]) * w_h[s0 + 1] : 0.0f;
+              const int s0 = sb + 8 * c8 + 2 * e, i0 = 8 * c8 + 2 * e;
+              const float m0 = s0 <= row ? g[i0] * ex2_approx(cum - cum_s[s0]) * w_s[s0] : 0.0f;
+              const float m1 = s0 + 1 <= row ? g[i0 + 1] * ex2_approx(cum - cum_s[s0 + 1]) * w_s[s0 + 1] : 0.0f;
               op[e] = pack_bf16(m0, m1);
             }
-            *reinterpret_cast<uint4*>(mrow + c8 * 128) = make_uint4(op[0], op[1], op[2], op[3]);
+            *reinterpret_cast<uint4*>(mrow + (4 * ch + c8) * 128) = make_uint4(op[0], op[1], op[2], op[3]);
           }
         }
       }
@@ -484,23 +480,22 @@ ssd_chunk_kernel(const SsdArgs a) {
     tc_fence_after();
     if (tid == 0 && ok_run) {
 #pragma unroll
-      for (int hh = 0; hh < kSsdHeads; ++hh) {
-        if (hh == 1 && !pair) break;
-        const uint32_t xs = ox + hh * L::kX;
+      for (int hh = 0; hh < 2; ++hh) {
         if (!AGG) {
+          // Y half hh (channels 32 hh ..): M X then + C~ S_in
           const uint32_t dy = tmem + hh * d_off + kColY;
-          const uint32_t ms = L::kM + hh * (kSsdQ * kSsdQ * 2);
 #pragma unroll
-          for (int k = 0; k < kSsdQ / 16; ++k) umma_bf16(dy, at(dM, ms + k * 256), at(dX, xs + k * 2048), kIdY, k > 0);
-          const uint32_t cts = L::kCt + hh * L::kBC;
-          const uint32_t ss = L::kS + hh * (kSsdP * N * 2);
+          for (int k = 0; k < kSsdQ / 16; ++k)
+            umma_bf16(dy, at(dM, L::kM + k * 256), at(dX, ox + 512 * hh + k * 2048), kIdY, k > 0);
 #pragma unroll
-          for (int k = 0; k < N / 16; ++k) umma_bf16(dy, at(dBC, cts + k * 256), at(dBC, ss + k * 256), kIdOff, true);
+          for (int k = 0; k < N / 16; ++k)
+            umma_bf16(dy, at(dBC, L::kCt + k * 256), at(dBC, L::kS + 4 * hh * L::kSboBC + k * 256), kIdOff, true);
         }
-        const uint32_t bws = L::kBw + hh * L::kBC;
+        // dS^T over tokens 32 hh .. 32 hh + 31
 #pragma unroll
-        for (int k = 0; k < kSsdQ / 16; ++k)
-          umma_bf16(tmem + hh * d_off + kColS, at(dX, xs + k * 2048), at(dBw, bws + k * 2 * L::kSboBC), kIdS, k > 0);
+        for (int k = 2 * hh; k < 2 * hh + 2; ++k)
+          umma_bf16(tmem + hh * d_off + kColS, at(dX, ox + k * 2048), at(dBw, L::kBw + k * 2 * L::kSboBC), kIdS,
+                    k > 2 * hh);
       }
       umma_commit(bar_y);
       if (!AGG && c + 1 < nchunks) issue_g((c + 1) % L::kStages);
@@ -516,16 +511,37 @@ ssd_chunk_kernel(const SsdArgs a) {
     }
     tc_fence_after();
     if (ok_run) {
-      if (!AGG) {
-        // y = Y + D x for row `row` of head hd -> bf16 -> 16-byte stores
-        const float* Dh = Ds + hd * kSsdP;
-        const unsigned char* xrow = smem + ox + hd * L::kX + (row >> 3) * 1024 + (row & 7) * 16;
-        const bool store = hok && t0 + row < t_end;
-        __nv_bfloat16* yrow = a.y + (b * a.len + t0 + row) * channels + (int64_t)hc * kSsdP;
-        float yv[64];
-        tmem_ld64(t_lane + kColY, yv);
+      // this thread's half row of Y and its partial dS^T row: one round
+      // trip to tensor memory
+      float yv[32], ds[N];
+      {
+        uint32_t ry[2][16], rs[N / 16][16];
+        if (!AGG) {
+          tmem_ld16_nowait(t_lane + kColY, ry[0]);
+          tmem_ld16_nowait(t_lane + kColY + 16, ry[1]);
+        }
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
+        for (int q = 0; q < N / 16; ++q) tmem_ld16_nowait(t_lane + kColS + 16 * q, rs[q]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          yv[i] = AGG ? 0.0f : __uint_as_float(ry[0][i]);
+          yv[16 + i] = AGG ? 0.0f : __uint_as_float(ry[1][i]);
+        }
+#pragma unroll
+        for (int q = 0; q < N / 16; ++q)
+#pragma unroll
+          for (int i = 0; i < 16; ++i) ds[16 * q + i] = __uint_as_float(rs[q][i]);
+      }
+      if (!AGG) {
+        // y = Y + D x for row `row`, channels 32 ch .. 32 ch + 31 -> bf16 ->
+        // 16-byte stores
+        const float* Dh = Ds + 32 * ch;
+        const unsigned char* xrow = smem + ox + (row >> 3) * 1024 + (row & 7) * 16 + 4 * ch * 128;
+        const bool store = t0 + row < t_end;
+        __nv_bfloat16* yrow = a.y + (b * a.len + t0 + row) * channels + (int64_t)h * kSsdP + 32 * ch;
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
           const uint4 xv = *reinterpret_cast<const uint4*>(xrow + c8 * 128);
           const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
           const float4 da = *reinterpret_cast<const float4*>(Dh + 8 * c8);
@@ -541,14 +557,15 @@ ssd_chunk_kernel(const SsdArgs a) {
           if (store) *reinterpret_cast<uint4*>(yrow + 8 * c8) = make_uint4(op[0], op[1], op[2], op[3]);
         }
       }
-      // S = e^{a cum_end} S + dS for channel `row` of head hd; its bf16 copy
-      // feeds the next chunk's C~ S_in (this chunk's products are done)
+      // S = e^{a cum_end} S + dS for channel `row`: this thread holds the
+      // partial sum over tokens 32 ch .. of every state; it keeps states
+      // ch NH .. and swaps the other half with the row's other thread
       const float dec = ex2_approx(cum_end);
-      {
-        float ds[N];
-        tmem_ldN<N>(t_lane + kColS, ds);
 #pragma unroll
-        for (int i = 0; i < N; ++i) S[i] = fmaf(dec, S[i], ds[i]);
+      for (int i = 0; i < NH; ++i) {
+        const float keep = ch ? ds[NH + i] : ds[i];
+        const float give = ch ? ds[i] : ds[NH + i];
+        S[i] = fmaf(dec, S[i], keep + __shfl_xor_sync(0xffffffffu, give, 16));
       }
       if (!AGG) store_state_copy();
     }
@@ -557,21 +574,21 @@ ssd_chunk_kernel(const SsdArgs a) {
     // chunk c + kStages into the slot chunk c used
     if (c + L::kStages < nchunks) load_chunk(c + L::kStages, slot);
     cp_async_commit();
-    dt = ndt;
+    dt_raw = ndt_raw;
   }
   cp_async_wait<0>();
 
   griddep_launch_dependents();
-  if (ok_run && hok) {
+  if (ok_run) {
     if (AGG) {
       const int64_t agg = (b * a.heads + h) * (a.supers - 1) + j;
-      float* as = a.agg_state + (agg * kSsdP + row) * N;
+      float* as = a.agg_state + (agg * kSsdP + row) * N + ch * NH;
 #pragma unroll
-      for (int n = 0; n < N; ++n) as[n] = S[n];
-      if ((lane & 15) == 0 && warp == 0) a.agg_decay[agg] = total_log2;
+      for (int n = 0; n < NH; ++n) as[n] = S[n];
+      if (tid == 0) a.agg_decay[agg] = total_log2;
     } else if (a.final_state && j == a.supers - 1) {
 #pragma unroll
-      for (int n = 0; n < N; ++n) a.final_state[sidx + n] = S[n];
+      for (int n = 0; n < NH; ++n) a.final_state[sidx + n] = S[n];
     }
   }
   tc_fence_before();
