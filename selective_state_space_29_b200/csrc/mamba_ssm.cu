@@ -170,8 +170,8 @@ struct Plan {
 // fewer than the resident consumer warps, sequences are cut into
 // super-chunks that run from zero side by side and are joined afterwards by
 // the correction kernel (about as many streams as warps: each extra
-// super-chunk adds a correction walk, which is short once the decay has
-// underflowed).  Within a stream the sequence is cut into chunks so that
+// super-chunk adds a correction walk, which ends once the carried decay is
+// below 2^-32).  Within a stream the sequence is cut into chunks so that
 // there are about kJobsPerWarp jobs per warp for dynamic balance, each at
 // least two tiles long.  A positive `user_chunk` forces super-chunks of that
 // length.

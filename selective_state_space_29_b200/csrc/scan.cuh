@@ -32,9 +32,11 @@
 //     second kernel adds their effect to the outputs:
 //         y_t += sum_n C_t[n] exp(A_n cum_t) h_in[n],
 //     cum_t the sum of Delta from the super-chunk's start through t.  It
-//     walks each super-chunk only until exp2 of the slowest decay underflows
-//     to zero in fp32, beyond which the term is exactly zero, and writes the
-//     final state H + exp(A sum Delta) h_in of the last super-chunk.
+//     walks each super-chunk only while the slowest decay exp(A_n cum_t) is
+//     at least 2^-kFixStopLog2 (2^-32): past that every term is below 2^-32
+//     of |C_t[n] h_in[n]|, 256 times under the fp32 rounding of y.  It also
+//     writes the final state H + exp(A sum Delta) h_in of the last
+//     super-chunk (exactly, not truncated).
 //
 // Arithmetic per token and state (all fp32; the state is kept scaled,
 // g_n = A_n h_n, so that 1/A_n leaves the inner loop):
@@ -67,6 +69,7 @@ namespace mamba {
 
 constexpr int kCPW = 32;   // channels per warp: one lane per channel
 constexpr int kFixSegTiles = 1;  // tiles per segment of the super-chunk correction
+constexpr float kFixStopLog2 = 32.0f;  // the correction stops where the carried decay is below 2^-32
 constexpr int kHandQ = 8;  // hand-off flags a consumer may leave for the producer to publish
 
 enum Discretisation : int { kZOH = 0, kEuler = 1, kTrapezoid = 2 };
@@ -855,9 +858,9 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES, R>& cx, 
     for (int k = 0; k < NS / 2; ++k) g[k] = f2(h[2 * k] * an[2 * k], h[2 * k + 1] * an[2 * k + 1]);
   }
   // super-chunks 1..S-1 ran from zero: leave the correction kernel the sum
-  // of Delta at every segment start, until exp2 of the slowest decay
-  // underflows to zero on every lane (then the carried state's term is
-  // exactly zero in fp32 for the rest of the super-chunk)
+  // of Delta at every segment start, until the slowest decay falls below
+  // 2^-kFixStopLog2 on every lane (the carried state's term is negligible
+  // in fp32 for the rest of the super-chunk)
   bool track = p.supers > 1 && jb.super_idx > 0;
   float kmax = 0.0f;
   if (track) {
@@ -897,7 +900,7 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES, R>& cx, 
     const int64_t tt0 = jb.t0 + (int64_t)it * TILE;
     const int rows = (int)(jb.t1 - tt0 < (int64_t)TILE ? jb.t1 - tt0 : (int64_t)TILE);
     if (track && (tile0 + it) % kFixSegTiles == 0) {
-      if (__all_sync(0xffffffffu, !active || ex2_approx(sd * kmax) == 0.0f)) {
+      if (__all_sync(0xffffffffu, !active || sd * kmax < -kFixStopLog2)) {
         track = false;
       } else {
         const int seg = (int)((tile0 + it) / kFixSegTiles);
@@ -1054,8 +1057,8 @@ scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__
 //     sum_n C_t[n] exp(A_n cum_t) h_in[n],   cum_t = sum of Delta from the
 //                                            super-chunk's start through t.
 // The main pass left cum at the start of every tile, up to the tile where
-// exp2 of the slowest decay underflows to zero on every lane (from there on
-// the term is exactly zero in fp32), and the number of such tiles per
+// the slowest decay falls below 2^-kFixStopLog2 on every lane (from there on
+// the term is below 2^-32 of its size), and the number of such tiles per
 // stream.  One warp per (stream of a super-chunk j >= 1, phase w), a lane per
 // channel, takes tiles w, w + phases, ...: it stages the tile's Delta, y
 // and C rows in its shared memory (16-byte cp.async copies, all in flight
@@ -1217,8 +1220,8 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
       }
     }
     __syncwarp();
-    if (__all_sync(0xffffffffu, !active || ex2_approx(cum * kmax) == 0.0f))
-      break;  // later tiles of this warp add exactly zero (their cum is larger)
+    if (__all_sync(0xffffffffu, !active || cum * kmax < -kFixStopLog2))
+      break;  // later tiles of this warp add less (their cum is larger)
   }
 }
 

@@ -240,13 +240,16 @@ ssd_chunk_kernel(const SsdArgs a) {
   const __nv_bfloat16* xg = a.x + (b * a.len) * channels + (int64_t)h * kSsdP;
   const unsigned short* dtg = reinterpret_cast<const unsigned short*>(a.dt) + (b * a.len) * a.heads + h;
 
-  // stage one chunk's x, B (and C) into ring slot `slot`
+  // Stage one chunk's x, B (and C) into ring slot `slot`.  Piece i of 16
+  // bytes: i % 8 is the token within a group of 8, so the 8 lanes of a
+  // quarter-warp fill one core matrix (128 contiguous bytes of shared memory,
+  // one wavefront), while a warp reads 8 token rows, whole 32-byte sectors.
   auto load_chunk = [&](int c, int slot) {
     const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
     const uint32_t sx = sbase + slot * L::kStage;
 #pragma unroll
     for (int i = tid; i < kSsdQ * 8; i += kSsdWarps * 32) {
-      const int t = i >> 3, c8 = i & 7;
+      const int t = (i & 7) + 8 * (i >> 6), c8 = (i >> 3) & 7;
       const bool ok = t0 + t < t_end;
       const __nv_bfloat16* src = xg + (t0 + t) * channels + c8 * 8;
       cp_async16(sx + (t >> 3) * 1024 + c8 * 128 + (t & 7) * 16, ok ? (const void*)src : (const void*)a.x, ok);
@@ -254,7 +257,7 @@ ssd_chunk_kernel(const SsdArgs a) {
     const uint32_t sb = sx + L::kX;
 #pragma unroll
     for (int i = tid; i < kSsdQ * (N / 8); i += kSsdWarps * 32) {
-      const int t = i / (N / 8), n8 = i % (N / 8);
+      const int n8 = (i >> 3) % (N / 8), t = (i & 7) + 8 * (i / (8 * (N / 8)));
       const bool ok = t0 + t < t_end;
       const uint32_t off = (t >> 3) * L::kSboBC + n8 * 128 + (t & 7) * 16;
       cp_async16(sb + off, ok ? (const void*)(Bg + (t0 + t) * N + n8 * 8) : (const void*)a.B, ok);
