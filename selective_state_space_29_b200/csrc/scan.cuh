@@ -1103,23 +1103,48 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
   for (int k = 0; k < NS; ++k)
     an[k] = structured ? (float)(k + 1) * cm.x : (active ? __ldg(p.A + (int64_t)d * NS + k) : -1.0f);
 
-  // the entering state
+  // exp(A_n sd) for every state: one exponential and a product chain when
+  // A is structured (exp((n+1) A_0 sd) = exp(A_0 sd)^(n+1)), else one each
+  auto decays = [&](float sd, float (&e)[NS]) {
+    if (structured) {
+      const float r = ex2_approx(sd * an[0] * kLog2e);
+      e[0] = r;
+#pragma unroll
+      for (int k = 1; k < NS; ++k) e[k] = e[k - 1] * r;
+    } else {
+#pragma unroll
+      for (int k = 0; k < NS; ++k) e[k] = ex2_approx(sd * an[k] * kLog2e);
+    }
+  };
+  // the entering state: h <- exp(A sum Delta_j) h + H_j over the earlier
+  // super-chunks (the loads of a step do not wait for the previous step)
   float h[NS];
 #pragma unroll
   for (int k = 0; k < NS; ++k) h[k] = 0.0f;
+#pragma unroll 2
   for (int j = 0; j < super_idx; ++j) {
     const int64_t sj = (int64_t)j * p.groups + grp;
     const float sdj = __ldcg(p.agg_sd + sj * kCPW + lane);
-    const float* H = p.agg_h + (sj * kCPW + lane) * NS;
+    const float4* H = reinterpret_cast<const float4*>(p.agg_h + (sj * kCPW + lane) * NS);
+    float e[NS];
+    decays(sdj, e);
 #pragma unroll
-    for (int k = 0; k < NS; ++k) h[k] = fmaf(expf(an[k] * sdj), h[k], __ldcg(H + k));
+    for (int k = 0; k < NS / 4; ++k) {
+      const float4 v = __ldcg(H + k);
+      h[4 * k] = fmaf(e[4 * k], h[4 * k], v.x);
+      h[4 * k + 1] = fmaf(e[4 * k + 1], h[4 * k + 1], v.y);
+      h[4 * k + 2] = fmaf(e[4 * k + 2], h[4 * k + 2], v.z);
+      h[4 * k + 3] = fmaf(e[4 * k + 3], h[4 * k + 3], v.w);
+    }
   }
   if (super_idx == p.supers - 1 && w == 0 && p.final_state && active) {
     const float sdl = __ldcg(p.agg_sd + (int64_t)stream * kCPW + lane);
     const float* H = p.agg_h + ((int64_t)stream * kCPW + lane) * NS;
     float* dst = p.final_state + ((int64_t)b * p.channels + d) * NS;
+    float e[NS];
+    decays(sdl, e);
 #pragma unroll
-    for (int k = 0; k < NS; ++k) dst[k] = fmaf(expf(an[k] * sdl), h[k], __ldcg(H + k));
+    for (int k = 0; k < NS; ++k) dst[k] = fmaf(e[k], h[k], __ldcg(H + k));
   }
 
   const float a0l = cm.x * kLog2e;  // structured: every decay is a power of exp(A_0 cum)
@@ -1181,25 +1206,41 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
         }
       }
       cum += to_f32(sdl[r * kCPW + lane]);
-      // the carried state's decay to this token: rho_n = exp(A_n cum)
-      float ph[NS];
-      if (structured) {
-        const float rho = ex2_approx(cum * a0l);
-        float pw = rho;
+      // the carried state's decay to this token, exp(A_n cum)
+      const float rho = ex2_approx(cum * a0l);
+      float ev[NS];
+      if (!structured) {
 #pragma unroll
-        for (int n = 0; n < NS; ++n) {
-          ph[n] = pw * h[n];
-          pw *= rho;
-        }
-      } else {
-#pragma unroll
-        for (int n = 0; n < NS; ++n) ph[n] = ex2_approx(cum * an[n] * kLog2e) * h[n];
+        for (int n = 0; n < NS; ++n) ev[n] = ex2_approx(cum * an[n] * kLog2e);
       }
 #pragma unroll
       for (int q = 0; q < R; ++q) {  // output q reads the state with its own C row
-        float corr = 0.0f;
+        float cv[NS];
+        const TIO* crow = sc + (r * R + q) * NS;
+        if constexpr ((NS * sizeof(TIO)) % 16 == 0) {
 #pragma unroll
-        for (int n = 0; n < NS; ++n) corr = fmaf(to_f32(sc[(r * R + q) * NS + n]), ph[n], corr);
+          for (int i = 0; i < NS; i += kChunk) {
+            const uint4 v = *reinterpret_cast<const uint4*>(crow + i);
+            const TIO* e = reinterpret_cast<const TIO*>(&v);
+#pragma unroll
+            for (int k2 = 0; k2 < kChunk; ++k2) cv[i + k2] = to_f32(e[k2]);
+          }
+        } else {
+#pragma unroll
+          for (int n = 0; n < NS; ++n) cv[n] = to_f32(crow[n]);
+        }
+        float corr;
+        if (structured) {
+          // sum_n C_n h_n rho^(n+1), Horner in rho
+          corr = cv[NS - 1] * h[NS - 1];
+#pragma unroll
+          for (int n = NS - 2; n >= 0; --n) corr = fmaf(corr, rho, cv[n] * h[n]);
+          corr *= rho;
+        } else {
+          corr = 0.0f;
+#pragma unroll
+          for (int n = 0; n < NS; ++n) corr = fmaf(cv[n], ev[n] * h[n], corr);
+        }
         TIO& yv = sy[(r * R + q) * kCPW + lane];
         yv = from_f32<TIO>(to_f32(yv) + corr);
       }
