@@ -74,6 +74,10 @@ def parse_args():
     ap.add_argument("--no-ssd", action="store_true", help="skip Mamba-2's scalar-A scan (state space duality) leg")
     ap.add_argument("--only-backward", action="store_true",
                     help="run only the backward on the workload's shape (steps = timed calls) and print its object")
+    ap.add_argument("--only-complex", action="store_true",
+                    help="time only the complex-valued state scan on --workload (a small case for ncu)")
+    ap.add_argument("--only-mimo", action="store_true",
+                    help="time only the multi-input multi-output scan and step (a small case for ncu)")
     ap.add_argument("--only-ssd", action="store_true",
                     help="run only the scalar-A scan leg (steps/warmup as given) and print its object")
     ap.add_argument("--length-sweep", action="store_true",
@@ -487,7 +491,8 @@ def run_ours(args):
     roofline = {"bound": "hbm", "achieved": round(hbm_ach, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(hbm_ach / hbm_peak, 4),
                 "traffic": profiled_traffic("scan_chunks_kernel", args.workload),
-                "peak_source": f"{hbm_src} (MEASURED_PEAKS.json hbm_gbs)",
+                "peak_source": ("measured (MEASURED_PEAKS.json hbm_gbs)" if hbm_src == "measured" else
+                                f"fallback: the profiling recipe's {FALLBACK_HBM_GBS:.0f} GB/s (no MEASURED_PEAKS.json)"),
                 "kernel": "scan_chunks_kernel (timed per call: the call's pre-pass included)",
                 "call_ms": round(call_ms, 5), "algorithmic_bytes_per_launch": nbytes,
                 "bytes_per_tc": round(nbytes / tc, 4),
@@ -818,6 +823,46 @@ def run_mimo(dev, stream, dist, world, rank, hbm_peak, reps: int = 20) -> dict:
     return res
 
 
+def run_complex(w, dev, stream, dist, world, rank, reps: int = 20) -> dict:
+    """ms per call of the complex-valued state scan on the workload's shape
+    (complex diagonal A with imaginary parts pi n, complex state)."""
+    import torch
+
+    from selective_state_space_29_b200 import mamba_ssm as m
+    from selective_state_space_29_b200 import workloads as wl
+
+    lib = m.library()
+    dtc = m.dtype_code(w.torch_dtype)
+    tc = w.batch * w.length * w.channels
+    inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
+    A_im = wl.complex_a_imag(w.channels, w.nstate, dev)
+    y = torch.empty_like(inp["u"])
+    hf = torch.empty((w.batch, w.channels, w.nstate, 2), device=dev, dtype=torch.float32)
+
+    def cstep():
+        st = lib.mamba_selective_scan_complex(inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(),
+                                              A_im.data_ptr(), inp["B"].data_ptr(), inp["C"].data_ptr(),
+                                              inp["D"].data_ptr(), None, y.data_ptr(), hf.data_ptr(), w.batch,
+                                              w.length, w.channels, w.nstate, 0, dtc, stream.cuda_stream)
+        if st != 0:
+            raise m.MambaError(st, "mamba_selective_scan_complex")
+
+    for _ in range(3):
+        cstep()
+    torch.cuda.synchronize()
+    barrier(dist, world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        cstep()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(dist, world, a.elapsed_time(b)) / reps
+    del inp, A_im, y, hf
+    return {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
+            "nstate": w.nstate, "note": "complex diagonal A (imaginary parts pi n), complex state"}
+
+
 def run_variants(w, dev, stream, dist, world, rank, reps: int = 20):
     """ms per call and token·channels/s of the scan's options on the workload's
     shape: MAMBA_SCAN_GENERAL_A, MAMBA_SCAN_EULER, MAMBA_SCAN_TRAPEZOID, and 4, 8
@@ -861,35 +906,7 @@ def run_variants(w, dev, stream, dist, world, rank, reps: int = 20):
         res[name] = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
                      "nstate": wv.nstate}
         del inp, y, hf
-    # the complex-valued state (A_im = pi n), the same shape
-    inp = wl.scan_inputs(w, dev, seed=rank_seed(w.seed, rank))
-    A_im = wl.complex_a_imag(w.channels, w.nstate, dev)
-    y = torch.empty_like(inp["u"])
-    hf = torch.empty((w.batch, w.channels, w.nstate, 2), device=dev, dtype=torch.float32)
-
-    def cstep():
-        st = lib.mamba_selective_scan_complex(inp["u"].data_ptr(), inp["delta"].data_ptr(), inp["A"].data_ptr(),
-                                              A_im.data_ptr(), inp["B"].data_ptr(), inp["C"].data_ptr(),
-                                              inp["D"].data_ptr(), None, y.data_ptr(), hf.data_ptr(), w.batch,
-                                              w.length, w.channels, w.nstate, 0, dtc, stream.cuda_stream)
-        if st != 0:
-            raise m.MambaError(st, "mamba_selective_scan_complex")
-
-    for _ in range(3):
-        cstep()
-    torch.cuda.synchronize()
-    barrier(dist, world)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(reps):
-        cstep()
-    b.record(stream)
-    torch.cuda.synchronize()
-    ms = max_over_ranks(dist, world, a.elapsed_time(b)) / reps
-    res["complex_state"] = {"ms_per_call": round(ms, 5), "token_channels_per_s": world * tc / (ms * 1e-3),
-                            "nstate": w.nstate, "note": "complex diagonal A (imaginary parts pi n), complex state"}
-    del inp, A_im, y, hf
-
+    res["complex_state"] = run_complex(w, dev, stream, dist, world, rank, reps)
     res["backward"] = run_backward(w, dev, stream, dist, world, rank)
     res["note"] = (f"{w.name} shape; general A and the other discretisations take one exp2 per state "
                    f"(MUFU); nstate_* are zero-order hold with structured A")
@@ -1030,6 +1047,24 @@ def main():
             dist.destroy_process_group()
         if rank == 0:
             print(json.dumps({"backward": res}), flush=True)
+    elif args.only_complex or args.only_mimo:
+        import torch
+        from selective_state_space_29_b200 import workloads as wl
+        rank, world, local = dist_setup(args.gpus)
+        torch.cuda.set_device(local)
+        dist = init_pg(world, local)
+        dev, st = torch.device("cuda", local), torch.cuda.current_stream()
+        if args.only_complex:
+            res = {"complex_state": run_complex(wl.SCAN_WORKLOADS[args.workload], dev, st, dist, world, rank,
+                                                reps=max(1, args.steps))}
+        else:
+            peaks = measured_peaks()
+            res = {"mimo": run_mimo(dev, st, dist, world, rank, float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS)),
+                                    reps=max(1, args.steps))}
+        if world > 1:
+            dist.destroy_process_group()
+        if rank == 0:
+            print(json.dumps(res), flush=True)
     elif args.only_ssd:
         import torch
         rank, world, local = dist_setup(args.gpus)
