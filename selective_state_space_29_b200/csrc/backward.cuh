@@ -176,6 +176,24 @@ __device__ __forceinline__ void load_row(const TIO* row, float (&v)[NS], bool ve
 // Sum over the 32 lanes of v[0..31]; lane i returns the sum of v[i]
 // (butterfly reduce-scatter: at each step a lane keeps the half of its
 // values whose index has the lane's bit, and receives the partner's copy).
+// The state scratch is written once and read once per half tile: its
+// stores ask L2 to keep the lines (evict-last policy), and once a slot has
+// been read its lines are discarded from L2, so that dead states are never
+// written back to DRAM.
+__device__ __forceinline__ uint64_t l2_keep_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void st_keep(float* p, float4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void l2_discard128(const void* p) {  // p: 128-byte aligned
+  asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ float reduce_scatter32(float (&v)[32], int lane) {
 #pragma unroll
   for (int w = 16; w >= 1; w >>= 1) {
@@ -335,6 +353,7 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
   const int64_t streams = a.batch * a.groups_d;
   const int T = a.tile;
   const int64_t ntiles = (a.len + T - 1) / T;
+  const uint64_t keep = l2_keep_policy();  // for the state scratch
   float iA[NS], lam[NS], dA[NS];
 #pragma unroll
   for (int n = 0; n < NS; ++n) {
@@ -411,7 +430,7 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
     auto put = [&](int slot, const float (&v)[NS]) {
 #pragma unroll
       for (int n = 0; n < NS; n += 4)
-        *reinterpret_cast<float4*>(S + (size_t)slot * 32 * NS + n) = make_float4(v[n], v[n + 1], v[n + 2], v[n + 3]);
+        st_keep(S + (size_t)slot * 32 * NS + n, make_float4(v[n], v[n + 1], v[n + 2], v[n + 3]), keep);
     };
     float h[NS];
 #pragma unroll
@@ -427,7 +446,7 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
 #pragma unroll
       for (int n = 0; n < NS; ++n) h[n] = fmaf(1.0f + q[n], h[n], q[n] * iA[n] * bv[n] * x);
       if (k == start - 1) put(0, h);
-      if (k >= start) put(k - start + 1, h);
+      if (k >= start && k < end - 1) put(k - start + 1, h);  // (h after the half's last token: kept in h)
     }
     // reverse over the half; h holds h_t, hp is read back as h_{t-1}, one
     // token ahead of its use (hn)
@@ -505,7 +524,12 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
       const float s = reduce_scatter32(red, lane);
       if (lane < NS) atomicAdd(a.dB + tok * NS + lane, s);
       else if (lane < 2 * NS) atomicAdd(a.dC + tok * NS + (lane - NS), s);
+      // slot k - start (h_{t-1} of this token) has been read by every lane:
+      // drop its NS lines of 128 bytes from L2 without a write-back
+      __syncwarp();
+      if (lane < NS) l2_discard128(S - (size_t)lane * NS + (size_t)(k - start) * 32 * NS + (size_t)lane * 32);
     }
+    __syncwarp();  // every discard before the next half's stores into the same lines
     }  // half
   }
   if (active) {
