@@ -354,20 +354,27 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
   const int T = a.tile;
   const int64_t ntiles = (a.len + T - 1) / T;
   const uint64_t keep = l2_keep_policy();  // for the state scratch
-  float iA[NS], lam[NS], dA[NS];
+  // adjoints lam and the dA sums in pairs of states (n, n+1), so that the
+  // reverse step runs as packed FFMA2; LAM(n) / DA(n) / IA(n) name one state
+  float2 lam2[NS / 2], dA2[NS / 2], iA2[NS / 2], An2[NS / 2];
+  auto LAM = [&](int n) -> float& { return (n & 1) ? lam2[n >> 1].y : lam2[n >> 1].x; };
+  auto DA = [&](int n) -> float& { return (n & 1) ? dA2[n >> 1].y : dA2[n >> 1].x; };
+  auto IA = [&](int n) -> float { return (n & 1) ? iA2[n >> 1].y : iA2[n >> 1].x; };
 #pragma unroll
-  for (int n = 0; n < NS; ++n) {
-    iA[n] = 1.0f / An[n];
-    lam[n] = (active && a.dh_final) ? a.dh_final[(b * a.channels + d) * NS + n] : 0.0f;
-    dA[n] = 0.0f;
+  for (int p = 0; p < NS / 2; ++p) {
+    An2[p] = make_float2(An[2 * p], An[2 * p + 1]);
+    iA2[p] = make_float2(1.0f / An[2 * p], 1.0f / An[2 * p + 1]);
+    dA2[p] = make_float2(0.0f, 0.0f);
   }
+#pragma unroll
+  for (int n = 0; n < NS; ++n) LAM(n) = (active && a.dh_final) ? a.dh_final[(b * a.channels + d) * NS + n] : 0.0f;
   // the adjoint entering super-chunk j from the later ones:
   //   mu <- M_k + exp(A sumDelta_k) mu,  k = S-1 .. j+1,  mu_S = d h_final
   for (int k = a.supers - 1; k > j; --k) {
     const size_t base = ((size_t)k * streams + stream) * 32 + lane;
     const float sdk = a.agg_sd[base];
 #pragma unroll
-    for (int n = 0; n < NS; ++n) lam[n] = fmaf(expf(An[n] * sdk), lam[n], a.agg_mu[base * NS + n]);
+    for (int n = 0; n < NS; ++n) LAM(n) = fmaf(expf(An[n] * sdk), LAM(n), a.agg_mu[base * NS + n]);
   }
   const float Dd = (active && a.D) ? __ldg(a.D + d) : 0.0f;
   float dD = 0.0f;
@@ -444,7 +451,7 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
       get_B(k, tok, bv);
       decays<NS, STRUCT>(dt, An, q);
 #pragma unroll
-      for (int n = 0; n < NS; ++n) h[n] = fmaf(1.0f + q[n], h[n], q[n] * iA[n] * bv[n] * x);
+      for (int n = 0; n < NS; ++n) h[n] = fmaf(1.0f + q[n], h[n], q[n] * IA(n) * bv[n] * x);
       if (k == start - 1) put(0, h);
       if (k >= start && k < end - 1) put(k - start + 1, h);  // (h after the half's last token: kept in h)
     }
@@ -470,50 +477,81 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
       const float gy = get_dy(k, tok);
       float du = Dd * gy, ddt = 0.0f;
       dD = fmaf(gy, x, dD);
-      float bv[NS], cv[NS], q[NS];
+      float bv[NS], cv[NS];
       get_B(k, tok, bv);
       get_C(k, tok, cv);
       // structured A: q_n from the decay chain, and d_n = q_n - z_n exactly
       // from d_n = e^{z_0} d_{n-1} + n z_0 q_0 + d_0 (every term of one sign,
       // so nothing cancels); the B x part of dA_n is then
       // B x Delta^2 psi(z_n) = B x (z_n q_n - d_n) / A_n^2
-      float q0 = 0.0f, d0 = 0.0f;
+      float red[32];
       if constexpr (STRUCT) {
+        // q_n from the decay chain, and nd_n = -(q_n - z_n) exactly from
+        // d_n = e^{z_0} d_{n-1} + n z_0 q_0 + d_0 (every term of one sign, so
+        // nothing cancels); the B x part of dA_n is then
+        // B x Delta^2 psi(z_n) = B x (z_n q_n - d_n) / A_n^2.  Pairs of
+        // states go through packed FFMA2.
+        float q0, d0;
         expm1_parts(dt * An[0], q0, d0);
         float2 e2[NS / 2];
         decay_chain<NS>(1.0f + q0, q0, e2);
+        const float r0 = 1.0f + q0, zq0 = dt * An[0] * q0;
+        float nd[NS];
+        nd[0] = -d0;
 #pragma unroll
-        for (int kk = 0; kk < NS / 2; ++kk) {
-          q[2 * kk] = e2[kk].x;
-          q[2 * kk + 1] = e2[kk].y;
+        for (int n = 1; n < NS; ++n) nd[n] = fmaf(r0, nd[n - 1], fmaf(-(float)n, zq0, -d0));
+        const float2 x2 = make_float2(x, x), gy2 = make_float2(gy, gy), dt2 = make_float2(dt, dt);
+        const float2 one2 = make_float2(1.0f, 1.0f);
+        float2 du2 = make_float2(0.0f, 0.0f), ddt2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+        for (int pp = 0; pp < NS / 2; ++pp) {
+          const int n = 2 * pp;
+          const float2 q2 = e2[pp];
+          const float2 r2 = __fadd2_rn(q2, one2);
+          const float2 b2 = make_float2(bv[n], bv[n + 1]);
+          const float2 c2 = make_float2(cv[n], cv[n + 1]);
+          const float2 hp2 = make_float2(hp[n], hp[n + 1]);
+          const float2 bx2 = __fmul2_rn(b2, x2);
+          const float2 qa2 = __fmul2_rn(q2, iA2[pp]);
+          const float2 rc = __fmul2_rn(gy2, make_float2(h[n], h[n + 1]));  // dC_{t,n} part: dy_t h_t
+          red[NS + n] = rc.x;
+          red[NS + n + 1] = rc.y;
+          const float2 L = __ffma2_rn(c2, gy2, lam2[pp]);
+          du2 = __ffma2_rn(L, __fmul2_rn(qa2, b2), du2);
+          ddt2 = __ffma2_rn(__fmul2_rn(L, r2), __ffma2_rn(An2[pp], hp2, bx2), ddt2);
+          // d h_t / d A_n = Delta r h_{t-1} + B x Delta^2 psi(Delta A_n)
+          const float2 z2 = __fmul2_rn(dt2, An2[pp]);
+          const float2 bpsi2 = __fmul2_rn(bx2, __fmul2_rn(__ffma2_rn(z2, q2, make_float2(nd[n], nd[n + 1])),
+                                                          __fmul2_rn(iA2[pp], iA2[pp])));
+          dA2[pp] = __ffma2_rn(L, __ffma2_rn(__fmul2_rn(dt2, r2), hp2, bpsi2), dA2[pp]);
+          const float2 rb = __fmul2_rn(__fmul2_rn(L, x2), qa2);  // dB_{t,n} part
+          red[n] = rb.x;
+          red[n + 1] = rb.y;
+          lam2[pp] = __fmul2_rn(L, r2);
+          h[n] = hp[n];
+          h[n + 1] = hp[n + 1];
         }
+        du += du2.x + du2.y;
+        ddt = ddt2.x + ddt2.y;
       } else {
+        float q[NS];
         decays<NS, STRUCT>(dt, An, q);
-      }
-      const float r0 = 1.0f + q0, zq0 = dt * An[0] * q0;
-      float dn = d0;
-      float red[32];
 #pragma unroll
-      for (int n = 0; n < NS; ++n) {
-        const float r = 1.0f + q[n];
-        const float bx = bv[n] * x;
-        const float qa = q[n] * iA[n];
-        red[NS + n] = gy * h[n];                      // dC_{t,n} part: dy_t h_t
-        lam[n] = fmaf(cv[n], gy, lam[n]);
-        du = fmaf(lam[n], qa * bv[n], du);
-        ddt = fmaf(lam[n] * r, fmaf(An[n], hp[n], bx), ddt);
-        // d h_t / d A_n = Delta r h_{t-1} + B x Delta^2 psi(Delta A_n)
-        float bpsi;
-        if constexpr (STRUCT) {
-          if (n > 0) dn = fmaf(r0, dn, fmaf((float)n, zq0, d0));
-          bpsi = bx * fmaf(dt * An[n], q[n], -dn) * (iA[n] * iA[n]);
-        } else {
-          bpsi = bx * (dt * dt) * psi_f(dt * An[n], q[n]);
+        for (int n = 0; n < NS; ++n) {
+          const float r = 1.0f + q[n];
+          const float bx = bv[n] * x;
+          const float qa = q[n] * IA(n);
+          red[NS + n] = gy * h[n];                      // dC_{t,n} part: dy_t h_t
+          LAM(n) = fmaf(cv[n], gy, LAM(n));
+          du = fmaf(LAM(n), qa * bv[n], du);
+          ddt = fmaf(LAM(n) * r, fmaf(An[n], hp[n], bx), ddt);
+          // d h_t / d A_n = Delta r h_{t-1} + B x Delta^2 psi(Delta A_n)
+          const float bpsi = bx * (dt * dt) * psi_f(dt * An[n], q[n]);
+          DA(n) = fmaf(LAM(n), fmaf(dt * r, hp[n], bpsi), DA(n));
+          red[n] = LAM(n) * x * qa;                     // dB_{t,n} part
+          LAM(n) *= r;
+          h[n] = hp[n];
         }
-        dA[n] = fmaf(lam[n], fmaf(dt * r, hp[n], bpsi), dA[n]);
-        red[n] = lam[n] * x * qa;                     // dB_{t,n} part
-        lam[n] *= r;
-        h[n] = hp[n];
       }
 #pragma unroll
       for (int n = 2 * NS; n < 32; ++n) red[n] = 0.0f;
@@ -534,11 +572,11 @@ __device__ __forceinline__ void bwd_item(const BwdArgs<TIO>& a, int j, int64_t s
   }
   if (active) {
 #pragma unroll
-    for (int n = 0; n < NS; ++n) atomicAdd(a.dA + d * NS + n, dA[n]);
+    for (int n = 0; n < NS; ++n) atomicAdd(a.dA + d * NS + n, DA(n));
     if (a.dD) atomicAdd(a.dD + d, dD);
     if (a.dh0 && j == 0) {
 #pragma unroll
-      for (int n = 0; n < NS; ++n) a.dh0[(b * a.channels + d) * NS + n] = lam[n];
+      for (int n = 0; n < NS; ++n) a.dh0[(b * a.channels + d) * NS + n] = LAM(n);
     }
   }
 }
