@@ -74,8 +74,11 @@ struct ComplexArgs {
   int async;                    // u, delta, y, B and C rows come in 16-byte pieces (cp.async staging)
 };
 
+#ifndef MAMBA_CPLX_LANES
+#define MAMBA_CPLX_LANES 2  // lanes per channel from 8 states on (1 or 2)
+#endif
 template <int N>
-__host__ __device__ constexpr int cplx_lanes_per_channel() { return N >= 8 ? 2 : 1; }
+__host__ __device__ constexpr int cplx_lanes_per_channel() { return N >= 8 ? MAMBA_CPLX_LANES : 1; }
 template <int N>
 __host__ __device__ constexpr int cplx_channels_per_warp() { return 32 / cplx_lanes_per_channel<N>(); }
 

@@ -222,7 +222,7 @@ ssd_chunk_kernel(const SsdArgs a) {
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L::kTslot);
   if (tid == 0) {
     mbar_init(bar_g, 1);
-    mbar_init(bar_y, 1);
+    mbar_init(bar_y, 2);  // one commit from each of the two issuing threads
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -481,9 +481,10 @@ ssd_chunk_kernel(const SsdArgs a) {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (tid == 0 && ok_run) {
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
+    // two issuing threads in different warps, one per column half
+    if ((tid == 0 || tid == 32) && ok_run) {
+      {
+        const int hh = tid >> 5;
         if (!AGG) {
           // Y half hh (channels 32 hh ..): M X then + C~ S_in
           const uint32_t dy = tmem + hh * d_off + kColY;
@@ -501,7 +502,7 @@ ssd_chunk_kernel(const SsdArgs a) {
                     k > 2 * hh);
       }
       umma_commit(bar_y);
-      if (!AGG && c + 1 < nchunks) issue_g((c + 1) % L::kStages);
+      if (tid == 0 && !AGG && c + 1 < nchunks) issue_g((c + 1) % L::kStages);
     }
 
     if (ok_run) {
