@@ -310,9 +310,12 @@ int mamba_selective_scan_backward(const void *u, const void *delta, const float 
  *
  * supers: super-chunks per (batch row, head) run in parallel (0 = chosen
  * from the shape and the device; a forced value is clamped to the chunk
- * count).  With more than one, a first kernel computes each super-chunk's
- * end state from zero (stream-ordered scratch of 4 (64 nstate + 1) bytes per
- * super-chunk) and the main kernel folds them in.
+ * count).  With more than one, every super-chunk runs from zero (the first
+ * from initial_state) and records its end state (stream-ordered scratch of
+ * 4 (64 nstate + 1) bytes per super-chunk and head); a second kernel adds
+ * the entering states' effect to y while their decay is at least 2^-32
+ * (the terms left out are below 2^-32 of their size) and writes
+ * final_state.
  *
  * Supported: dtype MAMBA_BF16, headdim 64, nstate 16, 32 or 64, flags 0 or
  * MAMBA_SCAN_EULER (MAMBA_SCAN_GENERAL_A is accepted and has no effect: A

@@ -616,9 +616,8 @@ __global__ void expire_wait_kernel(uint64_t limit_ns) {
 // --- Mamba-2's restricted scan (ssd.cuh) ------------------------------------
 // Super-chunks per sequence (a CTA's unit): one when the sequences fill at
 // least half of the resident CTA slots, else enough for two waves of slots
-// (each super-chunk but the last costs an extra, state-only pass over its
-// x and B, but a CTA walks its chunks in order, so parallelism wins for
-// long sequences).
+// (a CTA walks its chunks in order, so parallelism wins for long sequences;
+// each super-chunk after the first adds a correction walk of a few chunks).
 int64_t ssd_supers(int64_t seqs, int64_t chunks, int64_t slots, int64_t requested) {
   int64_t s = requested > 0 ? requested
                             : (seqs * 2 >= slots ? 1 : std::max<int64_t>(1, (2 * slots + seqs - 1) / seqs));
@@ -628,10 +627,8 @@ int64_t ssd_supers(int64_t seqs, int64_t chunks, int64_t slots, int64_t requeste
 template <int N>
 int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream) {
   using L = SsdSmem<N>;
-  auto main_k = ssd_chunk_kernel<N, false>;
-  auto agg_k = ssd_chunk_kernel<N, true>;
-  if (cudaFuncSetAttribute(main_k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(agg_k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
+  auto main_k = ssd_chunk_kernel<N>;
+  if (cudaFuncSetAttribute(main_k, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes) != cudaSuccess)
     return MAMBA_ERR_CUDA;
   int sms = 0, per_sm = 0;
   if (current_sms(&sms) != MAMBA_OK) return MAMBA_ERR_CUDA;
@@ -650,21 +647,20 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
   a.supers = (int)S;
   if (seqs * S >= (int64_t(1) << 31)) return MAMBA_ERR_UNSUPPORTED;
   unsigned char* mem = nullptr;
-  if (S > 1) {
-    const size_t n_agg = (size_t)(batch * a.heads) * (size_t)(S - 1);
+  if (S > 1) {  // every super-chunk's end state from zero and its decay
+    const size_t n_agg = (size_t)seqs * (size_t)S;
     const size_t st_bytes = n_agg * kSsdP * N * sizeof(float);
     if (scratch_alloc(reinterpret_cast<void**>(&mem), st_bytes + n_agg * sizeof(float), stream) != cudaSuccess)
       return MAMBA_ERR_CUDA;
     a.agg_state = reinterpret_cast<float*>(mem);
     a.agg_decay = reinterpret_cast<float*>(mem + st_bytes);
-    if (launch_pdl(agg_k, dim3((unsigned)(seqs * (S - 1))), dim3(kSsdWarps * 32), L::kBytes, stream, a) !=
-        cudaSuccess) {
-      cudaFreeAsync(mem, stream);
-      return MAMBA_ERR_CUDA;
-    }
   }
   int st = MAMBA_OK;
   if (launch_pdl(main_k, dim3((unsigned)(seqs * S)), dim3(kSsdWarps * 32), L::kBytes, stream, a) != cudaSuccess)
+    st = MAMBA_ERR_CUDA;
+  // the states entering super-chunks 1..S-1, their effect on y, the final state
+  if (st == MAMBA_OK && S > 1 &&
+      launch_pdl(ssd_fix_kernel<N>, dim3((unsigned)(seqs * (S - 1))), dim3(128), 0, stream, a) != cudaSuccess)
     st = MAMBA_ERR_CUDA;
   if (mem && cudaFreeAsync(mem, stream) != cudaSuccess && st == MAMBA_OK) st = MAMBA_ERR_CUDA;
   return st;

@@ -38,10 +38,13 @@
 // so four CTAs share an SM and their chunk pipelines overlap.
 //
 // Long sequences with few (batch row, head) pairs are cut into
-// super-chunks: an aggregate kernel (the same kernel, state only) runs each
-// super-chunk but the last from a zero state and records its end state and
-// total decay; the main kernel folds the aggregates of the earlier
-// super-chunks into its entering state.
+// super-chunks that run side by side, each from a zero state (the first
+// from the initial state); each records its end state H_j and its total
+// decay.  A correction kernel then composes the state entering super-chunk
+// j, S_in(j) = e^{a sum_{j-1}} S_in(j-1) + H_{j-1} (the scan's monoid with a
+// scalar decay), adds its effect e^{a cum_t} C_t . S_in(j) to the outputs
+// while that decay is at least 2^-32 (the terms left out are 256 times
+// under the fp32 rounding of y), and writes the final state.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -66,8 +69,8 @@ struct SsdArgs {
   const float* h0;              // (batch, heads*64, N) or null
   __nv_bfloat16* y;             // (batch, len, heads*64)
   float* final_state;           // (batch, heads*64, N) or null
-  float* agg_state;             // (batch*heads, supers-1, 64, N): super-chunk end state from zero
-  float* agg_decay;             // (batch*heads, supers-1): log2 of its total decay
+  float* agg_state;             // (batch*heads, supers, 64, N): super-chunk end state from zero
+  float* agg_decay;             // (batch*heads, supers): log2 of its total decay
   int64_t len;
   int heads;
   int supers;                   // super-chunks per (batch row, head)
@@ -190,7 +193,7 @@ struct SsdSmem {
   static constexpr int kSboBC = (N / 8) * 128;           // K-major [rows][N]
 };
 
-template <int N, bool AGG>
+template <int N>
 __global__ void __launch_bounds__(kSsdWarps * 32)
 ssd_chunk_kernel(const SsdArgs a) {
   using L = SsdSmem<N>;
@@ -206,9 +209,8 @@ ssd_chunk_kernel(const SsdArgs a) {
   const int row = 16 * warp + (lane & 15);  // its row (token) or channel
   const int64_t channels = (int64_t)a.heads * kSsdP;
 
-  // job: (batch row, head, super-chunk); the aggregate kernel has one
-  // super-chunk fewer per head
-  const int per_seq = AGG ? a.supers - 1 : a.supers;
+  // job: (batch row, head, super-chunk)
+  const int per_seq = a.supers;
   const int64_t seq = blockIdx.x / per_seq;  // batch row * heads + head
   const int j = (int)(blockIdx.x % per_seq);
   const int64_t b = seq / a.heads;
@@ -261,7 +263,7 @@ ssd_chunk_kernel(const SsdArgs a) {
       const bool ok = t0 + t < t_end;
       const uint32_t off = (t >> 3) * L::kSboBC + n8 * 128 + (t & 7) * 16;
       cp_async16(sb + off, ok ? (const void*)(Bg + (t0 + t) * N + n8 * 8) : (const void*)a.B, ok);
-      if (!AGG) cp_async16(sb + L::kBC + off, ok ? (const void*)(Cg + (t0 + t) * N + n8 * 8) : (const void*)a.C, ok);
+      cp_async16(sb + L::kBC + off, ok ? (const void*)(Cg + (t0 + t) * N + n8 * 8) : (const void*)a.C, ok);
     }
   };
   // this thread's (token, head) step as raw bf16 bits (0 for padding tokens:
@@ -279,20 +281,9 @@ ssd_chunk_kernel(const SsdArgs a) {
 #pragma unroll
   for (int n = 0; n < NH; ++n) S[n] = 0.0f;
   const int64_t sidx = ((b * a.heads + h) * kSsdP + row) * N + ch * NH;  // (batch, channel, n) offset
-  if (!AGG) {
-    if (a.h0) {
+  if (a.h0 && j == 0) {  // later super-chunks run from zero (the correction kernel adds their carry)
 #pragma unroll
-      for (int n = 0; n < NH; ++n) S[n] = __ldg(a.h0 + sidx + n);
-    }
-    // fold in the super-chunks before this one
-    const int64_t aseq = b * a.heads + h;
-    for (int k = 0; k < j; ++k) {
-      const int64_t agg = aseq * (a.supers - 1) + k;
-      const float dec = exp2f(__ldg(a.agg_decay + agg));
-      const float* as = a.agg_state + (agg * kSsdP + row) * N + ch * NH;
-#pragma unroll
-      for (int n = 0; n < NH; ++n) S[n] = fmaf(dec, S[n], __ldg(as + n));
-    }
+    for (int n = 0; n < NH; ++n) S[n] = __ldg(a.h0 + sidx + n);
   }
   // bf16 copy of the state (K-major [channel][n]) for the next chunk's C~ S_in
   auto store_state_copy = [&]() {
@@ -307,7 +298,7 @@ ssd_chunk_kernel(const SsdArgs a) {
       *reinterpret_cast<uint4*>(st + (ch * (NH / 8) + q) * 128) = v;
     }
   };
-  if (!AGG) store_state_copy();
+  store_state_copy();
 
   float* Ds = reinterpret_cast<float*>(smem + L::kDs);  // [64] D of the head (0 without D)
   if (ch == 0) Ds[row] = a.D ? __ldg(a.D + (int64_t)h * kSsdP + row) : 0.0f;
@@ -357,7 +348,7 @@ ssd_chunk_kernel(const SsdArgs a) {
   cp_async_wait<L::kStages - 1>();  // chunk 0
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
-  if (!AGG && tid == 0 && nchunks > 0) issue_g(0);
+  if (tid == 0 && nchunks > 0) issue_g(0);
   uint32_t dt_raw = load_dt(0);
   bool ok_run = true;
 
@@ -419,12 +410,12 @@ ssd_chunk_kernel(const SsdArgs a) {
       for (int q = 0; q < N / 16; ++q) {
         const int n8 = ch * (N / 16) + q;
         scaled(smem + ob + roff + n8 * 128, smem + L::kBw + roff + n8 * 128, fB);
-        if (!AGG) scaled(smem + oc + roff + n8 * 128, smem + L::kCt + roff + n8 * 128, fC);
+        scaled(smem + oc + roff + n8 * 128, smem + L::kCt + roff + n8 * 128, fC);
       }
     }
     __syncthreads();  // cum and w of the chunk are in shared memory
 
-    if (!AGG) {
+    {
       // M row `row`, columns s = 32 ch .. 32 ch + 31, from G: causal mask,
       // decay and input weight
       bool got = mbar_wait_bounded(bar_g, (uint32_t)(c & 1), a.wait_limit_ns);
@@ -485,7 +476,7 @@ ssd_chunk_kernel(const SsdArgs a) {
     if ((tid == 0 || tid == 32) && ok_run) {
       {
         const int hh = tid >> 5;
-        if (!AGG) {
+        {
           // Y half hh (channels 32 hh ..): M X then + C~ S_in
           const uint32_t dy = tmem + hh * d_off + kColY;
 #pragma unroll
@@ -502,7 +493,7 @@ ssd_chunk_kernel(const SsdArgs a) {
                     k > 2 * hh);
       }
       umma_commit(bar_y);
-      if (tid == 0 && !AGG && c + 1 < nchunks) issue_g((c + 1) % L::kStages);
+      if (tid == 0 && c + 1 < nchunks) issue_g((c + 1) % L::kStages);
     }
 
     if (ok_run) {
@@ -520,7 +511,7 @@ ssd_chunk_kernel(const SsdArgs a) {
       float yv[32], ds[N];
       {
         uint32_t ry[2][16], rs[N / 16][16];
-        if (!AGG) {
+        {
           tmem_ld16_nowait(t_lane + kColY, ry[0]);
           tmem_ld16_nowait(t_lane + kColY + 16, ry[1]);
         }
@@ -529,15 +520,15 @@ ssd_chunk_kernel(const SsdArgs a) {
         tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          yv[i] = AGG ? 0.0f : __uint_as_float(ry[0][i]);
-          yv[16 + i] = AGG ? 0.0f : __uint_as_float(ry[1][i]);
+          yv[i] = __uint_as_float(ry[0][i]);
+          yv[16 + i] = __uint_as_float(ry[1][i]);
         }
 #pragma unroll
         for (int q = 0; q < N / 16; ++q)
 #pragma unroll
           for (int i = 0; i < 16; ++i) ds[16 * q + i] = __uint_as_float(rs[q][i]);
       }
-      if (!AGG) {
+      {
         // y = Y + D x for row `row`, channels 32 ch .. 32 ch + 31 -> bf16 ->
         // 16-byte stores
         const float* Dh = Ds + 32 * ch;
@@ -571,7 +562,7 @@ ssd_chunk_kernel(const SsdArgs a) {
         const float give = ch ? ds[i] : ds[NH + i];
         S[i] = fmaf(dec, S[i], keep + __shfl_xor_sync(0xffffffffu, give, 16));
       }
-      if (!AGG) store_state_copy();
+      store_state_copy();
     }
     tc_fence_before();
     ok_run = __syncthreads_and(ok_run) != 0;  // slot c is read; every read of Y / dS is done
@@ -584,13 +575,13 @@ ssd_chunk_kernel(const SsdArgs a) {
 
   griddep_launch_dependents();
   if (ok_run) {
-    if (AGG) {
-      const int64_t agg = (b * a.heads + h) * (a.supers - 1) + j;
+    if (a.supers > 1) {  // the end state from zero and the total decay, for the correction kernel
+      const int64_t agg = (b * a.heads + h) * a.supers + j;
       float* as = a.agg_state + (agg * kSsdP + row) * N + ch * NH;
 #pragma unroll
       for (int n = 0; n < NH; ++n) as[n] = S[n];
       if (tid == 0) a.agg_decay[agg] = total_log2;
-    } else if (a.final_state && j == a.supers - 1) {
+    } else if (a.final_state) {
 #pragma unroll
       for (int n = 0; n < NH; ++n) a.final_state[sidx + n] = S[n];
     }
@@ -600,6 +591,111 @@ ssd_chunk_kernel(const SsdArgs a) {
   tc_fence_after();
   if (warp == 0)
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "n"(kSsdTmemCols) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Correction of super-chunks 1..S-1 (one CTA of 128 threads per (batch row,
+// head, super-chunk j >= 1)).  Thread (p, half) owns channel p of the head
+// and half of each chunk's tokens.  It composes the state entering j from
+// the end states and decays the main kernel recorded,
+//     S_in = 0;  S_in <- e^{a sum_k} S_in + H_k   for k = 0 .. j-1,
+// (H_0 carries the initial state), then walks j's chunks while the carried
+// decay e^{a cum} is at least 2^-kSsdFixStopLog2 and adds
+//     y_t[p] += e^{a cum_t} sum_n C_t[n] S_in[p][n]
+// (cum_t: the sum of dt from the super-chunk's start through t).  The last
+// super-chunk's CTA writes the final state e^{a sum_{S-1}} S_in + H_{S-1}.
+// ---------------------------------------------------------------------------
+constexpr float kSsdFixStopLog2 = 32.0f;
+
+template <int N>
+__global__ void __launch_bounds__(128)
+ssd_fix_kernel(const SsdArgs a) {
+  __shared__ float s_cum[kSsdQ];      // a cum_t in log2 units
+  __shared__ float s_wsum[4];
+  __shared__ float s_C[kSsdQ * N];    // the chunk's C rows, fp32
+  griddep_wait();  // the main kernel's outputs, end states and decays
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int p = 32 * (warp & 1) + lane;  // channel of the head (consecutive lanes: consecutive channels)
+  const int half = warp >> 1;            // tokens half * 32 .. of a chunk
+  const int per = a.supers - 1;
+  const int64_t seq = blockIdx.x / per;  // batch row * heads + head
+  const int j = 1 + (int)(blockIdx.x % per);
+  const int64_t b = seq / a.heads;
+  const int h = (int)(seq % a.heads);
+  const int64_t channels = (int64_t)a.heads * kSsdP;
+  const float a2 = __ldg(a.A + h) * 1.4426950408889634f;
+
+  // the entering state of channel p
+  float Sin[N];
+#pragma unroll
+  for (int n = 0; n < N; ++n) Sin[n] = 0.0f;
+  for (int k = 0; k < j; ++k) {
+    const int64_t agg = seq * a.supers + k;
+    const float dec = exp2f(__ldcg(a.agg_decay + agg));
+    const float4* H = reinterpret_cast<const float4*>(a.agg_state + (agg * kSsdP + p) * N);
+#pragma unroll
+    for (int q = 0; q < N / 4; ++q) {
+      const float4 v = __ldcg(H + q);
+      Sin[4 * q] = fmaf(dec, Sin[4 * q], v.x);
+      Sin[4 * q + 1] = fmaf(dec, Sin[4 * q + 1], v.y);
+      Sin[4 * q + 2] = fmaf(dec, Sin[4 * q + 2], v.z);
+      Sin[4 * q + 3] = fmaf(dec, Sin[4 * q + 3], v.w);
+    }
+  }
+  if (j == a.supers - 1 && a.final_state && half == 0) {
+    const int64_t agg = seq * a.supers + j;
+    const float dec = exp2f(__ldcg(a.agg_decay + agg));
+    const float* H = a.agg_state + (agg * kSsdP + p) * N;
+    float* dst = a.final_state + ((b * a.heads + h) * kSsdP + p) * N;
+#pragma unroll
+    for (int n = 0; n < N; ++n) dst[n] = fmaf(dec, Sin[n], __ldcg(H + n));
+  }
+
+  const int64_t t_begin = (int64_t)j * a.super_len;
+  const int64_t t_end = t_begin + a.super_len < a.len ? t_begin + a.super_len : a.len;
+  const unsigned short* dtg = reinterpret_cast<const unsigned short*>(a.dt) + (b * a.len) * a.heads + h;
+  const __nv_bfloat16* Cg = a.C + (b * a.len) * N;
+  __nv_bfloat16* yg = a.y + (b * a.len) * channels + (int64_t)h * kSsdP + p;
+  float carry = 0.0f;  // a cum at the chunk's start, log2 units
+  for (int64_t t0 = t_begin; t0 < t_end && carry >= -kSsdFixStopLog2; t0 += kSsdQ) {
+    const int nt = t_end - t0 < kSsdQ ? (int)(t_end - t0) : kSsdQ;
+    __syncthreads();  // the previous chunk's rows are no longer read
+    // the chunk's running decay (threads 0..63, one token each) and C rows
+    if (tid < kSsdQ) {
+      float v = tid < nt ? __uint_as_float((uint32_t)__ldg(dtg + (t0 + tid) * a.heads) << 16) * a2 : 0.0f;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float nb = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += nb;
+      }
+      if (lane == 31) s_wsum[warp] = v;
+      s_cum[tid] = v;
+    }
+    for (int i = tid; i < kSsdQ * N; i += 128) {
+      const int t = i / N;
+      s_C[i] = t < nt ? __bfloat162float(Cg[(t0 + t) * N + (i - t * N)]) : 0.0f;
+    }
+    __syncthreads();
+    const float w0 = s_wsum[0];
+    // the 32 outputs of this thread's half of the chunk: loads all issued
+    // first, then the arithmetic, then the stores
+    float yv[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      const int t = 32 * half + r;
+      yv[r] = t < nt ? __bfloat162float(yg[(t0 + t) * channels]) : 0.0f;
+    }
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      const int t = 32 * half + r;
+      const float cum = carry + s_cum[t] + (half ? w0 : 0.0f);
+      float acc = 0.0f;
+#pragma unroll
+      for (int n = 0; n < N; ++n) acc = fmaf(s_C[t * N + n], Sin[n], acc);
+      if (t < nt) yg[(t0 + t) * channels] = __float2bfloat16_rn(yv[r] + ex2_approx(cum) * acc);
+    }
+    carry += w0 + (nt > 32 ? s_wsum[1] : 0.0f);
+  }
 }
 
 }  // namespace mamba
