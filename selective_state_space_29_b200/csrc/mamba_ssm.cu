@@ -125,6 +125,24 @@ bool make_map_2d(CUtensorMap* m, const void* base, int dtype, uint64_t cols, uin
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 5-D map that lands a [64 tokens][8 g] tile of a bf16 [batch][len][row]
+// array in the tensor core's no-swizzle core-matrix layout: dimensions
+// (8 elements, token % 8, row / 8, token / 8, batch row), box (8, 8, g, 8, 1)
+// walked innermost first, so the tile's byte offset of (token t, element e)
+// is (t/8) (128 g) + (e/8) 128 + (t%8) 16 + (e%8) 2.  Needs len % 8 == 0 (the
+// token split stays inside a batch row) and row % 8 == 0.
+bool make_map_core_tiles(CUtensorMap* m, const void* base, uint64_t row, uint64_t len, uint64_t batch, uint32_t g) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || row % 8 != 0 || len % 8 != 0 || len < 64) return false;
+  const cuuint64_t dims[5] = {8, 8, row / 8, len / 8, batch};
+  const cuuint64_t strides[4] = {row * 2, 16, 8 * row * 2, len * row * 2};
+  const cuuint32_t box[5] = {8, 8, g, 8, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // --- scan configuration per element type and state count -------------------
 // A CTA is kScanConsumers consumer warps (one per SM sub-partition) and one
 // producer warp; a consumer's ring holds kStages tiles of kTile tokens (the
@@ -655,8 +673,20 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
     a.agg_state = reinterpret_cast<float*>(mem);
     a.agg_decay = reinterpret_cast<float*>(mem + st_bytes);
   }
+  // x, B and C tiles by TMA when the maps can be made (else cp.async)
+  CUtensorMap mx, mb, mc;
+  std::memset(&mx, 0, sizeof(mx));
+  std::memset(&mb, 0, sizeof(mb));
+  std::memset(&mc, 0, sizeof(mc));
+  const uint64_t channels = (uint64_t)a.heads * kSsdP;
+  a.tma = (make_map_core_tiles(&mx, a.x, channels, (uint64_t)a.len, (uint64_t)batch, 8) &&
+           make_map_core_tiles(&mb, a.B, N, (uint64_t)a.len, (uint64_t)batch, N / 8) &&
+           make_map_core_tiles(&mc, a.C, N, (uint64_t)a.len, (uint64_t)batch, N / 8))
+              ? 1
+              : 0;
   int st = MAMBA_OK;
-  if (launch_pdl(main_k, dim3((unsigned)(seqs * S)), dim3(kSsdWarps * 32), L::kBytes, stream, a) != cudaSuccess)
+  if (launch_pdl(main_k, dim3((unsigned)(seqs * S)), dim3(kSsdWarps * 32), L::kBytes, stream, a, mx, mb, mc) !=
+      cudaSuccess)
     st = MAMBA_ERR_CUDA;
   // the states entering super-chunks 1..S-1, their effect on y, the final state
   if (st == MAMBA_OK && S > 1 &&

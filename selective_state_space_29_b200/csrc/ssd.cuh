@@ -76,6 +76,7 @@ struct SsdArgs {
   int supers;                   // super-chunks per (batch row, head)
   int64_t super_len;            // tokens per super-chunk, a multiple of 64
   int euler;                    // input weight dt (exponential Euler) instead of the ZOH weight
+  int tma;                      // x, B, C tiles by TMA (5-D core-matrix maps) instead of cp.async
   uint64_t wait_limit_ns;
 };
 
@@ -187,15 +188,16 @@ struct SsdSmem {
   static constexpr int kCum = kS + kSsdP * N * 2;        // [64] cum (log2), [64] w, [64] u
   static constexpr int kWsum = kCum + 3 * kSsdQ * 4;     // [4 warps] partial sums
   static constexpr int kDs = kWsum + 16;                 // [64] D
-  static constexpr int kBar = kDs + kSsdP * 4;           // 2 mbarriers
-  static constexpr int kTslot = kBar + 16;
+  static constexpr int kBar = kDs + kSsdP * 4;           // mbarriers: G, Y, then one per ring slot (TMA)
+  static constexpr int kTslot = kBar + 8 * (2 + kStages);
   static constexpr int kBytes = kTslot + 16 + 1024;      // + room to align the base to 1024
   static constexpr int kSboBC = (N / 8) * 128;           // K-major [rows][N]
 };
 
 template <int N>
 __global__ void __launch_bounds__(kSsdWarps * 32)
-ssd_chunk_kernel(const SsdArgs a) {
+ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mb,
+                 const __grid_constant__ CUtensorMap mc) {
   using L = SsdSmem<N>;
   static_assert(N % 16 == 0 && N <= 64, "states in steps of 16, at most 64 (tensor-memory columns)");
   constexpr int NH = N / 2;                 // states per thread
@@ -221,10 +223,12 @@ ssd_chunk_kernel(const SsdArgs a) {
 
   uint64_t* bar_g = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* bar_y = bar_g + 1;
+  uint64_t* bar_full = bar_g + 2;  // [kStages]: the slot's TMA tiles have landed
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L::kTslot);
   if (tid == 0) {
     mbar_init(bar_g, 1);
     mbar_init(bar_y, 2);  // one commit from each of the two issuing threads
+    for (int s2 = 0; s2 < L::kStages; ++s2) mbar_init(bar_full + s2, 1);
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -248,6 +252,16 @@ ssd_chunk_kernel(const SsdArgs a) {
   // one wavefront), while a warp reads 8 token rows, whole 32-byte sectors.
   auto load_chunk = [&](int c, int slot) {
     const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
+    if (a.tma) {  // one thread, three tiles, completion on the slot's barrier
+      if (tid == 0) {
+        unsigned char* dx = smem + slot * L::kStage;
+        mbar_arrive_expect_tx(bar_full + slot, (uint32_t)(L::kX + 2 * L::kBC));
+        tma_load_5d(dx, &mx, bar_full + slot, 0, 0, 8 * h, (int)(t0 / 8), (int)b);
+        tma_load_5d(dx + L::kX, &mb, bar_full + slot, 0, 0, 0, (int)(t0 / 8), (int)b);
+        tma_load_5d(dx + L::kX + L::kBC, &mc, bar_full + slot, 0, 0, 0, (int)(t0 / 8), (int)b);
+      }
+      return;
+    }
     const uint32_t sx = sbase + slot * L::kStage;
 #pragma unroll
     for (int i = tid; i < kSsdQ * 8; i += kSsdWarps * 32) {
@@ -348,9 +362,28 @@ ssd_chunk_kernel(const SsdArgs a) {
   cp_async_wait<L::kStages - 1>();  // chunk 0
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
-  if (tid == 0 && nchunks > 0) issue_g(0);
-  uint32_t dt_raw = load_dt(0);
+  // TMA: the tiles of chunk k have landed (bounded wait on the slot's
+  // barrier).  Thread 0 counts the chunks it issued and the highest one it
+  // saw land, so that it can drain the copies still in flight if the CTA
+  // leaves early.
+  int n_issued = nchunks < L::kStages ? nchunks : L::kStages, n_landed = 0;
+  auto tiles_ready = [&](int k) -> bool {
+    if (!a.tma) return true;
+    const bool ok = mbar_wait_bounded(bar_full + k % L::kStages, (uint32_t)((k / L::kStages) & 1), a.wait_limit_ns);
+    if (ok && k + 1 > n_landed) n_landed = k + 1;
+    return ok;
+  };
   bool ok_run = true;
+  if (tid == 0 && nchunks > 0) {
+    if (tiles_ready(0)) {
+      issue_g(0);
+    } else {
+      record_device_error(MAMBA_ERR_TIMEOUT);
+      ok_run = false;
+    }
+  }
+  ok_run = __syncthreads_and(ok_run) != 0;
+  uint32_t dt_raw = load_dt(0);
 
   for (int c = 0; c < nchunks && ok_run; ++c) {
     const int slot = c % L::kStages;
@@ -372,7 +405,9 @@ ssd_chunk_kernel(const SsdArgs a) {
     }
     if (lane == 15) wsum[warp] = v;
     const float wgt = a.euler ? dt : expm1f(dt * a_h) / a_h;
-    __syncthreads();  // the warp sums
+    bool landed = tiles_ready(c);  // (TMA) the chunk's tiles are in its slot
+    if (!landed && tid == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+    ok_run = __syncthreads_and(ok_run && landed) != 0;  // the warp sums, and the vote
     float pre = 0.0f;
     for (int w2 = 0; w2 < warp; ++w2) pre += wsum[w2];
     const float cum = v + pre;
@@ -493,7 +528,14 @@ ssd_chunk_kernel(const SsdArgs a) {
                     k > 2 * hh);
       }
       umma_commit(bar_y);
-      if (tid == 0 && c + 1 < nchunks) issue_g((c + 1) % L::kStages);
+      if (tid == 0 && c + 1 < nchunks) {
+        if (tiles_ready(c + 1)) {
+          issue_g((c + 1) % L::kStages);
+        } else {
+          record_device_error(MAMBA_ERR_TIMEOUT);
+          ok_run = false;
+        }
+      }
     }
 
     if (ok_run) {
@@ -566,12 +608,19 @@ ssd_chunk_kernel(const SsdArgs a) {
     }
     tc_fence_before();
     ok_run = __syncthreads_and(ok_run) != 0;  // slot c is read; every read of Y / dS is done
-    // chunk c + kStages into the slot chunk c used
-    if (c + L::kStages < nchunks) load_chunk(c + L::kStages, slot);
+    // chunk c + kStages into the slot chunk c used (its reads, and the
+    // products that read it, are complete)
+    if (a.tma && tid == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (ok_run && c + L::kStages < nchunks) {
+      load_chunk(c + L::kStages, slot);
+      n_issued = c + L::kStages + 1;
+    }
     cp_async_commit();
     dt_raw = ndt_raw;
   }
   cp_async_wait<0>();
+  if (a.tma && tid == 0)  // (only after a timeout) copies issued but never seen to land
+    for (int k = n_landed; k < n_issued; ++k) tiles_ready(k);
 
   griddep_launch_dependents();
   if (ok_run) {
