@@ -355,15 +355,31 @@ complex_scan_kernel(const ComplexArgs a) {
       gi2[p] = make_float2(giv[0], giv[1]);
     }
     // One token.  The decays of the lane's states come from a product chain
-    // of pair steps from (E_n0, E_n0+1): E_0 = expm1(dt a), E_1 = E_0 + F +
-    // E_0 F, then E <- E + F2 + E F2; the second half of a channel's states
-    // starts from (E_0, E_1) stepped once by F_{N/2} (F_{2k} = F_k (2 + F_k)).
+    // of pair steps from (E_n0, E_n0+1): E_n0+1 = E_n0 + F + E_n0 F, then
+    // E <- E + F2 + E F2 (F2 = F (2 + F)).  The exponential's inputs per
+    // lane: (a, w/2) for the first lane of a channel, ((n0+1) a, n0 w/2) for
+    // the second.
+    const float xa = half ? (float)(n0 + 1) * sa : sa, xw = half ? (float)n0 * sw : sw;
     auto token = [&](int k, const TIO* u0, const TIO* dt0) {
       const float x = to_f32(u0[k * CPW + cl]);
       const float dt = to_f32(dt0[k * CPW + cl]);
       if (AGG) sd_total += (double)dt;
+      // one complex exponential per lane: the first lane of a channel takes
+      // F = exp(dt (a + i w)) - 1 (and m = expm1(dt a) = E_0), the second
+      // E_{n0} = exp(dt A_{n0}) - 1 directly (A_{n0} = (n0+1) a + i n0 w) and
+      // F from its partner
       float fr, fi, m;
-      expm1_complex(dt * sa, dt * sw, &fr, &fi, &m);
+      expm1_complex(dt * xa, dt * xw, &fr, &fi, &m);
+      float e1r = m, e1i = 0.0f;  // the lane's first state's E
+      if constexpr (LPC == 2) {
+        const float pr = __shfl_xor_sync(0xffffffffu, fr, 1), pi = __shfl_xor_sync(0xffffffffu, fi, 1);
+        if (half) {
+          e1r = fr;
+          e1i = fi;
+          fr = pr;
+          fi = pi;
+        }
+      }
       const float f2r = fmaf(fr, 2.0f + fr, -fi * fi);
       const float f2i = fi * fmaf(2.0f, fr, 2.0f);
       auto step = [](float2& er, float2& ei, float2 gr, float2 gi, float2 ngi) {
@@ -372,22 +388,9 @@ complex_scan_kernel(const ComplexArgs a) {
         er = nr;
         ei = ni;
       };
-      float2 er = make_float2(m, fmaf(m, fr, m + fr));
-      float2 ei = make_float2(0.0f, fmaf(m, fi, fi));
-      if constexpr (LPC == 2) {
-        float hr_ = f2r, hi_ = f2i;  // F_{N/2} by squaring F2
-#pragma unroll
-        for (int q = 4; q <= N / 2; q *= 2) {
-          const float nr = fmaf(hr_, 2.0f + hr_, -hi_ * hi_);
-          hi_ = hi_ * fmaf(2.0f, hr_, 2.0f);
-          hr_ = nr;
-        }
-        if (!half) {  // first half: a step by 0 leaves (E_0, E_1)
-          hr_ = 0.0f;
-          hi_ = 0.0f;
-        }
-        step(er, ei, make_float2(hr_, hr_), make_float2(hi_, hi_), make_float2(-hi_, -hi_));
-      }
+      // (E_n0, E_n0+1), E_n0+1 = E_n0 + F + E_n0 F
+      float2 er = make_float2(e1r, e1r + fr + fmaf(e1r, fr, -e1i * fi));
+      float2 ei = make_float2(e1i, e1i + fi + fmaf(e1r, fi, e1i * fr));
       const float2 Fr = make_float2(f2r, f2r), Fi = make_float2(f2i, f2i), nFi = make_float2(-f2i, -f2i);
       const float2 x2 = make_float2(x, x);
       const float4* Bt = reinterpret_cast<const float4*>(sB + k * N + n0);

@@ -66,6 +66,10 @@ namespace mamba {
 #ifndef MAMBA_SCAN_PIPE
 #define MAMBA_SCAN_PIPE 0
 #endif
+#ifndef MAMBA_SCAN_UNROLL
+#define MAMBA_SCAN_UNROLL 4
+#endif
+constexpr int kScanUnroll = MAMBA_SCAN_UNROLL;  // token pairs per unrolled step of a full tile
 
 constexpr int kCPW = 32;   // channels per warp: one lane per channel
 constexpr int kFixSegTiles = 1;  // tiles per segment of the super-chunk correction
@@ -396,7 +400,7 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
       db = ndb;
     }
 #else
-#pragma unroll 4
+#pragma unroll kScanUnroll
     for (; r < TILE; r += 2) pair(r);
 #endif
   } else {
