@@ -428,7 +428,7 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
     const int64_t zero_words = (int64_t)((sl.ctr + sl.done + sl.fix_segs) / sizeof(int));
     const int64_t total_c = batch * len * R * NS;
     const int64_t chan_padded = (int64_t)pl.groups_d * kCPW;
-    const int64_t total = zero_words + total_c + chan_padded;
+    const int64_t total = zero_words + total_c / 4 + chan_padded;  // (four C and B elements per thread)
     if ((total + 255) / 256 > 0x7fffffff) return MAMBA_ERR_UNSUPPORTED;
     scan_prep_kernel<TIO, NS><<<(unsigned)((total + 255) / 256), 256, 0, stream>>>(
         counters, zero_words, static_cast<const TIO*>(C), cs, static_cast<const TIO*>(B), bs, total_c, A, D, chan,

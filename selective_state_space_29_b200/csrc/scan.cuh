@@ -1072,7 +1072,10 @@ scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__
 // before every walked tile gets exp(A_n cum) h_in[n] added.
 // ---------------------------------------------------------------------------
 constexpr int kFixWarps = 4;
-constexpr int kFixPhases = 32;
+#ifndef MAMBA_FIX_PHASES
+#define MAMBA_FIX_PHASES 32
+#endif
+constexpr int kFixPhases = MAMBA_FIX_PHASES;  // warps per stream of the correction (tiles w, w + phases, ...)
 
 template <typename TIO, int NS, int TILE, int R>
 __host__ __device__ constexpr int fix_stage_bytes() {  // one warp: Delta [TILE][32], y [TILE*R][32], C [TILE*R][NS]
@@ -1274,7 +1277,7 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
 // pre-pass, one thread per element of three ranges:
 //   [0, zero_words):          the job counters and progress flags = 0
 //   C' = C / (n+1) in fp32 for every (token row, state), and B widened to
-//   fp32 when bs is given (bf16 data)
+//   fp32 when bs is given (bf16 data): four consecutive states per thread
 //   per channel {A[d,0], 1/A[d,0], D[d], structured}, where "structured"
 //   means A[d,n] == (n+1) A[d,0] exactly for every n, A[d,0] < 0 and the
 //   general path was not forced; padding channels get {-1, -1, 0, 1}.
@@ -1293,13 +1296,18 @@ __global__ void scan_prep_kernel(int* __restrict__ zero, int64_t zero_words, con
     return;
   }
   i -= zero_words;
-  if (i < total_c) {
-    const int n = (int)(i % NS);
-    cs[i] = to_f32(C[i]) / (float)(n + 1);
-    if (bs) bs[i] = to_f32(B[i]);
+  const int64_t quads = total_c / 4;  // four consecutive elements of a row per thread (NS % 4 == 0)
+  if (i < quads) {
+    const int64_t e = 4 * i;
+    const int n = (int)(e % NS);
+    reinterpret_cast<float4*>(cs)[i] =
+        make_float4(to_f32(C[e]) / (float)(n + 1), to_f32(C[e + 1]) / (float)(n + 2),
+                    to_f32(C[e + 2]) / (float)(n + 3), to_f32(C[e + 3]) / (float)(n + 4));
+    if (bs)
+      reinterpret_cast<float4*>(bs)[i] = make_float4(to_f32(B[e]), to_f32(B[e + 1]), to_f32(B[e + 2]), to_f32(B[e + 3]));
     return;
   }
-  const int64_t d = i - total_c;
+  const int64_t d = i - quads;
   if (d >= chan_padded) return;
   if (d >= channels) {
     chan[d] = make_float4(-1.0f, -1.0f, 0.0f, 1.0f);
