@@ -650,7 +650,7 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
     return MAMBA_ERR_CUDA;
   int sms = 0, per_sm = 0;
   if (current_sms(&sms) != MAMBA_OK) return MAMBA_ERR_CUDA;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, main_k, kSsdWarps * 32, L::kBytes) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, main_k, kSsdThreads, L::kBytes) != cudaSuccess ||
       per_sm < 1)
     return MAMBA_ERR_CUDA;
   // tensor memory: kSsdTmemCols columns per CTA out of 512 per SM
@@ -685,7 +685,7 @@ int launch_ssd(SsdArgs a, int64_t batch, int64_t supers_req, cudaStream_t stream
               ? 1
               : 0;
   int st = MAMBA_OK;
-  if (launch_pdl(main_k, dim3((unsigned)(seqs * S)), dim3(kSsdWarps * 32), L::kBytes, stream, a, mx, mb, mc) !=
+  if (launch_pdl(main_k, dim3((unsigned)(seqs * S)), dim3(kSsdThreads), L::kBytes, stream, a, mx, mb, mc) !=
       cudaSuccess)
     st = MAMBA_ERR_CUDA;
   // the states entering super-chunks 1..S-1, their effect on y, the final state

@@ -13,10 +13,11 @@
 // the input weight of the discretisation: (e^{a dt} - 1)/a for the
 // zero-order hold, dt for exponential Euler.
 //
-// A CTA of four warps owns one head of one batch row over one super-chunk
-// and walks its chunks of 64 tokens in order.  Per chunk, all products are
-// tcgen05.mma (bf16 operands from shared memory, fp32 accumulators in
-// tensor memory), issued by one thread:
+// A CTA of four builder warps and one issuing warp owns one head of one
+// batch row over one super-chunk and walks its chunks of 64 tokens in order.
+// Per chunk, all products are tcgen05.mma (bf16 operands from shared memory,
+// fp32 accumulators in tensor memory), issued by one thread of the fifth
+// warp while the builders prepare the next chunk:
 //   G   = C B^T                     64 x 64, K = N
 //   Y   = M X + C~ S_in             64 x 64, K = 64 + N  (M = G o e^{a(cum_t - cum_s)} o w_s,
 //                                                         masked s > t; C~ = e^{a cum_t} C)
@@ -56,7 +57,8 @@ namespace mamba {
 
 constexpr int kSsdQ = 64;       // tokens per chunk
 constexpr int kSsdP = 64;       // channels per head
-constexpr int kSsdWarps = 4;    // one warpgroup per CTA
+constexpr int kSsdWarps = 4;    // builder warps (one warpgroup: one per tensor-memory sub-partition)
+constexpr int kSsdThreads = (kSsdWarps + 1) * 32;  // + one warp that issues the tensor-core products
 constexpr int kSsdTmemCols = 128;  // dS^T in columns [0, 64), Y in [64, 96), G in [96, 128)
 
 struct SsdArgs {
@@ -164,6 +166,31 @@ __device__ __forceinline__ void tmem_ldN(uint32_t taddr, float (&v)[N]) {
   }
 }
 
+// e^z - 1 for z <= 0 without a branch: the Taylor polynomial through z^6
+// for |z| <= 1/4 (truncation below 1.2e-8 relative), the hardware exp2
+// minus one otherwise (|e^z - 1| > 0.22 there); both are evaluated
+__device__ __forceinline__ float ssd_expm1(float z) {
+  const float z2 = z * z;
+  const float lo = fmaf(z, 1.0f / 6.0f, 0.5f);
+  const float hi = fmaf(z2, 1.0f / 720.0f, fmaf(z, 1.0f / 120.0f, 1.0f / 24.0f));
+  const float poly = fmaf(z2 * z2, hi, fmaf(z2, lo, z));
+  const float viaexp2 = ex2_approx(z * 1.4426950408889634f) - 1.0f;
+  return fabsf(z) <= 0.25f ? poly : viaexp2;
+}
+
+// named barrier 1 over the four builder warps (the issuer warp is not in it)
+__device__ __forceinline__ void builders_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ bool builders_and(bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred ip, op;\n\tsetp.ne.u32 ip, %1, 0;\n\tbar.red.and.pred op, 1, 128, ip;\n\t"
+      "selp.u32 %0, 1, 0, op;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)p)
+      : "memory");
+  return r != 0;
+}
+
 // ---------------------------------------------------------------------------
 // shared-memory layout (bytes), every tile in the no-swizzle core-matrix
 // form: a core matrix is 8 rows x 16 bytes, stored contiguously (128 B)
@@ -175,27 +202,31 @@ __device__ __forceinline__ void tmem_ldN(uint32_t taddr, float (&v)[N]) {
 // ---------------------------------------------------------------------------
 template <int N>
 struct SsdSmem {
-  static constexpr int kStages = N >= 64 ? 2 : 3;
+  static constexpr int kStages = 3;
   static_assert(kStages >= 2, "chunk c+1 must be resident while chunk c is finished");
   static constexpr int kX = kSsdQ * kSsdP * 2;           // the head's x tile (8 KB)
   static constexpr int kBC = kSsdQ * N * 2;              // one B or C tile
   static constexpr int kStage = kX + 2 * kBC;            // x, B, C
   static constexpr int kRing = kStages * kStage;
-  static constexpr int kM = kRing;                       // M tile, 64 x 64
-  static constexpr int kCt = kM + kSsdQ * kSsdQ * 2;     // C~ tile, 64 x N
-  static constexpr int kBw = kCt + kBC;                  // Bw tile, 64 x N
-  static constexpr int kS = kBw + kBC;                   // bf16 state copy, 64 ch x N
+  // M, C~ and Bw of two chunks (by chunk parity): the warps build chunk
+  // c+1's while the tensor core reads chunk c's
+  static constexpr int kMtile = kSsdQ * kSsdQ * 2;
+  static constexpr int kM = kRing;                       // [2] M tiles, 64 x 64
+  static constexpr int kCt = kM + 2 * kMtile;            // [2] C~ tiles, 64 x N
+  static constexpr int kBw = kCt + 2 * kBC;              // [2] Bw tiles, 64 x N
+  static constexpr int kS = kBw + 2 * kBC;               // bf16 state copy, 64 ch x N
   static constexpr int kCum = kS + kSsdP * N * 2;        // [64] cum (log2), [64] w, [64] u
   static constexpr int kWsum = kCum + 3 * kSsdQ * 4;     // [4 warps] partial sums
   static constexpr int kDs = kWsum + 16;                 // [64] D
-  static constexpr int kBar = kDs + kSsdP * 4;           // mbarriers: G, Y, then one per ring slot (TMA)
-  static constexpr int kTslot = kBar + 8 * (2 + kStages);
+  // mbarriers: G, Y, one per ring slot (TMA), operands ready, drain
+  static constexpr int kBar = kDs + kSsdP * 4;
+  static constexpr int kTslot = kBar + 8 * (4 + kStages);  // tensor-memory address, then the stop flag
   static constexpr int kBytes = kTslot + 16 + 1024;      // + room to align the base to 1024
   static constexpr int kSboBC = (N / 8) * 128;           // K-major [rows][N]
 };
 
 template <int N>
-__global__ void __launch_bounds__(kSsdWarps * 32)
+__global__ void __launch_bounds__(kSsdThreads)
 ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const __grid_constant__ CUtensorMap mb,
                  const __grid_constant__ CUtensorMap mc) {
   using L = SsdSmem<N>;
@@ -223,12 +254,19 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
 
   uint64_t* bar_g = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint64_t* bar_y = bar_g + 1;
-  uint64_t* bar_full = bar_g + 2;  // [kStages]: the slot's TMA tiles have landed
+  uint64_t* bar_full = bar_g + 2;                 // [kStages]: the slot's TMA tiles have landed
+  uint64_t* bar_ops = bar_full + L::kStages;      // the builders' operands of a chunk are ready
+  uint64_t* bar_drain = bar_ops + 1;              // the issuer's last products have completed
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + L::kTslot);
+  volatile int* s_stop = reinterpret_cast<volatile int*>(smem + L::kTslot + 4);  // the builders left early
+  const bool builder = warp < kSsdWarps;
   if (tid == 0) {
     mbar_init(bar_g, 1);
-    mbar_init(bar_y, 2);  // one commit from each of the two issuing threads
+    mbar_init(bar_y, 1);
     for (int s2 = 0; s2 < L::kStages; ++s2) mbar_init(bar_full + s2, 1);
+    mbar_init(bar_ops, 1);
+    mbar_init(bar_drain, 1);
+    *s_stop = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -240,6 +278,7 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
   griddep_wait();  // inputs (and the aggregates) may come from the previous kernel
 
   const float a_h = __ldg(a.A + h);
+  const float inv_a = 1.0f / a_h;
   const float a2 = a_h * 1.4426950408889634f;  // a in log2 units
   const __nv_bfloat16* Bg = a.B + (b * a.len) * N;
   const __nv_bfloat16* Cg = a.C + (b * a.len) * N;
@@ -295,7 +334,7 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
 #pragma unroll
   for (int n = 0; n < NH; ++n) S[n] = 0.0f;
   const int64_t sidx = ((b * a.heads + h) * kSsdP + row) * N + ch * NH;  // (batch, channel, n) offset
-  if (a.h0 && j == 0) {  // later super-chunks run from zero (the correction kernel adds their carry)
+  if (builder && a.h0 && j == 0) {  // later super-chunks run from zero (the correction kernel adds their carry)
 #pragma unroll
     for (int n = 0; n < NH; ++n) S[n] = __ldg(a.h0 + sidx + n);
   }
@@ -312,15 +351,14 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
       *reinterpret_cast<uint4*>(st + (ch * (NH / 8) + q) * 128) = v;
     }
   };
-  store_state_copy();
+  if (builder) store_state_copy();
 
   float* Ds = reinterpret_cast<float*>(smem + L::kDs);  // [64] D of the head (0 without D)
-  if (ch == 0) Ds[row] = a.D ? __ldg(a.D + (int64_t)h * kSsdP + row) : 0.0f;
+  if (builder && ch == 0) Ds[row] = a.D ? __ldg(a.D + (int64_t)h * kSsdP + row) : 0.0f;
   float* cum_s = reinterpret_cast<float*>(smem + L::kCum);  // [64]
   float* w_s = cum_s + kSsdQ;                                // [64]
   float* u_s = w_s + kSsdQ;                                  // [64] e^{-a cum_s} w_s
   float* wsum = reinterpret_cast<float*>(smem + L::kWsum);   // [4]
-  float total_log2 = 0.0f;
 
   tc_fence_before();
   __syncthreads();
@@ -353,15 +391,6 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
     umma_commit(bar_g);
   };
 
-  // prologue: the first kStages chunks, and G of chunk 0
-#pragma unroll
-  for (int s2 = 0; s2 < L::kStages; ++s2) {
-    if (s2 < nchunks) load_chunk(s2, s2);
-    cp_async_commit();
-  }
-  cp_async_wait<L::kStages - 1>();  // chunk 0
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncthreads();
   // TMA: the tiles of chunk k have landed (bounded wait on the slot's
   // barrier).  Thread 0 counts the chunks it issued and the highest one it
   // saw land, so that it can drain the copies still in flight if the CTA
@@ -374,26 +403,19 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
     return ok;
   };
   bool ok_run = true;
-  if (tid == 0 && nchunks > 0) {
-    if (tiles_ready(0)) {
-      issue_g(0);
-    } else {
-      record_device_error(MAMBA_ERR_TIMEOUT);
-      ok_run = false;
-    }
-  }
-  ok_run = __syncthreads_and(ok_run) != 0;
   uint32_t dt_raw = load_dt(0);
+  float total_log2 = 0.0f;
 
-  for (int c = 0; c < nchunks && ok_run; ++c) {
-    const int slot = c % L::kStages;
-    const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
+  // ---- the front of chunk f: Delta scan, C~ and Bw, then M from G (the
+  // operands the warps build; buffers f & 1).  Returns the chunk's total
+  // log2 decay.
+  auto front = [&](int f) -> float {
+    const int slot = f % L::kStages;
+    const uint32_t ob = slot * L::kStage + L::kX;  // B tile
+    const uint32_t oc = ob + L::kBC;               // C tile
+    const int pb = f & 1;
     const float dt = __uint_as_float(dt_raw << 16);
-    const uint32_t ndt_raw = load_dt(c + 1);
-    const uint32_t ox = slot * L::kStage;                 // x tile of the slot
-    const uint32_t ob = ox + L::kX;                       // B tile
-    const uint32_t oc = ob + L::kBC;                      // C tile
-
+    dt_raw = load_dt(f + 1);
     // running log2 decay inside the chunk: an inclusive scan over the 16
     // rows of the half-warp (both halves of a warp hold the same rows), then
     // across warps
@@ -404,15 +426,19 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
       if ((lane & 15) >= o) v += nb;
     }
     if (lane == 15) wsum[warp] = v;
-    const float wgt = a.euler ? dt : expm1f(dt * a_h) / a_h;
-    bool landed = tiles_ready(c);  // (TMA) the chunk's tiles are in its slot
+    const float wgt = a.euler ? dt : ssd_expm1(dt * a_h) * inv_a;
+    // the chunk's tiles are resident: by TMA (the slot's barrier), or by
+    // this thread's cp.async groups (the ones of later chunks may still fly;
+    // the builders' barrier below makes every thread's copies visible, and
+    // the tensor core reads them only after the next fenced bar_ops arrival)
+    cp_async_wait<L::kStages - 2>();
+    bool landed = tiles_ready(f);
     if (!landed && tid == 0) record_device_error(MAMBA_ERR_TIMEOUT);
-    ok_run = __syncthreads_and(ok_run && landed) != 0;  // the warp sums, and the vote
+    ok_run = builders_and(ok_run && landed);  // the warp sums, the copies, and the vote
     float pre = 0.0f;
     for (int w2 = 0; w2 < warp; ++w2) pre += wsum[w2];
     const float cum = v + pre;
     const float cum_end = (wsum[0] + wsum[1]) + (wsum[2] + wsum[3]);
-    total_log2 += cum_end;
     // the decay from s to t factors as e^{a cum_t} e^{-a cum_s} while the
     // factors stay in range (the chunk decays by less than 2^-100)
     const bool split = cum_end > -100.0f;
@@ -421,18 +447,17 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
       w_s[row] = wgt;
       u_s[row] = split ? ex2_approx(-cum) * wgt : 0.0f;
     }
-
     // C~ = e^{a cum_t} C_t and Bw = e^{a(cum_end - cum_s)} w_s B_s for row
     // `row`: each of the row's two threads takes half of the 16-byte pieces
     {
-      auto scaled = [&](const unsigned char* src, unsigned char* dst, float f) {
-        const uint4 v = *reinterpret_cast<const uint4*>(src);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      auto scaled = [&](const unsigned char* src, unsigned char* dst, float fac) {
+        const uint4 w = *reinterpret_cast<const uint4*>(src);
+        const uint32_t w4[4] = {w.x, w.y, w.z, w.w};
         uint32_t op[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float2 x2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[q]));
-          op[q] = pack_bf16(x2.x * f, x2.y * f);
+          op[q] = pack_bf16(x2.x * fac, x2.y * fac);
         }
         *reinterpret_cast<uint4*>(dst) = make_uint4(op[0], op[1], op[2], op[3]);
       };
@@ -444,186 +469,255 @@ ssd_chunk_kernel(const SsdArgs a, const __grid_constant__ CUtensorMap mx, const 
 #pragma unroll
       for (int q = 0; q < N / 16; ++q) {
         const int n8 = ch * (N / 16) + q;
-        scaled(smem + ob + roff + n8 * 128, smem + L::kBw + roff + n8 * 128, fB);
-        scaled(smem + oc + roff + n8 * 128, smem + L::kCt + roff + n8 * 128, fC);
+        scaled(smem + ob + roff + n8 * 128, smem + L::kBw + pb * L::kBC + roff + n8 * 128, fB);
+        scaled(smem + oc + roff + n8 * 128, smem + L::kCt + pb * L::kBC + roff + n8 * 128, fC);
       }
     }
-    __syncthreads();  // cum and w of the chunk are in shared memory
-
-    {
-      // M row `row`, columns s = 32 ch .. 32 ch + 31, from G: causal mask,
-      // decay and input weight
-      bool got = mbar_wait_bounded(bar_g, (uint32_t)(c & 1), a.wait_limit_ns);
-      got = __all_sync(0xffffffffu, got);  // warp-uniform: the tensor-memory loads are warp-wide
-      if (!got) {
-        if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
-        ok_run = false;
-      }
-      tc_fence_after();
-      unsigned char* mrow = smem + L::kM + (row >> 3) * 1024 + (row & 7) * 16;
-      if (ok_run) {
-        float g[32];
-        tmem_ldN<32>(t_lane + kColG, g);
-        const int sb = 32 * ch;
-        if (split) {
-          // M[t][s] = G[t][s] e^{a cum_t} (e^{-a cum_s} w_s), s <= t
-          const float et = ex2_approx(cum);
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            const float4 ua = *reinterpret_cast<const float4*>(u_s + sb + 8 * c8);
-            const float4 ub = *reinterpret_cast<const float4*>(u_s + sb + 8 * c8 + 4);
-            const float uu[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
-            uint32_t op[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int s0 = sb + 8 * c8 + 2 * e, i0 = 8 * c8 + 2 * e;
-              const float m0 = s0 <= row ? g[i0] * et * uu[2 * e] : 0.0f;
-              const float m1 = s0 + 1 <= row ? g[i0 + 1] * et * uu[2 * e + 1] : 0.0f;
-              op[e] = pack_bf16(m0, m1);
-            }
-            *reinterpret_cast<uint4*>(mrow + (4 * ch + c8) * 128) = make_uint4(op[0], op[1], op[2], op[3]);
-          }
-        } else {
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            uint32_t op[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int s0 = sb + 8 * c8 + 2 * e, i0 = 8 * c8 + 2 * e;
-              const float m0 = s0 <= row ? g[i0] * ex2_approx(cum - cum_s[s0]) * w_s[s0] : 0.0f;
-              const float m1 = s0 + 1 <= row ? g[i0 + 1] * ex2_approx(cum - cum_s[s0 + 1]) * w_s[s0 + 1] : 0.0f;
-              op[e] = pack_bf16(m0, m1);
-            }
-            *reinterpret_cast<uint4*>(mrow + (4 * ch + c8) * 128) = make_uint4(op[0], op[1], op[2], op[3]);
-          }
-        }
-      }
-    }
-
-    // the operands built by the warps, and chunk c+1's copies, are complete:
-    // issue Y and dS^T of chunk c, then G of chunk c+1 behind them
-    cp_async_wait<L::kStages - 2>();
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    // two issuing threads in different warps, one per column half
-    if ((tid == 0 || tid == 32) && ok_run) {
-      {
-        const int hh = tid >> 5;
-        {
-          // Y half hh (channels 32 hh ..): M X then + C~ S_in
-          const uint32_t dy = tmem + hh * d_off + kColY;
-#pragma unroll
-          for (int k = 0; k < kSsdQ / 16; ++k)
-            umma_bf16(dy, at(dM, L::kM + k * 256), at(dX, ox + 512 * hh + k * 2048), kIdY, k > 0);
-#pragma unroll
-          for (int k = 0; k < N / 16; ++k)
-            umma_bf16(dy, at(dBC, L::kCt + k * 256), at(dBC, L::kS + 4 * hh * L::kSboBC + k * 256), kIdOff, true);
-        }
-        // dS^T over tokens 32 hh .. 32 hh + 31
-#pragma unroll
-        for (int k = 2 * hh; k < 2 * hh + 2; ++k)
-          umma_bf16(tmem + hh * d_off + kColS, at(dX, ox + k * 2048), at(dBw, L::kBw + k * 2 * L::kSboBC), kIdS,
-                    k > 2 * hh);
-      }
-      umma_commit(bar_y);
-      if (tid == 0 && c + 1 < nchunks) {
-        if (tiles_ready(c + 1)) {
-          issue_g((c + 1) % L::kStages);
-        } else {
-          record_device_error(MAMBA_ERR_TIMEOUT);
-          ok_run = false;
-        }
-      }
-    }
-
-    if (ok_run) {
-      bool got = mbar_wait_bounded(bar_y, (uint32_t)(c & 1), a.wait_limit_ns);
-      got = __all_sync(0xffffffffu, got);
-      if (!got) {
-        if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
-        ok_run = false;
-      }
+    builders_sync();  // cum and w of the chunk are in shared memory
+    // M row `row`, columns s = 32 ch .. 32 ch + 31, from G: causal mask,
+    // decay and input weight
+    bool got = ok_run && mbar_wait_bounded(bar_g, (uint32_t)(f & 1), a.wait_limit_ns);
+    got = __all_sync(0xffffffffu, got);  // warp-uniform: the tensor-memory loads are warp-wide
+    if (!got && ok_run) {
+      if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+      ok_run = false;
     }
     tc_fence_after();
+    unsigned char* mrow = smem + L::kM + pb * L::kMtile + (row >> 3) * 1024 + (row & 7) * 16;
     if (ok_run) {
-      // this thread's half row of Y and its partial dS^T row: one round
-      // trip to tensor memory
-      float yv[32], ds[N];
-      {
-        uint32_t ry[2][16], rs[N / 16][16];
-        {
-          tmem_ld16_nowait(t_lane + kColY, ry[0]);
-          tmem_ld16_nowait(t_lane + kColY + 16, ry[1]);
-        }
-#pragma unroll
-        for (int q = 0; q < N / 16; ++q) tmem_ld16_nowait(t_lane + kColS + 16 * q, rs[q]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          yv[i] = __uint_as_float(ry[0][i]);
-          yv[16 + i] = __uint_as_float(ry[1][i]);
-        }
-#pragma unroll
-        for (int q = 0; q < N / 16; ++q)
-#pragma unroll
-          for (int i = 0; i < 16; ++i) ds[16 * q + i] = __uint_as_float(rs[q][i]);
-      }
-      {
-        // y = Y + D x for row `row`, channels 32 ch .. 32 ch + 31 -> bf16 ->
-        // 16-byte stores
-        const float* Dh = Ds + 32 * ch;
-        const unsigned char* xrow = smem + ox + (row >> 3) * 1024 + (row & 7) * 16 + 4 * ch * 128;
-        const bool store = t0 + row < t_end;
-        __nv_bfloat16* yrow = a.y + (b * a.len + t0 + row) * channels + (int64_t)h * kSsdP + 32 * ch;
+      float g[32];
+      tmem_ldN<32>(t_lane + kColG, g);
+      const int sb = 32 * ch;
+      if (split) {
+        // M[t][s] = G[t][s] e^{a cum_t} (e^{-a cum_s} w_s), s <= t
+        const float et = ex2_approx(cum);
 #pragma unroll
         for (int c8 = 0; c8 < 4; ++c8) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(xrow + c8 * 128);
-          const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-          const float4 da = *reinterpret_cast<const float4*>(Dh + 8 * c8);
-          const float4 db = *reinterpret_cast<const float4*>(Dh + 8 * c8 + 4);
-          const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+          const float4 ua = *reinterpret_cast<const float4*>(u_s + sb + 8 * c8);
+          const float4 ub = *reinterpret_cast<const float4*>(u_s + sb + 8 * c8 + 4);
+          const float uu[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
           uint32_t op[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[e]));
-            const int p = 8 * c8 + 2 * e;
-            op[e] = pack_bf16(fmaf(dd[2 * e], xf.x, yv[p]), fmaf(dd[2 * e + 1], xf.y, yv[p + 1]));
+            const int s0 = sb + 8 * c8 + 2 * e, i0 = 8 * c8 + 2 * e;
+            const float m0 = s0 <= row ? g[i0] * et * uu[2 * e] : 0.0f;
+            const float m1 = s0 + 1 <= row ? g[i0 + 1] * et * uu[2 * e + 1] : 0.0f;
+            op[e] = pack_bf16(m0, m1);
           }
-          if (store) *reinterpret_cast<uint4*>(yrow + 8 * c8) = make_uint4(op[0], op[1], op[2], op[3]);
+          *reinterpret_cast<uint4*>(mrow + (4 * ch + c8) * 128) = make_uint4(op[0], op[1], op[2], op[3]);
+        }
+      } else {
+#pragma unroll
+        for (int c8 = 0; c8 < 4; ++c8) {
+          uint32_t op[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int s0 = sb + 8 * c8 + 2 * e, i0 = 8 * c8 + 2 * e;
+            const float m0 = s0 <= row ? g[i0] * ex2_approx(cum - cum_s[s0]) * w_s[s0] : 0.0f;
+            const float m1 = s0 + 1 <= row ? g[i0 + 1] * ex2_approx(cum - cum_s[s0 + 1]) * w_s[s0 + 1] : 0.0f;
+            op[e] = pack_bf16(m0, m1);
+          }
+          *reinterpret_cast<uint4*>(mrow + (4 * ch + c8) * 128) = make_uint4(op[0], op[1], op[2], op[3]);
         }
       }
-      // S = e^{a cum_end} S + dS for channel `row`: this thread holds the
-      // partial sum over tokens 32 ch .. of every state; it keeps states
-      // ch NH .. and swaps the other half with the row's other thread
-      const float dec = ex2_approx(cum_end);
+    }
+    return cum_end;
+  };
+
+  // ---- the epilogue of chunk c: y = Y + D x, S = e^{a cum_end} S + dS and its
+  // bf16 copy (the next chunk's C~ S_in operand)
+  auto epilogue = [&](int c, float cum_end) {
+    bool got = ok_run && mbar_wait_bounded(bar_y, (uint32_t)(c & 1), a.wait_limit_ns);
+    got = __all_sync(0xffffffffu, got);
+    if (!got && ok_run) {
+      if (lane == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+      ok_run = false;
+    }
+    tc_fence_after();
+    if (!ok_run) return;
+    const int64_t t0 = t_begin + (int64_t)c * kSsdQ;
+    const uint32_t ox = (c % L::kStages) * L::kStage;
+    // this thread's half row of Y and its partial dS^T row: one round
+    // trip to tensor memory
+    float yv[32], ds[N];
+    {
+      uint32_t ry[2][16], rs[N / 16][16];
+      tmem_ld16_nowait(t_lane + kColY, ry[0]);
+      tmem_ld16_nowait(t_lane + kColY + 16, ry[1]);
 #pragma unroll
-      for (int i = 0; i < NH; ++i) {
-        const float keep = ch ? ds[NH + i] : ds[i];
-        const float give = ch ? ds[i] : ds[NH + i];
-        S[i] = fmaf(dec, S[i], keep + __shfl_xor_sync(0xffffffffu, give, 16));
+      for (int q = 0; q < N / 16; ++q) tmem_ld16_nowait(t_lane + kColS + 16 * q, rs[q]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        yv[i] = __uint_as_float(ry[0][i]);
+        yv[16 + i] = __uint_as_float(ry[1][i]);
       }
-      store_state_copy();
+#pragma unroll
+      for (int q = 0; q < N / 16; ++q)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) ds[16 * q + i] = __uint_as_float(rs[q][i]);
     }
-    tc_fence_before();
-    ok_run = __syncthreads_and(ok_run) != 0;  // slot c is read; every read of Y / dS is done
-    // chunk c + kStages into the slot chunk c used (its reads, and the
-    // products that read it, are complete)
-    if (a.tma && tid == 0) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    if (ok_run && c + L::kStages < nchunks) {
-      load_chunk(c + L::kStages, slot);
-      n_issued = c + L::kStages + 1;
+    {
+      // y = Y + D x for row `row`, channels 32 ch .. 32 ch + 31 -> bf16 ->
+      // 16-byte stores
+      const float* Dh = Ds + 32 * ch;
+      const unsigned char* xrow = smem + ox + (row >> 3) * 1024 + (row & 7) * 16 + 4 * ch * 128;
+      const bool store = t0 + row < t_end;
+      __nv_bfloat16* yrow = a.y + (b * a.len + t0 + row) * channels + (int64_t)h * kSsdP + 32 * ch;
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        const uint4 xv = *reinterpret_cast<const uint4*>(xrow + c8 * 128);
+        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+        const float4 da = *reinterpret_cast<const float4*>(Dh + 8 * c8);
+        const float4 db = *reinterpret_cast<const float4*>(Dh + 8 * c8 + 4);
+        const float dd[8] = {da.x, da.y, da.z, da.w, db.x, db.y, db.z, db.w};
+        uint32_t op[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[e]));
+          const int p = 8 * c8 + 2 * e;
+          op[e] = pack_bf16(fmaf(dd[2 * e], xf.x, yv[p]), fmaf(dd[2 * e + 1], xf.y, yv[p + 1]));
+        }
+        if (store) *reinterpret_cast<uint4*>(yrow + 8 * c8) = make_uint4(op[0], op[1], op[2], op[3]);
+      }
     }
-    cp_async_commit();
-    dt_raw = ndt_raw;
+    // S = e^{a cum_end} S + dS for channel `row`: this thread holds the
+    // partial sum over tokens 32 ch .. of every state; it keeps states
+    // ch NH .. and swaps the other half with the row's other thread
+    const float dec = ex2_approx(cum_end);
+#pragma unroll
+    for (int i = 0; i < NH; ++i) {
+      const float keep = ch ? ds[NH + i] : ds[i];
+      const float give = ch ? ds[i] : ds[NH + i];
+      S[i] = fmaf(dec, S[i], keep + __shfl_xor_sync(0xffffffffu, give, 16));
+    }
+    store_state_copy();
+  };
+
+  // ---- the pipeline.  The issuer warp (one thread) waits on bar_ops,
+  // whose phase 0 means chunk 0's tiles are resident and phase c+1 that the
+  // builders have chunk c's operands (M, C~, Bw, the state copy) in shared
+  // memory, chunk c+1's tiles resident and chunk c-1's tensor-memory results
+  // read; it then issues G(c+1) and chunk c's products.  The builders run,
+  // per chunk c, the front of c+1 (while the tensor core works on c), the
+  // epilogue of c, a vote, the copies of chunk c + kStages into c's slot
+  // and the next bar_ops arrival: they never wait for the issue itself.
+  if (!builder) {
+    if (lane == 0) {
+      bool ok = true;
+      auto wait_ops = [&](int phase) -> bool {
+        const bool got = mbar_wait_bounded(bar_ops, (uint32_t)(phase & 1), a.wait_limit_ns);
+        if (!got) record_device_error(MAMBA_ERR_TIMEOUT);
+        tc_fence_after();
+        return got && *s_stop == 0;
+      };
+      if (nchunks > 0 && wait_ops(0)) {
+        if (tiles_ready(0)) {
+          issue_g(0);
+        } else {
+          record_device_error(MAMBA_ERR_TIMEOUT);
+          ok = false;
+        }
+        for (int c = 0; c < nchunks && ok; ++c) {
+          if (!wait_ops(c + 1)) break;
+          if (c + 1 < nchunks) {
+            if (tiles_ready(c + 1)) {
+              issue_g((c + 1) % L::kStages);
+            } else {
+              record_device_error(MAMBA_ERR_TIMEOUT);
+              ok = false;
+            }
+          }
+          const uint32_t ox = (c % L::kStages) * L::kStage;
+          const int pb = c & 1;
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            // Y half hh (channels 32 hh ..): M X then + C~ S_in
+            const uint32_t dy = tmem + hh * d_off + kColY;
+#pragma unroll
+            for (int k = 0; k < kSsdQ / 16; ++k)
+              umma_bf16(dy, at(dM, L::kM + pb * L::kMtile + k * 256), at(dX, ox + 512 * hh + k * 2048), kIdY, k > 0);
+#pragma unroll
+            for (int k = 0; k < N / 16; ++k)
+              umma_bf16(dy, at(dBC, L::kCt + pb * L::kBC + k * 256), at(dBC, L::kS + 4 * hh * L::kSboBC + k * 256),
+                        kIdOff, true);
+            // dS^T over tokens 32 hh .. 32 hh + 31
+#pragma unroll
+            for (int k = 2 * hh; k < 2 * hh + 2; ++k)
+              umma_bf16(tmem + hh * d_off + kColS, at(dX, ox + k * 2048),
+                        at(dBw, L::kBw + pb * L::kBC + k * 2 * L::kSboBC), kIdS, k > 2 * hh);
+          }
+          umma_commit(bar_y);
+        }
+      }
+      // every product issued has completed before tensor memory is released
+      umma_commit(bar_drain);
+      if (!mbar_wait_bounded(bar_drain, 0u, a.wait_limit_ns)) record_device_error(MAMBA_ERR_TIMEOUT);
+    }
+    __syncwarp();
+  } else {
+    // builders: the first kStages chunks' copies
+#pragma unroll
+    for (int s2 = 0; s2 < L::kStages; ++s2) {
+      if (s2 < nchunks) load_chunk(s2, s2);
+      cp_async_commit();
+    }
+    // one arrival on bar_ops by builder thread 0; a stop flag goes first when
+    // the builders are leaving early (the issuer then leaves too)
+    auto arrive_ops = [&]() {
+      if (tid == 0) {
+        if (!ok_run) *s_stop = 1;
+        mbar_arrive(bar_ops);
+      }
+    };
+    float cum_end_c = 0.0f;
+    if (nchunks > 0) {
+      cp_async_wait<L::kStages - 1>();  // chunk 0
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const bool landed = tiles_ready(0);
+      if (!landed && tid == 0) record_device_error(MAMBA_ERR_TIMEOUT);
+      ok_run = builders_and(ok_run && landed);
+      arrive_ops();  // phase 0: G(0) may go
+      if (ok_run) {
+        cum_end_c = front(0);
+        total_log2 += cum_end_c;
+        cp_async_wait<0>();  // (chunks 1, 2 for G ahead)
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc_fence_before();
+        ok_run = builders_and(ok_run);
+        tc_fence_after();
+        arrive_ops();  // phase 1: chunk 0's products and G(1) may go
+      }
+    }
+    for (int c = 0; c < nchunks && ok_run; ++c) {
+      float cum_end_n = 0.0f;
+      if (c + 1 < nchunks) {
+        cum_end_n = front(c + 1);
+        total_log2 += cum_end_n;
+      }
+      epilogue(c, cum_end_c);
+      // chunk c+2's copies, the operands of c+1 and the state copy are
+      // complete; every read of chunk c's slot and of Y / dS is done
+      cp_async_wait<0>();
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      ok_run = builders_and(ok_run);
+      tc_fence_after();
+      if (ok_run && c + L::kStages < nchunks) {
+        load_chunk(c + L::kStages, c % L::kStages);
+        n_issued = c + L::kStages + 1;
+      }
+      cp_async_commit();
+      if (c + 1 < nchunks) arrive_ops();  // phase c+2: chunk c+1's products and G(c+2) may go
+      cum_end_c = cum_end_n;
+    }
   }
   cp_async_wait<0>();
   if (a.tma && tid == 0)  // (only after a timeout) copies issued but never seen to land
     for (int k = n_landed; k < n_issued; ++k) tiles_ready(k);
 
   griddep_launch_dependents();
-  if (ok_run) {
+  if (builder && ok_run) {
     if (a.supers > 1) {  // the end state from zero and the total decay, for the correction kernel
       const int64_t agg = (b * a.heads + h) * a.supers + j;
       float* as = a.agg_state + (agg * kSsdP + row) * N + ch * NH;
