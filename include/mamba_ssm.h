@@ -423,7 +423,8 @@ int mamba_state_update_mimo(float *state, const void *x, const void *delta,
 /* 1 if mamba_selective_scan_mimo implements this number of inputs/outputs and states. */
 int mamba_mimo_supported(int64_t ranks, int64_t nstate);
 
-/* How mamba_selective_scan_ex would split a problem (host-side planning only). */
+/* How mamba_selective_scan_ex (zero-order hold, default flags) would split a
+ * problem (host-side planning only). */
 typedef struct {
     int64_t supers;        /* super-chunks per sequence, run side by side from zero (1: no correction kernel) */
     int64_t super_len;     /* tokens per super-chunk (all but the last) */
@@ -432,6 +433,9 @@ typedef struct {
     int64_t kernels;       /* kernels one call launches (pre-pass, chunked scan, correction when supers > 1) */
     int64_t scratch_bytes; /* stream-ordered scratch one call allocates */
     int64_t ctas;          /* CTAs of the chunked kernel (persistent: at most one per SM) */
+    int64_t consumer_warps; /* consumer warps per CTA: 4, or 8 (two per SM sub-partition) for
+                               super-chunks of >= 65,536 tokens of the bf16 zero-order-hold scan
+                               with 16 states */
 } mamba_scan_plan_t;
 
 /*

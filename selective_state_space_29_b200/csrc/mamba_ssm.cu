@@ -144,23 +144,19 @@ bool make_map_core_tiles(CUtensorMap* m, const void* base, uint64_t row, uint64_
 }
 
 // --- scan configuration per element type and state count -------------------
-// A CTA is kScanConsumers consumer warps (one per SM sub-partition) and one
+// A CTA is CW consumer warps (4: one per SM sub-partition; 8: two) and one
 // producer warp; a consumer's ring holds kStages tiles of kTile tokens (the
 // ring of four consumers fits the 227 KB of shared memory of a CTA).
 // With R inputs per token (multi-input multi-output) a tile holds 1/R as
 // many tokens, so that its u, B and C' rows stay the same size.  With eight
-// consumer warps (two per sub-partition) tiles are half as long and the
-// ring two deep, so that eight rings fit the shared memory of a CTA.
-#ifndef MAMBA_SCAN_CONSUMERS
-#define MAMBA_SCAN_CONSUMERS 4
-#endif
-constexpr int kScanConsumers = MAMBA_SCAN_CONSUMERS;
-static_assert(kScanConsumers == 4 || kScanConsumers == 8, "one or two consumer warps per sub-partition");
-template <typename TIO, int NS, int R = 1>
+// consumer warps tiles are half as long and the ring two deep, so that
+// eight rings fit the shared memory of a CTA.
+template <typename TIO, int NS, int R = 1, int CW = 4>
 struct ScanCfg {
+  static_assert(CW == 4 || CW == 8, "one or two consumer warps per sub-partition");
   static constexpr bool kBf16 = sizeof(TIO) == 2;
-  static constexpr int kTile = (kBf16 ? 64 : 32) / R / (kScanConsumers / 4);
-  static constexpr int kStages = (kScanConsumers == 8 || (kBf16 && NS >= 32)) ? 2 : 3;
+  static constexpr int kTile = (kBf16 ? 64 : 32) / R / (CW / 4);
+  static constexpr int kStages = (CW == 8 || (kBf16 && NS >= 32)) ? 2 : 3;
 };
 #ifndef MAMBA_SCAN_JOBS_PER_WARP
 #define MAMBA_SCAN_JOBS_PER_WARP 8
@@ -176,7 +172,8 @@ constexpr int64_t kStreamsPerWarpPct = MAMBA_SCAN_STREAMS_PCT;
 struct Plan {
   int groups_d = 0;         // ceil(channels / 32)
   int64_t groups = 0;       // batch * groups_d
-  int warps_total = 0;      // resident consumer warps: SMs * kScanConsumers
+  int cw = 4;               // consumer warps per CTA
+  int warps_total = 0;      // resident consumer warps: SMs * cw
   int supers = 1;
   int64_t super_len = 0;
   int64_t chunk_len = 0;
@@ -193,9 +190,10 @@ struct Plan {
 // there are about kJobsPerWarp jobs per warp for dynamic balance, each at
 // least two tiles long.  A positive `user_chunk` forces super-chunks of that
 // length.
-Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, int64_t user_chunk) {
+Plan plan_scan(int64_t batch, int64_t len, int64_t channels, int sms, int tile, int64_t user_chunk, int cw = 4) {
   Plan pl;
-  pl.warps_total = sms * kScanConsumers;
+  pl.cw = cw;
+  pl.warps_total = sms * cw;
   pl.groups_d = (int)((channels + kCPW - 1) / kCPW);
   pl.groups = batch * pl.groups_d;
   const int64_t groups = std::max<int64_t>(1, pl.groups);
@@ -259,7 +257,32 @@ int64_t full_jobs(const Plan& pl) {
   return (int64_t)pl.chunks_last * streams + (int64_t)(pl.chunks_full - pl.chunks_last) * streams_early;
 }
 
-int tile_for(int dtype) { return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16, 16>::kTile : ScanCfg<float, 16>::kTile; }
+int tile_for(int dtype, int cw = 4) {
+  if (cw == 8) return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16, 16, 1, 8>::kTile : ScanCfg<float, 16, 1, 8>::kTile;
+  return dtype == MAMBA_BF16 ? ScanCfg<__nv_bfloat16, 16>::kTile : ScanCfg<float, 16>::kTile;
+}
+
+// Consumer warps for a scan.  Two per sub-partition hide more of a token's
+// latency but need twice the streams, i.e. twice the super-chunks, each of
+// which adds a correction walk of ~1,500 tokens, and halve the tile, i.e.
+// double the barrier traffic per token; that pays off only for bf16 data
+// in very long super-chunks (measured on 2048 channels: 2-4% faster at 2^20
+// tokens, even at 2^19, slower at 2^18 and below, and 50% slower for fp32
+// data, whose 16-token tiles hide too little of the load latency).  Built
+// for the zero-order-hold scan with one input and 16 states (`eligible`);
+// a forced chunk length keeps four.
+#ifndef MAMBA_LONG_SUPER_CHUNK
+#define MAMBA_LONG_SUPER_CHUNK 65536
+#endif
+constexpr int64_t kLongSuperChunk = MAMBA_LONG_SUPER_CHUNK;
+Plan choose_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate, int sms, int dtype,
+                 int64_t user_chunk, bool eligible) {
+  Plan pl = plan_scan(batch, len, channels, sms, tile_for(dtype), user_chunk);
+  if (eligible && dtype == MAMBA_BF16 && nstate == 16 && user_chunk == 0 && pl.supers > 1 &&
+      pl.super_len >= kLongSuperChunk)
+    pl = plan_scan(batch, len, channels, sms, tile_for(dtype, 8), 0, 8);
+  return pl;
+}
 
 // state counts the kernels are built for
 template <typename F>
@@ -334,13 +357,13 @@ int noalloc_scratch_address(void** out) {
 // by scratch_layout): pre-pass, chunked pass, [correction].  R > 1: the
 // multi-input multi-output scan (u, y [batch][len][R][channels], B, C
 // [batch][len][R][nstate]).
-template <typename TIO, int NS, int METHOD, bool CKPT = false, int R = 1>
+template <typename TIO, int NS, int METHOD, bool CKPT = false, int R = 1, int CW = 4>
 int launch_scan_on(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
                    const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
                    unsigned flags, int dtype, cudaStream_t stream, const Plan& pl, int sms,
                    unsigned char* scratch, float* ckpt = nullptr) {
-  constexpr int TILE = ScanCfg<TIO, NS, R>::kTile;
-  constexpr int STAGES = ScanCfg<TIO, NS, R>::kStages;
+  constexpr int TILE = ScanCfg<TIO, NS, R, CW>::kTile;
+  constexpr int STAGES = ScanCfg<TIO, NS, R, CW>::kStages;
   constexpr bool kWidenB = sizeof(TIO) == 2;
   const ScratchLayout sl = scratch_layout(pl, NS, batch, len, TILE, kWidenB, R);
   unsigned char* cur = scratch;
@@ -393,9 +416,9 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   p.use_tma = tma ? 1 : 0;
   p.wait_limit_ns = kWaitLimitNs;
 
-  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES, kScanConsumers, R>();
+  constexpr size_t smem = scan_smem_bytes<TIO, NS, TILE, STAGES, CW, R>();
   static_assert(smem <= 232448, "scan CTA exceeds the shared memory of an SM");
-  auto kern = scan_chunks_kernel<TIO, NS, kScanConsumers, TILE, STAGES, METHOD, CKPT, R>;
+  auto kern = scan_chunks_kernel<TIO, NS, CW, TILE, STAGES, METHOD, CKPT, R>;
   {
     // the dynamic shared-memory limit is a per-device attribute of the kernel
     static std::mutex mu_attr;
@@ -438,8 +461,8 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   }
   // one persistent pass over every super-chunk from zero (super-chunk 0
   // from the initial state) ...
-  const int64_t ctas = std::min<int64_t>(sms, (jobs + kScanConsumers - 1) / kScanConsumers);
-  if (launch_pdl(kern, dim3((unsigned)ctas), dim3((kScanConsumers + 1) * 32), smem, stream, p, mu, mdl, mb, mc) !=
+  const int64_t ctas = std::min<int64_t>(sms, (jobs + CW - 1) / CW);
+  if (launch_pdl(kern, dim3((unsigned)ctas), dim3((CW + 1) * 32), smem, stream, p, mu, mdl, mb, mc) !=
       cudaSuccess)
     return MAMBA_ERR_CUDA;
   // ... then the states entering super-chunks 1..S-1 and their effect on y
@@ -456,6 +479,18 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
   return MAMBA_OK;
 }
 
+// The eight-consumer scan exists for 16 states only (choose_plan)
+template <typename TIO, int NS>
+int launch_cw8(const void* u, const void* delta, const float* A, const void* B, const void* C, const float* D,
+               const float* h0, void* y, float* final_state, int64_t batch, int64_t len, int64_t channels,
+               unsigned flags, int dtype, cudaStream_t stream, const Plan& pl, int sms, unsigned char* scratch) {
+  if constexpr (NS == 16)
+    return launch_scan_on<TIO, NS, kZOH, false, 1, 8>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels,
+                                                      flags, dtype, stream, pl, sms, scratch);
+  else
+    return MAMBA_ERR_UNSUPPORTED;
+}
+
 // Plan, get scratch (stream-ordered allocation, or the fixed array when
 // `noalloc`), enqueue, release the allocation.
 template <typename TIO, int NS>
@@ -465,9 +500,10 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
                 float* ckpt = nullptr) {
   int sms = 0;
   if (int st = current_sms(&sms)) return st;
-  const Plan pl = plan_scan(batch, len, channels, sms, ScanCfg<TIO, NS>::kTile, user_chunk);
+  const bool zoh = !(flags & (MAMBA_SCAN_EULER | MAMBA_SCAN_TRAPEZOID));
+  const Plan pl = choose_plan(batch, len, channels, NS, sms, dtype, user_chunk, zoh && !ckpt);
   if (pl.groups > (1 << 30)) return MAMBA_ERR_UNSUPPORTED;
-  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, ScanCfg<TIO, NS>::kTile, sizeof(TIO) == 2);
+  const ScratchLayout sl = scratch_layout(pl, NS, batch, len, tile_for(dtype, pl.cw), sizeof(TIO) == 2);
   unsigned char* scratch = nullptr;
   if (noalloc) {
     if (sl.total > kNoAllocScratchBytes) return MAMBA_ERR_UNSUPPORTED;  // needs more than the fixed array
@@ -487,6 +523,9 @@ int launch_scan(const void* u, const void* delta, const float* A, const void* B,
   else if (ckpt)
     status = launch_scan_on<TIO, NS, kZOH, true>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels,
                                                  flags, dtype, stream, pl, sms, scratch, ckpt);
+  else if (pl.cw == 8)
+    status = launch_cw8<TIO, NS>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags, dtype, stream,
+                                 pl, sms, scratch);
   else
     status = launch_scan_on<TIO, NS, kZOH>(u, delta, A, B, C, D, h0, y, final_state, batch, len, channels, flags,
                                            dtype, stream, pl, sms, scratch);
@@ -784,14 +823,16 @@ int mamba_scan_plan(int64_t batch, int64_t len, int64_t channels, int64_t nstate
   if (sms <= 0) {
     if (int st = current_sms(&sms)) return st;
   }
-  const Plan pl = plan_scan(batch, len, channels, sms, tile_for(dtype), chunk_len);
+  const Plan pl = choose_plan(batch, len, channels, nstate, sms, dtype, chunk_len, true);
   out->supers = pl.supers;
   out->super_len = pl.super_len;
   out->chunk_len = pl.chunk_len;
   out->jobs = full_jobs(pl);
   out->kernels = kernels_per_call(pl);
-  out->scratch_bytes = (int64_t)scratch_layout(pl, (int)nstate, batch, len, tile_for(dtype), dtype == MAMBA_BF16).total;
-  out->ctas = std::min<int64_t>(sms, (out->jobs + kScanConsumers - 1) / kScanConsumers);
+  out->scratch_bytes =
+      (int64_t)scratch_layout(pl, (int)nstate, batch, len, tile_for(dtype, pl.cw), dtype == MAMBA_BF16).total;
+  out->ctas = std::min<int64_t>(sms, (out->jobs + pl.cw - 1) / pl.cw);
+  out->consumer_warps = pl.cw;
   return MAMBA_OK;
 }
 

@@ -30,7 +30,7 @@ class ScanPlan(ctypes.Structure):
     """mamba_scan_plan_t"""
     _fields_ = [("supers", ctypes.c_int64), ("super_len", ctypes.c_int64), ("chunk_len", ctypes.c_int64),
                 ("jobs", ctypes.c_int64), ("kernels", ctypes.c_int64), ("scratch_bytes", ctypes.c_int64),
-                ("ctas", ctypes.c_int64)]
+                ("ctas", ctypes.c_int64), ("consumer_warps", ctypes.c_int64)]
 
     def as_dict(self):
         return {k: int(getattr(self, k)) for k, _ in self._fields_}

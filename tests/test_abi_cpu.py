@@ -236,17 +236,23 @@ def test_scan_plan_host_logic(lib):
     sms = 148
     # mid workload: 8 x 3072 channels = 768 groups >= 592 warps -> no split
     p = m.mamba_scan_plan(8, 2048, 3072, 16, 0, m.MAMBA_BF16, sms)
-    assert p.supers == 1 and p.kernels == 2
+    assert p.supers == 1 and p.kernels == 2 and p.consumer_warps == 4
     assert p.jobs * p.chunk_len >= 768 * 2048 and p.jobs >= 8 * 592 * 0.9
     assert p.ctas == sms
     # long workload: 64 groups -> split into super-chunks that run from zero
-    # side by side; pre-pass, chunked kernel, correction kernel
+    # side by side; pre-pass, chunked kernel, correction kernel.  The
+    # super-chunks are long, so the CTAs carry eight consumer warps
     p = m.mamba_scan_plan(1, 1 << 20, 2048, 16, 0, m.MAMBA_BF16, sms)
-    assert p.supers > 1 and p.kernels == 3
-    assert p.supers * 64 >= 592
+    assert p.supers > 1 and p.kernels == 3 and p.consumer_warps == 8
+    assert p.supers * 64 >= sms * 8
     assert p.super_len * p.supers >= 1 << 20 and p.super_len * (p.supers - 1) < 1 << 20
     # every job is a chunk of a main stream: the jobs cover each stream once
     assert p.jobs * p.chunk_len >= 64 * (1 << 20) and (p.jobs - 64 * p.supers) * p.chunk_len < 64 * (1 << 20)
+    # shorter super-chunks, other state counts and forced chunking keep four
+    assert m.mamba_scan_plan(1, 1 << 19, 2048, 16, 0, m.MAMBA_BF16, sms).consumer_warps == 4
+    assert m.mamba_scan_plan(1, 1 << 20, 2048, 16, 0, m.MAMBA_F32, sms).consumer_warps == 4
+    assert m.mamba_scan_plan(1, 1 << 20, 2048, 32, 0, m.MAMBA_BF16, sms).consumer_warps == 4
+    assert m.mamba_scan_plan(1, 1 << 20, 2048, 16, 4096, m.MAMBA_BF16, sms).consumer_warps == 4
     # forced chunking
     p = m.mamba_scan_plan(2, 1000, 200, 16, 37, m.MAMBA_BF16, sms)
     assert p.super_len == 37 and p.supers == 28 and p.kernels == 3
