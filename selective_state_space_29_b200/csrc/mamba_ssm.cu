@@ -1020,26 +1020,44 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
         const size_t sc_bytes = al(sizeof(float) * (size_t)ctas * kBwdWarps * (T / 2 + 1) * 32 * NS);
         const size_t mu_bytes = al(sizeof(float) * (size_t)supers * (size_t)streams * 32 * NS);
         const size_t sd_bytes = al(sizeof(float) * (size_t)supers * (size_t)streams * 32);
+        // bf16 B and C are widened to fp32 once (fp32 B and C are read in place)
+        constexpr bool kWiden = sizeof(TIO) == 2;
+        const size_t row_elems = (size_t)batch * (size_t)len * NS;
+        const size_t wd_bytes = kWiden ? al(sizeof(float) * row_elems) : 0;
         unsigned char* mem = nullptr;
-        if (scratch_alloc(reinterpret_cast<void**>(&mem), ck_bytes + sc_bytes + mu_bytes + sd_bytes, stream) !=
-            cudaSuccess)
+        if (scratch_alloc(reinterpret_cast<void**>(&mem), ck_bytes + sc_bytes + mu_bytes + sd_bytes + 2 * wd_bytes,
+                          stream) != cudaSuccess)
           return MAMBA_ERR_CUDA;
         float* ckpt = reinterpret_cast<float*>(mem);
+        unsigned char* wd = mem + ck_bytes + sc_bytes + mu_bytes + sd_bytes;
+        const float* Bf = kWiden ? reinterpret_cast<const float*>(wd) : static_cast<const float*>(B);
+        const float* Cf = kWiden ? reinterpret_cast<const float*>(wd + wd_bytes) : static_cast<const float*>(C);
+        int st = MAMBA_OK;
+        if constexpr (kWiden) {
+          const int vec = (aligned(B, 16) && aligned(C, 16) && row_elems % 8 == 0) ? 1 : 0;
+          const int64_t work = vec ? (int64_t)(row_elems / 8) : (int64_t)row_elems;
+          const unsigned blocks = (unsigned)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, 8 * sms));
+          if (launch_pdl(bwd_widen_kernel, dim3(blocks), dim3(256), 0, stream,
+                         static_cast<const __nv_bfloat16*>(B), static_cast<const __nv_bfloat16*>(C),
+                         const_cast<float*>(Bf), const_cast<float*>(Cf), (int64_t)row_elems, vec) != cudaSuccess)
+            st = MAMBA_ERR_CUDA;
+        }
         // forward pass that only leaves the state before every tile
-        int st = launch_scan<TIO, NS>(u, delta, A, B, C, D, initial_state, nullptr, nullptr, batch, len, channels, 0,
-                                      0u, dtype, stream, false, ckpt);
+        if (st == MAMBA_OK)
+          st = launch_scan<TIO, NS>(u, delta, A, B, C, D, initial_state, nullptr, nullptr, batch, len, channels, 0,
+                                    0u, dtype, stream, false, ckpt);
         if (st == MAMBA_OK) {
-          BwdArgs<TIO> a{static_cast<const TIO*>(u), static_cast<const TIO*>(delta), A, static_cast<const TIO*>(B),
-                         static_cast<const TIO*>(C), D, static_cast<const TIO*>(dy), d_final_state, ckpt,
-                         reinterpret_cast<float*>(mem + ck_bytes), static_cast<TIO*>(du), static_cast<TIO*>(ddelta),
-                         dA, dB, dC, D ? dD : nullptr, d_initial_state, batch, len, channels, (int)groups_d, T,
-                         (aligned(B, 16) && aligned(C, 16) && (NS * sizeof(TIO)) % 16 == 0) ? 1 : 0, (int)supers,
-                         (int)super_tiles, reinterpret_cast<float*>(mem + ck_bytes + sc_bytes),
+          BwdArgs<TIO> a{static_cast<const TIO*>(u), static_cast<const TIO*>(delta), A, Bf, Cf, D,
+                         static_cast<const TIO*>(dy), d_final_state, ckpt, reinterpret_cast<float*>(mem + ck_bytes),
+                         static_cast<TIO*>(du), static_cast<TIO*>(ddelta), dA, dB, dC, D ? dD : nullptr,
+                         d_initial_state, batch, len, channels, (int)groups_d, T,
+                         (aligned(Bf, 16) && aligned(Cf, 16)) ? 1 : 0, (int)supers, (int)super_tiles,
+                         reinterpret_cast<float*>(mem + ck_bytes + sc_bytes),
                          reinterpret_cast<float*>(mem + ck_bytes + sc_bytes + mu_bytes), 0};
           // tiles staged in shared memory when every row piece is a whole,
           // aligned 16-byte copy
-          a.staged = ((channels * (int64_t)es) % 16 == 0 && (NS * es) % 16 == 0 && aligned(u, 16) &&
-                      aligned(delta, 16) && aligned(dy, 16) && aligned(B, 16) && aligned(C, 16))
+          a.staged = ((channels * (int64_t)es) % 16 == 0 && aligned(u, 16) && aligned(delta, 16) &&
+                      aligned(dy, 16) && aligned(Bf, 16) && aligned(Cf, 16))
                          ? 1
                          : 0;
           if (supers > 1) {
@@ -1055,8 +1073,8 @@ int mamba_selective_scan_backward(const void* u, const void* delta, const float*
                            (size_t)agg_smem, stream, a) != cudaSuccess)
               st = MAMBA_ERR_CUDA;
           }
-          const int smem = a.staged ? kBwdWarps * bwd_stage_bytes<TIO, NS>(T) : 0;
-          if (st == MAMBA_OK && smem > 0 &&
+          const int smem = kBwdWarps * bwd_warp_smem<TIO, NS>(T, a.staged != 0);
+          if (st == MAMBA_OK &&
               cudaFuncSetAttribute(scan_backward_kernel<TIO, NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    smem) != cudaSuccess)
             st = MAMBA_ERR_CUDA;
