@@ -471,7 +471,11 @@ int launch_scan_on(const void* u, const void* delta, const float* A, const void*
     const int phases = (int)fix_phases;
     const int64_t blocks = (fix_warps + kFixWarps - 1) / kFixWarps;
     constexpr int fix_smem = kFixWarps * fix_stage_bytes<TIO, NS, TILE, R>();
-    static_assert(fix_smem <= 48 * 1024, "correction staging within the default shared-memory limit");
+    if constexpr (fix_smem > 48 * 1024) {
+      if (cudaFuncSetAttribute(scan_fix_kernel<TIO, NS, TILE, CKPT, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               fix_smem) != cudaSuccess)
+        return MAMBA_ERR_CUDA;
+    }
     if (launch_pdl(scan_fix_kernel<TIO, NS, TILE, CKPT, R>, dim3((unsigned)blocks), dim3(kFixWarps * 32), fix_smem,
                    stream, p, phases) != cudaSuccess)
       return MAMBA_ERR_CUDA;

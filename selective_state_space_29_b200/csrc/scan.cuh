@@ -33,10 +33,11 @@
 //         y_t += sum_n C_t[n] exp(A_n cum_t) h_in[n],
 //     cum_t the sum of Delta from the super-chunk's start through t.  It
 //     walks each super-chunk only while the slowest decay exp(A_n cum_t) is
-//     at least 2^-kFixStopLog2 (2^-32): past that every term is below 2^-32
-//     of |C_t[n] h_in[n]|, 256 times under the fp32 rounding of y.  It also
-//     writes the final state H + exp(A sum Delta) h_in of the last
-//     super-chunk (exactly, not truncated).
+//     at least 2^-s, s = fix_stop_log2: past that every term is below 2^-s
+//     of |C_t[n] h_in[n]|.  s = 32 for fp32 data (256 times under the fp32
+//     rounding of y), 20 for bf16 data (2^11 times under the bf16 rounding
+//     of y).  It also writes the final state H + exp(A sum Delta) h_in of
+//     the last super-chunk (exactly, not truncated).
 //
 // Arithmetic per token and state (all fp32; the state is kept scaled,
 // g_n = A_n h_n, so that 1/A_n leaves the inner loop):
@@ -73,7 +74,9 @@ constexpr int kScanUnroll = MAMBA_SCAN_UNROLL;  // token pairs per unrolled step
 
 constexpr int kCPW = 32;   // channels per warp: one lane per channel
 constexpr int kFixSegTiles = 1;  // tiles per segment of the super-chunk correction
-constexpr float kFixStopLog2 = 32.0f;  // the correction stops where the carried decay is below 2^-32
+// the correction stops where the carried decay is below 2^-fix_stop_log2
+template <typename TIO>
+__host__ __device__ constexpr float fix_stop_log2() { return sizeof(TIO) == 2 ? 20.0f : 32.0f; }
 constexpr int kHandQ = 8;  // hand-off flags a consumer may leave for the producer to publish
 
 enum Discretisation : int { kZOH = 0, kEuler = 1, kTrapezoid = 2 };
@@ -863,8 +866,8 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES, R>& cx, 
   }
   // super-chunks 1..S-1 ran from zero: leave the correction kernel the sum
   // of Delta at every segment start, until the slowest decay falls below
-  // 2^-kFixStopLog2 on every lane (the carried state's term is negligible
-  // in fp32 for the rest of the super-chunk)
+  // 2^-fix_stop_log2 on every lane (the carried state's term is negligible
+  // at the output's precision for the rest of the super-chunk)
   bool track = p.supers > 1 && jb.super_idx > 0;
   float kmax = 0.0f;
   if (track) {
@@ -904,7 +907,7 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES, R>& cx, 
     const int64_t tt0 = jb.t0 + (int64_t)it * TILE;
     const int rows = (int)(jb.t1 - tt0 < (int64_t)TILE ? jb.t1 - tt0 : (int64_t)TILE);
     if (track && (tile0 + it) % kFixSegTiles == 0) {
-      if (__all_sync(0xffffffffu, !active || sd * kmax < -kFixStopLog2)) {
+      if (__all_sync(0xffffffffu, !active || sd * kmax < -fix_stop_log2<TIO>())) {
         track = false;
       } else {
         const int seg = (int)((tile0 + it) / kFixSegTiles);
@@ -1061,13 +1064,17 @@ scan_chunks_kernel(const __grid_constant__ ScanParams p, const __grid_constant__
 //     sum_n C_t[n] exp(A_n cum_t) h_in[n],   cum_t = sum of Delta from the
 //                                            super-chunk's start through t.
 // The main pass left cum at the start of every tile, up to the tile where
-// the slowest decay falls below 2^-kFixStopLog2 on every lane (from there on
-// the term is below 2^-32 of its size), and the number of such tiles per
-// stream.  One warp per (stream of a super-chunk j >= 1, phase w), a lane per
-// channel, takes tiles w, w + phases, ...: it stages the tile's Delta, y
-// and C rows in its shared memory (16-byte cp.async copies, all in flight
-// at once; plain loads when rows are not 16-byte pieces), adds the term
-// token by token, and writes y back.  Phase 0 of the last super-chunk writes
+// the slowest decay falls below 2^-fix_stop_log2 on every lane (from there
+// on the term is below that fraction of its size), and the number of such
+// tiles per stream.  One warp per (stream of a super-chunk j >= 1, phase w),
+// a lane per channel, takes tiles w, w + phases, ...: it stages the tile's
+// Delta and y rows and the pre-pass's fp32 C' = C / (n+1) rows in its shared
+// memory (16-byte cp.async copies, all in flight at once; plain loads when
+// rows are not 16-byte pieces), adds the term token by token, and writes y
+// back.  With C' the carried state is taken as hs_n = (n+1) h_n, and for
+// structured A the term sum_n C'_n hs_n rho^(n+1) is a Horner scheme in
+// rho^2 over pairs of states (even states in one half of a packed FFMA2,
+// odd ones in the other).  Phase 0 of the last super-chunk writes
 // the final state H + exp(A sum Delta) h_in.  CKPT: the state checkpointed
 // before every walked tile gets exp(A_n cum) h_in[n] added.
 // ---------------------------------------------------------------------------
@@ -1078,8 +1085,8 @@ constexpr int kFixWarps = 4;
 constexpr int kFixPhases = MAMBA_FIX_PHASES;  // warps per stream of the correction (tiles w, w + phases, ...)
 
 template <typename TIO, int NS, int TILE, int R>
-__host__ __device__ constexpr int fix_stage_bytes() {  // one warp: Delta [TILE][32], y [TILE*R][32], C [TILE*R][NS]
-  return (TILE * kCPW + TILE * R * kCPW + TILE * R * NS) * (int)sizeof(TIO);
+__host__ __device__ constexpr int fix_stage_bytes() {  // one warp: Delta [TILE][32], y [TILE*R][32], C' [TILE*R][NS] fp32
+  return (TILE * kCPW + TILE * R * kCPW) * (int)sizeof(TIO) + TILE * R * NS * (int)sizeof(float);
 }
 
 template <typename TIO, int NS, int TILE, bool CKPT, int R = 1>
@@ -1163,13 +1170,17 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
   const int64_t s_end = (s_begin + p.super_len < p.len) ? s_begin + p.super_len : p.len;
   const int tiles = ld_volatile(p.fix_segs + stream);
   const TIO* dl = static_cast<const TIO*>(p.delta);
-  const TIO* Cg = static_cast<const TIO*>(p.C);
+  const float* Cs = p.cs;  // C' = C / (n+1), fp32
   TIO* y = static_cast<TIO*>(p.y);
   // this warp's staging area
   TIO* sdl = reinterpret_cast<TIO*>(fix_smem + wl * fix_stage_bytes<TIO, NS, TILE, R>());  // [TILE][32]
   TIO* sy = sdl + TILE * kCPW;                                                              // [TILE*R][32]
-  TIO* sc = sy + TILE * R * kCPW;                                                            // [TILE*R][NS]
+  float* sc = reinterpret_cast<float*>(sy + TILE * R * kCPW);                               // [TILE*R][NS]
   const uint32_t s_dl = smem_addr(sdl), s_y = smem_addr(sy), s_c = smem_addr(sc);
+  // the carried state against C': C_n h_n = C'_n hs_n, hs_n = (n+1) h_n
+  float2 hs2[NS / 2];
+#pragma unroll
+  for (int k = 0; k < NS / 2; ++k) hs2[k] = make_float2((float)(2 * k + 1) * h[2 * k], (float)(2 * k + 2) * h[2 * k + 1]);
 
   for (int k = w; k < tiles; k += phases) {
     float cum = __ldcg(p.cum + ((int64_t)stream * p.segs_max + k) * kCPW + lane);
@@ -1192,16 +1203,16 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
           cp_async16_zfill(s_y + (uint32_t)(r * kCPW + c * kChunk) * sizeof(TIO),
                            in ? (const void*)(y + (row0 * R + r) * p.channels + d0 + c * kChunk) : p.delta, in);
         }
-      constexpr int kCPieces = NS / kChunk;  // 16-byte pieces of a C row
+      constexpr int kCPieces = NS / 4;  // 16-byte pieces of an fp32 C' row
       for (int i = lane; i < nt * R * kCPieces; i += 32)
-        cp_async16_zfill(s_c + (uint32_t)i * 16u, Cg + row0 * R * NS + (int64_t)i * kChunk, true);
+        cp_async16_zfill(s_c + (uint32_t)i * 16u, Cs + row0 * R * NS + (int64_t)i * 4, true);
       asm volatile("cp.async.wait_all;" ::: "memory");
     } else {
       for (int r = 0; r < nt; ++r) sdl[r * kCPW + lane] = active ? dl[(row0 + r) * p.channels + d] : from_f32<TIO>(0.0f);
       if (y != nullptr)
         for (int r = 0; r < nt * R; ++r)
           sy[r * kCPW + lane] = active ? y[(row0 * R + r) * p.channels + d] : from_f32<TIO>(0.0f);
-      for (int i = lane; i < nt * R * NS; i += 32) sc[i] = Cg[row0 * R * NS + i];
+      for (int i = lane; i < nt * R * NS; i += 32) sc[i] = Cs[row0 * R * NS + i];
     }
     __syncwarp();
     for (int r = 0; r < nt; ++r) {
@@ -1222,31 +1233,29 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
       }
 #pragma unroll
       for (int q = 0; q < R; ++q) {  // output q reads the state with its own C row
-        float cv[NS];
-        const TIO* crow = sc + (r * R + q) * NS;
-        if constexpr ((NS * sizeof(TIO)) % 16 == 0) {
+        // the products C'_n hs_n in pairs (n, n+1)
+        float2 pc[NS / 2];
+        const float4* crow = reinterpret_cast<const float4*>(sc + (r * R + q) * NS);
 #pragma unroll
-          for (int i = 0; i < NS; i += kChunk) {
-            const uint4 v = *reinterpret_cast<const uint4*>(crow + i);
-            const TIO* e = reinterpret_cast<const TIO*>(&v);
-#pragma unroll
-            for (int k2 = 0; k2 < kChunk; ++k2) cv[i + k2] = to_f32(e[k2]);
-          }
-        } else {
-#pragma unroll
-          for (int n = 0; n < NS; ++n) cv[n] = to_f32(crow[n]);
+        for (int i = 0; i < NS / 4; ++i) {
+          const float4 v = crow[i];
+          pc[2 * i] = __fmul2_rn(make_float2(v.x, v.y), hs2[2 * i]);
+          pc[2 * i + 1] = __fmul2_rn(make_float2(v.z, v.w), hs2[2 * i + 1]);
         }
         float corr;
         if (structured) {
-          // sum_n C_n h_n rho^(n+1), Horner in rho
-          corr = cv[NS - 1] * h[NS - 1];
+          // sum_n C_n h_n rho^(n+1) = rho (E(rho^2) + rho O(rho^2)), E and O
+          // the polynomials of the even and the odd states, Horner together
+          const float rho2 = rho * rho;
+          const float2 rr = make_float2(rho2, rho2);
+          float2 acc = pc[NS / 2 - 1];
 #pragma unroll
-          for (int n = NS - 2; n >= 0; --n) corr = fmaf(corr, rho, cv[n] * h[n]);
-          corr *= rho;
+          for (int k = NS / 2 - 2; k >= 0; --k) acc = __ffma2_rn(acc, rr, pc[k]);
+          corr = fmaf(acc.y, rho, acc.x) * rho;
         } else {
           corr = 0.0f;
 #pragma unroll
-          for (int n = 0; n < NS; ++n) corr = fmaf(cv[n], ev[n] * h[n], corr);
+          for (int k = 0; k < NS / 2; ++k) corr = fmaf(ev[2 * k], pc[k].x, fmaf(ev[2 * k + 1], pc[k].y, corr));
         }
         TIO& yv = sy[(r * R + q) * kCPW + lane];
         yv = from_f32<TIO>(to_f32(yv) + corr);
@@ -1268,7 +1277,7 @@ scan_fix_kernel(const __grid_constant__ ScanParams p, int phases) {
       }
     }
     __syncwarp();
-    if (__all_sync(0xffffffffu, !active || cum * kmax < -kFixStopLog2))
+    if (__all_sync(0xffffffffu, !active || cum * kmax < -fix_stop_log2<TIO>()))
       break;  // later tiles of this warp add less (their cum is larger)
   }
 }
