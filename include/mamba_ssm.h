@@ -119,8 +119,9 @@ typedef enum {
  * that run side by side, their end states and step sums (mamba_scan_plan
  * reports the size).  With super-chunks a third kernel adds the state
  * entering each super-chunk to its outputs; it walks a super-chunk only
- * while that state's decay is at least 2^-32 (the terms left out are below
- * 2^-32 of their size, under fp32 rounding of y; the final state is
+ * while that state's decay is at least 2^-32 for MAMBA_F32 data, 2^-20 for
+ * MAMBA_BF16 data (the terms left out are below that fraction of their
+ * size: under the fp32, resp. bf16, rounding of y; the final state is
  * composed exactly).  batch == 0 or
  * channels == 0 is a no-op that returns MAMBA_OK.
  * The call enqueues only stream-ordered work (allocation, kernels, free), so

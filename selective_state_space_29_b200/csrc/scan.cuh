@@ -756,8 +756,11 @@ __device__ void producer_loop(const ScanParams& p, WarpSmem<TIO, NS, TILE, STAGE
               mbar_arrive_expect_tx(&sm.full[s], tile_bytes<TIO, NS, R>(TILE) + (first ? kChanBytes : 0u));
               tma_load_2d(&sm.u[s][0][0], mu, &sm.full[s], f[w].d0, row * R);
               tma_load_2d(&sm.dl[s][0][0], mdl, &sm.full[s], f[w].d0, row);
-              tma_load_2d(&sm.b[s][0][0], mb, &sm.full[s], 0, row * R);
-              tma_load_2d(&sm.cs[s][0][0], mc, &sm.full[s], 0, row * R);
+              // B and C' rows are read by every channel group of the
+              // batch row: keep them in L2 ahead of the u and Delta lines
+              const uint64_t keep = l2_policy_evict_last();
+              tma_load_2d_hint(&sm.b[s][0][0], mb, &sm.full[s], 0, row * R, keep);
+              tma_load_2d_hint(&sm.cs[s][0][0], mc, &sm.full[s], 0, row * R, keep);
               if (first) bulk_load(&sm.chan[s][0], p.chan + f[w].d0, kChanBytes, &sm.full[s]);
             } else {
               mbar_arrive(&sm.full[s]);
