@@ -162,13 +162,14 @@ struct ScanCfg {
 #define MAMBA_SCAN_JOBS_PER_WARP 8
 #endif
 constexpr int kJobsPerWarp = MAMBA_SCAN_JOBS_PER_WARP;  // chunks per consumer warp, for dynamic balance
-// With eight consumers (very long super-chunks) the jobs are four times as
-// many and as short: two warps reading the two halves of the same 128-byte
-// u and Delta lines (neighbouring channel groups) then stay close enough in
-// time for the second read to hit L2 (measured at 2^20 tokens x 2048
-// channels: DRAM reads 14.2 -> 11.5 GB per launch, 8.73 -> 8.48 ms); with
-// four consumers the extra job hand-offs cost more than they save.
-constexpr int kJobsPerWarpCw8 = 4 * MAMBA_SCAN_JOBS_PER_WARP;
+// With eight consumers (very long super-chunks) the jobs are twice as many
+// and as short (measured at 2^20 tokens x 2048 channels: 8.47 ms with 8 jobs
+// per warp, 8.19 with 16, 8.23 with 32); with four consumers more jobs cost
+// more hand-offs than they gain in balance.
+#ifndef MAMBA_SCAN_JOBS_PER_WARP_CW8
+#define MAMBA_SCAN_JOBS_PER_WARP_CW8 (2 * MAMBA_SCAN_JOBS_PER_WARP)
+#endif
+constexpr int kJobsPerWarpCw8 = MAMBA_SCAN_JOBS_PER_WARP_CW8;
 // streams (channel group x super-chunk) per resident consumer warp, in percent,
 // below which sequences are cut into super-chunks
 #ifndef MAMBA_SCAN_STREAMS_PCT
