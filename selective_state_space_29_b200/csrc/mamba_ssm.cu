@@ -1194,7 +1194,13 @@ int mamba_state_update_mimo(float* state, const void* x, const void* delta, cons
     return MAMBA_ERR_INVALID_ARG;
   cudaGetLastError();
   constexpr int NS = 16;
-  constexpr int kRows = 2;  // batch rows per thread
+  // batch rows per thread: one keeps the registers low enough for more
+  // resident warps, which the step needs to keep loads in flight (256 x 5120
+  // rows, 4 inputs and outputs: 68 us with one row, 77 with two, 103 with four)
+#ifndef MAMBA_MIMO_DECODE_ROWS
+#define MAMBA_MIMO_DECODE_ROWS 1
+#endif
+  constexpr int kRows = MAMBA_MIMO_DECODE_ROWS;
   constexpr int kChanPerCta = kDecodeWarps * (32 / (NS / 4));
   const int64_t gx = (channels + kChanPerCta - 1) / kChanPerCta;
   const int64_t gy = (batch + kRows - 1) / kRows;
