@@ -297,10 +297,11 @@ __device__ __forceinline__ void decay_chain(float r, float q, float2 (&e2)[NS / 
 }
 
 // One token for one lane: g <- g + e (g + B x) for all states; returns
-// sum_n C'_n g_n.  States as N/2 float2 pairs, every step a packed FFMA2
-// (B x is exact in fp32 for bf16 operands, so this equals the mixed-precision
-// product of the raw bf16 values).
-template <typename TIO, int NS>
+// sum_n C'_n g_n (Y; without Y, only the state steps: the checkpointing pass
+// of the backward writes no output).  States as N/2 float2 pairs, every step
+// a packed FFMA2 (B x is exact in fp32 for bf16 operands, so this equals the
+// mixed-precision product of the raw bf16 values).
+template <typename TIO, int NS, bool Y = true>
 __device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const float* brow, const float* csrow, TIO xr,
                                               float2 (&g)[NS / 2]) {
   float2 acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
@@ -309,14 +310,16 @@ __device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const f
 #pragma unroll
   for (int n4 = 0; n4 < NS / 4; ++n4) {
     const float4 bv = reinterpret_cast<const float4*>(brow)[n4];
-    const float4 cv = reinterpret_cast<const float4*>(csrow)[n4];
     const int p0 = 2 * n4, p1 = 2 * n4 + 1;
     const float2 v0 = __ffma2_rn(f2(bv.x, bv.y), x2, g[p0]);
     const float2 v1 = __ffma2_rn(f2(bv.z, bv.w), x2, g[p1]);
     g[p0] = __ffma2_rn(e[p0], v0, g[p0]);
     g[p1] = __ffma2_rn(e[p1], v1, g[p1]);
-    acc0 = __ffma2_rn(f2(cv.x, cv.y), g[p0], acc0);
-    acc1 = __ffma2_rn(f2(cv.z, cv.w), g[p1], acc1);
+    if constexpr (Y) {
+      const float4 cv = reinterpret_cast<const float4*>(csrow)[n4];
+      acc0 = __ffma2_rn(f2(cv.x, cv.y), g[p0], acc0);
+      acc1 = __ffma2_rn(f2(cv.z, cv.w), g[p1], acc1);
+    }
   }
   return (acc0.x + acc0.y) + (acc1.x + acc1.y);
 }
@@ -329,7 +332,7 @@ __device__ __forceinline__ float token_update(const float2 (&e)[NS / 2], const f
 // expm1 and r = 1 + q.  Two tokens per step:
 // their decay chains are independent work for the scheduler while the state
 // updates wait on each other.
-template <typename TIO, int NS, int TILE, bool FASTQ>
+template <typename TIO, int NS, int TILE, bool FASTQ, bool Y = true>
 __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, const float (*bt)[NS],
                                                 const float (*ct)[NS], int rows, float a0, float inv_a0, float Dd,
                                                 float2 (&g)[NS / 2], float& sd, TIO* yp, int64_t ystride,
@@ -349,8 +352,10 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
     }
   };
   auto emit = [&](float s, TIO xr, float dt) {
-    st_global_pred(yp, from_f32<TIO>(fmaf(s, inv_a0, Dd * to_f32(xr))), active);
-    yp += ystride;
+    if constexpr (Y) {
+      st_global_pred(yp, from_f32<TIO>(fmaf(s, inv_a0, Dd * to_f32(xr))), active);
+      yp += ystride;
+    }
     sd += dt;
   };
   auto pair = [&](int r) {
@@ -359,8 +364,8 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
     float2 e0[NS / 2], e1[NS / 2];
     chain(d0, e0);
     chain(d1, e1);
-    const float s0 = token_update<TIO, NS>(e0, bt[r], ct[r], x0, g);
-    const float s1 = token_update<TIO, NS>(e1, bt[r + 1], ct[r + 1], x1, g);
+    const float s0 = token_update<TIO, NS, Y>(e0, bt[r], ct[r], x0, g);
+    const float s1 = token_update<TIO, NS, Y>(e1, bt[r + 1], ct[r + 1], x1, g);
     emit(s0, x0, d0);
     emit(s1, x1, d1);
   };
@@ -388,8 +393,8 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
         chain(nda, na);
         chain(ndb, nb);
       }
-      const float s0 = token_update<TIO, NS>(ea, bt[r], ct[r], xa, g);
-      const float s1 = token_update<TIO, NS>(eb, bt[r + 1], ct[r + 1], xb, g);
+      const float s0 = token_update<TIO, NS, Y>(ea, bt[r], ct[r], xa, g);
+      const float s1 = token_update<TIO, NS, Y>(eb, bt[r + 1], ct[r + 1], xb, g);
       emit(s0, xa, da);
       emit(s1, xb, db);
 #pragma unroll
@@ -413,7 +418,7 @@ __device__ __forceinline__ void tile_structured(const TIO* su, const TIO* sdl, c
       const float d0 = to_f32(sdl[r * kCPW]);
       float2 e0[NS / 2];
       chain(d0, e0);
-      emit(token_update<TIO, NS>(e0, bt[r], ct[r], x0, g), x0, d0);
+      emit(token_update<TIO, NS, Y>(e0, bt[r], ct[r], x0, g), x0, d0);
     }
   }
 }
@@ -947,8 +952,8 @@ __device__ __forceinline__ bool run_job(Consumer<TIO, NS, TILE, STAGES, R>& cx, 
       tile_mimo<TIO, NS, R, STRUCT, kFastQ>(su, sdl, sm.b[slot], sm.cs[slot], rows, a0, cm.y, kA, kC, Dd, g, sd,
                                             yrow, p.channels, store_y);
     } else if constexpr (STRUCT) {
-      tile_structured<TIO, NS, TILE, kFastQ>(su, sdl, sm.b[slot], sm.cs[slot], rows, a0, cm.y, Dd, g, sd, yrow,
-                                             p.channels, store_y);
+      tile_structured<TIO, NS, TILE, kFastQ, !CKPT>(su, sdl, sm.b[slot], sm.cs[slot], rows, a0, cm.y, Dd, g, sd,
+                                                    yrow, p.channels, store_y);
     } else {
       tile_general<TIO, NS, METHOD>(su, sdl, sm.b[slot], sm.cs[slot], rows, kA, kC, Dd, g, sd, vp, yrow,
                                     p.channels, store_y);
