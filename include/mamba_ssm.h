@@ -314,8 +314,9 @@ int mamba_selective_scan_backward(const void *u, const void *delta, const float 
  * count).  With more than one, every super-chunk runs from zero (the first
  * from initial_state) and records its end state (stream-ordered scratch of
  * 4 (64 nstate + 1) bytes per super-chunk and head); a second kernel adds
- * the entering states' effect to y while their decay is at least 2^-32
- * (the terms left out are below 2^-32 of their size) and writes
+ * the entering states' effect to y while their decay is at least 2^-20
+ * (the terms left out are below 2^-20 of their size, 2^11 times under the
+ * bf16 rounding of y) and writes
  * final_state.
  *
  * Supported: dtype MAMBA_BF16, headdim 64, nstate 16, 32 or 64, flags 0 or
